@@ -1,0 +1,199 @@
+"""CPU oracle of the MoGE layer forward (fp64, single thread, plain C in oracle.c).
+
+TEST INFRASTRUCTURE ONLY: the tests, the package smoke check and the benchmark's
+CPU-baseline leg use it; the product path never imports it. It shares no code
+with the CUDA library; both sides only share the seeded inputs of ``synth``.
+
+Functions with no independent pin are listed in the header of oracle.c and in
+the design notes ("parity unpinned"); every function here is pinned by
+tests/test_oracle.py against closed forms, brute force or library routines.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+F32, BF16 = 0, 1
+_DT = {"f32": F32, "bf16": BF16}
+
+
+def build(force: bool = False) -> str:
+    """Compile liboracle.so (gcc -O2, strict IEEE double, one thread)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp%d" % os.getpid()
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
+                               "-shared", "-fPIC", _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def _l():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        vp, i32 = ctypes.c_void_p, ctypes.c_int
+        lib.oracle_router_probs.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp]
+        lib.oracle_select_grouped.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp]
+        lib.oracle_select_global.argtypes = [vp, i32, i32, i32, vp]
+        lib.oracle_route.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp]
+        lib.oracle_imbalance.argtypes = [vp, i32, i32, i32, i32, vp]
+        lib.oracle_imbalance.restype = ctypes.c_double
+        lib.oracle_dispatch.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp]
+        lib.oracle_expert_ffn.argtypes = [vp, vp, vp, vp, i32, i32, i32, vp]
+        lib.oracle_layer.argtypes = [vp, i32, i32, i32, i32, i32, i32, i32, i32,
+                                     vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp]
+        lib.oracle_rmsnorm.argtypes = [vp, i32, i32, ctypes.c_double, vp]
+        _lib = lib
+    return _lib
+
+
+def _p(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data
+
+
+def _chk(rc: int, what: str):
+    if rc != 0:
+        raise ValueError("oracle %s failed (code %d)" % (what, rc))
+
+
+def to_double(a: np.ndarray, dtype: str) -> np.ndarray:
+    """Widen stored values (bf16 bit patterns or float32) to float64 exactly."""
+    if dtype == "bf16":
+        return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return np.asarray(a, dtype=np.float32).astype(np.float64)
+
+
+def _w(a: np.ndarray, dtype: str) -> np.ndarray:
+    want = np.uint16 if dtype == "bf16" else np.float32
+    if a.dtype != want:
+        raise TypeError("weights must be %s for dtype %s" % (want, dtype))
+    return np.ascontiguousarray(a)
+
+
+def router_probs(x: np.ndarray, w_router: np.ndarray, bias: Optional[np.ndarray],
+                 dtype: str) -> np.ndarray:
+    """Global softmax scores p [T][N] (x given as float64 [T][d])."""
+    x = np.ascontiguousarray(x, np.float64)
+    wr = _w(w_router, dtype)
+    T, d = x.shape
+    N = wr.shape[0]
+    b = None if bias is None else np.ascontiguousarray(bias, np.float32)
+    p = np.empty((T, N), np.float64)
+    _chk(_l().oracle_router_probs(_p(x), _p(wr), _p(b), _DT[dtype], T, d, N, _p(p)), "router_probs")
+    return p
+
+
+def select_grouped(p: np.ndarray, M: int, Kp: int):
+    """Per-group top-Kp on scores p [T][N] -> (idx [T][M*Kp] int32, w float64, margin [T])."""
+    p = np.ascontiguousarray(p, np.float64)
+    T, N = p.shape
+    idx = np.empty((T, M * Kp), np.int32)
+    w = np.empty((T, M * Kp), np.float64)
+    mg = np.empty(T, np.float64)
+    _chk(_l().oracle_select_grouped(_p(p), T, N, M, Kp, _p(idx), _p(w), _p(mg)), "select_grouped")
+    return idx, w, mg
+
+
+def select_global(p: np.ndarray, K: int) -> np.ndarray:
+    """Conventional global top-K on scores p [T][N] -> idx [T][K]."""
+    p = np.ascontiguousarray(p, np.float64)
+    T, N = p.shape
+    idx = np.empty((T, K), np.int32)
+    _chk(_l().oracle_select_global(_p(p), T, N, K, _p(idx)), "select_global")
+    return idx
+
+
+def route(x: np.ndarray, w_router: np.ndarray, bias, dtype: str, M: int, Kp: int):
+    """Scores + group-balanced selection for a batch -> (idx, w, margin)."""
+    x = np.ascontiguousarray(x, np.float64)
+    wr = _w(w_router, dtype)
+    T, d = x.shape
+    N = wr.shape[0]
+    b = None if bias is None else np.ascontiguousarray(bias, np.float32)
+    idx = np.empty((T, M * Kp), np.int32)
+    w = np.empty((T, M * Kp), np.float64)
+    mg = np.empty(T, np.float64)
+    _chk(_l().oracle_route(_p(x), _p(wr), _p(b), _DT[dtype], T, d, N, M, Kp,
+                           _p(idx), _p(w), _p(mg)), "route")
+    return idx, w, mg
+
+
+def imbalance(idx: np.ndarray, N: int, M: int):
+    """(imbalance score, per-group loads [M]) of an assignment matrix [T][K]."""
+    idx = np.ascontiguousarray(idx, np.int32)
+    T, K = idx.shape
+    loads = np.empty(M, np.int64)
+    s = _l().oracle_imbalance(_p(idx), T, K, N, M, _p(loads))
+    return float(s), loads
+
+
+def dispatch(idx: np.ndarray, N: int):
+    """(counts [N], offsets [N+1], perm_src [T*K], perm_dst [T][K]) of idx [T][K]."""
+    idx = np.ascontiguousarray(idx, np.int32)
+    T, K = idx.shape
+    counts = np.empty(N, np.int32)
+    offsets = np.empty(N + 1, np.int32)
+    ps = np.empty(T * K, np.int32)
+    pd = np.empty((T, K), np.int32)
+    _chk(_l().oracle_dispatch(_p(idx), T, K, N, _p(counts), _p(offsets), _p(ps), _p(pd)), "dispatch")
+    return counts, offsets, ps, pd
+
+
+def expert_ffn(x_row: np.ndarray, wg: np.ndarray, wu: np.ndarray, wd: np.ndarray,
+               dtype: str) -> np.ndarray:
+    """One SwiGLU expert on one token (x_row float64 [d]; wg,wu [I][d]; wd [d][I])."""
+    x = np.ascontiguousarray(x_row, np.float64)
+    wg, wu, wd = _w(wg, dtype), _w(wu, dtype), _w(wd, dtype)
+    I, d = wg.shape
+    y = np.empty(d, np.float64)
+    _chk(_l().oracle_expert_ffn(_p(x), _p(wg), _p(wu), _p(wd), _DT[dtype], d, I, _p(y)), "expert_ffn")
+    return y
+
+
+def layer(x: np.ndarray, inp: dict, M: int, Kp: int, dtype: str,
+          tokens: Optional[Sequence[int]] = None):
+    """MoGE layer output for the listed tokens (all when None).
+
+    x: float64 [T][d]; inp: the weight dict of synth.layer_inputs.
+    Returns (y [n][d] float64, idx [n][K], w [n][K], margin [n]).
+    """
+    x = np.ascontiguousarray(x, np.float64)
+    T, d = x.shape
+    wr = _w(inp["w_router"], dtype)
+    wg, wu, wd = _w(inp["w_gate"], dtype), _w(inp["w_up"], dtype), _w(inp["w_down"], dtype)
+    N, I = wg.shape[0], wg.shape[1]
+    S = inp["s_gate"].shape[0]
+    sg, su, sd = (_w(inp[k], dtype) if S > 0 else None for k in ("s_gate", "s_up", "s_down"))
+    b = inp.get("logit_bias")
+    b = None if b is None else np.ascontiguousarray(b, np.float32)
+    toks = np.arange(T, dtype=np.int32) if tokens is None else np.asarray(tokens, np.int32)
+    n = len(toks)
+    K = M * Kp
+    y = np.empty((n, d), np.float64)
+    idx = np.empty((n, K), np.int32)
+    w = np.empty((n, K), np.float64)
+    mg = np.empty(n, np.float64)
+    _chk(_l().oracle_layer(_p(x), T, d, N, M, Kp, S, I, _DT[dtype], _p(wr), _p(b),
+                           _p(wg), _p(wu), _p(wd), _p(sg), _p(su), _p(sd),
+                           _p(toks), n, _p(y), _p(idx), _p(w), _p(mg)), "layer")
+    return y, idx, w, mg
+
+
+def rmsnorm(x: np.ndarray, eps: float = 1e-6) -> np.ndarray:
+    """u = x / sqrt(mean(x^2) + eps), unit gain, per row."""
+    x = np.ascontiguousarray(x, np.float64)
+    T, d = x.shape
+    u = np.empty_like(x)
+    _chk(_l().oracle_rmsnorm(_p(x), T, d, eps, _p(u)), "rmsnorm")
+    return u

@@ -1,0 +1,328 @@
+/*
+ * oracle.c -- plain, slow, single-threaded CPU reference of the MoGE FFN layer
+ * forward pass, in fp64.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing on the product path may call, link or load
+ * this file: it is used by the tests, by the package's smoke check and by the
+ * timed CPU baseline of the benchmark. It shares no code, header, table or
+ * helper with the CUDA library.
+ *
+ * Sources (web pages on Huawei's Pangu Pro MoE; the method is stated in prose
+ * only, the formulas below restate it):
+ *  [A] "Huawei releases Pangu Pro MoE: the first 72B sparse language model,
+ *      designed for Ascend NPUs" (techwalker.com), section 1 "Innovative
+ *      architecture: the design of the mixture of grouped experts" --
+ *      N experts split evenly into M groups of N/M; per token K' = K/M experts
+ *      are chosen inside EVERY group; the scores are a GLOBAL softmax over all
+ *      N experts, taken BEFORE the in-group top-K'; the imbalance score is the
+ *      load gap between the busiest and the idlest device (group) in a batch.
+ *  [B] same page, section 2 "Hardware co-design" -- 64 routed experts plus 4
+ *      shared experts, hidden size 5120.
+ *  [C] reportify.cn concept page "Mixture of grouped experts", bullet
+ *      "technical innovation details" -- each group does its own top-K
+ *      routing, the inter-group load difference is zero.
+ *  [D] mokono.cn news page, "three breakthroughs of MoGE", item 1 -- 64
+ *      routed experts in 8 groups, 1 active per group, 4 shared experts kept
+ *      for general work.
+ *
+ * Readings where the pages are silent (each also listed in the design notes):
+ *  - the chosen experts' weights are their global-softmax probabilities, not
+ *    renormalised;
+ *  - shared experts are always on and enter with weight 1;
+ *  - an expert is a SwiGLU FFN: W_down (silu(W_gate x) * (W_up x)),
+ *    silu(z) = z / (1 + e^-z), no biases;
+ *  - group g holds the contiguous experts [g*N/M, (g+1)*N/M);
+ *  - inside a group the K' picks are taken in descending score order, equal
+ *    scores going to the lower expert index; the selection compares the
+ *    scores rounded to fp32, the precision the GPU path decides in;
+ *  - the imbalance score is (max_g L_g - min_g L_g) / (T K), L_g the number
+ *    of (token, expert) assignments that land in group g;
+ *  - within one expert's block of permuted rows, tokens keep ascending order.
+ *
+ * Layouts are row-major: x [T][d]; w_router [N][d]; w_gate, w_up [E][I][d];
+ * w_down [E][d][I] (E = N routed or S shared). Weights are fp32 (dtype 0) or
+ * bf16 bit patterns (dtype 1); every element is widened to double exactly.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define OR_F32 0
+#define OR_BF16 1
+
+static double bf16_bits_to_double(uint16_t h) {
+    uint32_t b = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &b, 4);
+    return (double)f;
+}
+
+/* row of a weight matrix widened to double */
+static void load_row(const void *base, int dtype, size_t first, int n, double *out) {
+    if (dtype == OR_F32) {
+        const float *p = (const float *)base + first;
+        for (int j = 0; j < n; ++j) out[j] = (double)p[j];
+    } else {
+        const uint16_t *p = (const uint16_t *)base + first;
+        for (int j = 0; j < n; ++j) out[j] = bf16_bits_to_double(p[j]);
+    }
+}
+
+static double dot(const double *a, const double *b, int n) {
+    double s = 0.0;
+    for (int j = 0; j < n; ++j) s += a[j] * b[j];
+    return s;
+}
+
+/* ---------------------------------------------------------------------------
+ * Router scores [A]: logits l_e = x . w_router[e] (+ bias_e), then ONE softmax
+ * over all N experts (max subtracted for range only).
+ * x: [T][d] double; p_out: [T][N] double.
+ */
+int oracle_router_probs(const double *x, const void *w_router, const float *bias, int dtype,
+                        int T, int d, int N, double *p_out) {
+    if (T < 0 || d <= 0 || N <= 0) return 1;
+    double *w = (double *)malloc(sizeof(double) * (size_t)d);
+    double *l = (double *)malloc(sizeof(double) * (size_t)N);
+    if (!w || !l) { free(w); free(l); return 2; }
+    for (int t = 0; t < T; ++t) {
+        const double *xt = x + (size_t)t * d;
+        for (int e = 0; e < N; ++e) {
+            load_row(w_router, dtype, (size_t)e * d, d, w);
+            l[e] = dot(xt, w, d) + (bias ? (double)bias[e] : 0.0);
+        }
+        double m = l[0];
+        for (int e = 1; e < N; ++e) if (l[e] > m) m = l[e];
+        double z = 0.0;
+        for (int e = 0; e < N; ++e) z += exp(l[e] - m);
+        for (int e = 0; e < N; ++e) p_out[(size_t)t * N + e] = exp(l[e] - m) / z;
+    }
+    free(w);
+    free(l);
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------
+ * Group-balanced selection [A][C] on given scores p [T][N]: for every group g,
+ * the Kp experts of [g*G, (g+1)*G) with the largest score (G = N/M).
+ * idx/w: [T][M*Kp], group-major, picks inside a group in descending order.
+ * margin[t]: min over groups of p(Kp-th pick) - p(best unpicked), in fp64;
+ * +inf when a group has no unpicked expert.
+ */
+int oracle_select_grouped(const double *p, int T, int N, int M, int Kp,
+                          int32_t *idx, double *w, double *margin) {
+    if (M <= 0 || N % M != 0 || Kp < 1 || Kp > N / M) return 1;
+    int G = N / M, K = M * Kp;
+    unsigned char *taken = (unsigned char *)malloc((size_t)N);
+    if (!taken) return 2;
+    for (int t = 0; t < T; ++t) {
+        const double *pt = p + (size_t)t * N;
+        memset(taken, 0, (size_t)N);
+        double mg = INFINITY;
+        for (int g = 0; g < M; ++g) {
+            double last = 0.0;
+            for (int j = 0; j < Kp; ++j) {
+                int best = -1;
+                float bv = 0.0f;
+                for (int e = g * G; e < (g + 1) * G; ++e) {
+                    if (taken[e]) continue;
+                    float v = (float)pt[e];
+                    if (best < 0 || v > bv) { best = e; bv = v; }  /* ties: lower index stays */
+                }
+                taken[best] = 1;
+                idx[(size_t)t * K + g * Kp + j] = best;
+                w[(size_t)t * K + g * Kp + j] = pt[best];
+                last = pt[best];
+            }
+            double next = -INFINITY;
+            for (int e = g * G; e < (g + 1) * G; ++e)
+                if (!taken[e] && pt[e] > next) next = pt[e];
+            if (next > -INFINITY && last - next < mg) mg = last - next;
+        }
+        if (margin) margin[t] = mg;
+    }
+    free(taken);
+    return 0;
+}
+
+/* Conventional global top-K [A] (the routing MoGE replaces): the K largest
+ * scores over all N experts, same ordering and tie rule. */
+int oracle_select_global(const double *p, int T, int N, int K, int32_t *idx) {
+    if (K < 1 || K > N) return 1;
+    unsigned char *taken = (unsigned char *)malloc((size_t)N);
+    if (!taken) return 2;
+    for (int t = 0; t < T; ++t) {
+        const double *pt = p + (size_t)t * N;
+        memset(taken, 0, (size_t)N);
+        for (int j = 0; j < K; ++j) {
+            int best = -1;
+            float bv = 0.0f;
+            for (int e = 0; e < N; ++e) {
+                if (taken[e]) continue;
+                float v = (float)pt[e];
+                if (best < 0 || v > bv) { best = e; bv = v; }
+            }
+            taken[best] = 1;
+            idx[(size_t)t * K + j] = best;
+        }
+    }
+    free(taken);
+    return 0;
+}
+
+/* Routing of a whole batch [A]: scores then group-balanced selection. */
+int oracle_route(const double *x, const void *w_router, const float *bias, int dtype,
+                 int T, int d, int N, int M, int Kp,
+                 int32_t *idx, double *w, double *margin) {
+    double *p = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1) * N);
+    if (!p) return 2;
+    int rc = oracle_router_probs(x, w_router, bias, dtype, T, d, N, p);
+    if (rc == 0) rc = oracle_select_grouped(p, T, N, M, Kp, idx, w, margin);
+    free(p);
+    return rc;
+}
+
+/* ---------------------------------------------------------------------------
+ * Imbalance score [A]: loads L_g = number of assignments in group g (experts
+ * [g*N/M, (g+1)*N/M)); loads_out[M] receives them; returns (max - min)/(T K).
+ */
+double oracle_imbalance(const int32_t *idx, int T, int K, int N, int M, int64_t *loads_out) {
+    int G = N / M;
+    int64_t *L = (int64_t *)calloc((size_t)M, sizeof(int64_t));
+    if (!L) return NAN;
+    for (size_t a = 0; a < (size_t)T * K; ++a) L[idx[a] / G] += 1;
+    int64_t mx = L[0], mn = L[0];
+    for (int g = 1; g < M; ++g) { if (L[g] > mx) mx = L[g]; if (L[g] < mn) mn = L[g]; }
+    if (loads_out) memcpy(loads_out, L, sizeof(int64_t) * (size_t)M);
+    free(L);
+    return (T > 0 && K > 0) ? (double)(mx - mn) / ((double)T * K) : 0.0;
+}
+
+/* ---------------------------------------------------------------------------
+ * Expert-major dispatch, written from its definition: counts[e] = number of
+ * assignments to e; offsets = exclusive prefix sum (offsets[N] = T K); the
+ * rows of expert e are offsets[e] .. offsets[e+1]-1, holding its tokens in
+ * ascending token order; perm_src[row] = token, perm_dst[t][k] = row.
+ */
+int oracle_dispatch(const int32_t *idx, int T, int K, int N,
+                    int32_t *counts, int32_t *offsets, int32_t *perm_src, int32_t *perm_dst) {
+    for (int e = 0; e < N; ++e) counts[e] = 0;
+    for (size_t a = 0; a < (size_t)T * K; ++a) {
+        if (idx[a] < 0 || idx[a] >= N) return 1;
+        counts[idx[a]] += 1;
+    }
+    offsets[0] = 0;
+    for (int e = 0; e < N; ++e) offsets[e + 1] = offsets[e] + counts[e];
+    for (int e = 0; e < N; ++e) {
+        int32_t row = offsets[e];
+        for (int t = 0; t < T; ++t)
+            for (int k = 0; k < K; ++k)
+                if (idx[(size_t)t * K + k] == e) {
+                    perm_src[row] = t;
+                    perm_dst[(size_t)t * K + k] = row;
+                    ++row;
+                }
+    }
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------
+ * One expert on one token: y = W_down (silu(W_gate x) * (W_up x)).
+ * wg, wu point at the expert's [I][d] matrices, wd at its [d][I] matrix.
+ */
+int oracle_expert_ffn(const double *x, const void *wg, const void *wu, const void *wd,
+                      int dtype, int d, int I, double *y) {
+    double *w = (double *)malloc(sizeof(double) * (size_t)(d > I ? d : I));
+    double *h = (double *)malloc(sizeof(double) * (size_t)I);
+    if (!w || !h) { free(w); free(h); return 2; }
+    for (int i = 0; i < I; ++i) {
+        load_row(wg, dtype, (size_t)i * d, d, w);
+        double g = dot(x, w, d);
+        load_row(wu, dtype, (size_t)i * d, d, w);
+        double u = dot(x, w, d);
+        h[i] = (g / (1.0 + exp(-g))) * u;
+    }
+    for (int o = 0; o < d; ++o) {
+        load_row(wd, dtype, (size_t)o * I, I, w);
+        y[o] = dot(h, w, I);
+    }
+    free(w);
+    free(h);
+    return 0;
+}
+
+static const void *expert_ptr(const void *base, int dtype, size_t e, size_t per_expert) {
+    size_t esz = dtype == OR_F32 ? 4 : 2;
+    return (const char *)base + e * per_expert * esz;
+}
+
+/* ---------------------------------------------------------------------------
+ * The layer [A][B][D] for the listed tokens only (each token is independent):
+ *   y_t = sum_g sum_{e picked in g} p_e FFN_e(x_t)  +  sum_s FFN_s(x_t)
+ * summed in pick order (group-major), then the shared experts in index order.
+ * x [T][d] double (all tokens; only listed rows are read); y_out [n][d].
+ * idx_out/w_out [n][M*Kp] and margin_out [n] may be NULL.
+ */
+int oracle_layer(const double *x, int T, int d, int N, int M, int Kp, int S, int I, int dtype,
+                 const void *w_router, const float *bias,
+                 const void *w_gate, const void *w_up, const void *w_down,
+                 const void *s_gate, const void *s_up, const void *s_down,
+                 const int32_t *tokens, int n, double *y_out,
+                 int32_t *idx_out, double *w_out, double *margin_out) {
+    if (N % M != 0 || Kp < 1 || Kp > N / M) return 1;
+    int K = M * Kp;
+    size_t per = (size_t)I * d;
+    double *tmp = (double *)malloc(sizeof(double) * (size_t)d);
+    int32_t *idx = (int32_t *)malloc(sizeof(int32_t) * (size_t)K);
+    double *w = (double *)malloc(sizeof(double) * (size_t)K);
+    if (!tmp || !idx || !w) { free(tmp); free(idx); free(w); return 2; }
+    int rc = 0;
+    for (int q = 0; q < n && rc == 0; ++q) {
+        int t = tokens[q];
+        if (t < 0 || t >= T) { rc = 1; break; }
+        const double *xt = x + (size_t)t * d;
+        double *yt = y_out + (size_t)q * d;
+        double mg;
+        rc = oracle_route(xt, w_router, bias, dtype, 1, d, N, M, Kp, idx, w, &mg);
+        if (rc) break;
+        for (int o = 0; o < d; ++o) yt[o] = 0.0;
+        for (int k = 0; k < K; ++k) {
+            size_t e = (size_t)idx[k];
+            rc = oracle_expert_ffn(xt, expert_ptr(w_gate, dtype, e, per),
+                                   expert_ptr(w_up, dtype, e, per),
+                                   expert_ptr(w_down, dtype, e, per), dtype, d, I, tmp);
+            if (rc) break;
+            for (int o = 0; o < d; ++o) yt[o] += w[k] * tmp[o];
+        }
+        for (int s = 0; s < S && rc == 0; ++s) {
+            rc = oracle_expert_ffn(xt, expert_ptr(s_gate, dtype, (size_t)s, per),
+                                   expert_ptr(s_up, dtype, (size_t)s, per),
+                                   expert_ptr(s_down, dtype, (size_t)s, per), dtype, d, I, tmp);
+            for (int o = 0; o < d; ++o) yt[o] += tmp[o];
+        }
+        if (idx_out) memcpy(idx_out + (size_t)q * K, idx, sizeof(int32_t) * (size_t)K);
+        if (w_out) memcpy(w_out + (size_t)q * K, w, sizeof(double) * (size_t)K);
+        if (margin_out) margin_out[q] = mg;
+    }
+    free(tmp);
+    free(idx);
+    free(w);
+    return rc;
+}
+
+/* ---------------------------------------------------------------------------
+ * RMSNorm with unit gain (pre-norm of the 12-layer stack; the page mentions
+ * RMSNorm in section 2, the form and eps are spec choices):
+ *   u = x / sqrt(mean(x^2) + eps)
+ */
+int oracle_rmsnorm(const double *x, int T, int d, double eps, double *u) {
+    for (int t = 0; t < T; ++t) {
+        const double *xt = x + (size_t)t * d;
+        double ss = 0.0;
+        for (int j = 0; j < d; ++j) ss += xt[j] * xt[j];
+        double r = 1.0 / sqrt(ss / d + eps);
+        for (int j = 0; j < d; ++j) u[(size_t)t * d + j] = xt[j] * r;
+    }
+    return 0;
+}
