@@ -1,0 +1,343 @@
+#!/usr/bin/env python
+"""Benchmark of the MoGE FFN layer forward on B200 (one JSON line on rank 0).
+
+A step is one moge_layer_forward over one batch: router GEMM + global softmax +
+per-group top-K', scan/permute, grouped SwiGLU up- and down-projection
+(tcgen05), combine with the shared experts. Workload: the decode layer
+(T=456 tokens, d=5120, 64 experts in 8 groups, K'=1, 4 shared experts,
+intermediate 1344, bf16), synthetic seeded inputs. The 2.8 GB of expert
+weights read per step exceed the 126 MB L2, so no L2 flush is needed.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl moge|reference]
+
+N > 1 (torchrun): every rank runs its own batch with replicated weights, no
+collective on the data path (weak scaling); time = max over ranks.
+--impl reference times the CPU oracle (fp64, 1 thread) on a bounded sample.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "MoGE layer tokens/s; % of HBM roofline (decode) / bf16 TC peak (prefill)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------- work model
+def up_bytes(cfg, n_used):
+    """Algorithmic bytes of one up-projection launch: gate+up weights of every
+    expert that received a token, the B rows it reads (routed rows + x for the
+    shared experts), and the h rows it writes; bf16."""
+    T, d, I, K, S = cfg.T, cfg.d, cfg.I, cfg.K, cfg.S
+    return 2 * ((n_used + S) * 2 * I * d + (T * K + T) * d + T * (K + S) * I)
+
+
+def down_bytes(cfg, n_used):
+    T, d, I, K, S = cfg.T, cfg.d, cfg.I, cfg.K, cfg.S
+    return 2 * ((n_used + S) * d * I + T * (K + S) * I + T * (K + S) * d)
+
+
+def up_flops(cfg):
+    return 2.0 * (cfg.T * cfg.K + cfg.S * cfg.T) * cfg.d * 2 * cfg.I
+
+
+def layer_flops(cfg):
+    return (cfg.T * cfg.K + cfg.S * cfg.T) * 6.0 * cfg.d * cfg.I + 2.0 * cfg.T * cfg.d * cfg.N
+
+
+def layer_bytes(cfg, n_used):
+    """Algorithmic bytes of the layer: each used expert's three matrices once,
+    the router, x in and y out (no padding, no permute traffic)."""
+    return 2 * ((n_used + cfg.S) * 3 * cfg.I * cfg.d + cfg.N * cfg.d + 2 * cfg.T * cfg.d)
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), "--query-gpu=" + self.Q,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), f[4:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i in range(4) if r[i + 1] == "Active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- oracle legs
+def oracle_sample(cfg, inp, tokens):
+    """Time the CPU oracle on the listed tokens (full layer each)."""
+    import oracle
+    xd = oracle.to_double(inp["x"], cfg.dtype)
+    t0 = time.perf_counter()
+    oracle.layer(xd, inp, cfg.M, cfg.Kp, cfg.dtype, tokens=tokens)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(cfg, inp, n_tokens):
+    toks = list(range(0, cfg.T, max(1, cfg.T // n_tokens)))[:n_tokens]
+    dt = oracle_sample(cfg, inp, toks)
+    return {"value": len(toks) / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": "%d of the %d tokens of the %s layer, full layer per token (routing over "
+                      "%d experts, %d routed + %d shared SwiGLU experts), fp64 C, one thread; %.1f s"
+                      % (len(toks), cfg.T, cfg.name, cfg.N, cfg.K, cfg.S, dt)}
+
+
+def workload_config(cfg):
+    return {"workload": "MoGE FFN layer forward, %s: T=%d tokens, d=%d, N=%d experts in M=%d groups, "
+                        "K'=%d (K=%d), S=%d shared, SwiGLU I=%d, %s" % (
+                            cfg.name, cfg.T, cfg.d, cfg.N, cfg.M, cfg.Kp, cfg.K, cfg.S, cfg.I, cfg.dtype),
+            "T": cfg.T, "d": cfg.d, "N": cfg.N, "M": cfg.M, "Kp": cfg.Kp, "S": cfg.S, "I": cfg.I,
+            "seed": cfg.seed,
+            "l2": "inputs larger than L2: %.2f GB of expert weights read per step, no flush"
+                  % (layer_bytes(cfg, cfg.N) / 1e9)}
+
+
+def run_reference(args, cfg):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    inp = synth.layer_inputs(cfg)
+    per_step = max(1, args.ref_tokens)
+    rng = np.random.default_rng(0)
+    for _ in range(args.warmup):
+        oracle_sample(cfg, inp, rng.choice(cfg.T, per_step, replace=False).tolist())
+    t = 0.0
+    for _ in range(args.steps):
+        t += oracle_sample(cfg, inp, rng.choice(cfg.T, per_step, replace=False).tolist())
+    value = args.steps * per_step / t
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000.0 * t / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded normal inputs)",
+            "config": workload_config(cfg),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": "each step: %d random tokens of the %d-token batch, full layer "
+                                       "per token, fp64 C oracle, one thread" % (per_step, cfg.T)},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def measure(cfg, inp, steps, warmup, dist_on=False, with_e2e=True):
+    """Device-timed layer steps (+ per-launch stage times, + end-to-end through
+    the host-buffer entry point). Returns a dict of raw measurements."""
+    import torch
+    import mixture_grouped_experts_b200 as mg
+
+    s = mg.shape_of(cfg)
+    x = mg.to_device(inp["x"], cfg.dtype)
+    w = mg.weights_to_device(inp, cfg.dtype)
+    ws = mg.alloc_workspace(s)
+    y = torch.empty_like(x)
+    for _ in range(max(warmup, 3)):
+        mg.moge_layer_forward(s, x, w, ws, y=y)
+    torch.cuda.synchronize()
+    mg.check_device_errors()
+    counts = mg.moge_workspace_routing(s, ws)[2].cpu().numpy()
+    n_used = int((counts > 0).sum())
+
+    stream = torch.cuda.current_stream()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    mg.moge_stage_timing(True)
+    if dist_on:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(steps):
+        mg.moge_layer_forward(s, x, w, ws, y=y)
+    end.record(stream)
+    torch.cuda.synchronize()
+    if dist_on:
+        torch.distributed.barrier()
+    stage_ms, calls = mg.moge_stage_times()
+    mg.moge_stage_timing(False)
+    mg.check_device_errors()
+    ms = start.elapsed_time(end) / steps
+    out = {"ms": ms, "stage_ms": {k: v / calls for k, v in stage_ms.items()}, "n_used": n_used,
+           "counts": counts}
+    if with_e2e:
+        xh = x.cpu().pin_memory()
+        yh = torch.empty_like(xh).pin_memory()
+        xd, yd = torch.empty_like(x), torch.empty_like(x)
+        for _ in range(3):
+            mg.moge_layer_forward_host(s, xh, w, ws, yh, xd, yd)
+        if dist_on:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        start.record(stream)
+        for _ in range(steps):
+            mg.moge_layer_forward_host(s, xh, w, ws, yh, xd, yd)
+        end.record(stream)
+        torch.cuda.synchronize()
+        out["e2e_ms"] = start.elapsed_time(end) / steps
+        out["io_bytes"] = xh.numel() * xh.element_size()
+    del x, w, ws, y
+    torch.cuda.empty_cache()
+    return out
+
+
+def max_over_ranks(v, dist_on):
+    if not dist_on:
+        return v
+    import torch
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="moge", choices=["moge", "reference"])
+    ap.add_argument("--config", default="decode", choices=["decode", "prefill", "skew"])
+    ap.add_argument("--no-secondary", action="store_true", help="skip the prefill side measurement")
+    ap.add_argument("--cpu-tokens", type=int, default=16, help="tokens in the CPU-baseline sample")
+    ap.add_argument("--ref-tokens", type=int, default=2, help="tokens per step of --impl reference")
+    args = ap.parse_args()
+    cfg = synth.CONFIGS[args.config]
+    if args.impl == "reference":
+        run_reference(args, cfg)
+        return
+
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist_on = world > 1
+    if dist_on:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    import mixture_grouped_experts_b200 as mg
+    mg.lib()
+    peaks, peak_kind = load_peaks()
+
+    inp = synth.layer_inputs(cfg, x_stream_offset=rank)
+    sampler = ClockSampler(local)
+    sampler.start()
+    m = measure(cfg, inp, args.steps, args.warmup, dist_on)
+    clocks = sampler.stop()
+    ms = max_over_ranks(m["ms"], dist_on)
+    e2e_ms = max_over_ranks(m["e2e_ms"], dist_on)
+    n = world
+    value = n * cfg.T / (ms / 1e3)
+
+    su = m["stage_ms"]
+    hbm = peaks["hbm_gbs"]
+    ub = up_bytes(cfg, m["n_used"])
+    ach = ub / (su["ffn_up"] / 1e3) / 1e9
+    roofline = {"bound": "hbm", "kernel": "ffn_tc_kernel<up> (grouped gate+up GEMM, SwiGLU epilogue)",
+                "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind if peak_kind == "measured"
+                else "fallback 6650 GB/s", "traffic": None,
+                "algorithmic_bytes_per_launch": ub,
+                "kernel_ms": su["ffn_up"]}
+    lb = layer_bytes(cfg, m["n_used"])
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": n, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded normal inputs, random-init weights)",
+            "config": dict(workload_config(cfg), parallelism="replicas (dp%d), no collective" % n),
+            "roofline": roofline,
+            "layer_roofline": {"bound": "hbm", "achieved": lb / (ms / 1e3) / 1e9, "peak": hbm,
+                               "unit": "GB/s", "frac": lb / (ms / 1e3) / 1e9 / hbm,
+                               "algorithmic_bytes": lb},
+            "stage_ms": su,
+            "e2e": {"value": n * cfg.T / (e2e_ms / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": m["io_bytes"], "d2h_bytes_per_step": m["io_bytes"],
+                    "api": "moge_layer_forward_host (pinned host x in, host y out, synchronised per step)"},
+            "gpu_launches": 6 * args.steps,
+            "clocks": clocks}
+    if rank == 0 and n == 1:
+        line["cpu_baseline"] = cpu_baseline(cfg, inp, args.cpu_tokens)
+    del inp
+    if rank == 0 and n == 1 and not args.no_secondary and args.config == "decode":
+        pcfg = synth.CONFIGS["prefill"]
+        pinp = synth.layer_inputs(pcfg)
+        ps = ClockSampler(local)
+        ps.start()
+        pm = measure(pcfg, pinp, max(5, args.steps // 2), args.warmup, False, with_e2e=False)
+        pclk = ps.stop()
+        tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        tfs = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+        up_tf = up_flops(pcfg) / (pm["stage_ms"]["ffn_up"] / 1e3) / 1e12
+        lay_tf = layer_flops(pcfg) / (pm["ms"] / 1e3) / 1e12
+        line["prefill"] = {
+            "workload": workload_config(pcfg)["workload"],
+            "value": pcfg.T / (pm["ms"] / 1e3), "unit": "tokens/s", "ms_per_step": pm["ms"],
+            "roofline": {"bound": "tensor", "kernel": "ffn_tc_kernel<up>", "achieved": up_tf,
+                         "peak": tf, "unit": "TFLOP/s", "frac": up_tf / tf,
+                         "peak_source": "%s bf16_tflops (burst)" % peak_kind},
+            "layer_tflops": lay_tf, "layer_frac_sustained": lay_tf / tfs,
+            "stage_ms": pm["stage_ms"], "clocks": pclk}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist_on:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

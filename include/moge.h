@@ -1,0 +1,181 @@
+/*
+ * moge.h -- C ABI of the MoGE (Mixture of Grouped Experts) FFN layer forward
+ * pass for NVIDIA B200 (sm_100a).
+ *
+ * The operation (restated from "Huawei releases Pangu Pro MoE: the first 72B
+ * sparse language model, designed for Ascend NPUs", techwalker.com,
+ * section 1 "Innovative architecture", and section 2 for the shared experts):
+ *
+ *   for every token t, with x_t its hidden vector (length d):
+ *     l_e   = x_t . w_router[e] (+ logit_bias[e])          e = 0 .. N-1
+ *     p     = softmax(l) over ALL N experts (global softmax, before selection)
+ *     group g holds experts [g*G, (g+1)*G), G = N/M; inside EVERY group the
+ *     Kp = K/M experts with the largest p are picked (ties: lower index)
+ *     y_t   = sum_{picked e} p_e * FFN_e(x_t)  +  sum_{s<S} FFN_s(x_t)
+ *     FFN(x) = W_down (silu(W_gate x) * (W_up x)),  silu(z) = z / (1 + e^-z)
+ *
+ * Every group receives exactly T*Kp (token, expert) assignments, so the
+ * per-group load is equal by construction (imbalance score 0). The picked
+ * weights are NOT renormalised; shared experts enter with weight 1.
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are caller-owned DEVICE pointers on the current CUDA
+ *    device, 16-byte aligned, row-major, densely packed. The library never
+ *    allocates device memory in these calls and never synchronises the host
+ *    (except moge_check_device_errors).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Work is enqueued asynchronously on it.
+ *  - dtype MOGE_BF16: x, weights and every activation are bf16 (bit patterns,
+ *    2 bytes); router logits, softmax, SwiGLU epilogue and all sums are fp32.
+ *    dtype MOGE_F32: everything is fp32 (CUDA-core arithmetic, no TF32).
+ *    Scores (topk_w) and logit_bias are always fp32; indices are int32.
+ *  - Return value: MOGE_OK or an error code; nothing is enqueued when a host
+ *    check fails. moge_last_error() gives a message (thread-local).
+ *    Errors found by the kernels (a bounded wait that timed out, a violated
+ *    routing invariant) are recorded in a device-side word and reported by
+ *    moge_check_device_errors().
+ *
+ * Weight layouts follow the nn.Linear [out][in] convention:
+ *   w_router [N][d]; w_gate, w_up [N][I][d]; w_down [N][d][I]
+ *   s_gate, s_up [S][I][d]; s_down [S][d][I]
+ * Size limits: 1 <= N <= 256, N % M == 0, 1 <= Kp <= N/M, d % 8 == 0,
+ * I % 8 == 0, T*(M*Kp+S) < 2^31 (else MOGE_ERR_UNSUPPORTED).
+ */
+#ifndef MOGE_H
+#define MOGE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOGE_API __attribute__((visibility("default")))
+#else
+#define MOGE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOGE_OK 0
+#define MOGE_ERR_INVALID_ARG 1 /* null pointer, negative size, bad dtype */
+#define MOGE_ERR_UNSUPPORTED 2 /* a size limit above, or a misaligned pointer */
+#define MOGE_ERR_CUDA 3        /* a CUDA runtime/driver call failed */
+#define MOGE_ERR_TIMEOUT 4     /* a bounded device wait gave up (device word) */
+#define MOGE_ERR_DEVICE 5      /* a kernel found a violated invariant (device word) */
+
+#define MOGE_F32 0
+#define MOGE_BF16 1
+
+typedef struct moge_config {
+    int T;     /* tokens in the batch (>= 0) */
+    int d;     /* hidden size */
+    int N;     /* routed experts */
+    int M;     /* groups (N/M experts each) */
+    int Kp;    /* experts picked per group per token (K = M*Kp per token) */
+    int S;     /* always-on shared experts (>= 0) */
+    int I;     /* SwiGLU intermediate size of every expert */
+    int dtype; /* MOGE_BF16 or MOGE_F32 */
+} moge_config;
+
+/* Bytes of device workspace the calls below need for this configuration
+ * (0 for an invalid one). The caller allocates it once (256-byte aligned) and
+ * may reuse it across calls on the same stream. */
+MOGE_API size_t moge_workspace_size(const moge_config *cfg);
+
+/* Message of the last failing call on this host thread ("" if none). */
+MOGE_API const char *moge_last_error(void);
+
+/* Synchronises `stream`, reads and clears the device error word of the
+ * current device: MOGE_OK, MOGE_ERR_TIMEOUT or MOGE_ERR_DEVICE. */
+MOGE_API int moge_check_device_errors(void *stream);
+
+/* Routing: router GEMM, global fp32 softmax, per-group top-Kp, per-expert
+ * counts and the expert-major permutation (section 1 of the article above;
+ * equal per-group load from the reportify "mixture of grouped experts" page).
+ *   x [T][d] dtype, w_router [N][d] dtype, logit_bias [N] fp32 or NULL
+ *   out topk_idx [T][K] int32  picks, group-major, descending score inside a group
+ *   out topk_w   [T][K] fp32   the picks' global softmax scores (no renorm)
+ *   out counts   [N]    int32  assignments per expert
+ *   out offsets  [N+1]  int32  exclusive prefix sum of counts (offsets[N] = T*K)
+ *   out perm_src [T*K]  int32  token held by each expert-major row
+ *   out perm_dst [T][K] int32  expert-major row of each (token, pick)
+ * Rows of one expert keep ascending token order. */
+MOGE_API int moge_route(const moge_config *cfg, const void *x, const void *w_router,
+               const float *logit_bias, int32_t *topk_idx, float *topk_w, int32_t *counts,
+               int32_t *offsets, int32_t *perm_src, int32_t *perm_dst, void *workspace,
+               void *stream);
+
+/* Permute: x_perm[r] = x[perm_src[r]] for r < T*K (rows of d, dtype). */
+MOGE_API int moge_permute(const moge_config *cfg, const void *x, const int32_t *perm_src, void *x_perm,
+                 void *stream);
+
+/* Grouped routed-expert FFN over expert-major rows: for every expert e and
+ * row r in [offsets[e], offsets[e+1]):
+ *   y_perm[r] = W_down[e] (silu(W_gate[e] x_perm[r]) * (W_up[e] x_perm[r]))
+ * x_perm, y_perm [T*K][d] dtype; offsets [N+1] int32 on the device.
+ * bf16: tcgen05 tensor-core GEMMs (TMA-fed, TMEM accumulators), the SwiGLU
+ * product rounded to bf16 between the two GEMMs. */
+MOGE_API int moge_grouped_ffn(const moge_config *cfg, const void *x_perm, const int32_t *offsets,
+                     const void *w_gate, const void *w_up, const void *w_down, void *y_perm,
+                     void *workspace, void *stream);
+
+/* Shared experts: y_shared[t] = sum_{s<S} FFN_s(x[t]); x, y_shared [T][d]. */
+MOGE_API int moge_shared_ffn(const moge_config *cfg, const void *x, const void *s_gate,
+                    const void *s_up, const void *s_down, void *y_shared, void *workspace,
+                    void *stream);
+
+/* Combine: y[t] = residual[t] + sum_{k<K} topk_w[t][k] * y_perm[perm_dst[t][k]]
+ *                 + y_shared[t]
+ * summed in fp32 in this order (k ascending); residual and y_shared may be
+ * NULL (treated as zero). y may alias residual. */
+MOGE_API int moge_combine(const moge_config *cfg, const void *y_perm, const float *topk_w,
+                 const int32_t *perm_dst, const void *y_shared, const void *residual, void *y,
+                 void *stream);
+
+/* Whole layer: route, permute, one grouped up-projection launch and one
+ * grouped down-projection launch covering routed AND shared experts, combine.
+ *   y[t] = residual[t] (if not NULL) + MoGE(x)[t];  y may alias residual, not x.
+ * s_* may be NULL when S == 0; logit_bias may be NULL. The routing of the
+ * call stays readable in the workspace (moge_workspace_routing). */
+MOGE_API int moge_layer_forward(const moge_config *cfg, const void *x, const void *w_router,
+                       const float *logit_bias, const void *w_gate, const void *w_up,
+                       const void *w_down, const void *s_gate, const void *s_up,
+                       const void *s_down, const void *residual, void *y, void *workspace,
+                       void *stream);
+
+/* moge_layer_forward with x and y in HOST memory (pinned for full speed):
+ * copies x in, runs the layer, copies y out, all on `stream`, and returns after
+ * synchronising the stream. Weights and workspace stay device pointers. */
+MOGE_API int moge_layer_forward_host(const moge_config *cfg, const void *x_host, const void *w_router,
+                            const float *logit_bias, const void *w_gate, const void *w_up,
+                            const void *w_down, const void *s_gate, const void *s_up,
+                            const void *s_down, void *y_host, void *x_dev, void *y_dev,
+                            void *workspace, void *stream);
+
+/* Device pointers, inside `workspace`, of the routing written by the last
+ * moge_layer_forward on it: topk_idx [T][K], topk_w [T][K], counts [N],
+ * offsets [N+1] (any out pointer may be NULL). Host-only arithmetic. */
+MOGE_API int moge_workspace_routing(const moge_config *cfg, void *workspace, int32_t **topk_idx,
+                           float **topk_w, int32_t **counts, int32_t **offsets);
+
+/* RMSNorm with unit gain, per row of x [T][d] (dtype): u = x / sqrt(mean(x^2) + eps),
+ * fp32 arithmetic (pre-norm of a stack of MoGE blocks; RMSNorm is named in
+ * section 2 of the article above, its form here is a stated choice). */
+MOGE_API int moge_rmsnorm(const moge_config *cfg, const void *x, float eps, void *u, void *stream);
+
+/* Stage timing (measurement aid): while enabled, every moge_layer_forward
+ * records CUDA events around its six launches -- router, scan, permute,
+ * up-projection, down-projection, combine -- and the library adds up their
+ * durations. moge_stage_timing(1) resets the totals and starts, (0) stops.
+ * moge_stage_times waits for the recorded events and returns the totals in
+ * milliseconds per stage (ms_total[6]) and the number of timed calls. For one
+ * host thread and one device; not for use during CUDA stream capture. */
+MOGE_API int moge_stage_timing(int enable);
+MOGE_API int moge_stage_times(double *ms_total, int64_t *calls);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOGE_H */

@@ -1,0 +1,269 @@
+"""Thin Python binding of libmoge.so, the B200 (sm_100a) MoGE layer forward.
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels. PyTorch provides device memory and streams. The entry points carry
+the names of the C ABI in include/moge.h; each takes torch tensors on the
+current CUDA device (bf16 tensors for a bf16 layer, float32 for an fp32 one,
+int32 indices, float32 scores) and enqueues on the current torch stream.
+
+There is no fallback: if libmoge.so is missing or cannot be loaded, loading
+it raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoge.so")
+
+MOGE_F32, MOGE_BF16 = 0, 1
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE = range(6)
+_DT = {"f32": MOGE_F32, "bf16": MOGE_BF16}
+_TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+EXPORTS = ["moge_workspace_size", "moge_last_error", "moge_check_device_errors", "moge_route",
+           "moge_permute", "moge_grouped_ffn", "moge_shared_ffn", "moge_combine",
+           "moge_layer_forward", "moge_layer_forward_host", "moge_workspace_routing",
+           "moge_rmsnorm", "moge_stage_timing", "moge_stage_times"]
+STAGES = ("router", "scan", "permute", "ffn_up", "ffn_down", "combine")
+
+
+class MogeError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__("moge error %d: %s" % (code, msg))
+        self.code = code
+
+
+class moge_config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("T", "d", "N", "M", "Kp", "S", "I", "dtype")]
+
+
+@dataclass(frozen=True)
+class LayerShape:
+    """Sizes of one MoGE layer: T tokens, hidden d, N routed experts in M
+    groups, Kp picked per group, S shared experts, SwiGLU intermediate I."""
+    T: int
+    d: int
+    N: int
+    M: int
+    Kp: int
+    S: int
+    I: int
+    dtype: str = "bf16"
+
+    @property
+    def K(self) -> int:
+        return self.M * self.Kp
+
+
+def shape_of(obj, **over) -> LayerShape:
+    """LayerShape from any object with the fields T, d, N, M, Kp, S, I, dtype."""
+    kw = {f: getattr(obj, f) for f in ("T", "d", "N", "M", "Kp", "S", "I", "dtype")}
+    kw.update(over)
+    return LayerShape(**kw)
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmoge.so (raises when it is missing: there is no fallback path)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError("libmoge.so not built: run `python -m mixture_grouped_experts_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, cp, i32 = ctypes.c_void_p, ctypes.POINTER(moge_config), ctypes.c_int
+        L.moge_workspace_size.argtypes = [cp]
+        L.moge_workspace_size.restype = ctypes.c_size_t
+        L.moge_last_error.argtypes = []
+        L.moge_last_error.restype = ctypes.c_char_p
+        L.moge_check_device_errors.argtypes = [vp]
+        L.moge_route.argtypes = [cp] + [vp] * 11
+        L.moge_permute.argtypes = [cp, vp, vp, vp, vp]
+        L.moge_grouped_ffn.argtypes = [cp] + [vp] * 8
+        L.moge_shared_ffn.argtypes = [cp] + [vp] * 7
+        L.moge_combine.argtypes = [cp] + [vp] * 7
+        L.moge_layer_forward.argtypes = [cp] + [vp] * 13
+        L.moge_layer_forward_host.argtypes = [cp] + [vp] * 14
+        L.moge_workspace_routing.argtypes = [cp, vp] + [ctypes.POINTER(vp)] * 4
+        L.moge_rmsnorm.argtypes = [cp, vp, ctypes.c_float, vp, vp]
+        L.moge_stage_timing.argtypes = [i32]
+        L.moge_stage_times.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]
+        for n in EXPORTS:
+            if n not in ("moge_workspace_size", "moge_last_error"):
+                getattr(L, n).restype = i32
+        _lib = L
+    return _lib
+
+
+def _cfg(s: LayerShape) -> moge_config:
+    return moge_config(s.T, s.d, s.N, s.M, s.Kp, s.S, s.I, _DT[s.dtype])
+
+
+def _p(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libmoge must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _chk(rc: int):
+    if rc != OK:
+        raise MogeError(rc, lib().moge_last_error().decode())
+
+
+def workspace_size(s: LayerShape) -> int:
+    n = lib().moge_workspace_size(ctypes.byref(_cfg(s)))
+    if n == 0:
+        raise MogeError(ERR_INVALID_ARG, lib().moge_last_error().decode())
+    return n
+
+
+def alloc_workspace(s: LayerShape, device=None) -> torch.Tensor:
+    return torch.empty(workspace_size(s), dtype=torch.uint8, device=device or "cuda")
+
+
+def check_device_errors(stream=None):
+    _chk(lib().moge_check_device_errors(_stream(stream)))
+
+
+def moge_route(s: LayerShape, x, w_router, logit_bias, workspace, stream=None):
+    """-> (topk_idx [T][K] i32, topk_w [T][K] f32, counts [N], offsets [N+1], perm_src [T*K], perm_dst [T][K])"""
+    dev = x.device
+    T, K, N = s.T, s.K, s.N
+    idx = torch.empty((T, K), dtype=torch.int32, device=dev)
+    w = torch.empty((T, K), dtype=torch.float32, device=dev)
+    counts = torch.empty(N, dtype=torch.int32, device=dev)
+    offsets = torch.empty(N + 1, dtype=torch.int32, device=dev)
+    ps = torch.empty(max(T * K, 1), dtype=torch.int32, device=dev)
+    pd = torch.empty((T, K), dtype=torch.int32, device=dev)
+    _chk(lib().moge_route(ctypes.byref(_cfg(s)), _p(x), _p(w_router), _p(logit_bias), _p(idx),
+                          _p(w), _p(counts), _p(offsets), _p(ps), _p(pd), _p(workspace),
+                          _stream(stream)))
+    return idx, w, counts, offsets, ps[:T * K], pd
+
+
+def moge_permute(s: LayerShape, x, perm_src, x_perm=None, stream=None):
+    if x_perm is None:
+        x_perm = torch.empty((s.T * s.K, s.d), dtype=x.dtype, device=x.device)
+    _chk(lib().moge_permute(ctypes.byref(_cfg(s)), _p(x), _p(perm_src), _p(x_perm), _stream(stream)))
+    return x_perm
+
+
+def moge_grouped_ffn(s: LayerShape, x_perm, offsets, w_gate, w_up, w_down, workspace,
+                     y_perm=None, stream=None):
+    if y_perm is None:
+        y_perm = torch.empty((s.T * s.K, s.d), dtype=x_perm.dtype, device=x_perm.device)
+    _chk(lib().moge_grouped_ffn(ctypes.byref(_cfg(s)), _p(x_perm), _p(offsets), _p(w_gate),
+                                _p(w_up), _p(w_down), _p(y_perm), _p(workspace), _stream(stream)))
+    return y_perm
+
+
+def moge_shared_ffn(s: LayerShape, x, s_gate, s_up, s_down, workspace, y_shared=None, stream=None):
+    if y_shared is None:
+        y_shared = torch.empty((s.T, s.d), dtype=x.dtype, device=x.device)
+    _chk(lib().moge_shared_ffn(ctypes.byref(_cfg(s)), _p(x), _p(s_gate), _p(s_up), _p(s_down),
+                               _p(y_shared), _p(workspace), _stream(stream)))
+    return y_shared
+
+
+def moge_combine(s: LayerShape, y_perm, topk_w, perm_dst, y_shared=None, residual=None, y=None,
+                 stream=None):
+    if y is None:
+        y = torch.empty((s.T, s.d), dtype=y_perm.dtype, device=y_perm.device)
+    _chk(lib().moge_combine(ctypes.byref(_cfg(s)), _p(y_perm), _p(topk_w), _p(perm_dst),
+                            _p(y_shared), _p(residual), _p(y), _stream(stream)))
+    return y
+
+
+def moge_layer_forward(s: LayerShape, x, w: dict, workspace, residual=None, y=None, stream=None):
+    """w: dict with w_router, logit_bias (or None), w_gate, w_up, w_down, s_gate, s_up, s_down."""
+    if y is None:
+        y = torch.empty((s.T, s.d), dtype=x.dtype, device=x.device)
+    _chk(lib().moge_layer_forward(ctypes.byref(_cfg(s)), _p(x), _p(w["w_router"]),
+                                  _p(w.get("logit_bias")), _p(w["w_gate"]), _p(w["w_up"]),
+                                  _p(w["w_down"]), _p(w.get("s_gate")), _p(w.get("s_up")),
+                                  _p(w.get("s_down")), _p(residual), _p(y), _p(workspace),
+                                  _stream(stream)))
+    return y
+
+
+def moge_layer_forward_host(s: LayerShape, x_host, w: dict, workspace, y_host, x_dev, y_dev,
+                            stream=None):
+    """Host x in, host y out (pinned CPU tensors); returns after the stream is synchronised."""
+    _chk(lib().moge_layer_forward_host(ctypes.byref(_cfg(s)), _p(x_host), _p(w["w_router"]),
+                                       _p(w.get("logit_bias")), _p(w["w_gate"]), _p(w["w_up"]),
+                                       _p(w["w_down"]), _p(w.get("s_gate")), _p(w.get("s_up")),
+                                       _p(w.get("s_down")), _p(y_host), _p(x_dev), _p(y_dev),
+                                       _p(workspace), _stream(stream)))
+    return y_host
+
+
+def moge_workspace_routing(s: LayerShape, workspace):
+    """Views of the routing the last moge_layer_forward wrote into `workspace`:
+    (topk_idx [T][K], topk_w [T][K], counts [N], offsets [N+1])."""
+    ptrs = [ctypes.c_void_p() for _ in range(4)]
+    _chk(lib().moge_workspace_routing(ctypes.byref(_cfg(s)), _p(workspace),
+                                      *[ctypes.byref(p) for p in ptrs]))
+    base = workspace.data_ptr()
+    out = []
+    for p, n, dt in zip(ptrs, (s.T * s.K, s.T * s.K, s.N, s.N + 1),
+                        (torch.int32, torch.float32, torch.int32, torch.int32)):
+        off = p.value - base
+        out.append(workspace[off:off + 4 * n].view(dt))
+    return out[0].view(s.T, s.K), out[1].view(s.T, s.K), out[2], out[3]
+
+
+def moge_rmsnorm(s: LayerShape, x, eps: float = 1e-6, u=None, stream=None):
+    if u is None:
+        u = torch.empty_like(x)
+    _chk(lib().moge_rmsnorm(ctypes.byref(_cfg(s)), _p(x), float(eps), _p(u), _stream(stream)))
+    return u
+
+
+def to_device(a, dtype: str, device="cuda") -> torch.Tensor:
+    """Host array (uint16 bf16 bit patterns or float32) -> device tensor of the layer dtype."""
+    import numpy as np
+    if a is None:
+        return None
+    if dtype == "bf16" and a.dtype == np.uint16:
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+
+def weights_to_device(inp: dict, dtype: str, device="cuda") -> dict:
+    """The weight dict of a layer (host arrays) moved to the device; logit_bias stays fp32."""
+    out = {}
+    for k in ("w_router", "w_gate", "w_up", "w_down", "s_gate", "s_up", "s_down"):
+        out[k] = to_device(inp[k], dtype, device) if inp.get(k) is not None and inp[k].size else None
+    lb = inp.get("logit_bias")
+    out["logit_bias"] = None if lb is None else torch.from_numpy(lb).to(device)
+    return out
+
+
+def moge_stage_timing(enable: bool):
+    """Start (reset) or stop the per-launch CUDA-event timing of moge_layer_forward."""
+    _chk(lib().moge_stage_timing(1 if enable else 0))
+
+
+def moge_stage_times():
+    """-> ({stage: total ms}, timed calls) accumulated since moge_stage_timing(True)."""
+    ms = (ctypes.c_double * len(STAGES))()
+    n = ctypes.c_int64()
+    _chk(lib().moge_stage_times(ms, ctypes.byref(n)))
+    return {k: ms[i] for i, k in enumerate(STAGES)}, n.value

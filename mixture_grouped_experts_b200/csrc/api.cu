@@ -1,0 +1,424 @@
+// C ABI of the MoGE layer (declared in include/moge.h): argument checks,
+// workspace carve-up and the launch sequences. No entry point allocates
+// device memory; all of them only enqueue work on the caller's stream.
+#include <string.h>
+
+#include <string>
+
+#include "common.cuh"
+#include "moge_internal.h"
+
+namespace moge {
+
+static thread_local std::string g_last_error;
+
+static int fail(int code, const std::string &msg) {
+    g_last_error = msg;
+    return code;
+}
+static int cuda_fail(cudaError_t e, const char *where) {
+    return fail(MOGE_ERR_CUDA, std::string(where) + ": " + cudaGetErrorString(e));
+}
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+static int check_config(const moge_config *c) {
+    if (!c) return fail(MOGE_ERR_INVALID_ARG, "config is NULL");
+    if (c->T < 0 || c->d <= 0 || c->N <= 0 || c->M <= 0 || c->Kp <= 0 || c->S < 0 || c->I <= 0)
+        return fail(MOGE_ERR_INVALID_ARG, "config has a non-positive size");
+    if (c->dtype != MOGE_F32 && c->dtype != MOGE_BF16)
+        return fail(MOGE_ERR_INVALID_ARG, "dtype must be MOGE_F32 or MOGE_BF16");
+    if (c->N > kMaxExperts) return fail(MOGE_ERR_UNSUPPORTED, "N > 256");
+    if (c->N % c->M != 0) return fail(MOGE_ERR_UNSUPPORTED, "N is not a multiple of M");
+    if (c->Kp > c->N / c->M) return fail(MOGE_ERR_UNSUPPORTED, "Kp > N/M");
+    if (c->d % 8 != 0 || c->I % 8 != 0)
+        return fail(MOGE_ERR_UNSUPPORTED, "d and I must be multiples of 8");
+    if (c->dtype == MOGE_BF16 && c->N % 8 != 0)
+        return fail(MOGE_ERR_UNSUPPORTED, "bf16 router needs N % 8 == 0");
+    const long long rows = (long long)c->T * (c->M * c->Kp + c->S);
+    if (rows >= (1ll << 31) || (long long)c->T * c->M * c->Kp * (long long)c->d >= (1ll << 62))
+        return fail(MOGE_ERR_UNSUPPORTED, "T*(K+S) rows exceed int32");
+    return MOGE_OK;
+}
+
+static size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+Workspace carve_workspace(const moge_config &c, void *base) {
+    Workspace w;
+    const size_t K = (size_t)c.M * c.Kp, T = (size_t)c.T, N = (size_t)c.N;
+    const size_t tiles = (T + kRouterTile - 1) / kRouterTile;
+    const size_t E = N + (size_t)c.S;
+    const size_t esz = c.dtype == MOGE_BF16 ? 2 : 4;
+    char *p = static_cast<char *>(base);
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        char *r = p ? p + off : nullptr;
+        off += align256(bytes > 0 ? bytes : 1);
+        return r;
+    };
+    w.hist = (int32_t *)take(tiles * N * 4);
+    w.base = (int32_t *)take(tiles * N * 4);
+    w.rank = (int32_t *)take(T * K * 4);
+    w.topk_idx = (int32_t *)take(T * K * 4);
+    w.topk_w = (float *)take(T * K * 4);
+    w.counts = (int32_t *)take(N * 4);
+    w.offsets = (int32_t *)take((N + 1) * 4);
+    w.perm_src = (int32_t *)take(T * K * 4);
+    w.perm_dst = (int32_t *)take(T * K * 4);
+    w.plan.up = (ExpertWork *)take(E * sizeof(ExpertWork));
+    w.plan.down = (ExpertWork *)take(E * sizeof(ExpertWork));
+    w.plan.up_start = (int *)take((E + 1) * 4);
+    w.plan.down_start = (int *)take((E + 1) * 4);
+    w.x_perm = take(T * K * c.d * esz);
+    w.h = take(T * (K + c.S) * c.I * esz);
+    w.y_perm = take(T * (K + c.S) * c.d * esz);
+    w.total = off;
+    return w;
+}
+
+static int num_sms() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+#define MOGE_NEED(p, what)                                                       \
+    do {                                                                         \
+        if (!(p)) return fail(MOGE_ERR_INVALID_ARG, std::string(what) + " is NULL"); \
+        if (!aligned16(p))                                                       \
+            return fail(MOGE_ERR_UNSUPPORTED, std::string(what) + " is not 16-byte aligned"); \
+    } while (0)
+#define MOGE_NEED4(p, what)                                                      \
+    do {                                                                         \
+        if (!(p)) return fail(MOGE_ERR_INVALID_ARG, std::string(what) + " is NULL"); \
+        if (!aligned4(p))                                                        \
+            return fail(MOGE_ERR_UNSUPPORTED, std::string(what) + " is not 4-byte aligned"); \
+    } while (0)
+#define MOGE_CU(expr, where)                       \
+    do {                                           \
+        cudaError_t e_ = (expr);                   \
+        if (e_ != cudaSuccess) return cuda_fail(e_, where); \
+    } while (0)
+
+// ---------------------------------------------------------------- stage timing
+// Optional CUDA-event timing of the six launches of moge_layer_forward
+// (router, scan, permute, up-projection, down-projection, combine). Host state
+// for one host thread and one device; not for use under stream capture.
+constexpr int kTimedStages = 6;
+constexpr int kEventSets = 32;
+struct StageTimer {
+    bool enabled = false;
+    cudaEvent_t ev[kEventSets][kTimedStages + 1] = {};
+    bool pending[kEventSets] = {};
+    int next = 0;
+    double total_ms[kTimedStages] = {};
+    long long calls = 0;
+};
+static StageTimer g_timer;
+
+static cudaError_t timer_harvest(int i) {
+    if (!g_timer.pending[i]) return cudaSuccess;
+    cudaError_t e = cudaEventSynchronize(g_timer.ev[i][kTimedStages]);
+    if (e != cudaSuccess) return e;
+    for (int s = 0; s < kTimedStages; ++s) {
+        float ms = 0.0f;
+        e = cudaEventElapsedTime(&ms, g_timer.ev[i][s], g_timer.ev[i][s + 1]);
+        if (e != cudaSuccess) return e;
+        g_timer.total_ms[s] += ms;
+    }
+    g_timer.pending[i] = false;
+    g_timer.calls += 1;
+    return cudaSuccess;
+}
+
+// Event set for the next layer call, or nullptr when timing is off.
+static cudaEvent_t *timer_slot() {
+    if (!g_timer.enabled) return nullptr;
+    const int i = g_timer.next;
+    g_timer.next = (i + 1) % kEventSets;
+    if (timer_harvest(i) != cudaSuccess) return nullptr;
+    for (int s = 0; s <= kTimedStages; ++s)
+        if (!g_timer.ev[i][s] && cudaEventCreate(&g_timer.ev[i][s]) != cudaSuccess) return nullptr;
+    g_timer.pending[i] = true;
+    return g_timer.ev[i];
+}
+
+}  // namespace moge
+
+using namespace moge;
+
+extern "C" {
+
+size_t moge_workspace_size(const moge_config *cfg) {
+    if (check_config(cfg) != MOGE_OK) return 0;
+    return carve_workspace(*cfg, nullptr).total;
+}
+
+const char *moge_last_error(void) { return g_last_error.c_str(); }
+
+int moge_check_device_errors(void *stream) {
+    MOGE_CU(cudaStreamSynchronize((cudaStream_t)stream), "cudaStreamSynchronize");
+    uint32_t w = 0, zero = 0;
+    MOGE_CU(cudaMemcpyFromSymbol(&w, g_error_word, sizeof(w)), "read device error word");
+    MOGE_CU(cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)), "clear device error word");
+    if (w & ERRBIT_TIMEOUT) return fail(MOGE_ERR_TIMEOUT, "a device-side wait timed out");
+    if (w & ERRBIT_INVARIANT) return fail(MOGE_ERR_DEVICE, "a kernel found a violated invariant");
+    return MOGE_OK;
+}
+
+int moge_route(const moge_config *cfg, const void *x, const void *w_router,
+               const float *logit_bias, int32_t *topk_idx, float *topk_w, int32_t *counts,
+               int32_t *offsets, int32_t *perm_src, int32_t *perm_dst, void *workspace,
+               void *stream) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    const moge_config c = *cfg;
+    cudaStream_t st = (cudaStream_t)stream;
+    MOGE_NEED4(counts, "counts");
+    MOGE_NEED4(offsets, "offsets");
+    if (c.T == 0) {
+        MOGE_CU(cudaMemsetAsync(counts, 0, sizeof(int32_t) * c.N, st), "memset counts");
+        MOGE_CU(cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (c.N + 1), st), "memset offsets");
+        return MOGE_OK;
+    }
+    MOGE_NEED(x, "x");
+    MOGE_NEED(w_router, "w_router");
+    if (logit_bias && !aligned4(logit_bias)) return fail(MOGE_ERR_UNSUPPORTED, "logit_bias misaligned");
+    MOGE_NEED4(topk_idx, "topk_idx");
+    MOGE_NEED4(topk_w, "topk_w");
+    MOGE_NEED4(perm_src, "perm_src");
+    MOGE_NEED4(perm_dst, "perm_dst");
+    MOGE_NEED(workspace, "workspace");
+    Workspace ws = carve_workspace(c, workspace);
+    MOGE_CU(launch_router(c, x, w_router, logit_bias, topk_idx, topk_w, ws.hist, ws.rank, num_sms(),
+                          st), "router launch");
+    MOGE_CU(launch_scan(c, ws.hist, ws.base, counts, offsets, nullptr, false, false, st),
+            "scan launch");
+    MOGE_CU(launch_finalize(c, topk_idx, ws.rank, ws.base, offsets, perm_src, perm_dst, st),
+            "finalize launch");
+    return MOGE_OK;
+}
+
+int moge_permute(const moge_config *cfg, const void *x, const int32_t *perm_src, void *x_perm,
+                 void *stream) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    if (cfg->T == 0) return MOGE_OK;
+    MOGE_NEED(x, "x");
+    MOGE_NEED4(perm_src, "perm_src");
+    MOGE_NEED(x_perm, "x_perm");
+    MOGE_CU(launch_gather_rows(*cfg, x, perm_src, x_perm, (cudaStream_t)stream), "permute launch");
+    return MOGE_OK;
+}
+
+static int run_ffn(const moge_config &c, const Plan &plan, int n_entries, const FfnOperands &op,
+                   cudaStream_t st, cudaEvent_t mid = nullptr) {
+    if (c.dtype == MOGE_BF16)
+        MOGE_CU(launch_ffn_tc(c, plan, n_entries, op, num_sms(), st, mid),
+                "grouped FFN (tcgen05) launch");
+    else
+        MOGE_CU(launch_ffn_f32(c, plan, n_entries, op, st, mid), "grouped FFN (fp32) launch");
+    return MOGE_OK;
+}
+
+int moge_grouped_ffn(const moge_config *cfg, const void *x_perm, const int32_t *offsets,
+                     const void *w_gate, const void *w_up, const void *w_down, void *y_perm,
+                     void *workspace, void *stream) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    const moge_config c = *cfg;
+    if (c.T == 0) return MOGE_OK;
+    MOGE_NEED(x_perm, "x_perm");
+    MOGE_NEED4(offsets, "offsets");
+    MOGE_NEED(w_gate, "w_gate");
+    MOGE_NEED(w_up, "w_up");
+    MOGE_NEED(w_down, "w_down");
+    MOGE_NEED(y_perm, "y_perm");
+    MOGE_NEED(workspace, "workspace");
+    cudaStream_t st = (cudaStream_t)stream;
+    Workspace ws = carve_workspace(c, workspace);
+    MOGE_CU(launch_plan(c, offsets, ws.plan, true, false, st), "plan launch");
+    const int64_t rows = (int64_t)c.T * c.M * c.Kp;
+    FfnOperands op{x_perm, nullptr, rows, 0, w_gate, w_up, w_down, nullptr, nullptr, nullptr,
+                   ws.h, rows, y_perm};
+    return run_ffn(c, ws.plan, c.N, op, st);
+}
+
+int moge_shared_ffn(const moge_config *cfg, const void *x, const void *s_gate, const void *s_up,
+                    const void *s_down, void *y_shared, void *workspace, void *stream) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    const moge_config c = *cfg;
+    if (c.T == 0) return MOGE_OK;
+    cudaStream_t st = (cudaStream_t)stream;
+    MOGE_NEED(y_shared, "y_shared");
+    const size_t esz = c.dtype == MOGE_BF16 ? 2 : 4;
+    if (c.S == 0) {
+        MOGE_CU(cudaMemsetAsync(y_shared, 0, (size_t)c.T * c.d * esz, st), "memset y_shared");
+        return MOGE_OK;
+    }
+    MOGE_NEED(x, "x");
+    MOGE_NEED(s_gate, "s_gate");
+    MOGE_NEED(s_up, "s_up");
+    MOGE_NEED(s_down, "s_down");
+    MOGE_NEED(workspace, "workspace");
+    Workspace ws = carve_workspace(c, workspace);
+    MOGE_CU(launch_plan(c, nullptr, ws.plan, false, true, st), "plan launch");
+    const int64_t rows = (int64_t)c.T * c.S;
+    FfnOperands op{nullptr, x, 0, c.T, nullptr, nullptr, nullptr, s_gate, s_up, s_down,
+                   ws.h, rows, ws.y_perm};
+    rc = run_ffn(c, ws.plan, c.S, op, st);
+    if (rc) return rc;
+    MOGE_CU(launch_combine(c, nullptr, nullptr, nullptr, 0, ws.y_perm, c.S, nullptr, y_shared, st),
+            "shared sum launch");
+    return MOGE_OK;
+}
+
+int moge_combine(const moge_config *cfg, const void *y_perm, const float *topk_w,
+                 const int32_t *perm_dst, const void *y_shared, const void *residual, void *y,
+                 void *stream) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    const moge_config c = *cfg;
+    if (c.T == 0) return MOGE_OK;
+    MOGE_NEED(y_perm, "y_perm");
+    MOGE_NEED4(topk_w, "topk_w");
+    MOGE_NEED4(perm_dst, "perm_dst");
+    MOGE_NEED(y, "y");
+    if (y_shared && !aligned16(y_shared)) return fail(MOGE_ERR_UNSUPPORTED, "y_shared misaligned");
+    if (residual && !aligned16(residual)) return fail(MOGE_ERR_UNSUPPORTED, "residual misaligned");
+    MOGE_CU(launch_combine(c, y_perm, topk_w, perm_dst, c.M * c.Kp, y_shared, y_shared ? 1 : 0,
+                           residual, y, (cudaStream_t)stream),
+            "combine launch");
+    return MOGE_OK;
+}
+
+int moge_layer_forward(const moge_config *cfg, const void *x, const void *w_router,
+                       const float *logit_bias, const void *w_gate, const void *w_up,
+                       const void *w_down, const void *s_gate, const void *s_up,
+                       const void *s_down, const void *residual, void *y, void *workspace,
+                       void *stream) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    const moge_config c = *cfg;
+    if (c.T == 0) return MOGE_OK;
+    MOGE_NEED(x, "x");
+    MOGE_NEED(w_router, "w_router");
+    MOGE_NEED(w_gate, "w_gate");
+    MOGE_NEED(w_up, "w_up");
+    MOGE_NEED(w_down, "w_down");
+    if (c.S > 0) {
+        MOGE_NEED(s_gate, "s_gate");
+        MOGE_NEED(s_up, "s_up");
+        MOGE_NEED(s_down, "s_down");
+    }
+    if (logit_bias && !aligned4(logit_bias)) return fail(MOGE_ERR_UNSUPPORTED, "logit_bias misaligned");
+    if (residual && !aligned16(residual)) return fail(MOGE_ERR_UNSUPPORTED, "residual misaligned");
+    MOGE_NEED(y, "y");
+    MOGE_NEED(workspace, "workspace");
+    if (y == x) return fail(MOGE_ERR_INVALID_ARG, "y must not alias x");
+    cudaStream_t st = (cudaStream_t)stream;
+    Workspace ws = carve_workspace(c, workspace);
+    const int K = c.M * c.Kp;
+    cudaEvent_t *ev = timer_slot();
+    if (ev) MOGE_CU(cudaEventRecord(ev[0], st), "event");
+    MOGE_CU(launch_router(c, x, w_router, logit_bias, ws.topk_idx, ws.topk_w, ws.hist, ws.rank,
+                          num_sms(), st), "router launch");
+    if (ev) MOGE_CU(cudaEventRecord(ev[1], st), "event");
+    MOGE_CU(launch_scan(c, ws.hist, ws.base, ws.counts, ws.offsets, &ws.plan, true, c.S > 0, st),
+            "scan launch");
+    if (ev) MOGE_CU(cudaEventRecord(ev[2], st), "event");
+    MOGE_CU(launch_scatter_rows(c, x, ws.topk_idx, ws.rank, ws.base, ws.offsets, ws.perm_src,
+                                ws.perm_dst, ws.x_perm, st), "permute launch");
+    if (ev) MOGE_CU(cudaEventRecord(ev[3], st), "event");
+    const int64_t rrows = (int64_t)c.T * K;
+    FfnOperands op{ws.x_perm, x, rrows, c.T, w_gate, w_up, w_down,
+                   c.S > 0 ? s_gate : nullptr, c.S > 0 ? s_up : nullptr, c.S > 0 ? s_down : nullptr,
+                   ws.h, rrows + (int64_t)c.T * c.S, ws.y_perm};
+    rc = run_ffn(c, ws.plan, c.N + c.S, op, st, ev ? ev[4] : nullptr);
+    if (rc) return rc;
+    if (ev) MOGE_CU(cudaEventRecord(ev[5], st), "event");
+    const size_t esz = c.dtype == MOGE_BF16 ? 2 : 4;
+    const void *shared_rows = static_cast<const char *>(ws.y_perm) + (size_t)rrows * c.d * esz;
+    MOGE_CU(launch_combine(c, ws.y_perm, ws.topk_w, ws.perm_dst, K, shared_rows, c.S, residual, y,
+                           st), "combine launch");
+    if (ev) MOGE_CU(cudaEventRecord(ev[6], st), "event");
+    return MOGE_OK;
+}
+
+int moge_layer_forward_host(const moge_config *cfg, const void *x_host, const void *w_router,
+                            const float *logit_bias, const void *w_gate, const void *w_up,
+                            const void *w_down, const void *s_gate, const void *s_up,
+                            const void *s_down, void *y_host, void *x_dev, void *y_dev,
+                            void *workspace, void *stream) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    const moge_config c = *cfg;
+    if (c.T == 0) return MOGE_OK;
+    if (!x_host || !y_host) return fail(MOGE_ERR_INVALID_ARG, "host buffer is NULL");
+    MOGE_NEED(x_dev, "x_dev");
+    MOGE_NEED(y_dev, "y_dev");
+    cudaStream_t st = (cudaStream_t)stream;
+    const size_t bytes = (size_t)c.T * c.d * (c.dtype == MOGE_BF16 ? 2 : 4);
+    MOGE_CU(cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, st), "copy x in");
+    rc = moge_layer_forward(cfg, x_dev, w_router, logit_bias, w_gate, w_up, w_down, s_gate, s_up,
+                            s_down, nullptr, y_dev, workspace, stream);
+    if (rc) return rc;
+    MOGE_CU(cudaMemcpyAsync(y_host, y_dev, bytes, cudaMemcpyDeviceToHost, st), "copy y out");
+    MOGE_CU(cudaStreamSynchronize(st), "cudaStreamSynchronize");
+    return MOGE_OK;
+}
+
+int moge_workspace_routing(const moge_config *cfg, void *workspace, int32_t **topk_idx,
+                           float **topk_w, int32_t **counts, int32_t **offsets) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    if (!workspace) return fail(MOGE_ERR_INVALID_ARG, "workspace is NULL");
+    Workspace ws = carve_workspace(*cfg, workspace);
+    if (topk_idx) *topk_idx = ws.topk_idx;
+    if (topk_w) *topk_w = ws.topk_w;
+    if (counts) *counts = ws.counts;
+    if (offsets) *offsets = ws.offsets;
+    return MOGE_OK;
+}
+
+int moge_rmsnorm(const moge_config *cfg, const void *x, float eps, void *u, void *stream) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    if (cfg->T == 0) return MOGE_OK;
+    MOGE_NEED(x, "x");
+    MOGE_NEED(u, "u");
+    if (!(eps >= 0.0f)) return fail(MOGE_ERR_INVALID_ARG, "eps must be >= 0");
+    MOGE_CU(launch_rmsnorm(*cfg, x, eps, u, (cudaStream_t)stream), "rmsnorm launch");
+    return MOGE_OK;
+}
+
+int moge_stage_timing(int enable) {
+    if (enable) {
+        for (int i = 0; i < kEventSets; ++i) g_timer.pending[i] = false;
+        for (int k = 0; k < kTimedStages; ++k) g_timer.total_ms[k] = 0.0;
+        g_timer.calls = 0;
+        g_timer.next = 0;
+    }
+    g_timer.enabled = enable != 0;
+    return MOGE_OK;
+}
+
+int moge_stage_times(double *ms_total, int64_t *calls) {
+    for (int i = 0; i < kEventSets; ++i)
+        MOGE_CU(timer_harvest(i), "stage timing events");
+    if (ms_total)
+        for (int k = 0; k < kTimedStages; ++k) ms_total[k] = g_timer.total_ms[k];
+    if (calls) *calls = g_timer.calls;
+    return MOGE_OK;
+}
+
+}  // extern "C"

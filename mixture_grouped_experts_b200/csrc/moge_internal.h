@@ -1,0 +1,110 @@
+// Internal declarations shared by the MoGE CUDA sources: the grouped-GEMM
+// work plan, the workspace layout and the kernel launchers used by api.cu.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/moge.h"
+
+namespace moge {
+
+// Tokens handled by one router tile (one CTA, or one cluster of CTAs that
+// split the hidden dimension).
+constexpr int kRouterTile = 16;
+constexpr int kMaxExperts = 256;
+
+// One expert's block of rows in a grouped GEMM launch.
+//   rows      rows of this expert (routed: counts[e]; shared: T)
+//   src_row0  first row in the B-operand matrix (x_perm / x / h)
+//   dst_row0  first row in the output matrix (h / y_perm)
+//   a_sel     0: routed weight tensors, 1: shared weight tensors
+//   a_idx     expert index inside the selected weight tensor
+//   b_sel     0: first B matrix (x_perm, or h), 1: second (x)
+//   bn        token-tile width (multiple of 16, <= 256)
+//   ntb       token tiles of this expert (ceil(rows / bn)), 0 if rows == 0
+struct ExpertWork {
+    int rows, src_row0, dst_row0, a_sel, a_idx, b_sel, bn, ntb;
+};
+
+// Token-tile widths: an expert with at most kStreamRows rows is one
+// "streaming" tile (two K-chunks per pipeline stage, weights are the
+// bandwidth-bound stream); larger experts use tensor tiles of up to 256 rows.
+constexpr int kStreamRows = 64;
+constexpr int kMaxTileN = 256;
+
+// Work plan of one layer call: an up-projection list and a down-projection list.
+struct Plan {
+    ExpertWork *up;     // [n_entries]
+    ExpertWork *down;   // [n_entries]
+    int *up_start;      // [n_entries + 1] prefix sum of items (ntb * feature blocks)
+    int *down_start;    // [n_entries + 1]
+};
+
+// Workspace carve-up (all regions 256-byte aligned).
+struct Workspace {
+    int32_t *hist;      // [tiles][N] per-tile expert counts
+    int32_t *base;      // [tiles][N] rows of expert e taken by earlier tiles
+    int32_t *rank;      // [T][K]     rank of (t, k) among its tile's tokens of that expert
+    int32_t *topk_idx;  // [T][K]
+    float *topk_w;      // [T][K]
+    int32_t *counts;    // [N]
+    int32_t *offsets;   // [N+1]
+    int32_t *perm_src;  // [T*K]
+    int32_t *perm_dst;  // [T][K]
+    Plan plan;          // N + S entries per list
+    void *x_perm;       // [T*K][d]      dtype
+    void *h;            // [T*(K+S)][I]  dtype
+    void *y_perm;       // [T*(K+S)][d]  dtype
+    size_t total;
+};
+Workspace carve_workspace(const moge_config &c, void *base);
+
+// ---------------------------------------------------------------- launchers
+// Each returns a cudaError_t of the launch.
+cudaError_t launch_router(const moge_config &c, const void *x, const void *w_router,
+                          const float *bias, int32_t *topk_idx, float *topk_w, int32_t *hist,
+                          int32_t *rank, int num_sms, cudaStream_t st);
+// counts/offsets/base from hist; when plan_* are given also the layer's GEMM plan
+cudaError_t launch_scan(const moge_config &c, const int32_t *hist, int32_t *base, int32_t *counts,
+                        int32_t *offsets, const Plan *plan, bool with_routed, bool with_shared,
+                        cudaStream_t st);
+// plan from caller offsets (routed only) or for shared experts only
+cudaError_t launch_plan(const moge_config &c, const int32_t *offsets, const Plan &plan,
+                        bool with_routed, bool with_shared, cudaStream_t st);
+cudaError_t launch_finalize(const moge_config &c, const int32_t *topk_idx, const int32_t *rank,
+                            const int32_t *base, const int32_t *offsets, int32_t *perm_src,
+                            int32_t *perm_dst, cudaStream_t st);
+cudaError_t launch_scatter_rows(const moge_config &c, const void *x, const int32_t *topk_idx,
+                                const int32_t *rank, const int32_t *base, const int32_t *offsets,
+                                int32_t *perm_src, int32_t *perm_dst, void *x_perm,
+                                cudaStream_t st);
+cudaError_t launch_gather_rows(const moge_config &c, const void *x, const int32_t *perm_src,
+                               void *x_perm, cudaStream_t st);
+cudaError_t launch_combine(const moge_config &c, const void *y_perm, const float *topk_w,
+                           const int32_t *perm_dst, int K, const void *shared_rows,
+                           int n_shared_blocks, const void *residual, void *y, cudaStream_t st);
+cudaError_t launch_rmsnorm(const moge_config &c, const void *x, float eps, void *u,
+                           cudaStream_t st);
+
+// Grouped SwiGLU FFN over a plan list (n_entries experts).
+struct FfnOperands {
+    const void *b0;          // up: x_perm (routed rows) ; down: h
+    const void *b1;          // up: x (shared rows)      ; down: unused
+    int64_t b0_rows, b1_rows;
+    const void *wg, *wu, *wd;  // routed weights [N][I][d], [N][I][d], [N][d][I]
+    const void *sg, *su, *sd;  // shared weights [S][I][d], [S][I][d], [S][d][I]
+    void *h;                 // [h_rows][I]
+    int64_t h_rows;
+    void *y;                 // [h_rows][d]
+};
+// `mid` (may be null) is recorded on the stream between the up- and the
+// down-projection launches.
+cudaError_t launch_ffn_tc(const moge_config &c, const Plan &plan, int n_entries,
+                          const FfnOperands &op, int num_sms, cudaStream_t st, cudaEvent_t mid);
+cudaError_t launch_ffn_f32(const moge_config &c, const Plan &plan, int n_entries,
+                           const FfnOperands &op, cudaStream_t st, cudaEvent_t mid);
+
+}  // namespace moge

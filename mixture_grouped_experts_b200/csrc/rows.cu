@@ -1,0 +1,215 @@
+// Row-wise kernels of the MoGE layer: the expert-major permutation of the
+// token rows (scatter form fused with the index finalisation, and the plain
+// gather form), the score-weighted combine with the shared experts and an
+// optional residual, and RMSNorm. All move rows as 16-byte vectors; these are
+// HBM-bound copies, so they use plain coalesced vector loads/stores and a
+// grid of one CTA per row.
+//
+// Combine weights are the picked experts' global softmax scores ("Huawei
+// releases Pangu Pro MoE", techwalker.com, section 1); shared experts are
+// always on with weight 1 (same page, section 2).
+#include "common.cuh"
+#include "moge_internal.h"
+
+namespace moge {
+
+constexpr int kRowThreads = 128;
+
+__device__ __forceinline__ int vec_elems(int dtype) { return dtype == MOGE_F32 ? 4 : 8; }
+
+// One CTA per token: computes the token's K destination rows, writes the
+// permutation indices and copies x[t] into each destination row.
+__global__ void __launch_bounds__(kRowThreads) scatter_rows_kernel(
+    moge_config c, const uint4 *__restrict__ x, const int32_t *__restrict__ topk_idx,
+    const int32_t *__restrict__ rank, const int32_t *__restrict__ base,
+    const int32_t *__restrict__ offsets, int32_t *perm_src, int32_t *perm_dst, uint4 *x_perm) {
+    __shared__ int dst_s[kMaxExperts];
+    const int t = blockIdx.x;
+    const int K = c.M * c.Kp;
+    const int nvec = c.d / vec_elems(c.dtype);
+    for (int k = threadIdx.x; k < K; k += blockDim.x) {
+        const size_t i = (size_t)t * K + k;
+        const int e = topk_idx[i];
+        int row = -1;
+        if (e >= 0 && e < c.N) {
+            row = offsets[e] + base[(size_t)(t / kRouterTile) * c.N + e] + rank[i];
+            perm_dst[i] = row;
+            perm_src[row] = t;
+        } else {
+            raise_error(ERRBIT_INVARIANT);
+        }
+        dst_s[k] = row;
+    }
+    __syncthreads();
+    const uint4 *src = x + (size_t)t * nvec;
+    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+        const uint4 val = src[v];
+        for (int k = 0; k < K; ++k) {
+            const int row = dst_s[k];
+            if (row >= 0) x_perm[(size_t)row * nvec + v] = val;
+        }
+    }
+}
+
+cudaError_t launch_scatter_rows(const moge_config &c, const void *x, const int32_t *topk_idx,
+                                const int32_t *rank, const int32_t *base, const int32_t *offsets,
+                                int32_t *perm_src, int32_t *perm_dst, void *x_perm,
+                                cudaStream_t st) {
+    scatter_rows_kernel<<<c.T, kRowThreads, 0, st>>>(c, (const uint4 *)x, topk_idx, rank, base,
+                                                     offsets, perm_src, perm_dst, (uint4 *)x_perm);
+    return cudaGetLastError();
+}
+
+// x_perm[r] = x[perm_src[r]], one CTA per destination row
+__global__ void __launch_bounds__(kRowThreads) gather_rows_kernel(
+    moge_config c, const uint4 *__restrict__ x, const int32_t *__restrict__ perm_src,
+    uint4 *x_perm) {
+    const int r = blockIdx.x;
+    const int nvec = c.d / vec_elems(c.dtype);
+    const int t = perm_src[r];
+    if (t < 0 || t >= c.T) {
+        if (threadIdx.x == 0) raise_error(ERRBIT_INVARIANT);
+        return;
+    }
+    const uint4 *src = x + (size_t)t * nvec;
+    uint4 *dst = x_perm + (size_t)r * nvec;
+    for (int v = threadIdx.x; v < nvec; v += blockDim.x) dst[v] = src[v];
+}
+
+cudaError_t launch_gather_rows(const moge_config &c, const void *x, const int32_t *perm_src,
+                               void *x_perm, cudaStream_t st) {
+    const int rows = c.T * c.M * c.Kp;
+    gather_rows_kernel<<<rows, kRowThreads, 0, st>>>(c, (const uint4 *)x, perm_src,
+                                                     (uint4 *)x_perm);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// y[t] = residual[t] + sum_k w[t][k] * y_perm[perm_dst[t][k]] + sum_b shared_b[t]
+// fp32 sums, k ascending, then the shared blocks in order, then the residual.
+template <int DT>
+__device__ __forceinline__ void load_vec(const void *p, size_t v, float (&f)[8]) {
+    if (DT == MOGE_BF16) {
+        const uint4 u = reinterpret_cast<const uint4 *>(p)[v];
+        f[0] = bf16_lo(u.x); f[1] = bf16_hi(u.x); f[2] = bf16_lo(u.y); f[3] = bf16_hi(u.y);
+        f[4] = bf16_lo(u.z); f[5] = bf16_hi(u.z); f[6] = bf16_lo(u.w); f[7] = bf16_hi(u.w);
+    } else {
+        const float4 a = reinterpret_cast<const float4 *>(p)[2 * v];
+        const float4 b = reinterpret_cast<const float4 *>(p)[2 * v + 1];
+        f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+        f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+    }
+}
+template <int DT>
+__device__ __forceinline__ void store_vec(void *p, size_t v, const float (&f)[8]) {
+    if (DT == MOGE_BF16) {
+        uint4 u;
+        u.x = pack_bf16x2(f[0], f[1]); u.y = pack_bf16x2(f[2], f[3]);
+        u.z = pack_bf16x2(f[4], f[5]); u.w = pack_bf16x2(f[6], f[7]);
+        reinterpret_cast<uint4 *>(p)[v] = u;
+    } else {
+        reinterpret_cast<float4 *>(p)[2 * v] = make_float4(f[0], f[1], f[2], f[3]);
+        reinterpret_cast<float4 *>(p)[2 * v + 1] = make_float4(f[4], f[5], f[6], f[7]);
+    }
+}
+
+// Vectors here are 8 elements (16 B in bf16, 32 B in fp32); d % 8 == 0.
+template <int DT>
+__global__ void __launch_bounds__(kRowThreads) combine_kernel(
+    int T, int d, int N, const void *__restrict__ y_perm, const float *__restrict__ topk_w,
+    const int32_t *__restrict__ perm_dst, int K, const void *__restrict__ shared_rows,
+    int n_shared, const void *residual, void *y) {
+    __shared__ int dst_s[kMaxExperts];
+    __shared__ float w_s[kMaxExperts];
+    const int t = blockIdx.x;
+    const int nvec = d / 8;
+    const size_t esz = DT == MOGE_BF16 ? 2 : 4;
+    for (int k = threadIdx.x; k < K; k += blockDim.x) {
+        const int row = perm_dst[(size_t)t * K + k];
+        if (row < 0 || row >= T * K) raise_error(ERRBIT_INVARIANT);
+        dst_s[k] = (row < 0 || row >= T * K) ? 0 : row;
+        w_s[k] = topk_w[(size_t)t * K + k];
+    }
+    __syncthreads();
+    (void)N;
+    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+        float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        for (int k = 0; k < K; ++k) {
+            float f[8];
+            load_vec<DT>((const char *)y_perm + (size_t)dst_s[k] * d * esz, v, f);
+            const float w = w_s[k];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] = fmaf(w, f[j], acc[j]);
+        }
+        for (int b = 0; b < n_shared; ++b) {
+            float f[8];
+            load_vec<DT>((const char *)shared_rows + ((size_t)b * T + t) * d * esz, v, f);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] += f[j];
+        }
+        if (residual) {
+            float f[8];
+            load_vec<DT>((const char *)residual + (size_t)t * d * esz, v, f);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] = f[j] + acc[j];
+        }
+        store_vec<DT>((char *)y + (size_t)t * d * esz, v, acc);
+    }
+}
+
+cudaError_t launch_combine(const moge_config &c, const void *y_perm, const float *topk_w,
+                           const int32_t *perm_dst, int K, const void *shared_rows,
+                           int n_shared_blocks, const void *residual, void *y, cudaStream_t st) {
+    if (c.dtype == MOGE_BF16)
+        combine_kernel<MOGE_BF16><<<c.T, kRowThreads, 0, st>>>(
+            c.T, c.d, c.N, y_perm, topk_w, perm_dst, K, shared_rows, n_shared_blocks, residual, y);
+    else
+        combine_kernel<MOGE_F32><<<c.T, kRowThreads, 0, st>>>(
+            c.T, c.d, c.N, y_perm, topk_w, perm_dst, K, shared_rows, n_shared_blocks, residual, y);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// u = x / sqrt(mean(x^2) + eps), unit gain; fp32 sum in a fixed tree order.
+template <int DT>
+__global__ void __launch_bounds__(kRowThreads) rmsnorm_kernel(int d, const void *__restrict__ x,
+                                                              float eps, void *u) {
+    __shared__ float red[kRowThreads / 32];
+    const int t = blockIdx.x;
+    const int nvec = d / 8;
+    const size_t esz = DT == MOGE_BF16 ? 2 : 4;
+    const char *xr = (const char *)x + (size_t)t * d * esz;
+    float ss = 0.0f;
+    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+        float f[8];
+        load_vec<DT>(xr, v, f);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) ss = fmaf(f[j], f[j], ss);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    float tot = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kRowThreads / 32; ++w) tot += red[w];
+    const float r = rsqrtf(tot / (float)d + eps);
+    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+        float f[8];
+        load_vec<DT>(xr, v, f);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) f[j] *= r;
+        store_vec<DT>((char *)u + (size_t)t * d * esz, v, f);
+    }
+}
+
+cudaError_t launch_rmsnorm(const moge_config &c, const void *x, float eps, void *u,
+                           cudaStream_t st) {
+    if (c.dtype == MOGE_BF16)
+        rmsnorm_kernel<MOGE_BF16><<<c.T, kRowThreads, 0, st>>>(c.d, x, eps, u);
+    else
+        rmsnorm_kernel<MOGE_F32><<<c.T, kRowThreads, 0, st>>>(c.d, x, eps, u);
+    return cudaGetLastError();
+}
+
+}  // namespace moge

@@ -1,0 +1,96 @@
+"""The C-ABI library loads and exports every symbol include/moge.h declares;
+host-side argument checks reject bad calls before any device work (no GPU needed)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import mixture_grouped_experts_b200 as mg
+from mixture_grouped_experts_b200 import build as mbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moge.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    mbuild.build()
+    return mg.lib()
+
+
+def declared_symbols():
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"MOGE_API\s+[\w\s\*]*?\b(moge_\w+)\s*\(", txt)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_symbols()
+    for n in ("moge_route", "moge_permute", "moge_grouped_ffn", "moge_combine", "moge_layer_forward"):
+        assert n in names
+    assert set(names) == set(mg.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    out = subprocess.check_output(["nm", "-D", "--defined-only", mg.LIB_PATH], text=True)
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    for n in declared_symbols():
+        assert n in exported, n
+        assert getattr(L, n) is not None
+    # nothing else leaks out of the library under the moge_ prefix
+    assert {e for e in exported if e.startswith("moge_")} == set(declared_symbols())
+
+
+def _shape(**kw):
+    base = dict(T=64, d=256, N=16, M=4, Kp=1, S=1, I=128, dtype="f32")
+    base.update(kw)
+    return mg.LayerShape(**base)
+
+
+def test_workspace_size_matches_layout(L):
+    s = _shape()
+    n = mg.workspace_size(s)
+    K = s.M * s.Kp
+    big = s.T * K * s.d * 4 + s.T * (K + s.S) * (s.I + s.d) * 4
+    assert big < n < big + 64 * 1024
+    b = mg.workspace_size(_shape(dtype="bf16"))
+    assert b < n                                   # bf16 rows take half the bytes
+    assert mg.workspace_size(_shape(T=0)) > 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(N=15), mg.ERR_UNSUPPORTED),               # N % M != 0
+    (dict(Kp=5), mg.ERR_UNSUPPORTED),               # Kp > N/M
+    (dict(d=100), mg.ERR_UNSUPPORTED),              # d % 8 != 0
+    (dict(I=12), mg.ERR_UNSUPPORTED),               # I % 8 != 0
+    (dict(N=512, M=4), mg.ERR_UNSUPPORTED),         # N > 256
+    (dict(T=-1), mg.ERR_INVALID_ARG),
+    (dict(M=0), mg.ERR_INVALID_ARG),
+    (dict(N=12, M=4, dtype="bf16"), mg.ERR_UNSUPPORTED),  # bf16 router needs N % 8 == 0
+])
+def test_invalid_configs_rejected_on_host(L, kw, code):
+    s = _shape(**kw)
+    assert L.moge_workspace_size(ctypes.byref(mg._cfg(s))) == 0
+    rc = L.moge_route(ctypes.byref(mg._cfg(s)), *([None] * 11))
+    assert rc == code
+    assert len(L.moge_last_error()) > 0
+
+
+def test_null_and_misaligned_pointers_rejected(L):
+    s = _shape()
+    c = ctypes.byref(mg._cfg(s))
+    assert L.moge_layer_forward(c, *([None] * 13)) == mg.ERR_INVALID_ARG
+    assert b"x" in L.moge_last_error()
+    # misaligned (odd) pointers are refused before anything is enqueued
+    rc = L.moge_permute(c, 0x1001, 0x2000, 0x3000, None)
+    assert rc == mg.ERR_UNSUPPORTED and b"aligned" in L.moge_last_error()
+    rc = L.moge_rmsnorm(c, 0x1000, ctypes.c_float(-1.0), 0x2000, None)
+    assert rc == mg.ERR_INVALID_ARG
+
+
+def test_no_cpu_fallback_when_library_missing(monkeypatch):
+    monkeypatch.setattr(mg, "_lib", None)
+    monkeypatch.setattr(mg, "LIB_PATH", "/nonexistent/libmoge.so")
+    with pytest.raises(ImportError):
+        mg.lib()
