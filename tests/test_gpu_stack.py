@@ -5,9 +5,12 @@ Two checks per layer and one end to end:
   * teacher forcing: the GPU's own layer input bytes (RMSNorm output) are fed
     to the oracle; the GPU layer output (no residual) on sampled tokens must
     match it, routing bit-exact above the margin;
-  * end to end: candidate tokens carried through the oracle's fp64 stack;
-    those whose picks agree with the GPU's at every layer (a pick under the
-    margin may legitimately flip with bf16 drift) must match at the end.
+  * end to end: bf16 drift may flip a pick whose margin is small, after which
+    the two stacks legitimately differ. So the oracle's scores on the GPU's own
+    layer inputs give every token its smallest in-group margin over the 12
+    layers; the tokens with the widest margins (all > 1e-3) are carried
+    through the oracle's fp64 stack, must keep the GPU's picks at every layer,
+    and must match at the end.
 """
 import gc
 
@@ -23,17 +26,21 @@ from gpu_helpers import MARGIN, TOL, normwise_err, to_host_f64
 pytestmark = pytest.mark.gpu
 
 
+def _free():
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
 def test_stack12_teacher_forced_and_end_to_end():
     cfg = synth.CONFIGS["stack12"]
     s = mg.shape_of(cfg)
     ws = mg.alloc_workspace(s)
     x0 = synth.normal(cfg.seed, synth.STREAM_X, cfg.T * cfg.d, cfg.x_std, "bf16").reshape(cfg.T, cfg.d)
     x_dev = mg.to_device(x0, "bf16")
-    cand = np.array([3, 50, 101, 222, 333, 455])
-    xo = oracle.to_double(x0, "bf16")[cand]
-    agree = np.ones(len(cand), bool)
+    min_margin = np.full(cfg.T, np.inf)
+    idx_all = []
     checked = 0
-    for l in range(cfg.layers):
+    for l in range(cfg.layers):                   # pass 1: the GPU stack
         inp = synth.layer_inputs(cfg, layer=l, with_x=False)
         w = mg.weights_to_device(inp, "bf16")
         u = mg.moge_rmsnorm(s, x_dev, 1e-6)
@@ -42,8 +49,12 @@ def test_stack12_teacher_forced_and_end_to_end():
         idx_g = mg.moge_workspace_routing(s, ws)[0].cpu().numpy()
         torch.cuda.synchronize()
         mg.check_device_errors()
-        # teacher forcing on two tokens per layer
+        idx_all.append(idx_g)
         u_h = to_host_f64(u)
+        p = oracle.router_probs(u_h, inp["w_router"], None, "bf16")
+        _, _, mgn = oracle.select_grouped(p, cfg.M, cfg.Kp)
+        min_margin = np.minimum(min_margin, mgn)
+        # teacher forcing on two tokens per layer
         tf = np.array([(37 * l + 11) % cfg.T, (91 * l + 5) % cfg.T])
         y_ref, idx_ref, _, mg_ref = oracle.layer(u_h, inp, cfg.M, cfg.Kp, "bf16", tokens=tf)
         yg = to_host_f64(y_only)[tf]
@@ -52,17 +63,18 @@ def test_stack12_teacher_forced_and_end_to_end():
                 assert np.array_equal(idx_ref[j], idx_g[t]), (l, t)
                 assert normwise_err(yg[j], y_ref[j]) <= TOL["bf16"], (l, t)
                 checked += 1
-        # the oracle's own fp64 stack for the candidates
-        uo = oracle.rmsnorm(xo, 1e-6)
-        yo, idx_o, _, _ = oracle.layer(uo, inp, cfg.M, cfg.Kp, "bf16")
-        agree &= (idx_o == idx_g[cand]).all(1)
-        xo = xo + yo
         x_dev = x_next
         del w, inp, u, y_only
-        gc.collect()
-        torch.cuda.empty_cache()
+        _free()
     assert checked >= cfg.layers
-    assert agree.sum() >= 2, agree
-    xg = to_host_f64(x_dev)[cand[agree]]
-    err = normwise_err(xg, xo[agree])
+    cand = np.argsort(-min_margin)[:4]
+    assert np.all(min_margin[cand] > 1e-3), min_margin[cand]
+    xo = oracle.to_double(x0, "bf16")[cand]
+    for l in range(cfg.layers):                   # pass 2: the oracle's fp64 stack
+        inp = synth.layer_inputs(cfg, layer=l, with_x=False)
+        yo, idx_o, _, _ = oracle.layer(oracle.rmsnorm(xo, 1e-6), inp, cfg.M, cfg.Kp, "bf16")
+        assert np.array_equal(idx_o, idx_all[l][cand]), l
+        xo = xo + yo
+        del inp
+    err = normwise_err(to_host_f64(x_dev)[cand], xo)
     assert err <= TOL["bf16"], err
