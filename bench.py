@@ -252,7 +252,8 @@ def main():
     ap.add_argument("--impl", default="moge", choices=["moge", "reference"])
     ap.add_argument("--config", default="decode", choices=["decode", "prefill", "skew"])
     ap.add_argument("--no-secondary", action="store_true", help="skip the prefill side measurement")
-    ap.add_argument("--cpu-tokens", type=int, default=16, help="tokens in the CPU-baseline sample")
+    ap.add_argument("--cpu-tokens", type=int, default=16, help="tokens in the CPU-baseline sample (0: skip)")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--ref-tokens", type=int, default=2, help="tokens per step of --impl reference")
     args = ap.parse_args()
     cfg = synth.CONFIGS[args.config]
@@ -279,10 +280,10 @@ def main():
     inp = synth.layer_inputs(cfg, x_stream_offset=rank)
     sampler = ClockSampler(local)
     sampler.start()
-    m = measure(cfg, inp, args.steps, args.warmup, dist_on)
+    m = measure(cfg, inp, args.steps, args.warmup, dist_on, with_e2e=not args.no_e2e)
     clocks = sampler.stop()
     ms = max_over_ranks(m["ms"], dist_on)
-    e2e_ms = max_over_ranks(m["e2e_ms"], dist_on)
+    e2e_ms = max_over_ranks(m.get("e2e_ms", float("nan")), dist_on)
     n = world
     value = n * cfg.T / (ms / 1e3)
 
@@ -307,11 +308,11 @@ def main():
                                "algorithmic_bytes": lb},
             "stage_ms": su,
             "e2e": {"value": n * cfg.T / (e2e_ms / 1e3), "unit": "tokens/s",
-                    "h2d_bytes_per_step": m["io_bytes"], "d2h_bytes_per_step": m["io_bytes"],
+                    "h2d_bytes_per_step": m.get("io_bytes"), "d2h_bytes_per_step": m.get("io_bytes"),
                     "api": "moge_layer_forward_host (pinned host x in, host y out, synchronised per step)"},
             "gpu_launches": 6 * args.steps,
             "clocks": clocks}
-    if rank == 0 and n == 1:
+    if rank == 0 and n == 1 and args.cpu_tokens > 0:
         line["cpu_baseline"] = cpu_baseline(cfg, inp, args.cpu_tokens)
     del inp
     if rank == 0 and n == 1 and not args.no_secondary and args.config == "decode":

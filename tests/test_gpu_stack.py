@@ -8,7 +8,7 @@ Two checks per layer and one end to end:
   * end to end: bf16 drift may flip a pick whose margin is small, after which
     the two stacks legitimately differ. So the oracle's scores on the GPU's own
     layer inputs give every token its smallest in-group margin over the 12
-    layers; the tokens with the widest margins (all > 1e-3) are carried
+    layers; the tokens with the widest margins (all > 5e-4) are carried
     through the oracle's fp64 stack, must keep the GPU's picks at every layer,
     and must match at the end.
 """
@@ -68,7 +68,7 @@ def test_stack12_teacher_forced_and_end_to_end():
         _free()
     assert checked >= cfg.layers
     cand = np.argsort(-min_margin)[:4]
-    assert np.all(min_margin[cand] > 1e-3), min_margin[cand]
+    assert np.all(min_margin[cand] > 5e-4), min_margin[cand]
     xo = oracle.to_double(x0, "bf16")[cand]
     for l in range(cfg.layers):                   # pass 2: the oracle's fp64 stack
         inp = synth.layer_inputs(cfg, layer=l, with_x=False)
