@@ -10,7 +10,10 @@ Two checks per layer and one end to end:
     layer inputs give every token its smallest in-group margin over the 12
     layers; the tokens with the widest margins (all > 5e-4) are carried
     through the oracle's fp64 stack, must keep the GPU's picks at every layer,
-    and must match at the end.
+    and must match at the end within sqrt(L) * 1e-2: every layer is held to
+    1e-2 of its own output (checked above) and the L layers' independent bf16
+    rounding errors, plus the bf16 rounding of the residual after each layer,
+    add up roughly in quadrature.
 """
 import gc
 
@@ -77,4 +80,4 @@ def test_stack12_teacher_forced_and_end_to_end():
         xo = xo + yo
         del inp
     err = normwise_err(to_host_f64(x_dev)[cand], xo)
-    assert err <= TOL["bf16"], err
+    assert err <= np.sqrt(cfg.layers) * TOL["bf16"], err
