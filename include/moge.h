@@ -164,6 +164,27 @@ MOGE_API int moge_workspace_routing(const moge_config *cfg, void *workspace, int
  * section 2 of the article above, its form here is a stated choice). */
 MOGE_API int moge_rmsnorm(const moge_config *cfg, const void *x, float eps, void *u, void *stream);
 
+/* moge_route without a workspace, for callers that may not allocate device
+ * memory on their calling path (a plugin inside a runtime whose device memory
+ * is all pre-reserved by its own pool; a latency-bound serving loop where
+ * cudaMalloc/cudaFree would synchronise the device). The pages describe no
+ * such call; it exists for this library's users only.
+ * Same arguments and results as moge_route, minus `workspace`: the routing
+ * scratch (per-tile histograms, row bases, ranks) lives in a fixed 1 MiB array
+ * inside the library's device image, held by every GPU that loads the library
+ * until the process exits. Limit: 2*round256(ceil(T/16)*N*4) +
+ * round256(T*K*4) <= 1048576 bytes (e.g. T <= 16384 at N = 64, K = 8);
+ * larger batches return MOGE_ERR_UNSUPPORTED with a message. Allocates
+ * nothing. The first call on a device (with that device current) looks up the
+ * array's device address; make that first call before any stream capture.
+ * All calls on a device share the array: calls that overlap on the GPU race,
+ * so order them on one stream. Nothing in the array needs clearing between
+ * calls (each call writes every scratch word it reads). */
+MOGE_API int moge_route_noalloc(const moge_config *cfg, const void *x, const void *w_router,
+                                const float *logit_bias, int32_t *topk_idx, float *topk_w,
+                                int32_t *counts, int32_t *offsets, int32_t *perm_src,
+                                int32_t *perm_dst, void *stream);
+
 /* Stage timing (measurement aid): while enabled, every moge_layer_forward
  * records CUDA events around its six launches -- router, scan, permute,
  * up-projection, down-projection, combine -- and the library adds up their

@@ -29,7 +29,7 @@ _TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16}
 EXPORTS = ["moge_workspace_size", "moge_last_error", "moge_check_device_errors", "moge_route",
            "moge_permute", "moge_grouped_ffn", "moge_shared_ffn", "moge_combine",
            "moge_layer_forward", "moge_layer_forward_host", "moge_workspace_routing",
-           "moge_rmsnorm", "moge_stage_timing", "moge_stage_times"]
+           "moge_rmsnorm", "moge_stage_timing", "moge_stage_times", "moge_route_noalloc"]
 STAGES = ("router", "scan", "permute", "ffn_up", "ffn_down", "combine")
 
 
@@ -94,6 +94,7 @@ def lib() -> ctypes.CDLL:
         L.moge_workspace_routing.argtypes = [cp, vp] + [ctypes.POINTER(vp)] * 4
         L.moge_rmsnorm.argtypes = [cp, vp, ctypes.c_float, vp, vp]
         L.moge_stage_timing.argtypes = [i32]
+        L.moge_route_noalloc.argtypes = [cp] + [vp] * 10
         L.moge_stage_times.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]
         for n in EXPORTS:
             if n not in ("moge_workspace_size", "moge_last_error"):
@@ -155,6 +156,23 @@ def moge_route(s: LayerShape, x, w_router, logit_bias, workspace, stream=None):
     _chk(lib().moge_route(ctypes.byref(_cfg(s)), _p(x), _p(w_router), _p(logit_bias), _p(idx),
                           _p(w), _p(counts), _p(offsets), _p(ps), _p(pd), _p(workspace),
                           _stream(stream)))
+    return idx, w, counts, offsets, ps[:T * K], pd
+
+
+def moge_route_noalloc(s: LayerShape, x, w_router, logit_bias, stream=None):
+    """moge_route with its scratch in the library's fixed device array (no
+    workspace, nothing allocated by the library); same results."""
+    dev = x.device
+    T, K, N = s.T, s.K, s.N
+    idx = torch.empty((T, K), dtype=torch.int32, device=dev)
+    w = torch.empty((T, K), dtype=torch.float32, device=dev)
+    counts = torch.empty(N, dtype=torch.int32, device=dev)
+    offsets = torch.empty(N + 1, dtype=torch.int32, device=dev)
+    ps = torch.empty(max(T * K, 1), dtype=torch.int32, device=dev)
+    pd = torch.empty((T, K), dtype=torch.int32, device=dev)
+    _chk(lib().moge_route_noalloc(ctypes.byref(_cfg(s)), _p(x), _p(w_router), _p(logit_bias),
+                                  _p(idx), _p(w), _p(counts), _p(offsets), _p(ps), _p(pd),
+                                  _stream(stream)))
     return idx, w, counts, offsets, ps[:T * K], pd
 
 

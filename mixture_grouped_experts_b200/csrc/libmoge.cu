@@ -4,3 +4,4 @@
 #include "gemm_f32.cu"
 #include "gemm_tc.cu"
 #include "api.cu"
+#include "route_noalloc.cu"
