@@ -38,7 +38,7 @@
  * Weight layouts follow the nn.Linear [out][in] convention:
  *   w_router [N][d]; w_gate, w_up [N][I][d]; w_down [N][d][I]
  *   s_gate, s_up [S][I][d]; s_down [S][d][I]
- * Size limits: 1 <= N <= 256, N % M == 0, 1 <= Kp <= N/M, d % 8 == 0,
+ * Size limits: 1 <= N <= 256, 0 <= S <= 256, N % M == 0, 1 <= Kp <= N/M, d % 8 == 0,
  * I % 8 == 0, T*(M*Kp+S) < 2^31 (else MOGE_ERR_UNSUPPORTED).
  */
 #ifndef MOGE_H

@@ -30,6 +30,7 @@ static int check_config(const moge_config *c) {
     if (c->dtype != MOGE_F32 && c->dtype != MOGE_BF16)
         return fail(MOGE_ERR_INVALID_ARG, "dtype must be MOGE_F32 or MOGE_BF16");
     if (c->N > kMaxExperts) return fail(MOGE_ERR_UNSUPPORTED, "N > 256");
+    if (c->S > kMaxExperts) return fail(MOGE_ERR_UNSUPPORTED, "S > 256");
     if (c->N % c->M != 0) return fail(MOGE_ERR_UNSUPPORTED, "N is not a multiple of M");
     if (c->Kp > c->N / c->M) return fail(MOGE_ERR_UNSUPPORTED, "Kp > N/M");
     if (c->d % 8 != 0 || c->I % 8 != 0)

@@ -36,10 +36,17 @@ constexpr int kStageBytes = 48 * 1024;
 constexpr int kEpiBytes = 12 * 1024;
 constexpr int kTcThreads = 192;
 constexpr int kChunkK = 64;          // bf16 elements per K-chunk (128 bytes, one swizzle row)
-constexpr int kBoxRows = 32;         // token rows per TMA box
+constexpr int kBoxRows = 64;         // token rows per TMA box (one 8 KB copy per chunk)
 constexpr uint32_t kTmemCols = 512;  // two accumulators of 256 columns
 
+// How the up-projection's 128-row weight tile is fetched, per weight side
+// (routed / shared): one 16 KB copy from a 4-D map over both tensors when
+// w_up lies wholly after w_gate (kGateUpFused) or wholly before it
+// (kUpGateFused: the tile then holds up rows first), else two 8 KB copies.
+enum : int { kGateUpSplit = 0, kGateUpFused = 1, kUpGateFused = 2 };
+
 struct TcParams {
+    int gu_mode[2];  // per a_sel
     const ExpertWork *work;
     const int *item_start;
     int n_entries;
@@ -82,6 +89,16 @@ struct TcShared {
     int abort;
     int epi_ok;
 };
+
+// K-chunk processed at step i of an item of feature block fb: items of the
+// same expert run side by side and read the same token rows, so each feature
+// block starts at a different chunk (an L2 hot spot otherwise). The order is
+// fixed per item, so results stay deterministic.
+__device__ __forceinline__ int chunk_at(int i, int fb, int k_chunks) {
+    const int r = (fb * 2 * 5) % k_chunks;  // even start: streaming pairs stay aligned
+    const int c = i + r;
+    return c >= k_chunks ? c - k_chunks : c;
+}
 
 // smem byte offsets of chunk c of a stage
 __device__ __forceinline__ uint32_t a_off(bool stream, int c) { return stream ? c * 24576u : 0u; }
@@ -166,12 +183,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
                     armed |= 1u << stage;
                     armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
                     for (int c = 0; c < nch; ++c) {
-                        const int k = (kc + c) * kChunkK;
+                        const int k = chunk_at(kc + c, it.fb, p.k_chunks) * kChunkK;
                         unsigned char *sa = sbase + a_off(it.stream, c);
                         unsigned char *sb = sbase + b_off(it.stream, c);
                         if (UP) {
-                            tma_load_3d(sa, ma0, &sh.full[stage], k, arow0, it.w.a_idx, pol_w);
-                            tma_load_3d(sa + 8192, ma1, &sh.full[stage], k, arow0, it.w.a_idx, pol_w);
+                            if (p.gu_mode[it.w.a_sel] != kGateUpSplit) {
+                                tma_load_4d(sa, ma0, &sh.full[stage], k, arow0, it.w.a_idx, 0, pol_w);
+                            } else {
+                                tma_load_3d(sa, ma0, &sh.full[stage], k, arow0, it.w.a_idx, pol_w);
+                                tma_load_3d(sa + 8192, ma1, &sh.full[stage], k, arow0, it.w.a_idx, pol_w);
+                            }
                         } else {
                             tma_load_3d(sa, ma0, &sh.full[stage], k, arow0, it.w.a_idx, pol_w);
                         }
@@ -254,14 +275,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
                 if (UP) {
                     float *U = reinterpret_cast<float *>(epi);                 // [32 cols][64 features]
                     uint16_t *H = reinterpret_cast<uint16_t *>(epi + 8192);    // [32 cols][64 features]
-                    if (q >= 2) {
-                        const int f = (q - 2) * 32 + lane;
+                    // lanes 0-63 hold gate and 64-127 up, or the reverse for an up-first tile
+                    const bool gate_hi = p.gu_mode[it.w.a_sel] == kUpGateFused;
+                    const bool is_gate = (q < 2) != gate_hi;
+                    const int f = (q & 1) * 32 + lane;
+                    if (!is_gate) {
 #pragma unroll
                         for (int j = 0; j < 32; ++j) U[j * 64 + f] = __uint_as_float(v[j]);
                     }
                     named_bar_sync(1, 128);
-                    if (q < 2) {
-                        const int f = q * 32 + lane;
+                    if (is_gate) {
 #pragma unroll
                         for (int j = 0; j < 32; ++j) {
                             const float g = __uint_as_float(v[j]);
@@ -336,10 +359,6 @@ static bool encode_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t
     const cuuint32_t box[3] = {(cuuint32_t)kChunkK, box_rows, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     const cuuint32_t rank = outer > 1 ? 3 : 2;
-    if (rank == 2) {
-        // a 2-D map still receives the 3-D coordinate form only for weights;
-        // weights always use rank 3 below (outer may be 1)
-    }
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), dims,
                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -358,6 +377,42 @@ static bool encode_weights(CUtensorMap *m, const void *base, uint64_t cols, uint
               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+// One map over both the gate and the up tensor ([E][rows][cols] each, dense):
+// dims {cols, rows, E, 2}, the last dimension stepping from one tensor to the
+// other, so a {64, 64, 1, 2} box is one 16 KB copy of 64 gate rows followed by
+// the 64 matching up rows. Strides must increase, so this needs the two
+// tensors not to overlap; the tensor at the lower address becomes the first
+// half of the tile. Returns kGateUpSplit when they overlap (or on failure),
+// and the caller then uses two 3-D maps.
+static int encode_gate_up(CUtensorMap *m, const void *gate, const void *up, uint64_t cols,
+                          uint64_t rows, uint64_t experts) {
+    EncodeTiledFn fn = get_encode_fn();
+    if (!fn) return kGateUpSplit;
+    const int64_t bytes = (int64_t)(cols * rows * experts * 2);
+    const int64_t delta = static_cast<const char *>(up) - static_cast<const char *>(gate);
+    int mode;
+    const void *base;
+    if (delta >= bytes) {
+        mode = kGateUpFused;
+        base = gate;
+    } else if (-delta >= bytes) {
+        mode = kUpGateFused;
+        base = up;
+    } else {
+        return kGateUpSplit;
+    }
+    const uint64_t step = (uint64_t)(delta >= 0 ? delta : -delta);
+    if (step % 16 != 0 || step >= (1ull << 40)) return kGateUpSplit;
+    const cuuint64_t dims[4] = {cols, rows, experts, 2};
+    const cuuint64_t strides[3] = {cols * 2, cols * rows * 2, step};
+    const cuuint32_t box[4] = {(cuuint32_t)kChunkK, 64, 1, 2};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? mode : kGateUpSplit;
+}
+
 static bool encode_rows(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows) {
     return encode_map(m, base, cols, rows, 1, kBoxRows);
 }
@@ -380,9 +435,16 @@ cudaError_t launch_ffn_tc(const moge_config &c, const Plan &plan, int n_entries,
     const int64_t r0 = op.b0 ? op.b0_rows : op.b1_rows, r1 = op.b1 ? op.b1_rows : op.b0_rows;
 
     CUtensorMap mWg, mWu, mSg, mSu, mX0, mX1, mWd, mSd, mH;
-    if (!encode_weights(&mWg, wg, d, I, ne, 64) || !encode_weights(&mWu, wu, d, I, ne, 64) ||
-        !encode_weights(&mSg, sg, d, I, ns, 64) || !encode_weights(&mSu, su, d, I, ns, 64) ||
-        !encode_rows(&mX0, b0, d, (uint64_t)r0) || !encode_rows(&mX1, b1, d, (uint64_t)r1) ||
+    int gu_mode[2];
+    gu_mode[0] = encode_gate_up(&mWg, wg, wu, d, I, ne);
+    gu_mode[1] = encode_gate_up(&mSg, sg, su, d, I, ns);
+    if (gu_mode[0] != kGateUpSplit) mWu = mWg;
+    else if (!encode_weights(&mWg, wg, d, I, ne, 64) || !encode_weights(&mWu, wu, d, I, ne, 64))
+        return cudaErrorInvalidValue;
+    if (gu_mode[1] != kGateUpSplit) mSu = mSg;
+    else if (!encode_weights(&mSg, sg, d, I, ns, 64) || !encode_weights(&mSu, su, d, I, ns, 64))
+        return cudaErrorInvalidValue;
+    if (!encode_rows(&mX0, b0, d, (uint64_t)r0) || !encode_rows(&mX1, b1, d, (uint64_t)r1) ||
         !encode_weights(&mWd, wd, I, d, ne, 128) || !encode_weights(&mSd, sd, I, d, ns, 128) ||
         !encode_rows(&mH, op.h, I, (uint64_t)op.h_rows))
         return cudaErrorInvalidValue;
@@ -395,14 +457,14 @@ cudaError_t launch_ffn_tc(const moge_config &c, const Plan &plan, int n_entries,
                              (int)smem);
     if (e != cudaSuccess) return e;
 
-    TcParams pu{plan.up, plan.up_start, n_entries, (d + kChunkK - 1) / kChunkK, I,
-                (uint16_t *)op.h};
+    TcParams pu{{gu_mode[0], gu_mode[1]}, plan.up, plan.up_start, n_entries,
+                (d + kChunkK - 1) / kChunkK, I, (uint16_t *)op.h};
     ffn_tc_kernel<true><<<num_sms, kTcThreads, smem, st>>>(pu, mWg, mWu, mSg, mSu, mX0, mX1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (mid && (e = cudaEventRecord(mid, st)) != cudaSuccess) return e;
-    TcParams pd{plan.down, plan.down_start, n_entries, (I + kChunkK - 1) / kChunkK, d,
-                (uint16_t *)op.y};
+    TcParams pd{{kGateUpSplit, kGateUpSplit}, plan.down, plan.down_start, n_entries,
+                (I + kChunkK - 1) / kChunkK, d, (uint16_t *)op.y};
     ffn_tc_kernel<false><<<num_sms, kTcThreads, smem, st>>>(pd, mWd, mWd, mSd, mSd, mH, mH);
     return cudaGetLastError();
 }

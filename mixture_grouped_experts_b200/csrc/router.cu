@@ -23,8 +23,7 @@ constexpr int kRouterThreads = kRouterWarps * 32;
 // -> scores, picks, per-tile histogram, in-tile ranks.
 struct RouterSmem {
     float logits[kRouterTile][kMaxExperts];
-    float part[kRouterWarps][kRouterTile][64];  // per-warp partial sums (bf16 path)
-    int ids[kRouterTile][kMaxExperts];          // picks, [t][k], k < K
+    int16_t ids[kRouterTile][kMaxExperts];  // picks, [t][k], k < K
 };
 
 // Order of candidates inside a group: higher score first, equal scores ->
@@ -37,9 +36,10 @@ __device__ void router_epilogue(RouterSmem &sm, const moge_config &c, const floa
                                 int32_t *topk_idx, float *topk_w, int32_t *hist, int32_t *rank) {
     const int N = c.N, M = c.M, Kp = c.Kp, K = M * Kp, G = N / M;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nwarps = blockDim.x >> 5;
     const int ntok = min(kRouterTile, c.T - t0);
     // one warp per token: global softmax over all N experts, fp32
-    for (int tt = warp; tt < ntok; tt += kRouterWarps) {
+    for (int tt = warp; tt < ntok; tt += nwarps) {
         float m = -INFINITY;
         for (int e = lane; e < N; e += 32) {
             float l = sm.logits[tt][e] + (bias ? bias[e] : 0.0f);
@@ -71,7 +71,7 @@ __device__ void router_epilogue(RouterSmem &sm, const moge_config &c, const floa
                     if (prev >= 0 && !ranks_before(pprev, prev, pe, e)) continue;
                     if (best < 0 || ranks_before(pe, e, pb, best)) { best = e; pb = pe; }
                 }
-                sm.ids[tt][g * Kp + j] = best;
+                sm.ids[tt][g * Kp + j] = (int16_t)best;
                 const size_t o = (size_t)(t0 + tt) * K + g * Kp + j;
                 topk_idx[o] = best;
                 topk_w[o] = pb;
@@ -103,15 +103,21 @@ __device__ void router_epilogue(RouterSmem &sm, const moge_config &c, const floa
 
 // ---------------------------------------------------------------------------
 // bf16 router GEMM with mma.sync m16n8k16 (the N <= 256 output columns are far
-// too narrow for a tcgen05 tile to pay). A cluster of `ks` CTAs splits the
-// hidden dimension of one 16-token tile; rank 0 reduces the partial logits
-// through distributed shared memory in a fixed order (deterministic).
+// too narrow for a tcgen05 tile to pay). One CTA owns 16 tokens and a slice of
+// the hidden dimension; a cluster of `ks` CTAs splits the hidden dimension of
+// one tile and the leader adds the partial logits in rank order
+// (deterministic). The CTA copies its x rows and router rows block by block
+// into shared memory with cp.async (every load of a block in flight at once,
+// two blocks double-buffered); warp w owns the n-tiles w, w+8, ... (8 experts
+// each), so no reduction across warps is needed.
 //
 // k-slot mapping: for each 32-wide chunk of the hidden dimension, the thread
-// with quad index q loads hidden elements [8q, 8q+8) of its A rows and of its
-// B rows, and feeds them to two m16n8k16 steps as the k-slots {2q, 2q+1,
+// with quad index q reads hidden elements [8q, 8q+8) of its A rows and of its
+// B rows and feeds them to two m16n8k16 steps as the k-slots {2q, 2q+1,
 // 2q+8, 2q+9}. A and B use the same mapping, so every product pairs equal
 // hidden indices; the sum over the chunk is unchanged.
+constexpr int kRouterStageBytes = 40 * 1024;
+
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                                uint32_t a3, uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -121,88 +127,132 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__global__ void __launch_bounds__(kRouterThreads) router_bf16_kernel(
+// 16-byte async copy global -> shared; src_bytes = 0 fills zeros.
+__device__ __forceinline__ void cp_async_16(void *dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int NPEND>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(NPEND) : "memory");
+}
+
+// hidden elements per staged block for N experts (multiple of 32, >= 32):
+// (16 + N) rows of (2*LB + 64) bytes fit one stage
+__host__ __device__ inline int router_block_len(int N) {
+    int lb = ((kRouterStageBytes / (kRouterTile + N) - 64) / 2) & ~31;
+    if (lb >= 64) lb &= ~63;
+    return lb < 32 ? 32 : lb;
+}
+
+__global__ void __launch_bounds__(kRouterThreads, 2) router_bf16_kernel(
     moge_config c, const uint16_t *__restrict__ x, const uint16_t *__restrict__ wr,
     const float *__restrict__ bias, int32_t *topk_idx, float *topk_w, int32_t *hist, int32_t *rank,
     int ks) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    RouterSmem &sm = *reinterpret_cast<RouterSmem *>(smem_raw);
+    unsigned char *stage = smem_raw;  // [2][kRouterStageBytes]
+    RouterSmem &sm = *reinterpret_cast<RouterSmem *>(smem_raw + 2 * kRouterStageBytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, q = lane & 3;
     const int crank = blockIdx.x % ks;
     const int t0 = (blockIdx.x / ks) * kRouterTile;
     const int d = c.d, N = c.N;
+    const int LB = router_block_len(N);
+    const int pitch = 2 * LB + 64;  // bytes per staged row
+    const int rows = kRouterTile + N;
+    // this CTA's slice of the hidden dimension, in whole 32-element chunks
     const int nchunk = (d + 31) / 32;
-    const int c_begin = (int)((long long)nchunk * crank / ks);
-    const int c_end = (int)((long long)nchunk * (crank + 1) / ks);
-    const int ra = t0 + g, rb = t0 + g + 8;
-    const bool va = ra < c.T, vb = rb < c.T;
-    const uint16_t *xa = x + (size_t)(va ? ra : 0) * d;
-    const uint16_t *xb = x + (size_t)(vb ? rb : 0) * d;
+    const int kb = 32 * (int)((long long)nchunk * crank / ks);
+    const int ke = min(d, 32 * (int)((long long)nchunk * (crank + 1) / ks));
+    const int nblk = (ke - kb + LB - 1) / LB;
+    const int vpr = LB / 8;  // 16-byte vectors per staged row
 
-    for (int n0 = 0; n0 < N; n0 += 64) {  // pass over 64 experts (8 n-tiles)
-        const int ntile = min(8, (N - n0) / 8);
-        float acc[8][4];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.0f;
-        for (int ch = c_begin + warp; ch < c_end; ch += kRouterWarps) {
-            const int k = ch * 32 + 8 * q;
-            const bool kv = k < d;  // d % 8 == 0: a 16-byte vector is all in or all out
-            uint4 av = make_uint4(0, 0, 0, 0), bv = make_uint4(0, 0, 0, 0);
-            if (kv && va) av = __ldg(reinterpret_cast<const uint4 *>(xa + k));
-            if (kv && vb) bv = __ldg(reinterpret_cast<const uint4 *>(xb + k));
-            uint4 wv[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                wv[i] = make_uint4(0, 0, 0, 0);
-                if (i < ntile && kv)
-                    wv[i] = __ldg(reinterpret_cast<const uint4 *>(wr + (size_t)(n0 + i * 8 + g) * d + k));
+    auto load_block = [&](int b, unsigned char *dst) {
+        const int k0 = kb + b * LB;
+        for (int i = threadIdx.x; i < rows * vpr; i += blockDim.x) {
+            const int r = i / vpr, v = i % vpr;
+            const int k = k0 + 8 * v;
+            const uint16_t *src;
+            bool ok = k < ke;
+            if (r < kRouterTile) {
+                ok = ok && (t0 + r) < c.T;
+                src = x + (size_t)(ok ? t0 + r : 0) * d + (ok ? k : 0);
+            } else {
+                src = wr + (size_t)(r - kRouterTile) * d + (ok ? k : 0);
             }
+            cp_async_16(dst + (size_t)r * pitch + 16 * v, src, ok ? 16u : 0u);
+        }
+        cp_async_commit();
+    };
+
+    float acc[4][4];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                if (i < ntile) {
-                    mma_bf16_16816(acc[i], av.x, bv.x, av.y, bv.y, wv[i].x, wv[i].y);
-                    mma_bf16_16816(acc[i], av.z, bv.z, av.w, bv.w, wv[i].z, wv[i].w);
+    for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.0f;
+    const int ntiles = N / 8;
+    // Tiles start at different blocks of their slice, so the CTAs that run at
+    // the same time do not all read the same router rows (an L2 hot spot).
+    const int rot = nblk > 0 ? (blockIdx.x / ks) % nblk : 0;
+    if (nblk > 0) load_block(rot, stage);
+    for (int i = 0; i < nblk; ++i) {
+        const int b = (i + rot) % nblk;
+        if (i + 1 < nblk) {
+            load_block((i + 1 + rot) % nblk, stage + ((i + 1) & 1) * kRouterStageBytes);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();
+        const unsigned char *st = stage + (i & 1) * kRouterStageBytes;
+        const int len = min(LB, ke - (kb + b * LB));
+        for (int ch = 0; ch < (len + 31) / 32; ++ch) {
+            const int off = 64 * ch + 16 * q;  // bytes into the row
+            const uint4 av = *reinterpret_cast<const uint4 *>(st + (size_t)g * pitch + off);
+            const uint4 bv = *reinterpret_cast<const uint4 *>(st + (size_t)(g + 8) * pitch + off);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int nt = warp + 8 * i;
+                if (nt < ntiles) {
+                    const uint4 wv = *reinterpret_cast<const uint4 *>(
+                        st + (size_t)(kRouterTile + nt * 8 + g) * pitch + off);
+                    mma_bf16_16816(acc[i], av.x, bv.x, av.y, bv.y, wv.x, wv.y);
+                    mma_bf16_16816(acc[i], av.z, bv.z, av.w, bv.w, wv.z, wv.w);
                 }
             }
         }
-        // per-warp partials -> smem, then a fixed-order sum over warps
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            if (i < ntile) {
-                sm.part[warp][g][i * 8 + 2 * q] = acc[i][0];
-                sm.part[warp][g][i * 8 + 2 * q + 1] = acc[i][1];
-                sm.part[warp][g + 8][i * 8 + 2 * q] = acc[i][2];
-                sm.part[warp][g + 8][i * 8 + 2 * q + 1] = acc[i][3];
-            }
-        }
-        __syncthreads();
-        for (int o = threadIdx.x; o < kRouterTile * ntile * 8; o += blockDim.x) {
-            const int tt = o / (ntile * 8), e = o % (ntile * 8);
-            float s = 0.0f;
-#pragma unroll
-            for (int w = 0; w < kRouterWarps; ++w) s += sm.part[w][tt][e];
-            sm.logits[tt][n0 + e] = s;
-        }
-        __syncthreads();
+        __syncthreads();  // the stage is refilled two blocks later
     }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int nt = warp + 8 * i;
+        if (nt < ntiles) {
+            sm.logits[g][nt * 8 + 2 * q] = acc[i][0];
+            sm.logits[g][nt * 8 + 2 * q + 1] = acc[i][1];
+            sm.logits[g + 8][nt * 8 + 2 * q] = acc[i][2];
+            sm.logits[g + 8][nt * 8 + 2 * q + 1] = acc[i][3];
+        }
+    }
+    __syncthreads();
 
     if (ks > 1) {
+        // peers push their partial logits into the leader's (now idle) stage
+        // buffers; the leader adds them in rank order
         cg::cluster_group cluster = cg::this_cluster();
-        cluster.sync();  // every CTA's partial logits are complete
-        if (crank == 0) {
-            for (int o = threadIdx.x; o < kRouterTile * N; o += blockDim.x) {
-                const int tt = o / N, e = o % N;
-                float s = sm.logits[tt][e];
-                for (int r = 1; r < ks; ++r) {
-                    const RouterSmem *rs = cluster.map_shared_rank(&sm, r);
-                    s += rs->logits[tt][e];
-                }
-                sm.logits[tt][e] = s;
-            }
+        cluster.sync();  // all partial logits are final; every CTA is past its K-loop
+        float *land = reinterpret_cast<float *>(stage);
+        if (crank != 0) {
+            float *dst = cluster.map_shared_rank(land, 0) + (size_t)(crank - 1) * kRouterTile * N;
+            for (int o = threadIdx.x; o < kRouterTile * N; o += blockDim.x)
+                dst[o] = sm.logits[o / N][o % N];
         }
-        cluster.sync();  // peers keep their shared memory until rank 0 has read it
+        cluster.sync();  // the pushes are visible to the leader
         if (crank != 0) return;
+        for (int o = threadIdx.x; o < kRouterTile * N; o += blockDim.x) {
+            float s = sm.logits[o / N][o % N];
+            for (int r = 1; r < ks; ++r) s += land[(size_t)(r - 1) * kRouterTile * N + o];
+            sm.logits[o / N][o % N] = s;
+        }
         __syncthreads();
     }
     router_epilogue(sm, c, bias, t0, topk_idx, topk_w, hist, rank);
@@ -235,8 +285,8 @@ cudaError_t launch_router(const moge_config &c, const void *x, const void *w_rou
                           const float *bias, int32_t *topk_idx, float *topk_w, int32_t *hist,
                           int32_t *rank, int num_sms, cudaStream_t st) {
     const int tiles = (c.T + kRouterTile - 1) / kRouterTile;
-    const size_t smem = sizeof(RouterSmem);
     if (c.dtype == MOGE_F32) {
+        const size_t smem = sizeof(RouterSmem);
         cudaError_t e = cudaFuncSetAttribute(router_f32_kernel,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
@@ -244,9 +294,15 @@ cudaError_t launch_router(const moge_config &c, const void *x, const void *w_rou
             c, (const float *)x, (const float *)w_router, bias, topk_idx, topk_w, hist, rank);
         return cudaGetLastError();
     }
-    // split the hidden dimension over a cluster when there are few tiles
+    // Split the hidden dimension over a cluster of up to 8 CTAs while the
+    // grid stays within two CTAs per SM, each CTA keeps >= 2 blocks of work,
+    // and the leader's landing buffer (two stages) holds (ks - 1) partial tiles.
+    const int lb = router_block_len(c.N);
     int ks = 1;
-    while (ks < 8 && tiles * ks * 2 <= 2 * num_sms && (c.d / 32) >= ks * 2 * kRouterWarps) ks *= 2;
+    while (ks < 8 && tiles * ks * 2 <= 2 * num_sms && c.d >= ks * 2 * 2 * lb &&
+           (2 * ks - 1) * kRouterTile * c.N * 4 <= 2 * kRouterStageBytes)
+        ks *= 2;
+    const size_t smem = 2 * kRouterStageBytes + sizeof(RouterSmem);
     cudaError_t e = cudaFuncSetAttribute(router_bf16_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -267,67 +323,110 @@ cudaError_t launch_router(const moge_config &c, const void *x, const void *w_rou
 }
 
 // ---------------------------------------------------------------------------
-// Work plan of the grouped FFN. Entries: routed experts 0..N-1 (if
-// with_routed), then shared experts 0..S-1 (if with_shared).
-__device__ void build_plan(const moge_config &c, const int32_t *offsets, Plan plan,
-                           bool with_routed, bool with_shared, int shared_row_base) {
-    const int K = c.M * c.Kp;
+// Exclusive prefix sum across a block of exactly 1024 threads: returns the sum
+// of v over the threads before this one; *total receives the block sum.
+// Every thread must call it (it synchronises the block).
+__device__ int block_exclusive_scan_1024(int v, int *wbuf /* [32] */, int *total) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) wbuf[w] = x;
+    __syncthreads();
+    if (w == 0) {
+        int t = wbuf[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, t, o);
+            if (lane >= o) t += y;
+        }
+        wbuf[lane] = t;
+    }
+    __syncthreads();
+    const int pre = (w > 0 ? wbuf[w - 1] : 0) + x - v;
+    *total = wbuf[31];
+    __syncthreads();
+    return pre;
+}
+
+// Work plan of the grouped FFN, one entry per thread: routed experts 0..N-1
+// (if with_routed, rows from offs[]), then shared experts 0..S-1 (if
+// with_shared, T rows each, their h / y rows after shared_row_base).
+// Token-tile width: <= kStreamRows rows -> one streaming tile of
+// round16(rows); more -> ceil(rows / 256) balanced tiles of round16 width.
+// Called by all 1024 threads of the block.
+__device__ void build_plan_block(const moge_config &c, const int32_t *offs, Plan plan,
+                                 bool with_routed, bool with_shared, int shared_row_base,
+                                 int *wbuf) {
     const int fb_up = (c.I + 63) / 64;      // 64 gate + 64 up rows per tile
     const int fb_down = (c.d + 127) / 128;  // 128 output features per tile
-    int n = 0, su = 0, sd = 0;
-    auto add = [&](int rows, int a_sel, int a_idx, int up_src, int up_bsel, int mid_row) {
-        ExpertWork w;
-        w.rows = rows;
-        w.a_sel = a_sel;
-        w.a_idx = a_idx;
-        if (rows <= 0) {
-            w.bn = 16;
-            w.ntb = 0;
-        } else if (rows <= kStreamRows) {
-            w.bn = (rows + 15) & ~15;
-            w.ntb = 1;
+    const int nr = with_routed ? c.N : 0;
+    const int n = nr + (with_shared ? c.S : 0);
+    const int i = threadIdx.x;
+    ExpertWork u = {}, dn = {};
+    int items_up = 0, items_down = 0;
+    if (i < n) {
+        int rows, a_sel, a_idx, up_src, up_bsel, mid;
+        if (i < nr) {
+            rows = offs[i + 1] - offs[i];
+            a_sel = 0; a_idx = i; up_src = offs[i]; up_bsel = 0; mid = offs[i];
         } else {
-            const int ntb = (rows + kMaxTileN - 1) / kMaxTileN;
-            const int per = (rows + ntb - 1) / ntb;
-            w.bn = (per + 15) & ~15;
-            w.ntb = (rows + w.bn - 1) / w.bn;
+            const int sidx = i - nr;
+            rows = c.T;
+            a_sel = 1; a_idx = sidx; up_src = 0; up_bsel = 1; mid = shared_row_base + sidx * c.T;
         }
-        ExpertWork u = w, dn = w;
-        u.src_row0 = up_src;
-        u.b_sel = up_bsel;
-        u.dst_row0 = mid_row;
-        dn.src_row0 = mid_row;
-        dn.b_sel = 0;
-        dn.dst_row0 = mid_row;
-        plan.up[n] = u;
-        plan.down[n] = dn;
-        plan.up_start[n] = su;
-        plan.down_start[n] = sd;
-        su += w.ntb * fb_up;
-        sd += w.ntb * fb_down;
-        ++n;
-    };
-    (void)K;
-    if (with_routed)
-        for (int e = 0; e < c.N; ++e)
-            add(offsets[e + 1] - offsets[e], 0, e, offsets[e], 0, offsets[e]);
-    if (with_shared)
-        for (int s = 0; s < c.S; ++s) add(c.T, 1, s, 0, 1, shared_row_base + s * c.T);
-    plan.up_start[n] = su;
-    plan.down_start[n] = sd;
+        int bn, ntb;
+        if (rows <= 0) {
+            bn = 16; ntb = 0;
+        } else if (rows <= kStreamRows) {
+            bn = (rows + 15) & ~15; ntb = 1;
+        } else {
+            const int nt = (rows + kMaxTileN - 1) / kMaxTileN;
+            bn = (((rows + nt - 1) / nt) + 15) & ~15;
+            ntb = (rows + bn - 1) / bn;
+        }
+        u.rows = dn.rows = rows;
+        u.a_sel = dn.a_sel = a_sel;
+        u.a_idx = dn.a_idx = a_idx;
+        u.bn = dn.bn = bn;
+        u.ntb = dn.ntb = ntb;
+        u.src_row0 = up_src; u.b_sel = up_bsel; u.dst_row0 = mid;
+        dn.src_row0 = mid; dn.b_sel = 0; dn.dst_row0 = mid;
+        items_up = ntb * fb_up;
+        items_down = ntb * fb_down;
+    }
+    int tot_up, tot_down;
+    const int pre_up = block_exclusive_scan_1024(items_up, wbuf, &tot_up);
+    const int pre_down = block_exclusive_scan_1024(items_down, wbuf, &tot_down);
+    if (i < n) {
+        plan.up[i] = u;
+        plan.down[i] = dn;
+        plan.up_start[i] = pre_up;
+        plan.down_start[i] = pre_down;
+    }
+    if (i == 0) {
+        plan.up_start[n] = tot_up;
+        plan.down_start[n] = tot_down;
+    }
 }
 
 // Column sums of hist over tiles -> base (exclusive), counts, offsets;
 // checks the equal group load; optionally writes the layer's GEMM plan.
+// One block of 1024 threads.
 __global__ void __launch_bounds__(1024) scan_kernel(moge_config c, const int32_t *__restrict__ hist,
                                                      int32_t *base, int32_t *counts,
                                                      int32_t *offsets, Plan plan, int make_plan,
                                                      int with_routed, int with_shared) {
     __shared__ int32_t part[1024];
-    __shared__ int32_t cnt_s[kMaxExperts + 1];
+    __shared__ int32_t cnt_s[kMaxExperts];
+    __shared__ int32_t off_s[kMaxExperts + 1];
+    __shared__ int wbuf[32];
     const int N = c.N;
     const int tiles = (c.T + kRouterTile - 1) / kRouterTile;
-    const int P = blockDim.x / N;  // chunks of tiles
+    const int P = 1024 / N;  // chunks of tiles
     const int e = threadIdx.x % N, p = threadIdx.x / N;
     const bool act = p < P;
     const int tb = act ? (int)((long long)tiles * p / P) : 0;
@@ -344,7 +443,6 @@ __global__ void __launch_bounds__(1024) scan_kernel(moge_config c, const int32_t
             run += v;
         }
         cnt_s[threadIdx.x] = run;
-        counts[threadIdx.x] = run;
     }
     __syncthreads();
     if (act) {
@@ -354,47 +452,54 @@ __global__ void __launch_bounds__(1024) scan_kernel(moge_config c, const int32_t
             run += hist[(size_t)t * N + e];
         }
     }
+    const int v = threadIdx.x < N ? cnt_s[threadIdx.x] : 0;
+    int total;
+    const int pre = block_exclusive_scan_1024(v, wbuf, &total);
+    if (threadIdx.x < N) {
+        counts[threadIdx.x] = v;
+        offsets[threadIdx.x] = pre;
+        off_s[threadIdx.x] = pre;
+    }
     if (threadIdx.x == 0) {
+        offsets[N] = total;
+        off_s[N] = total;
+    }
+    if (threadIdx.x < c.M) {  // every group carries exactly T*Kp assignments
         const int G = N / c.M;
-        int run = 0;
-        for (int i = 0; i < N; ++i) {
-            offsets[i] = run;
-            run += cnt_s[i];
-        }
-        offsets[N] = run;
-        for (int g = 0; g < c.M; ++g) {  // every group carries exactly T*Kp assignments
-            int lg = 0;
-            for (int i = g * G; i < (g + 1) * G; ++i) lg += cnt_s[i];
-            if (lg != c.T * c.Kp) raise_error(ERRBIT_INVARIANT);
-        }
+        int lg = 0;
+        for (int i = threadIdx.x * G; i < (threadIdx.x + 1) * G; ++i) lg += cnt_s[i];
+        if (lg != c.T * c.Kp) raise_error(ERRBIT_INVARIANT);
     }
     if (make_plan) {
         __syncthreads();
-        if (threadIdx.x == 0)
-            build_plan(c, offsets, plan, with_routed != 0, with_shared != 0, c.T * c.M * c.Kp);
+        build_plan_block(c, off_s, plan, with_routed != 0, with_shared != 0, c.T * c.M * c.Kp, wbuf);
     }
 }
 
 cudaError_t launch_scan(const moge_config &c, const int32_t *hist, int32_t *base, int32_t *counts,
                         int32_t *offsets, const Plan *plan, bool with_routed, bool with_shared,
                         cudaStream_t st) {
-    const int threads = (1024 / c.N) * c.N;
     Plan p = plan ? *plan : Plan{nullptr, nullptr, nullptr, nullptr};
-    scan_kernel<<<1, threads, 0, st>>>(c, hist, base, counts, offsets, p, plan ? 1 : 0,
-                                        with_routed ? 1 : 0, with_shared ? 1 : 0);
+    scan_kernel<<<1, 1024, 0, st>>>(c, hist, base, counts, offsets, p, plan ? 1 : 0,
+                                    with_routed ? 1 : 0, with_shared ? 1 : 0);
     return cudaGetLastError();
 }
 
-__global__ void plan_kernel(moge_config c, const int32_t *offsets, Plan plan, int with_routed,
-                            int with_shared) {
-    if (threadIdx.x == 0 && blockIdx.x == 0)
-        build_plan(c, offsets, plan, with_routed != 0, with_shared != 0,
-                   with_routed ? c.T * c.M * c.Kp : 0);
+// Plan from the caller's offsets (routed only) or for the shared experts only.
+__global__ void __launch_bounds__(1024) plan_kernel(moge_config c, const int32_t *offsets, Plan plan,
+                                                     int with_routed, int with_shared) {
+    __shared__ int32_t off_s[kMaxExperts + 1];
+    __shared__ int wbuf[32];
+    if (with_routed)
+        for (int i = threadIdx.x; i <= c.N; i += blockDim.x) off_s[i] = offsets[i];
+    __syncthreads();
+    build_plan_block(c, off_s, plan, with_routed != 0, with_shared != 0,
+                     with_routed ? c.T * c.M * c.Kp : 0, wbuf);
 }
 
 cudaError_t launch_plan(const moge_config &c, const int32_t *offsets, const Plan &plan,
                         bool with_routed, bool with_shared, cudaStream_t st) {
-    plan_kernel<<<1, 32, 0, st>>>(c, offsets, plan, with_routed ? 1 : 0, with_shared ? 1 : 0);
+    plan_kernel<<<1, 1024, 0, st>>>(c, offsets, plan, with_routed ? 1 : 0, with_shared ? 1 : 0);
     return cudaGetLastError();
 }
 

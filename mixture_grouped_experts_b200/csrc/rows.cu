@@ -114,46 +114,92 @@ __device__ __forceinline__ void store_vec(void *p, size_t v, const float (&f)[8]
 }
 
 // Vectors here are 8 elements (16 B in bf16, 32 B in fp32); d % 8 == 0.
+// The row loads of one vector are issued in batches of 8 before any of them
+// is used, so that the kernel waits for memory once per batch, not per row.
+struct Raw8 {
+    uint4 a, b;  // bf16: a only; fp32: a and b
+};
+template <int DT>
+__device__ __forceinline__ Raw8 load_raw(const void *row, int v) {
+    Raw8 r;
+    if (DT == MOGE_BF16) {
+        r.a = reinterpret_cast<const uint4 *>(row)[v];
+        r.b = make_uint4(0, 0, 0, 0);
+    } else {
+        r.a = reinterpret_cast<const uint4 *>(row)[2 * v];
+        r.b = reinterpret_cast<const uint4 *>(row)[2 * v + 1];
+    }
+    return r;
+}
+template <int DT>
+__device__ __forceinline__ void unpack8(const Raw8 &r, float (&f)[8]) {
+    if (DT == MOGE_BF16) {
+        f[0] = bf16_lo(r.a.x); f[1] = bf16_hi(r.a.x); f[2] = bf16_lo(r.a.y); f[3] = bf16_hi(r.a.y);
+        f[4] = bf16_lo(r.a.z); f[5] = bf16_hi(r.a.z); f[6] = bf16_lo(r.a.w); f[7] = bf16_hi(r.a.w);
+    } else {
+        f[0] = __uint_as_float(r.a.x); f[1] = __uint_as_float(r.a.y);
+        f[2] = __uint_as_float(r.a.z); f[3] = __uint_as_float(r.a.w);
+        f[4] = __uint_as_float(r.b.x); f[5] = __uint_as_float(r.b.y);
+        f[6] = __uint_as_float(r.b.z); f[7] = __uint_as_float(r.b.w);
+    }
+}
+
 template <int DT>
 __global__ void __launch_bounds__(kRowThreads) combine_kernel(
     int T, int d, int N, const void *__restrict__ y_perm, const float *__restrict__ topk_w,
     const int32_t *__restrict__ perm_dst, int K, const void *__restrict__ shared_rows,
     int n_shared, const void *residual, void *y) {
-    __shared__ int dst_s[kMaxExperts];
+    __shared__ const char *src_s[2 * kMaxExperts + 1];
     __shared__ float w_s[kMaxExperts];
     const int t = blockIdx.x;
     const int nvec = d / 8;
-    const size_t esz = DT == MOGE_BF16 ? 2 : 4;
+    const size_t row_bytes = (size_t)d * (DT == MOGE_BF16 ? 2 : 4);
+    (void)N;
+    // source rows in summation order: K routed rows, then the shared blocks
     for (int k = threadIdx.x; k < K; k += blockDim.x) {
-        const int row = perm_dst[(size_t)t * K + k];
-        if (row < 0 || row >= T * K) raise_error(ERRBIT_INVARIANT);
-        dst_s[k] = (row < 0 || row >= T * K) ? 0 : row;
+        int row = perm_dst[(size_t)t * K + k];
+        if (row < 0 || row >= T * K) {
+            raise_error(ERRBIT_INVARIANT);
+            row = 0;
+        }
+        src_s[k] = static_cast<const char *>(y_perm) + (size_t)row * row_bytes;
         w_s[k] = topk_w[(size_t)t * K + k];
     }
+    for (int b = threadIdx.x; b < n_shared; b += blockDim.x)
+        src_s[K + b] = static_cast<const char *>(shared_rows) + ((size_t)b * T + t) * row_bytes;
     __syncthreads();
-    (void)N;
+    const int nsrc = K + n_shared;
     for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
         float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-        for (int k = 0; k < K; ++k) {
-            float f[8];
-            load_vec<DT>((const char *)y_perm + (size_t)dst_s[k] * d * esz, v, f);
-            const float w = w_s[k];
+        for (int k0 = 0; k0 < nsrc; k0 += 8) {
+            Raw8 raw[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) acc[j] = fmaf(w, f[j], acc[j]);
-        }
-        for (int b = 0; b < n_shared; ++b) {
-            float f[8];
-            load_vec<DT>((const char *)shared_rows + ((size_t)b * T + t) * d * esz, v, f);
+            for (int j = 0; j < 8; ++j)
+                if (k0 + j < nsrc) raw[j] = load_raw<DT>(src_s[k0 + j], v);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) acc[j] += f[j];
+            for (int j = 0; j < 8; ++j) {
+                const int k = k0 + j;
+                if (k < nsrc) {
+                    float f[8];
+                    unpack8<DT>(raw[j], f);
+                    if (k < K) {
+                        const float w = w_s[k];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) acc[q] = fmaf(w, f[q], acc[q]);
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) acc[q] += f[q];
+                    }
+                }
+            }
         }
         if (residual) {
             float f[8];
-            load_vec<DT>((const char *)residual + (size_t)t * d * esz, v, f);
+            load_vec<DT>((const char *)residual + (size_t)t * row_bytes, v, f);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) acc[j] = f[j] + acc[j];
+            for (int q = 0; q < 8; ++q) acc[q] = f[q] + acc[q];
         }
-        store_vec<DT>((char *)y + (size_t)t * d * esz, v, acc);
+        store_vec<DT>((char *)y + (size_t)t * row_bytes, v, acc);
     }
 }
 

@@ -183,3 +183,34 @@ def test_host_buffer_entry_point():
     xd, yd = torch.empty_like(x), torch.empty_like(x)
     mg.moge_layer_forward_host(s, xh, w, ws, yh, xd, yd)
     assert torch.equal(yh.view(torch.int16), ref.cpu().view(torch.int16))
+
+
+@pytest.mark.parametrize("layout", ["gate_first", "up_first", "same_tensor"])
+def test_gate_up_weight_placements(layout):
+    """The up-projection fetches its gate+up tile in one copy when w_up lies
+    wholly after (or before) w_gate, and in two copies when they overlap (here:
+    w_up is w_gate itself). All three give the oracle's result."""
+    cfg = MED.replace(name="gu_" + layout, T=120, seed=27)
+    inp = synth.layer_inputs(cfg)
+    if layout == "same_tensor":
+        inp["w_up"] = inp["w_gate"]
+    x, w = device_inputs(cfg, inp)
+    if layout in ("gate_first", "up_first"):
+        n = w["w_gate"].numel()
+        both = torch.empty(2 * n, dtype=torch.bfloat16, device="cuda")
+        first, second = (both[:n], both[n:])
+        g, u = (first, second) if layout == "gate_first" else (second, first)
+        g.copy_(w["w_gate"].reshape(-1))
+        u.copy_(w["w_up"].reshape(-1))
+        w["w_gate"], w["w_up"] = g.view_as(w["w_gate"]), u.view_as(w["w_up"])
+        assert (w["w_gate"].data_ptr() < w["w_up"].data_ptr()) == (layout == "gate_first")
+    s = mg.shape_of(cfg)
+    ws = mg.alloc_workspace(s)
+    y, idx_g, w_g, counts_g, offsets_g = run_layer(cfg, x, w, ws)
+    xd = x_double(inp, cfg)
+    p = oracle.router_probs(xd, inp["w_router"], None, cfg.dtype)
+    idx_o, _, mg_o = oracle.select_grouped(p, cfg.M, cfg.Kp)
+    safe = check_routing(cfg, p, idx_o, mg_o, idx_g, w_g)
+    toks = np.nonzero(safe)[0]
+    y_ref, _, _, _ = oracle.layer(xd, inp, cfg.M, cfg.Kp, cfg.dtype, tokens=toks)
+    assert normwise_err(to_host_f64(y)[toks], y_ref) <= TOL["bf16"]
