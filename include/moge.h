@@ -133,8 +133,8 @@ MOGE_API int moge_combine(const moge_config *cfg, const void *y_perm, const floa
                  const int32_t *perm_dst, const void *y_shared, const void *residual, void *y,
                  void *stream);
 
-/* Whole layer: route, permute, one grouped up-projection launch and one
- * grouped down-projection launch covering routed AND shared experts, combine.
+/* Whole layer: route, permute, one grouped-FFN launch covering both
+ * projections of routed AND shared experts, combine.
  *   y[t] = residual[t] (if not NULL) + MoGE(x)[t];  y may alias residual, not x.
  * s_* may be NULL when S == 0; logit_bias may be NULL. The routing of the
  * call stays readable in the workspace (moge_workspace_routing). */
@@ -186,11 +186,11 @@ MOGE_API int moge_route_noalloc(const moge_config *cfg, const void *x, const voi
                                 int32_t *perm_dst, void *stream);
 
 /* Stage timing (measurement aid): while enabled, every moge_layer_forward
- * records CUDA events around its six launches -- router, scan, permute,
- * up-projection, down-projection, combine -- and the library adds up their
+ * records CUDA events around its five launches -- router, scan, permute,
+ * grouped FFN (both projections), combine -- and the library adds up their
  * durations. moge_stage_timing(1) resets the totals and starts, (0) stops.
  * moge_stage_times waits for the recorded events and returns the totals in
- * milliseconds per stage (ms_total[6]) and the number of timed calls. For one
+ * milliseconds per stage (ms_total[5]) and the number of timed calls. For one
  * host thread and one device; not for use during CUDA stream capture. */
 MOGE_API int moge_stage_timing(int enable);
 MOGE_API int moge_stage_times(double *ms_total, int64_t *calls);

@@ -30,7 +30,7 @@ EXPORTS = ["moge_workspace_size", "moge_last_error", "moge_check_device_errors",
            "moge_permute", "moge_grouped_ffn", "moge_shared_ffn", "moge_combine",
            "moge_layer_forward", "moge_layer_forward_host", "moge_workspace_routing",
            "moge_rmsnorm", "moge_stage_timing", "moge_stage_times", "moge_route_noalloc"]
-STAGES = ("router", "scan", "permute", "ffn_up", "ffn_down", "combine")
+STAGES = ("router", "scan", "permute", "ffn", "combine")
 
 
 class MogeError(RuntimeError):

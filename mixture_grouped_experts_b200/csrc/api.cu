@@ -71,6 +71,7 @@ Workspace carve_workspace(const moge_config &c, void *base) {
     w.plan.down = (ExpertWork *)take(E * sizeof(ExpertWork));
     w.plan.up_start = (int *)take((E + 1) * 4);
     w.plan.down_start = (int *)take((E + 1) * 4);
+    w.plan.sync = (int *)take((E + 1) * 4);
     w.x_perm = take(T * K * c.d * esz);
     w.h = take(T * (K + c.S) * c.I * esz);
     w.y_perm = take(T * (K + c.S) * c.d * esz);
@@ -110,10 +111,10 @@ static int num_sms() {
     } while (0)
 
 // ---------------------------------------------------------------- stage timing
-// Optional CUDA-event timing of the six launches of moge_layer_forward
-// (router, scan, permute, up-projection, down-projection, combine). Host state
-// for one host thread and one device; not for use under stream capture.
-constexpr int kTimedStages = 6;
+// Optional CUDA-event timing of the five launches of moge_layer_forward
+// (router, scan, permute, grouped FFN, combine). Host state for one host
+// thread and one device; not for use under stream capture.
+constexpr int kTimedStages = 5;
 constexpr int kEventSets = 32;
 struct StageTimer {
     bool enabled = false;
@@ -344,14 +345,14 @@ int moge_layer_forward(const moge_config *cfg, const void *x, const void *w_rout
     FfnOperands op{ws.x_perm, x, rrows, c.T, w_gate, w_up, w_down,
                    c.S > 0 ? s_gate : nullptr, c.S > 0 ? s_up : nullptr, c.S > 0 ? s_down : nullptr,
                    ws.h, rrows + (int64_t)c.T * c.S, ws.y_perm};
-    rc = run_ffn(c, ws.plan, c.N + c.S, op, st, ev ? ev[4] : nullptr);
+    rc = run_ffn(c, ws.plan, c.N + c.S, op, st, nullptr);
     if (rc) return rc;
-    if (ev) MOGE_CU(cudaEventRecord(ev[5], st), "event");
+    if (ev) MOGE_CU(cudaEventRecord(ev[4], st), "event");
     const size_t esz = c.dtype == MOGE_BF16 ? 2 : 4;
     const void *shared_rows = static_cast<const char *>(ws.y_perm) + (size_t)rrows * c.d * esz;
     MOGE_CU(launch_combine(c, ws.y_perm, ws.topk_w, ws.perm_dst, K, shared_rows, c.S, residual, y,
                            st), "combine launch");
-    if (ev) MOGE_CU(cudaEventRecord(ev[6], st), "event");
+    if (ev) MOGE_CU(cudaEventRecord(ev[5], st), "event");
     return MOGE_OK;
 }
 

@@ -18,6 +18,7 @@ __global__ void __launch_bounds__(256) ffn_up_f32_kernel(moge_config c, const Ex
     __shared__ float xs[kF32K][kF32Tile + 1];
     __shared__ float gs[kF32K][kF32Tile + 1];
     __shared__ float us[kF32K][kF32Tile + 1];
+    grid_dependency_wait();
     const ExpertWork w = work[blockIdx.z];
     const int r0 = blockIdx.y * kF32Tile, i0 = blockIdx.x * kF32Tile;
     if (r0 >= w.rows) return;
@@ -76,6 +77,7 @@ __global__ void __launch_bounds__(256) ffn_down_f32_kernel(moge_config c, const 
                                                            FfnOperands op) {
     __shared__ float hs[kF32K][kF32Tile + 1];
     __shared__ float ws[kF32K][kF32Tile + 1];
+    grid_dependency_wait();
     const ExpertWork w = work[blockIdx.z];
     const int r0 = blockIdx.y * kF32Tile, o0 = blockIdx.x * kF32Tile;
     if (r0 >= w.rows) return;
@@ -125,13 +127,11 @@ cudaError_t launch_ffn_f32(const moge_config &c, const Plan &plan, int n_entries
     if (n_entries <= 0 || c.T <= 0) return cudaSuccess;
     const int rt = (c.T + kF32Tile - 1) / kF32Tile;
     dim3 gu((c.I + kF32Tile - 1) / kF32Tile, rt, n_entries);
-    ffn_up_f32_kernel<<<gu, 256, 0, st>>>(c, plan.up, op);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(ffn_up_f32_kernel, gu, dim3(256), 0, st, c, plan.up, op);
     if (e != cudaSuccess) return e;
     if (mid && (e = cudaEventRecord(mid, st)) != cudaSuccess) return e;
     dim3 gd((c.d + kF32Tile - 1) / kF32Tile, rt, n_entries);
-    ffn_down_f32_kernel<<<gd, 256, 0, st>>>(c, plan.down, op);
-    return cudaGetLastError();
+    return launch_pdl(ffn_down_f32_kernel, gd, dim3(256), 0, st, c, plan.down, op);
 }
 
 }  // namespace moge

@@ -1,26 +1,37 @@
 // Grouped SwiGLU expert FFN on the 5th-generation tensor cores (sm_100a).
 //
-// One persistent kernel per projection (up: gate+up with the SwiGLU epilogue,
-// down: plain), one CTA per SM, warp-specialised:
-//   warp 0   TMA producer   (weights: 3-D tensor maps over [E][rows][K],
-//                             tokens: 2-D maps over the row matrices)
-//   warp 1   MMA issuer     (tcgen05.mma kind::f16, M = 128, N = token tile,
-//                             fp32 accumulators in TMEM, double-buffered)
-//   warps 2-5 epilogue      (tcgen05.ld -> registers -> smem -> coalesced
-//                             16-byte global stores, rows masked per expert)
+// One persistent kernel runs both projections of every expert -- the
+// up-projection (gate and up, SwiGLU epilogue, h rows out) and the
+// down-projection (y rows out) -- one CTA per SM, warp-specialised:
+//   warp 0    scheduler + TMA producer: takes work items from a global queue
+//             (an atomic counter), publishes them to the other roles through
+//             a small shared-memory ring, and streams their operands with TMA
+//   warp 1    MMA issuer   (tcgen05.mma kind::f16, M = 128, N = token tile,
+//                           fp32 accumulators in TMEM, double-buffered)
+//   warps 2-5 epilogue     (tcgen05.ld -> registers -> smem -> coalesced
+//                           16-byte global stores, rows masked per expert)
+//
+// The queue hands out every up-projection item before any down-projection
+// item, shared experts first (the heaviest items go first, the tail is made
+// of small ones). A down-projection item of an expert waits -- bounded -- until
+// all up-projection items of that expert have stored their h rows (a per-
+// expert counter), so no kernel boundary separates the two phases. Every item
+// it waits for was handed out earlier to a running CTA whose pipeline finishes
+// it without waiting on anything, so the wait always ends.
 //
 // Orientation ("swap AB"): the weight tile is the MMA's M = 128 operand and the
 // tokens of one expert are its N operand, N = 16 .. 256. A decode-sized expert
-// (<= 64 rows) is one "streaming" tile: its weight rows are the HBM-bound
-// stream, so every pipeline stage carries two 64-wide K-chunks (32 KB of
-// weights) to keep more bytes in flight. Larger experts are split into token
-// tiles of <= 256 rows ("tensor" tiles: one K-chunk per stage, compute-bound).
-// The choice is made per expert from its token count, on the device.
+// (<= 64 rows) is one "streaming" tile: its weights are the HBM-bound stream,
+// and every 48 KB pipeline stage carries two 64-wide K-chunks (32 KB of
+// weights). Larger experts are split into token tiles of <= 256 rows
+// ("tensor" tiles: one K-chunk per stage). The choice is made per expert from
+// its token count, on the device.
 //
-// The up tile stacks 64 gate rows over the matching 64 up rows (two TMA boxes
-// into one 128-row operand), so the accumulator lanes 0-63 hold gate and lanes
-// 64-127 hold up for the same 64 features; the epilogue pairs them through
-// shared memory. This needs no repacking of the [E][I][d] weights.
+// The up tile stacks 64 gate rows over the matching 64 up rows, fetched with
+// one 16 KB copy from a 4-D tensor map that spans both weight tensors (or two
+// 8 KB copies if the tensors overlap), so the accumulator lanes 0-63 hold gate
+// and lanes 64-127 hold up for the same 64 features; the epilogue pairs them
+// through shared memory. No repacking of the [E][I][d] weights is needed.
 //
 // The grouped expert GEMM ("GroupMatmul") of the Pangu Pro MoE article
 // (techwalker.com, section 3) and its SwiftGMM GEMV/GEMM switch (reportify.cn
@@ -38,6 +49,7 @@ constexpr int kTcThreads = 192;
 constexpr int kChunkK = 64;          // bf16 elements per K-chunk (128 bytes, one swizzle row)
 constexpr int kBoxRows = 64;         // token rows per TMA box (one 8 KB copy per chunk)
 constexpr uint32_t kTmemCols = 512;  // two accumulators of 256 columns
+constexpr int kSlots = 8;            // depth of the work-item ring
 
 // How the up-projection's 128-row weight tile is fetched, per weight side
 // (routed / shared): one 16 KB copy from a 4-D map over both tensors when
@@ -47,27 +59,32 @@ enum : int { kGateUpSplit = 0, kGateUpFused = 1, kUpGateFused = 2 };
 
 struct TcParams {
     int gu_mode[2];  // per a_sel
-    const ExpertWork *work;
-    const int *item_start;
+    Plan plan;
     int n_entries;
-    int k_chunks;  // ceil(K / 64)
-    int out_cols;  // I (up) or d (down): valid output features
-    uint16_t *out; // h (up) or y_perm (down), row stride out_cols
+    int kc_up, kc_down;  // K-chunks of the two projections: ceil(d/64), ceil(I/64)
+    int I, d;
+    uint16_t *h;         // [rows][I]
+    uint16_t *y;         // [rows][d]
+    int *sync;           // [0] queue counter, [1 + e] finished up items of entry e
 };
 
 struct TcItem {
     ExpertWork w;
-    int fb, tb, n_valid;
-    bool stream;
+    int entry, fb, tb, n_valid;
+    bool up, stream;
 };
 
-__device__ __forceinline__ void decode_item(const TcParams &p, int item, TcItem &it) {
+// Decode global item q: the up-projection items first, then the down-projection ones.
+__device__ __forceinline__ void decode_item(const TcParams &p, int tot_up, int q, TcItem &it) {
+    it.up = q < tot_up;
+    const int local = it.up ? q : q - tot_up;
+    const int *start = it.up ? p.plan.up_start : p.plan.down_start;
     int lo = 0, hi = p.n_entries - 1;
-    while (lo < hi) {  // last entry whose first item is <= item (entries may be empty)
+    while (lo < hi) {  // last entry whose first item is <= local (entries may be empty)
         const int mid = (lo + hi + 1) >> 1;
-        if (__ldg(p.item_start + mid) <= item) lo = mid; else hi = mid - 1;
+        if (__ldg(start + mid) <= local) lo = mid; else hi = mid - 1;
     }
-    const int *wp = reinterpret_cast<const int *>(p.work + lo);
+    const int *wp = reinterpret_cast<const int *>((it.up ? p.plan.up : p.plan.down) + lo);
     it.w.rows = __ldg(wp + 0);
     it.w.src_row0 = __ldg(wp + 1);
     it.w.dst_row0 = __ldg(wp + 2);
@@ -76,29 +93,32 @@ __device__ __forceinline__ void decode_item(const TcParams &p, int item, TcItem 
     it.w.b_sel = __ldg(wp + 5);
     it.w.bn = __ldg(wp + 6);
     it.w.ntb = __ldg(wp + 7);
-    const int local = item - __ldg(p.item_start + lo);
-    it.fb = local / it.w.ntb;  // feature block major, token tile fastest
-    it.tb = local % it.w.ntb;
+    it.entry = lo;
+    const int r = local - __ldg(start + lo);
+    it.fb = r / it.w.ntb;  // feature block major, token tile fastest
+    it.tb = r % it.w.ntb;
     it.n_valid = min(it.w.bn, it.w.rows - it.tb * it.w.bn);
     it.stream = it.w.rows <= kStreamRows;
 }
 
-struct TcShared {
-    uint64_t full[kStages], empty[kStages], tfull[2], tempty[2], drain;
-    uint32_t tmem_base;
-    int abort;
-    int epi_ok;
-};
-
 // K-chunk processed at step i of an item of feature block fb: items of the
 // same expert run side by side and read the same token rows, so each feature
-// block starts at a different chunk (an L2 hot spot otherwise). The order is
-// fixed per item, so results stay deterministic.
+// block starts at a different chunk. The order is fixed per item, so results
+// stay deterministic.
 __device__ __forceinline__ int chunk_at(int i, int fb, int k_chunks) {
     const int r = (fb * 2 * 5) % k_chunks;  // even start: streaming pairs stay aligned
     const int c = i + r;
     return c >= k_chunks ? c - k_chunks : c;
 }
+
+struct TcShared {
+    uint64_t full[kStages], empty[kStages], tfull[2], tempty[2], drain;
+    uint64_t slot_full[kSlots], slot_empty[kSlots];
+    int slot_item[kSlots];
+    uint32_t tmem_base;
+    int abort;
+    int epi_item;
+};
 
 // smem byte offsets of chunk c of a stage
 __device__ __forceinline__ uint32_t a_off(bool stream, int c) { return stream ? c * 24576u : 0u; }
@@ -106,11 +126,39 @@ __device__ __forceinline__ uint32_t b_off(bool stream, int c) {
     return stream ? c * 24576u + 16384u : 16384u;
 }
 
-template <bool UP>
+__device__ __forceinline__ int ld_acquire(const int *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Bounded wait until *ctr >= need (an up-projection's h rows of one expert).
+__device__ bool wait_counter(const int *ctr, int need, volatile int *abort) {
+    if (ld_acquire(ctr) >= need) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        __nanosleep(64);
+        if (ld_acquire(ctr) >= need) return true;
+        if ((it & 63u) == 0) {
+            if (*abort) return false;
+            if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+                raise_error(ERRBIT_TIMEOUT);
+                *abort = 1;
+                return false;
+            }
+        }
+    }
+}
+
 __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
-    TcParams p, const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
-    const __grid_constant__ CUtensorMap tmS0, const __grid_constant__ CUtensorMap tmS1,
-    const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1) {
+    const __grid_constant__ TcParams p, const __grid_constant__ CUtensorMap tmWg,
+    const __grid_constant__ CUtensorMap tmWu, const __grid_constant__ CUtensorMap tmSg,
+    const __grid_constant__ CUtensorMap tmSu, const __grid_constant__ CUtensorMap tmX0,
+    const __grid_constant__ CUtensorMap tmX1, const __grid_constant__ CUtensorMap tmWd,
+    const __grid_constant__ CUtensorMap tmSd, const __grid_constant__ CUtensorMap tmH) {
     extern __shared__ __align__(1024) unsigned char smem_dyn[];
     // 1024-byte alignment for the 128-byte swizzle atoms
     unsigned char *smem = reinterpret_cast<unsigned char *>(
@@ -119,9 +167,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
     unsigned char *epi = smem + kStages * kStageBytes;
     TcShared &sh = *reinterpret_cast<TcShared *>(epi + kEpiBytes);
     volatile int *abort = &sh.abort;
-
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int total = __ldg(p.item_start + p.n_entries);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -132,19 +178,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
             mbar_init(&sh.tfull[a], 1);
             mbar_init(&sh.tempty[a], 128);
         }
+        for (int s = 0; s < kSlots; ++s) {
+            mbar_init(&sh.slot_full[s], 1);
+            mbar_init(&sh.slot_empty[s], 2);  // the MMA thread and the epilogue leader
+        }
         mbar_init(&sh.drain, 1);
         sh.abort = 0;
         fence_barrier_init();
     }
     if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&tmA0);
-        tma_prefetch_desc(&tmS0);
-        tma_prefetch_desc(&tmB0);
-        if (UP) {
-            tma_prefetch_desc(&tmA1);
-            tma_prefetch_desc(&tmS1);
-            tma_prefetch_desc(&tmB1);
-        }
+        tma_prefetch_desc(&tmWg);
+        tma_prefetch_desc(&tmWu);
+        tma_prefetch_desc(&tmSg);
+        tma_prefetch_desc(&tmSu);
+        tma_prefetch_desc(&tmX0);
+        tma_prefetch_desc(&tmX1);
+        tma_prefetch_desc(&tmWd);
+        tma_prefetch_desc(&tmSd);
+        tma_prefetch_desc(&tmH);
     }
     if (warp == 1) {
         tmem_alloc(&sh.tmem_base, kTmemCols);
@@ -154,45 +205,68 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = sh.tmem_base;
+    // everything above overlapped the previous kernel; its results are needed from here on
+    grid_dependency_wait();
+    const int tot_up = __ldg(p.plan.up_start + p.n_entries);
+    const int total = tot_up + __ldg(p.plan.down_start + p.n_entries);
+    const int fb_up = (p.I + 63) / 64;
 
     if (warp == 0) {
-        // ------------------------------------------------------------ producer
+        // ------------------------------------------------------ scheduler + producer
         if (lane == 0) {
             const uint64_t pol_w = policy_evict_first();  // weights: read once
-            const uint64_t pol_b = policy_evict_last();   // token rows: reused by every feature block
+            const uint64_t pol_b = policy_evict_last();   // token / h rows: reused across feature blocks
             int stage = 0;
             uint32_t phase = 0;
             uint32_t armed = 0, armed_par = 0;  // per stage: a load issued / its parity
-            for (int item = blockIdx.x; item < total && !*abort; item += gridDim.x) {
+            int next = atomicAdd(p.sync, 1);
+            for (int s = 0;; ++s) {
+                const int slot = s % kSlots;
+                if (!mbar_wait(&sh.slot_empty[slot], ((uint32_t)(s / kSlots) & 1u) ^ 1u, abort)) break;
+                const int q = *abort ? total : next;
+                sh.slot_item[slot] = q;
+                mbar_arrive(&sh.slot_full[slot]);
+                if (q >= total) break;
+                next = atomicAdd(p.sync, 1);
                 TcItem it;
-                decode_item(p, item, it);
-                const CUtensorMap *ma0 = it.w.a_sel ? &tmS0 : &tmA0;
-                const CUtensorMap *ma1 = it.w.a_sel ? &tmS1 : &tmA1;
-                const CUtensorMap *mb = it.w.b_sel ? &tmB1 : &tmB0;
+                decode_item(p, tot_up, q, it);
+                if (!it.up) {  // the h rows of this expert must all be stored
+                    if (!wait_counter(p.sync + 1 + it.entry, it.w.ntb * fb_up, abort)) break;
+                    fence_proxy_async_global();
+                }
+                const CUtensorMap *ma0, *ma1, *mb;
+                if (it.up) {
+                    ma0 = it.w.a_sel ? &tmSg : &tmWg;
+                    ma1 = it.w.a_sel ? &tmSu : &tmWu;
+                    mb = it.w.b_sel ? &tmX1 : &tmX0;
+                } else {
+                    ma0 = ma1 = it.w.a_sel ? &tmSd : &tmWd;
+                    mb = &tmH;
+                }
+                const int gu = p.gu_mode[it.w.a_sel];
+                const int kcs = it.up ? p.kc_up : p.kc_down;
                 const int per = it.stream ? 2 : 1;
                 const int nbox = (it.w.bn + kBoxRows - 1) / kBoxRows;
                 const int brow0 = it.w.src_row0 + it.tb * it.w.bn;
-                const int arow0 = UP ? it.fb * 64 : it.fb * 128;
+                const int arow0 = it.up ? it.fb * 64 : it.fb * 128;
                 bool ok = true;
-                for (int kc = 0; kc < p.k_chunks; kc += per) {
+                for (int kc = 0; kc < kcs; kc += per) {
                     if (!mbar_wait(&sh.empty[stage], phase ^ 1u, abort)) { ok = false; break; }
-                    const int nch = min(per, p.k_chunks - kc);
+                    const int nch = min(per, kcs - kc);
                     unsigned char *sbase = stages + stage * kStageBytes;
                     mbar_arrive_expect_tx(&sh.full[stage],
                                           (uint32_t)nch * (16384u + (uint32_t)nbox * kBoxRows * 128u));
                     armed |= 1u << stage;
                     armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
                     for (int c = 0; c < nch; ++c) {
-                        const int k = chunk_at(kc + c, it.fb, p.k_chunks) * kChunkK;
+                        const int k = chunk_at(kc + c, it.fb, kcs) * kChunkK;
                         unsigned char *sa = sbase + a_off(it.stream, c);
                         unsigned char *sb = sbase + b_off(it.stream, c);
-                        if (UP) {
-                            if (p.gu_mode[it.w.a_sel] != kGateUpSplit) {
-                                tma_load_4d(sa, ma0, &sh.full[stage], k, arow0, it.w.a_idx, 0, pol_w);
-                            } else {
-                                tma_load_3d(sa, ma0, &sh.full[stage], k, arow0, it.w.a_idx, pol_w);
-                                tma_load_3d(sa + 8192, ma1, &sh.full[stage], k, arow0, it.w.a_idx, pol_w);
-                            }
+                        if (it.up && gu != kGateUpSplit) {
+                            tma_load_4d(sa, ma0, &sh.full[stage], k, arow0, it.w.a_idx, 0, pol_w);
+                        } else if (it.up) {
+                            tma_load_3d(sa, ma0, &sh.full[stage], k, arow0, it.w.a_idx, pol_w);
+                            tma_load_3d(sa + 8192, ma1, &sh.full[stage], k, arow0, it.w.a_idx, pol_w);
                         } else {
                             tma_load_3d(sa, ma0, &sh.full[stage], k, arow0, it.w.a_idx, pol_w);
                         }
@@ -210,26 +284,31 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
+        // ------------------------------------------------------ MMA issuer
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            int li = 0;
-            for (int item = blockIdx.x; item < total && !*abort; item += gridDim.x, ++li) {
+            for (int s = 0;; ++s) {
+                const int slot = s % kSlots;
+                if (!mbar_wait(&sh.slot_full[slot], (uint32_t)(s / kSlots) & 1u, abort)) break;
+                const int q = sh.slot_item[slot];
+                mbar_arrive(&sh.slot_empty[slot]);
+                if (q >= total) break;
                 TcItem it;
-                decode_item(p, item, it);
-                const int acc = li & 1;
-                const uint32_t use = (uint32_t)(li >> 1);
+                decode_item(p, tot_up, q, it);
+                const int acc = s & 1;
+                const uint32_t use = (uint32_t)(s >> 1);
                 if (!mbar_wait(&sh.tempty[acc], (use & 1u) ^ 1u, abort)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)acc * 256u;
                 const uint32_t idesc = idesc_bf16_f32(128, (uint32_t)it.w.bn);
+                const int kcs = it.up ? p.kc_up : p.kc_down;
                 const int per = it.stream ? 2 : 1;
                 bool ok = true;
-                for (int kc = 0; kc < p.k_chunks; kc += per) {
+                for (int kc = 0; kc < kcs; kc += per) {
                     if (!mbar_wait(&sh.full[stage], phase, abort)) { ok = false; break; }
                     tc_fence_after();
-                    const int nch = min(per, p.k_chunks - kc);
+                    const int nch = min(per, kcs - kc);
                     const uint32_t sbase = smem_u32(stages + stage * kStageBytes);
                     for (int c = 0; c < nch; ++c) {
                         const uint32_t sa = sbase + a_off(it.stream, c);
@@ -250,35 +329,44 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
             mbar_wait(&sh.drain, 0, nullptr);
         }
     } else {
-        // ------------------------------------------------------------ epilogue
-        const int q = warp & 3;            // TMEM lane quarter this warp may read
+        // ------------------------------------------------------ epilogue
+        const int q4 = warp & 3;           // TMEM lane quarter this warp may read
         const int et = threadIdx.x - 64;   // 0 .. 127
-        int li = 0;
-        for (int item = blockIdx.x; item < total; item += gridDim.x, ++li) {
-            TcItem it;
-            decode_item(p, item, it);
-            const int acc = li & 1;
-            const uint32_t use = (uint32_t)(li >> 1);
-            // one thread waits, all 128 take the same decision
-            if (et == 0) sh.epi_ok = mbar_wait(&sh.tfull[acc], use & 1u, abort) ? 1 : 0;
+        for (int s = 0;; ++s) {
+            // the leader takes the next item and waits for its accumulator;
+            // all 128 threads then act on the same decision
+            if (et == 0) {
+                const int slot = s % kSlots;
+                int q = -1;
+                if (mbar_wait(&sh.slot_full[slot], (uint32_t)(s / kSlots) & 1u, abort)) {
+                    q = sh.slot_item[slot];
+                    mbar_arrive(&sh.slot_empty[slot]);
+                    if (q < total && !mbar_wait(&sh.tfull[s & 1], (uint32_t)(s >> 1) & 1u, abort))
+                        q = -1;
+                }
+                sh.epi_item = q;
+            }
             named_bar_sync(1, 128);
-            const int ok = *(volatile int *)&sh.epi_ok;
+            const int q = *(volatile int *)&sh.epi_item;
             named_bar_sync(1, 128);
-            if (!ok) break;
+            if (q < 0 || q >= total) break;
             tc_fence_after();
-            const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)acc * 256u;
+            TcItem it;
+            decode_item(p, tot_up, q, it);
+            const int acc = s & 1;
+            const uint32_t tbase = tmem_base + ((uint32_t)(32 * q4) << 16) + (uint32_t)acc * 256u;
             const size_t row0 = (size_t)it.w.dst_row0 + (size_t)it.tb * it.w.bn;
             for (int c0 = 0; c0 < it.n_valid; c0 += 32) {
                 uint32_t v[32];
                 tmem_ld_32x32b_x32(tbase + (uint32_t)c0, v);
                 tmem_ld_wait();
-                if (UP) {
+                if (it.up) {
                     float *U = reinterpret_cast<float *>(epi);                 // [32 cols][64 features]
                     uint16_t *H = reinterpret_cast<uint16_t *>(epi + 8192);    // [32 cols][64 features]
                     // lanes 0-63 hold gate and 64-127 up, or the reverse for an up-first tile
                     const bool gate_hi = p.gu_mode[it.w.a_sel] == kUpGateFused;
-                    const bool is_gate = (q < 2) != gate_hi;
-                    const int f = (q & 1) * 32 + lane;
+                    const bool is_gate = (q4 < 2) != gate_hi;
+                    const int f = (q4 & 1) * 32 + lane;
                     if (!is_gate) {
 #pragma unroll
                         for (int j = 0; j < 32; ++j) U[j * 64 + f] = __uint_as_float(v[j]);
@@ -296,22 +384,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
                     for (int idx = et; idx < 32 * 8; idx += 128) {
                         const int r = idx >> 3, vv = idx & 7;
                         const int col = c0 + r, feat = it.fb * 64 + vv * 8;
-                        if (col < it.n_valid && feat < p.out_cols)
-                            *reinterpret_cast<uint4 *>(p.out + (row0 + col) * p.out_cols + feat) =
+                        if (col < it.n_valid && feat < p.I)
+                            *reinterpret_cast<uint4 *>(p.h + (row0 + col) * p.I + feat) =
                                 *reinterpret_cast<const uint4 *>(H + r * 64 + vv * 8);
                     }
                     named_bar_sync(1, 128);
                 } else {
                     uint16_t *Y = reinterpret_cast<uint16_t *>(epi);  // [32 cols][128 features]
-                    const int f = q * 32 + lane;
+                    const int f = q4 * 32 + lane;
 #pragma unroll
                     for (int j = 0; j < 32; ++j) Y[j * 128 + f] = to_bf16_bits(__uint_as_float(v[j]));
                     named_bar_sync(1, 128);
                     for (int idx = et; idx < 32 * 16; idx += 128) {
                         const int r = idx >> 4, vv = idx & 15;
                         const int col = c0 + r, feat = it.fb * 128 + vv * 8;
-                        if (col < it.n_valid && feat < p.out_cols)
-                            *reinterpret_cast<uint4 *>(p.out + (row0 + col) * p.out_cols + feat) =
+                        if (col < it.n_valid && feat < p.d)
+                            *reinterpret_cast<uint4 *>(p.y + (row0 + col) * p.d + feat) =
                                 *reinterpret_cast<const uint4 *>(Y + r * 128 + vv * 8);
                     }
                     named_bar_sync(1, 128);
@@ -319,6 +407,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
             }
             tc_fence_before();
             mbar_arrive(&sh.tempty[acc]);
+            if (it.up) {
+                // publish this item's h rows to the down-projection items of the expert
+                fence_proxy_async_global();
+                __threadfence();
+                named_bar_sync(1, 128);
+                if (et == 0) atomicAdd(p.sync + 1 + it.entry, 1);
+            }
         }
     }
 
@@ -329,7 +424,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// Host side: tensor maps and launches.
+// Host side: tensor maps and the launch.
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -348,35 +443,33 @@ static EncodeTiledFn get_encode_fn() {
     return fn;
 }
 
-// bf16 map over a row-major [outer][rows][cols] tensor (outer = 1 for 2-D),
-// box = [box_rows][64 cols], 128-byte swizzle, zero fill out of bounds.
-static bool encode_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows,
-                       uint64_t outer, uint32_t box_rows) {
+static bool encode(CUtensorMap *m, const void *base, cuuint32_t rank, const cuuint64_t *dims,
+                   const cuuint64_t *strides, const cuuint32_t *box) {
     EncodeTiledFn fn = get_encode_fn();
     if (!fn) return false;
-    const cuuint64_t dims[3] = {cols, rows, outer};
-    const cuuint64_t strides[2] = {cols * 2, cols * rows * 2};
-    const cuuint32_t box[3] = {(cuuint32_t)kChunkK, box_rows, 1};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    const cuuint32_t rank = outer > 1 ? 3 : 2;
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), dims,
-                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), dims, strides,
+              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+// bf16 [experts][rows][cols] weights, box = [box_rows][64 cols] of one expert
 static bool encode_weights(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows,
                            uint64_t experts, uint32_t box_rows) {
-    EncodeTiledFn fn = get_encode_fn();
-    if (!fn) return false;
     const cuuint64_t dims[3] = {cols, rows, experts};
     const cuuint64_t strides[2] = {cols * 2, cols * rows * 2};
     const cuuint32_t box[3] = {(cuuint32_t)kChunkK, box_rows, 1};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
-              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return encode(m, base, 3, dims, strides, box);
 }
+
+// bf16 [rows][cols] row matrix, box = [64 rows][64 cols]
+static bool encode_rows(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows) {
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kChunkK, (cuuint32_t)kBoxRows};
+    return encode(m, base, 2, dims, strides, box);
+}
+
 // One map over both the gate and the up tensor ([E][rows][cols] each, dense):
 // dims {cols, rows, E, 2}, the last dimension stepping from one tensor to the
 // other, so a {64, 64, 1, 2} box is one 16 KB copy of 64 gate rows followed by
@@ -386,8 +479,6 @@ static bool encode_weights(CUtensorMap *m, const void *base, uint64_t cols, uint
 // and the caller then uses two 3-D maps.
 static int encode_gate_up(CUtensorMap *m, const void *gate, const void *up, uint64_t cols,
                           uint64_t rows, uint64_t experts) {
-    EncodeTiledFn fn = get_encode_fn();
-    if (!fn) return kGateUpSplit;
     const int64_t bytes = (int64_t)(cols * rows * experts * 2);
     const int64_t delta = static_cast<const char *>(up) - static_cast<const char *>(gate);
     int mode;
@@ -406,15 +497,7 @@ static int encode_gate_up(CUtensorMap *m, const void *gate, const void *up, uint
     const cuuint64_t dims[4] = {cols, rows, experts, 2};
     const cuuint64_t strides[3] = {cols * 2, cols * rows * 2, step};
     const cuuint32_t box[4] = {(cuuint32_t)kChunkK, 64, 1, 2};
-    const cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
-                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? mode : kGateUpSplit;
-}
-
-static bool encode_rows(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows) {
-    return encode_map(m, base, cols, rows, 1, kBoxRows);
+    return encode(m, base, 4, dims, strides, box) ? mode : kGateUpSplit;
 }
 
 static size_t tc_smem_bytes() {
@@ -423,6 +506,7 @@ static size_t tc_smem_bytes() {
 
 cudaError_t launch_ffn_tc(const moge_config &c, const Plan &plan, int n_entries,
                           const FfnOperands &op, int num_sms, cudaStream_t st, cudaEvent_t mid) {
+    (void)mid;
     if (n_entries <= 0 || c.T <= 0) return cudaSuccess;
     const int N = c.N, S = c.S, d = c.d, I = c.I;
     // routed / shared weight tensors; a missing side borrows the other's
@@ -435,38 +519,35 @@ cudaError_t launch_ffn_tc(const moge_config &c, const Plan &plan, int n_entries,
     const int64_t r0 = op.b0 ? op.b0_rows : op.b1_rows, r1 = op.b1 ? op.b1_rows : op.b0_rows;
 
     CUtensorMap mWg, mWu, mSg, mSu, mX0, mX1, mWd, mSd, mH;
-    int gu_mode[2];
-    gu_mode[0] = encode_gate_up(&mWg, wg, wu, d, I, ne);
-    gu_mode[1] = encode_gate_up(&mSg, sg, su, d, I, ns);
-    if (gu_mode[0] != kGateUpSplit) mWu = mWg;
+    TcParams p;
+    p.gu_mode[0] = encode_gate_up(&mWg, wg, wu, d, I, ne);
+    p.gu_mode[1] = encode_gate_up(&mSg, sg, su, d, I, ns);
+    if (p.gu_mode[0] != kGateUpSplit) mWu = mWg;
     else if (!encode_weights(&mWg, wg, d, I, ne, 64) || !encode_weights(&mWu, wu, d, I, ne, 64))
         return cudaErrorInvalidValue;
-    if (gu_mode[1] != kGateUpSplit) mSu = mSg;
+    if (p.gu_mode[1] != kGateUpSplit) mSu = mSg;
     else if (!encode_weights(&mSg, sg, d, I, ns, 64) || !encode_weights(&mSu, su, d, I, ns, 64))
         return cudaErrorInvalidValue;
     if (!encode_rows(&mX0, b0, d, (uint64_t)r0) || !encode_rows(&mX1, b1, d, (uint64_t)r1) ||
         !encode_weights(&mWd, wd, I, d, ne, 128) || !encode_weights(&mSd, sd, I, d, ns, 128) ||
         !encode_rows(&mH, op.h, I, (uint64_t)op.h_rows))
         return cudaErrorInvalidValue;
+    p.plan = plan;
+    p.n_entries = n_entries;
+    p.kc_up = (d + kChunkK - 1) / kChunkK;
+    p.kc_down = (I + kChunkK - 1) / kChunkK;
+    p.I = I;
+    p.d = d;
+    p.h = (uint16_t *)op.h;
+    p.y = (uint16_t *)op.y;
+    p.sync = plan.sync;
 
     const size_t smem = tc_smem_bytes();
-    cudaError_t e = cudaFuncSetAttribute(ffn_tc_kernel<true>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(ffn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(ffn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-    if (e != cudaSuccess) return e;
-
-    TcParams pu{{gu_mode[0], gu_mode[1]}, plan.up, plan.up_start, n_entries,
-                (d + kChunkK - 1) / kChunkK, I, (uint16_t *)op.h};
-    ffn_tc_kernel<true><<<num_sms, kTcThreads, smem, st>>>(pu, mWg, mWu, mSg, mSu, mX0, mX1);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    if (mid && (e = cudaEventRecord(mid, st)) != cudaSuccess) return e;
-    TcParams pd{{kGateUpSplit, kGateUpSplit}, plan.down, plan.down_start, n_entries,
-                (I + kChunkK - 1) / kChunkK, d, (uint16_t *)op.y};
-    ffn_tc_kernel<false><<<num_sms, kTcThreads, smem, st>>>(pd, mWd, mWd, mSd, mSd, mH, mH);
-    return cudaGetLastError();
+    return launch_pdl(ffn_tc_kernel, dim3(num_sms), dim3(kTcThreads), smem, st, p, mWg, mWu, mSg,
+                      mSu, mX0, mX1, mWd, mSd, mH);
 }
 
 }  // namespace moge

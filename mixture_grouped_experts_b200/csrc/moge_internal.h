@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/moge.h"
 
 namespace moge {
@@ -41,6 +43,8 @@ struct Plan {
     ExpertWork *down;   // [n_entries]
     int *up_start;      // [n_entries + 1] prefix sum of items (ntb * feature blocks)
     int *down_start;    // [n_entries + 1]
+    int *sync;          // [n_entries + 1] work-queue counter and per-entry finished
+                        // up-projection items; zeroed by the kernel that writes the plan
 };
 
 // Workspace carve-up (all regions 256-byte aligned).
@@ -61,6 +65,26 @@ struct Workspace {
     size_t total;
 };
 Workspace carve_workspace(const moge_config &c, void *base);
+
+// Launch with programmatic stream serialisation (the kernel starts its
+// prologue while the previous kernel on the stream drains; every kernel of
+// this library calls grid_dependency_wait() before its first global access),
+// optionally as clusters of `cluster` CTAs.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // ---------------------------------------------------------------- launchers
 // Each returns a cudaError_t of the launch.

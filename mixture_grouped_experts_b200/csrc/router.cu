@@ -154,6 +154,7 @@ __global__ void __launch_bounds__(kRouterThreads, 2) router_bf16_kernel(
     extern __shared__ __align__(16) unsigned char smem_raw[];
     unsigned char *stage = smem_raw;  // [2][kRouterStageBytes]
     RouterSmem &sm = *reinterpret_cast<RouterSmem *>(smem_raw + 2 * kRouterStageBytes);
+    grid_dependency_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, q = lane & 3;
     const int crank = blockIdx.x % ks;
@@ -266,6 +267,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_f32_kernel(
     extern __shared__ __align__(16) unsigned char smem_raw[];
     RouterSmem &sm = *reinterpret_cast<RouterSmem *>(smem_raw);
     const int t0 = blockIdx.x * kRouterTile;
+    grid_dependency_wait();
     const int ntok = min(kRouterTile, c.T - t0);
     for (int o = threadIdx.x; o < kRouterTile * c.N; o += blockDim.x) {
         const int tt = o / c.N, e = o % c.N;
@@ -290,9 +292,9 @@ cudaError_t launch_router(const moge_config &c, const void *x, const void *w_rou
         cudaError_t e = cudaFuncSetAttribute(router_f32_kernel,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        router_f32_kernel<<<tiles, kRouterThreads, smem, st>>>(
-            c, (const float *)x, (const float *)w_router, bias, topk_idx, topk_w, hist, rank);
-        return cudaGetLastError();
+        return launch_pdl(router_f32_kernel, dim3(tiles), dim3(kRouterThreads), smem, st, c,
+                          (const float *)x, (const float *)w_router, bias, topk_idx, topk_w, hist,
+                          rank);
     }
     // Split the hidden dimension over a cluster of up to 8 CTAs while the
     // grid stays within two CTAs per SM, each CTA keeps >= 2 blocks of work,
@@ -311,13 +313,15 @@ cudaError_t launch_router(const moge_config &c, const void *x, const void *w_rou
     cfg.blockDim = dim3(kRouterThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = ks;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, router_bf16_kernel, c, (const uint16_t *)x,
                               (const uint16_t *)w_router, bias, topk_idx, topk_w, hist, rank, ks);
 }
@@ -352,33 +356,36 @@ __device__ int block_exclusive_scan_1024(int v, int *wbuf /* [32] */, int *total
     return pre;
 }
 
-// Work plan of the grouped FFN, one entry per thread: routed experts 0..N-1
-// (if with_routed, rows from offs[]), then shared experts 0..S-1 (if
-// with_shared, T rows each, their h / y rows after shared_row_base).
-// Token-tile width: <= kStreamRows rows -> one streaming tile of
+// Work plan of the grouped FFN, one entry per thread: shared experts 0..S-1
+// first (if with_shared; T rows each, their h / y rows after shared_row_base),
+// then routed experts 0..N-1 (if with_routed, rows from offs[]). The grouped
+// FFN hands its work out in this order, so the heavy shared-expert items come
+// first. Token-tile width: <= kStreamRows rows -> one streaming tile of
 // round16(rows); more -> ceil(rows / 256) balanced tiles of round16 width.
+// Also zeroes the FFN's work-queue counter and per-entry completion counters.
 // Called by all 1024 threads of the block.
 __device__ void build_plan_block(const moge_config &c, const int32_t *offs, Plan plan,
                                  bool with_routed, bool with_shared, int shared_row_base,
                                  int *wbuf) {
     const int fb_up = (c.I + 63) / 64;      // 64 gate + 64 up rows per tile
     const int fb_down = (c.d + 127) / 128;  // 128 output features per tile
-    const int nr = with_routed ? c.N : 0;
-    const int n = nr + (with_shared ? c.S : 0);
+    const int ns = with_shared ? c.S : 0;
+    const int n = ns + (with_routed ? c.N : 0);
     const int i = threadIdx.x;
     ExpertWork u = {}, dn = {};
     int items_up = 0, items_down = 0;
+    if (i <= n) plan.sync[i] = 0;
     if (i < n) {
         int rows, a_sel, a_idx, up_src, up_bsel, mid;
-        if (i < nr) {
-            rows = offs[i + 1] - offs[i];
-            a_sel = 0; a_idx = i; up_src = offs[i]; up_bsel = 0; mid = offs[i];
+        if (i >= ns) {
+            const int e = i - ns;
+            rows = offs[e + 1] - offs[e];
+            a_sel = 0; a_idx = e; up_src = offs[e]; up_bsel = 0; mid = offs[e];
         } else {
-            const int sidx = i - nr;
             rows = c.T;
-            a_sel = 1; a_idx = sidx; up_src = 0; up_bsel = 1; mid = shared_row_base + sidx * c.T;
+            a_sel = 1; a_idx = i; up_src = 0; up_bsel = 1; mid = shared_row_base + i * c.T;
         }
-        int bn, ntb;
+    int bn, ntb;
         if (rows <= 0) {
             bn = 16; ntb = 0;
         } else if (rows <= kStreamRows) {
@@ -424,6 +431,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(moge_config c, const int32_t
     __shared__ int32_t cnt_s[kMaxExperts];
     __shared__ int32_t off_s[kMaxExperts + 1];
     __shared__ int wbuf[32];
+    grid_dependency_wait();
     const int N = c.N;
     const int tiles = (c.T + kRouterTile - 1) / kRouterTile;
     const int P = 1024 / N;  // chunks of tiles
@@ -480,9 +488,8 @@ cudaError_t launch_scan(const moge_config &c, const int32_t *hist, int32_t *base
                         int32_t *offsets, const Plan *plan, bool with_routed, bool with_shared,
                         cudaStream_t st) {
     Plan p = plan ? *plan : Plan{nullptr, nullptr, nullptr, nullptr};
-    scan_kernel<<<1, 1024, 0, st>>>(c, hist, base, counts, offsets, p, plan ? 1 : 0,
-                                    with_routed ? 1 : 0, with_shared ? 1 : 0);
-    return cudaGetLastError();
+    return launch_pdl(scan_kernel, dim3(1), dim3(1024), 0, st, c, hist, base, counts, offsets, p,
+                      plan ? 1 : 0, with_routed ? 1 : 0, with_shared ? 1 : 0);
 }
 
 // Plan from the caller's offsets (routed only) or for the shared experts only.
@@ -490,6 +497,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(moge_config c, const int32_t
                                                      int with_routed, int with_shared) {
     __shared__ int32_t off_s[kMaxExperts + 1];
     __shared__ int wbuf[32];
+    grid_dependency_wait();
     if (with_routed)
         for (int i = threadIdx.x; i <= c.N; i += blockDim.x) off_s[i] = offsets[i];
     __syncthreads();
@@ -499,8 +507,8 @@ __global__ void __launch_bounds__(1024) plan_kernel(moge_config c, const int32_t
 
 cudaError_t launch_plan(const moge_config &c, const int32_t *offsets, const Plan &plan,
                         bool with_routed, bool with_shared, cudaStream_t st) {
-    plan_kernel<<<1, 1024, 0, st>>>(c, offsets, plan, with_routed ? 1 : 0, with_shared ? 1 : 0);
-    return cudaGetLastError();
+    return launch_pdl(plan_kernel, dim3(1), dim3(1024), 0, st, c, offsets, plan,
+                      with_routed ? 1 : 0, with_shared ? 1 : 0);
 }
 
 // ---------------------------------------------------------------------------
@@ -509,6 +517,7 @@ __global__ void finalize_kernel(moge_config c, const int32_t *__restrict__ topk_
                                 const int32_t *__restrict__ rank, const int32_t *__restrict__ base,
                                 const int32_t *__restrict__ offsets, int32_t *perm_src,
                                 int32_t *perm_dst) {
+    grid_dependency_wait();
     const int K = c.M * c.Kp;
     const long long n = (long long)c.T * K;
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
@@ -530,9 +539,8 @@ cudaError_t launch_finalize(const moge_config &c, const int32_t *topk_idx, const
                             int32_t *perm_dst, cudaStream_t st) {
     const long long n = (long long)c.T * c.M * c.Kp;
     const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
-    finalize_kernel<<<blocks > 0 ? blocks : 1, 256, 0, st>>>(c, topk_idx, rank, base, offsets,
-                                                             perm_src, perm_dst);
-    return cudaGetLastError();
+    return launch_pdl(finalize_kernel, dim3(blocks > 0 ? blocks : 1), dim3(256), 0, st, c, topk_idx,
+                      rank, base, offsets, perm_src, perm_dst);
 }
 
 }  // namespace moge

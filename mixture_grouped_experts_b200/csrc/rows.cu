@@ -24,6 +24,7 @@ __global__ void __launch_bounds__(kRowThreads) scatter_rows_kernel(
     const int32_t *__restrict__ rank, const int32_t *__restrict__ base,
     const int32_t *__restrict__ offsets, int32_t *perm_src, int32_t *perm_dst, uint4 *x_perm) {
     __shared__ int dst_s[kMaxExperts];
+    grid_dependency_wait();
     const int t = blockIdx.x;
     const int K = c.M * c.Kp;
     const int nvec = c.d / vec_elems(c.dtype);
@@ -55,15 +56,15 @@ cudaError_t launch_scatter_rows(const moge_config &c, const void *x, const int32
                                 const int32_t *rank, const int32_t *base, const int32_t *offsets,
                                 int32_t *perm_src, int32_t *perm_dst, void *x_perm,
                                 cudaStream_t st) {
-    scatter_rows_kernel<<<c.T, kRowThreads, 0, st>>>(c, (const uint4 *)x, topk_idx, rank, base,
-                                                     offsets, perm_src, perm_dst, (uint4 *)x_perm);
-    return cudaGetLastError();
+    return launch_pdl(scatter_rows_kernel, dim3(c.T), dim3(kRowThreads), 0, st, c, (const uint4 *)x,
+                      topk_idx, rank, base, offsets, perm_src, perm_dst, (uint4 *)x_perm);
 }
 
 // x_perm[r] = x[perm_src[r]], one CTA per destination row
 __global__ void __launch_bounds__(kRowThreads) gather_rows_kernel(
     moge_config c, const uint4 *__restrict__ x, const int32_t *__restrict__ perm_src,
     uint4 *x_perm) {
+    grid_dependency_wait();
     const int r = blockIdx.x;
     const int nvec = c.d / vec_elems(c.dtype);
     const int t = perm_src[r];
@@ -79,9 +80,8 @@ __global__ void __launch_bounds__(kRowThreads) gather_rows_kernel(
 cudaError_t launch_gather_rows(const moge_config &c, const void *x, const int32_t *perm_src,
                                void *x_perm, cudaStream_t st) {
     const int rows = c.T * c.M * c.Kp;
-    gather_rows_kernel<<<rows, kRowThreads, 0, st>>>(c, (const uint4 *)x, perm_src,
-                                                     (uint4 *)x_perm);
-    return cudaGetLastError();
+    return launch_pdl(gather_rows_kernel, dim3(rows), dim3(kRowThreads), 0, st, c, (const uint4 *)x,
+                      perm_src, (uint4 *)x_perm);
 }
 
 // ---------------------------------------------------------------------------
@@ -151,6 +151,7 @@ __global__ void __launch_bounds__(kRowThreads) combine_kernel(
     int n_shared, const void *residual, void *y) {
     __shared__ const char *src_s[2 * kMaxExperts + 1];
     __shared__ float w_s[kMaxExperts];
+    grid_dependency_wait();
     const int t = blockIdx.x;
     const int nvec = d / 8;
     const size_t row_bytes = (size_t)d * (DT == MOGE_BF16 ? 2 : 4);
@@ -206,13 +207,9 @@ __global__ void __launch_bounds__(kRowThreads) combine_kernel(
 cudaError_t launch_combine(const moge_config &c, const void *y_perm, const float *topk_w,
                            const int32_t *perm_dst, int K, const void *shared_rows,
                            int n_shared_blocks, const void *residual, void *y, cudaStream_t st) {
-    if (c.dtype == MOGE_BF16)
-        combine_kernel<MOGE_BF16><<<c.T, kRowThreads, 0, st>>>(
-            c.T, c.d, c.N, y_perm, topk_w, perm_dst, K, shared_rows, n_shared_blocks, residual, y);
-    else
-        combine_kernel<MOGE_F32><<<c.T, kRowThreads, 0, st>>>(
-            c.T, c.d, c.N, y_perm, topk_w, perm_dst, K, shared_rows, n_shared_blocks, residual, y);
-    return cudaGetLastError();
+    auto kern = c.dtype == MOGE_BF16 ? combine_kernel<MOGE_BF16> : combine_kernel<MOGE_F32>;
+    return launch_pdl(kern, dim3(c.T), dim3(kRowThreads), 0, st, c.T, c.d, c.N, y_perm, topk_w,
+                      perm_dst, K, shared_rows, n_shared_blocks, residual, y);
 }
 
 // ---------------------------------------------------------------------------
@@ -221,6 +218,7 @@ template <int DT>
 __global__ void __launch_bounds__(kRowThreads) rmsnorm_kernel(int d, const void *__restrict__ x,
                                                               float eps, void *u) {
     __shared__ float red[kRowThreads / 32];
+    grid_dependency_wait();
     const int t = blockIdx.x;
     const int nvec = d / 8;
     const size_t esz = DT == MOGE_BF16 ? 2 : 4;
@@ -251,11 +249,8 @@ __global__ void __launch_bounds__(kRowThreads) rmsnorm_kernel(int d, const void 
 
 cudaError_t launch_rmsnorm(const moge_config &c, const void *x, float eps, void *u,
                            cudaStream_t st) {
-    if (c.dtype == MOGE_BF16)
-        rmsnorm_kernel<MOGE_BF16><<<c.T, kRowThreads, 0, st>>>(c.d, x, eps, u);
-    else
-        rmsnorm_kernel<MOGE_F32><<<c.T, kRowThreads, 0, st>>>(c.d, x, eps, u);
-    return cudaGetLastError();
+    auto kern = c.dtype == MOGE_BF16 ? rmsnorm_kernel<MOGE_BF16> : rmsnorm_kernel<MOGE_F32>;
+    return launch_pdl(kern, dim3(c.T), dim3(kRowThreads), 0, st, c.d, x, eps, u);
 }
 
 }  // namespace moge
