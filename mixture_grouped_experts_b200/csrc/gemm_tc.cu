@@ -6,6 +6,7 @@
 //   warp 0    scheduler + TMA producer: takes work items from a global queue
 //             (an atomic counter), publishes them to the other roles through
 //             a small shared-memory ring, and streams their operands with TMA
+//             (the copies of a stage issued by several lanes at once)
 //   warp 1    MMA issuer   (tcgen05.mma kind::f16, M = 128, N = token tile,
 //                           fp32 accumulators in TMEM, double-buffered)
 //   warps 2-5 epilogue     (tcgen05.ld -> registers -> smem -> coalesced
@@ -213,75 +214,95 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
 
     if (warp == 0) {
         // ------------------------------------------------------ scheduler + producer
-        if (lane == 0) {
-            const uint64_t pol_w = policy_evict_first();  // weights: read once
-            const uint64_t pol_b = policy_evict_last();   // token / h rows: reused across feature blocks
-            int stage = 0;
-            uint32_t phase = 0;
-            uint32_t armed = 0, armed_par = 0;  // per stage: a load issued / its parity
-            int next = atomicAdd(p.sync, 1);
-            for (int s = 0;; ++s) {
-                const int slot = s % kSlots;
-                if (!mbar_wait(&sh.slot_empty[slot], ((uint32_t)(s / kSlots) & 1u) ^ 1u, abort)) break;
-                const int q = *abort ? total : next;
-                sh.slot_item[slot] = q;
-                mbar_arrive(&sh.slot_full[slot]);
-                if (q >= total) break;
-                next = atomicAdd(p.sync, 1);
-                TcItem it;
-                decode_item(p, tot_up, q, it);
-                if (!it.up) {  // the h rows of this expert must all be stored
-                    if (!wait_counter(p.sync + 1 + it.entry, it.w.ntb * fb_up, abort)) break;
-                    fence_proxy_async_global();
-                }
-                const CUtensorMap *ma0, *ma1, *mb;
-                if (it.up) {
-                    ma0 = it.w.a_sel ? &tmSg : &tmWg;
-                    ma1 = it.w.a_sel ? &tmSu : &tmWu;
-                    mb = it.w.b_sel ? &tmX1 : &tmX0;
+        // Lane 0 schedules and keeps the stage ring; the copies of a stage are
+        // issued by several lanes at once (one copy per lane): a single thread
+        // issuing them one after another cannot keep up with the tensor cores.
+        const uint64_t pol_w = policy_evict_first();  // weights: read once
+        const uint64_t pol_b = policy_evict_last();   // token / h rows: reused across feature blocks
+        int stage = 0;
+        uint32_t phase = 0;
+        uint32_t armed = 0, armed_par = 0;  // lane 0: per stage, a load issued / its parity
+        int next = lane == 0 ? atomicAdd(p.sync, 1) : 0;
+        for (int s = 0;; ++s) {
+            const int slot = s % kSlots;
+            int q = 0;
+            if (lane == 0) {
+                if (mbar_wait(&sh.slot_empty[slot], ((uint32_t)(s / kSlots) & 1u) ^ 1u, abort)) {
+                    q = *abort ? total : next;
+                    sh.slot_item[slot] = q;
+                    mbar_arrive(&sh.slot_full[slot]);
+                    if (q < total) next = atomicAdd(p.sync, 1);
                 } else {
-                    ma0 = ma1 = it.w.a_sel ? &tmSd : &tmWd;
-                    mb = &tmH;
+                    q = -1;
                 }
-                const int gu = p.gu_mode[it.w.a_sel];
-                const int kcs = it.up ? p.kc_up : p.kc_down;
-                const int per = it.stream ? 2 : 1;
-                const int nbox = (it.w.bn + kBoxRows - 1) / kBoxRows;
-                const int brow0 = it.w.src_row0 + it.tb * it.w.bn;
-                const int arow0 = it.up ? it.fb * 64 : it.fb * 128;
-                bool ok = true;
-                for (int kc = 0; kc < kcs; kc += per) {
-                    if (!mbar_wait(&sh.empty[stage], phase ^ 1u, abort)) { ok = false; break; }
-                    const int nch = min(per, kcs - kc);
-                    unsigned char *sbase = stages + stage * kStageBytes;
+            }
+            q = __shfl_sync(0xffffffffu, q, 0);
+            if (q < 0 || q >= total) break;
+            TcItem it;
+            decode_item(p, tot_up, q, it);
+            if (!it.up) {  // the h rows of this expert must all be stored
+                int ok = 1;
+                if (lane == 0) ok = wait_counter(p.sync + 1 + it.entry, it.w.ntb * fb_up, abort);
+                if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+                fence_proxy_async_global();
+            }
+            const CUtensorMap *ma0, *ma1, *mb;
+            if (it.up) {
+                ma0 = it.w.a_sel ? &tmSg : &tmWg;
+                ma1 = it.w.a_sel ? &tmSu : &tmWu;
+                mb = it.w.b_sel ? &tmX1 : &tmX0;
+            } else {
+                ma0 = ma1 = it.w.a_sel ? &tmSd : &tmWd;
+                mb = &tmH;
+            }
+            const int gu = p.gu_mode[it.w.a_sel];
+            const int na = (it.up && gu == kGateUpSplit) ? 2 : 1;  // weight copies per chunk
+            const int kcs = it.up ? p.kc_up : p.kc_down;
+            const int per = it.stream ? 2 : 1;
+            const int nbox = (it.w.bn + kBoxRows - 1) / kBoxRows;
+            const int brow0 = it.w.src_row0 + it.tb * it.w.bn;
+            const int arow0 = it.up ? it.fb * 64 : it.fb * 128;
+            // this lane's copy in every stage: chunk c, copy r of that chunk
+            const int ops = na + nbox;
+            const int my_c = lane / ops, my_r = lane % ops;
+            bool ok = true;
+            for (int kc = 0; kc < kcs; kc += per) {
+                int got = 1;
+                if (lane == 0) got = mbar_wait(&sh.empty[stage], phase ^ 1u, abort);
+                if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
+                const int nch = min(per, kcs - kc);
+                unsigned char *sbase = stages + stage * kStageBytes;
+                if (lane == 0) {
                     mbar_arrive_expect_tx(&sh.full[stage],
                                           (uint32_t)nch * (16384u + (uint32_t)nbox * kBoxRows * 128u));
                     armed |= 1u << stage;
                     armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
-                    for (int c = 0; c < nch; ++c) {
-                        const int k = chunk_at(kc + c, it.fb, kcs) * kChunkK;
-                        unsigned char *sa = sbase + a_off(it.stream, c);
-                        unsigned char *sb = sbase + b_off(it.stream, c);
-                        if (it.up && gu != kGateUpSplit) {
-                            tma_load_4d(sa, ma0, &sh.full[stage], k, arow0, it.w.a_idx, 0, pol_w);
-                        } else if (it.up) {
-                            tma_load_3d(sa, ma0, &sh.full[stage], k, arow0, it.w.a_idx, pol_w);
-                            tma_load_3d(sa + 8192, ma1, &sh.full[stage], k, arow0, it.w.a_idx, pol_w);
-                        } else {
-                            tma_load_3d(sa, ma0, &sh.full[stage], k, arow0, it.w.a_idx, pol_w);
-                        }
-                        for (int j = 0; j < nbox; ++j)
-                            tma_load_2d(sb + j * kBoxRows * 128, mb, &sh.full[stage], k,
-                                        brow0 + j * kBoxRows, pol_b);
-                    }
-                    if (++stage == kStages) { stage = 0; phase ^= 1u; }
                 }
-                if (!ok) break;
+                __syncwarp();
+                if (my_c < nch) {
+                    const int k = chunk_at(kc + my_c, it.fb, kcs) * kChunkK;
+                    unsigned char *sa = sbase + a_off(it.stream, my_c);
+                    unsigned char *sb = sbase + b_off(it.stream, my_c);
+                    if (my_r >= na) {
+                        const int j = my_r - na;
+                        tma_load_2d(sb + j * kBoxRows * 128, mb, &sh.full[stage], k,
+                                    brow0 + j * kBoxRows, pol_b);
+                    } else if (it.up && gu != kGateUpSplit) {
+                        tma_load_4d(sa, ma0, &sh.full[stage], k, arow0, it.w.a_idx, 0, pol_w);
+                    } else if (it.up) {
+                        tma_load_3d(sa + 8192 * my_r, my_r ? ma1 : ma0, &sh.full[stage], k, arow0,
+                                    it.w.a_idx, pol_w);
+                    } else {
+                        tma_load_3d(sa, ma0, &sh.full[stage], k, arow0, it.w.a_idx, pol_w);
+                    }
+                }
+                if (++stage == kStages) { stage = 0; phase ^= 1u; }
             }
-            if (*abort) {  // let every issued copy land before the CTA can exit
-                for (int s = 0; s < kStages; ++s)
-                    if (armed & (1u << s)) mbar_wait(&sh.full[s], (armed_par >> s) & 1u, nullptr);
-            }
+            if (!ok) break;
+        }
+        if (lane == 0 && *abort) {  // let every issued copy land before the CTA can exit
+            for (int s = 0; s < kStages; ++s)
+                if (armed & (1u << s)) mbar_wait(&sh.full[s], (armed_par >> s) & 1u, nullptr);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer
