@@ -253,12 +253,29 @@ def measure(cfg, inp, steps, warmup, dist_on=False, with_e2e=True):
 
 
 def max_over_ranks(v, dist_on):
+    """Max of a per-rank scalar over all ranks (identity on one process).
+    Uses a CUDA tensor under NCCL and a CPU tensor under gloo."""
     if not dist_on:
         return v
     import torch
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_inputs(cfg, rank, with_weights=True):
+    """Inputs of one data-parallel rank: every rank holds the same weights
+    (replicas) and its own token batch (x drawn from a rank-specific stream)."""
+    inp = synth.layer_inputs(cfg, x_stream_offset=rank) if with_weights else {
+        "x": synth.normal(cfg.seed, synth.STREAM_X + 1000 * rank, cfg.T * cfg.d, cfg.x_std,
+                          cfg.dtype).reshape(cfg.T, cfg.d)}
+    return inp
+
+
+def job_throughput(tokens_per_rank, world, max_ms):
+    """Whole-job tokens/s: all ranks' tokens over the slowest rank's step time."""
+    return world * tokens_per_rank / (max_ms / 1e3)
 
 
 def main():
@@ -294,7 +311,7 @@ def main():
     mg.lib()
     peaks, peak_kind = load_peaks()
 
-    inp = synth.layer_inputs(cfg, x_stream_offset=rank)
+    inp = rank_inputs(cfg, rank)
     sampler = ClockSampler(local)
     sampler.start()
     m = measure(cfg, inp, args.steps, args.warmup, dist_on, with_e2e=not args.no_e2e)
@@ -302,7 +319,7 @@ def main():
     ms = max_over_ranks(m["ms"], dist_on)
     e2e_ms = max_over_ranks(m.get("e2e_ms", float("nan")), dist_on)
     n = world
-    value = n * cfg.T / (ms / 1e3)
+    value = job_throughput(cfg.T, n, ms)
 
     su = m["stage_ms"]
     hbm = peaks["hbm_gbs"]
@@ -325,7 +342,7 @@ def main():
                                "unit": "GB/s", "frac": lb / (ms / 1e3) / 1e9 / hbm,
                                "algorithmic_bytes": lb},
             "stage_ms": su,
-            "e2e": {"value": n * cfg.T / (e2e_ms / 1e3), "unit": "tokens/s",
+            "e2e": {"value": job_throughput(cfg.T, n, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": m.get("io_bytes"), "d2h_bytes_per_step": m.get("io_bytes"),
                     "api": "moge_layer_forward_host (pinned host x in, host y out, synchronised per step)"},
             "gpu_launches": 5 * args.steps,
