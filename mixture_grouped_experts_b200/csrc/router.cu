@@ -19,11 +19,13 @@ constexpr int kRouterWarps = 8;
 constexpr int kRouterThreads = kRouterWarps * 32;
 
 // ---------------------------------------------------------------------------
-// Shared epilogue: logits [kRouterTile][N] fp32 in smem (bias not yet added)
-// -> scores, picks, per-tile histogram, in-tile ranks.
-struct RouterSmem {
-    float logits[kRouterTile][kMaxExperts];
-    int16_t ids[kRouterTile][kMaxExperts];  // picks, [t][k], k < K
+// Shared epilogue. The CTA's tile of tb tokens has its logits [tb][N] (fp32,
+// bias not yet added) in shared memory; this computes the scores, the picks,
+// and for every 16-token sub-tile the expert histogram and the in-tile ranks.
+struct RouterView {
+    float *logits;  // [tb][N]
+    int16_t *ids;   // [tb][K] picks
+    int tb;
 };
 
 // Order of candidates inside a group: higher score first, equal scores ->
@@ -32,31 +34,84 @@ __device__ __forceinline__ bool ranks_before(float pa, int a, float pb, int b) {
     return pa > pb || (pa == pb && a < b);
 }
 
-__device__ void router_epilogue(RouterSmem &sm, const moge_config &c, const float *bias, int t0,
-                                int32_t *topk_idx, float *topk_w, int32_t *hist, int32_t *rank) {
+__device__ void router_epilogue(const RouterView &sm, const moge_config &c, const float *bias,
+                                int t0, int32_t *topk_idx, float *topk_w, int32_t *hist,
+                                int32_t *rank) {
     const int N = c.N, M = c.M, Kp = c.Kp, K = M * Kp, G = N / M;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nwarps = blockDim.x >> 5;
-    const int ntok = min(kRouterTile, c.T - t0);
-    // one warp per token: global softmax over all N experts, fp32
+    const int ntok = min(sm.tb, c.T - t0);
+    // register path: every lane holds N/32 scores; a group of G (a power of
+    // two <= 32) lies inside one 32-lane segment, so its top-Kp is found with
+    // xor-shuffles inside G-lane segments
+    const bool shuffle = (N % 32 == 0) && G <= 32 && (G & (G - 1)) == 0;
     for (int tt = warp; tt < ntok; tt += nwarps) {
+        float *lg = sm.logits + (size_t)tt * N;
+        if (shuffle) {
+            const int J = N / 32;
+            float v[kMaxExperts / 32];
+            float m = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < kMaxExperts / 32; ++j) {
+                if (j < J) {
+                    const int e = lane + 32 * j;
+                    v[j] = lg[e] + (bias ? bias[e] : 0.0f);
+                    m = fmaxf(m, v[j]);
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            float z = 0.0f;
+#pragma unroll
+            for (int j = 0; j < kMaxExperts / 32; ++j)
+                if (j < J) {
+                    v[j] = expf(v[j] - m);
+                    z += v[j];
+                }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+#pragma unroll
+            for (int j = 0; j < kMaxExperts / 32; ++j) {
+                if (j >= J) continue;
+                float pv = v[j] / z;  // this lane's candidate; -inf once picked
+                for (int k = 0; k < Kp; ++k) {
+                    float bp = pv;
+                    int bi = lane + 32 * j;
+                    for (int o = G >> 1; o > 0; o >>= 1) {
+                        const float op = __shfl_xor_sync(0xffffffffu, bp, o);
+                        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                        if (ranks_before(op, oi, bp, bi)) { bp = op; bi = oi; }
+                    }
+                    if (bi == lane + 32 * j) pv = -INFINITY;
+                    if ((lane & (G - 1)) == 0) {
+                        const int g = (lane + 32 * j) / G;
+                        const size_t o = (size_t)(t0 + tt) * K + g * Kp + k;
+                        topk_idx[o] = bi;
+                        topk_w[o] = bp;
+                        sm.ids[(size_t)tt * K + g * Kp + k] = (int16_t)bi;
+                    }
+                }
+            }
+            continue;
+        }
+        // shared-memory path (any group size)
         float m = -INFINITY;
         for (int e = lane; e < N; e += 32) {
-            float l = sm.logits[tt][e] + (bias ? bias[e] : 0.0f);
-            sm.logits[tt][e] = l;
+            float l = lg[e] + (bias ? bias[e] : 0.0f);
+            lg[e] = l;
             m = fmaxf(m, l);
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        float s = 0.0f;
+        float z = 0.0f;
         for (int e = lane; e < N; e += 32) {
-            float v = expf(sm.logits[tt][e] - m);
-            sm.logits[tt][e] = v;
-            s += v;
+            float v = expf(lg[e] - m);
+            lg[e] = v;
+            z += v;
         }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        for (int e = lane; e < N; e += 32) sm.logits[tt][e] = sm.logits[tt][e] / s;
+        for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+        for (int e = lane; e < N; e += 32) lg[e] = lg[e] / z;
         __syncwarp();
         // per-group top-Kp: the j-th pick is the first candidate (in the order
         // above) that ranks after the (j-1)-th pick
@@ -67,11 +122,11 @@ __device__ void router_epilogue(RouterSmem &sm, const moge_config &c, const floa
                 int best = -1;
                 float pb = 0.0f;
                 for (int e = g * G; e < (g + 1) * G; ++e) {
-                    float pe = sm.logits[tt][e];
+                    const float pe = lg[e];
                     if (prev >= 0 && !ranks_before(pprev, prev, pe, e)) continue;
                     if (best < 0 || ranks_before(pe, e, pb, best)) { best = e; pb = pe; }
                 }
-                sm.ids[tt][g * Kp + j] = (int16_t)best;
+                sm.ids[(size_t)tt * K + g * Kp + j] = (int16_t)best;
                 const size_t o = (size_t)(t0 + tt) * K + g * Kp + j;
                 topk_idx[o] = best;
                 topk_w[o] = pb;
@@ -81,35 +136,37 @@ __device__ void router_epilogue(RouterSmem &sm, const moge_config &c, const floa
         }
     }
     __syncthreads();
-    // histogram of this tile, and the rank of each (t, k) among the tile's
-    // earlier tokens that picked the same expert (ascending token order)
-    const int tile = t0 / kRouterTile;
-    for (int e = threadIdx.x; e < N; e += blockDim.x) {
-        const int g = e / G;
+    // per 16-token sub-tile: histogram, and the rank of each (t, k) among the
+    // sub-tile's earlier tokens that picked the same expert (ascending tokens)
+    const int nsub = (ntok + kRouterTile - 1) / kRouterTile;
+    for (int i = threadIdx.x; i < nsub * N; i += blockDim.x) {
+        const int sub = i / N, e = i % N, g = e / G;
+        const int ta = sub * kRouterTile, tz = min(ntok, ta + kRouterTile);
         int cnt = 0;
-        for (int tt = 0; tt < ntok; ++tt)
-            for (int j = 0; j < Kp; ++j) cnt += sm.ids[tt][g * Kp + j] == e;
-        hist[(size_t)tile * N + e] = cnt;
+        for (int tt = ta; tt < tz; ++tt)
+            for (int j = 0; j < Kp; ++j) cnt += sm.ids[(size_t)tt * K + g * Kp + j] == e;
+        hist[(size_t)(t0 / kRouterTile + sub) * N + e] = cnt;
     }
-    for (int s = threadIdx.x; s < ntok * K; s += blockDim.x) {
-        const int tt = s / K, k = s % K, g = k / Kp;
-        const int e = sm.ids[tt][k];
+    for (int i = threadIdx.x; i < ntok * K; i += blockDim.x) {
+        const int tt = i / K, k = i % K, g = k / Kp;
+        const int e = sm.ids[i];
         int r = 0;
-        for (int t2 = 0; t2 < tt; ++t2)
-            for (int j = 0; j < Kp; ++j) r += sm.ids[t2][g * Kp + j] == e;
+        for (int t2 = (tt / kRouterTile) * kRouterTile; t2 < tt; ++t2)
+            for (int j = 0; j < Kp; ++j) r += sm.ids[(size_t)t2 * K + g * Kp + j] == e;
         rank[(size_t)(t0 + tt) * K + k] = r;
     }
 }
 
 // ---------------------------------------------------------------------------
 // bf16 router GEMM with mma.sync m16n8k16 (the N <= 256 output columns are far
-// too narrow for a tcgen05 tile to pay). One CTA owns 16 tokens and a slice of
-// the hidden dimension; a cluster of `ks` CTAs splits the hidden dimension of
-// one tile and the leader adds the partial logits in rank order
-// (deterministic). The CTA copies its x rows and router rows block by block
-// into shared memory with cp.async (every load of a block in flight at once,
-// two blocks double-buffered); warp w owns the n-tiles w, w+8, ... (8 experts
-// each), so no reduction across warps is needed.
+// too narrow for a tcgen05 tile to pay). One CTA owns a tile of TB = 16*TBM
+// tokens and a slice of the hidden dimension; a cluster of `ks` CTAs splits
+// the hidden dimension of one tile and the leader adds the partial logits in
+// rank order (deterministic). The CTA copies its x rows and router rows block
+// by block into shared memory with cp.async, NST blocks in flight; warp w owns
+// the n-tiles w, w+8, ... (8 experts each), so no reduction across warps is
+// needed. Long batches use 64-token tiles, which read the router matrix a
+// quarter as often.
 //
 // k-slot mapping: for each 32-wide chunk of the hidden dimension, the thread
 // with quad index q reads hidden elements [8q, 8q+8) of its A rows and of its
@@ -134,35 +191,43 @@ __device__ __forceinline__ void cp_async_16(void *dst, const void *src, uint32_t
                  : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int NPEND>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(NPEND) : "memory");
+__device__ __forceinline__ void cp_async_wait_pending(int n) {
+    // wait until at most n copy groups are outstanding (n < 4)
+    if (n <= 0) asm volatile("cp.async.wait_group 0;" ::: "memory");
+    else if (n == 1) asm volatile("cp.async.wait_group 1;" ::: "memory");
+    else if (n == 2) asm volatile("cp.async.wait_group 2;" ::: "memory");
+    else asm volatile("cp.async.wait_group 3;" ::: "memory");
 }
 
-// hidden elements per staged block for N experts (multiple of 32, >= 32):
-// (16 + N) rows of (2*LB + 64) bytes fit one stage
-__host__ __device__ inline int router_block_len(int N) {
-    int lb = ((kRouterStageBytes / (kRouterTile + N) - 64) / 2) & ~31;
+// hidden elements per staged block for a tile of tb tokens and N experts
+// (multiple of 32, >= 32): (tb + N) rows of (2*LB + 64) bytes fit one stage
+__host__ __device__ inline int router_block_len(int N, int tb) {
+    int lb = ((kRouterStageBytes / (tb + N) - 64) / 2) & ~31;
     if (lb >= 64) lb &= ~63;
     return lb < 32 ? 32 : lb;
 }
 
-__global__ void __launch_bounds__(kRouterThreads, 2) router_bf16_kernel(
+template <int TBM, int NST>
+__global__ void __launch_bounds__(kRouterThreads, (NST <= 2 ? 2 : 1)) router_bf16_kernel(
     moge_config c, const uint16_t *__restrict__ x, const uint16_t *__restrict__ wr,
     const float *__restrict__ bias, int32_t *topk_idx, float *topk_w, int32_t *hist, int32_t *rank,
     int ks) {
+    constexpr int TB = kRouterTile * TBM;
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    unsigned char *stage = smem_raw;  // [2][kRouterStageBytes]
-    RouterSmem &sm = *reinterpret_cast<RouterSmem *>(smem_raw + 2 * kRouterStageBytes);
+    unsigned char *stage = smem_raw;  // [NST][kRouterStageBytes]
+    RouterView sm;
+    sm.logits = reinterpret_cast<float *>(smem_raw + NST * kRouterStageBytes);
+    sm.ids = reinterpret_cast<int16_t *>(sm.logits + TB * c.N);
+    sm.tb = TB;
     grid_dependency_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, q = lane & 3;
     const int crank = blockIdx.x % ks;
-    const int t0 = (blockIdx.x / ks) * kRouterTile;
+    const int t0 = (blockIdx.x / ks) * TB;
     const int d = c.d, N = c.N;
-    const int LB = router_block_len(N);
-    const int pitch = 2 * LB + 64;  // bytes per staged row
-    const int rows = kRouterTile + N;
+    const int LB = router_block_len(N, TB);
+    const int pitch = 2 * LB + 64;  // bytes per staged row (64 B pad: conflict-free 16-byte loads)
+    const int rows = TB + N;
     // this CTA's slice of the hidden dimension, in whole 32-element chunks
     const int nchunk = (d + 31) / 32;
     const int kb = 32 * (int)((long long)nchunk * crank / ks);
@@ -170,70 +235,88 @@ __global__ void __launch_bounds__(kRouterThreads, 2) router_bf16_kernel(
     const int nblk = (ke - kb + LB - 1) / LB;
     const int vpr = LB / 8;  // 16-byte vectors per staged row
 
+    // warp w copies rows w, w+8, ...; lane l copies 16-byte vectors l, l+32, ... of a row
     auto load_block = [&](int b, unsigned char *dst) {
         const int k0 = kb + b * LB;
-        for (int i = threadIdx.x; i < rows * vpr; i += blockDim.x) {
-            const int r = i / vpr, v = i % vpr;
-            const int k = k0 + 8 * v;
-            const uint16_t *src;
-            bool ok = k < ke;
-            if (r < kRouterTile) {
-                ok = ok && (t0 + r) < c.T;
-                src = x + (size_t)(ok ? t0 + r : 0) * d + (ok ? k : 0);
+        for (int r = warp; r < rows; r += kRouterWarps) {
+            bool row_ok = true;
+            const uint16_t *src_row;
+            if (r < TB) {
+                row_ok = (t0 + r) < c.T;
+                src_row = x + (size_t)(row_ok ? t0 + r : 0) * d;
             } else {
-                src = wr + (size_t)(r - kRouterTile) * d + (ok ? k : 0);
+                src_row = wr + (size_t)(r - TB) * d;
             }
-            cp_async_16(dst + (size_t)r * pitch + 16 * v, src, ok ? 16u : 0u);
+            unsigned char *dst_row = dst + (size_t)r * pitch;
+            for (int v = lane; v < vpr; v += 32) {
+                const int k = k0 + 8 * v;
+                const bool ok = row_ok && k < ke;
+                cp_async_16(dst_row + 16 * v, src_row + (ok ? k : 0), ok ? 16u : 0u);
+            }
         }
         cp_async_commit();
     };
 
-    float acc[4][4];
+    float acc[TBM][4][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.0f;
+    for (int m = 0; m < TBM; ++m)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[m][i][0] = acc[m][i][1] = acc[m][i][2] = acc[m][i][3] = 0.0f;
     const int ntiles = N / 8;
-    // Tiles start at different blocks of their slice, so the CTAs that run at
-    // the same time do not all read the same router rows (an L2 hot spot).
+    // tiles start at different blocks of their slice, so concurrently running
+    // CTAs do not all read the same router rows at the same time
     const int rot = nblk > 0 ? (blockIdx.x / ks) % nblk : 0;
-    if (nblk > 0) load_block(rot, stage);
+    for (int i = 0; i < NST - 1 && i < nblk; ++i)
+        load_block((i + rot) % nblk, stage + i * kRouterStageBytes);
     for (int i = 0; i < nblk; ++i) {
         const int b = (i + rot) % nblk;
-        if (i + 1 < nblk) {
-            load_block((i + 1 + rot) % nblk, stage + ((i + 1) & 1) * kRouterStageBytes);
-            cp_async_wait<1>();
+        if (i + NST - 1 < nblk) {
+            load_block((i + NST - 1 + rot) % nblk, stage + ((i + NST - 1) % NST) * kRouterStageBytes);
+            cp_async_wait_pending(NST - 1);
         } else {
-            cp_async_wait<0>();
+            cp_async_wait_pending(nblk - 1 - i);
         }
         __syncthreads();
-        const unsigned char *st = stage + (i & 1) * kRouterStageBytes;
+        const unsigned char *st = stage + (i % NST) * kRouterStageBytes;
         const int len = min(LB, ke - (kb + b * LB));
         for (int ch = 0; ch < (len + 31) / 32; ++ch) {
             const int off = 64 * ch + 16 * q;  // bytes into the row
-            const uint4 av = *reinterpret_cast<const uint4 *>(st + (size_t)g * pitch + off);
-            const uint4 bv = *reinterpret_cast<const uint4 *>(st + (size_t)(g + 8) * pitch + off);
+            uint4 a_lo[TBM], a_hi[TBM];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int nt = warp + 8 * i;
+            for (int m = 0; m < TBM; ++m) {
+                a_lo[m] = *reinterpret_cast<const uint4 *>(st + (size_t)(16 * m + g) * pitch + off);
+                a_hi[m] = *reinterpret_cast<const uint4 *>(st + (size_t)(16 * m + g + 8) * pitch + off);
+            }
+#pragma unroll
+            for (int i2 = 0; i2 < 4; ++i2) {
+                const int nt = warp + 8 * i2;
                 if (nt < ntiles) {
                     const uint4 wv = *reinterpret_cast<const uint4 *>(
-                        st + (size_t)(kRouterTile + nt * 8 + g) * pitch + off);
-                    mma_bf16_16816(acc[i], av.x, bv.x, av.y, bv.y, wv.x, wv.y);
-                    mma_bf16_16816(acc[i], av.z, bv.z, av.w, bv.w, wv.z, wv.w);
+                        st + (size_t)(TB + nt * 8 + g) * pitch + off);
+#pragma unroll
+                    for (int m = 0; m < TBM; ++m) {
+                        mma_bf16_16816(acc[m][i2], a_lo[m].x, a_hi[m].x, a_lo[m].y, a_hi[m].y, wv.x, wv.y);
+                        mma_bf16_16816(acc[m][i2], a_lo[m].z, a_hi[m].z, a_lo[m].w, a_hi[m].w, wv.z, wv.w);
+                    }
                 }
             }
         }
-        __syncthreads();  // the stage is refilled two blocks later
+        __syncthreads();  // this stage is refilled NST blocks later
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int nt = warp + 8 * i;
-        if (nt < ntiles) {
-            sm.logits[g][nt * 8 + 2 * q] = acc[i][0];
-            sm.logits[g][nt * 8 + 2 * q + 1] = acc[i][1];
-            sm.logits[g + 8][nt * 8 + 2 * q] = acc[i][2];
-            sm.logits[g + 8][nt * 8 + 2 * q + 1] = acc[i][3];
+    for (int m = 0; m < TBM; ++m)
+#pragma unroll
+        for (int i2 = 0; i2 < 4; ++i2) {
+            const int nt = warp + 8 * i2;
+            if (nt < ntiles) {
+                float *r0 = sm.logits + (size_t)(16 * m + g) * N + nt * 8 + 2 * q;
+                float *r1 = sm.logits + (size_t)(16 * m + g + 8) * N + nt * 8 + 2 * q;
+                r0[0] = acc[m][i2][0];
+                r0[1] = acc[m][i2][1];
+                r1[0] = acc[m][i2][2];
+                r1[1] = acc[m][i2][3];
+            }
         }
-    }
     __syncthreads();
 
     if (ks > 1) {
@@ -243,16 +326,15 @@ __global__ void __launch_bounds__(kRouterThreads, 2) router_bf16_kernel(
         cluster.sync();  // all partial logits are final; every CTA is past its K-loop
         float *land = reinterpret_cast<float *>(stage);
         if (crank != 0) {
-            float *dst = cluster.map_shared_rank(land, 0) + (size_t)(crank - 1) * kRouterTile * N;
-            for (int o = threadIdx.x; o < kRouterTile * N; o += blockDim.x)
-                dst[o] = sm.logits[o / N][o % N];
+            float *dst = cluster.map_shared_rank(land, 0) + (size_t)(crank - 1) * TB * N;
+            for (int o = threadIdx.x; o < TB * N; o += blockDim.x) dst[o] = sm.logits[o];
         }
         cluster.sync();  // the pushes are visible to the leader
         if (crank != 0) return;
-        for (int o = threadIdx.x; o < kRouterTile * N; o += blockDim.x) {
-            float s = sm.logits[o / N][o % N];
-            for (int r = 1; r < ks; ++r) s += land[(size_t)(r - 1) * kRouterTile * N + o];
-            sm.logits[o / N][o % N] = s;
+        for (int o = threadIdx.x; o < TB * N; o += blockDim.x) {
+            float sum = sm.logits[o];
+            for (int r = 1; r < ks; ++r) sum += land[(size_t)(r - 1) * TB * N + o];
+            sm.logits[o] = sum;
         }
         __syncthreads();
     }
@@ -265,9 +347,12 @@ __global__ void __launch_bounds__(kRouterThreads) router_f32_kernel(
     const float *__restrict__ bias, int32_t *topk_idx, float *topk_w, int32_t *hist,
     int32_t *rank) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    RouterSmem &sm = *reinterpret_cast<RouterSmem *>(smem_raw);
-    const int t0 = blockIdx.x * kRouterTile;
+    RouterView sm;
+    sm.logits = reinterpret_cast<float *>(smem_raw);
+    sm.ids = reinterpret_cast<int16_t *>(sm.logits + kRouterTile * c.N);
+    sm.tb = kRouterTile;
     grid_dependency_wait();
+    const int t0 = blockIdx.x * kRouterTile;
     const int ntok = min(kRouterTile, c.T - t0);
     for (int o = threadIdx.x; o < kRouterTile * c.N; o += blockDim.x) {
         const int tt = o / c.N, e = o % c.N;
@@ -277,36 +362,31 @@ __global__ void __launch_bounds__(kRouterThreads) router_f32_kernel(
             const float *wrow = wr + (size_t)e * c.d;
             for (int k = 0; k < c.d; ++k) s = fmaf(xr[k], wrow[k], s);
         }
-        sm.logits[tt][e] = s;
+        sm.logits[o] = s;
     }
     __syncthreads();
     router_epilogue(sm, c, bias, t0, topk_idx, topk_w, hist, rank);
 }
 
-cudaError_t launch_router(const moge_config &c, const void *x, const void *w_router,
-                          const float *bias, int32_t *topk_idx, float *topk_w, int32_t *hist,
-                          int32_t *rank, int num_sms, cudaStream_t st) {
-    const int tiles = (c.T + kRouterTile - 1) / kRouterTile;
-    if (c.dtype == MOGE_F32) {
-        const size_t smem = sizeof(RouterSmem);
-        cudaError_t e = cudaFuncSetAttribute(router_f32_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        return launch_pdl(router_f32_kernel, dim3(tiles), dim3(kRouterThreads), smem, st, c,
-                          (const float *)x, (const float *)w_router, bias, topk_idx, topk_w, hist,
-                          rank);
-    }
-    // Split the hidden dimension over a cluster of up to 8 CTAs while the
-    // grid stays within two CTAs per SM, each CTA keeps >= 2 blocks of work,
-    // and the leader's landing buffer (two stages) holds (ks - 1) partial tiles.
-    const int lb = router_block_len(c.N);
+template <int TBM, int NST>
+static cudaError_t launch_router_bf16(const moge_config &c, const void *x, const void *w_router,
+                                      const float *bias, int32_t *topk_idx, float *topk_w,
+                                      int32_t *hist, int32_t *rank, int num_sms, cudaStream_t st) {
+    constexpr int TB = kRouterTile * TBM;
+    const int tiles = (c.T + TB - 1) / TB;
+    const int per_sm = NST <= 2 ? 2 : 1;
+    // Split the hidden dimension over a cluster of up to 8 CTAs while the grid
+    // stays within one wave, each CTA keeps >= 2 blocks of work, and the
+    // leader's landing buffer (its stages) holds the (ks - 1) partial tiles.
+    const int lb = router_block_len(c.N, TB);
     int ks = 1;
-    while (ks < 8 && tiles * ks * 2 <= 2 * num_sms && c.d >= ks * 2 * 2 * lb &&
-           (2 * ks - 1) * kRouterTile * c.N * 4 <= 2 * kRouterStageBytes)
+    while (ks < 8 && tiles * ks * 2 <= per_sm * num_sms && c.d >= ks * 2 * 2 * lb &&
+           (size_t)(2 * ks - 1) * TB * c.N * 4 <= (size_t)NST * kRouterStageBytes)
         ks *= 2;
-    const size_t smem = 2 * kRouterStageBytes + sizeof(RouterSmem);
-    cudaError_t e = cudaFuncSetAttribute(router_bf16_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const size_t smem = (size_t)NST * kRouterStageBytes + (size_t)TB * c.N * 4 +
+                        (size_t)TB * c.M * c.Kp * 2;
+    auto kern = router_bf16_kernel<TBM, NST>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(tiles * ks);
@@ -322,8 +402,29 @@ cudaError_t launch_router(const moge_config &c, const void *x, const void *w_rou
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, router_bf16_kernel, c, (const uint16_t *)x,
-                              (const uint16_t *)w_router, bias, topk_idx, topk_w, hist, rank, ks);
+    return cudaLaunchKernelEx(&cfg, kern, c, (const uint16_t *)x, (const uint16_t *)w_router, bias,
+                              topk_idx, topk_w, hist, rank, ks);
+}
+
+cudaError_t launch_router(const moge_config &c, const void *x, const void *w_router,
+                          const float *bias, int32_t *topk_idx, float *topk_w, int32_t *hist,
+                          int32_t *rank, int num_sms, cudaStream_t st) {
+    if (c.dtype == MOGE_F32) {
+        const int tiles = (c.T + kRouterTile - 1) / kRouterTile;
+        const size_t smem = (size_t)kRouterTile * c.N * 4 + (size_t)kRouterTile * c.M * c.Kp * 2;
+        cudaError_t e = cudaFuncSetAttribute(router_f32_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        return launch_pdl(router_f32_kernel, dim3(tiles), dim3(kRouterThreads), smem, st, c,
+                          (const float *)x, (const float *)w_router, bias, topk_idx, topk_w, hist,
+                          rank);
+    }
+    // long batches with few experts: 64-token tiles, four blocks in flight
+    // (one CTA per SM); otherwise 16-token tiles, two blocks in flight (two
+    // CTAs per SM, up to 8-CTA clusters over the hidden dimension)
+    if (c.N <= 64 && c.T >= 1024)
+        return launch_router_bf16<4, 4>(c, x, w_router, bias, topk_idx, topk_w, hist, rank, num_sms, st);
+    return launch_router_bf16<1, 2>(c, x, w_router, bias, topk_idx, topk_w, hist, rank, num_sms, st);
 }
 
 // ---------------------------------------------------------------------------
