@@ -1,19 +1,23 @@
 """12-layer stack of MoGE blocks with pre-RMSNorm and residual:
 x_{l+1} = x_l + MoGE_l(RMSNorm(x_l)), residual stream stored in bf16.
 
-Two checks per layer and one end to end:
-  * teacher forcing: the GPU's own layer input bytes (RMSNorm output) are fed
-    to the oracle; the GPU layer output (no residual) on sampled tokens must
-    match it, routing bit-exact above the margin;
-  * end to end: bf16 drift may flip a pick whose margin is small, after which
-    the two stacks legitimately differ. So the oracle's scores on the GPU's own
-    layer inputs give every token its smallest in-group margin over the 12
-    layers; the tokens with the widest margins (all > 5e-4) are carried
-    through the oracle's fp64 stack, must keep the GPU's picks at every layer,
-    and must match at the end within sqrt(L) * 1e-2: every layer is held to
-    1e-2 of its own output (checked above) and the L layers' independent bf16
-    rounding errors, plus the bf16 rounding of the residual after each layer,
-    add up roughly in quadrature.
+Three checks per layer and one end to end:
+  * routing: on the GPU's own layer inputs (RMSNorm output) the GPU's picks
+    equal the oracle's for every token whose margin is above 1e-4;
+  * teacher forcing: those input bytes are fed to the oracle; the GPU layer
+    output (no residual) on sampled tokens must match it within 1e-2;
+  * end to end: the 8 tokens with the widest routing margins on the GPU's
+    trajectory are carried through the oracle's fp64 stack. The two stacks
+    drift apart by bf16 rounding, so their router scores p (oracle) and p'
+    (oracle arithmetic on the GPU's inputs) differ a little; an argmax in a
+    group can only flip if the oracle's margin is at most 2 max|p - p'| (plus
+    the 1e-4 rule for the GPU side). Every disagreement must be explained by
+    that measured drift, and the token is followed no further (from there the
+    stacks legitimately differ). At least two tokens must keep their picks
+    through all 12 layers, and those must match at the end within
+    sqrt(L) * 1e-2: every layer is held to 1e-2 of its own output (checked
+    above) and the L layers' independent bf16 rounding errors, plus the bf16
+    rounding of the residual after each layer, add up roughly in quadrature.
 """
 import gc
 
@@ -42,6 +46,7 @@ def test_stack12_teacher_forced_and_end_to_end():
     x_dev = mg.to_device(x0, "bf16")
     min_margin = np.full(cfg.T, np.inf)
     idx_all = []
+    p_all = []
     checked = 0
     for l in range(cfg.layers):                   # pass 1: the GPU stack
         inp = synth.layer_inputs(cfg, layer=l, with_x=False)
@@ -55,8 +60,11 @@ def test_stack12_teacher_forced_and_end_to_end():
         idx_all.append(idx_g)
         u_h = to_host_f64(u)
         p = oracle.router_probs(u_h, inp["w_router"], None, "bf16")
-        _, _, mgn = oracle.select_grouped(p, cfg.M, cfg.Kp)
+        idx_p, _, mgn = oracle.select_grouped(p, cfg.M, cfg.Kp)
+        clear = mgn > MARGIN
+        assert np.array_equal(idx_p[clear], idx_g[clear]), l
         min_margin = np.minimum(min_margin, mgn)
+        p_all.append(p)
         # teacher forcing on two tokens per layer
         tf = np.array([(37 * l + 11) % cfg.T, (91 * l + 5) % cfg.T])
         y_ref, idx_ref, _, mg_ref = oracle.layer(u_h, inp, cfg.M, cfg.Kp, "bf16", tokens=tf)
@@ -70,14 +78,22 @@ def test_stack12_teacher_forced_and_end_to_end():
         del w, inp, u, y_only
         _free()
     assert checked >= cfg.layers
-    cand = np.argsort(-min_margin)[:4]
-    assert np.all(min_margin[cand] > 5e-4), min_margin[cand]
+    cand = np.argsort(-min_margin)[:8]
     xo = oracle.to_double(x0, "bf16")[cand]
+    kept = np.ones(len(cand), bool)       # same picks as the GPU at every layer so far
     for l in range(cfg.layers):                   # pass 2: the oracle's fp64 stack
         inp = synth.layer_inputs(cfg, layer=l, with_x=False)
-        yo, idx_o, _, _ = oracle.layer(oracle.rmsnorm(xo, 1e-6), inp, cfg.M, cfg.Kp, "bf16")
-        assert np.array_equal(idx_o, idx_all[l][cand]), l
+        uo = oracle.rmsnorm(xo, 1e-6)
+        yo, idx_o, _, mg_o = oracle.layer(uo, inp, cfg.M, cfg.Kp, "bf16")
+        drift = np.abs(oracle.router_probs(uo, inp["w_router"], None, "bf16") - p_all[l][cand])
+        idx_g = idx_all[l][cand]
+        for j in range(len(cand)):
+            if kept[j] and not np.array_equal(idx_o[j], idx_g[j]):
+                assert mg_o[j] <= 2 * drift[j].max() + MARGIN, (l, int(cand[j]), float(mg_o[j]),
+                                                                 float(drift[j].max()))
+                kept[j] = False           # a flip explained by drift: the stacks part here
         xo = xo + yo
         del inp
-    err = normwise_err(to_host_f64(x_dev)[cand], xo)
+    assert kept.sum() >= 2, (min_margin[cand], kept)
+    err = normwise_err(to_host_f64(x_dev)[cand[kept]], xo[kept])
     assert err <= np.sqrt(cfg.layers) * TOL["bf16"], err
