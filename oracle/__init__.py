@@ -54,6 +54,16 @@ def _l():
         lib.oracle_layer.argtypes = [vp, i32, i32, i32, i32, i32, i32, i32, i32,
                                      vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp]
         lib.oracle_rmsnorm.argtypes = [vp, i32, i32, ctypes.c_double, vp]
+        lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_decode.restype = ctypes.c_double
+        lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+        i64 = ctypes.c_int64
+        lib.oracle_quantize_rows_fp8.argtypes = [vp, i64, i64, vp, vp]
+        lib.oracle_expert_ffn_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, vp]
+        lib.oracle_layer_fp8.argtypes = [vp, i32, i32, i32, i32, i32, i32, i32, i32, vp, vp,
+                                         vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                         vp, i32, vp, vp, vp, vp]
         _lib = lib
     return _lib
 
@@ -197,3 +207,89 @@ def rmsnorm(x: np.ndarray, eps: float = 1e-6) -> np.ndarray:
     u = np.empty_like(x)
     _chk(_l().oracle_rmsnorm(_p(x), T, d, eps, _p(u)), "rmsnorm")
     return u
+
+
+# ----------------------------------------------------------------------------- fp8 weights
+def e4m3_decode(code: int) -> float:
+    """Value of one OCP FP8 E4M3 code (NaN for S.1111.111)."""
+    return float(_l().oracle_e4m3_decode(int(code) & 0xFF))
+
+
+def e4m3_encode(v: float) -> int:
+    """Nearest E4M3 code to the fp32 value v (ties to even, saturating at 448)."""
+    return int(_l().oracle_e4m3_encode(float(np.float32(v))))
+
+
+def e4m3_values() -> np.ndarray:
+    """Values of all 256 codes (float64; NaN at 0x7F and 0xFF)."""
+    return np.array([e4m3_decode(c) for c in range(256)], np.float64)
+
+
+def quantize_rows_fp8(w: np.ndarray):
+    """Per-row fp8 quantisation of bf16 rows (uint16 bit patterns, [..., cols]).
+
+    Returns (q uint8 of the same shape, scale float32 of shape w.shape[:-1]):
+    scale = amax / 448 in fp32 (1 for an all-zero row), q = E4M3(fp32(w / scale)).
+    """
+    w = np.ascontiguousarray(w)
+    if w.dtype != np.uint16:
+        raise TypeError("quantize_rows_fp8 takes bf16 bit patterns (uint16)")
+    cols = w.shape[-1]
+    rows = w.size // cols
+    q = np.empty(w.shape, np.uint8)
+    sc = np.empty(w.shape[:-1], np.float32)
+    _chk(_l().oracle_quantize_rows_fp8(_p(w), rows, cols, _p(q), _p(sc)), "quantize_rows_fp8")
+    return q, sc
+
+
+def dequantize_fp8(q: np.ndarray, scale: np.ndarray) -> np.ndarray:
+    """decode(q) * scale per row, float64 (exact)."""
+    return e4m3_values()[q] * np.asarray(scale, np.float64)[..., None]
+
+
+def quantize_experts_fp8(inp: dict) -> dict:
+    """Quantise every expert matrix of a synth.layer_inputs weight dict (bf16)."""
+    out = {}
+    for k in ("w_gate", "w_up", "w_down", "s_gate", "s_up", "s_down"):
+        out[k], out[k + "_scale"] = quantize_rows_fp8(inp[k])
+    return out
+
+
+def expert_ffn_fp8(x_row: np.ndarray, qg, sg, qu, su, qd, sd) -> np.ndarray:
+    """One SwiGLU expert on one token with fp8 weights (qg, qu [I][d]; qd [d][I])."""
+    x = np.ascontiguousarray(x_row, np.float64)
+    qg, qu, qd = (np.ascontiguousarray(a, np.uint8) for a in (qg, qu, qd))
+    sg, su, sd = (np.ascontiguousarray(a, np.float32) for a in (sg, su, sd))
+    I, d = qg.shape
+    y = np.empty(d, np.float64)
+    _chk(_l().oracle_expert_ffn_fp8(_p(x), _p(qg), _p(sg), _p(qu), _p(su), _p(qd), _p(sd),
+                                    d, I, _p(y)), "expert_ffn_fp8")
+    return y
+
+
+def layer_fp8(x: np.ndarray, inp: dict, q: dict, M: int, Kp: int, dtype: str,
+              tokens: Optional[Sequence[int]] = None):
+    """MoGE layer output with fp8 expert weights q (quantize_experts_fp8 form);
+    router weights and logit bias from inp. Same returns as layer()."""
+    x = np.ascontiguousarray(x, np.float64)
+    T, d = x.shape
+    wr = _w(inp["w_router"], dtype)
+    N, I = q["w_gate"].shape[0], q["w_gate"].shape[1]
+    S = q["s_gate"].shape[0]
+    a = {k: np.ascontiguousarray(v) for k, v in q.items()}
+    b = inp.get("logit_bias")
+    b = None if b is None else np.ascontiguousarray(b, np.float32)
+    toks = np.arange(T, dtype=np.int32) if tokens is None else np.asarray(tokens, np.int32)
+    n = len(toks)
+    K = M * Kp
+    y = np.empty((n, d), np.float64)
+    idx = np.empty((n, K), np.int32)
+    w = np.empty((n, K), np.float64)
+    mg = np.empty(n, np.float64)
+    _chk(_l().oracle_layer_fp8(_p(x), T, d, N, M, Kp, S, I, _DT[dtype], _p(wr), _p(b),
+                               _p(a["w_gate"]), _p(a["w_gate_scale"]), _p(a["w_up"]),
+                               _p(a["w_up_scale"]), _p(a["w_down"]), _p(a["w_down_scale"]),
+                               _p(a["s_gate"]), _p(a["s_gate_scale"]), _p(a["s_up"]),
+                               _p(a["s_up_scale"]), _p(a["s_down"]), _p(a["s_down_scale"]),
+                               _p(toks), n, _p(y), _p(idx), _p(w), _p(mg)), "layer_fp8")
+    return y, idx, w, mg

@@ -326,3 +326,149 @@ int oracle_rmsnorm(const double *x, int T, int d, double eps, double *u) {
     }
     return 0;
 }
+
+/* ---------------------------------------------------------------------------
+ * 8-bit expert weights. The pages report 8-bit weight quantisation of the
+ * model (hwcomputing.csdn.net news piece, deployment section: W8A8 with a
+ * small accuracy loss) and an expert-aware quantisation method (techwalker.com
+ * article, section 3), but fix no number format. Reading taken: weights-only
+ * 8-bit, OCP FP8 E4M3 codes (1 sign bit, 4 exponent bits with bias 7, 3
+ * mantissa bits; no infinities; S.1111.111 is NaN; largest finite 448;
+ * subnormals m * 2^-9), one fp32 scale per weight row (output channel):
+ *   scale_r = amax_r / 448 (fp32 division; 1 for an all-zero row),
+ *   q[r][c] = E4M3 round-to-nearest-even, saturating, of fp32(w[r][c] / scale_r),
+ *   dequantised weight = decode(q) * scale_r.
+ * Activations stay at the layer's precision (bf16).
+ */
+
+/* value of an E4M3 code (NaN codes decode to NaN) */
+double oracle_e4m3_decode(uint8_t code) {
+    int sign = code >> 7, e = (code >> 3) & 15, m = code & 7;
+    if (e == 15 && m == 7) return NAN;
+    double mag = e == 0 ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+    return sign ? -mag : mag;
+}
+
+/* nearest E4M3 code to v, ties to even mantissa, finite results saturating at
+ * +-448 (so every finite input maps to a finite code) */
+uint8_t oracle_e4m3_encode(float v) {
+    double a = fabs((double)v);
+    uint8_t sign = signbit(v) ? 0x80 : 0;
+    if (isnan(v)) return (uint8_t)(sign | 0x7F);
+    if (a >= 448.0) return (uint8_t)(sign | 0x7E);
+    if (a < ldexp(1.0, -6)) {               /* subnormal range: steps of 2^-9 */
+        double n = rint(ldexp(a, 9));       /* current rounding mode: to nearest even */
+        return (uint8_t)(sign | (uint8_t)n); /* n == 8 is the smallest normal, code 0x08 */
+    }
+    int ex;
+    double fr = frexp(a, &ex);              /* a = fr * 2^ex, fr in [0.5, 1) */
+    int e = ex - 1;                         /* a = (2 fr) * 2^e, 2 fr in [1, 2) */
+    double mm = rint((2.0 * fr - 1.0) * 8.0);
+    if (mm >= 8.0) { mm = 0.0; e += 1; }
+    int be = e + 7;
+    if (be > 15 || (be == 15 && mm >= 7.0)) return (uint8_t)(sign | 0x7E);
+    return (uint8_t)(sign | (be << 3) | (int)mm);
+}
+
+/* per-row quantisation of bf16 rows (bit patterns) w [rows][cols] */
+int oracle_quantize_rows_fp8(const uint16_t *w, int64_t rows, int64_t cols, uint8_t *q,
+                             float *scale) {
+    for (int64_t r = 0; r < rows; ++r) {
+        const uint16_t *wr = w + r * cols;
+        float amax = 0.0f;
+        for (int64_t c = 0; c < cols; ++c) {
+            float a = (float)fabs(bf16_bits_to_double(wr[c]));
+            if (a > amax) amax = a;
+        }
+        volatile float s = amax > 0.0f ? amax / 448.0f : 1.0f;  /* one fp32 division */
+        scale[r] = s;
+        for (int64_t c = 0; c < cols; ++c) {
+            volatile float v = (float)bf16_bits_to_double(wr[c]) / s;
+            q[r * cols + c] = oracle_e4m3_encode(v);
+        }
+    }
+    return 0;
+}
+
+/* row of an fp8 matrix, dequantised: decode(q) * scale (exact in double) */
+static void load_row_fp8(const uint8_t *q, const float *scale, size_t row, int n, double *out) {
+    const uint8_t *p = q + row * (size_t)n;
+    double s = (double)scale[row];
+    for (int j = 0; j < n; ++j) out[j] = oracle_e4m3_decode(p[j]) * s;
+}
+
+/* One expert on one token with fp8 weights: the same SwiGLU expert as
+ * oracle_expert_ffn, on the dequantised matrices. qg, qu [I][d] with scales
+ * sg, su [I]; qd [d][I] with scales sd [d]. */
+int oracle_expert_ffn_fp8(const double *x, const uint8_t *qg, const float *sg, const uint8_t *qu,
+                          const float *su, const uint8_t *qd, const float *sd, int d, int I,
+                          double *y) {
+    double *w = (double *)malloc(sizeof(double) * (size_t)(d > I ? d : I));
+    double *h = (double *)malloc(sizeof(double) * (size_t)I);
+    if (!w || !h) { free(w); free(h); return 2; }
+    for (int i = 0; i < I; ++i) {
+        load_row_fp8(qg, sg, (size_t)i, d, w);
+        double g = dot(x, w, d);
+        load_row_fp8(qu, su, (size_t)i, d, w);
+        double u = dot(x, w, d);
+        h[i] = (g / (1.0 + exp(-g))) * u;
+    }
+    for (int o = 0; o < d; ++o) {
+        load_row_fp8(qd, sd, (size_t)o, I, w);
+        y[o] = dot(h, w, I);
+    }
+    free(w);
+    free(h);
+    return 0;
+}
+
+/* The layer [A][B][D] with fp8 expert weights (routed and shared), router
+ * weights and activations as in oracle_layer (dtype of x / w_router):
+ * routed expert e uses qg + e I d, sg + e I, ..., qd + e d I, sd + e d. */
+int oracle_layer_fp8(const double *x, int T, int d, int N, int M, int Kp, int S, int I, int dtype,
+                     const void *w_router, const float *bias,
+                     const uint8_t *qg, const float *sg, const uint8_t *qu, const float *su,
+                     const uint8_t *qd, const float *sd,
+                     const uint8_t *sqg, const float *ssg, const uint8_t *squ, const float *ssu,
+                     const uint8_t *sqd, const float *ssd,
+                     const int32_t *tokens, int n, double *y_out,
+                     int32_t *idx_out, double *w_out, double *margin_out) {
+    if (N % M != 0 || Kp < 1 || Kp > N / M) return 1;
+    int K = M * Kp;
+    size_t per = (size_t)I * d;
+    double *tmp = (double *)malloc(sizeof(double) * (size_t)d);
+    int32_t *idx = (int32_t *)malloc(sizeof(int32_t) * (size_t)K);
+    double *w = (double *)malloc(sizeof(double) * (size_t)K);
+    if (!tmp || !idx || !w) { free(tmp); free(idx); free(w); return 2; }
+    int rc = 0;
+    for (int q = 0; q < n && rc == 0; ++q) {
+        int t = tokens[q];
+        if (t < 0 || t >= T) { rc = 1; break; }
+        const double *xt = x + (size_t)t * d;
+        double *yt = y_out + (size_t)q * d;
+        double mg;
+        rc = oracle_route(xt, w_router, bias, dtype, 1, d, N, M, Kp, idx, w, &mg);
+        if (rc) break;
+        for (int o = 0; o < d; ++o) yt[o] = 0.0;
+        for (int k = 0; k < K; ++k) {
+            size_t e = (size_t)idx[k];
+            rc = oracle_expert_ffn_fp8(xt, qg + e * per, sg + e * I, qu + e * per, su + e * I,
+                                       qd + e * per, sd + e * d, d, I, tmp);
+            if (rc) break;
+            for (int o = 0; o < d; ++o) yt[o] += w[k] * tmp[o];
+        }
+        for (int s = 0; s < S && rc == 0; ++s) {
+            size_t e = (size_t)s;
+            rc = oracle_expert_ffn_fp8(xt, sqg + e * per, ssg + e * I, squ + e * per, ssu + e * I,
+                                       sqd + e * per, ssd + e * d, d, I, tmp);
+            for (int o = 0; o < d; ++o) yt[o] += tmp[o];
+        }
+        if (idx_out) memcpy(idx_out + (size_t)q * K, idx, sizeof(int32_t) * (size_t)K);
+        if (w_out) memcpy(w_out + (size_t)q * K, w, sizeof(double) * (size_t)K);
+        if (margin_out) margin_out[q] = mg;
+    }
+    free(tmp);
+    free(idx);
+    free(w);
+    return rc;
+}
