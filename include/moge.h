@@ -195,6 +195,44 @@ MOGE_API int moge_route_noalloc(const moge_config *cfg, const void *x, const voi
 MOGE_API int moge_stage_timing(int enable);
 MOGE_API int moge_stage_times(double *ms_total, int64_t *calls);
 
+/* ---------------------------------------------------------------- 8-bit expert weights
+ * The pages report 8-bit weight quantisation of the model (hwcomputing.csdn.net
+ * news piece, deployment section) and an expert-aware quantisation method
+ * (techwalker.com article, section 3) without a number format. This library
+ * reads it as weights-only FP8: OCP E4M3 codes with one fp32 scale per weight
+ * row (output channel); activations, h and y stay bf16. Calibration (the
+ * pages' smoothing and routing-alignment steps) is not part of it.
+ *
+ * Quantise rows of a bf16 matrix w [rows][cols] (device):
+ *   scale[r] = amax_r / 448 (fp32 division; 1 for an all-zero row)
+ *   q[r][c]  = E4M3 of fp32(w[r][c] / scale[r]), round to nearest even,
+ *              saturating at +-448
+ * q [rows][cols] bytes, scale [rows] fp32, both caller-owned device memory.
+ * cols % 8 == 0; w 16-byte and q 8-byte aligned. Asynchronous on `stream`.
+ * Expert tensors [E][R][C] are quantised as E*R rows. */
+MOGE_API int moge_quantize_fp8_rows(const void *w, int64_t rows, int64_t cols, void *q,
+                                    float *scale, void *stream);
+
+/* One side's (routed or shared) expert weights in FP8: codes in the layouts of
+ * the bf16 weights (gate, up [E][I][d]; down [E][d][I], one byte each) and
+ * their row scales (gate_scale, up_scale [E][I]; down_scale [E][d]). The
+ * dequantised weight is decode(code) * scale of its row. */
+typedef struct {
+    const void *gate, *up, *down;
+    const float *gate_scale, *up_scale, *down_scale;
+} moge_fp8_experts;
+
+/* moge_layer_forward with FP8 expert weights (routed and shared; the router
+ * stays bf16). cfg->dtype must be MOGE_BF16; d % 16 == 0 and I % 16 == 0
+ * (16-byte rows of codes). `shared` may be NULL when S == 0. Same workspace,
+ * routing, residual and aliasing rules as moge_layer_forward. The FFN streams
+ * the codes (half the bf16 bytes), widens them exactly to bf16 in shared
+ * memory and applies the row scales to the fp32 accumulators. */
+MOGE_API int moge_layer_forward_fp8(const moge_config *cfg, const void *x, const void *w_router,
+                                    const float *logit_bias, const moge_fp8_experts *routed,
+                                    const moge_fp8_experts *shared, const void *residual, void *y,
+                                    void *workspace, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

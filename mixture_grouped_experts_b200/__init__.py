@@ -29,7 +29,8 @@ _TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16}
 EXPORTS = ["moge_workspace_size", "moge_last_error", "moge_check_device_errors", "moge_route",
            "moge_permute", "moge_grouped_ffn", "moge_shared_ffn", "moge_combine",
            "moge_layer_forward", "moge_layer_forward_host", "moge_workspace_routing",
-           "moge_rmsnorm", "moge_stage_timing", "moge_stage_times", "moge_route_noalloc"]
+           "moge_rmsnorm", "moge_stage_timing", "moge_stage_times", "moge_route_noalloc",
+           "moge_quantize_fp8_rows", "moge_layer_forward_fp8"]
 STAGES = ("router", "scan", "permute", "ffn", "combine")
 
 
@@ -41,6 +42,11 @@ class MogeError(RuntimeError):
 
 class moge_config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in ("T", "d", "N", "M", "Kp", "S", "I", "dtype")]
+
+
+class moge_fp8_experts(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("gate", "up", "down", "gate_scale", "up_scale",
+                                               "down_scale")]
 
 
 @dataclass(frozen=True)
@@ -96,6 +102,9 @@ def lib() -> ctypes.CDLL:
         L.moge_stage_timing.argtypes = [i32]
         L.moge_route_noalloc.argtypes = [cp] + [vp] * 10
         L.moge_stage_times.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]
+        L.moge_quantize_fp8_rows.argtypes = [vp, ctypes.c_int64, ctypes.c_int64, vp, vp, vp]
+        fp = ctypes.POINTER(moge_fp8_experts)
+        L.moge_layer_forward_fp8.argtypes = [cp, vp, vp, vp, fp, fp, vp, vp, vp, vp]
         for n in EXPORTS:
             if n not in ("moge_workspace_size", "moge_last_error"):
                 getattr(L, n).restype = i32
@@ -285,3 +294,55 @@ def moge_stage_times():
     n = ctypes.c_int64()
     _chk(lib().moge_stage_times(ms, ctypes.byref(n)))
     return {k: ms[i] for i, k in enumerate(STAGES)}, n.value
+
+
+# ----------------------------------------------------------------------------- fp8 weights
+FP8_KEYS = ("w_gate", "w_up", "w_down", "s_gate", "s_up", "s_down")
+
+
+def moge_quantize_fp8_rows(w, stream=None):
+    """Per-row E4M3 quantisation of a bf16 device tensor [..., cols] ->
+    (codes uint8 of the same shape, fp32 scales of shape w.shape[:-1])."""
+    if w.dtype != torch.bfloat16:
+        raise TypeError("moge_quantize_fp8_rows takes a bf16 tensor")
+    cols = w.shape[-1]
+    rows = w.numel() // cols
+    q = torch.empty(w.shape, dtype=torch.uint8, device=w.device)
+    sc = torch.empty(w.shape[:-1], dtype=torch.float32, device=w.device)
+    _chk(lib().moge_quantize_fp8_rows(_p(w), rows, cols, _p(q), _p(sc), _stream(stream)))
+    return q, sc
+
+
+def experts_to_fp8(w: dict, stream=None) -> dict:
+    """FP8 codes and row scales of every expert matrix of a device weight dict
+    (keys w_gate ... s_down, and the same keys + "_scale"); router weights and
+    logit_bias are not touched."""
+    out = {}
+    for k in FP8_KEYS:
+        if w.get(k) is not None:
+            out[k], out[k + "_scale"] = moge_quantize_fp8_rows(w[k], stream)
+        else:
+            out[k] = out[k + "_scale"] = None
+    return out
+
+
+def _fp8_side(w8: dict, prefix: str):
+    if w8.get(prefix + "_gate") is None:
+        return None
+    return moge_fp8_experts(*[_p(w8[prefix + n]) for n in ("_gate", "_up", "_down", "_gate_scale",
+                                                            "_up_scale", "_down_scale")])
+
+
+def moge_layer_forward_fp8(s: LayerShape, x, w: dict, w8: dict, workspace, residual=None, y=None,
+                           stream=None):
+    """Layer with FP8 expert weights w8 (experts_to_fp8 form); w gives w_router
+    and logit_bias."""
+    if y is None:
+        y = torch.empty((s.T, s.d), dtype=x.dtype, device=x.device)
+    routed, shared = _fp8_side(w8, "w"), _fp8_side(w8, "s")
+    _chk(lib().moge_layer_forward_fp8(ctypes.byref(_cfg(s)), _p(x), _p(w["w_router"]),
+                                      _p(w.get("logit_bias")),
+                                      ctypes.byref(routed) if routed is not None else None,
+                                      ctypes.byref(shared) if shared is not None else None,
+                                      _p(residual), _p(y), _p(workspace), _stream(stream)))
+    return y

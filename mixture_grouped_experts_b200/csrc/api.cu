@@ -157,6 +157,59 @@ static cudaEvent_t *timer_slot() {
 
 using namespace moge;
 
+static int run_ffn(const moge_config &c, const Plan &plan, int n_entries, const FfnOperands &op,
+                   cudaStream_t st, cudaEvent_t mid = nullptr) {
+    if (c.dtype == MOGE_BF16)
+        MOGE_CU(launch_ffn_tc(c, plan, n_entries, op, num_sms(), st, mid),
+                "grouped FFN (tcgen05) launch");
+    else
+        MOGE_CU(launch_ffn_f32(c, plan, n_entries, op, st, mid), "grouped FFN (fp32) launch");
+    return MOGE_OK;
+}
+
+// The five launches of the layer (router, scan + plan, permute, grouped FFN,
+// combine) after the entry point validated its arguments. `op` carries the
+// expert weight pointers (and, for fp8, their row scales); the activation
+// pointers are filled in here.
+static int layer_run(const moge_config &c, const void *x, const void *w_router,
+                     const float *logit_bias, FfnOperands op, bool fp8, const void *residual,
+                     void *y, void *workspace, cudaStream_t st) {
+    Workspace ws = carve_workspace(c, workspace);
+    const int K = c.M * c.Kp;
+    cudaEvent_t *ev = timer_slot();
+    if (ev) MOGE_CU(cudaEventRecord(ev[0], st), "event");
+    MOGE_CU(launch_router(c, x, w_router, logit_bias, ws.topk_idx, ws.topk_w, ws.hist, ws.rank,
+                          num_sms(), st), "router launch");
+    if (ev) MOGE_CU(cudaEventRecord(ev[1], st), "event");
+    MOGE_CU(launch_scan(c, ws.hist, ws.base, ws.counts, ws.offsets, &ws.plan, true, c.S > 0, st),
+            "scan launch");
+    if (ev) MOGE_CU(cudaEventRecord(ev[2], st), "event");
+    MOGE_CU(launch_scatter_rows(c, x, ws.topk_idx, ws.rank, ws.base, ws.offsets, ws.perm_src,
+                                ws.perm_dst, ws.x_perm, st), "permute launch");
+    if (ev) MOGE_CU(cudaEventRecord(ev[3], st), "event");
+    const int64_t rrows = (int64_t)c.T * K;
+    op.b0 = ws.x_perm;
+    op.b1 = x;
+    op.b0_rows = rrows;
+    op.b1_rows = c.T;
+    op.h = ws.h;
+    op.h_rows = rrows + (int64_t)c.T * c.S;
+    op.y = ws.y_perm;
+    if (fp8) {
+        MOGE_CU(launch_ffn_fp8(c, ws.plan, c.N + c.S, op, num_sms(), st), "grouped FFN (fp8) launch");
+    } else {
+        int rc = run_ffn(c, ws.plan, c.N + c.S, op, st, nullptr);
+        if (rc) return rc;
+    }
+    if (ev) MOGE_CU(cudaEventRecord(ev[4], st), "event");
+    const size_t esz = c.dtype == MOGE_BF16 ? 2 : 4;
+    const void *shared_rows = static_cast<const char *>(ws.y_perm) + (size_t)rrows * c.d * esz;
+    MOGE_CU(launch_combine(c, ws.y_perm, ws.topk_w, ws.perm_dst, K, shared_rows, c.S, residual, y,
+                           st), "combine launch");
+    if (ev) MOGE_CU(cudaEventRecord(ev[5], st), "event");
+    return MOGE_OK;
+}
+
 extern "C" {
 
 size_t moge_workspace_size(const moge_config *cfg) {
@@ -221,15 +274,6 @@ int moge_permute(const moge_config *cfg, const void *x, const int32_t *perm_src,
     return MOGE_OK;
 }
 
-static int run_ffn(const moge_config &c, const Plan &plan, int n_entries, const FfnOperands &op,
-                   cudaStream_t st, cudaEvent_t mid = nullptr) {
-    if (c.dtype == MOGE_BF16)
-        MOGE_CU(launch_ffn_tc(c, plan, n_entries, op, num_sms(), st, mid),
-                "grouped FFN (tcgen05) launch");
-    else
-        MOGE_CU(launch_ffn_f32(c, plan, n_entries, op, st, mid), "grouped FFN (fp32) launch");
-    return MOGE_OK;
-}
 
 int moge_grouped_ffn(const moge_config *cfg, const void *x_perm, const int32_t *offsets,
                      const void *w_gate, const void *w_up, const void *w_down, void *y_perm,
@@ -327,33 +371,11 @@ int moge_layer_forward(const moge_config *cfg, const void *x, const void *w_rout
     MOGE_NEED(y, "y");
     MOGE_NEED(workspace, "workspace");
     if (y == x) return fail(MOGE_ERR_INVALID_ARG, "y must not alias x");
-    cudaStream_t st = (cudaStream_t)stream;
-    Workspace ws = carve_workspace(c, workspace);
-    const int K = c.M * c.Kp;
-    cudaEvent_t *ev = timer_slot();
-    if (ev) MOGE_CU(cudaEventRecord(ev[0], st), "event");
-    MOGE_CU(launch_router(c, x, w_router, logit_bias, ws.topk_idx, ws.topk_w, ws.hist, ws.rank,
-                          num_sms(), st), "router launch");
-    if (ev) MOGE_CU(cudaEventRecord(ev[1], st), "event");
-    MOGE_CU(launch_scan(c, ws.hist, ws.base, ws.counts, ws.offsets, &ws.plan, true, c.S > 0, st),
-            "scan launch");
-    if (ev) MOGE_CU(cudaEventRecord(ev[2], st), "event");
-    MOGE_CU(launch_scatter_rows(c, x, ws.topk_idx, ws.rank, ws.base, ws.offsets, ws.perm_src,
-                                ws.perm_dst, ws.x_perm, st), "permute launch");
-    if (ev) MOGE_CU(cudaEventRecord(ev[3], st), "event");
-    const int64_t rrows = (int64_t)c.T * K;
-    FfnOperands op{ws.x_perm, x, rrows, c.T, w_gate, w_up, w_down,
-                   c.S > 0 ? s_gate : nullptr, c.S > 0 ? s_up : nullptr, c.S > 0 ? s_down : nullptr,
-                   ws.h, rrows + (int64_t)c.T * c.S, ws.y_perm};
-    rc = run_ffn(c, ws.plan, c.N + c.S, op, st, nullptr);
-    if (rc) return rc;
-    if (ev) MOGE_CU(cudaEventRecord(ev[4], st), "event");
-    const size_t esz = c.dtype == MOGE_BF16 ? 2 : 4;
-    const void *shared_rows = static_cast<const char *>(ws.y_perm) + (size_t)rrows * c.d * esz;
-    MOGE_CU(launch_combine(c, ws.y_perm, ws.topk_w, ws.perm_dst, K, shared_rows, c.S, residual, y,
-                           st), "combine launch");
-    if (ev) MOGE_CU(cudaEventRecord(ev[5], st), "event");
-    return MOGE_OK;
+    FfnOperands wts{};
+    wts.wg = w_gate; wts.wu = w_up; wts.wd = w_down;
+    if (c.S > 0) { wts.sg = s_gate; wts.su = s_up; wts.sd = s_down; }
+    return layer_run(c, x, w_router, logit_bias, wts, false, residual, y, workspace,
+                     (cudaStream_t)stream);
 }
 
 int moge_layer_forward_host(const moge_config *cfg, const void *x_host, const void *w_router,
@@ -401,6 +423,62 @@ int moge_rmsnorm(const moge_config *cfg, const void *x, float eps, void *u, void
     if (!(eps >= 0.0f)) return fail(MOGE_ERR_INVALID_ARG, "eps must be >= 0");
     MOGE_CU(launch_rmsnorm(*cfg, x, eps, u, (cudaStream_t)stream), "rmsnorm launch");
     return MOGE_OK;
+}
+
+int moge_quantize_fp8_rows(const void *w, int64_t rows, int64_t cols, void *q, float *scale,
+                           void *stream) {
+    if (rows < 0 || cols <= 0) return fail(MOGE_ERR_INVALID_ARG, "rows must be >= 0, cols > 0");
+    if (cols % 8 != 0) return fail(MOGE_ERR_UNSUPPORTED, "cols must be a multiple of 8");
+    if (rows == 0) return MOGE_OK;
+    MOGE_NEED(w, "w");
+    if (!q) return fail(MOGE_ERR_INVALID_ARG, "q is NULL");
+    if (reinterpret_cast<uintptr_t>(q) % 8 != 0)
+        return fail(MOGE_ERR_UNSUPPORTED, "q is not 8-byte aligned");
+    MOGE_NEED4(scale, "scale");
+    MOGE_CU(launch_quantize_fp8(w, rows, cols, q, scale, (cudaStream_t)stream), "quantize launch");
+    return MOGE_OK;
+}
+
+static int check_fp8_side(const moge_fp8_experts *e, const char *side) {
+    if (!e) return fail(MOGE_ERR_INVALID_ARG, std::string(side) + " fp8 experts are NULL");
+    MOGE_NEED(e->gate, std::string(side) + ".gate");
+    MOGE_NEED(e->up, std::string(side) + ".up");
+    MOGE_NEED(e->down, std::string(side) + ".down");
+    MOGE_NEED4(e->gate_scale, std::string(side) + ".gate_scale");
+    MOGE_NEED4(e->up_scale, std::string(side) + ".up_scale");
+    MOGE_NEED4(e->down_scale, std::string(side) + ".down_scale");
+    return MOGE_OK;
+}
+
+int moge_layer_forward_fp8(const moge_config *cfg, const void *x, const void *w_router,
+                           const float *logit_bias, const moge_fp8_experts *routed,
+                           const moge_fp8_experts *shared, const void *residual, void *y,
+                           void *workspace, void *stream) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    const moge_config c = *cfg;
+    if (c.dtype != MOGE_BF16) return fail(MOGE_ERR_UNSUPPORTED, "fp8 experts need dtype MOGE_BF16");
+    if (c.d % 16 != 0 || c.I % 16 != 0)
+        return fail(MOGE_ERR_UNSUPPORTED, "fp8 experts need d % 16 == 0 and I % 16 == 0");
+    if (c.T == 0) return MOGE_OK;
+    MOGE_NEED(x, "x");
+    MOGE_NEED(w_router, "w_router");
+    if ((rc = check_fp8_side(routed, "routed"))) return rc;
+    if (c.S > 0 && (rc = check_fp8_side(shared, "shared"))) return rc;
+    if (logit_bias && !aligned4(logit_bias)) return fail(MOGE_ERR_UNSUPPORTED, "logit_bias misaligned");
+    if (residual && !aligned16(residual)) return fail(MOGE_ERR_UNSUPPORTED, "residual misaligned");
+    MOGE_NEED(y, "y");
+    MOGE_NEED(workspace, "workspace");
+    if (y == x) return fail(MOGE_ERR_INVALID_ARG, "y must not alias x");
+    FfnOperands op{};
+    op.wg = routed->gate; op.wu = routed->up; op.wd = routed->down;
+    op.wg_s = routed->gate_scale; op.wu_s = routed->up_scale; op.wd_s = routed->down_scale;
+    if (c.S > 0) {
+        op.sg = shared->gate; op.su = shared->up; op.sd = shared->down;
+        op.sg_s = shared->gate_scale; op.su_s = shared->up_scale; op.sd_s = shared->down_scale;
+    }
+    return layer_run(c, x, w_router, logit_bias, op, true, residual, y, workspace,
+                     (cudaStream_t)stream);
 }
 
 int moge_stage_timing(int enable) {

@@ -3,5 +3,6 @@
 #include "rows.cu"
 #include "gemm_f32.cu"
 #include "gemm_tc.cu"
+#include "gemm_fp8.cu"
 #include "api.cu"
 #include "route_noalloc.cu"

@@ -123,6 +123,10 @@ struct FfnOperands {
     void *h;                 // [h_rows][I]
     int64_t h_rows;
     void *y;                 // [h_rows][d]
+    // FP8 weights only (launch_ffn_fp8): the w*/s* pointers above are E4M3
+    // codes and these their per-row fp32 scales ([E][I], [E][I], [E][d])
+    const float *wg_s, *wu_s, *wd_s;
+    const float *sg_s, *su_s, *sd_s;
 };
 // `mid` (may be null) is recorded on the stream between the up- and the
 // down-projection launches.
@@ -130,5 +134,11 @@ cudaError_t launch_ffn_tc(const moge_config &c, const Plan &plan, int n_entries,
                           const FfnOperands &op, int num_sms, cudaStream_t st, cudaEvent_t mid);
 cudaError_t launch_ffn_f32(const moge_config &c, const Plan &plan, int n_entries,
                            const FfnOperands &op, cudaStream_t st, cudaEvent_t mid);
+// grouped FFN with FP8 (E4M3, per-row scale) weights and bf16 activations
+cudaError_t launch_ffn_fp8(const moge_config &c, const Plan &plan, int n_entries,
+                           const FfnOperands &op, int num_sms, cudaStream_t st);
+// per-row FP8 quantisation of bf16 rows
+cudaError_t launch_quantize_fp8(const void *w, int64_t rows, int64_t cols, void *q, float *scale,
+                                cudaStream_t st);
 
 }  // namespace moge

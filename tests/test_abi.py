@@ -94,3 +94,29 @@ def test_no_cpu_fallback_when_library_missing(monkeypatch):
     monkeypatch.setattr(mg, "LIB_PATH", "/nonexistent/libmoge.so")
     with pytest.raises(ImportError):
         mg.lib()
+
+
+def test_fp8_entry_points_validate_on_host(L):
+    # quantiser: shape and alignment rules before anything is enqueued
+    assert L.moge_quantize_fp8_rows(0x1000, 4, 12, 0x2000, 0x3000, None) == mg.ERR_UNSUPPORTED
+    assert b"multiple of 8" in L.moge_last_error()
+    assert L.moge_quantize_fp8_rows(0x1000, 4, 16, 0x2004, 0x3000, None) == mg.ERR_UNSUPPORTED
+    assert L.moge_quantize_fp8_rows(None, 4, 16, 0x2000, 0x3000, None) == mg.ERR_INVALID_ARG
+    assert L.moge_quantize_fp8_rows(None, 0, 16, None, None, None) == mg.OK
+    # layer: bf16 only, 16-byte rows of codes, both sides' pointers present
+    f8 = mg.moge_fp8_experts(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000)
+    args = (0x7000, 0x8000, None, ctypes.byref(f8), ctypes.byref(f8), None, 0x9000, 0xA000, None)
+    rc = L.moge_layer_forward_fp8(ctypes.byref(mg._cfg(_shape(dtype="f32"))), *args)
+    assert rc == mg.ERR_UNSUPPORTED and b"BF16" in L.moge_last_error()
+    rc = L.moge_layer_forward_fp8(ctypes.byref(mg._cfg(_shape(dtype="bf16", I=136))), *args)
+    assert rc == mg.ERR_UNSUPPORTED and b"% 16" in L.moge_last_error()
+    rc = L.moge_layer_forward_fp8(ctypes.byref(mg._cfg(_shape(dtype="bf16"))), 0x7000, 0x8000, None,
+                                  None, ctypes.byref(f8), None, 0x9000, 0xA000, None)
+    assert rc == mg.ERR_INVALID_ARG and b"routed" in L.moge_last_error()
+    rc = L.moge_layer_forward_fp8(ctypes.byref(mg._cfg(_shape(dtype="bf16"))), 0x7000, 0x8000, None,
+                                  ctypes.byref(f8), None, None, 0x9000, 0xA000, None)
+    assert rc == mg.ERR_INVALID_ARG and b"shared" in L.moge_last_error()
+    bad = mg.moge_fp8_experts(0x1000, 0x2000, 0x3000, 0x4002, 0x5000, 0x6000)
+    rc = L.moge_layer_forward_fp8(ctypes.byref(mg._cfg(_shape(dtype="bf16"))), 0x7000, 0x8000, None,
+                                  ctypes.byref(bad), ctypes.byref(f8), None, 0x9000, 0xA000, None)
+    assert rc == mg.ERR_UNSUPPORTED and b"gate_scale" in L.moge_last_error()
