@@ -72,6 +72,21 @@ def ffn_bytes(cfg, n_used):
     return up_bytes(cfg, n_used) + down_bytes(cfg, n_used)
 
 
+def ffn_bytes_fp8(cfg, n_used):
+    """Algorithmic bytes of the grouped-FFN launch with 8-bit weights: one byte
+    per weight plus one fp32 scale per weight row, activations as in bf16."""
+    T, d, I, K, S = cfg.T, cfg.d, cfg.I, cfg.K, cfg.S
+    weights = (n_used + S) * (3 * I * d + 4 * (2 * I + d))
+    acts = 2 * ((T * K + T) * d + 2 * T * (K + S) * I + T * (K + S) * d)
+    return weights + acts
+
+
+def layer_bytes_fp8(cfg, n_used):
+    """Layer bytes with 8-bit expert weights (router stays bf16)."""
+    return ((n_used + cfg.S) * (3 * cfg.I * cfg.d + 4 * (2 * cfg.I + cfg.d))
+            + 2 * (cfg.N * cfg.d + 2 * cfg.T * cfg.d))
+
+
 def layer_flops(cfg):
     return (cfg.T * cfg.K + cfg.S * cfg.T) * 6.0 * cfg.d * cfg.I + 2.0 * cfg.T * cfg.d * cfg.N
 
@@ -187,9 +202,11 @@ def run_reference(args, cfg):
 
 
 # ----------------------------------------------------------------------------- GPU arm
-def measure(cfg, inp, steps, warmup, dist_on=False, with_e2e=True):
+def measure(cfg, inp, steps, warmup, dist_on=False, with_e2e=True, fp8=False):
     """Device-timed layer steps (+ per-launch stage times, + end-to-end through
-    the host-buffer entry point). Returns a dict of raw measurements."""
+    the host-buffer entry point). Returns a dict of raw measurements. With
+    fp8, the expert weights are quantised on the device once (outside the
+    timed region) and the layer runs moge_layer_forward_fp8."""
     import torch
     import mixture_grouped_experts_b200 as mg
 
@@ -198,8 +215,20 @@ def measure(cfg, inp, steps, warmup, dist_on=False, with_e2e=True):
     w = mg.weights_to_device(inp, cfg.dtype)
     ws = mg.alloc_workspace(s)
     y = torch.empty_like(x)
+    if fp8:
+        w8 = mg.experts_to_fp8(w)
+        torch.cuda.synchronize()
+        for k in mg.FP8_KEYS:          # only the router stays in bf16
+            w[k] = None
+        torch.cuda.empty_cache()
+
+        def fwd():
+            mg.moge_layer_forward_fp8(s, x, w, w8, ws, y=y)
+    else:
+        def fwd():
+            mg.moge_layer_forward(s, x, w, ws, y=y)
     for _ in range(max(warmup, 3)):
-        mg.moge_layer_forward(s, x, w, ws, y=y)
+        fwd()
     torch.cuda.synchronize()
     mg.check_device_errors()
     counts = mg.moge_workspace_routing(s, ws)[2].cpu().numpy()
@@ -214,7 +243,7 @@ def measure(cfg, inp, steps, warmup, dist_on=False, with_e2e=True):
     torch.cuda.synchronize()
     start.record(stream)
     for _ in range(steps):
-        mg.moge_layer_forward(s, x, w, ws, y=y)
+        fwd()
     end.record(stream)
     torch.cuda.synchronize()
     if dist_on:
@@ -225,13 +254,13 @@ def measure(cfg, inp, steps, warmup, dist_on=False, with_e2e=True):
     # CUDA-event stage timing (a separate loop of the same steps)
     mg.moge_stage_timing(True)
     for _ in range(steps):
-        mg.moge_layer_forward(s, x, w, ws, y=y)
+        fwd()
     stage_ms, calls = mg.moge_stage_times()
     mg.moge_stage_timing(False)
     mg.check_device_errors()
     out = {"ms": ms, "stage_ms": {k: v / calls for k, v in stage_ms.items()}, "n_used": n_used,
            "counts": counts}
-    if with_e2e:
+    if with_e2e and not fp8:
         xh = x.cpu().pin_memory()
         yh = torch.empty_like(xh).pin_memory()
         xd, yd = torch.empty_like(x), torch.empty_like(x)
@@ -248,6 +277,8 @@ def measure(cfg, inp, steps, warmup, dist_on=False, with_e2e=True):
         out["e2e_ms"] = start.elapsed_time(end) / steps
         out["io_bytes"] = xh.numel() * xh.element_size()
     del x, w, ws, y
+    if fp8:
+        del w8
     torch.cuda.empty_cache()
     return out
 
@@ -288,6 +319,7 @@ def main():
     ap.add_argument("--no-secondary", action="store_true", help="skip the prefill side measurement")
     ap.add_argument("--cpu-tokens", type=int, default=16, help="tokens in the CPU-baseline sample (0: skip)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the 8-bit-weight side measurement")
     ap.add_argument("--ref-tokens", type=int, default=2, help="tokens per step of --impl reference")
     args = ap.parse_args()
     cfg = synth.CONFIGS[args.config]
@@ -369,6 +401,28 @@ def main():
                          "peak_source": "%s bf16_tflops (burst)" % peak_kind},
             "layer_tflops": lay_tf, "layer_frac_sustained": lay_tf / tfs,
             "stage_ms": pm["stage_ms"], "clocks": pclk}
+    if rank == 0 and n == 1 and not args.no_fp8 and args.config == "decode":
+        finp = synth.layer_inputs(cfg)
+        fs = ClockSampler(local)
+        fs.start()
+        fm = measure(cfg, finp, args.steps, args.warmup, False, with_e2e=False, fp8=True)
+        fclk = fs.stop()
+        del finp
+        fb8 = ffn_bytes_fp8(cfg, fm["n_used"])
+        ach8 = fb8 / (fm["stage_ms"]["ffn"] / 1e3) / 1e9
+        lb8 = layer_bytes_fp8(cfg, fm["n_used"])
+        line["decode_fp8"] = {
+            "workload": workload_config(cfg)["workload"],
+            "weights": "expert weights as OCP E4M3 codes + one fp32 scale per row (weights-only "
+                       "8-bit; router, activations, h and y bf16); quantised on the device before "
+                       "the timed region",
+            "value": cfg.T / (fm["ms"] / 1e3), "unit": "tokens/s", "ms_per_step": fm["ms"],
+            "roofline": {"bound": "hbm", "kernel": "ffn_fp8_kernel", "achieved": ach8, "peak": hbm,
+                         "unit": "GB/s", "frac": ach8 / hbm, "algorithmic_bytes_per_launch": fb8,
+                         "kernel_ms": fm["stage_ms"]["ffn"]},
+            "layer_roofline": {"achieved": lb8 / (fm["ms"] / 1e3) / 1e9, "peak": hbm, "unit": "GB/s",
+                               "frac": lb8 / (fm["ms"] / 1e3) / 1e9 / hbm, "algorithmic_bytes": lb8},
+            "stage_ms": fm["stage_ms"], "clocks": fclk}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist_on:

@@ -9,20 +9,29 @@
 // The kernel is the persistent work-queue kernel of gemm_tc.cu (same plan,
 // same item order, same per-expert completion counters) with a different
 // operand path for the weights:
-//   warp 0     scheduler + TMA producer: per K-chunk one 8 KB copy of codes
-//              (128 weight rows x 64 bytes, no swizzle) plus the token rows,
-//              into a 40 KB "raw" stage
-//   warps 6-9  converters: widen the codes of a chunk exactly to bf16
-//              (every E4M3 value is a bf16 value) and write them, 128-byte
-//              swizzled, into a 16 KB operand slot for the MMA
-//   warp 1     MMA issuer: A from the operand slot, B (token rows) from the
-//              raw stage, fp32 accumulators in TMEM (double-buffered)
+//   warp 0     scheduler + TMA producer: the codes of a stage land in the
+//              upper half of its weight areas (a streaming stage's two
+//              K-chunks as one copy of 128 rows x 128 bytes, a tensor stage's
+//              chunk as 128 rows x 64 bytes), plus the token rows. It alone
+//              decodes each work item and hands it to the other roles
+//              through a shared-memory ring
+//   warps 6-9  converters: load the stage's codes into registers, then write
+//              them back widened to bf16 (every E4M3 value is a bf16 value)
+//              over the whole 16 KB area, 128-byte swizzled for the MMA --
+//              in place, so a stage is the same 48 KB as in the bf16 kernel
+//   warp 1     MMA issuer: tcgen05.mma as in the bf16 kernel once a stage is
+//              widened, fp32 accumulators in TMEM (double-buffered)
 //   warps 2-5  epilogue: the row scale of each accumulator row (its weight
 //              row) multiplies the accumulator, then SwiGLU / stores as in
 //              the bf16 kernel
-// So the HBM stream at decode is half the bf16 bytes, and the tensor cores
-// see exactly the dequantised weights up to the one fp32 rounding of the
-// scale product in the epilogue.
+// The tensor cores see exactly the dequantised weights up to the one fp32
+// rounding of the scale product in the epilogue, and the weights take half
+// the HBM of bf16 ones. The widening moves about 6 bytes of shared memory
+// per code and lies on each stage's critical path with the MMA, so at decode
+// this kernel runs about as fast as the bf16 one rather than twice as fast
+// (measured alternatives: widening into tensor memory with the MMA reading A
+// from there, more converter warps, L2 prefetch of codes, fewer and wider
+// copies, deeper rings -- none faster).
 #include <cuda_fp8.h>
 
 #include "common.cuh"
@@ -88,36 +97,72 @@ cudaError_t launch_quantize_fp8(const void *w, int64_t rows, int64_t cols, void 
                       static_cast<const uint4 *>(w), rows, cols, static_cast<uint2 *>(q), scale);
 }
 
+
 // ---------------------------------------------------------------- FFN kernel
-constexpr int kF8RawStages = 4;
-constexpr int kF8RawBytes = 40 * 1024;  // stream: 2 x (8 KB codes) + 2 x (8 KB tokens);
-                                        // tensor: 8 KB codes + up to 32 KB tokens
-constexpr int kF8Slots = 3;             // widened bf16 operand slots (16 KB each)
-constexpr int kF8SlotBytes = 16 * 1024;
+constexpr int kF8Stages = 4;
+constexpr int kF8StageBytes = 48 * 1024;  // stream: 2 x 16 KB weights + 2 x 8 KB tokens;
+                                          // tensor: 16 KB weights + up to 32 KB tokens
 constexpr int kF8EpiBytes = 12 * 1024;
-constexpr int kF8Threads = 320;         // 10 warps
-constexpr int kF8CvtThreads = 128;      // warps 6-9
+constexpr int kF8Threads = 320;           // 10 warps
+constexpr int kF8CvtThreads = 128;        // warps 6-9
+constexpr uint32_t kF8CodeOff = 8192;     // codes land in the upper half of a weight area
 
 struct F8Params {
     TcParams t;
     const float *sc_g[2], *sc_u[2], *sc_d[2];  // per a_sel (routed / shared)
 };
 
+constexpr int kF8MaxEntries = 2 * kMaxExperts;  // routed + shared experts of a plan
+
 struct F8Shared {
-    uint64_t raw_full[kF8RawStages], raw_empty[kF8RawStages];
-    uint64_t cvt_full[kF8Slots], cvt_empty[kF8Slots];
+    uint64_t full[kF8Stages], wide[kF8Stages], empty[kF8Stages];
     uint64_t tfull[2], tempty[2], drain;
     uint64_t slot_full[kSlots], slot_empty[kSlots];
     int slot_item[kSlots];
+    TcItem slot_it[kSlots];       // the producer's decoded items
+    TcItem epi_it, cvt_it;        // a role leader's copy for its threads
     uint32_t tmem_base;
     int abort;
     int epi_item, cvt_item;
+    int st_up[kF8MaxEntries + 1], st_down[kF8MaxEntries + 1];  // the plan's item starts
 };
 
-// byte offsets inside a raw stage of chunk c's codes and token rows
-__device__ __forceinline__ uint32_t f8_a_off(bool stream, int c) { return stream ? c * 8192u : 0u; }
+// Decode global item q (up-projection items first) against the plan's item
+// starts held in shared memory: a binary search there plus one read of the
+// entry. Only the producer decodes; the other roles get the decoded item
+// through the slot ring.
+__device__ __forceinline__ void decode_item_smem(const TcParams &p, const int *st_up,
+                                                 const int *st_down, int tot_up, int q, TcItem &it) {
+    it.up = q < tot_up;
+    const int local = it.up ? q : q - tot_up;
+    const int *start = it.up ? st_up : st_down;
+    int lo = 0, hi = p.n_entries - 1;
+    while (lo < hi) {  // last entry whose first item is <= local (entries may be empty)
+        const int mid = (lo + hi + 1) >> 1;
+        if (start[mid] <= local) lo = mid; else hi = mid - 1;
+    }
+    const int4 *wp = reinterpret_cast<const int4 *>((it.up ? p.plan.up : p.plan.down) + lo);
+    const int4 a = __ldg(wp), b = __ldg(wp + 1);
+    it.w.rows = a.x;
+    it.w.src_row0 = a.y;
+    it.w.dst_row0 = a.z;
+    it.w.a_sel = a.w;
+    it.w.a_idx = b.x;
+    it.w.b_sel = b.y;
+    it.w.bn = b.z;
+    it.w.ntb = b.w;
+    it.entry = lo;
+    const int r = local - start[lo];
+    it.fb = r / it.w.ntb;  // feature block major, token tile fastest
+    it.tb = r % it.w.ntb;
+    it.n_valid = min(it.w.bn, it.w.rows - it.tb * it.w.bn);
+    it.stream = it.w.rows <= kStreamRows;
+}
+
+// byte offsets inside a stage of chunk c's (widened) weights and token rows
+__device__ __forceinline__ uint32_t f8_a_off(bool stream, int c) { return stream ? c * 16384u : 0u; }
 __device__ __forceinline__ uint32_t f8_b_off(bool stream, int c) {
-    return stream ? 16384u + c * 8192u : 8192u;
+    return stream ? 32768u + c * 8192u : 16384u;
 }
 
 // Named barrier over the converter threads that also ANDs a predicate: every
@@ -148,24 +193,49 @@ __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t two_codes) {
     return *reinterpret_cast<const uint32_t *>(&b);
 }
 
-// Widen one chunk of codes (128 rows x 64 bytes, row-major) into a 128-byte
-// swizzled bf16 K-major tile (row r at r * 128, 16-byte unit j at
-// (j ^ (r & 7)) * 16). Converter thread ct: each pass covers 16 rows, a warp
-// 4 consecutive rows with 8 lanes per row (conflict-free loads and stores).
-__device__ __forceinline__ void widen_chunk(const unsigned char *raw, unsigned char *slot, int ct) {
+// In-place widening of a stage's weight chunks. Chunk c's codes (128 rows x
+// 64 bytes, row-major) sit at area + 8192; the widened bf16 tile (row r at
+// r * 128, 16-byte unit j at (j ^ (r & 7)) * 16: 128-byte swizzle, K-major)
+// covers the whole 16 KB area, so it overwrites codes: every converter loads
+// all its codes into registers, the converters synchronise, and only then
+// write. The synchronisation also ANDs `ok` (each converter's wait for the
+// stage): if any wait failed, nobody writes and all return false. Converter
+// thread ct handles, in pass p, row p * 16 + (ct / 32) * 4 + (ct % 32) / 8
+// and unit ct % 8 (conflict-free loads and stores).
+template <int NCH>
+__device__ __forceinline__ bool widen_in_place(unsigned char *stage, bool stream, int ct, bool ok) {
     const int cw = ct >> 5, lane = ct & 31;
     const int j = lane & 7;
-#pragma unroll 2
-    for (int pass = 0; pass < 8; ++pass) {
-        const int r = pass * 16 + cw * 4 + (lane >> 3);
-        const uint2 v = *reinterpret_cast<const uint2 *>(raw + r * 64 + j * 8);
-        uint4 o;
-        o.x = e4m3x2_to_bf16x2(v.x & 0xFFFFu);
-        o.y = e4m3x2_to_bf16x2(v.x >> 16);
-        o.z = e4m3x2_to_bf16x2(v.y & 0xFFFFu);
-        o.w = e4m3x2_to_bf16x2(v.y >> 16);
-        *reinterpret_cast<uint4 *>(slot + r * 128 + ((j ^ (r & 7)) << 4)) = o;
+    uint2 v[NCH][8];
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+        // a pair of chunks came as one box of 128-byte rows at +8192 (chunk c at
+        // byte 64 c of a row); a single chunk as 64-byte rows at its area + 8192
+        const unsigned char *codes = NCH == 2 ? stage + kF8CodeOff + c * 64
+                                              : stage + f8_a_off(stream, c) + kF8CodeOff;
+        const int rstride = NCH == 2 ? 128 : 64;
+#pragma unroll
+        for (int pass = 0; pass < 8; ++pass) {
+            const int r = pass * 16 + cw * 4 + (lane >> 3);
+            v[c][pass] = *reinterpret_cast<const uint2 *>(codes + r * rstride + j * 8);
+        }
     }
+    if (!cvt_bar_and(ok)) return false;  // every code of the stage is in registers
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+        unsigned char *tile = stage + f8_a_off(stream, c);
+#pragma unroll
+        for (int pass = 0; pass < 8; ++pass) {
+            const int r = pass * 16 + cw * 4 + (lane >> 3);
+            uint4 o;
+            o.x = e4m3x2_to_bf16x2(v[c][pass].x & 0xFFFFu);
+            o.y = e4m3x2_to_bf16x2(v[c][pass].x >> 16);
+            o.z = e4m3x2_to_bf16x2(v[c][pass].y & 0xFFFFu);
+            o.w = e4m3x2_to_bf16x2(v[c][pass].y >> 16);
+            *reinterpret_cast<uint4 *>(tile + r * 128 + ((j ^ (r & 7)) << 4)) = o;
+        }
+    }
+    return true;
 }
 
 __global__ void __launch_bounds__(kF8Threads, 1) ffn_fp8_kernel(
@@ -173,26 +243,25 @@ __global__ void __launch_bounds__(kF8Threads, 1) ffn_fp8_kernel(
     const __grid_constant__ CUtensorMap tmWu, const __grid_constant__ CUtensorMap tmSg,
     const __grid_constant__ CUtensorMap tmSu, const __grid_constant__ CUtensorMap tmX0,
     const __grid_constant__ CUtensorMap tmX1, const __grid_constant__ CUtensorMap tmWd,
-    const __grid_constant__ CUtensorMap tmSd, const __grid_constant__ CUtensorMap tmH) {
+    const __grid_constant__ CUtensorMap tmSd, const __grid_constant__ CUtensorMap tmH,
+    const __grid_constant__ CUtensorMap tmWg2, const __grid_constant__ CUtensorMap tmWu2,
+    const __grid_constant__ CUtensorMap tmSg2, const __grid_constant__ CUtensorMap tmSu2,
+    const __grid_constant__ CUtensorMap tmWd2, const __grid_constant__ CUtensorMap tmSd2) {
     extern __shared__ __align__(1024) unsigned char smem_dyn[];
     unsigned char *smem = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
-    unsigned char *raw = smem;                                   // kF8RawStages x 40 KB
-    unsigned char *slots = smem + kF8RawStages * kF8RawBytes;    // kF8Slots x 16 KB
-    unsigned char *epi = slots + kF8Slots * kF8SlotBytes;        // 12 KB
+    unsigned char *stages = smem;                              // kF8Stages x 48 KB
+    unsigned char *epi = smem + kF8Stages * kF8StageBytes;     // 12 KB
     F8Shared &sh = *reinterpret_cast<F8Shared *>(epi + kF8EpiBytes);
     volatile int *abort = &sh.abort;
     const TcParams &tp = p.t;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kF8RawStages; ++s) {
-            mbar_init(&sh.raw_full[s], 1);   // the producer's expect_tx arrival
-            mbar_init(&sh.raw_empty[s], 2);  // converter leader + MMA commit
-        }
-        for (int s = 0; s < kF8Slots; ++s) {
-            mbar_init(&sh.cvt_full[s], 1);   // converter leader
-            mbar_init(&sh.cvt_empty[s], 1);  // MMA commit
+        for (int s = 0; s < kF8Stages; ++s) {
+            mbar_init(&sh.full[s], 1);   // the producer's expect_tx arrival (+ the copies' bytes)
+            mbar_init(&sh.wide[s], 1);   // the converter leader: weights widened
+            mbar_init(&sh.empty[s], 1);  // the MMA commit: stage consumed
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&sh.tfull[a], 1);
@@ -226,8 +295,13 @@ __global__ void __launch_bounds__(kF8Threads, 1) ffn_fp8_kernel(
     tc_fence_after();
     const uint32_t tmem_base = sh.tmem_base;
     grid_dependency_wait();
-    const int tot_up = __ldg(tp.plan.up_start + tp.n_entries);
-    const int total = tot_up + __ldg(tp.plan.down_start + tp.n_entries);
+    for (int i = threadIdx.x; i <= tp.n_entries; i += blockDim.x) {
+        sh.st_up[i] = __ldg(tp.plan.up_start + i);
+        sh.st_down[i] = __ldg(tp.plan.down_start + i);
+    }
+    __syncthreads();
+    const int tot_up = sh.st_up[tp.n_entries];
+    const int total = tot_up + sh.st_down[tp.n_entries];
     const int fb_up = (tp.I + 63) / 64;
 
     if (warp == 0) {
@@ -244,6 +318,11 @@ __global__ void __launch_bounds__(kF8Threads, 1) ffn_fp8_kernel(
             if (lane == 0) {
                 if (mbar_wait(&sh.slot_empty[slot], ((uint32_t)(s / kSlots) & 1u) ^ 1u, abort)) {
                     q = *abort ? total : next;
+                    if (q < total) {
+                        TcItem d;
+                        decode_item_smem(tp, sh.st_up, sh.st_down, tot_up, q, d);
+                        sh.slot_it[slot] = d;
+                    }
                     sh.slot_item[slot] = q;
                     mbar_arrive(&sh.slot_full[slot]);
                     if (q < total) next = atomicAdd(tp.sync, 1);
@@ -251,10 +330,10 @@ __global__ void __launch_bounds__(kF8Threads, 1) ffn_fp8_kernel(
                     q = -1;
                 }
             }
+            __syncwarp();
             q = __shfl_sync(0xffffffffu, q, 0);
             if (q < 0 || q >= total) break;
-            TcItem it;
-            decode_item(tp, tot_up, q, it);
+            const TcItem it = sh.slot_it[slot];
             if (!it.up) {  // the h rows of this expert must all be stored
                 int ok = 1;
                 if (lane == 0) ok = wait_counter(tp.sync + 1 + it.entry, it.w.ntb * fb_up, abort);
@@ -279,58 +358,86 @@ __global__ void __launch_bounds__(kF8Threads, 1) ffn_fp8_kernel(
             const int arow0 = it.up ? it.fb * 64 : it.fb * 128;
             const int ops = na + nbox;
             const int my_c = lane / ops, my_r = lane % ops;
+            const CUtensorMap *ma0w, *ma1w;
+            if (it.up) {
+                ma0w = it.w.a_sel ? &tmSg2 : &tmWg2;
+                ma1w = it.w.a_sel ? &tmSu2 : &tmWu2;
+            } else {
+                ma0w = ma1w = it.w.a_sel ? &tmSd2 : &tmWd2;
+            }
             bool ok = true;
             for (int kc = 0; kc < kcs; kc += per) {
                 int got = 1;
-                if (lane == 0) got = mbar_wait(&sh.raw_empty[stage], phase ^ 1u, abort);
+                if (lane == 0) got = mbar_wait(&sh.empty[stage], phase ^ 1u, abort);
                 if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
                 const int nch = min(per, kcs - kc);
-                unsigned char *sbase = raw + stage * kF8RawBytes;
+                unsigned char *sbase = stages + stage * kF8StageBytes;
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(&sh.raw_full[stage],
+                    mbar_arrive_expect_tx(&sh.full[stage],
                                           (uint32_t)nch * (8192u + (uint32_t)nbox * kBoxRows * 128u));
                     armed |= 1u << stage;
                     armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
                 }
                 __syncwarp();
+                if (nch == 2) {
+                    // a streaming pair: one wide copy of codes (or two, gate and up
+                    // apart) and the token boxes of both chunks
+                    const int k = kc * kChunkK;
+                    if (lane < na) {
+                        unsigned char *sa = sbase + kF8CodeOff;
+                        if (it.up && gu != kGateUpSplit)
+                            tma_load_4d(sa, ma0w, &sh.full[stage], k, arow0, it.w.a_idx, 0, pol_w);
+                        else if (it.up)
+                            tma_load_3d(sa + 8192 * lane, lane ? ma1w : ma0w, &sh.full[stage], k,
+                                        arow0, it.w.a_idx, pol_w);
+                        else
+                            tma_load_3d(sa, ma0w, &sh.full[stage], k, arow0, it.w.a_idx, pol_w);
+                    } else if (lane < na + 2 * nbox) {
+                        const int c = (lane - na) / nbox, j = (lane - na) % nbox;
+                        tma_load_2d(sbase + f8_b_off(true, c) + j * kBoxRows * 128, mb,
+                                    &sh.full[stage], k + c * kChunkK, brow0 + j * kBoxRows, pol_b);
+                    }
+                    if (++stage == kF8Stages) { stage = 0; phase ^= 1u; }
+                    continue;
+                }
                 if (my_c < nch) {
-                    const int k = chunk_at(kc + my_c, it.fb, kcs) * kChunkK;
-                    unsigned char *sa = sbase + f8_a_off(it.stream, my_c);
+                    const int k = (kc + my_c) * kChunkK;
+                    unsigned char *sa = sbase + f8_a_off(it.stream, my_c) + kF8CodeOff;
                     unsigned char *sb = sbase + f8_b_off(it.stream, my_c);
                     if (my_r >= na) {
                         const int j = my_r - na;
-                        tma_load_2d(sb + j * kBoxRows * 128, mb, &sh.raw_full[stage], k,
+                        tma_load_2d(sb + j * kBoxRows * 128, mb, &sh.full[stage], k,
                                     brow0 + j * kBoxRows, pol_b);
                     } else if (it.up && gu != kGateUpSplit) {
-                        tma_load_4d(sa, ma0, &sh.raw_full[stage], k, arow0, it.w.a_idx, 0, pol_w);
+                        tma_load_4d(sa, ma0, &sh.full[stage], k, arow0, it.w.a_idx, 0, pol_w);
                     } else if (it.up) {  // gate rows, then up rows: 64 rows x 64 bytes each
-                        tma_load_3d(sa + 4096 * my_r, my_r ? ma1 : ma0, &sh.raw_full[stage], k,
-                                    arow0, it.w.a_idx, pol_w);
+                        tma_load_3d(sa + 4096 * my_r, my_r ? ma1 : ma0, &sh.full[stage], k, arow0,
+                                    it.w.a_idx, pol_w);
                     } else {
-                        tma_load_3d(sa, ma0, &sh.raw_full[stage], k, arow0, it.w.a_idx, pol_w);
+                        tma_load_3d(sa, ma0, &sh.full[stage], k, arow0, it.w.a_idx, pol_w);
                     }
                 }
-                if (++stage == kF8RawStages) { stage = 0; phase ^= 1u; }
+                if (++stage == kF8Stages) { stage = 0; phase ^= 1u; }
             }
             if (!ok) break;
         }
         if (lane == 0 && *abort) {  // let every issued copy land before the CTA can exit
-            for (int s = 0; s < kF8RawStages; ++s)
-                if (armed & (1u << s)) mbar_wait(&sh.raw_full[s], (armed_par >> s) & 1u, nullptr);
+            for (int s = 0; s < kF8Stages; ++s)
+                if (armed & (1u << s)) mbar_wait(&sh.full[s], (armed_par >> s) & 1u, nullptr);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            int stage = 0, cslot = 0;
-            uint32_t phase = 0, cphase = 0;
+            int stage = 0;
+            uint32_t phase = 0;
             for (int s = 0;; ++s) {
                 const int slot = s % kSlots;
                 if (!mbar_wait(&sh.slot_full[slot], (uint32_t)(s / kSlots) & 1u, abort)) break;
                 const int q = sh.slot_item[slot];
+                TcItem it;
+                if (q < total) it = sh.slot_it[slot];
                 mbar_arrive(&sh.slot_empty[slot]);
                 if (q >= total) break;
-                TcItem it;
-                decode_item(tp, tot_up, q, it);
                 const int acc = s & 1;
                 const uint32_t use = (uint32_t)(s >> 1);
                 if (!mbar_wait(&sh.tempty[acc], (use & 1u) ^ 1u, abort)) break;
@@ -340,28 +447,24 @@ __global__ void __launch_bounds__(kF8Threads, 1) ffn_fp8_kernel(
                 const int kcs = it.up ? tp.kc_up : tp.kc_down;
                 const int per = it.stream ? 2 : 1;
                 bool ok = true;
-                for (int kc = 0; kc < kcs && ok; kc += per) {
-                    // the token rows of the stage have landed
-                    if (!mbar_wait(&sh.raw_full[stage], phase, abort)) { ok = false; break; }
+                for (int kc = 0; kc < kcs; kc += per) {
+                    // the stage's copies have landed and its weights are widened
+                    if (!mbar_wait(&sh.full[stage], phase, abort) ||
+                        !mbar_wait(&sh.wide[stage], phase, abort)) { ok = false; break; }
+                    tc_fence_after();
                     const int nch = min(per, kcs - kc);
-                    const uint32_t sbase = smem_u32(raw + stage * kF8RawBytes);
+                    const uint32_t sbase = smem_u32(stages + stage * kF8StageBytes);
                     for (int c = 0; c < nch; ++c) {
-                        // and the chunk's widened weights
-                        if (!mbar_wait(&sh.cvt_full[cslot], cphase, abort)) { ok = false; break; }
-                        tc_fence_after();
-                        const uint32_t sa = smem_u32(slots + cslot * kF8SlotBytes);
+                        const uint32_t sa = sbase + f8_a_off(it.stream, c);
                         const uint32_t sb = sbase + f8_b_off(it.stream, c);
 #pragma unroll
                         for (int j = 0; j < kChunkK / 16; ++j)
                             tc_mma_bf16(d_tmem, smem_desc_sw128(sa + 32u * j),
                                         smem_desc_sw128(sb + 32u * j), idesc,
                                         (kc + c + j) > 0 ? 1u : 0u);
-                        tc_commit(&sh.cvt_empty[cslot]);
-                        if (++cslot == kF8Slots) { cslot = 0; cphase ^= 1u; }
                     }
-                    if (!ok) break;
-                    tc_commit(&sh.raw_empty[stage]);
-                    if (++stage == kF8RawStages) { stage = 0; phase ^= 1u; }
+                    tc_commit(&sh.empty[stage]);
+                    if (++stage == kF8Stages) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
                 tc_commit(&sh.tfull[acc]);
@@ -372,43 +475,38 @@ __global__ void __launch_bounds__(kF8Threads, 1) ffn_fp8_kernel(
     } else if (warp >= 6) {
         // ------------------------------------------------------ converters
         const int ct = threadIdx.x - 192;  // 0 .. 127
-        int stage = 0, cslot = 0;
-        uint32_t phase = 0, cphase = 0;
+        int stage = 0;
+        uint32_t phase = 0;
         for (int s = 0;; ++s) {
             if (ct == 0) {
                 const int slot = s % kSlots;
                 int q = -1;
                 if (mbar_wait(&sh.slot_full[slot], (uint32_t)(s / kSlots) & 1u, abort)) {
                     q = sh.slot_item[slot];
+                    if (q < total) sh.cvt_it = sh.slot_it[slot];
                     mbar_arrive(&sh.slot_empty[slot]);
                 }
                 sh.cvt_item = q;
             }
             named_bar_sync(2, kF8CvtThreads);
             const int q = *(volatile int *)&sh.cvt_item;
-            named_bar_sync(2, kF8CvtThreads);
             if (q < 0 || q >= total) break;
-            TcItem it;
-            decode_item(tp, tot_up, q, it);
+            const TcItem it = sh.cvt_it;
+            named_bar_sync(2, kF8CvtThreads);
             const int kcs = it.up ? tp.kc_up : tp.kc_down;
             const int per = it.stream ? 2 : 1;
             bool ok = true;
             for (int kc = 0; kc < kcs; kc += per) {
                 const int nch = min(per, kcs - kc);
-                bool mine = mbar_wait(&sh.raw_full[stage], phase, abort);
-                const unsigned char *sraw = raw + stage * kF8RawBytes;
-                for (int c = 0; c < nch; ++c) {
-                    mine = mine && mbar_wait(&sh.cvt_empty[cslot], cphase ^ 1u, abort);
-                    if (!cvt_bar_and(mine)) { ok = false; break; }  // all converters agree
-                    widen_chunk(sraw + f8_a_off(it.stream, c), slots + cslot * kF8SlotBytes, ct);
-                    fence_proxy_async_smem();  // generic-proxy writes -> the MMA's async reads
-                    named_bar_sync(2, kF8CvtThreads);
-                    if (ct == 0) mbar_arrive(&sh.cvt_full[cslot]);
-                    if (++cslot == kF8Slots) { cslot = 0; cphase ^= 1u; }
-                }
-                if (!ok) break;
-                if (ct == 0) mbar_arrive(&sh.raw_empty[stage]);  // the codes are read
-                if (++stage == kF8RawStages) { stage = 0; phase ^= 1u; }
+                const bool mine = mbar_wait(&sh.full[stage], phase, abort);
+                unsigned char *sbase = stages + stage * kF8StageBytes;
+                ok = nch == 2 ? widen_in_place<2>(sbase, it.stream, ct, mine)
+                              : widen_in_place<1>(sbase, it.stream, ct, mine);
+                if (!ok) break;  // every converter takes the same decision
+                fence_proxy_async_smem();  // generic-proxy writes -> the MMA's async reads
+                named_bar_sync(2, kF8CvtThreads);
+                if (ct == 0) mbar_arrive(&sh.wide[stage]);
+                if (++stage == kF8Stages) { stage = 0; phase ^= 1u; }
             }
             if (!ok) break;
         }
@@ -422,6 +520,7 @@ __global__ void __launch_bounds__(kF8Threads, 1) ffn_fp8_kernel(
                 int q = -1;
                 if (mbar_wait(&sh.slot_full[slot], (uint32_t)(s / kSlots) & 1u, abort)) {
                     q = sh.slot_item[slot];
+                    if (q < total) sh.epi_it = sh.slot_it[slot];
                     mbar_arrive(&sh.slot_empty[slot]);
                     if (q < total && !mbar_wait(&sh.tfull[s & 1], (uint32_t)(s >> 1) & 1u, abort))
                         q = -1;
@@ -430,11 +529,10 @@ __global__ void __launch_bounds__(kF8Threads, 1) ffn_fp8_kernel(
             }
             named_bar_sync(1, 128);
             const int q = *(volatile int *)&sh.epi_item;
-            named_bar_sync(1, 128);
             if (q < 0 || q >= total) break;
+            const TcItem it = sh.epi_it;
+            named_bar_sync(1, 128);
             tc_fence_after();
-            TcItem it;
-            decode_item(tp, tot_up, q, it);
             const int acc = s & 1;
             const uint32_t tbase = tmem_base + ((uint32_t)(32 * q4) << 16) + (uint32_t)acc * 256u;
             const size_t row0 = (size_t)it.w.dst_row0 + (size_t)it.tb * it.w.bn;
@@ -560,9 +658,26 @@ static int encode_codes_gate_up(CUtensorMap *m, const void *gate, const void *up
     return encode_u8(m, base, 4, dims, strides, box) ? mode : kGateUpSplit;
 }
 
+// Streaming stages fetch both K-chunks' codes of a weight row as one 128-byte
+// segment (boxes of 128 codes x rows); rows of the box keep the global layout
+// (no swizzle), chunk c being bytes 64 c .. 64 c + 63 of each row.
+static bool encode_codes_wide(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows,
+                              uint64_t experts, uint32_t box_rows) {
+    const cuuint64_t dims[3] = {cols, rows, experts};
+    const cuuint64_t strides[2] = {cols, cols * rows};
+    const cuuint32_t box[3] = {(cuuint32_t)(2 * kChunkK), box_rows, 1};
+    return encode_u8(m, base, 3, dims, strides, box);
+}
+static bool encode_codes_gate_up_wide(CUtensorMap *m, const void *base, uint64_t cols,
+                                      uint64_t rows, uint64_t experts, uint64_t step) {
+    const cuuint64_t dims[4] = {cols, rows, experts, 2};
+    const cuuint64_t strides[3] = {cols, cols * rows, step};
+    const cuuint32_t box[4] = {(cuuint32_t)(2 * kChunkK), 64, 1, 2};
+    return encode_u8(m, base, 4, dims, strides, box);
+}
+
 static size_t f8_smem_bytes() {
-    return 1024 + (size_t)kF8RawStages * kF8RawBytes + (size_t)kF8Slots * kF8SlotBytes +
-           kF8EpiBytes + sizeof(F8Shared);
+    return 1024 + (size_t)kF8Stages * kF8StageBytes + kF8EpiBytes + sizeof(F8Shared);
 }
 
 cudaError_t launch_ffn_fp8(const moge_config &c, const Plan &plan, int n_entries,
@@ -609,12 +724,28 @@ cudaError_t launch_ffn_fp8(const moge_config &c, const Plan &plan, int n_entries
     p.sc_g[0] = wgs; p.sc_u[0] = wus; p.sc_d[0] = wds;
     p.sc_g[1] = sgs; p.sc_u[1] = sus; p.sc_d[1] = sds;
 
+    // maps of the streaming stages: two K-chunks of codes per weight row
+    CUtensorMap mWg2, mWu2, mSg2, mSu2, mWd2, mSd2;
+    auto wide_gu = [&](CUtensorMap *g2, CUtensorMap *u2, int mode, const void *g, const void *u,
+                       int ex) -> bool {
+        if (mode == kGateUpSplit)
+            return encode_codes_wide(g2, g, d, I, ex, 64) && encode_codes_wide(u2, u, d, I, ex, 64);
+        const char *lo = static_cast<const char *>(mode == kGateUpFused ? g : u);
+        const char *hi = static_cast<const char *>(mode == kGateUpFused ? u : g);
+        if (!encode_codes_gate_up_wide(g2, lo, d, I, ex, (uint64_t)(hi - lo))) return false;
+        *u2 = *g2;
+        return true;
+    };
+    if (!wide_gu(&mWg2, &mWu2, t.gu_mode[0], wg, wu, ne) ||
+        !wide_gu(&mSg2, &mSu2, t.gu_mode[1], sg, su, ns) ||
+        !encode_codes_wide(&mWd2, wd, I, d, ne, 128) || !encode_codes_wide(&mSd2, sd, I, d, ns, 128))
+        return cudaErrorInvalidValue;
     const size_t smem = f8_smem_bytes();
     cudaError_t e = cudaFuncSetAttribute(ffn_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
     return launch_pdl(ffn_fp8_kernel, dim3(num_sms), dim3(kF8Threads), smem, st, p, mWg, mWu, mSg,
-                      mSu, mX0, mX1, mWd, mSd, mH);
+                      mSu, mX0, mX1, mWd, mSd, mH, mWg2, mWu2, mSg2, mSu2, mWd2, mSd2);
 }
 
 }  // namespace moge

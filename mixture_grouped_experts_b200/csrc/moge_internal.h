@@ -92,9 +92,10 @@ cudaError_t launch_router(const moge_config &c, const void *x, const void *w_rou
                           const float *bias, int32_t *topk_idx, float *topk_w, int32_t *hist,
                           int32_t *rank, int num_sms, cudaStream_t st);
 // counts/offsets/base from hist; when plan_* are given also the layer's GEMM plan
+// (token tiles of the plan: at most max_tile rows each)
 cudaError_t launch_scan(const moge_config &c, const int32_t *hist, int32_t *base, int32_t *counts,
                         int32_t *offsets, const Plan *plan, bool with_routed, bool with_shared,
-                        cudaStream_t st);
+                        cudaStream_t st, int max_tile = kMaxTileN);
 // plan from caller offsets (routed only) or for shared experts only
 cudaError_t launch_plan(const moge_config &c, const int32_t *offsets, const Plan &plan,
                         bool with_routed, bool with_shared, cudaStream_t st);

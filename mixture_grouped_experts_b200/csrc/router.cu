@@ -462,12 +462,13 @@ __device__ int block_exclusive_scan_1024(int v, int *wbuf /* [32] */, int *total
 // then routed experts 0..N-1 (if with_routed, rows from offs[]). The grouped
 // FFN hands its work out in this order, so the heavy shared-expert items come
 // first. Token-tile width: <= kStreamRows rows -> one streaming tile of
-// round16(rows); more -> ceil(rows / 256) balanced tiles of round16 width.
+// round16(rows); more -> ceil(rows / max_tile) balanced tiles of round16 width
+// (never above max_tile, a multiple of 16).
 // Also zeroes the FFN's work-queue counter and per-entry completion counters.
 // Called by all 1024 threads of the block.
 __device__ void build_plan_block(const moge_config &c, const int32_t *offs, Plan plan,
                                  bool with_routed, bool with_shared, int shared_row_base,
-                                 int *wbuf) {
+                                 int max_tile, int *wbuf) {
     const int fb_up = (c.I + 63) / 64;      // 64 gate + 64 up rows per tile
     const int fb_down = (c.d + 127) / 128;  // 128 output features per tile
     const int ns = with_shared ? c.S : 0;
@@ -492,7 +493,7 @@ __device__ void build_plan_block(const moge_config &c, const int32_t *offs, Plan
         } else if (rows <= kStreamRows) {
             bn = (rows + 15) & ~15; ntb = 1;
         } else {
-            const int nt = (rows + kMaxTileN - 1) / kMaxTileN;
+            const int nt = (rows + max_tile - 1) / max_tile;
             bn = (((rows + nt - 1) / nt) + 15) & ~15;
             ntb = (rows + bn - 1) / bn;
         }
@@ -527,7 +528,8 @@ __device__ void build_plan_block(const moge_config &c, const int32_t *offs, Plan
 __global__ void __launch_bounds__(1024) scan_kernel(moge_config c, const int32_t *__restrict__ hist,
                                                      int32_t *base, int32_t *counts,
                                                      int32_t *offsets, Plan plan, int make_plan,
-                                                     int with_routed, int with_shared) {
+                                                     int with_routed, int with_shared,
+                                                     int max_tile) {
     __shared__ int32_t part[1024];
     __shared__ int32_t cnt_s[kMaxExperts];
     __shared__ int32_t off_s[kMaxExperts + 1];
@@ -581,16 +583,17 @@ __global__ void __launch_bounds__(1024) scan_kernel(moge_config c, const int32_t
     }
     if (make_plan) {
         __syncthreads();
-        build_plan_block(c, off_s, plan, with_routed != 0, with_shared != 0, c.T * c.M * c.Kp, wbuf);
+        build_plan_block(c, off_s, plan, with_routed != 0, with_shared != 0, c.T * c.M * c.Kp,
+                         max_tile, wbuf);
     }
 }
 
 cudaError_t launch_scan(const moge_config &c, const int32_t *hist, int32_t *base, int32_t *counts,
                         int32_t *offsets, const Plan *plan, bool with_routed, bool with_shared,
-                        cudaStream_t st) {
+                        cudaStream_t st, int max_tile) {
     Plan p = plan ? *plan : Plan{nullptr, nullptr, nullptr, nullptr};
     return launch_pdl(scan_kernel, dim3(1), dim3(1024), 0, st, c, hist, base, counts, offsets, p,
-                      plan ? 1 : 0, with_routed ? 1 : 0, with_shared ? 1 : 0);
+                      plan ? 1 : 0, with_routed ? 1 : 0, with_shared ? 1 : 0, max_tile);
 }
 
 // Plan from the caller's offsets (routed only) or for the shared experts only.
@@ -603,7 +606,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(moge_config c, const int32_t
         for (int i = threadIdx.x; i <= c.N; i += blockDim.x) off_s[i] = offsets[i];
     __syncthreads();
     build_plan_block(c, off_s, plan, with_routed != 0, with_shared != 0,
-                     with_routed ? c.T * c.M * c.Kp : 0, wbuf);
+                     with_routed ? c.T * c.M * c.Kp : 0, kMaxTileN, wbuf);
 }
 
 cudaError_t launch_plan(const moge_config &c, const int32_t *offsets, const Plan &plan,
