@@ -446,34 +446,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
 
 // ---------------------------------------------------------------------------
 // Host side: tensor maps and the launch.
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn get_encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    }
-    return fn;
-}
-
-static bool encode(CUtensorMap *m, const void *base, cuuint32_t rank, const cuuint64_t *dims,
-                   const cuuint64_t *strides, const cuuint32_t *box) {
-    EncodeTiledFn fn = get_encode_fn();
-    if (!fn) return false;
-    const cuuint32_t estr[4] = {1, 1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), dims, strides,
-              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // bf16 [experts][rows][cols] weights, box = [box_rows][64 cols] of one expert
 static bool encode_weights(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows,
                            uint64_t experts, uint32_t box_rows) {

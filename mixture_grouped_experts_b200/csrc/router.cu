@@ -158,166 +158,139 @@ __device__ void router_epilogue(const RouterView &sm, const moge_config &c, cons
 }
 
 // ---------------------------------------------------------------------------
-// bf16 router GEMM with mma.sync m16n8k16 (the N <= 256 output columns are far
-// too narrow for a tcgen05 tile to pay). One CTA owns a tile of TB = 16*TBM
+// bf16 router GEMM on the tensor cores. One CTA owns a tile of TB = 16*TBM
 // tokens and a slice of the hidden dimension; a cluster of `ks` CTAs splits
 // the hidden dimension of one tile and the leader adds the partial logits in
-// rank order (deterministic). The CTA copies its x rows and router rows block
-// by block into shared memory with cp.async, NST blocks in flight; warp w owns
-// the n-tiles w, w+8, ... (8 experts each), so no reduction across warps is
-// needed. Long batches use 64-token tiles, which read the router matrix a
-// quarter as often.
-//
-// k-slot mapping: for each 32-wide chunk of the hidden dimension, the thread
-// with quad index q reads hidden elements [8q, 8q+8) of its A rows and of its
-// B rows and feeds them to two m16n8k16 steps as the k-slots {2q, 2q+1,
-// 2q+8, 2q+9}. A and B use the same mapping, so every product pairs equal
-// hidden indices; the sum over the chunk is unchanged.
-constexpr int kRouterStageBytes = 40 * 1024;
+// rank order (deterministic). Thread 0 streams the slice through a ring of
+// `nst` stages with TMA, one 64-wide K-chunk per stage: a box of TB token rows
+// and a box of 128 (or 256) router rows, rows past N arriving as zeros, both
+// 128-byte swizzled. Thread 32 issues tcgen05.mma with the router rows as A
+// (M = 128 per half) and the token rows as B (N = TB), fp32 accumulation in
+// tensor memory, and frees each stage with tcgen05.commit. The accumulator
+// D[expert][token] then goes to shared memory as logits [token][expert] for
+// the epilogue. (The warp-level mma.sync path it replaces was bound by that
+// instruction's low issue rate on this architecture.) Long batches use
+// 64-token tiles, which read the router matrix a quarter as often.
 
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                               uint32_t a3, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
+constexpr int kRouterChunk = 64;      // hidden elements per stage (128 bytes per row)
+constexpr int kRouterMaxStages = 12;
 
-// 16-byte async copy global -> shared; src_bytes = 0 fills zeros.
-__device__ __forceinline__ void cp_async_16(void *dst, const void *src, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
-                 "r"(src_bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_pending(int n) {
-    // wait until at most n copy groups are outstanding (n < 4)
-    if (n <= 0) asm volatile("cp.async.wait_group 0;" ::: "memory");
-    else if (n == 1) asm volatile("cp.async.wait_group 1;" ::: "memory");
-    else if (n == 2) asm volatile("cp.async.wait_group 2;" ::: "memory");
-    else asm volatile("cp.async.wait_group 3;" ::: "memory");
-}
+// bytes of one stage: TB token rows and N router rows of 128 bytes (a
+// multiple of 1024 since TB % 16 == 0 and N % 8 == 0)
+__host__ __device__ inline int router_stage_bytes(int tb, int n) { return (tb + n) * 128; }
 
-// hidden elements per staged block for a tile of tb tokens and N experts
-// (multiple of 32, >= 32): (tb + N) rows of (2*LB + 64) bytes fit one stage
-__host__ __device__ inline int router_block_len(int N, int tb) {
-    int lb = ((kRouterStageBytes / (tb + N) - 64) / 2) & ~31;
-    if (lb >= 64) lb &= ~63;
-    return lb < 32 ? 32 : lb;
-}
-
-template <int TBM, int NST>
-__global__ void __launch_bounds__(kRouterThreads, (NST <= 2 ? 2 : 1)) router_bf16_kernel(
-    moge_config c, const uint16_t *__restrict__ x, const uint16_t *__restrict__ wr,
+template <int TBM>
+__global__ void __launch_bounds__(kRouterThreads, TBM == 1 ? 2 : 1) router_bf16_kernel(
+    moge_config c, const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
     const float *__restrict__ bias, int32_t *topk_idx, float *topk_w, int32_t *hist, int32_t *rank,
-    int ks) {
+    int ks, int nst) {
     constexpr int TB = kRouterTile * TBM;
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    unsigned char *stage = smem_raw;  // [NST][kRouterStageBytes]
+    extern __shared__ __align__(1024) unsigned char smem_dyn[];
+    __shared__ uint64_t full[kRouterMaxStages], empty[kRouterMaxStages], done;
+    __shared__ uint32_t tmem_base;
+    __shared__ int abort_flag;
+    unsigned char *stage = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    const int N = c.N;
+    const int mh = N <= 128 ? 1 : 2;                 // 128-row halves of the router matrix
+    const int sbytes = router_stage_bytes(TB, 128 * mh);
     RouterView sm;
-    sm.logits = reinterpret_cast<float *>(smem_raw + NST * kRouterStageBytes);
-    sm.ids = reinterpret_cast<int16_t *>(sm.logits + TB * c.N);
+    sm.logits = reinterpret_cast<float *>(stage + (size_t)nst * sbytes);
+    sm.ids = reinterpret_cast<int16_t *>(sm.logits + TB * N);
     sm.tb = TB;
-    grid_dependency_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g = lane >> 2, q = lane & 3;
     const int crank = blockIdx.x % ks;
     const int t0 = (blockIdx.x / ks) * TB;
-    const int d = c.d, N = c.N;
-    const int LB = router_block_len(N, TB);
-    const int pitch = 2 * LB + 64;  // bytes per staged row (64 B pad: conflict-free 16-byte loads)
-    const int rows = TB + N;
-    // this CTA's slice of the hidden dimension, in whole 32-element chunks
-    const int nchunk = (d + 31) / 32;
-    const int kb = 32 * (int)((long long)nchunk * crank / ks);
-    const int ke = min(d, 32 * (int)((long long)nchunk * (crank + 1) / ks));
-    const int nblk = (ke - kb + LB - 1) / LB;
-    const int vpr = LB / 8;  // 16-byte vectors per staged row
-
-    // warp w copies rows w, w+8, ...; lane l copies 16-byte vectors l, l+32, ... of a row
-    auto load_block = [&](int b, unsigned char *dst) {
-        const int k0 = kb + b * LB;
-        for (int r = warp; r < rows; r += kRouterWarps) {
-            bool row_ok = true;
-            const uint16_t *src_row;
-            if (r < TB) {
-                row_ok = (t0 + r) < c.T;
-                src_row = x + (size_t)(row_ok ? t0 + r : 0) * d;
-            } else {
-                src_row = wr + (size_t)(r - TB) * d;
-            }
-            unsigned char *dst_row = dst + (size_t)r * pitch;
-            for (int v = lane; v < vpr; v += 32) {
-                const int k = k0 + 8 * v;
-                const bool ok = row_ok && k < ke;
-                cp_async_16(dst_row + 16 * v, src_row + (ok ? k : 0), ok ? 16u : 0u);
-            }
+    // this CTA's slice of the hidden dimension, in whole chunks
+    const int nck = (c.d + kRouterChunk - 1) / kRouterChunk;
+    const int cb = (int)((long long)nck * crank / ks), ce = (int)((long long)nck * (crank + 1) / ks);
+    const int nc = ce - cb;
+    // accumulator columns: half h at h * hs (hs >= 32, so every 32-column read
+    // below stays inside the allocation), allocation a power of two >= 32
+    constexpr int hs = TB < 32 ? 32 : TB;
+    uint32_t tcols = 32;
+    while (tcols < (uint32_t)(hs * mh)) tcols <<= 1;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < nst; ++s) {
+            mbar_init(&full[s], 1);   // the producer's expect_tx arrival (+ the copies' bytes)
+            mbar_init(&empty[s], 1);  // the MMA thread's commit
         }
-        cp_async_commit();
-    };
-
-    float acc[TBM][4][4];
-#pragma unroll
-    for (int m = 0; m < TBM; ++m)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[m][i][0] = acc[m][i][1] = acc[m][i][2] = acc[m][i][3] = 0.0f;
-    const int ntiles = N / 8;
-    // tiles start at different blocks of their slice, so concurrently running
-    // CTAs do not all read the same router rows at the same time
-    const int rot = nblk > 0 ? (blockIdx.x / ks) % nblk : 0;
-    for (int i = 0; i < NST - 1 && i < nblk; ++i)
-        load_block((i + rot) % nblk, stage + i * kRouterStageBytes);
-    for (int i = 0; i < nblk; ++i) {
-        const int b = (i + rot) % nblk;
-        if (i + NST - 1 < nblk) {
-            load_block((i + NST - 1 + rot) % nblk, stage + ((i + NST - 1) % NST) * kRouterStageBytes);
-            cp_async_wait_pending(NST - 1);
-        } else {
-            cp_async_wait_pending(nblk - 1 - i);
-        }
-        __syncthreads();
-        const unsigned char *st = stage + (i % NST) * kRouterStageBytes;
-        const int len = min(LB, ke - (kb + b * LB));
-        for (int ch = 0; ch < (len + 31) / 32; ++ch) {
-            const int off = 64 * ch + 16 * q;  // bytes into the row
-            uint4 a_lo[TBM], a_hi[TBM];
-#pragma unroll
-            for (int m = 0; m < TBM; ++m) {
-                a_lo[m] = *reinterpret_cast<const uint4 *>(st + (size_t)(16 * m + g) * pitch + off);
-                a_hi[m] = *reinterpret_cast<const uint4 *>(st + (size_t)(16 * m + g + 8) * pitch + off);
-            }
-#pragma unroll
-            for (int i2 = 0; i2 < 4; ++i2) {
-                const int nt = warp + 8 * i2;
-                if (nt < ntiles) {
-                    const uint4 wv = *reinterpret_cast<const uint4 *>(
-                        st + (size_t)(TB + nt * 8 + g) * pitch + off);
-#pragma unroll
-                    for (int m = 0; m < TBM; ++m) {
-                        mma_bf16_16816(acc[m][i2], a_lo[m].x, a_hi[m].x, a_lo[m].y, a_hi[m].y, wv.x, wv.y);
-                        mma_bf16_16816(acc[m][i2], a_lo[m].z, a_hi[m].z, a_lo[m].w, a_hi[m].w, wv.z, wv.w);
-                    }
-                }
-            }
-        }
-        __syncthreads();  // this stage is refilled NST blocks later
+        mbar_init(&done, 1);
+        abort_flag = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&tmX);
+        tma_prefetch_desc(&tmW);
     }
-#pragma unroll
-    for (int m = 0; m < TBM; ++m)
-#pragma unroll
-        for (int i2 = 0; i2 < 4; ++i2) {
-            const int nt = warp + 8 * i2;
-            if (nt < ntiles) {
-                float *r0 = sm.logits + (size_t)(16 * m + g) * N + nt * 8 + 2 * q;
-                float *r1 = sm.logits + (size_t)(16 * m + g + 8) * N + nt * 8 + 2 * q;
-                r0[0] = acc[m][i2][0];
-                r0[1] = acc[m][i2][1];
-                r1[0] = acc[m][i2][2];
-                r1[1] = acc[m][i2][3];
+    if (warp == 0) {
+        tmem_alloc(&tmem_base, tcols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = tmem_base;
+    grid_dependency_wait();
+    volatile int *abort = &abort_flag;
+
+    if (threadIdx.x == 0) {
+        // ---- producer: chunk i of the slice into stage i % nst, a box of TB
+        // token rows then the router rows (rows past T and past N come as zeros)
+        const uint64_t pol_x = policy_evict_first(), pol_w = policy_evict_last();
+        int issued = 0;
+        for (; issued < nc; ++issued) {
+            const int s = issued % nst;
+            if (issued >= nst && !mbar_wait(&empty[s], (uint32_t)(issued / nst - 1) & 1u, abort)) break;
+            unsigned char *st = stage + (size_t)s * sbytes;
+            mbar_arrive_expect_tx(&full[s], (uint32_t)sbytes);
+            tma_load_2d(st, &tmX, &full[s], (cb + issued) * kRouterChunk, t0, pol_x);
+            tma_load_2d(st + TB * 128, &tmW, &full[s], (cb + issued) * kRouterChunk, 0, pol_w);
+        }
+        if (*abort) {  // let the copies in flight land before the stages are reused
+            for (int s = 0; s < nst && s < issued; ++s) {
+                const int last = issued - 1 - ((issued - 1 - s) % nst);
+                mbar_wait(&full[s], (uint32_t)(last / nst) & 1u, nullptr);
             }
         }
+    } else if (threadIdx.x == 32) {
+        // ---- MMA issuer: D[expert][token] += W_chunk * x_chunk^T, M = 128 per half
+        const uint32_t idesc = idesc_bf16_f32(128, (uint32_t)TB);
+        for (int i = 0; i < nc; ++i) {
+            const int s = i % nst;
+            if (!mbar_wait(&full[s], (uint32_t)(i / nst) & 1u, abort)) break;
+            tc_fence_after();
+            const uint32_t sb = smem_u32(stage + (size_t)s * sbytes);
+            for (int h = 0; h < mh; ++h)
+#pragma unroll
+                for (int j = 0; j < kRouterChunk / 16; ++j)  // 16-wide K steps: +32 bytes
+                    tc_mma_bf16(tm + (uint32_t)(h * hs), smem_desc_sw128(sb + TB * 128 + h * 16384 + 32 * j),
+                                smem_desc_sw128(sb + 32 * j), idesc, (i | j) > 0 ? 1u : 0u);
+            tc_commit(&empty[s]);  // the stage may be refilled once these MMAs have read it
+        }
+        tc_commit(&done);  // every MMA of this CTA has completed after this
+    }
+    // ---- everyone: the accumulator is final; TMEM -> logits [token][expert]
+    const bool ok = mbar_wait(&done, 0u, nullptr) && !*abort;
     __syncthreads();
+    tc_fence_after();
+    {
+        const int q4 = warp & 3, wg = warp >> 2;   // TMEM lane quarter, warp group
+        const int ncb = (TB + 31) / 32;            // 32-column blocks per half
+        for (int idx = wg; idx < mh * ncb; idx += 2) {
+            const int h = idx / ncb, c0 = (idx % ncb) * 32;
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(tm + ((uint32_t)(32 * q4) << 16) + (uint32_t)(h * hs + c0), v);
+            tmem_ld_wait();
+            const int e = h * 128 + 32 * q4 + lane;
+            if (e < N) {
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj)
+                    if (c0 + jj < TB) sm.logits[(size_t)(c0 + jj) * N + e] = ok ? __uint_as_float(v[jj]) : 0.0f;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tm, tcols);  // before any CTA of the cluster returns
 
     if (ks > 1) {
         // peers push their partial logits into the leader's (now idle) stage
@@ -368,24 +341,44 @@ __global__ void __launch_bounds__(kRouterThreads) router_f32_kernel(
     router_epilogue(sm, c, bias, t0, topk_idx, topk_w, hist, rank);
 }
 
-template <int TBM, int NST>
+template <int TBM>
 static cudaError_t launch_router_bf16(const moge_config &c, const void *x, const void *w_router,
                                       const float *bias, int32_t *topk_idx, float *topk_w,
                                       int32_t *hist, int32_t *rank, int num_sms, cudaStream_t st) {
     constexpr int TB = kRouterTile * TBM;
     const int tiles = (c.T + TB - 1) / TB;
-    const int per_sm = NST <= 2 ? 2 : 1;
+    const int per_sm = TBM == 1 ? 2 : 1;
+    const int mh = c.N <= 128 ? 1 : 2;  // the router box is 128 (or 256) rows, zero past N
+    const int sb = router_stage_bytes(TB, 128 * mh);
+    // as many stages as the CTA's shared-memory budget holds (two CTAs per SM
+    // with 16-token tiles, one with 64-token tiles)
+    const size_t fixed = 1024 + (size_t)TB * c.N * 4 + (size_t)TB * c.M * c.Kp * 2;
+    const size_t budget = TBM == 1 ? 100 * 1024 : 200 * 1024;
+    int nst = budget > fixed ? (int)((budget - fixed) / sb) : 0;
+    nst = nst > kRouterMaxStages ? kRouterMaxStages : nst < 2 ? 2 : nst;
     // Split the hidden dimension over a cluster of up to 8 CTAs while the grid
-    // stays within one wave, each CTA keeps >= 2 blocks of work, and the
-    // leader's landing buffer (its stages) holds the (ks - 1) partial tiles.
-    const int lb = router_block_len(c.N, TB);
+    // stays within one wave, each CTA keeps >= 2 chunks, and the leader's
+    // landing buffer (its stages) holds the (ks - 1) partial tiles.
+    const int nck = (c.d + kRouterChunk - 1) / kRouterChunk;
     int ks = 1;
-    while (ks < 8 && tiles * ks * 2 <= per_sm * num_sms && c.d >= ks * 2 * 2 * lb &&
-           (size_t)(2 * ks - 1) * TB * c.N * 4 <= (size_t)NST * kRouterStageBytes)
+    while (ks < 8 && tiles * 2 * ks <= per_sm * num_sms && nck >= 2 * 2 * ks &&
+           (size_t)(2 * ks - 1) * TB * c.N * 4 <= (size_t)nst * sb)
         ks *= 2;
-    const size_t smem = (size_t)NST * kRouterStageBytes + (size_t)TB * c.N * 4 +
-                        (size_t)TB * c.M * c.Kp * 2;
-    auto kern = router_bf16_kernel<TBM, NST>;
+    CUtensorMap mX, mW;
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)c.d, (cuuint64_t)c.T};
+        const cuuint64_t strides[1] = {(cuuint64_t)c.d * 2};
+        const cuuint32_t box[2] = {(cuuint32_t)kRouterChunk, (cuuint32_t)TB};
+        if (!encode(&mX, x, 2, dims, strides, box)) return cudaErrorInvalidValue;
+    }
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)c.d, (cuuint64_t)c.N};
+        const cuuint64_t strides[1] = {(cuuint64_t)c.d * 2};
+        const cuuint32_t box[2] = {(cuuint32_t)kRouterChunk, (cuuint32_t)(128 * mh)};
+        if (!encode(&mW, w_router, 2, dims, strides, box)) return cudaErrorInvalidValue;
+    }
+    const size_t smem = fixed + (size_t)nst * sb;
+    auto kern = router_bf16_kernel<TBM>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -402,8 +395,7 @@ static cudaError_t launch_router_bf16(const moge_config &c, const void *x, const
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, kern, c, (const uint16_t *)x, (const uint16_t *)w_router, bias,
-                              topk_idx, topk_w, hist, rank, ks);
+    return cudaLaunchKernelEx(&cfg, kern, c, mX, mW, bias, topk_idx, topk_w, hist, rank, ks, nst);
 }
 
 cudaError_t launch_router(const moge_config &c, const void *x, const void *w_router,
@@ -419,12 +411,12 @@ cudaError_t launch_router(const moge_config &c, const void *x, const void *w_rou
                           (const float *)x, (const float *)w_router, bias, topk_idx, topk_w, hist,
                           rank);
     }
-    // long batches with few experts: 64-token tiles, four blocks in flight
-    // (one CTA per SM); otherwise 16-token tiles, two blocks in flight (two
-    // CTAs per SM, up to 8-CTA clusters over the hidden dimension)
+    // long batches with few experts: 64-token tiles (one CTA per SM);
+    // otherwise 16-token tiles (two CTAs per SM, up to 8-CTA clusters over the
+    // hidden dimension)
     if (c.N <= 64 && c.T >= 1024)
-        return launch_router_bf16<4, 4>(c, x, w_router, bias, topk_idx, topk_w, hist, rank, num_sms, st);
-    return launch_router_bf16<1, 2>(c, x, w_router, bias, topk_idx, topk_w, hist, rank, num_sms, st);
+        return launch_router_bf16<4>(c, x, w_router, bias, topk_idx, topk_w, hist, rank, num_sms, st);
+    return launch_router_bf16<1>(c, x, w_router, bias, topk_idx, topk_w, hist, rank, num_sms, st);
 }
 
 // ---------------------------------------------------------------------------

@@ -26,6 +26,8 @@ CASES = {
     "t17": MED.replace(name="t17", T=17, seed=16),                        # ragged router tile
     "s0": MED.replace(name="s0", T=50, S=0, seed=17),                     # no shared expert
     "big": MED.replace(name="big", T=1100, N=8, M=2, S=1, seed=18),       # > 256 rows per expert
+    "n256": MED.replace(name="n256", T=70, N=256, M=8, seed=41),          # router in two 128-row halves
+    "n160": MED.replace(name="n160", T=45, N=160, M=8, seed=42),          # groups of 20 (no shuffle path)
 }
 
 
