@@ -34,10 +34,92 @@ __device__ __forceinline__ bool ranks_before(float pa, int a, float pb, int b) {
     return pa > pb || (pa == pb && a < b);
 }
 
+// Lane-per-group epilogue (M a power of two <= 32, groups of G = 8, 16 or 32
+// experts, Kp <= 2): a token takes M consecutive lanes, lane g of its segment
+// holding the G scores of group g in registers, so a warp works on 32 / M
+// tokens at once; max and sum need log2(M) shuffle steps, the in-group top-Kp
+// is a scan of registers. Histogram and ranks of every 16-token sub-tile then
+// come from one warp per (sub-tile, group): its lanes hold the sub-tile's
+// picks in that group, __match_any_sync groups equal experts (rank = equal
+// picks of earlier tokens, ascending tokens), one ballot per expert counts.
+template <int G>
+__device__ void router_epilogue_lanes(const RouterView &sm, const moge_config &c, const float *bias,
+                                      int t0, int32_t *topk_idx, float *topk_w, int32_t *hist,
+                                      int32_t *rank) {
+    const int N = c.N, M = c.M, Kp = c.Kp, K = M * Kp;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nwarps = blockDim.x >> 5;
+    const int ntok = min(sm.tb, c.T - t0);
+    const int per_warp = 32 / M;  // tokens a warp handles at once
+    const int g = lane % M, seg = lane / M;
+    for (int tb0 = warp * per_warp; tb0 < ntok; tb0 += nwarps * per_warp) {
+        const int tt = tb0 + seg;
+        const bool live = tt < ntok;
+        float v[G];
+        float m = -INFINITY;
+        const float *lg = sm.logits + (size_t)(live ? tt : 0) * N + g * G;
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+            v[j] = lg[j] + (bias ? bias[g * G + j] : 0.0f);
+            m = fmaxf(m, v[j]);
+        }
+        for (int o = M >> 1; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        float z = 0.0f;
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+            v[j] = expf(v[j] - m);
+            z += v[j];
+        }
+        for (int o = M >> 1; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+#pragma unroll
+        for (int j = 0; j < G; ++j) v[j] = v[j] / z;
+        int prev = -1;
+        for (int k = 0; k < Kp; ++k) {
+            int best = -1;
+            float pb = 0.0f;
+#pragma unroll
+            for (int j = 0; j < G; ++j) {  // Kp <= 2: the second pick skips the first
+                if (j == prev) continue;
+                if (best < 0 || ranks_before(v[j], j, pb, best)) { best = j; pb = v[j]; }
+            }
+            if (live) {
+                const int e = g * G + best;
+                const size_t o = (size_t)(t0 + tt) * K + g * Kp + k;
+                topk_idx[o] = e;
+                topk_w[o] = pb;
+                sm.ids[(size_t)tt * K + g * Kp + k] = (int16_t)e;
+            }
+            prev = best;
+        }
+    }
+    __syncthreads();
+    const int nsub = (ntok + kRouterTile - 1) / kRouterTile;
+    for (int pr = warp; pr < nsub * M; pr += nwarps) {
+        const int sub = pr / M, gg = pr % M;
+        const int tl = lane / Kp, j = lane % Kp;       // token in the sub-tile, pick
+        const int tt = sub * kRouterTile + tl;
+        const bool valid = lane < kRouterTile * Kp && tt < ntok;
+        const int e = valid ? (int)sm.ids[(size_t)tt * K + gg * Kp + j] : -1 - lane;
+        const unsigned same = __match_any_sync(0xffffffffu, e);
+        if (valid) rank[(size_t)(t0 + tt) * K + gg * Kp + j] = __popc(same & ((1u << (tl * Kp)) - 1u));
+        int cnt = 0;
+        for (int x = 0; x < G; ++x) {
+            const int n = __popc(__ballot_sync(0xffffffffu, e == gg * G + x));
+            if (lane == x) cnt = n;
+        }
+        if (lane < G) hist[(size_t)(t0 / kRouterTile + sub) * N + gg * G + lane] = cnt;
+    }
+}
+
 __device__ void router_epilogue(const RouterView &sm, const moge_config &c, const float *bias,
                                 int t0, int32_t *topk_idx, float *topk_w, int32_t *hist,
                                 int32_t *rank) {
     const int N = c.N, M = c.M, Kp = c.Kp, K = M * Kp, G = N / M;
+    if (M <= 32 && 32 % M == 0 && Kp <= 2) {
+        if (G == 8) return router_epilogue_lanes<8>(sm, c, bias, t0, topk_idx, topk_w, hist, rank);
+        if (G == 16) return router_epilogue_lanes<16>(sm, c, bias, t0, topk_idx, topk_w, hist, rank);
+        if (G == 32) return router_epilogue_lanes<32>(sm, c, bias, t0, topk_idx, topk_w, hist, rank);
+    }
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nwarps = blockDim.x >> 5;
     const int ntok = min(sm.tb, c.T - t0);
@@ -232,6 +314,9 @@ __global__ void __launch_bounds__(kRouterThreads, TBM == 1 ? 2 : 1) router_bf16_
     grid_dependency_wait();
     volatile int *abort = &abort_flag;
 
+    // Lane 0 of warp 0 produces and lane 0 of warp 1 issues the MMAs; the other
+    // lanes of those two warps wait at __syncwarp (parked, not polling), so the
+    // working lane does not share its warp's issue slots with a wait loop.
     if (threadIdx.x == 0) {
         // ---- producer: chunk i of the slice into stage i % nst, a box of TB
         // token rows then the router rows (rows past T and past N come as zeros)
@@ -268,6 +353,7 @@ __global__ void __launch_bounds__(kRouterThreads, TBM == 1 ? 2 : 1) router_bf16_
         }
         tc_commit(&done);  // every MMA of this CTA has completed after this
     }
+    if (warp < 2) __syncwarp();
     // ---- everyone: the accumulator is final; TMEM -> logits [token][expert]
     const bool ok = mbar_wait(&done, 0u, nullptr) && !*abort;
     __syncthreads();

@@ -28,6 +28,7 @@ CASES = {
     "big": MED.replace(name="big", T=1100, N=8, M=2, S=1, seed=18),       # > 256 rows per expert
     "n256": MED.replace(name="n256", T=70, N=256, M=8, seed=41),          # router in two 128-row halves
     "n160": MED.replace(name="n160", T=45, N=160, M=8, seed=42),          # groups of 20 (no shuffle path)
+    "kp2g8": MED.replace(name="kp2g8", T=120, N=32, M=4, Kp=2, seed=43),  # lane-per-group path, 2 picks
 }
 
 
