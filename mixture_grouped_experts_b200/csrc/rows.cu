@@ -14,12 +14,16 @@
 namespace moge {
 
 constexpr int kRowThreads = 128;
+// The layer's scatter spreads one token's row over several CTAs of
+// kVecThreads threads, one 8-element vector (16 bytes in bf16) per thread.
+constexpr int kVecThreads = 256;
 
-__device__ __forceinline__ int vec_elems(int dtype) { return dtype == MOGE_F32 ? 4 : 8; }
+__host__ __device__ __forceinline__ int vec_elems(int dtype) { return dtype == MOGE_F32 ? 4 : 8; }
 
-// One CTA per token: computes the token's K destination rows, writes the
-// permutation indices and copies x[t] into each destination row.
-__global__ void __launch_bounds__(kRowThreads) scatter_rows_kernel(
+// CTA (t, part): computes the token's K destination rows, copies its part of
+// x[t] (one vector per thread) into each of them; part 0 also writes the
+// permutation indices.
+__global__ void __launch_bounds__(kVecThreads) scatter_rows_kernel(
     moge_config c, const uint4 *__restrict__ x, const int32_t *__restrict__ topk_idx,
     const int32_t *__restrict__ rank, const int32_t *__restrict__ base,
     const int32_t *__restrict__ offsets, int32_t *perm_src, int32_t *perm_dst, uint4 *x_perm) {
@@ -34,17 +38,19 @@ __global__ void __launch_bounds__(kRowThreads) scatter_rows_kernel(
         int row = -1;
         if (e >= 0 && e < c.N) {
             row = offsets[e] + base[(size_t)(t / kRouterTile) * c.N + e] + rank[i];
-            perm_dst[i] = row;
-            perm_src[row] = t;
-        } else {
+            if (blockIdx.y == 0) {
+                perm_dst[i] = row;
+                perm_src[row] = t;
+            }
+        } else if (blockIdx.y == 0) {
             raise_error(ERRBIT_INVARIANT);
         }
         dst_s[k] = row;
     }
     __syncthreads();
-    const uint4 *src = x + (size_t)t * nvec;
-    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
-        const uint4 val = src[v];
+    const int v = blockIdx.y * kVecThreads + threadIdx.x;
+    if (v < nvec) {
+        const uint4 val = x[(size_t)t * nvec + v];
         for (int k = 0; k < K; ++k) {
             const int row = dst_s[k];
             if (row >= 0) x_perm[(size_t)row * nvec + v] = val;
@@ -56,8 +62,10 @@ cudaError_t launch_scatter_rows(const moge_config &c, const void *x, const int32
                                 const int32_t *rank, const int32_t *base, const int32_t *offsets,
                                 int32_t *perm_src, int32_t *perm_dst, void *x_perm,
                                 cudaStream_t st) {
-    return launch_pdl(scatter_rows_kernel, dim3(c.T), dim3(kRowThreads), 0, st, c, (const uint4 *)x,
-                      topk_idx, rank, base, offsets, perm_src, perm_dst, (uint4 *)x_perm);
+    const int nvec = c.d / vec_elems(c.dtype);
+    return launch_pdl(scatter_rows_kernel, dim3(c.T, (nvec + kVecThreads - 1) / kVecThreads),
+                      dim3(kVecThreads), 0, st, c, (const uint4 *)x, topk_idx, rank, base, offsets,
+                      perm_src, perm_dst, (uint4 *)x_perm);
 }
 
 // x_perm[r] = x[perm_src[r]], one CTA per destination row
