@@ -195,6 +195,18 @@ MOGE_API int moge_route_noalloc(const moge_config *cfg, const void *x, const voi
 MOGE_API int moge_stage_timing(int enable);
 MOGE_API int moge_stage_times(double *ms_total, int64_t *calls);
 
+/* Failure-path check (test aid; the pages have no counterpart). Launches one
+ * small kernel whose two bounded device waits can never be satisfied -- an
+ * mbarrier phase that no thread completes and a completion counter that
+ * nothing increments, the same wait helpers the layer's pipelines use -- so
+ * both give up after limit_us microseconds (1 .. 2,000,000), record the
+ * timeout bit in the device error word and return. out: caller-owned device
+ * int32[3]; afterwards out[0] = 1 (mbarrier wait gave up), out[1] = 1
+ * (counter wait gave up), out[2] = 0. The next moge_check_device_errors then
+ * returns MOGE_ERR_TIMEOUT (and clears the word); the context stays usable.
+ * No fault, trap or hang is involved. */
+MOGE_API int moge_selftest_waits(int64_t limit_us, int32_t *out, void *stream);
+
 /* ---------------------------------------------------------------- 8-bit expert weights
  * The pages report 8-bit weight quantisation of the model (hwcomputing.csdn.net
  * news piece, deployment section) and an expert-aware quantisation method

@@ -30,7 +30,7 @@ EXPORTS = ["moge_workspace_size", "moge_last_error", "moge_check_device_errors",
            "moge_permute", "moge_grouped_ffn", "moge_shared_ffn", "moge_combine",
            "moge_layer_forward", "moge_layer_forward_host", "moge_workspace_routing",
            "moge_rmsnorm", "moge_stage_timing", "moge_stage_times", "moge_route_noalloc",
-           "moge_quantize_fp8_rows", "moge_layer_forward_fp8"]
+           "moge_quantize_fp8_rows", "moge_layer_forward_fp8", "moge_selftest_waits"]
 STAGES = ("router", "scan", "permute", "ffn", "combine")
 
 
@@ -103,6 +103,7 @@ def lib() -> ctypes.CDLL:
         L.moge_route_noalloc.argtypes = [cp] + [vp] * 10
         L.moge_stage_times.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]
         L.moge_quantize_fp8_rows.argtypes = [vp, ctypes.c_int64, ctypes.c_int64, vp, vp, vp]
+        L.moge_selftest_waits.argtypes = [ctypes.c_int64, vp, vp]
         fp = ctypes.POINTER(moge_fp8_experts)
         L.moge_layer_forward_fp8.argtypes = [cp, vp, vp, vp, fp, fp, vp, vp, vp, vp]
         for n in EXPORTS:
@@ -346,3 +347,11 @@ def moge_layer_forward_fp8(s: LayerShape, x, w: dict, w8: dict, workspace, resid
                                       ctypes.byref(shared) if shared is not None else None,
                                       _p(residual), _p(y), _p(workspace), _stream(stream)))
     return y
+
+
+def moge_selftest_waits(limit_us: int, out, stream=None):
+    """Run the bounded-wait check (see moge.h): out (device int32[3]) receives
+    [1, 1, 0] once both waits gave up; the next check_device_errors reports
+    the timeout."""
+    _chk(lib().moge_selftest_waits(int(limit_us), _p(out), _stream(stream)))
+    return out

@@ -425,6 +425,15 @@ int moge_rmsnorm(const moge_config *cfg, const void *x, float eps, void *u, void
     return MOGE_OK;
 }
 
+int moge_selftest_waits(int64_t limit_us, int32_t *out, void *stream) {
+    if (limit_us < 1 || limit_us > 2000000)
+        return fail(MOGE_ERR_INVALID_ARG, "limit_us must be in 1 .. 2000000");
+    MOGE_NEED4(out, "out");
+    MOGE_CU(launch_wait_selftest(out, (uint64_t)limit_us * 1000u, (cudaStream_t)stream),
+            "wait self-test launch");
+    return MOGE_OK;
+}
+
 int moge_quantize_fp8_rows(const void *w, int64_t rows, int64_t cols, void *q, float *scale,
                            void *stream) {
     if (rows < 0 || cols <= 0) return fail(MOGE_ERR_INVALID_ARG, "rows must be >= 0, cols > 0");

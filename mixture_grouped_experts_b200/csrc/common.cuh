@@ -81,16 +81,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 // Bounded wait for the phase with the given parity to complete. Returns false
-// (and records ERRBIT_TIMEOUT) after kWaitTimeoutNs, or at once when *abort
-// is set by another role of the CTA.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+// (and records ERRBIT_TIMEOUT) after limit_ns (kWaitTimeoutNs unless given),
+// or at once when *abort is set by another role of the CTA.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                          uint64_t limit_ns = kWaitTimeoutNs) {
     if (mbar_try_wait(bar, parity)) return true;
     uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 255u) == 0) {
             if (abort && *abort) return false;
-            if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+            if (globaltimer_ns() - t0 > limit_ns) {
                 raise_error(ERRBIT_TIMEOUT);
                 if (abort) *abort = 1;
                 return false;

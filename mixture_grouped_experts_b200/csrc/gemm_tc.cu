@@ -137,17 +137,20 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 }
 
 // Bounded wait until *ctr >= need (an up-projection's h rows of one expert).
-__device__ bool wait_counter(const int *ctr, int need, volatile int *abort) {
+// Gives up (records ERRBIT_TIMEOUT, sets *abort) after limit_ns, or at once
+// when *abort is set; abort may be NULL.
+__device__ bool wait_counter(const int *ctr, int need, volatile int *abort,
+                             uint64_t limit_ns = kWaitTimeoutNs) {
     if (ld_acquire(ctr) >= need) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
         __nanosleep(64);
         if (ld_acquire(ctr) >= need) return true;
         if ((it & 63u) == 0) {
-            if (*abort) return false;
-            if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+            if (abort && *abort) return false;
+            if (globaltimer_ns() - t0 > limit_ns) {
                 raise_error(ERRBIT_TIMEOUT);
-                *abort = 1;
+                if (abort) *abort = 1;
                 return false;
             }
         }

@@ -4,5 +4,6 @@
 #include "gemm_f32.cu"
 #include "gemm_tc.cu"
 #include "gemm_fp8.cu"
+#include "selftest.cu"
 #include "api.cu"
 #include "route_noalloc.cu"

@@ -138,6 +138,8 @@ cudaError_t launch_ffn_f32(const moge_config &c, const Plan &plan, int n_entries
 // grouped FFN with FP8 (E4M3, per-row scale) weights and bf16 activations
 cudaError_t launch_ffn_fp8(const moge_config &c, const Plan &plan, int n_entries,
                            const FfnOperands &op, int num_sms, cudaStream_t st);
+// kernel whose bounded waits run out after limit_ns (failure-path check)
+cudaError_t launch_wait_selftest(int32_t *out, uint64_t limit_ns, cudaStream_t st);
 // per-row FP8 quantisation of bf16 rows
 cudaError_t launch_quantize_fp8(const void *w, int64_t rows, int64_t cols, void *q, float *scale,
                                 cudaStream_t st);

@@ -120,3 +120,10 @@ def test_fp8_entry_points_validate_on_host(L):
     rc = L.moge_layer_forward_fp8(ctypes.byref(mg._cfg(_shape(dtype="bf16"))), 0x7000, 0x8000, None,
                                   ctypes.byref(bad), ctypes.byref(f8), None, 0x9000, 0xA000, None)
     assert rc == mg.ERR_UNSUPPORTED and b"gate_scale" in L.moge_last_error()
+
+
+def test_wait_selftest_validates_on_host(L):
+    assert L.moge_selftest_waits(0, 0x1000, None) == mg.ERR_INVALID_ARG
+    assert L.moge_selftest_waits(2000001, 0x1000, None) == mg.ERR_INVALID_ARG
+    assert L.moge_selftest_waits(1000, None, None) == mg.ERR_INVALID_ARG
+    assert L.moge_selftest_waits(1000, 0x1002, None) == mg.ERR_UNSUPPORTED
