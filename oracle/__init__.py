@@ -1,4 +1,4 @@
-"""CPU oracle of the MoGE layer forward (fp64, single thread, plain C in oracle.c).
+"""CPU oracle of the MoGE layer forward and backward (fp64, single thread, plain C in oracle.c).
 
 TEST INFRASTRUCTURE ONLY: the tests, the package smoke check and the benchmark's
 CPU-baseline leg use it; the product path never imports it. It shares no code
@@ -64,6 +64,9 @@ def _l():
         lib.oracle_layer_fp8.argtypes = [vp, i32, i32, i32, i32, i32, i32, i32, i32, vp, vp,
                                          vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                          vp, i32, vp, vp, vp, vp]
+        lib.oracle_layer_backward.argtypes = [vp, i32, i32, i32, i32, i32, i32, i32, i32,
+                                              vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                              ctypes.c_double, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         _lib = lib
     return _lib
 
@@ -198,6 +201,36 @@ def layer(x: np.ndarray, inp: dict, M: int, Kp: int, dtype: str,
                            _p(wg), _p(wu), _p(wd), _p(sg), _p(su), _p(sd),
                            _p(toks), n, _p(y), _p(idx), _p(w), _p(mg)), "layer")
     return y, idx, w, mg
+
+
+def layer_backward(x: np.ndarray, inp: dict, M: int, Kp: int, dtype: str, dy: np.ndarray,
+                   alpha: float = 0.0) -> dict:
+    """Gradients of sum_t dy_t . y_t + L_aux (routing held fixed) -- oracle.c,
+    oracle_layer_backward. x, dy: float64 [T][d]. Returns float64 arrays
+    dx [T][d], w_router [N][d], w_gate/w_up [N][I][d], w_down [N][d][I],
+    s_gate/s_up [S][I][d], s_down [S][d][I], and the scalar aux."""
+    x = np.ascontiguousarray(x, np.float64)
+    dy = np.ascontiguousarray(dy, np.float64)
+    T, d = x.shape
+    wr = _w(inp["w_router"], dtype)
+    wg, wu, wd = _w(inp["w_gate"], dtype), _w(inp["w_up"], dtype), _w(inp["w_down"], dtype)
+    N, I = wg.shape[0], wg.shape[1]
+    S = inp["s_gate"].shape[0]
+    sg, su, sd = (_w(inp[k], dtype) if S > 0 else None for k in ("s_gate", "s_up", "s_down"))
+    b = inp.get("logit_bias")
+    b = None if b is None else np.ascontiguousarray(b, np.float32)
+    out = {"dx": np.empty((T, d)), "w_router": np.empty((N, d)),
+           "w_gate": np.empty((N, I, d)), "w_up": np.empty((N, I, d)), "w_down": np.empty((N, d, I)),
+           "s_gate": np.empty((S, I, d)), "s_up": np.empty((S, I, d)), "s_down": np.empty((S, d, I))}
+    aux = np.zeros(1)
+    _chk(_l().oracle_layer_backward(_p(x), T, d, N, M, Kp, S, I, _DT[dtype], _p(wr), _p(b),
+                                    _p(wg), _p(wu), _p(wd), _p(sg), _p(su), _p(sd), _p(dy),
+                                    float(alpha), _p(out["dx"]), _p(out["w_router"]),
+                                    _p(out["w_gate"]), _p(out["w_up"]), _p(out["w_down"]),
+                                    _p(out["s_gate"]), _p(out["s_up"]), _p(out["s_down"]),
+                                    _p(aux)), "layer_backward")
+    out["aux"] = float(aux[0])
+    return out
 
 
 def rmsnorm(x: np.ndarray, eps: float = 1e-6) -> np.ndarray:

@@ -1,6 +1,6 @@
 /*
  * oracle.c -- plain, slow, single-threaded CPU reference of the MoGE FFN layer
- * forward pass, in fp64.
+ * forward and backward passes, in fp64.
  *
  * TEST INFRASTRUCTURE ONLY. Nothing on the product path may call, link or load
  * this file: it is used by the tests, by the package's smoke check and by the
@@ -470,5 +470,144 @@ int oracle_layer_fp8(const double *x, int T, int d, int N, int M, int Kp, int S,
     free(tmp);
     free(idx);
     free(w);
+    return rc;
+}
+
+/* ---------------------------------------------------------------------------
+ * Backward pass of the layer [A][B][D] for an upstream gradient dy [T][d],
+ * with the routing held at its forward value (the picks are piecewise
+ * constant in the inputs), plus the batch-level balance loss named in [E]:
+ *   L_aux = alpha * sum_i f_i P_i,  f_i = c_i / T,  P_i = (1/T) sum_t p[t][i],
+ * c_i the number of tokens routed to expert i in the batch; f_i is a count,
+ * so only P_i carries a gradient. ([E]: reportify.cn concept page "Mixture of
+ * grouped experts", bullet "technical innovation details": a batch-level
+ * auxiliary balance loss whose strength is alpha and whose f_i is the share of
+ * the batch's tokens routed to expert i; the page prints no formula, the
+ * product form above is a reading.)
+ *
+ * For token t and each picked expert e with weight w = p[t][e] (shared
+ * experts: w = 1), writing g = Wg x, u = Wu x, h = silu(g) * u, o = Wd h:
+ *   dp[t][e]  = dy_t . o                       (routed experts only)
+ *   dh        = w * Wd^T dy_t
+ *   dg        = dh * u * silu'(g),  du = dh * silu(g),
+ *               silu'(g) = s (1 + g (1 - s)),  s = 1 / (1 + e^-g)
+ *   dWd      += w * dy_t h^T,  dWg += dg x_t^T,  dWu += du x_t^T
+ *   dx_t     += Wg^T dg + Wu^T du
+ * then, with dp[t][i] += alpha * f_i / T for every expert i,
+ *   dl[t][i]  = p[t][i] (dp[t][i] - sum_j p[t][j] dp[t][j])   (softmax)
+ *   dWr[i]   += dl[t][i] x_t,   dx_t += sum_i dl[t][i] Wr[i].
+ * Every output array is overwritten. Shapes: dx [T][d], dwr [N][d],
+ * dwg/dwu [N][I][d], dwd [N][d][I], dsg/dsu [S][I][d], dsd [S][d][I].
+ * aux_out (may be NULL) receives L_aux.
+ */
+int oracle_layer_backward(const double *x, int T, int d, int N, int M, int Kp, int S, int I,
+                          int dtype, const void *w_router, const float *bias,
+                          const void *w_gate, const void *w_up, const void *w_down,
+                          const void *s_gate, const void *s_up, const void *s_down,
+                          const double *dy, double alpha, double *dx, double *dwr, double *dwg,
+                          double *dwu, double *dwd, double *dsg, double *dsu, double *dsd,
+                          double *aux_out) {
+    if (T < 0 || N <= 0 || M <= 0 || N % M != 0 || Kp < 1 || Kp > N / M) return 1;
+    const int K = M * Kp;
+    const size_t per = (size_t)I * d;
+    double *p = (double *)malloc(sizeof(double) * ((size_t)T * N + 1));
+    int32_t *idx = (int32_t *)malloc(sizeof(int32_t) * ((size_t)T * K + 1));
+    double *wk = (double *)malloc(sizeof(double) * ((size_t)T * K + 1));
+    double *f = (double *)calloc((size_t)N, sizeof(double));
+    double *dp = (double *)malloc(sizeof(double) * (size_t)N);
+    double *row = (double *)malloc(sizeof(double) * (size_t)(d > I ? d : I));
+    double *g = (double *)malloc(sizeof(double) * (size_t)I);
+    double *u = (double *)malloc(sizeof(double) * (size_t)I);
+    double *h = (double *)malloc(sizeof(double) * (size_t)I);
+    double *dh = (double *)malloc(sizeof(double) * (size_t)I);
+    if (!p || !idx || !wk || !f || !dp || !row || !g || !u || !h || !dh) {
+        free(p); free(idx); free(wk); free(f); free(dp); free(row); free(g); free(u); free(h);
+        free(dh);
+        return 2;
+    }
+    memset(dx, 0, sizeof(double) * (size_t)T * d);
+    memset(dwr, 0, sizeof(double) * (size_t)N * d);
+    memset(dwg, 0, sizeof(double) * (size_t)N * per);
+    memset(dwu, 0, sizeof(double) * (size_t)N * per);
+    memset(dwd, 0, sizeof(double) * (size_t)N * per);
+    if (S > 0) {
+        memset(dsg, 0, sizeof(double) * (size_t)S * per);
+        memset(dsu, 0, sizeof(double) * (size_t)S * per);
+        memset(dsd, 0, sizeof(double) * (size_t)S * per);
+    }
+    int rc = oracle_router_probs(x, w_router, bias, dtype, T, d, N, p);
+    if (!rc) rc = oracle_select_grouped(p, T, N, M, Kp, idx, wk, NULL);
+    double aux = 0.0;
+    if (!rc && T > 0) {
+        for (size_t i = 0; i < (size_t)T * K; ++i) f[idx[i]] += 1.0 / T;
+        for (int e = 0; e < N; ++e) {
+            double P = 0.0;
+            for (int t = 0; t < T; ++t) P += p[(size_t)t * N + e];
+            aux += alpha * f[e] * (P / T);
+        }
+    }
+    for (int t = 0; t < T && !rc; ++t) {
+        const double *xt = x + (size_t)t * d;
+        const double *dyt = dy + (size_t)t * d;
+        double *dxt = dx + (size_t)t * d;
+        for (int e = 0; e < N; ++e) dp[e] = alpha * f[e] / T;
+        for (int k = 0; k < K + S; ++k) {
+            const int routed = k < K;
+            const size_t e = routed ? (size_t)idx[(size_t)t * K + k] : (size_t)(k - K);
+            const double w = routed ? wk[(size_t)t * K + k] : 1.0;
+            const void *wg = routed ? expert_ptr(w_gate, dtype, e, per) : expert_ptr(s_gate, dtype, e, per);
+            const void *wu = routed ? expert_ptr(w_up, dtype, e, per) : expert_ptr(s_up, dtype, e, per);
+            const void *wd = routed ? expert_ptr(w_down, dtype, e, per) : expert_ptr(s_down, dtype, e, per);
+            double *gg = (routed ? dwg : dsg) + e * per;
+            double *gu = (routed ? dwu : dsu) + e * per;
+            double *gd = (routed ? dwd : dsd) + e * per;
+            for (int i = 0; i < I; ++i) {
+                load_row(wg, dtype, (size_t)i * d, d, row);
+                g[i] = dot(xt, row, d);
+                load_row(wu, dtype, (size_t)i * d, d, row);
+                u[i] = dot(xt, row, d);
+                h[i] = g[i] / (1.0 + exp(-g[i])) * u[i];
+                dh[i] = 0.0;
+            }
+            double o_dot = 0.0;  /* dy_t . (Wd h) */
+            for (int o = 0; o < d; ++o) {
+                load_row(wd, dtype, (size_t)o * I, I, row);
+                o_dot += dyt[o] * dot(h, row, I);
+                for (int i = 0; i < I; ++i) {
+                    dh[i] += w * dyt[o] * row[i];
+                    gd[(size_t)o * I + i] += w * dyt[o] * h[i];
+                }
+            }
+            if (routed) dp[e] += o_dot;
+            for (int i = 0; i < I; ++i) {
+                const double s = 1.0 / (1.0 + exp(-g[i]));
+                const double dg = dh[i] * u[i] * s * (1.0 + g[i] * (1.0 - s));
+                const double du = dh[i] * g[i] * s;
+                load_row(wg, dtype, (size_t)i * d, d, row);
+                for (int c = 0; c < d; ++c) {
+                    gg[(size_t)i * d + c] += dg * xt[c];
+                    dxt[c] += dg * row[c];
+                }
+                load_row(wu, dtype, (size_t)i * d, d, row);
+                for (int c = 0; c < d; ++c) {
+                    gu[(size_t)i * d + c] += du * xt[c];
+                    dxt[c] += du * row[c];
+                }
+            }
+        }
+        const double *pt = p + (size_t)t * N;
+        double pdp = 0.0;
+        for (int e = 0; e < N; ++e) pdp += pt[e] * dp[e];
+        for (int e = 0; e < N; ++e) {
+            const double dl = pt[e] * (dp[e] - pdp);
+            load_row(w_router, dtype, (size_t)e * d, d, row);
+            for (int c = 0; c < d; ++c) {
+                dwr[(size_t)e * d + c] += dl * xt[c];
+                dxt[c] += dl * row[c];
+            }
+        }
+    }
+    if (aux_out) *aux_out = aux;
+    free(p); free(idx); free(wk); free(f); free(dp); free(row); free(g); free(u); free(h); free(dh);
     return rc;
 }

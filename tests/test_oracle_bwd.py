@@ -1,0 +1,109 @@
+"""Pins of the oracle's backward pass (no GPU): central finite differences of
+the oracle's own forward layer, coordinate by coordinate, for every input and
+weight tensor, with the routing checked to stay put under each perturbation;
+the balance loss alone; the dense special case (every expert picked); and the
+softmax invariant that the router gradient's rows sum to zero."""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+WEIGHTS = ("w_router", "w_gate", "w_up", "w_down", "s_gate", "s_up", "s_down")
+
+
+def _loss(x, inp, M, Kp, dtype, dy, alpha, f):
+    """sum_t dy_t . y_t + alpha sum_i f_i P_i, f fixed (the balance loss's count share)."""
+    y, idx, _, _ = oracle.layer(x, inp, M, Kp, dtype)
+    p = oracle.router_probs(x, inp["w_router"], inp.get("logit_bias"), dtype)
+    return float((dy * y).sum() + alpha * (f * p.mean(0)).sum()), idx
+
+
+def _count_share(x, inp, M, Kp, dtype, N):
+    _, idx, _, _ = oracle.layer(x, inp, M, Kp, dtype)
+    return np.bincount(idx.ravel(), minlength=N) / x.shape[0], idx
+
+
+def _check_fd(cfg, alpha, n_coords=6, h_x=1e-5, h_w=1e-4, tensors=("x",) + WEIGHTS, seed=0):
+    inp = synth.layer_inputs(cfg)
+    x = oracle.to_double(inp["x"], cfg.dtype)
+    rng = np.random.default_rng(seed)
+    dy = rng.normal(size=x.shape)
+    g = oracle.layer_backward(x, inp, cfg.M, cfg.Kp, cfg.dtype, dy, alpha)
+    f, idx0 = _count_share(x, inp, cfg.M, cfg.Kp, cfg.dtype, cfg.N)
+    checked = 0
+    for name in tensors:
+        if name.startswith("s_") and cfg.S == 0:
+            continue
+        base = x if name == "x" else inp[name]
+        ana = g["dx"] if name == "x" else g[name]
+        for flat in rng.choice(base.size, size=min(n_coords, base.size), replace=False):
+            vals = []
+            for sgn in (1.0, -1.0):
+                if name == "x":
+                    xp = x.copy()
+                    xp.flat[flat] += sgn * h_x
+                    L, idx = _loss(xp, inp, cfg.M, cfg.Kp, cfg.dtype, dy, alpha, f)
+                    vals.append((L, xp.flat[flat]))
+                else:
+                    w = base.copy()
+                    w.flat[flat] = np.float32(w.flat[flat] + sgn * h_w)
+                    ip = dict(inp)
+                    ip[name] = w
+                    L, idx = _loss(x, ip, cfg.M, cfg.Kp, cfg.dtype, dy, alpha, f)
+                    vals.append((L, float(w.flat[flat])))
+                assert np.array_equal(idx, idx0), "routing moved under the perturbation"
+            fd = (vals[0][0] - vals[1][0]) / (vals[0][1] - vals[1][1])
+            an = ana.flat[flat]
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, flat, fd, an)
+            checked += 1
+    return checked
+
+
+SMALL = synth.Config("fd", T=7, d=24, N=8, M=4, Kp=1, S=2, I=12, dtype="f32", seed=21, w_std=0.3)
+
+
+def test_fd_every_tensor():
+    assert _check_fd(SMALL, alpha=0.0) >= 40
+
+
+def test_fd_with_balance_loss():
+    assert _check_fd(SMALL, alpha=0.37, seed=1) >= 40
+
+
+def test_fd_balance_loss_alone():
+    cfg = SMALL.replace(seed=22)
+    inp = synth.layer_inputs(cfg)
+    x = oracle.to_double(inp["x"], "f32")
+    g = oracle.layer_backward(x, inp, cfg.M, cfg.Kp, "f32", np.zeros_like(x), alpha=1.0)
+    # no upstream gradient: only the router and x move, every expert gradient is zero
+    for k in ("w_gate", "w_up", "w_down", "s_gate", "s_up", "s_down"):
+        assert not g[k].any()
+    assert np.abs(g["w_router"]).max() > 0
+    f, _ = _count_share(x, inp, cfg.M, cfg.Kp, "f32", cfg.N)
+    p = oracle.router_probs(x, inp["w_router"], None, "f32")
+    assert g["aux"] == pytest.approx(float((f * p.mean(0)).sum()), rel=1e-12)
+    assert _check_fd(cfg, alpha=1.0, tensors=("x", "w_router"), seed=2) >= 12
+
+
+def test_fd_dense_every_expert_picked():
+    # K' = N/M: the picks never change, the layer is sum_e p_e FFN_e(x) + shared
+    cfg = synth.Config("dense", T=5, d=16, N=8, M=2, Kp=4, S=1, I=8, dtype="f32", seed=23,
+                       w_std=0.3)
+    assert _check_fd(cfg, alpha=0.2, seed=3) >= 40
+
+
+def test_fd_bf16_weights_through_x():
+    cfg = SMALL.replace(dtype="bf16", seed=24)
+    assert _check_fd(cfg, alpha=0.1, tensors=("x",), n_coords=12, seed=4) == 12
+
+
+def test_router_gradient_rows_sum_to_zero_and_linearity():
+    inp = synth.layer_inputs(SMALL)
+    x = oracle.to_double(inp["x"], "f32")
+    dy = np.random.default_rng(5).normal(size=x.shape)
+    g1 = oracle.layer_backward(x, inp, SMALL.M, SMALL.Kp, "f32", dy, 0.0)
+    g2 = oracle.layer_backward(x, inp, SMALL.M, SMALL.Kp, "f32", 2.0 * dy, 0.0)
+    assert np.abs(g1["w_router"].sum(0)).max() < 1e-12
+    for k in ("dx",) + WEIGHTS:
+        np.testing.assert_allclose(g2[k], 2.0 * g1[k], rtol=1e-12, atol=1e-14)
