@@ -245,6 +245,58 @@ MOGE_API int moge_layer_forward_fp8(const moge_config *cfg, const void *x, const
                                     const moge_fp8_experts *shared, const void *residual, void *y,
                                     void *workspace, void *stream);
 
+
+/* ---------------------------------------------------------------- training
+ * Backward pass of the layer (the pages' models are trained, and they name a
+ * batch-level auxiliary balance loss: reportify.cn concept page "Mixture of
+ * grouped experts", bullet "technical innovation details" -- strength alpha,
+ * f_i = share of the batch's tokens routed to expert i; no formula is printed,
+ * this library reads it as L_aux = alpha * sum_i f_i * P_i with P_i the batch
+ * mean of the softmax score p[t][i]; f_i is a count and carries no gradient).
+ * The routing (picks) is held at its forward value, as in every top-K router.
+ *
+ * Only cfg->dtype == MOGE_BF16, with I % 64 == 0, N % 8 == 0, M * Kp <= 32.
+ *
+ * moge_train_workspace_size: bytes of the training workspace (the forward
+ * workspace plus the saved pre-activations and the backward's scratch), 0 for
+ * an unsupported config. */
+MOGE_API size_t moge_train_workspace_size(const moge_config *cfg);
+
+/* moge_layer_forward (no residual) that also keeps, in `workspace`, what the
+ * backward pass reads: the routing, the permuted rows, h, the expert outputs
+ * and the up-projection's pre-activations g and u. Same arguments and rules
+ * as moge_layer_forward; `workspace` is a training workspace and must be
+ * passed unchanged to the moge_layer_backward call that follows. */
+MOGE_API int moge_layer_forward_train(const moge_config *cfg, const void *x, const void *w_router,
+                                      const float *logit_bias, const void *w_gate,
+                                      const void *w_up, const void *w_down, const void *s_gate,
+                                      const void *s_up, const void *s_down, void *y,
+                                      void *workspace, void *stream);
+
+/* Gradients of  sum_t dy[t] . y[t] + L_aux  with respect to the layer's input
+ * and weights, for the forward of the preceding moge_layer_forward_train call
+ * (same cfg, x, weights, logit_bias and workspace; x and the weights must be
+ * unchanged). dy [T][d] bf16 (device). Outputs (caller-owned device memory,
+ * bf16, 16-byte aligned, overwritten, layouts of their forward tensors):
+ * dx [T][d]; dw_router [N][d]; dw_gate, dw_up [N][I][d]; dw_down [N][d][I];
+ * ds_gate, ds_up [S][I][d]; ds_down [S][d][I] (NULL when S == 0). An expert no
+ * token chose gets a zero gradient. aux: device float (nullable) receiving
+ * L_aux. logit_bias gets no gradient (it is an input, not a weight).
+ * The workspace's saved tensors are consumed (overwritten) by the call.
+ * Computation: the expert GEMMs (dh with the SwiGLU backward fused in its
+ * epilogue, dx, dW_down, dW_gate / dW_up over each expert's rows) and the
+ * router's (logits recomputed, dW_router, the router's share of dx) run on the
+ * tensor cores with fp32 accumulation; the softmax backward, the combine's
+ * backward (dy_perm = w * dy, dw = dy . expert output) and the un-permute are
+ * bandwidth-bound kernels. Asynchronous on `stream`. */
+MOGE_API int moge_layer_backward(const moge_config *cfg, float alpha, const void *x,
+                                 const void *w_router, const float *logit_bias,
+                                 const void *w_gate, const void *w_up, const void *w_down,
+                                 const void *s_gate, const void *s_up, const void *s_down,
+                                 const void *dy, void *dx, void *dw_router, void *dw_gate,
+                                 void *dw_up, void *dw_down, void *ds_gate, void *ds_up,
+                                 void *ds_down, float *aux, void *workspace, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -30,7 +30,8 @@ EXPORTS = ["moge_workspace_size", "moge_last_error", "moge_check_device_errors",
            "moge_permute", "moge_grouped_ffn", "moge_shared_ffn", "moge_combine",
            "moge_layer_forward", "moge_layer_forward_host", "moge_workspace_routing",
            "moge_rmsnorm", "moge_stage_timing", "moge_stage_times", "moge_route_noalloc",
-           "moge_quantize_fp8_rows", "moge_layer_forward_fp8", "moge_selftest_waits"]
+           "moge_quantize_fp8_rows", "moge_layer_forward_fp8", "moge_selftest_waits",
+           "moge_train_workspace_size", "moge_layer_forward_train", "moge_layer_backward"]
 STAGES = ("router", "scan", "permute", "ffn", "combine")
 
 
@@ -106,8 +107,12 @@ def lib() -> ctypes.CDLL:
         L.moge_selftest_waits.argtypes = [ctypes.c_int64, vp, vp]
         fp = ctypes.POINTER(moge_fp8_experts)
         L.moge_layer_forward_fp8.argtypes = [cp, vp, vp, vp, fp, fp, vp, vp, vp, vp]
+        L.moge_train_workspace_size.argtypes = [cp]
+        L.moge_train_workspace_size.restype = ctypes.c_size_t
+        L.moge_layer_forward_train.argtypes = [cp] + [vp] * 12
+        L.moge_layer_backward.argtypes = [cp, ctypes.c_float] + [vp] * 21
         for n in EXPORTS:
-            if n not in ("moge_workspace_size", "moge_last_error"):
+            if n not in ("moge_workspace_size", "moge_last_error", "moge_train_workspace_size"):
                 getattr(L, n).restype = i32
         _lib = L
     return _lib
@@ -147,6 +152,17 @@ def workspace_size(s: LayerShape) -> int:
 
 def alloc_workspace(s: LayerShape, device=None) -> torch.Tensor:
     return torch.empty(workspace_size(s), dtype=torch.uint8, device=device or "cuda")
+
+
+def train_workspace_size(s: LayerShape) -> int:
+    n = lib().moge_train_workspace_size(ctypes.byref(_cfg(s)))
+    if n == 0:
+        raise MogeError(ERR_UNSUPPORTED, lib().moge_last_error().decode())
+    return n
+
+
+def alloc_train_workspace(s: LayerShape, device=None) -> torch.Tensor:
+    return torch.empty(train_workspace_size(s), dtype=torch.uint8, device=device or "cuda")
 
 
 def check_device_errors(stream=None):
@@ -229,6 +245,39 @@ def moge_layer_forward(s: LayerShape, x, w: dict, workspace, residual=None, y=No
                                   _p(w.get("s_down")), _p(residual), _p(y), _p(workspace),
                                   _stream(stream)))
     return y
+
+
+def moge_layer_forward_train(s: LayerShape, x, w: dict, workspace, y=None, stream=None):
+    """Forward that keeps what moge_layer_backward needs in `workspace` (a training workspace)."""
+    if y is None:
+        y = torch.empty((s.T, s.d), dtype=x.dtype, device=x.device)
+    _chk(lib().moge_layer_forward_train(ctypes.byref(_cfg(s)), _p(x), _p(w["w_router"]),
+                                        _p(w.get("logit_bias")), _p(w["w_gate"]), _p(w["w_up"]),
+                                        _p(w["w_down"]), _p(w.get("s_gate")), _p(w.get("s_up")),
+                                        _p(w.get("s_down")), _p(y), _p(workspace),
+                                        _stream(stream)))
+    return y
+
+
+GRAD_KEYS = ("w_router", "w_gate", "w_up", "w_down", "s_gate", "s_up", "s_down")
+
+
+def moge_layer_backward(s: LayerShape, x, w: dict, dy, workspace, alpha: float = 0.0, grads=None,
+                        dx=None, aux=None, stream=None):
+    """Gradients for the preceding moge_layer_forward_train on the same workspace.
+    Returns (dx, grads) with grads keyed like the weights (GRAD_KEYS); `aux` (a
+    device float32 tensor of one element, optional) receives the balance loss."""
+    if dx is None:
+        dx = torch.empty_like(x)
+    if grads is None:
+        grads = {k: torch.empty_like(w[k]) for k in GRAD_KEYS if w.get(k) is not None}
+    _chk(lib().moge_layer_backward(ctypes.byref(_cfg(s)), float(alpha), _p(x), _p(w["w_router"]),
+                                   _p(w.get("logit_bias")), _p(w["w_gate"]), _p(w["w_up"]),
+                                   _p(w["w_down"]), _p(w.get("s_gate")), _p(w.get("s_up")),
+                                   _p(w.get("s_down")), _p(dy), _p(dx),
+                                   *[_p(grads.get(k)) for k in GRAD_KEYS], _p(aux),
+                                   _p(workspace), _stream(stream)))
+    return dx, grads
 
 
 def moge_layer_forward_host(s: LayerShape, x_host, w: dict, workspace, y_host, x_dev, y_dev,

@@ -210,6 +210,52 @@ static int layer_run(const moge_config &c, const void *x, const void *w_router,
     return MOGE_OK;
 }
 
+
+// Training workspace: the forward workspace, then what the backward pass needs
+// beyond it. dgu overwrites gu in place (the SwiGLU backward reads g, u and
+// writes dg, du at the same positions, each element by one thread) and dx_perm
+// overwrites y_perm (read only by the combine backward, which runs first).
+struct TrainSpace {
+    Workspace fw;
+    void *gu;        // [hrows][2I]
+    void *dy_perm;   // [rrows][d]
+    float *logits;   // [T][N]
+    void *dl;        // [T][N]
+    float *dx_r;     // [T][d]
+    float *dw;       // [T][K]
+    float *part;     // [router_bwd_parts][N]
+    size_t total;
+};
+static TrainSpace carve_train(const moge_config &c, void *base) {
+    TrainSpace s;
+    s.fw = carve_workspace(c, base);
+    const size_t K = (size_t)c.M * c.Kp, T = (size_t)c.T;
+    char *p = static_cast<char *>(base);
+    size_t off = s.fw.total;
+    auto take = [&](size_t bytes) {
+        char *r = p ? p + off : nullptr;
+        off += align256(bytes > 0 ? bytes : 1);
+        return r;
+    };
+    s.gu = take(T * (K + c.S) * 2 * (size_t)c.I * 2);
+    s.dy_perm = take(T * K * c.d * 2);
+    s.logits = (float *)take(T * c.N * 4);
+    s.dl = take(T * c.N * 2);
+    s.dx_r = (float *)take(T * c.d * 4);
+    s.dw = (float *)take(T * K * 4);
+    s.part = (float *)take((size_t)router_bwd_parts(c) * c.N * 4);
+    s.total = off;
+    return s;
+}
+
+static int check_train(const moge_config &c) {
+    if (c.dtype != MOGE_BF16) return fail(MOGE_ERR_UNSUPPORTED, "training needs dtype MOGE_BF16");
+    if (c.I % 64 != 0) return fail(MOGE_ERR_UNSUPPORTED, "training needs I % 64 == 0");
+    if (c.N % 8 != 0) return fail(MOGE_ERR_UNSUPPORTED, "training needs N % 8 == 0");
+    if (c.M * c.Kp > 32) return fail(MOGE_ERR_UNSUPPORTED, "training needs M * Kp <= 32");
+    return MOGE_OK;
+}
+
 extern "C" {
 
 size_t moge_workspace_size(const moge_config *cfg) {
@@ -507,6 +553,125 @@ int moge_stage_times(double *ms_total, int64_t *calls) {
     if (ms_total)
         for (int k = 0; k < kTimedStages; ++k) ms_total[k] = g_timer.total_ms[k];
     if (calls) *calls = g_timer.calls;
+    return MOGE_OK;
+}
+
+
+size_t moge_train_workspace_size(const moge_config *cfg) {
+    if (check_config(cfg) != MOGE_OK || check_train(*cfg) != MOGE_OK) return 0;
+    return carve_train(*cfg, nullptr).total;
+}
+
+int moge_layer_forward_train(const moge_config *cfg, const void *x, const void *w_router,
+                             const float *logit_bias, const void *w_gate, const void *w_up,
+                             const void *w_down, const void *s_gate, const void *s_up,
+                             const void *s_down, void *y, void *workspace, void *stream) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    const moge_config c = *cfg;
+    if ((rc = check_train(c))) return rc;
+    if (c.T == 0) return MOGE_OK;
+    MOGE_NEED(x, "x");
+    MOGE_NEED(w_router, "w_router");
+    MOGE_NEED(w_gate, "w_gate");
+    MOGE_NEED(w_up, "w_up");
+    MOGE_NEED(w_down, "w_down");
+    if (c.S > 0) {
+        MOGE_NEED(s_gate, "s_gate");
+        MOGE_NEED(s_up, "s_up");
+        MOGE_NEED(s_down, "s_down");
+    }
+    if (logit_bias && !aligned4(logit_bias)) return fail(MOGE_ERR_UNSUPPORTED, "logit_bias misaligned");
+    MOGE_NEED(y, "y");
+    MOGE_NEED(workspace, "workspace");
+    if (y == x) return fail(MOGE_ERR_INVALID_ARG, "y must not alias x");
+    TrainSpace ts = carve_train(c, workspace);
+    FfnOperands wts{};
+    wts.wg = w_gate; wts.wu = w_up; wts.wd = w_down;
+    if (c.S > 0) { wts.sg = s_gate; wts.su = s_up; wts.sd = s_down; }
+    wts.gu = ts.gu;
+    return layer_run(c, x, w_router, logit_bias, wts, false, nullptr, y, workspace,
+                     (cudaStream_t)stream);
+}
+
+int moge_layer_backward(const moge_config *cfg, float alpha, const void *x, const void *w_router,
+                        const float *logit_bias, const void *w_gate, const void *w_up,
+                        const void *w_down, const void *s_gate, const void *s_up,
+                        const void *s_down, const void *dy, void *dx, void *dw_router,
+                        void *dw_gate, void *dw_up, void *dw_down, void *ds_gate, void *ds_up,
+                        void *ds_down, float *aux, void *workspace, void *stream) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    const moge_config c = *cfg;
+    if ((rc = check_train(c))) return rc;
+    cudaStream_t st = (cudaStream_t)stream;
+    MOGE_NEED(dw_router, "dw_router");
+    MOGE_NEED(dw_gate, "dw_gate");
+    MOGE_NEED(dw_up, "dw_up");
+    MOGE_NEED(dw_down, "dw_down");
+    if (c.S > 0) {
+        MOGE_NEED(ds_gate, "ds_gate");
+        MOGE_NEED(ds_up, "ds_up");
+        MOGE_NEED(ds_down, "ds_down");
+    }
+    if (aux && !aligned4(aux)) return fail(MOGE_ERR_UNSUPPORTED, "aux misaligned");
+    const size_t wsz = (size_t)c.I * c.d * 2;
+    if (c.T == 0) {  // no tokens: every gradient is zero
+        MOGE_CU(cudaMemsetAsync(dw_router, 0, (size_t)c.N * c.d * 2, st), "memset");
+        MOGE_CU(cudaMemsetAsync(dw_gate, 0, c.N * wsz, st), "memset");
+        MOGE_CU(cudaMemsetAsync(dw_up, 0, c.N * wsz, st), "memset");
+        MOGE_CU(cudaMemsetAsync(dw_down, 0, c.N * wsz, st), "memset");
+        if (c.S > 0) {
+            MOGE_CU(cudaMemsetAsync(ds_gate, 0, c.S * wsz, st), "memset");
+            MOGE_CU(cudaMemsetAsync(ds_up, 0, c.S * wsz, st), "memset");
+            MOGE_CU(cudaMemsetAsync(ds_down, 0, c.S * wsz, st), "memset");
+        }
+        if (aux) MOGE_CU(cudaMemsetAsync(aux, 0, sizeof(float), st), "memset");
+        return MOGE_OK;
+    }
+    MOGE_NEED(x, "x");
+    MOGE_NEED(w_router, "w_router");
+    MOGE_NEED(w_gate, "w_gate");
+    MOGE_NEED(w_up, "w_up");
+    MOGE_NEED(w_down, "w_down");
+    if (c.S > 0) {
+        MOGE_NEED(s_gate, "s_gate");
+        MOGE_NEED(s_up, "s_up");
+        MOGE_NEED(s_down, "s_down");
+    }
+    if (logit_bias && !aligned4(logit_bias)) return fail(MOGE_ERR_UNSUPPORTED, "logit_bias misaligned");
+    MOGE_NEED(dy, "dy");
+    MOGE_NEED(dx, "dx");
+    MOGE_NEED(workspace, "workspace");
+    if (dx == dy || dx == x) return fail(MOGE_ERR_INVALID_ARG, "dx must not alias x or dy");
+    TrainSpace ts = carve_train(c, workspace);
+    const Workspace &ws = ts.fw;
+    const int E = c.N + c.S;
+    BwdTensors b{};
+    b.x = x; b.w_router = w_router; b.bias = logit_bias;
+    b.wg = w_gate; b.wu = w_up; b.wd = w_down;
+    if (c.S > 0) { b.sg = s_gate; b.su = s_up; b.sd = s_down; }
+    b.x_perm = ws.x_perm; b.h = ws.h; b.gu = ts.gu;
+    b.dy = dy; b.dy_perm = ts.dy_perm;
+    b.dgu = ts.gu;          // in place
+    b.dx_perm = ws.y_perm;  // y_perm is dead once the combine backward has run
+    b.logits = ts.logits; b.dl = ts.dl; b.dx_r = ts.dx_r;
+    b.dwg = dw_gate; b.dwu = dw_up; b.dwd = dw_down; b.dwr = dw_router;
+    b.dsg = ds_gate; b.dsu = ds_up; b.dsd = ds_down;
+    const int sms = num_sms();
+    const ExpertWork *ent = ws.plan.up;
+    MOGE_CU(launch_combine_bwd(c, dy, ws.y_perm, ws.topk_w, ws.perm_dst, ts.dy_perm, ts.dw, st),
+            "combine backward launch");
+    MOGE_CU(launch_bwd_gemm(kLOGITS, c, ent, E, b, sms, st), "logits launch");
+    MOGE_CU(launch_router_bwd(c, alpha, ts.logits, ws.topk_idx, ts.dw, ws.counts, ts.dl, ts.part,
+                              aux, st), "router backward launch");
+    MOGE_CU(launch_bwd_gemm(kDH, c, ent, E, b, sms, st), "dh launch");
+    MOGE_CU(launch_bwd_gemm(kDX, c, ent, E, b, sms, st), "dx launch");
+    MOGE_CU(launch_bwd_gemm(kDWD, c, ent, E, b, sms, st), "dW_down launch");
+    MOGE_CU(launch_bwd_gemm(kDWGU, c, ent, E, b, sms, st), "dW_gate/up launch");
+    MOGE_CU(launch_bwd_gemm(kDWR, c, ent, E, b, sms, st), "dW_router launch");
+    MOGE_CU(launch_bwd_gemm(kDXR, c, ent, E, b, sms, st), "dx router launch");
+    MOGE_CU(launch_unpermute_bwd(c, ws.y_perm, ws.perm_dst, ts.dx_r, dx, st), "un-permute launch");
     return MOGE_OK;
 }
 

@@ -1,0 +1,610 @@
+// Backward pass of the MoGE layer: its grouped GEMMs on the 5th-generation
+// tensor cores (sm_100a).
+//
+// One persistent kernel serves seven GEMM kinds; a launch runs one kind over
+// every expert entry of the forward's plan (shared experts first, then the
+// routed ones, rows in the forward's permuted order). With x, x_perm, h, the
+// saved SwiGLU pre-activations gu = [g | u] and dy_perm = w * dy (routed rows)
+// or dy (shared rows), for expert e:
+//   kDH     dh^T  = Wd^T dy^T      -> SwiGLU backward in the epilogue: dgu = [dg | du]
+//   kDX     dx^T  = Wg^T dg^T + Wu^T du^T   (K runs over [g | u]: 2I)
+//   kDWD    dWd   = dy^T h         (K = the expert's rows)
+//   kDWGU   dWg   = dg^T x,  dWu = du^T x   (K = the expert's rows)
+// and for the router (one entry, all T tokens):
+//   kLOGITS l     = x Wr^T + bias  (recomputed logits, fp32)
+//   kDWR    dWr   = dl^T x         (K = T)
+//   kDXR    dx_r  = dl Wr          (K = N, fp32)
+// D = A B^T with the MMA's M = 128 rows of A in TMEM lanes and N <= 256
+// columns. Operands are staged by TMA in 64 x 64 boxes with the 128-byte
+// swizzle; a row-major matrix read along its rows is a "K-major" operand, read
+// across them an "MN-major" one (tcgen05 descriptor: 8-row groups 1024 bytes
+// apart, 64-element blocks 8 KB apart). Gradients over an expert's rows have a
+// ragged last K-chunk: its rows past the expert are zeroed in shared memory in
+// the A operand (they belong to the next expert) and the MMAs past them are
+// skipped.
+//
+// Roles per CTA (one per SM, 192 threads): warp 0 TMA producer, warp 1 MMA
+// issuer (one thread; the warp zeroes ragged rows), warps 2-5 epilogue. Items
+// are dealt out statically (item blockIdx.x + i * gridDim.x), all three roles
+// walk the same sequence; two 256-column accumulators let the epilogue of one
+// item overlap the MMAs of the next. Every wait is bounded.
+#include "common.cuh"
+#include "moge_internal.h"
+
+namespace moge {
+
+constexpr int kGStages = 4;
+constexpr int kGStageBytes = 48 * 1024;  // A: 2 boxes (16 KB), B: up to 4 boxes (32 KB)
+constexpr int kGThreads = 192;
+constexpr uint32_t kGTmemCols = 512;
+constexpr int kGMaxEntries = kMaxExperts + 64;
+
+struct GMaps {
+    CUtensorMap m[6];
+};
+
+struct GParams {
+    int kind;
+    const ExpertWork *ent;  // forward plan entries (token and weight-gradient kinds)
+    int n_entries;
+    int T, d, I, N;
+    int m_tiles;            // M tiles per entry (per part for kDWGU)
+    int n_tiles, bn;        // weight-gradient and router kinds: N tiles and their width
+    int kc;                 // K chunks of the fixed-K kinds
+    void *out[4];
+    const uint16_t *gu;     // kDH: [rows][2I]
+    const float *bias;      // kLOGITS, nullable
+};
+
+struct GItem {
+    int entry, mt, nt, bn, n_valid, nck, kv_last;
+};
+
+struct GShared {
+    uint64_t full[kGStages], empty[kGStages], tfull[2], tempty[2], drain;
+    uint32_t tmem_base;
+    int abort;
+    int total;
+    int start[kGMaxEntries + 1];  // token kinds: prefix sum of items per entry
+};
+
+__device__ __forceinline__ bool g_token_kind(int kind) { return kind == kDH || kind == kDX; }
+__device__ __forceinline__ bool g_wgrad_kind(int kind) { return kind == kDWD || kind == kDWGU; }
+// (A, B) is MN-major?
+__device__ __forceinline__ bool g_a_mn(int kind) { return kind != kLOGITS; }
+__device__ __forceinline__ bool g_b_mn(int kind) {
+    return kind == kDWD || kind == kDWGU || kind == kDWR;
+}
+
+__device__ void g_decode(const GParams &p, const GShared &sh, int q, GItem &it) {
+    it.kv_last = 64;
+    if (g_token_kind(p.kind)) {
+        int lo = 0, hi = p.n_entries - 1;
+        while (lo < hi) {  // last entry whose first item is <= q
+            const int mid = (lo + hi + 1) >> 1;
+            if (sh.start[mid] <= q) lo = mid; else hi = mid - 1;
+        }
+        const ExpertWork &w = p.ent[lo];
+        const int r = q - sh.start[lo];
+        it.entry = lo;
+        it.mt = r / w.ntb;
+        it.nt = r % w.ntb;
+        it.bn = w.bn;
+        it.n_valid = min(w.bn, w.rows - it.nt * w.bn);
+        it.nck = p.kc;
+    } else if (g_wgrad_kind(p.kind)) {
+        const int mt_all = p.kind == kDWGU ? 2 * p.m_tiles : p.m_tiles;
+        const int per = mt_all * p.n_tiles;
+        it.entry = q / per;
+        const int r = q % per;
+        it.mt = r / p.n_tiles;
+        it.nt = r % p.n_tiles;
+        it.bn = p.bn;
+        it.n_valid = p.bn;
+        const int rows = p.ent[it.entry].rows;
+        it.nck = (rows + 63) / 64;
+        it.kv_last = rows - 64 * (it.nck - 1);
+    } else {
+        it.entry = 0;
+        it.mt = q / p.n_tiles;
+        it.nt = q % p.n_tiles;
+        it.bn = p.bn;
+        const int ncols = p.kind == kDWR ? p.d : p.T;
+        it.n_valid = min(p.bn, ncols - it.nt * p.bn);
+        it.nck = p.kind == kDWR ? (p.T + 63) / 64 : p.kc;
+    }
+}
+
+// Issue box `j` of operand A (j < 2) or B (j >= 2: box j - 2) of chunk kc.
+__device__ __forceinline__ void g_load(const GParams &p, const GMaps &mp, const GItem &it, int kc,
+                                       int j, unsigned char *stage, uint64_t *bar, uint64_t pol_a,
+                                       uint64_t pol_b) {
+    const ExpertWork *w = g_token_kind(p.kind) || g_wgrad_kind(p.kind) ? &p.ent[it.entry] : nullptr;
+    const int k = 64 * kc;
+    if (j < 2) {
+        unsigned char *dst = stage + 8192 * j;
+        const int mn = it.mt * 128 + 64 * j;
+        switch (p.kind) {
+            case kDH:  // Wd[e] as [d][I]: rows are K
+                tma_load_3d(dst, &mp.m[w->a_sel], bar, mn, k, w->a_idx, pol_a);
+                break;
+            case kDX: {  // Wg[e] then Wu[e], as [I][d]: rows are K
+                const int kh = p.I / 64;
+                const int sel = (kc < kh ? 0 : 2) + w->a_sel;
+                tma_load_3d(dst, &mp.m[sel], bar, mn, kc < kh ? k : k - p.I, w->a_idx, pol_a);
+                break;
+            }
+            case kDWD:  // dy rows (dy_perm / dy) read across: rows are K
+                tma_load_2d(dst, &mp.m[w->b_sel], bar, mn, w->src_row0 + k, pol_a);
+                break;
+            case kDWGU: {  // [g | u] rows read across
+                const int part = it.mt / p.m_tiles;
+                const int m0 = (it.mt - part * p.m_tiles) * 128 + 64 * j + part * p.I;
+                tma_load_2d(dst, &mp.m[0], bar, m0, w->dst_row0 + k, pol_a);
+                break;
+            }
+            case kLOGITS:  // Wr rows, K-major
+                tma_load_2d(dst, &mp.m[0], bar, k, mn, pol_a);
+                break;
+            default:  // kDWR: dl read across (rows are tokens = K); kDXR: Wr read across
+                tma_load_2d(dst, &mp.m[0], bar, mn, k, pol_a);
+                break;
+        }
+    } else {
+        const int jb = j - 2;
+        unsigned char *dst = stage + 16384 + 8192 * jb;
+        const int r0 = it.nt * it.bn + 64 * jb;  // first N element of the box
+        switch (p.kind) {
+            case kDH:  // dy rows, K-major
+                tma_load_2d(dst, &mp.m[2 + w->b_sel], bar, k, w->src_row0 + r0, pol_b);
+                break;
+            case kDX:  // [dg | du] rows, K-major
+                tma_load_2d(dst, &mp.m[4], bar, k, w->dst_row0 + r0, pol_b);
+                break;
+            case kDWD:  // h rows read across
+                tma_load_2d(dst, &mp.m[2], bar, r0, w->dst_row0 + k, pol_b);
+                break;
+            case kDWGU:  // x rows (x_perm / x) read across
+                tma_load_2d(dst, &mp.m[2 + w->b_sel], bar, r0, w->src_row0 + k, pol_b);
+                break;
+            case kDWR:  // x read across
+                tma_load_2d(dst, &mp.m[1], bar, r0, k, pol_b);
+                break;
+            default:  // kLOGITS: x rows; kDXR: dl rows (K-major)
+                tma_load_2d(dst, &mp.m[1], bar, k, r0, pol_b);
+                break;
+        }
+    }
+}
+
+// Instruction descriptor of kind::f16 with the operands' majors (bit 15: A
+// MN-major, bit 16: B MN-major).
+__device__ __forceinline__ uint32_t g_idesc(int kind, uint32_t n) {
+    return idesc_bf16_f32(128, n) | (g_a_mn(kind) ? (1u << 15) : 0u) |
+           (g_b_mn(kind) ? (1u << 16) : 0u);
+}
+
+// Shared-memory descriptor of a 128-byte-swizzled operand: K-major (8-row
+// groups 1024 bytes apart) or MN-major (64-element blocks 8 KB apart, 8-row K
+// groups 1024 bytes apart).
+__device__ __forceinline__ uint64_t g_sdesc(uint32_t saddr, bool mn) {
+    uint64_t dsc = 0;
+    dsc |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    dsc |= (uint64_t)((mn ? 8192u : 16u) >> 4) << 16;
+    dsc |= (uint64_t)(1024u >> 4) << 32;
+    dsc |= (uint64_t)1u << 46;
+    dsc |= (uint64_t)2u << 61;
+    return dsc;
+}
+
+
+__device__ __forceinline__ float bits_to_f32(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
+
+// Epilogue of one item: 32 accumulator columns (c0 ...) of TMEM lane `m`
+// (M row m of the tile) in v; `zero`: the item had no K (an expert no token
+// chose: its weight gradient is zero).
+__device__ __forceinline__ void g_store(const GParams &p, const GItem &it, int m, int c0,
+                                        const uint32_t (&v)[32], bool zero) {
+    switch (p.kind) {
+        case kDH: {
+            const ExpertWork &w = p.ent[it.entry];
+            const int i = it.mt * 128 + m;
+            if (i >= p.I) return;
+            uint16_t *dgu = static_cast<uint16_t *>(p.out[0]);
+            const size_t ld = 2 * (size_t)p.I;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int c = c0 + j;
+                if (c >= it.n_valid) continue;
+                const size_t row = (size_t)w.dst_row0 + (size_t)it.nt * it.bn + c;
+                const float g = bits_to_f32(p.gu[row * ld + i]);
+                const float u = bits_to_f32(p.gu[row * ld + p.I + i]);
+                const float dh = __uint_as_float(v[j]);
+                const float s = 1.0f / (1.0f + expf(-g));
+                dgu[row * ld + i] = to_bf16_bits(dh * u * s * (1.0f + g * (1.0f - s)));
+                dgu[row * ld + p.I + i] = to_bf16_bits(dh * g * s);
+            }
+            break;
+        }
+        case kDX: {
+            const ExpertWork &w = p.ent[it.entry];
+            const int jf = it.mt * 128 + m;
+            if (jf >= p.d) return;
+            uint16_t *dxp = static_cast<uint16_t *>(p.out[0]);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int c = c0 + j;
+                if (c >= it.n_valid) continue;
+                const size_t row = (size_t)w.dst_row0 + (size_t)it.nt * it.bn + c;
+                dxp[row * p.d + jf] = to_bf16_bits(__uint_as_float(v[j]));
+            }
+            break;
+        }
+        case kLOGITS: {
+            const int e = it.mt * 128 + m;
+            if (e >= p.N) return;
+            float *l = static_cast<float *>(p.out[0]);
+            const float b = p.bias ? p.bias[e] : 0.0f;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int c = c0 + j;
+                if (c >= it.n_valid) continue;
+                l[(size_t)(it.nt * it.bn + c) * p.N + e] = __uint_as_float(v[j]) + b;
+            }
+            break;
+        }
+        case kDXR: {
+            const int jf = it.mt * 128 + m;
+            if (jf >= p.d) return;
+            float *o = static_cast<float *>(p.out[0]);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int c = c0 + j;
+                if (c >= it.n_valid) continue;
+                o[(size_t)(it.nt * it.bn + c) * p.d + jf] = __uint_as_float(v[j]);
+            }
+            break;
+        }
+        default: {  // weight gradients: row-major [rows][cols] bf16, 32 columns per thread
+            int row, rows, cols;
+            uint16_t *base;
+            if (p.kind == kDWR) {
+                row = it.mt * 128 + m; rows = p.N; cols = p.d;
+                base = static_cast<uint16_t *>(p.out[0]);
+            } else {
+                const ExpertWork &w = p.ent[it.entry];
+                if (p.kind == kDWD) {
+                    row = it.mt * 128 + m; rows = p.d; cols = p.I;
+                    base = static_cast<uint16_t *>(p.out[w.a_sel]);
+                } else {
+                    const int part = it.mt / p.m_tiles;
+                    row = (it.mt - part * p.m_tiles) * 128 + m; rows = p.I; cols = p.d;
+                    base = static_cast<uint16_t *>(p.out[2 * part + w.a_sel]);
+                }
+                base += (size_t)w.a_idx * (size_t)rows * cols;
+            }
+            if (row >= rows) return;
+            const int col0 = it.nt * it.bn + c0;
+            const int lim = min(min(32, it.bn - c0), cols - col0);
+            if (lim <= 0) return;
+            uint16_t *dst = base + (size_t)row * cols + col0;
+            if (lim == 32) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    uint4 o;
+                    o.x = zero ? 0u : pack_bf16x2(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1]));
+                    o.y = zero ? 0u : pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
+                    o.z = zero ? 0u : pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
+                    o.w = zero ? 0u : pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
+                    reinterpret_cast<uint4 *>(dst)[q] = o;
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (j < lim) dst[j] = zero ? (uint16_t)0 : to_bf16_bits(__uint_as_float(v[j]));
+            }
+            break;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kGThreads, 1) bwd_gemm_kernel(const __grid_constant__ GParams p,
+                                                                 const __grid_constant__ GMaps mp) {
+    extern __shared__ __align__(1024) unsigned char smem_dyn[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    unsigned char *stages = smem;
+    GShared &sh = *reinterpret_cast<GShared *>(smem + kGStages * kGStageBytes);
+    volatile int *abort = &sh.abort;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kGStages; ++s) {
+            mbar_init(&sh.full[s], 1);
+            mbar_init(&sh.empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&sh.tfull[a], 1);
+            mbar_init(&sh.tempty[a], 128);
+        }
+        mbar_init(&sh.drain, 1);
+        sh.abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0)
+        for (int i = 0; i < 6; ++i) tma_prefetch_desc(&mp.m[i]);
+    if (warp == 1) {
+        tmem_alloc(&sh.tmem_base, kGTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = sh.tmem_base;
+    grid_dependency_wait();
+    // item count (token kinds: from the plan's token tiles)
+    if (threadIdx.x == 0) {
+        int tot;
+        if (g_token_kind(p.kind)) {
+            tot = 0;
+            for (int e = 0; e < p.n_entries; ++e) {
+                sh.start[e] = tot;
+                tot += p.m_tiles * p.ent[e].ntb;
+            }
+            sh.start[p.n_entries] = tot;
+        } else if (g_wgrad_kind(p.kind)) {
+            tot = p.n_entries * (p.kind == kDWGU ? 2 : 1) * p.m_tiles * p.n_tiles;
+        } else {
+            tot = p.m_tiles * p.n_tiles;
+        }
+        sh.total = tot;
+    }
+    __syncthreads();
+    const int total = sh.total;
+    const bool a_mn = g_a_mn(p.kind), b_mn = g_b_mn(p.kind);
+
+    if (warp == 0) {
+        // ------------------------------------------------------ TMA producer
+        const uint64_t pol_a = policy_evict_first();
+        const uint64_t pol_b = policy_evict_last();
+        int stage = 0;
+        uint32_t phase = 0;
+        uint32_t armed = 0, armed_par = 0;
+        bool ok = true;
+        for (int q = blockIdx.x; q < total && ok; q += gridDim.x) {
+            GItem it;
+            g_decode(p, sh, q, it);
+            const int nbb = (it.bn + 63) / 64;
+            const uint32_t bytes = 16384u + 8192u * (uint32_t)nbb;
+            for (int kc = 0; kc < it.nck; ++kc) {
+                int got = 1;
+                if (lane == 0) got = mbar_wait(&sh.empty[stage], phase ^ 1u, abort);
+                if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
+                unsigned char *sbase = stages + stage * kGStageBytes;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&sh.full[stage], bytes);
+                    armed |= 1u << stage;
+                    armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+                }
+                __syncwarp();
+                if (lane < 2 + nbb) g_load(p, mp, it, kc, lane, sbase, &sh.full[stage], pol_a, pol_b);
+                if (++stage == kGStages) { stage = 0; phase ^= 1u; }
+            }
+        }
+        if (lane == 0 && *abort) {  // let every issued copy land before the CTA can exit
+            for (int s = 0; s < kGStages; ++s)
+                if (armed & (1u << s)) mbar_wait(&sh.full[s], (armed_par >> s) & 1u, nullptr);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------ MMA issuer
+        int stage = 0;
+        uint32_t phase = 0;
+        int i = 0;
+        bool ok = true;
+        for (int q = blockIdx.x; q < total && ok; q += gridDim.x, ++i) {
+            GItem it;
+            g_decode(p, sh, q, it);
+            const int acc = i & 1;
+            int got = 1;
+            if (lane == 0) got = mbar_wait(&sh.tempty[acc], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort);
+            if (!__shfl_sync(0xffffffffu, got, 0)) break;
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + (uint32_t)acc * 256u;
+            const uint32_t idesc = g_idesc(p.kind, (uint32_t)it.bn);
+            for (int kc = 0; kc < it.nck; ++kc) {
+                got = 1;
+                if (lane == 0) got = mbar_wait(&sh.full[stage], phase, abort);
+                if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
+                unsigned char *sbase = stages + stage * kGStageBytes;
+                int steps = 4;
+                if (kc == it.nck - 1 && it.kv_last < 64) {
+                    // ragged K: rows kv_last .. (next multiple of 16) of A hold the
+                    // next expert's rows; zero them, skip the MMAs past them
+                    __syncwarp();  // order the lanes after lane 0's wait (TMA has landed)
+                    const int kv = it.kv_last;
+                    steps = (kv + 15) / 16;
+                    const int nz = 16 * steps - kv;  // rows to clear in each of A's two boxes
+                    for (int z = lane; z < 2 * nz * 8; z += 32) {
+                        const int box = z / (nz * 8), r = (z / 8) % nz, c16 = z % 8;
+                        *reinterpret_cast<uint4 *>(sbase + 8192 * box + (kv + r) * 128 + 16 * c16) =
+                            make_uint4(0u, 0u, 0u, 0u);
+                    }
+                    fence_proxy_async();
+                    __syncwarp();
+                }
+                if (lane == 0) {
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(sbase), sb = sa + 16384u;
+                    for (int j = 0; j < steps; ++j) {
+                        const uint32_t adv_a = a_mn ? 2048u * j : 32u * j;
+                        const uint32_t adv_b = b_mn ? 2048u * j : 32u * j;
+                        tc_mma_bf16(d_tmem, g_sdesc(sa + adv_a, a_mn), g_sdesc(sb + adv_b, b_mn), idesc,
+                                    (kc + j) > 0 ? 1u : 0u);
+                    }
+                    tc_commit(&sh.empty[stage]);
+                }
+                __syncwarp();
+                if (++stage == kGStages) { stage = 0; phase ^= 1u; }
+            }
+            if (!ok) break;
+            if (lane == 0) tc_commit(&sh.tfull[acc]);  // (no MMA: arrives at once)
+            __syncwarp();
+        }
+        if (lane == 0) {
+            tc_commit(&sh.drain);
+            mbar_wait(&sh.drain, 0, nullptr);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------ epilogue
+        const int q4 = warp & 3;
+        const int m = 32 * q4 + lane;
+        int i = 0;
+        for (int q = blockIdx.x; q < total; q += gridDim.x, ++i) {
+            GItem it;
+            g_decode(p, sh, q, it);
+            const int acc = i & 1;
+            if (!mbar_wait(&sh.tfull[acc], (uint32_t)(i >> 1) & 1u, abort)) break;
+            tc_fence_after();
+            const uint32_t tbase = tmem_base + ((uint32_t)(32 * q4) << 16) + (uint32_t)acc * 256u;
+            const bool zero = it.nck == 0;
+            for (int c0 = 0; c0 < it.n_valid; c0 += 32) {
+                uint32_t v[32];
+                if (!zero) {
+                    tmem_ld_32x32b_x32(tbase + (uint32_t)c0, v);
+                    tmem_ld_wait();
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = 0u;
+                }
+                g_store(p, it, m, c0, v, zero);
+            }
+            tc_fence_before();
+            mbar_arrive(&sh.tempty[acc]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, kGTmemCols);
+}
+
+// ---------------------------------------------------------------------------
+// Host side.
+static bool g_rows(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows) {
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {64, 64};
+    return encode(m, base, 2, dims, strides, box);
+}
+static bool g_experts(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint64_t E) {
+    const cuuint64_t dims[3] = {cols, rows, E};
+    const cuuint64_t strides[2] = {cols * 2, cols * rows * 2};
+    const cuuint32_t box[3] = {64, 64, 1};
+    return encode(m, base, 3, dims, strides, box);
+}
+// N tiles of at most 256 columns over n columns, each a multiple of 16 wide
+static void g_ntiles(int n, int &tiles, int &bn) {
+    tiles = (n + 255) / 256;
+    if (tiles < 1) tiles = 1;
+    bn = (((n + tiles - 1) / tiles) + 15) & ~15;
+    if (bn < 16) bn = 16;
+}
+
+static size_t g_smem_bytes() { return 1024 + (size_t)kGStages * kGStageBytes + sizeof(GShared); }
+
+cudaError_t launch_bwd_gemm(int kind, const moge_config &c, const ExpertWork *ent, int n_entries,
+                            const BwdTensors &b, int num_sms, cudaStream_t st) {
+    const int T = c.T, d = c.d, I = c.I, N = c.N, S = c.S;
+    const int K = c.M * c.Kp;
+    const uint64_t rrows = (uint64_t)T * K, hrows = (uint64_t)T * (K + S);
+    // a missing shared side borrows the routed tensors (no entry selects it)
+    const void *sg = S ? b.sg : b.wg, *su = S ? b.su : b.wu, *sd = S ? b.sd : b.wd;
+    const int ns = S ? S : N;
+    GMaps mp;
+    GParams p = {};
+    p.kind = kind;
+    p.ent = ent;
+    p.n_entries = n_entries;
+    p.T = T; p.d = d; p.I = I; p.N = N;
+    bool ok = true;
+    int total = -1;  // unknown on the host (token kinds)
+    switch (kind) {
+        case kDH:
+            ok = g_experts(&mp.m[0], b.wd, I, d, N) && g_experts(&mp.m[1], sd, I, d, ns) &&
+                 g_rows(&mp.m[2], b.dy_perm, d, rrows) && g_rows(&mp.m[3], b.dy, d, T);
+            mp.m[4] = mp.m[5] = mp.m[0];
+            p.m_tiles = (I + 127) / 128;
+            p.kc = (d + 63) / 64;
+            p.out[0] = b.dgu;
+            p.gu = (const uint16_t *)b.gu;
+            break;
+        case kDX:
+            ok = g_experts(&mp.m[0], b.wg, d, I, N) && g_experts(&mp.m[1], sg, d, I, ns) &&
+                 g_experts(&mp.m[2], b.wu, d, I, N) && g_experts(&mp.m[3], su, d, I, ns) &&
+                 g_rows(&mp.m[4], b.dgu, 2 * (uint64_t)I, hrows);
+            mp.m[5] = mp.m[0];
+            p.m_tiles = (d + 127) / 128;
+            p.kc = 2 * I / 64;
+            p.out[0] = b.dx_perm;
+            break;
+        case kDWD:
+            ok = g_rows(&mp.m[0], b.dy_perm, d, rrows) && g_rows(&mp.m[1], b.dy, d, T) &&
+                 g_rows(&mp.m[2], b.h, I, hrows);
+            mp.m[3] = mp.m[4] = mp.m[5] = mp.m[0];
+            p.m_tiles = (d + 127) / 128;
+            g_ntiles(I, p.n_tiles, p.bn);
+            p.out[0] = b.dwd; p.out[1] = b.dsd;
+            total = n_entries * p.m_tiles * p.n_tiles;
+            break;
+        case kDWGU:
+            ok = g_rows(&mp.m[0], b.dgu, 2 * (uint64_t)I, hrows) &&
+                 g_rows(&mp.m[2], b.x_perm, d, rrows) && g_rows(&mp.m[3], b.x, d, T);
+            mp.m[1] = mp.m[4] = mp.m[5] = mp.m[0];
+            p.m_tiles = (I + 127) / 128;
+            g_ntiles(d, p.n_tiles, p.bn);
+            p.out[0] = b.dwg; p.out[1] = b.dsg; p.out[2] = b.dwu; p.out[3] = b.dsu;
+            total = n_entries * 2 * p.m_tiles * p.n_tiles;
+            break;
+        case kLOGITS:
+            ok = g_rows(&mp.m[0], b.w_router, d, N) && g_rows(&mp.m[1], b.x, d, T);
+            mp.m[2] = mp.m[3] = mp.m[4] = mp.m[5] = mp.m[0];
+            p.m_tiles = (N + 127) / 128;
+            p.kc = (d + 63) / 64;
+            g_ntiles(T, p.n_tiles, p.bn);
+            p.out[0] = b.logits;
+            p.bias = b.bias;
+            total = p.m_tiles * p.n_tiles;
+            break;
+        case kDWR:
+            ok = g_rows(&mp.m[0], b.dl, N, T) && g_rows(&mp.m[1], b.x, d, T);
+            mp.m[2] = mp.m[3] = mp.m[4] = mp.m[5] = mp.m[0];
+            p.m_tiles = (N + 127) / 128;
+            g_ntiles(d, p.n_tiles, p.bn);
+            p.out[0] = b.dwr;
+            total = p.m_tiles * p.n_tiles;
+            break;
+        case kDXR:
+            ok = g_rows(&mp.m[0], b.w_router, d, N) && g_rows(&mp.m[1], b.dl, N, T);
+            mp.m[2] = mp.m[3] = mp.m[4] = mp.m[5] = mp.m[0];
+            p.m_tiles = (d + 127) / 128;
+            p.kc = (N + 63) / 64;
+            g_ntiles(T, p.n_tiles, p.bn);
+            p.out[0] = b.dx_r;
+            total = p.m_tiles * p.n_tiles;
+            break;
+        default:
+            return cudaErrorInvalidValue;
+    }
+    if (!ok) return cudaErrorInvalidValue;
+    if (total == 0) return cudaSuccess;
+    const int grid = total < 0 ? num_sms : (total < num_sms ? total : num_sms);
+    const size_t smem = g_smem_bytes();
+    cudaError_t e = cudaFuncSetAttribute(bwd_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(bwd_gemm_kernel, dim3(grid), dim3(kGThreads), smem, st, p, mp);
+}
+
+}  // namespace moge

@@ -67,6 +67,7 @@ struct TcParams {
     uint16_t *h;         // [rows][I]
     uint16_t *y;         // [rows][d]
     int *sync;           // [0] queue counter, [1 + e] finished up items of entry e
+    uint16_t *gu;        // null, or [rows][2I]: the up-projection's g and u (training forward)
 };
 
 struct TcItem {
@@ -391,6 +392,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
                     const bool gate_hi = p.gu_mode[it.w.a_sel] == kUpGateFused;
                     const bool is_gate = (q4 < 2) != gate_hi;
                     const int f = (q4 & 1) * 32 + lane;
+                    if (p.gu && it.fb * 64 + f < p.I) {  // keep g / u for the backward pass
+                        uint16_t *dst = p.gu + (row0 + c0) * 2 * (size_t)p.I + (is_gate ? 0 : p.I) +
+                                        it.fb * 64 + f;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (c0 + j < it.n_valid)
+                                dst[(size_t)j * 2 * p.I] = to_bf16_bits(__uint_as_float(v[j]));
+                    }
                     if (!is_gate) {
 #pragma unroll
                         for (int j = 0; j < 32; ++j) U[j * 64 + f] = __uint_as_float(v[j]);
@@ -537,6 +546,7 @@ cudaError_t launch_ffn_tc(const moge_config &c, const Plan &plan, int n_entries,
     p.h = (uint16_t *)op.h;
     p.y = (uint16_t *)op.y;
     p.sync = plan.sync;
+    p.gu = (uint16_t *)op.gu;
 
     const size_t smem = tc_smem_bytes();
     cudaError_t e = cudaFuncSetAttribute(ffn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

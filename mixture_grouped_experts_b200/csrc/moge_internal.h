@@ -124,6 +124,9 @@ struct FfnOperands {
     void *h;                 // [h_rows][I]
     int64_t h_rows;
     void *y;                 // [h_rows][d]
+    // Optional (bf16 tensor-core FFN only, training forward): the
+    // up-projection's pre-activations, [h_rows][2I] = [g | u] per row.
+    void *gu;
     // FP8 weights only (launch_ffn_fp8): the w*/s* pointers above are E4M3
     // codes and these their per-row fp32 scales ([E][I], [E][I], [E][d])
     const float *wg_s, *wu_s, *wd_s;
@@ -138,6 +141,41 @@ cudaError_t launch_ffn_f32(const moge_config &c, const Plan &plan, int n_entries
 // grouped FFN with FP8 (E4M3, per-row scale) weights and bf16 activations
 cudaError_t launch_ffn_fp8(const moge_config &c, const Plan &plan, int n_entries,
                            const FfnOperands &op, int num_sms, cudaStream_t st);
+
+// ---------------------------------------------------------------- backward
+// Tensors of the backward pass (bf16 unless noted; rows as in the forward:
+// rrows = T*K routed rows in permuted order, hrows = T*(K+S) with the shared
+// experts' rows after the routed ones).
+struct BwdTensors {
+    const void *x, *w_router;            // [T][d], [N][d]
+    const float *bias;                   // [N] or null
+    const void *wg, *wu, *wd;            // routed weights [N][I][d], [N][I][d], [N][d][I]
+    const void *sg, *su, *sd;            // shared weights (null when S == 0)
+    const void *x_perm, *h;              // [rrows][d], [hrows][I]   (forward)
+    const void *gu;                      // [hrows][2I] pre-activations [g | u] (forward)
+    const void *dy, *dy_perm;            // [T][d], [rrows][d]
+    void *dgu;                           // [hrows][2I] (may alias gu)
+    void *dx_perm;                       // [hrows][d]
+    float *logits;                       // [T][N] fp32
+    void *dl;                            // [T][N]
+    float *dx_r;                         // [T][d] fp32
+    void *dwg, *dwu, *dwd, *dsg, *dsu, *dsd, *dwr;  // weight gradients (layouts of the weights)
+};
+// GEMM kinds of the backward pass: dh (with the SwiGLU backward), dx, dW_down,
+// dW_gate / dW_up, the router's logits, dW_router, the router's share of dx
+enum : int { kDH = 0, kDX = 1, kDWD = 2, kDWGU = 3, kLOGITS = 4, kDWR = 5, kDXR = 6 };
+cudaError_t launch_bwd_gemm(int kind, const moge_config &c, const ExpertWork *ent, int n_entries,
+                            const BwdTensors &b, int num_sms, cudaStream_t st);
+cudaError_t launch_combine_bwd(const moge_config &c, const void *dy, const void *y_perm,
+                               const float *topk_w, const int32_t *perm_dst, void *dy_perm,
+                               float *dw, cudaStream_t st);
+int router_bwd_parts(const moge_config &c);
+cudaError_t launch_router_bwd(const moge_config &c, float alpha, const float *logits,
+                              const int32_t *topk_idx, const float *dw, const int32_t *counts,
+                              void *dl, float *part, float *aux, cudaStream_t st);
+cudaError_t launch_unpermute_bwd(const moge_config &c, const void *dx_perm, const int32_t *perm_dst,
+                                 const float *dx_r, void *dx, cudaStream_t st);
+
 // kernel whose bounded waits run out after limit_ns (failure-path check)
 cudaError_t launch_wait_selftest(int32_t *out, uint64_t limit_ns, cudaStream_t st);
 // per-row FP8 quantisation of bf16 rows

@@ -66,7 +66,8 @@ def _l():
                                          vp, i32, vp, vp, vp, vp]
         lib.oracle_layer_backward.argtypes = [vp, i32, i32, i32, i32, i32, i32, i32, i32,
                                               vp, vp, vp, vp, vp, vp, vp, vp, vp,
-                                              ctypes.c_double, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+                                              ctypes.c_double, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                              vp]
         _lib = lib
     return _lib
 
@@ -204,9 +205,10 @@ def layer(x: np.ndarray, inp: dict, M: int, Kp: int, dtype: str,
 
 
 def layer_backward(x: np.ndarray, inp: dict, M: int, Kp: int, dtype: str, dy: np.ndarray,
-                   alpha: float = 0.0) -> dict:
+                   alpha: float = 0.0, idx: Optional[np.ndarray] = None) -> dict:
     """Gradients of sum_t dy_t . y_t + L_aux (routing held fixed) -- oracle.c,
-    oracle_layer_backward. x, dy: float64 [T][d]. Returns float64 arrays
+    oracle_layer_backward. x, dy: float64 [T][d]; idx: optional picks [T][M*Kp]
+    to hold the routing at (default: the oracle's own). Returns float64 arrays
     dx [T][d], w_router [N][d], w_gate/w_up [N][I][d], w_down [N][d][I],
     s_gate/s_up [S][I][d], s_down [S][d][I], and the scalar aux."""
     x = np.ascontiguousarray(x, np.float64)
@@ -223,9 +225,10 @@ def layer_backward(x: np.ndarray, inp: dict, M: int, Kp: int, dtype: str, dy: np
            "w_gate": np.empty((N, I, d)), "w_up": np.empty((N, I, d)), "w_down": np.empty((N, d, I)),
            "s_gate": np.empty((S, I, d)), "s_up": np.empty((S, I, d)), "s_down": np.empty((S, d, I))}
     aux = np.zeros(1)
+    picks = None if idx is None else np.ascontiguousarray(idx, np.int32)
     _chk(_l().oracle_layer_backward(_p(x), T, d, N, M, Kp, S, I, _DT[dtype], _p(wr), _p(b),
                                     _p(wg), _p(wu), _p(wd), _p(sg), _p(su), _p(sd), _p(dy),
-                                    float(alpha), _p(out["dx"]), _p(out["w_router"]),
+                                    float(alpha), _p(picks), _p(out["dx"]), _p(out["w_router"]),
                                     _p(out["w_gate"]), _p(out["w_up"]), _p(out["w_down"]),
                                     _p(out["s_gate"]), _p(out["s_up"]), _p(out["s_down"]),
                                     _p(aux)), "layer_backward")

@@ -496,6 +496,9 @@ int oracle_layer_fp8(const double *x, int T, int d, int N, int M, int Kp, int S,
  * then, with dp[t][i] += alpha * f_i / T for every expert i,
  *   dl[t][i]  = p[t][i] (dp[t][i] - sum_j p[t][j] dp[t][j])   (softmax)
  *   dWr[i]   += dl[t][i] x_t,   dx_t += sum_i dl[t][i] Wr[i].
+ * idx_in (may be NULL): picks [T][M*Kp] to hold the routing at instead of the
+ * oracle's own selection (tokens whose top scores tie within rounding have
+ * more than one correct pick; each must lie in its group).
  * Every output array is overwritten. Shapes: dx [T][d], dwr [N][d],
  * dwg/dwu [N][I][d], dwd [N][d][I], dsg/dsu [S][I][d], dsd [S][d][I].
  * aux_out (may be NULL) receives L_aux.
@@ -504,7 +507,8 @@ int oracle_layer_backward(const double *x, int T, int d, int N, int M, int Kp, i
                           int dtype, const void *w_router, const float *bias,
                           const void *w_gate, const void *w_up, const void *w_down,
                           const void *s_gate, const void *s_up, const void *s_down,
-                          const double *dy, double alpha, double *dx, double *dwr, double *dwg,
+                          const double *dy, double alpha, const int32_t *idx_in, double *dx,
+                          double *dwr, double *dwg,
                           double *dwu, double *dwd, double *dsg, double *dsu, double *dsd,
                           double *aux_out) {
     if (T < 0 || N <= 0 || M <= 0 || N % M != 0 || Kp < 1 || Kp > N / M) return 1;
@@ -537,6 +541,16 @@ int oracle_layer_backward(const double *x, int T, int d, int N, int M, int Kp, i
     }
     int rc = oracle_router_probs(x, w_router, bias, dtype, T, d, N, p);
     if (!rc) rc = oracle_select_grouped(p, T, N, M, Kp, idx, wk, NULL);
+    if (!rc && idx_in) {
+        const int G = N / M;
+        for (int t = 0; t < T && !rc; ++t)
+            for (int k = 0; k < K; ++k) {
+                const int e = idx_in[(size_t)t * K + k];
+                if (e < (k / Kp) * G || e >= (k / Kp + 1) * G) { rc = 1; break; }
+                idx[(size_t)t * K + k] = e;
+                wk[(size_t)t * K + k] = p[(size_t)t * N + e];
+            }
+    }
     double aux = 0.0;
     if (!rc && T > 0) {
         for (size_t i = 0; i < (size_t)T * K; ++i) f[idx[i]] += 1.0 / T;

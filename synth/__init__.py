@@ -29,6 +29,7 @@ _LIB = os.path.join(_HERE, "libsynth.so")
 # tensor stream ids; a layer l of a stack adds 16 * l
 STREAM_X, STREAM_WR, STREAM_WG, STREAM_WU, STREAM_WD = 1, 2, 3, 4, 5
 STREAM_SG, STREAM_SU, STREAM_SD = 6, 7, 8
+STREAM_DY = 9  # upstream gradient of the backward pass
 
 
 def build(force: bool = False) -> str:
@@ -163,3 +164,9 @@ def layer_inputs(cfg: Config, layer: int = 0, x_stream_offset: int = 0,
     out["s_down"] = normal(cfg.seed, STREAM_SD + base, S * d * I, cfg.w_std, dt).reshape(S, d, I)
     out["logit_bias"] = zipf_bias(cfg)
     return out
+
+
+def upstream_grad(cfg: Config, std: float = 1.0) -> np.ndarray:
+    """Seeded upstream gradient dy [T][d] for the backward pass (bf16 bit
+    patterns for bf16 configs, float32 otherwise)."""
+    return normal(cfg.seed, STREAM_DY, cfg.T * cfg.d, std, cfg.dtype).reshape(cfg.T, cfg.d)

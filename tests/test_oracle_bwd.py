@@ -107,3 +107,25 @@ def test_router_gradient_rows_sum_to_zero_and_linearity():
     assert np.abs(g1["w_router"].sum(0)).max() < 1e-12
     for k in ("dx",) + WEIGHTS:
         np.testing.assert_allclose(g2[k], 2.0 * g1[k], rtol=1e-12, atol=1e-14)
+
+
+def test_routing_override():
+    # held at its own picks the override changes nothing; at another valid pick
+    # of a group the gradients move; a pick outside its group is refused
+    inp = synth.layer_inputs(SMALL)
+    x = oracle.to_double(inp["x"], "f32")
+    dy = np.random.default_rng(6).normal(size=x.shape)
+    _, idx, _, _ = oracle.layer(x, inp, SMALL.M, SMALL.Kp, "f32")
+    a = oracle.layer_backward(x, inp, SMALL.M, SMALL.Kp, "f32", dy, 0.2)
+    b = oracle.layer_backward(x, inp, SMALL.M, SMALL.Kp, "f32", dy, 0.2, idx=idx)
+    for k in ("dx",) + WEIGHTS:
+        assert np.array_equal(a[k], b[k])
+    G = SMALL.N // SMALL.M
+    other = idx.copy()
+    other[0, 0] = (other[0, 0] + 1) % G  # group 0 holds experts 0 .. G-1
+    c = oracle.layer_backward(x, inp, SMALL.M, SMALL.Kp, "f32", dy, 0.2, idx=other)
+    assert not np.array_equal(a["w_gate"], c["w_gate"])
+    bad = idx.copy()
+    bad[0, 0] = SMALL.N - 1
+    with pytest.raises(ValueError):
+        oracle.layer_backward(x, inp, SMALL.M, SMALL.Kp, "f32", dy, 0.2, idx=bad)
