@@ -38,9 +38,12 @@ constexpr int kGStageBytes = 48 * 1024;  // A: 2 boxes (16 KB), B: up to 4 boxes
 constexpr int kGThreads = 192;
 constexpr uint32_t kGTmemCols = 512;
 constexpr int kGMaxEntries = kMaxExperts + 64;
+constexpr int kGEpiBytes = 4 * 2 * 2048;  // per epilogue warp: two [32][32] bf16 staging tiles
 
+// m[0..5]: operand maps (per kind); m[6..9]: weight-gradient outputs, stored
+// by TMA from a staging tile ([32 rows][32 cols] bf16 per epilogue warp)
 struct GMaps {
-    CUtensorMap m[6];
+    CUtensorMap m[10];
 };
 
 struct GParams {
@@ -51,6 +54,8 @@ struct GParams {
     int m_tiles;            // M tiles per entry (per part for kDWGU)
     int n_tiles, bn;        // weight-gradient and router kinds: N tiles and their width
     int kc;                 // K chunks of the fixed-K kinds
+    int nst;                // pipeline stages in use (3 for the weight-gradient kinds, whose
+                            // freed stage holds the epilogue's store staging tiles)
     void *out[4];
     const uint16_t *gu;     // kDH: [rows][2I]
     const float *bias;      // kLOGITS, nullable
@@ -200,46 +205,85 @@ __device__ __forceinline__ uint64_t g_sdesc(uint32_t saddr, bool mn) {
 
 __device__ __forceinline__ float bits_to_f32(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
 
+// Epilogue of the token kinds for one 32-column chunk (32 rows of the expert):
+// every epilogue thread stages its feature's 32 values in S (row-major
+// [32 rows][128 features], fp32), then each thread takes 16-byte vectors of
+// 8 features of one row. kDH: dg, du from dh and the saved g, u (read as
+// vectors before any store: dgu overwrites gu in place); kDX: dx_perm rows.
+__device__ __forceinline__ void g_store_rows(const GParams &p, const GItem &it, int m, int et,
+                                             int c0, const uint32_t (&v)[32], float *S) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) S[j * 128 + m] = __uint_as_float(v[j]);
+    named_bar_sync(1, 128);
+    const ExpertWork &w = p.ent[it.entry];
+    const size_t row_base = (size_t)w.dst_row0 + (size_t)it.nt * it.bn + c0;
+    const int f0 = it.mt * 128;
+    if (p.kind == kDH) {
+        const size_t ld = 2 * (size_t)p.I;
+        uint4 gv[4], uv[4];
+        bool ok[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int idx = et + 128 * q, j = idx >> 4, fv = (idx & 15) * 8;
+            ok[q] = c0 + j < it.n_valid && f0 + fv < p.I;
+            if (ok[q]) {
+                const uint16_t *src = p.gu + (row_base + j) * ld + f0 + fv;
+                gv[q] = *reinterpret_cast<const uint4 *>(src);
+                uv[q] = *reinterpret_cast<const uint4 *>(src + p.I);
+            }
+        }
+        uint16_t *dgu = static_cast<uint16_t *>(p.out[0]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            if (!ok[q]) continue;
+            const int idx = et + 128 * q, j = idx >> 4, fv = (idx & 15) * 8;
+            const float4 d0 = *reinterpret_cast<const float4 *>(S + j * 128 + fv);
+            const float4 d1 = *reinterpret_cast<const float4 *>(S + j * 128 + fv + 4);
+            const float dh[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+            const uint32_t gw[4] = {gv[q].x, gv[q].y, gv[q].z, gv[q].w};
+            const uint32_t uw[4] = {uv[q].x, uv[q].y, uv[q].z, uv[q].w};
+            uint32_t og[4], ou[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                float dg2[2], du2[2];
+#pragma unroll
+                for (int b = 0; b < 2; ++b) {
+                    const float g = b ? bf16_hi(gw[h]) : bf16_lo(gw[h]);
+                    const float u = b ? bf16_hi(uw[h]) : bf16_lo(uw[h]);
+                    const float sg = 1.0f / (1.0f + expf(-g));
+                    const float x = dh[2 * h + b];
+                    dg2[b] = x * u * sg * (1.0f + g * (1.0f - sg));
+                    du2[b] = x * g * sg;
+                }
+                og[h] = pack_bf16x2(dg2[0], dg2[1]);
+                ou[h] = pack_bf16x2(du2[0], du2[1]);
+            }
+            uint16_t *dst = dgu + (row_base + j) * ld + f0 + fv;
+            *reinterpret_cast<uint4 *>(dst) = make_uint4(og[0], og[1], og[2], og[3]);
+            *reinterpret_cast<uint4 *>(dst + p.I) = make_uint4(ou[0], ou[1], ou[2], ou[3]);
+        }
+    } else {  // kDX
+        uint16_t *dxp = static_cast<uint16_t *>(p.out[0]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int idx = et + 128 * q, j = idx >> 4, fv = (idx & 15) * 8;
+            if (c0 + j >= it.n_valid || f0 + fv >= p.d) continue;
+            const float4 a = *reinterpret_cast<const float4 *>(S + j * 128 + fv);
+            const float4 b = *reinterpret_cast<const float4 *>(S + j * 128 + fv + 4);
+            *reinterpret_cast<uint4 *>(dxp + (row_base + j) * p.d + f0 + fv) =
+                make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y),
+                           pack_bf16x2(b.z, b.w));
+        }
+    }
+    named_bar_sync(1, 128);  // S is rewritten by the next chunk
+}
+
 // Epilogue of one item: 32 accumulator columns (c0 ...) of TMEM lane `m`
 // (M row m of the tile) in v; `zero`: the item had no K (an expert no token
 // chose: its weight gradient is zero).
 __device__ __forceinline__ void g_store(const GParams &p, const GItem &it, int m, int c0,
                                         const uint32_t (&v)[32], bool zero) {
     switch (p.kind) {
-        case kDH: {
-            const ExpertWork &w = p.ent[it.entry];
-            const int i = it.mt * 128 + m;
-            if (i >= p.I) return;
-            uint16_t *dgu = static_cast<uint16_t *>(p.out[0]);
-            const size_t ld = 2 * (size_t)p.I;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int c = c0 + j;
-                if (c >= it.n_valid) continue;
-                const size_t row = (size_t)w.dst_row0 + (size_t)it.nt * it.bn + c;
-                const float g = bits_to_f32(p.gu[row * ld + i]);
-                const float u = bits_to_f32(p.gu[row * ld + p.I + i]);
-                const float dh = __uint_as_float(v[j]);
-                const float s = 1.0f / (1.0f + expf(-g));
-                dgu[row * ld + i] = to_bf16_bits(dh * u * s * (1.0f + g * (1.0f - s)));
-                dgu[row * ld + p.I + i] = to_bf16_bits(dh * g * s);
-            }
-            break;
-        }
-        case kDX: {
-            const ExpertWork &w = p.ent[it.entry];
-            const int jf = it.mt * 128 + m;
-            if (jf >= p.d) return;
-            uint16_t *dxp = static_cast<uint16_t *>(p.out[0]);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int c = c0 + j;
-                if (c >= it.n_valid) continue;
-                const size_t row = (size_t)w.dst_row0 + (size_t)it.nt * it.bn + c;
-                dxp[row * p.d + jf] = to_bf16_bits(__uint_as_float(v[j]));
-            }
-            break;
-        }
         case kLOGITS: {
             const int e = it.mt * 128 + m;
             if (e >= p.N) return;
@@ -265,46 +309,73 @@ __device__ __forceinline__ void g_store(const GParams &p, const GItem &it, int m
             }
             break;
         }
-        default: {  // weight gradients: row-major [rows][cols] bf16, 32 columns per thread
-            int row, rows, cols;
-            uint16_t *base;
-            if (p.kind == kDWR) {
-                row = it.mt * 128 + m; rows = p.N; cols = p.d;
-                base = static_cast<uint16_t *>(p.out[0]);
-            } else {
-                const ExpertWork &w = p.ent[it.entry];
-                if (p.kind == kDWD) {
-                    row = it.mt * 128 + m; rows = p.d; cols = p.I;
-                    base = static_cast<uint16_t *>(p.out[w.a_sel]);
-                } else {
-                    const int part = it.mt / p.m_tiles;
-                    row = (it.mt - part * p.m_tiles) * 128 + m; rows = p.I; cols = p.d;
-                    base = static_cast<uint16_t *>(p.out[2 * part + w.a_sel]);
-                }
-                base += (size_t)w.a_idx * (size_t)rows * cols;
-            }
-            if (row >= rows) return;
-            const int col0 = it.nt * it.bn + c0;
-            const int lim = min(min(32, it.bn - c0), cols - col0);
-            if (lim <= 0) return;
-            uint16_t *dst = base + (size_t)row * cols + col0;
-            if (lim == 32) {
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint4 o;
-                    o.x = zero ? 0u : pack_bf16x2(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1]));
-                    o.y = zero ? 0u : pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
-                    o.z = zero ? 0u : pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
-                    o.w = zero ? 0u : pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
-                    reinterpret_cast<uint4 *>(dst)[q] = o;
-                }
-            } else {
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    if (j < lim) dst[j] = zero ? (uint16_t)0 : to_bf16_bits(__uint_as_float(v[j]));
-            }
+        default:  // weight gradients: staged and stored by TMA (g_store_wgrad)
             break;
+    }
+}
+
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap *m, const void *src, int c0, int c1,
+                                             int c2) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];"
+                 ::"l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// at most one committed store group may still be reading shared memory
+__device__ __forceinline__ void bulk_wait_read_1() {
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read_7() {
+    asm volatile("cp.async.bulk.wait_group.read 7;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Weight-gradient epilogue of one 32-column chunk for one warp: lane r holds
+// row (32 q4 + r) of the tile; the warp writes its [32][32] bf16 block into a
+// staging tile (a ring of 8 per warp, or 2 when no stage was freed: `deep`)
+// and lane 0 stores it with TMA.
+// Rows and columns past the tensor are clipped by the copy.
+__device__ __forceinline__ void g_store_wgrad(const GParams &p, const GMaps &mp, const GItem &it,
+                                              int q4, int lane, int c0, const uint32_t (&v)[32],
+                                              unsigned char *stage_tile, bool deep) {
+    const CUtensorMap *map;
+    int row0, e, rows, cols;
+    if (p.kind == kDWR) {
+        map = &mp.m[6]; row0 = it.mt * 128; e = 0; rows = p.N; cols = p.d;
+    } else {
+        const ExpertWork &w = p.ent[it.entry];
+        e = w.a_idx;
+        if (p.kind == kDWD) {
+            map = &mp.m[6 + w.a_sel]; row0 = it.mt * 128; rows = p.d; cols = p.I;
+        } else {
+            const int part = it.mt / p.m_tiles;
+            map = &mp.m[6 + 2 * part + w.a_sel]; row0 = (it.mt - part * p.m_tiles) * 128;
+            rows = p.I; cols = p.d;
         }
+    }
+    row0 += 32 * q4;
+    const int col0 = it.nt * it.bn + c0;
+    if (row0 >= rows || col0 >= cols) return;  // wholly past the tensor: nothing to store
+    if (lane == 0) {  // this staging tile's previous store has read it
+        if (deep) bulk_wait_read_7(); else bulk_wait_read_1();
+    }
+    __syncwarp();
+    // 64-byte swizzle (the map's): 16-byte chunk q of row r at q ^ ((r >> 1) & 3)
+    uint4 *dst = reinterpret_cast<uint4 *>(stage_tile + lane * 64);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint4 o;
+        o.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1]));
+        o.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
+        o.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
+        o.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
+        dst[q ^ ((lane >> 1) & 3)] = o;
+    }
+    fence_proxy_async();
+    __syncwarp();
+    if (lane == 0) {
+        tma_store_3d(map, stage_tile, col0, row0, e);
+        bulk_commit();
     }
 }
 
@@ -314,7 +385,8 @@ __global__ void __launch_bounds__(kGThreads, 1) bwd_gemm_kernel(const __grid_con
     unsigned char *smem = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
     unsigned char *stages = smem;
-    GShared &sh = *reinterpret_cast<GShared *>(smem + kGStages * kGStageBytes);
+    unsigned char *epi = smem + kGStages * kGStageBytes;
+    GShared &sh = *reinterpret_cast<GShared *>(epi + kGEpiBytes);
     volatile int *abort = &sh.abort;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -332,7 +404,7 @@ __global__ void __launch_bounds__(kGThreads, 1) bwd_gemm_kernel(const __grid_con
         fence_barrier_init();
     }
     if (warp == 0 && lane == 0)
-        for (int i = 0; i < 6; ++i) tma_prefetch_desc(&mp.m[i]);
+        for (int i = 0; i < 10; ++i) tma_prefetch_desc(&mp.m[i]);
     if (warp == 1) {
         tmem_alloc(&sh.tmem_base, kGTmemCols);
         tmem_relinquish();
@@ -362,6 +434,7 @@ __global__ void __launch_bounds__(kGThreads, 1) bwd_gemm_kernel(const __grid_con
     __syncthreads();
     const int total = sh.total;
     const bool a_mn = g_a_mn(p.kind), b_mn = g_b_mn(p.kind);
+    const int nst = p.nst;
 
     if (warp == 0) {
         // ------------------------------------------------------ TMA producer
@@ -388,7 +461,7 @@ __global__ void __launch_bounds__(kGThreads, 1) bwd_gemm_kernel(const __grid_con
                 }
                 __syncwarp();
                 if (lane < 2 + nbb) g_load(p, mp, it, kc, lane, sbase, &sh.full[stage], pol_a, pol_b);
-                if (++stage == kGStages) { stage = 0; phase ^= 1u; }
+                if (++stage == nst) { stage = 0; phase ^= 1u; }
             }
         }
         if (lane == 0 && *abort) {  // let every issued copy land before the CTA can exit
@@ -444,7 +517,7 @@ __global__ void __launch_bounds__(kGThreads, 1) bwd_gemm_kernel(const __grid_con
                     tc_commit(&sh.empty[stage]);
                 }
                 __syncwarp();
-                if (++stage == kGStages) { stage = 0; phase ^= 1u; }
+                if (++stage == nst) { stage = 0; phase ^= 1u; }
             }
             if (!ok) break;
             if (lane == 0) tc_commit(&sh.tfull[acc]);  // (no MMA: arrives at once)
@@ -459,7 +532,15 @@ __global__ void __launch_bounds__(kGThreads, 1) bwd_gemm_kernel(const __grid_con
         // ------------------------------------------------------ epilogue
         const int q4 = warp & 3;
         const int m = 32 * q4 + lane;
-        int i = 0;
+        const bool wgrad = g_wgrad_kind(p.kind) || p.kind == kDWR;
+        const bool rowk = g_token_kind(p.kind);
+        const int et = threadIdx.x - 64;
+        // weight-gradient staging: the freed 4th stage and the epilogue area (64 KB,
+        // 16 KB per warp) when 3 stages run, else the epilogue area alone
+        const bool deep = nst < kGStages;
+        unsigned char *wstage = deep ? stages + (size_t)nst * kGStageBytes : epi;
+        const int nbuf = deep ? 8 : 2;
+        int i = 0, chunk = 0;
         for (int q = blockIdx.x; q < total; q += gridDim.x, ++i) {
             GItem it;
             g_decode(p, sh, q, it);
@@ -477,11 +558,21 @@ __global__ void __launch_bounds__(kGThreads, 1) bwd_gemm_kernel(const __grid_con
 #pragma unroll
                     for (int j = 0; j < 32; ++j) v[j] = 0u;
                 }
-                g_store(p, it, m, c0, v, zero);
+                if (wgrad) {
+                    g_store_wgrad(p, mp, it, q4, lane, c0, v,
+                                  wstage + (size_t)(q4 * nbuf + chunk % nbuf) * 2048, deep);
+                    ++chunk;
+                } else if (rowk) {
+                    g_store_rows(p, it, m, et, c0, v, reinterpret_cast<float *>(epi));
+                } else {
+                    g_store(p, it, m, c0, v, zero);
+                }
             }
             tc_fence_before();
             mbar_arrive(&sh.tempty[acc]);
         }
+        if (lane == 0) bulk_wait_all();  // every gradient store has completed
+        __syncwarp();
     }
 
     tc_fence_before();
@@ -505,14 +596,28 @@ static bool g_experts(CUtensorMap *m, const void *base, uint64_t cols, uint64_t 
     return encode(m, base, 3, dims, strides, box);
 }
 // N tiles of at most 256 columns over n columns, each a multiple of 16 wide
-static void g_ntiles(int n, int &tiles, int &bn) {
+static void g_ntiles(int n, int &tiles, int &bn, int align = 16) {
     tiles = (n + 255) / 256;
     if (tiles < 1) tiles = 1;
-    bn = (((n + tiles - 1) / tiles) + 15) & ~15;
-    if (bn < 16) bn = 16;
+    bn = (((n + tiles - 1) / tiles) + align - 1) / align * align;
+    if (bn < align) bn = align;
+}
+// bf16 [E][rows][cols] gradient written in [32 rows][32 cols] boxes (64-byte swizzle)
+static bool g_out(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint64_t E) {
+    EncodeTiledFn fn = get_encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {cols, rows, E};
+    const cuuint64_t strides[2] = {cols * 2, cols * rows * 2};
+    const cuuint32_t box[3] = {32, 32, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-static size_t g_smem_bytes() { return 1024 + (size_t)kGStages * kGStageBytes + sizeof(GShared); }
+static size_t g_smem_bytes() {
+    return 1024 + (size_t)kGStages * kGStageBytes + kGEpiBytes + sizeof(GShared);
+}
 
 cudaError_t launch_bwd_gemm(int kind, const moge_config &c, const ExpertWork *ent, int n_entries,
                             const BwdTensors &b, int num_sms, cudaStream_t st) {
@@ -552,18 +657,22 @@ cudaError_t launch_bwd_gemm(int kind, const moge_config &c, const ExpertWork *en
         case kDWD:
             ok = g_rows(&mp.m[0], b.dy_perm, d, rrows) && g_rows(&mp.m[1], b.dy, d, T) &&
                  g_rows(&mp.m[2], b.h, I, hrows);
+            ok = ok && g_out(&mp.m[6], b.dwd, I, d, N) && g_out(&mp.m[7], S ? b.dsd : b.dwd, I, d, ns);
             mp.m[3] = mp.m[4] = mp.m[5] = mp.m[0];
+            mp.m[8] = mp.m[9] = mp.m[6];
             p.m_tiles = (d + 127) / 128;
-            g_ntiles(I, p.n_tiles, p.bn);
+            g_ntiles(I, p.n_tiles, p.bn, 32);
             p.out[0] = b.dwd; p.out[1] = b.dsd;
             total = n_entries * p.m_tiles * p.n_tiles;
             break;
         case kDWGU:
             ok = g_rows(&mp.m[0], b.dgu, 2 * (uint64_t)I, hrows) &&
                  g_rows(&mp.m[2], b.x_perm, d, rrows) && g_rows(&mp.m[3], b.x, d, T);
+            ok = ok && g_out(&mp.m[6], b.dwg, d, I, N) && g_out(&mp.m[7], S ? b.dsg : b.dwg, d, I, ns) &&
+                 g_out(&mp.m[8], b.dwu, d, I, N) && g_out(&mp.m[9], S ? b.dsu : b.dwu, d, I, ns);
             mp.m[1] = mp.m[4] = mp.m[5] = mp.m[0];
             p.m_tiles = (I + 127) / 128;
-            g_ntiles(d, p.n_tiles, p.bn);
+            g_ntiles(d, p.n_tiles, p.bn, 32);
             p.out[0] = b.dwg; p.out[1] = b.dsg; p.out[2] = b.dwu; p.out[3] = b.dsu;
             total = n_entries * 2 * p.m_tiles * p.n_tiles;
             break;
@@ -578,10 +687,12 @@ cudaError_t launch_bwd_gemm(int kind, const moge_config &c, const ExpertWork *en
             total = p.m_tiles * p.n_tiles;
             break;
         case kDWR:
-            ok = g_rows(&mp.m[0], b.dl, N, T) && g_rows(&mp.m[1], b.x, d, T);
+            ok = g_rows(&mp.m[0], b.dl, N, T) && g_rows(&mp.m[1], b.x, d, T) &&
+                 g_out(&mp.m[6], b.dwr, d, N, 1);
             mp.m[2] = mp.m[3] = mp.m[4] = mp.m[5] = mp.m[0];
+            mp.m[7] = mp.m[8] = mp.m[9] = mp.m[6];
             p.m_tiles = (N + 127) / 128;
-            g_ntiles(d, p.n_tiles, p.bn);
+            g_ntiles(d, p.n_tiles, p.bn, 32);
             p.out[0] = b.dwr;
             total = p.m_tiles * p.n_tiles;
             break;
@@ -598,6 +709,9 @@ cudaError_t launch_bwd_gemm(int kind, const moge_config &c, const ExpertWork *en
             return cudaErrorInvalidValue;
     }
     if (!ok) return cudaErrorInvalidValue;
+    p.nst = (kind == kDWD || kind == kDWGU || kind == kDWR) ? 3 : kGStages;
+    if (kind == kDH || kind == kDX || kind == kLOGITS || kind == kDXR)
+        mp.m[6] = mp.m[7] = mp.m[8] = mp.m[9] = mp.m[0];  // no gradient output (never stored to)
     if (total == 0) return cudaSuccess;
     const int grid = total < 0 ? num_sms : (total < num_sms ? total : num_sms);
     const size_t smem = g_smem_bytes();

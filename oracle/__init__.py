@@ -66,8 +66,10 @@ def _l():
                                          vp, i32, vp, vp, vp, vp]
         lib.oracle_layer_backward.argtypes = [vp, i32, i32, i32, i32, i32, i32, i32, i32,
                                               vp, vp, vp, vp, vp, vp, vp, vp, vp,
-                                              ctypes.c_double, vp, vp, vp, vp, vp, vp, vp, vp, vp,
-                                              vp]
+                                              ctypes.c_double, vp, vp, i32, vp, vp, vp, vp, vp,
+                                              vp, vp, vp, vp]
+        lib.oracle_expert_backward.argtypes = [vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, vp, vp,
+                                               vp]
         _lib = lib
     return _lib
 
@@ -205,10 +207,13 @@ def layer(x: np.ndarray, inp: dict, M: int, Kp: int, dtype: str,
 
 
 def layer_backward(x: np.ndarray, inp: dict, M: int, Kp: int, dtype: str, dy: np.ndarray,
-                   alpha: float = 0.0, idx: Optional[np.ndarray] = None) -> dict:
+                   alpha: float = 0.0, idx: Optional[np.ndarray] = None,
+                   tokens: Optional[Sequence[int]] = None, weights: bool = True) -> dict:
     """Gradients of sum_t dy_t . y_t + L_aux (routing held fixed) -- oracle.c,
     oracle_layer_backward. x, dy: float64 [T][d]; idx: optional picks [T][M*Kp]
-    to hold the routing at (default: the oracle's own). Returns float64 arrays
+    to hold the routing at (default: the oracle's own); tokens: only these
+    tokens' terms (their dx rows exact, weight gradients partial); weights=False:
+    dx alone (no weight-gradient arrays, for full-size samples). Returns float64 arrays
     dx [T][d], w_router [N][d], w_gate/w_up [N][I][d], w_down [N][d][I],
     s_gate/s_up [S][I][d], s_down [S][d][I], and the scalar aux."""
     x = np.ascontiguousarray(x, np.float64)
@@ -221,19 +226,41 @@ def layer_backward(x: np.ndarray, inp: dict, M: int, Kp: int, dtype: str, dy: np
     sg, su, sd = (_w(inp[k], dtype) if S > 0 else None for k in ("s_gate", "s_up", "s_down"))
     b = inp.get("logit_bias")
     b = None if b is None else np.ascontiguousarray(b, np.float32)
-    out = {"dx": np.empty((T, d)), "w_router": np.empty((N, d)),
-           "w_gate": np.empty((N, I, d)), "w_up": np.empty((N, I, d)), "w_down": np.empty((N, d, I)),
-           "s_gate": np.empty((S, I, d)), "s_up": np.empty((S, I, d)), "s_down": np.empty((S, d, I))}
+    out = {"dx": np.empty((T, d))}
+    if weights:
+        out.update({"w_router": np.empty((N, d)), "w_gate": np.empty((N, I, d)),
+                    "w_up": np.empty((N, I, d)), "w_down": np.empty((N, d, I)),
+                    "s_gate": np.empty((S, I, d)), "s_up": np.empty((S, I, d)),
+                    "s_down": np.empty((S, d, I))})
     aux = np.zeros(1)
     picks = None if idx is None else np.ascontiguousarray(idx, np.int32)
+    toks = None if tokens is None else np.ascontiguousarray(tokens, np.int32)
     _chk(_l().oracle_layer_backward(_p(x), T, d, N, M, Kp, S, I, _DT[dtype], _p(wr), _p(b),
                                     _p(wg), _p(wu), _p(wd), _p(sg), _p(su), _p(sd), _p(dy),
-                                    float(alpha), _p(picks), _p(out["dx"]), _p(out["w_router"]),
-                                    _p(out["w_gate"]), _p(out["w_up"]), _p(out["w_down"]),
-                                    _p(out["s_gate"]), _p(out["s_up"]), _p(out["s_down"]),
+                                    float(alpha), _p(picks), _p(toks), 0 if toks is None else len(toks),
+                                    _p(out["dx"]), *[_p(out.get(k)) for k in
+                                                     ("w_router", "w_gate", "w_up", "w_down",
+                                                      "s_gate", "s_up", "s_down")],
                                     _p(aux)), "layer_backward")
     out["aux"] = float(aux[0])
     return out
+
+
+def expert_backward(x_rows: np.ndarray, dy_rows: np.ndarray, w: np.ndarray, wg: np.ndarray,
+                    wu: np.ndarray, wd: np.ndarray, dtype: str):
+    """One expert's weight gradients from the tokens that chose it (oracle.c,
+    oracle_expert_backward): x_rows, dy_rows float64 [n][d], w [n] the tokens'
+    routing weights. Returns (dw_gate [I][d], dw_up [I][d], dw_down [d][I])."""
+    x_rows = np.ascontiguousarray(x_rows, np.float64)
+    dy_rows = np.ascontiguousarray(dy_rows, np.float64)
+    w = np.ascontiguousarray(w, np.float64)
+    wg, wu, wd = _w(wg, dtype), _w(wu, dtype), _w(wd, dtype)
+    I, d = wg.shape
+    dwg, dwu, dwd = np.empty((I, d)), np.empty((I, d)), np.empty((d, I))
+    _chk(_l().oracle_expert_backward(_p(x_rows), _p(dy_rows), _p(w), len(w), _p(wg), _p(wu),
+                                     _p(wd), _DT[dtype], d, I, _p(dwg), _p(dwu), _p(dwd)),
+         "expert_backward")
+    return dwg, dwu, dwd
 
 
 def rmsnorm(x: np.ndarray, eps: float = 1e-6) -> np.ndarray:

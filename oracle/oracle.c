@@ -473,6 +473,49 @@ int oracle_layer_fp8(const double *x, int T, int d, int N, int M, int Kp, int S,
     return rc;
 }
 
+/* One (token, expert) term of the backward pass below, with the expert's
+ * weight w for this token: accumulates w dy h^T into gd, dg x^T into gg and
+ * du x^T into gu, and Wg^T dg + Wu^T du into dxt (any of them may be NULL); returns
+ * dy . (Wd h). Scratch: row [max(d, I)], g, u, h, dh [I]. */
+static double expert_token_backward(const double *xt, const double *dyt, double w,
+                                    const void *wg, const void *wu, const void *wd, int dtype,
+                                    int d, int I, double *gg, double *gu, double *gd, double *dxt,
+                                    double *row, double *g, double *u, double *h, double *dh) {
+    for (int i = 0; i < I; ++i) {
+        load_row(wg, dtype, (size_t)i * d, d, row);
+        g[i] = dot(xt, row, d);
+        load_row(wu, dtype, (size_t)i * d, d, row);
+        u[i] = dot(xt, row, d);
+        h[i] = g[i] / (1.0 + exp(-g[i])) * u[i];
+        dh[i] = 0.0;
+    }
+    double o_dot = 0.0;
+    for (int o = 0; o < d; ++o) {
+        load_row(wd, dtype, (size_t)o * I, I, row);
+        o_dot += dyt[o] * dot(h, row, I);
+        for (int i = 0; i < I; ++i) {
+            dh[i] += w * dyt[o] * row[i];
+            if (gd) gd[(size_t)o * I + i] += w * dyt[o] * h[i];
+        }
+    }
+    for (int i = 0; i < I; ++i) {
+        const double s = 1.0 / (1.0 + exp(-g[i]));
+        const double dg = dh[i] * u[i] * s * (1.0 + g[i] * (1.0 - s));
+        const double du = dh[i] * g[i] * s;
+        load_row(wg, dtype, (size_t)i * d, d, row);
+        for (int c = 0; c < d; ++c) {
+            if (gg) gg[(size_t)i * d + c] += dg * xt[c];
+            if (dxt) dxt[c] += dg * row[c];
+        }
+        load_row(wu, dtype, (size_t)i * d, d, row);
+        for (int c = 0; c < d; ++c) {
+            if (gu) gu[(size_t)i * d + c] += du * xt[c];
+            if (dxt) dxt[c] += du * row[c];
+        }
+    }
+    return o_dot;
+}
+
 /* ---------------------------------------------------------------------------
  * Backward pass of the layer [A][B][D] for an upstream gradient dy [T][d],
  * with the routing held at its forward value (the picks are piecewise
@@ -499,6 +542,10 @@ int oracle_layer_fp8(const double *x, int T, int d, int N, int M, int Kp, int S,
  * idx_in (may be NULL): picks [T][M*Kp] to hold the routing at instead of the
  * oracle's own selection (tokens whose top scores tie within rounding have
  * more than one correct pick; each must lie in its group).
+ * tokens (may be NULL): only these n_tokens tokens' terms are taken -- their
+ * dx rows are then exact (other rows zero), the weight gradients partial; the
+ * routing and the balance loss's f still come from the whole batch.
+ * The weight-gradient outputs (dwr ... dsd) may all be NULL together: only dx.
  * Every output array is overwritten. Shapes: dx [T][d], dwr [N][d],
  * dwg/dwu [N][I][d], dwd [N][d][I], dsg/dsu [S][I][d], dsd [S][d][I].
  * aux_out (may be NULL) receives L_aux.
@@ -507,7 +554,8 @@ int oracle_layer_backward(const double *x, int T, int d, int N, int M, int Kp, i
                           int dtype, const void *w_router, const float *bias,
                           const void *w_gate, const void *w_up, const void *w_down,
                           const void *s_gate, const void *s_up, const void *s_down,
-                          const double *dy, double alpha, const int32_t *idx_in, double *dx,
+                          const double *dy, double alpha, const int32_t *idx_in,
+                          const int32_t *tokens, int n_tokens, double *dx,
                           double *dwr, double *dwg,
                           double *dwu, double *dwd, double *dsg, double *dsu, double *dsd,
                           double *aux_out) {
@@ -529,12 +577,15 @@ int oracle_layer_backward(const double *x, int T, int d, int N, int M, int Kp, i
         free(dh);
         return 2;
     }
+    const int wgt = dwg != NULL;
     memset(dx, 0, sizeof(double) * (size_t)T * d);
-    memset(dwr, 0, sizeof(double) * (size_t)N * d);
-    memset(dwg, 0, sizeof(double) * (size_t)N * per);
-    memset(dwu, 0, sizeof(double) * (size_t)N * per);
-    memset(dwd, 0, sizeof(double) * (size_t)N * per);
-    if (S > 0) {
+    if (wgt) {
+        memset(dwr, 0, sizeof(double) * (size_t)N * d);
+        memset(dwg, 0, sizeof(double) * (size_t)N * per);
+        memset(dwu, 0, sizeof(double) * (size_t)N * per);
+        memset(dwd, 0, sizeof(double) * (size_t)N * per);
+    }
+    if (wgt && S > 0) {
         memset(dsg, 0, sizeof(double) * (size_t)S * per);
         memset(dsu, 0, sizeof(double) * (size_t)S * per);
         memset(dsd, 0, sizeof(double) * (size_t)S * per);
@@ -560,7 +611,10 @@ int oracle_layer_backward(const double *x, int T, int d, int N, int M, int Kp, i
             aux += alpha * f[e] * (P / T);
         }
     }
-    for (int t = 0; t < T && !rc; ++t) {
+    const int n_run = tokens ? n_tokens : T;
+    for (int q = 0; q < n_run && !rc; ++q) {
+        const int t = tokens ? tokens[q] : q;
+        if (t < 0 || t >= T) { rc = 1; break; }
         const double *xt = x + (size_t)t * d;
         const double *dyt = dy + (size_t)t * d;
         double *dxt = dx + (size_t)t * d;
@@ -569,45 +623,15 @@ int oracle_layer_backward(const double *x, int T, int d, int N, int M, int Kp, i
             const int routed = k < K;
             const size_t e = routed ? (size_t)idx[(size_t)t * K + k] : (size_t)(k - K);
             const double w = routed ? wk[(size_t)t * K + k] : 1.0;
-            const void *wg = routed ? expert_ptr(w_gate, dtype, e, per) : expert_ptr(s_gate, dtype, e, per);
-            const void *wu = routed ? expert_ptr(w_up, dtype, e, per) : expert_ptr(s_up, dtype, e, per);
-            const void *wd = routed ? expert_ptr(w_down, dtype, e, per) : expert_ptr(s_down, dtype, e, per);
-            double *gg = (routed ? dwg : dsg) + e * per;
-            double *gu = (routed ? dwu : dsu) + e * per;
-            double *gd = (routed ? dwd : dsd) + e * per;
-            for (int i = 0; i < I; ++i) {
-                load_row(wg, dtype, (size_t)i * d, d, row);
-                g[i] = dot(xt, row, d);
-                load_row(wu, dtype, (size_t)i * d, d, row);
-                u[i] = dot(xt, row, d);
-                h[i] = g[i] / (1.0 + exp(-g[i])) * u[i];
-                dh[i] = 0.0;
-            }
-            double o_dot = 0.0;  /* dy_t . (Wd h) */
-            for (int o = 0; o < d; ++o) {
-                load_row(wd, dtype, (size_t)o * I, I, row);
-                o_dot += dyt[o] * dot(h, row, I);
-                for (int i = 0; i < I; ++i) {
-                    dh[i] += w * dyt[o] * row[i];
-                    gd[(size_t)o * I + i] += w * dyt[o] * h[i];
-                }
-            }
+            const double o_dot = expert_token_backward(
+                xt, dyt, w,
+                routed ? expert_ptr(w_gate, dtype, e, per) : expert_ptr(s_gate, dtype, e, per),
+                routed ? expert_ptr(w_up, dtype, e, per) : expert_ptr(s_up, dtype, e, per),
+                routed ? expert_ptr(w_down, dtype, e, per) : expert_ptr(s_down, dtype, e, per),
+                dtype, d, I, wgt ? (routed ? dwg : dsg) + e * per : NULL,
+                wgt ? (routed ? dwu : dsu) + e * per : NULL,
+                wgt ? (routed ? dwd : dsd) + e * per : NULL, dxt, row, g, u, h, dh);
             if (routed) dp[e] += o_dot;
-            for (int i = 0; i < I; ++i) {
-                const double s = 1.0 / (1.0 + exp(-g[i]));
-                const double dg = dh[i] * u[i] * s * (1.0 + g[i] * (1.0 - s));
-                const double du = dh[i] * g[i] * s;
-                load_row(wg, dtype, (size_t)i * d, d, row);
-                for (int c = 0; c < d; ++c) {
-                    gg[(size_t)i * d + c] += dg * xt[c];
-                    dxt[c] += dg * row[c];
-                }
-                load_row(wu, dtype, (size_t)i * d, d, row);
-                for (int c = 0; c < d; ++c) {
-                    gu[(size_t)i * d + c] += du * xt[c];
-                    dxt[c] += du * row[c];
-                }
-            }
         }
         const double *pt = p + (size_t)t * N;
         double pdp = 0.0;
@@ -616,7 +640,7 @@ int oracle_layer_backward(const double *x, int T, int d, int N, int M, int Kp, i
             const double dl = pt[e] * (dp[e] - pdp);
             load_row(w_router, dtype, (size_t)e * d, d, row);
             for (int c = 0; c < d; ++c) {
-                dwr[(size_t)e * d + c] += dl * xt[c];
+                if (wgt) dwr[(size_t)e * d + c] += dl * xt[c];
                 dxt[c] += dl * row[c];
             }
         }
@@ -624,4 +648,34 @@ int oracle_layer_backward(const double *x, int T, int d, int N, int M, int Kp, i
     if (aux_out) *aux_out = aux;
     free(p); free(idx); free(wk); free(f); free(dp); free(row); free(g); free(u); free(h); free(dh);
     return rc;
+}
+
+/* ---------------------------------------------------------------------------
+ * Weight gradients of ONE expert from the n tokens that chose it (rows x and
+ * dy [n][d], weights w [n]: the tokens' routing scores, 1 for a shared expert):
+ * the same terms as oracle_layer_backward, summed over those tokens only --
+ * which is the whole of that expert's gradient. dwg, dwu [I][d], dwd [d][I]
+ * are overwritten. wg, wu point at the expert's [I][d], wd at its [d][I].
+ */
+int oracle_expert_backward(const double *x, const double *dy, const double *w, int n,
+                           const void *wg, const void *wu, const void *wd, int dtype, int d, int I,
+                           double *dwg, double *dwu, double *dwd) {
+    const size_t per = (size_t)I * d;
+    double *row = (double *)malloc(sizeof(double) * (size_t)(d > I ? d : I));
+    double *g = (double *)malloc(sizeof(double) * (size_t)I);
+    double *u = (double *)malloc(sizeof(double) * (size_t)I);
+    double *h = (double *)malloc(sizeof(double) * (size_t)I);
+    double *dh = (double *)malloc(sizeof(double) * (size_t)I);
+    if (!row || !g || !u || !h || !dh) {
+        free(row); free(g); free(u); free(h); free(dh);
+        return 2;
+    }
+    memset(dwg, 0, sizeof(double) * per);
+    memset(dwu, 0, sizeof(double) * per);
+    memset(dwd, 0, sizeof(double) * per);
+    for (int q = 0; q < n; ++q)
+        expert_token_backward(x + (size_t)q * d, dy + (size_t)q * d, w[q], wg, wu, wd, dtype, d, I,
+                              dwg, dwu, dwd, NULL, row, g, u, h, dh);
+    free(row); free(g); free(u); free(h); free(dh);
+    return 0;
 }

@@ -19,7 +19,7 @@ import torch
 import mixture_grouped_experts_b200 as mg
 import oracle
 import synth
-from gpu_helpers import check_routing, to_host_f64
+from gpu_helpers import check_routing, sample_tokens, to_host_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -98,3 +98,49 @@ def test_unchosen_experts_get_zero_gradient():
     for e in unused:
         for k in ("w_gate", "w_up", "w_down"):
             assert not grads[k][e].float().abs().max().item(), (k, e)
+
+
+def test_backward_full_size_prefill_sampled():
+    """The prefill workload (T = 4096, d = 5120, 64 experts in 8 groups,
+    K' = 1, 4 shared experts, I = 1344) in the launch configuration the
+    benchmark times. The oracle checks what it can compute one piece at a
+    time: dx of sampled tokens, and the complete weight gradients of the
+    routed expert with the fewest tokens (its gradient is the sum over exactly
+    those tokens). The router gradient is checked by a property that holds at
+    any size: its rows sum to zero (each token's softmax gradient does), up to
+    the bf16 rounding of dl."""
+    cfg = synth.CONFIGS["prefill"]
+    alpha = 0.01
+    inp = synth.layer_inputs(cfg)
+    x = oracle.to_double(inp["x"], cfg.dtype)
+    s = mg.shape_of(cfg)
+    xd = mg.to_device(inp["x"], cfg.dtype)
+    w = mg.weights_to_device(inp, cfg.dtype)
+    dy_h = synth.upstream_grad(cfg)
+    dy = mg.to_device(dy_h, "bf16")
+    ws = mg.alloc_train_workspace(s)
+    mg.moge_layer_forward_train(s, xd, w, ws)
+    idx_g, w_g, _, _ = mg.moge_workspace_routing(s, ws)
+    idx_g, w_g = idx_g.cpu().numpy(), w_g.cpu().numpy()
+    dx, grads = mg.moge_layer_backward(s, xd, w, dy, ws, alpha=alpha)
+    torch.cuda.synchronize()
+    mg.check_device_errors()
+    p = oracle.router_probs(x, inp["w_router"], None, cfg.dtype)
+    idx_o, _, mg_o = oracle.select_grouped(p, cfg.M, cfg.Kp)
+    check_routing(cfg, p, idx_o, mg_o, idx_g, w_g)
+    dyd = oracle.to_double(dy_h, "bf16")
+    toks = sample_tokens(cfg.T, 6)
+    ref = oracle.layer_backward(x, inp, cfg.M, cfg.Kp, cfg.dtype, dyd, alpha, idx=idx_g,
+                                tokens=toks, weights=False)
+    err = _normwise(to_host_f64(dx)[toks], ref["dx"][toks])
+    assert err <= TOL, ("dx", err)
+    cnt = np.bincount(idx_g.ravel(), minlength=cfg.N)
+    e = int(np.argmin(np.where(cnt > 0, cnt, 1 << 30)))
+    rows = np.nonzero((idx_g == e).any(1))[0]
+    ref_w = oracle.expert_backward(x[rows], dyd[rows], p[rows, e], inp["w_gate"][e],
+                                   inp["w_up"][e], inp["w_down"][e], cfg.dtype)
+    for k, r in zip(("w_gate", "w_up", "w_down"), ref_w):
+        err = _normwise(to_host_f64(grads[k][e]), r)
+        assert err <= TOL, (k, e, len(rows), err)
+    gr = grads["w_router"].float()
+    assert float(gr.sum(0).abs().max() / gr.abs().max()) <= 0.05

@@ -129,3 +129,41 @@ def test_routing_override():
     bad[0, 0] = SMALL.N - 1
     with pytest.raises(ValueError):
         oracle.layer_backward(x, inp, SMALL.M, SMALL.Kp, "f32", dy, 0.2, idx=bad)
+
+
+def test_token_subset_and_per_expert_gradients():
+    # a token subset gives those tokens' dx rows exactly; one expert's weight
+    # gradient from only the tokens that chose it is that expert's whole gradient
+    cfg = SMALL.replace(T=11, seed=25)
+    inp = synth.layer_inputs(cfg)
+    x = oracle.to_double(inp["x"], "f32")
+    dy = np.random.default_rng(7).normal(size=x.shape)
+    full = oracle.layer_backward(x, inp, cfg.M, cfg.Kp, "f32", dy, 0.3)
+    sub = [2, 5, 9]
+    part = oracle.layer_backward(x, inp, cfg.M, cfg.Kp, "f32", dy, 0.3, tokens=sub)
+    assert np.array_equal(part["dx"][sub], full["dx"][sub])
+    assert not part["dx"][[0, 1, 3]].any()
+    p = oracle.router_probs(x, inp["w_router"], None, "f32")
+    idx, _, _ = oracle.select_grouped(p, cfg.M, cfg.Kp)
+    for e in range(cfg.N):
+        rows = np.nonzero((idx == e).any(1))[0]
+        dwg, dwu, dwd = oracle.expert_backward(x[rows], dy[rows], p[rows, e], inp["w_gate"][e],
+                                               inp["w_up"][e], inp["w_down"][e], "f32")
+        assert np.array_equal(dwg, full["w_gate"][e])
+        assert np.array_equal(dwu, full["w_up"][e])
+        assert np.array_equal(dwd, full["w_down"][e])
+    one = np.ones(cfg.T)
+    dsg, dsu, dsd = oracle.expert_backward(x, dy, one, inp["s_gate"][1], inp["s_up"][1],
+                                           inp["s_down"][1], "f32")
+    assert np.array_equal(dsg, full["s_gate"][1]) and np.array_equal(dsd, full["s_down"][1])
+
+
+def test_dx_only():
+    cfg = SMALL.replace(T=9, seed=26)
+    inp = synth.layer_inputs(cfg)
+    x = oracle.to_double(inp["x"], "f32")
+    dy = np.random.default_rng(8).normal(size=x.shape)
+    full = oracle.layer_backward(x, inp, cfg.M, cfg.Kp, "f32", dy, 0.2)
+    only = oracle.layer_backward(x, inp, cfg.M, cfg.Kp, "f32", dy, 0.2, weights=False)
+    assert set(only) == {"dx", "aux"}
+    assert np.array_equal(only["dx"], full["dx"])
