@@ -91,6 +91,15 @@ def layer_flops(cfg):
     return (cfg.T * cfg.K + cfg.S * cfg.T) * 6.0 * cfg.d * cfg.I + 2.0 * cfg.T * cfg.d * cfg.N
 
 
+def train_flops(cfg):
+    """FLOPs of one training step of the layer (moge_layer_forward_train +
+    moge_layer_backward): the forward's, the backward's expert GEMMs (twice the
+    forward FFN: dh and dx on the input side, dW_down and dW_gate / dW_up on
+    the weight side) and the router's three (recomputed logits, dW_router, the
+    router's share of dx)."""
+    return layer_flops(cfg) + 2 * ffn_flops(cfg) + 3 * 2 * cfg.T * cfg.N * cfg.d
+
+
 def layer_bytes(cfg, n_used):
     """Algorithmic bytes of the layer: each used expert's three matrices once,
     the router, x in and y out (no padding, no permute traffic)."""
@@ -283,6 +292,49 @@ def measure(cfg, inp, steps, warmup, dist_on=False, with_e2e=True, fp8=False):
     return out
 
 
+def measure_train(cfg, inp, steps, warmup, alpha=0.01):
+    """Device-timed training steps: forward (keeping what the backward needs)
+    + backward with the balance loss; also the forward alone, same loop."""
+    import torch
+    import mixture_grouped_experts_b200 as mg
+
+    s = mg.shape_of(cfg)
+    x = mg.to_device(inp["x"], cfg.dtype)
+    w = mg.weights_to_device(inp, cfg.dtype)
+    dy = mg.to_device(synth.upstream_grad(cfg), "bf16")
+    ws = mg.alloc_train_workspace(s)
+    y = torch.empty_like(x)
+    dx = torch.empty_like(x)
+    grads = {k: torch.empty_like(w[k]) for k in mg.GRAD_KEYS if w.get(k) is not None}
+    aux = torch.zeros(1, dtype=torch.float32, device="cuda")
+
+    def fwd():
+        mg.moge_layer_forward_train(s, x, w, ws, y=y)
+
+    def step():
+        fwd()
+        mg.moge_layer_backward(s, x, w, dy, ws, alpha=alpha, grads=grads, dx=dx, aux=aux)
+
+    stream = torch.cuda.current_stream()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    out = {}
+    for name, fn in (("step", step), ("fwd", fwd)):
+        for _ in range(max(warmup, 3)):
+            fn()
+        torch.cuda.synchronize()
+        start.record(stream)
+        for _ in range(steps):
+            fn()
+        end.record(stream)
+        torch.cuda.synchronize()
+        out[name + "_ms"] = start.elapsed_time(end) / steps
+    mg.check_device_errors()
+    out["aux"] = float(aux.item())
+    del x, w, dy, ws, y, dx, grads
+    torch.cuda.empty_cache()
+    return out
+
+
 def max_over_ranks(v, dist_on):
     """Max of a per-rank scalar over all ranks (identity on one process).
     Uses a CUDA tensor under NCCL and a CPU tensor under gloo."""
@@ -320,6 +372,7 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=16, help="tokens in the CPU-baseline sample (0: skip)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--no-fp8", action="store_true", help="skip the 8-bit-weight side measurement")
+    ap.add_argument("--no-train", action="store_true", help="skip the training-step side measurement")
     ap.add_argument("--ref-tokens", type=int, default=2, help="tokens per step of --impl reference")
     args = ap.parse_args()
     cfg = synth.CONFIGS[args.config]
@@ -423,6 +476,29 @@ def main():
             "layer_roofline": {"achieved": lb8 / (fm["ms"] / 1e3) / 1e9, "peak": hbm, "unit": "GB/s",
                                "frac": lb8 / (fm["ms"] / 1e3) / 1e9 / hbm, "algorithmic_bytes": lb8},
             "stage_ms": fm["stage_ms"], "clocks": fclk}
+    if rank == 0 and n == 1 and not args.no_train and args.config == "decode":
+        tcfg = synth.CONFIGS["prefill"]
+        tinp = synth.layer_inputs(tcfg)
+        ts = ClockSampler(local)
+        ts.start()
+        tm = measure_train(tcfg, tinp, max(5, args.steps // 2), args.warmup)
+        tclk = ts.stop()
+        del tinp
+        tfs = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+        ach = train_flops(tcfg) / (tm["step_ms"] / 1e3) / 1e12
+        bwd_ms = tm["step_ms"] - tm["fwd_ms"]
+        bwd_tf = (train_flops(tcfg) - layer_flops(tcfg)) / (bwd_ms / 1e3) / 1e12
+        line["train_prefill"] = {
+            "workload": workload_config(tcfg)["workload"],
+            "step": "moge_layer_forward_train + moge_layer_backward (all weight and input "
+                    "gradients, batch balance loss alpha = 0.01)",
+            "value": tcfg.T / (tm["step_ms"] / 1e3), "unit": "tokens/s",
+            "ms_per_step": tm["step_ms"], "forward_ms": tm["fwd_ms"], "backward_ms": bwd_ms,
+            "roofline": {"bound": "tensor", "kernel": "training step (forward + backward GEMMs)",
+                         "achieved": ach, "peak": tfs, "unit": "TFLOP/s", "frac": ach / tfs,
+                         "flops_per_step": train_flops(tcfg),
+                         "peak_source": "%s bf16_tflops_sustained" % peak_kind},
+            "backward_tflops": bwd_tf, "clocks": tclk}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist_on:

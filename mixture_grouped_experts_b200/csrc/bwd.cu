@@ -14,7 +14,9 @@ namespace moge {
 
 constexpr int kBwdThreads = 128;
 constexpr int kMaxK = 32;
-constexpr int kRouterBwdTokens = 8;  // tokens per CTA (one warp each)
+constexpr int kRouterBwdWarps = 8;
+constexpr int kRouterBwdPerWarp = 8;  // tokens per warp, one after another
+constexpr int kRouterBwdTokens = kRouterBwdWarps * kRouterBwdPerWarp;  // tokens per CTA
 
 __device__ __forceinline__ void unpack8(const uint4 u, float (&f)[8]) {
     f[0] = bf16_lo(u.x); f[1] = bf16_hi(u.x); f[2] = bf16_lo(u.y); f[3] = bf16_hi(u.y);
@@ -72,21 +74,27 @@ __global__ void __launch_bounds__(kBwdThreads) combine_bwd_kernel(
     }
 }
 
-// One warp per token, lane l holding experts l, l + 32, ...; also each CTA's
-// sums of p over its tokens (part[blockIdx.x][e]) for the balance loss.
-__global__ void __launch_bounds__(32 * kRouterBwdTokens) router_bwd_kernel(
+// One warp per token (each warp takes kRouterBwdPerWarp tokens in turn), lane
+// l holding experts l, l + 32, ...; also each CTA's sums of p over its tokens
+// (part[blockIdx.x][e], fixed order) for the balance loss.
+__global__ void __launch_bounds__(32 * kRouterBwdWarps) router_bwd_kernel(
     moge_config c, float alpha, const float *__restrict__ logits,
     const int32_t *__restrict__ topk_idx, const float *__restrict__ dw,
     const int32_t *__restrict__ counts, uint16_t *dl, float *part) {
-    __shared__ float psum[kRouterBwdTokens][kMaxExperts];
+    __shared__ float psum[kRouterBwdWarps][kMaxExperts];
     grid_dependency_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t = blockIdx.x * kRouterBwdTokens + warp;
     const int N = c.N, K = c.M * c.Kp;
     const int per = (N + 31) / 32;
     constexpr int kPer = kMaxExperts / 32;
-    float pr[kPer], dp[kPer];
-    if (t < c.T) {
+    const float inv_t = 1.0f / (float)c.T;
+    float acc[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) acc[j] = 0.0f;
+    for (int r = 0; r < kRouterBwdPerWarp; ++r) {
+        const int t = blockIdx.x * kRouterBwdTokens + r * kRouterBwdWarps + warp;
+        if (t >= c.T) break;
+        float pr[kPer], dp[kPer];
         float mx = -INFINITY;
 #pragma unroll
         for (int j = 0; j < kPer; ++j) {
@@ -102,11 +110,11 @@ __global__ void __launch_bounds__(32 * kRouterBwdTokens) router_bwd_kernel(
             z += pr[j];
         }
         for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-        const float inv_t = 1.0f / (float)c.T;
 #pragma unroll
         for (int j = 0; j < kPer; ++j) {
             const int e = lane + 32 * j;
             pr[j] /= z;
+            acc[j] += pr[j];
             dp[j] = (j < per && e < N) ? alpha * ((float)counts[e] * inv_t) * inv_t : 0.0f;
         }
         for (int k = 0; k < K; ++k) {
@@ -125,18 +133,15 @@ __global__ void __launch_bounds__(32 * kRouterBwdTokens) router_bwd_kernel(
             const int e = lane + 32 * j;
             if (j < per && e < N) dl[(size_t)t * N + e] = to_bf16_bits(pr[j] * (dp[j] - pdp));
         }
-    } else {
-#pragma unroll
-        for (int j = 0; j < kPer; ++j) pr[j] = 0.0f;
     }
 #pragma unroll
     for (int j = 0; j < kPer; ++j)
-        if (lane + 32 * j < N) psum[warp][lane + 32 * j] = pr[j];
+        if (lane + 32 * j < N) psum[warp][lane + 32 * j] = acc[j];
     __syncthreads();
     for (int e = threadIdx.x; e < N; e += blockDim.x) {
-        float s = 0.0f;
-        for (int w = 0; w < kRouterBwdTokens; ++w) s += psum[w][e];
-        part[(size_t)blockIdx.x * N + e] = s;
+        float sum = 0.0f;
+        for (int w = 0; w < kRouterBwdWarps; ++w) sum += psum[w][e];
+        part[(size_t)blockIdx.x * N + e] = sum;
     }
 }
 
@@ -209,7 +214,7 @@ cudaError_t launch_router_bwd(const moge_config &c, float alpha, const float *lo
                               const int32_t *topk_idx, const float *dw, const int32_t *counts,
                               void *dl, float *part, float *aux, cudaStream_t st) {
     const int parts = router_bwd_parts(c);
-    cudaError_t e = launch_pdl(router_bwd_kernel, dim3(parts), dim3(32 * kRouterBwdTokens), 0, st, c,
+    cudaError_t e = launch_pdl(router_bwd_kernel, dim3(parts), dim3(32 * kRouterBwdWarps), 0, st, c,
                                alpha, logits, topk_idx, dw, counts, (uint16_t *)dl, part);
     if (e != cudaSuccess || !aux) return e;
     return launch_pdl(aux_loss_kernel, dim3(1), dim3(256), 0, st, c, alpha, (const float *)part,
