@@ -297,6 +297,53 @@ MOGE_API int moge_layer_backward(const moge_config *cfg, float alpha, const void
                                  void *dw_up, void *dw_down, void *ds_gate, void *ds_up,
                                  void *ds_down, float *aux, void *workspace, void *stream);
 
+
+/* ---------------------------------------------------------- expert parallelism
+ * The pages place one expert group per device (techwalker.com article,
+ * section 1: experts reorganised by device so that every device carries the
+ * same load; sections 2 and 5: AllGather / ReduceScatter around the grouped
+ * matmuls, shared experts split by tensor parallelism). Rank r of `world`
+ * ranks (world divides M and I) holds the routed experts of groups
+ * [r M/world, (r+1) M/world) -- experts [r N/world, (r+1) N/world), the
+ * layouts of the full tensors restricted to those experts -- and rows
+ * [r I/world, (r+1) I/world) of every shared expert's W_gate and W_up with
+ * the matching columns of its W_down (s_gate, s_up [S][I/world][d], s_down
+ * [S][d][I/world], contiguous). A layer step on `world` ranks, each with its
+ * own T/world tokens:
+ *   1. all-gather x into x_all [T][d]               (collective, caller's)
+ *   2. moge_layer_forward_ep_local -> y_part [T][d] fp32: this rank's routed
+ *      experts on the picks that fall in its groups (weighted by the global
+ *      softmax scores, routing replicated on every rank) plus its slice of
+ *      every shared expert
+ *   3. reduce-scatter (sum) of y_part into this rank's [T/world][d] rows
+ *                                                  (collective, caller's)
+ *   4. moge_ep_finish: y = that sum (+ residual) in the layer dtype.
+ * The sum over ranks of y_part is the layer's output for all T tokens.
+ * cfg describes the whole layer: T = all ranks' tokens, N, M, I of the full
+ * model. The Python binding's moge_layer_forward_ep runs the four steps with
+ * torch.distributed (NCCL).
+ *
+ * moge_ep_workspace_size(cfg, world): bytes of the workspace of step 2
+ * (0: unsupported). */
+MOGE_API size_t moge_ep_workspace_size(const moge_config *cfg, int world);
+
+/* Step 2 (see above). x_all [T][d] in cfg->dtype; w_gate, w_up
+ * [N/world][I][d], w_down [N/world][d][I]: this rank's routed experts; s_*:
+ * its shared-expert slices (NULL when S == 0); y_part [T][d] fp32 (device,
+ * 16-byte aligned, overwritten). Asynchronous on `stream`. */
+MOGE_API int moge_layer_forward_ep_local(const moge_config *cfg, int rank, int world,
+                                         const void *x_all, const void *w_router,
+                                         const float *logit_bias, const void *w_gate,
+                                         const void *w_up, const void *w_down,
+                                         const void *s_gate, const void *s_up,
+                                         const void *s_down, float *y_part, void *workspace,
+                                         void *stream);
+
+/* Step 4: y[t] = y_sum[t] (+ residual[t]) for `rows` rows of cfg->d, y and
+ * residual in cfg->dtype, y_sum fp32. */
+MOGE_API int moge_ep_finish(const moge_config *cfg, int64_t rows, const float *y_sum,
+                            const void *residual, void *y, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -31,7 +31,8 @@ EXPORTS = ["moge_workspace_size", "moge_last_error", "moge_check_device_errors",
            "moge_layer_forward", "moge_layer_forward_host", "moge_workspace_routing",
            "moge_rmsnorm", "moge_stage_timing", "moge_stage_times", "moge_route_noalloc",
            "moge_quantize_fp8_rows", "moge_layer_forward_fp8", "moge_selftest_waits",
-           "moge_train_workspace_size", "moge_layer_forward_train", "moge_layer_backward"]
+           "moge_train_workspace_size", "moge_layer_forward_train", "moge_layer_backward",
+           "moge_ep_workspace_size", "moge_layer_forward_ep_local", "moge_ep_finish"]
 STAGES = ("router", "scan", "permute", "ffn", "combine")
 
 
@@ -111,8 +112,13 @@ def lib() -> ctypes.CDLL:
         L.moge_train_workspace_size.restype = ctypes.c_size_t
         L.moge_layer_forward_train.argtypes = [cp] + [vp] * 12
         L.moge_layer_backward.argtypes = [cp, ctypes.c_float] + [vp] * 21
+        L.moge_ep_workspace_size.argtypes = [cp, i32]
+        L.moge_ep_workspace_size.restype = ctypes.c_size_t
+        L.moge_layer_forward_ep_local.argtypes = [cp, i32, i32] + [vp] * 12
+        L.moge_ep_finish.argtypes = [cp, ctypes.c_int64, vp, vp, vp, vp]
         for n in EXPORTS:
-            if n not in ("moge_workspace_size", "moge_last_error", "moge_train_workspace_size"):
+            if n not in ("moge_workspace_size", "moge_last_error", "moge_train_workspace_size",
+                         "moge_ep_workspace_size"):
                 getattr(L, n).restype = i32
         _lib = L
     return _lib
@@ -278,6 +284,81 @@ def moge_layer_backward(s: LayerShape, x, w: dict, dy, workspace, alpha: float =
                                    *[_p(grads.get(k)) for k in GRAD_KEYS], _p(aux),
                                    _p(workspace), _stream(stream)))
     return dx, grads
+
+
+# ---------------------------------------------------------------- expert parallelism
+def ep_workspace_size(s: LayerShape, world: int) -> int:
+    n = lib().moge_ep_workspace_size(ctypes.byref(_cfg(s)), int(world))
+    if n == 0:
+        raise MogeError(ERR_UNSUPPORTED, lib().moge_last_error().decode())
+    return n
+
+
+def alloc_ep_workspace(s: LayerShape, world: int, device=None) -> torch.Tensor:
+    return torch.empty(ep_workspace_size(s, world), dtype=torch.uint8, device=device or "cuda")
+
+
+def ep_shard_weights(w: dict, rank: int, world: int) -> dict:
+    """Rank `rank`'s expert-parallel share of a layer's weights (see moge.h):
+    the routed experts of its groups (views of the full tensors, contiguous)
+    and rows [r I/world, (r+1) I/world) of every shared expert's gate and up
+    with the matching columns of its down projection (contiguous copies). The
+    router is replicated."""
+    N, I = w["w_gate"].shape[0], w["w_gate"].shape[1]
+    if N % world or I % world:
+        raise ValueError("world must divide the expert count and I")
+    n_loc, i_s = N // world, I // world
+    e0, i0 = rank * n_loc, rank * i_s
+    out = {"w_router": w["w_router"], "logit_bias": w.get("logit_bias")}
+    for k in ("w_gate", "w_up", "w_down"):
+        out[k] = w[k][e0:e0 + n_loc]
+    if w.get("s_gate") is not None:
+        out["s_gate"] = w["s_gate"][:, i0:i0 + i_s].contiguous()
+        out["s_up"] = w["s_up"][:, i0:i0 + i_s].contiguous()
+        out["s_down"] = w["s_down"][:, :, i0:i0 + i_s].contiguous()
+    return out
+
+
+def moge_layer_forward_ep_local(s: LayerShape, rank: int, world: int, x_all, w_local: dict,
+                                workspace, y_part=None, stream=None):
+    """This rank's fp32 partial y [T][d] of the layer (s: the whole layer's shape)."""
+    if y_part is None:
+        y_part = torch.empty((s.T, s.d), dtype=torch.float32, device=x_all.device)
+    _chk(lib().moge_layer_forward_ep_local(ctypes.byref(_cfg(s)), int(rank), int(world), _p(x_all),
+                                           _p(w_local["w_router"]), _p(w_local.get("logit_bias")),
+                                           _p(w_local["w_gate"]), _p(w_local["w_up"]),
+                                           _p(w_local["w_down"]), _p(w_local.get("s_gate")),
+                                           _p(w_local.get("s_up")), _p(w_local.get("s_down")),
+                                           _p(y_part), _p(workspace), _stream(stream)))
+    return y_part
+
+
+def moge_ep_finish(s: LayerShape, y_sum, residual=None, y=None, stream=None):
+    """y = y_sum (+ residual) in the layer dtype."""
+    if y is None:
+        y = torch.empty(y_sum.shape, dtype=_TORCH_DT[s.dtype], device=y_sum.device)
+    _chk(lib().moge_ep_finish(ctypes.byref(_cfg(s)), int(y_sum.shape[0]), _p(y_sum), _p(residual),
+                              _p(y), _stream(stream)))
+    return y
+
+
+def moge_layer_forward_ep(s: LayerShape, x_local, w_local: dict, workspace, group=None,
+                          residual=None):
+    """One layer step under expert parallelism on the ranks of `group` (each
+    with its own x_local [T/world][d]; s is the whole layer's shape, T = all
+    ranks' tokens): all-gather x, this rank's partial, reduce-scatter of the
+    partials (NCCL), finish. Returns this rank's y [T/world][d]."""
+    import torch.distributed as dist
+    world, rank = dist.get_world_size(group), dist.get_rank(group)
+    rows = x_local.shape[0]
+    if rows * world != s.T:
+        raise ValueError("x_local must hold T / world rows")
+    x_all = torch.empty((s.T, s.d), dtype=x_local.dtype, device=x_local.device)
+    dist.all_gather_into_tensor(x_all, x_local, group=group)
+    y_part = moge_layer_forward_ep_local(s, rank, world, x_all, w_local, workspace)
+    y_sum = torch.empty((rows, s.d), dtype=torch.float32, device=x_local.device)
+    dist.reduce_scatter_tensor(y_sum, y_part, group=group)
+    return moge_ep_finish(s, y_sum, residual)
 
 
 def moge_layer_forward_host(s: LayerShape, x_host, w: dict, workspace, y_host, x_dev, y_dev,

@@ -23,7 +23,9 @@ static int cuda_fail(cudaError_t e, const char *where) {
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 static bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
-static int check_config(const moge_config *c) {
+// router: the config's router runs (the bf16 router needs N % 8 == 0); the
+// expert-parallel sub-problems route nothing themselves
+static int check_config(const moge_config *c, bool router = true) {
     if (!c) return fail(MOGE_ERR_INVALID_ARG, "config is NULL");
     if (c->T < 0 || c->d <= 0 || c->N <= 0 || c->M <= 0 || c->Kp <= 0 || c->S < 0 || c->I <= 0)
         return fail(MOGE_ERR_INVALID_ARG, "config has a non-positive size");
@@ -35,7 +37,7 @@ static int check_config(const moge_config *c) {
     if (c->Kp > c->N / c->M) return fail(MOGE_ERR_UNSUPPORTED, "Kp > N/M");
     if (c->d % 8 != 0 || c->I % 8 != 0)
         return fail(MOGE_ERR_UNSUPPORTED, "d and I must be multiples of 8");
-    if (c->dtype == MOGE_BF16 && c->N % 8 != 0)
+    if (router && c->dtype == MOGE_BF16 && c->N % 8 != 0)
         return fail(MOGE_ERR_UNSUPPORTED, "bf16 router needs N % 8 == 0");
     const long long rows = (long long)c->T * (c->M * c->Kp + c->S);
     if (rows >= (1ll << 31) || (long long)c->T * c->M * c->Kp * (long long)c->d >= (1ll << 62))
@@ -254,6 +256,62 @@ static int check_train(const moge_config &c) {
     if (c.N % 8 != 0) return fail(MOGE_ERR_UNSUPPORTED, "training needs N % 8 == 0");
     if (c.M * c.Kp > 32) return fail(MOGE_ERR_UNSUPPORTED, "training needs M * Kp <= 32");
     return MOGE_OK;
+}
+
+
+// Expert parallelism: rank `rank` of `world` holds the experts of groups
+// [rank M/world, (rank+1) M/world) and an I/world slice of every shared
+// expert. loc: the routed sub-problem (those experts and groups, all T
+// tokens, no shared experts); shr: the shared slice (S experts of I/world,
+// no routed experts).
+static int ep_configs(const moge_config &c, int rank, int world, moge_config &loc,
+                      moge_config &shr) {
+    if (world < 1 || rank < 0 || rank >= world)
+        return fail(MOGE_ERR_INVALID_ARG, "need 0 <= rank < world");
+    if (c.M % world != 0) return fail(MOGE_ERR_UNSUPPORTED, "expert parallelism needs M % world == 0");
+    if (c.I % world != 0) return fail(MOGE_ERR_UNSUPPORTED, "expert parallelism needs I % world == 0");
+    loc = c;
+    loc.N = c.N / world;
+    loc.M = c.M / world;
+    loc.S = 0;
+    shr = c;
+    shr.N = 1;
+    shr.M = 1;
+    shr.Kp = 1;
+    shr.I = c.I / world;
+    int rc = check_config(&loc, false);
+    if (!rc) rc = check_config(&shr, false);
+    return rc;
+}
+
+struct EpSpace {
+    int32_t *hist, *rank, *topk_idx;  // routing of all T tokens over all N experts
+    float *topk_w;
+    Workspace lw, sw;                 // the routed and the shared sub-problems
+    size_t total;
+};
+static EpSpace carve_ep(const moge_config &c, const moge_config &loc, const moge_config &shr,
+                        void *base) {
+    EpSpace e;
+    const size_t K = (size_t)c.M * c.Kp, T = (size_t)c.T;
+    const size_t tiles = (T + kRouterTile - 1) / kRouterTile;
+    char *p = static_cast<char *>(base);
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        char *r = p ? p + off : nullptr;
+        off += align256(bytes > 0 ? bytes : 1);
+        return r;
+    };
+    e.hist = (int32_t *)take(tiles * c.N * 4);
+    e.rank = (int32_t *)take(T * K * 4);
+    e.topk_idx = (int32_t *)take(T * K * 4);
+    e.topk_w = (float *)take(T * K * 4);
+    e.lw = carve_workspace(loc, p ? p + off : nullptr);
+    off += e.lw.total;
+    e.sw = carve_workspace(shr, p ? p + off : nullptr);
+    off += e.sw.total;
+    e.total = off;
+    return e;
 }
 
 extern "C" {
@@ -672,6 +730,86 @@ int moge_layer_backward(const moge_config *cfg, float alpha, const void *x, cons
     MOGE_CU(launch_bwd_gemm(kDWR, c, ent, E, b, sms, st), "dW_router launch");
     MOGE_CU(launch_bwd_gemm(kDXR, c, ent, E, b, sms, st), "dx router launch");
     MOGE_CU(launch_unpermute_bwd(c, ws.y_perm, ws.perm_dst, ts.dx_r, dx, st), "un-permute launch");
+    return MOGE_OK;
+}
+
+
+size_t moge_ep_workspace_size(const moge_config *cfg, int world) {
+    moge_config loc, shr;
+    if (check_config(cfg) != MOGE_OK || ep_configs(*cfg, 0, world, loc, shr) != MOGE_OK) return 0;
+    return carve_ep(*cfg, loc, shr, nullptr).total;
+}
+
+int moge_layer_forward_ep_local(const moge_config *cfg, int rank, int world, const void *x_all,
+                                const void *w_router, const float *logit_bias,
+                                const void *w_gate, const void *w_up, const void *w_down,
+                                const void *s_gate, const void *s_up, const void *s_down,
+                                float *y_part, void *workspace, void *stream) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    const moge_config c = *cfg;
+    moge_config loc, shr;
+    if ((rc = ep_configs(c, rank, world, loc, shr))) return rc;
+    MOGE_NEED(y_part, "y_part");
+    cudaStream_t st = (cudaStream_t)stream;
+    if (c.T == 0) return MOGE_OK;
+    MOGE_NEED(x_all, "x_all");
+    MOGE_NEED(w_router, "w_router");
+    MOGE_NEED(w_gate, "w_gate");
+    MOGE_NEED(w_up, "w_up");
+    MOGE_NEED(w_down, "w_down");
+    if (c.S > 0) {
+        MOGE_NEED(s_gate, "s_gate");
+        MOGE_NEED(s_up, "s_up");
+        MOGE_NEED(s_down, "s_down");
+    }
+    if (logit_bias && !aligned4(logit_bias)) return fail(MOGE_ERR_UNSUPPORTED, "logit_bias misaligned");
+    MOGE_NEED(workspace, "workspace");
+    EpSpace es = carve_ep(c, loc, shr, workspace);
+    const Workspace &lw = es.lw, &sw = es.sw;
+    const int K = c.M * c.Kp, K_loc = loc.M * loc.Kp;
+    const int tiles = (c.T + kRouterTile - 1) / kRouterTile;
+    MOGE_CU(launch_router(c, x_all, w_router, logit_bias, es.topk_idx, es.topk_w, es.hist, es.rank,
+                          num_sms(), st), "router launch");
+    MOGE_CU(launch_localize(c.T, c.N, K, rank * K_loc, K_loc, rank * loc.N, loc.N, tiles,
+                            es.topk_idx, es.topk_w, es.rank, es.hist, lw.topk_idx, lw.topk_w, lw.rank,
+                            lw.hist, st), "localize launch");
+    MOGE_CU(launch_scan(loc, lw.hist, lw.base, lw.counts, lw.offsets, &lw.plan, true, false, st),
+            "scan launch");
+    MOGE_CU(launch_scatter_rows(loc, x_all, lw.topk_idx, lw.rank, lw.base, lw.offsets, lw.perm_src,
+                                lw.perm_dst, lw.x_perm, st), "permute launch");
+    const int64_t rrows = (int64_t)c.T * K_loc;
+    FfnOperands op{};
+    op.b0 = lw.x_perm; op.b1 = x_all; op.b0_rows = rrows; op.b1_rows = c.T;
+    op.wg = w_gate; op.wu = w_up; op.wd = w_down;
+    op.h = lw.h; op.h_rows = rrows; op.y = lw.y_perm;
+    rc = run_ffn(loc, lw.plan, loc.N, op, st);
+    if (rc) return rc;
+    if (c.S > 0) {
+        MOGE_CU(launch_plan(shr, nullptr, sw.plan, false, true, st), "plan launch");
+        FfnOperands os{};
+        os.b1 = x_all; os.b1_rows = c.T;
+        os.sg = s_gate; os.su = s_up; os.sd = s_down;
+        os.h = sw.h; os.h_rows = (int64_t)c.T * c.S; os.y = sw.y_perm;
+        rc = run_ffn(shr, sw.plan, c.S, os, st);
+        if (rc) return rc;
+    }
+    MOGE_CU(launch_combine(loc, lw.y_perm, lw.topk_w, lw.perm_dst, K_loc, c.S ? sw.y_perm : nullptr,
+                           c.S, nullptr, y_part, st, true), "combine launch");
+    return MOGE_OK;
+}
+
+int moge_ep_finish(const moge_config *cfg, int64_t rows, const float *y_sum, const void *residual,
+                   void *y, void *stream) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    if (rows < 0) return fail(MOGE_ERR_INVALID_ARG, "rows < 0");
+    if (rows == 0) return MOGE_OK;
+    MOGE_NEED(y_sum, "y_sum");
+    MOGE_NEED(y, "y");
+    if (residual && !aligned16(residual)) return fail(MOGE_ERR_UNSUPPORTED, "residual misaligned");
+    MOGE_CU(launch_ep_finish(cfg->dtype, rows, cfg->d, y_sum, residual, y, (cudaStream_t)stream),
+            "finish launch");
     return MOGE_OK;
 }
 

@@ -110,7 +110,8 @@ cudaError_t launch_gather_rows(const moge_config &c, const void *x, const int32_
                                void *x_perm, cudaStream_t st);
 cudaError_t launch_combine(const moge_config &c, const void *y_perm, const float *topk_w,
                            const int32_t *perm_dst, int K, const void *shared_rows,
-                           int n_shared_blocks, const void *residual, void *y, cudaStream_t st);
+                           int n_shared_blocks, const void *residual, void *y, cudaStream_t st,
+                           bool out_f32 = false);
 cudaError_t launch_rmsnorm(const moge_config &c, const void *x, float eps, void *u,
                            cudaStream_t st);
 
@@ -181,5 +182,13 @@ cudaError_t launch_wait_selftest(int32_t *out, uint64_t limit_ns, cudaStream_t s
 // per-row FP8 quantisation of bf16 rows
 cudaError_t launch_quantize_fp8(const void *w, int64_t rows, int64_t cols, void *q, float *scale,
                                 cudaStream_t st);
+
+// ---------------------------------------------------------------- expert parallelism
+cudaError_t launch_localize(int T, int N, int K, int k0, int K_loc, int e0, int N_loc, int tiles,
+                            const int32_t *topk_idx, const float *topk_w, const int32_t *rank,
+                            const int32_t *hist, int32_t *idx_loc, float *w_loc, int32_t *rank_loc,
+                            int32_t *hist_loc, cudaStream_t st);
+cudaError_t launch_ep_finish(int dtype, long long rows, int d, const float *y_sum,
+                             const void *residual, void *y, cudaStream_t st);
 
 }  // namespace moge

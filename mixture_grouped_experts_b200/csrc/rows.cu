@@ -156,7 +156,7 @@ template <int DT>
 __global__ void __launch_bounds__(kRowThreads) combine_kernel(
     int T, int d, int N, const void *__restrict__ y_perm, const float *__restrict__ topk_w,
     const int32_t *__restrict__ perm_dst, int K, const void *__restrict__ shared_rows,
-    int n_shared, const void *residual, void *y) {
+    int n_shared, const void *residual, void *y, int out_f32) {
     __shared__ const char *src_s[2 * kMaxExperts + 1];
     __shared__ float w_s[kMaxExperts];
     grid_dependency_wait();
@@ -208,16 +208,20 @@ __global__ void __launch_bounds__(kRowThreads) combine_kernel(
 #pragma unroll
             for (int q = 0; q < 8; ++q) acc[q] = f[q] + acc[q];
         }
-        store_vec<DT>((char *)y + (size_t)t * row_bytes, v, acc);
+        if (out_f32)
+            store_vec<MOGE_F32>((char *)y + (size_t)t * d * 4, v, acc);
+        else
+            store_vec<DT>((char *)y + (size_t)t * row_bytes, v, acc);
     }
 }
 
 cudaError_t launch_combine(const moge_config &c, const void *y_perm, const float *topk_w,
                            const int32_t *perm_dst, int K, const void *shared_rows,
-                           int n_shared_blocks, const void *residual, void *y, cudaStream_t st) {
+                           int n_shared_blocks, const void *residual, void *y, cudaStream_t st,
+                           bool out_f32) {
     auto kern = c.dtype == MOGE_BF16 ? combine_kernel<MOGE_BF16> : combine_kernel<MOGE_F32>;
     return launch_pdl(kern, dim3(c.T), dim3(kRowThreads), 0, st, c.T, c.d, c.N, y_perm, topk_w,
-                      perm_dst, K, shared_rows, n_shared_blocks, residual, y);
+                      perm_dst, K, shared_rows, n_shared_blocks, residual, y, out_f32 ? 1 : 0);
 }
 
 // ---------------------------------------------------------------------------

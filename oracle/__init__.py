@@ -68,6 +68,8 @@ def _l():
                                               vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                               ctypes.c_double, vp, vp, i32, vp, vp, vp, vp, vp,
                                               vp, vp, vp, vp]
+        lib.oracle_layer_ep_partial.argtypes = [vp, i32, i32, i32, i32, i32, i32, i32, i32, vp, vp,
+                                                i32, i32, vp, vp, vp, i32, vp, vp, vp, vp, i32, vp]
         lib.oracle_expert_backward.argtypes = [vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, vp, vp,
                                                vp]
         _lib = lib
@@ -261,6 +263,29 @@ def expert_backward(x_rows: np.ndarray, dy_rows: np.ndarray, w: np.ndarray, wg: 
                                      _p(wd), _DT[dtype], d, I, _p(dwg), _p(dwu), _p(dwd)),
          "expert_backward")
     return dwg, dwu, dwd
+
+
+def layer_ep_partial(x: np.ndarray, w_router: np.ndarray, bias: Optional[np.ndarray], e0: int,
+                     routed: Sequence[np.ndarray], shared: Sequence[np.ndarray], N: int, M: int,
+                     Kp: int, dtype: str, tokens: Optional[Sequence[int]] = None) -> np.ndarray:
+    """One rank's share of the layer (oracle.c, oracle_layer_ep_partial): the
+    router over all N experts; routed = (w_gate, w_up, w_down) of experts
+    [e0, e0 + n_loc) only; shared = (s_gate [S][I_s][d], s_up, s_down [S][d][I_s])
+    slices (S may be 0). Returns y [n][d] float64 for the listed tokens."""
+    x = np.ascontiguousarray(x, np.float64)
+    T, d = x.shape
+    wr = _w(w_router, dtype)
+    wg, wu, wd = (_w(a, dtype) for a in routed)
+    n_loc, I = wg.shape[0], wg.shape[1]
+    sg, su, sd = (_w(a, dtype) for a in shared)
+    S, I_s = sg.shape[0], sg.shape[1]
+    b = None if bias is None else np.ascontiguousarray(bias, np.float32)
+    toks = np.arange(T, dtype=np.int32) if tokens is None else np.asarray(tokens, np.int32)
+    y = np.empty((len(toks), d))
+    _chk(_l().oracle_layer_ep_partial(_p(x), T, d, N, M, Kp, S, I, _DT[dtype], _p(wr), _p(b), e0,
+                                      n_loc, _p(wg), _p(wu), _p(wd), I_s, _p(sg), _p(su), _p(sd),
+                                      _p(toks), len(toks), _p(y)), "layer_ep_partial")
+    return y
 
 
 def rmsnorm(x: np.ndarray, eps: float = 1e-6) -> np.ndarray:

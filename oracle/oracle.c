@@ -679,3 +679,61 @@ int oracle_expert_backward(const double *x, const double *dy, const double *w, i
     free(row); free(g); free(u); free(h); free(dh);
     return 0;
 }
+
+/* ---------------------------------------------------------------------------
+ * One rank's share of the layer under expert parallelism ([A] section 1:
+ * experts reorganised by device, one group per device; section 2: the shared
+ * experts split across devices): with the router over ALL N experts, the
+ * picks that fall on experts [e0, e0 + n_loc) -- whose weights are given
+ * alone, wg/wu [n_loc][I][d], wd [n_loc][d][I] -- weighted by their global
+ * scores, plus every shared expert restricted to I_s of its intermediate
+ * features (sg/su [S][I_s][d], sd [S][d][I_s]; W_down's matching columns):
+ *   y_r(t) = sum_{picks e in [e0, e0 + n_loc)} p_e FFN_e(x_t)
+ *          + sum_s W_down,s[:, slice] (silu(W_gate,s[slice] x_t) * (W_up,s[slice] x_t)).
+ * Summed over a partition of the experts and of the shared features, the
+ * partials are the layer. Listed tokens only; y_out [n][d].
+ */
+int oracle_layer_ep_partial(const double *x, int T, int d, int N, int M, int Kp, int S, int I,
+                            int dtype, const void *w_router, const float *bias, int e0, int n_loc,
+                            const void *w_gate, const void *w_up, const void *w_down, int I_s,
+                            const void *s_gate, const void *s_up, const void *s_down,
+                            const int32_t *tokens, int n, double *y_out) {
+    if (N % M != 0 || Kp < 1 || Kp > N / M || e0 < 0 || n_loc < 0 || e0 + n_loc > N) return 1;
+    const int K = M * Kp;
+    const size_t per = (size_t)I * d, per_s = (size_t)I_s * d;
+    double *tmp = (double *)malloc(sizeof(double) * (size_t)d);
+    int32_t *idx = (int32_t *)malloc(sizeof(int32_t) * (size_t)K);
+    double *w = (double *)malloc(sizeof(double) * (size_t)K);
+    if (!tmp || !idx || !w) { free(tmp); free(idx); free(w); return 2; }
+    int rc = 0;
+    for (int q = 0; q < n && rc == 0; ++q) {
+        const int t = tokens[q];
+        if (t < 0 || t >= T) { rc = 1; break; }
+        const double *xt = x + (size_t)t * d;
+        double *yt = y_out + (size_t)q * d;
+        double mg;
+        rc = oracle_route(xt, w_router, bias, dtype, 1, d, N, M, Kp, idx, w, &mg);
+        if (rc) break;
+        for (int o = 0; o < d; ++o) yt[o] = 0.0;
+        for (int k = 0; k < K; ++k) {
+            const int e = idx[k];
+            if (e < e0 || e >= e0 + n_loc) continue;
+            const size_t le = (size_t)(e - e0);
+            rc = oracle_expert_ffn(xt, expert_ptr(w_gate, dtype, le, per),
+                                   expert_ptr(w_up, dtype, le, per),
+                                   expert_ptr(w_down, dtype, le, per), dtype, d, I, tmp);
+            if (rc) break;
+            for (int o = 0; o < d; ++o) yt[o] += w[k] * tmp[o];
+        }
+        for (int s = 0; s < S && rc == 0 && I_s > 0; ++s) {
+            rc = oracle_expert_ffn(xt, expert_ptr(s_gate, dtype, (size_t)s, per_s),
+                                   expert_ptr(s_up, dtype, (size_t)s, per_s),
+                                   expert_ptr(s_down, dtype, (size_t)s, per_s), dtype, d, I_s, tmp);
+            for (int o = 0; o < d; ++o) yt[o] += tmp[o];
+        }
+    }
+    free(tmp);
+    free(idx);
+    free(w);
+    return rc;
+}

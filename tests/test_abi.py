@@ -127,3 +127,16 @@ def test_wait_selftest_validates_on_host(L):
     assert L.moge_selftest_waits(2000001, 0x1000, None) == mg.ERR_INVALID_ARG
     assert L.moge_selftest_waits(1000, None, None) == mg.ERR_INVALID_ARG
     assert L.moge_selftest_waits(1000, 0x1002, None) == mg.ERR_UNSUPPORTED
+
+
+def test_expert_parallel_entry_points_validate_on_host(L):
+    c = mg.moge_config(64, 256, 16, 4, 1, 1, 128, mg.MOGE_BF16)
+    assert L.moge_ep_workspace_size(ctypes.byref(c), 4) > 0
+    assert L.moge_ep_workspace_size(ctypes.byref(c), 3) == 0   # 3 does not divide M = 4
+    assert L.moge_ep_workspace_size(ctypes.byref(c), 0) == 0
+    args = [None] * 12
+    assert L.moge_layer_forward_ep_local(ctypes.byref(c), 4, 4, *args) == mg.ERR_INVALID_ARG
+    assert L.moge_layer_forward_ep_local(ctypes.byref(c), 0, 3, *args) == mg.ERR_UNSUPPORTED
+    assert L.moge_layer_forward_ep_local(ctypes.byref(c), 0, 2, *args) == mg.ERR_INVALID_ARG  # y_part NULL
+    assert L.moge_ep_finish(ctypes.byref(c), -1, None, None, None, None) == mg.ERR_INVALID_ARG
+    assert L.moge_ep_finish(ctypes.byref(c), 4, 0x1008, None, 0x1000, None) == mg.ERR_UNSUPPORTED

@@ -49,9 +49,9 @@ def _worker(rank, world, port, out):
 
 def test_two_gloo_ranks_weak_scaling_aggregation():
     world = 2
-    mgr = mp.Manager()
-    out = mgr.dict()
     ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
     port = _free_port()
     procs = [ctx.Process(target=_worker, args=(r, world, port, out)) for r in range(world)]
     for p in procs:
