@@ -356,6 +356,84 @@ def rank_inputs(cfg, rank, with_weights=True):
     return inp
 
 
+def ep_rank_bytes(cfg, world):
+    """Expert-weight bytes one rank streams per expert-parallel step: its N/world
+    routed experts and an I/world slice of every shared expert."""
+    return (cfg.N // world + cfg.S / world) * 3 * cfg.I * cfg.d * 2
+
+
+def run_ep(args, cfg, world, rank, local, dist_on, peaks):
+    """--ep: the layer under expert parallelism (strong scaling: the workload's
+    T tokens split over the ranks; each rank holds N/world experts and an
+    I/world slice of the shared ones; all-gather + reduce-scatter over NCCL)."""
+    import socket
+    import torch
+    import torch.distributed as dist
+    import mixture_grouped_experts_b200 as mg
+    if not dist_on:  # one rank: a world-1 NCCL group, so that the same driver runs
+        sk = socket.socket()
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+        sk.close()
+        dist.init_process_group("nccl", init_method="tcp://127.0.0.1:%d" % port, rank=0,
+                                world_size=1)
+    if cfg.T % world or cfg.M % world or cfg.I % world:
+        raise SystemExit("--ep needs world to divide T, M and I")
+    s = mg.shape_of(cfg)
+    inp = synth.layer_inputs(cfg)
+    rows = cfg.T // world
+    x = mg.to_device(inp["x"][rank * rows:(rank + 1) * rows], cfg.dtype)
+    w = mg.weights_to_device(inp, cfg.dtype)
+    wl = mg.ep_shard_weights(w, rank, world)
+    wl = {k: (v.clone() if torch.is_tensor(v) else v) for k, v in wl.items()}
+    del w, inp
+    torch.cuda.empty_cache()
+    ws = mg.alloc_ep_workspace(s, world)
+
+    def step():
+        return mg.moge_layer_forward_ep(s, x, wl, ws)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    mg.check_device_errors()
+    sampler = ClockSampler(local)
+    sampler.start()
+    stream = torch.cuda.current_stream()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(args.steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    clocks = sampler.stop()
+    mg.check_device_errors()
+    ms = max_over_ranks(start.elapsed_time(end) / args.steps, True)
+    hbm = peaks["hbm_gbs"]
+    rb = ep_rank_bytes(cfg, world)
+    line = {"metric": METRIC, "value": cfg.T / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded normal inputs, random-init weights)",
+            "config": dict(workload_config(cfg),
+                           parallelism="ep%d: groups %d per rank, shared experts split by "
+                                       "features, all-gather + reduce-scatter (NCCL)"
+                                       % (world, cfg.M // world)),
+            "roofline": {"bound": "hbm", "kernel": "whole expert-parallel step (per rank)",
+                         "achieved": rb / (ms / 1e3) / 1e9, "peak": hbm, "unit": "GB/s",
+                         "frac": rb / (ms / 1e3) / 1e9 / hbm,
+                         "algorithmic_bytes_per_rank": rb, "traffic": None},
+            "e2e": None,
+            "gpu_launches": (8 + (2 if cfg.S else 0)) * args.steps,
+            "clocks": clocks}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.destroy_process_group()
+
+
 def job_throughput(tokens_per_rank, world, max_ms):
     """Whole-job tokens/s: all ranks' tokens over the slowest rank's step time."""
     return world * tokens_per_rank / (max_ms / 1e3)
@@ -374,6 +452,8 @@ def main():
     ap.add_argument("--no-fp8", action="store_true", help="skip the 8-bit-weight side measurement")
     ap.add_argument("--no-train", action="store_true", help="skip the training-step side measurement")
     ap.add_argument("--ref-tokens", type=int, default=2, help="tokens per step of --impl reference")
+    ap.add_argument("--ep", action="store_true",
+                    help="expert parallelism over the ranks instead of independent replicas")
     args = ap.parse_args()
     cfg = synth.CONFIGS[args.config]
     if args.impl == "reference":
@@ -395,6 +475,9 @@ def main():
     import mixture_grouped_experts_b200 as mg
     mg.lib()
     peaks, peak_kind = load_peaks()
+    if args.ep:
+        run_ep(args, cfg, world, rank, local, dist_on, peaks)
+        return
 
     inp = rank_inputs(cfg, rank)
     sampler = ClockSampler(local)
