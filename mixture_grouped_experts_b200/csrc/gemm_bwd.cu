@@ -61,8 +61,11 @@ struct GParams {
     const float *bias;      // kLOGITS, nullable
 };
 
+// One work item, with its plan entry's fields held in registers (the copy
+// issue and the epilogues read them every chunk)
 struct GItem {
     int entry, mt, nt, bn, n_valid, nck, kv_last;
+    int a_sel, a_idx, b_sel, src_row0, dst_row0;
 };
 
 struct GShared {
@@ -83,6 +86,7 @@ __device__ __forceinline__ bool g_b_mn(int kind) {
 
 __device__ void g_decode(const GParams &p, const GShared &sh, int q, GItem &it) {
     it.kv_last = 64;
+    it.a_sel = it.a_idx = it.b_sel = it.src_row0 = it.dst_row0 = 0;
     if (g_token_kind(p.kind)) {
         int lo = 0, hi = p.n_entries - 1;
         while (lo < hi) {  // last entry whose first item is <= q
@@ -92,6 +96,8 @@ __device__ void g_decode(const GParams &p, const GShared &sh, int q, GItem &it) 
         const ExpertWork &w = p.ent[lo];
         const int r = q - sh.start[lo];
         it.entry = lo;
+        it.a_sel = w.a_sel; it.a_idx = w.a_idx; it.b_sel = w.b_sel;
+        it.src_row0 = w.src_row0; it.dst_row0 = w.dst_row0;
         it.mt = r / w.ntb;
         it.nt = r % w.ntb;
         it.bn = w.bn;
@@ -106,7 +112,10 @@ __device__ void g_decode(const GParams &p, const GShared &sh, int q, GItem &it) 
         it.nt = r % p.n_tiles;
         it.bn = p.bn;
         it.n_valid = p.bn;
-        const int rows = p.ent[it.entry].rows;
+        const ExpertWork &w = p.ent[it.entry];
+        const int rows = w.rows;
+        it.a_sel = w.a_sel; it.a_idx = w.a_idx; it.b_sel = w.b_sel;
+        it.src_row0 = w.src_row0; it.dst_row0 = w.dst_row0;
         it.nck = (rows + 63) / 64;
         it.kv_last = rows - 64 * (it.nck - 1);
     } else {
@@ -124,28 +133,27 @@ __device__ void g_decode(const GParams &p, const GShared &sh, int q, GItem &it) 
 __device__ __forceinline__ void g_load(const GParams &p, const GMaps &mp, const GItem &it, int kc,
                                        int j, unsigned char *stage, uint64_t *bar, uint64_t pol_a,
                                        uint64_t pol_b) {
-    const ExpertWork *w = g_token_kind(p.kind) || g_wgrad_kind(p.kind) ? &p.ent[it.entry] : nullptr;
     const int k = 64 * kc;
     if (j < 2) {
         unsigned char *dst = stage + 8192 * j;
         const int mn = it.mt * 128 + 64 * j;
         switch (p.kind) {
             case kDH:  // Wd[e] as [d][I]: rows are K
-                tma_load_3d(dst, &mp.m[w->a_sel], bar, mn, k, w->a_idx, pol_a);
+                tma_load_3d(dst, &mp.m[it.a_sel], bar, mn, k, it.a_idx, pol_a);
                 break;
             case kDX: {  // Wg[e] then Wu[e], as [I][d]: rows are K
                 const int kh = p.I / 64;
-                const int sel = (kc < kh ? 0 : 2) + w->a_sel;
-                tma_load_3d(dst, &mp.m[sel], bar, mn, kc < kh ? k : k - p.I, w->a_idx, pol_a);
+                const int sel = (kc < kh ? 0 : 2) + it.a_sel;
+                tma_load_3d(dst, &mp.m[sel], bar, mn, kc < kh ? k : k - p.I, it.a_idx, pol_a);
                 break;
             }
             case kDWD:  // dy rows (dy_perm / dy) read across: rows are K
-                tma_load_2d(dst, &mp.m[w->b_sel], bar, mn, w->src_row0 + k, pol_a);
+                tma_load_2d(dst, &mp.m[it.b_sel], bar, mn, it.src_row0 + k, pol_a);
                 break;
             case kDWGU: {  // [g | u] rows read across
                 const int part = it.mt / p.m_tiles;
                 const int m0 = (it.mt - part * p.m_tiles) * 128 + 64 * j + part * p.I;
-                tma_load_2d(dst, &mp.m[0], bar, m0, w->dst_row0 + k, pol_a);
+                tma_load_2d(dst, &mp.m[0], bar, m0, it.dst_row0 + k, pol_a);
                 break;
             }
             case kLOGITS:  // Wr rows, K-major
@@ -161,16 +169,16 @@ __device__ __forceinline__ void g_load(const GParams &p, const GMaps &mp, const 
         const int r0 = it.nt * it.bn + 64 * jb;  // first N element of the box
         switch (p.kind) {
             case kDH:  // dy rows, K-major
-                tma_load_2d(dst, &mp.m[2 + w->b_sel], bar, k, w->src_row0 + r0, pol_b);
+                tma_load_2d(dst, &mp.m[2 + it.b_sel], bar, k, it.src_row0 + r0, pol_b);
                 break;
             case kDX:  // [dg | du] rows, K-major
-                tma_load_2d(dst, &mp.m[4], bar, k, w->dst_row0 + r0, pol_b);
+                tma_load_2d(dst, &mp.m[4], bar, k, it.dst_row0 + r0, pol_b);
                 break;
             case kDWD:  // h rows read across
-                tma_load_2d(dst, &mp.m[2], bar, r0, w->dst_row0 + k, pol_b);
+                tma_load_2d(dst, &mp.m[2], bar, r0, it.dst_row0 + k, pol_b);
                 break;
             case kDWGU:  // x rows (x_perm / x) read across
-                tma_load_2d(dst, &mp.m[2 + w->b_sel], bar, r0, w->src_row0 + k, pol_b);
+                tma_load_2d(dst, &mp.m[2 + it.b_sel], bar, r0, it.src_row0 + k, pol_b);
                 break;
             case kDWR:  // x read across
                 tma_load_2d(dst, &mp.m[1], bar, r0, k, pol_b);
@@ -215,8 +223,7 @@ __device__ __forceinline__ void g_store_rows(const GParams &p, const GItem &it, 
 #pragma unroll
     for (int j = 0; j < 32; ++j) S[j * 128 + m] = __uint_as_float(v[j]);
     named_bar_sync(1, 128);
-    const ExpertWork &w = p.ent[it.entry];
-    const size_t row_base = (size_t)w.dst_row0 + (size_t)it.nt * it.bn + c0;
+    const size_t row_base = (size_t)it.dst_row0 + (size_t)it.nt * it.bn + c0;
     const int f0 = it.mt * 128;
     if (p.kind == kDH) {
         const size_t ld = 2 * (size_t)p.I;
@@ -343,13 +350,12 @@ __device__ __forceinline__ void g_store_wgrad(const GParams &p, const GMaps &mp,
     if (p.kind == kDWR) {
         map = &mp.m[6]; row0 = it.mt * 128; e = 0; rows = p.N; cols = p.d;
     } else {
-        const ExpertWork &w = p.ent[it.entry];
-        e = w.a_idx;
+        e = it.a_idx;
         if (p.kind == kDWD) {
-            map = &mp.m[6 + w.a_sel]; row0 = it.mt * 128; rows = p.d; cols = p.I;
+            map = &mp.m[6 + it.a_sel]; row0 = it.mt * 128; rows = p.d; cols = p.I;
         } else {
             const int part = it.mt / p.m_tiles;
-            map = &mp.m[6 + 2 * part + w.a_sel]; row0 = (it.mt - part * p.m_tiles) * 128;
+            map = &mp.m[6 + 2 * part + it.a_sel]; row0 = (it.mt - part * p.m_tiles) * 128;
             rows = p.I; cols = p.d;
         }
     }

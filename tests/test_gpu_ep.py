@@ -18,7 +18,7 @@ import torch
 import mixture_grouped_experts_b200 as mg
 import oracle
 import synth
-from gpu_helpers import MARGIN, TOL, normwise_err, to_host_f64
+from gpu_helpers import MARGIN, TOL, normwise_err, sample_tokens, to_host_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -121,5 +121,37 @@ def test_nccl_driver_world_one():
     x = oracle.to_double(inp["x"], cfg.dtype)
     toks = _clear_tokens(cfg, inp, x)
     assert normwise_err(to_host_f64(y)[toks], to_host_f64(y1)[toks]) <= TOL[cfg.dtype]
+    y_ref, _, _, _ = oracle.layer(x, inp, cfg.M, cfg.Kp, cfg.dtype, tokens=toks)
+    assert normwise_err(to_host_f64(y)[toks], y_ref) <= TOL[cfg.dtype]
+
+
+def test_full_size_decode_eight_ranks_sampled():
+    """The decode workload (T = 456, d = 5120, 64 experts in 8 groups, K' = 1,
+    4 shared, I = 1344) split over 8 ranks, one group each and 168 features of
+    every shared expert, the ranks run in turn: sampled tokens of the summed
+    partials against the oracle's layer, and one rank's partial against the
+    oracle's partial for that rank."""
+    cfg = synth.CONFIGS["decode"]
+    world = 8
+    inp = synth.layer_inputs(cfg)
+    x = oracle.to_double(inp["x"], cfg.dtype)
+    s = mg.shape_of(cfg)
+    xd = mg.to_device(inp["x"], cfg.dtype)
+    w = mg.weights_to_device(inp, cfg.dtype)
+    ws = mg.alloc_ep_workspace(s, world)
+    clear = set(_clear_tokens(cfg, inp, x).tolist())
+    toks = np.array([t for t in sample_tokens(cfg.T, 12) if t in clear])
+    assert len(toks) >= 8
+    total = torch.zeros((cfg.T, cfg.d), dtype=torch.float32, device="cuda")
+    for r in range(world):
+        part = mg.moge_layer_forward_ep_local(s, r, world, xd, mg.ep_shard_weights(w, r, world), ws)
+        if r == 3:
+            ref = _oracle_partial(cfg, inp, x, r, world, toks)
+            torch.cuda.synchronize()
+            assert normwise_err(to_host_f64(part)[toks], ref) <= TOL[cfg.dtype]
+        total += part
+    torch.cuda.synchronize()
+    mg.check_device_errors()
+    y = mg.moge_ep_finish(s, total)
     y_ref, _, _, _ = oracle.layer(x, inp, cfg.M, cfg.Kp, cfg.dtype, tokens=toks)
     assert normwise_err(to_host_f64(y)[toks], y_ref) <= TOL[cfg.dtype]
