@@ -328,23 +328,34 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap *m, const void *s
                  : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// at most one committed store group may still be reading shared memory
-__device__ __forceinline__ void bulk_wait_read_1() {
-    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_read_7() {
-    asm volatile("cp.async.bulk.wait_group.read 7;" ::: "memory");
+__device__ __forceinline__ void bulk_wait_read_3() {
+    asm volatile("cp.async.bulk.wait_group.read 3;" ::: "memory");
 }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-// Weight-gradient epilogue of one 32-column chunk for one warp: lane r holds
-// row (32 q4 + r) of the tile; the warp writes its [32][32] bf16 block into a
-// staging tile (a ring of 8 per warp, or 2 when no stage was freed: `deep`)
-// and lane 0 stores it with TMA.
-// Rows and columns past the tensor are clipped by the copy.
+// Weight-gradient epilogue of 64 columns (two 32-column chunks: va, and vb
+// when `two`) for one warp: lane r holds row (32 q4 + r) of the tile; the warp
+// writes its two [32][32] bf16 blocks into a pair of staging tiles (a ring of
+// 4 pairs per warp; 64-byte swizzle, the output maps') and lane 0 stores them
+// with TMA as one bulk group. Blocks wholly past the tensor are skipped; rows
+// and columns partly past it are clipped by the copy.
+__device__ __forceinline__ void g_stage_block(unsigned char *tile, int lane, const uint32_t (&v)[32]) {
+    uint4 *dst = reinterpret_cast<uint4 *>(tile + lane * 64);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint4 o;
+        o.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1]));
+        o.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
+        o.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
+        o.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
+        dst[q ^ ((lane >> 1) & 3)] = o;  // 16-byte chunk q of row r at q ^ ((r >> 1) & 3)
+    }
+}
+
 __device__ __forceinline__ void g_store_wgrad(const GParams &p, const GMaps &mp, const GItem &it,
-                                              int q4, int lane, int c0, const uint32_t (&v)[32],
-                                              unsigned char *stage_tile, bool deep) {
+                                              int q4, int lane, int c0, const uint32_t (&va)[32],
+                                              const uint32_t (&vb)[32], bool two,
+                                              unsigned char *pair) {
     const CUtensorMap *map;
     int row0, e, rows, cols;
     if (p.kind == kDWR) {
@@ -362,25 +373,16 @@ __device__ __forceinline__ void g_store_wgrad(const GParams &p, const GMaps &mp,
     row0 += 32 * q4;
     const int col0 = it.nt * it.bn + c0;
     if (row0 >= rows || col0 >= cols) return;  // wholly past the tensor: nothing to store
-    if (lane == 0) {  // this staging tile's previous store has read it
-        if (deep) bulk_wait_read_7(); else bulk_wait_read_1();
-    }
+    const bool second = two && col0 + 32 < cols;
+    if (lane == 0) bulk_wait_read_3();  // this pair's previous stores have read it
     __syncwarp();
-    // 64-byte swizzle (the map's): 16-byte chunk q of row r at q ^ ((r >> 1) & 3)
-    uint4 *dst = reinterpret_cast<uint4 *>(stage_tile + lane * 64);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        uint4 o;
-        o.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1]));
-        o.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
-        o.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
-        o.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
-        dst[q ^ ((lane >> 1) & 3)] = o;
-    }
+    g_stage_block(pair, lane, va);
+    if (second) g_stage_block(pair + 2048, lane, vb);
     fence_proxy_async();
     __syncwarp();
     if (lane == 0) {
-        tma_store_3d(map, stage_tile, col0, row0, e);
+        tma_store_3d(map, pair, col0, row0, e);
+        if (second) tma_store_3d(map, pair + 2048, col0 + 32, row0, e);
         bulk_commit();
     }
 }
@@ -541,12 +543,10 @@ __global__ void __launch_bounds__(kGThreads, 1) bwd_gemm_kernel(const __grid_con
         const bool wgrad = g_wgrad_kind(p.kind) || p.kind == kDWR;
         const bool rowk = g_token_kind(p.kind);
         const int et = threadIdx.x - 64;
-        // weight-gradient staging: the freed 4th stage and the epilogue area (64 KB,
-        // 16 KB per warp) when 3 stages run, else the epilogue area alone
-        const bool deep = nst < kGStages;
-        unsigned char *wstage = deep ? stages + (size_t)nst * kGStageBytes : epi;
-        const int nbuf = deep ? 8 : 2;
-        int i = 0, chunk = 0;
+        // weight-gradient staging (these kinds run 3 stages): the freed 4th stage and
+        // the epilogue area, 64 KB, 16 KB per warp = 4 pairs of [32][32] bf16 tiles
+        unsigned char *wstage = stages + (size_t)(kGStages - 1) * kGStageBytes + q4 * 16384;
+        int i = 0, pairs = 0;
         for (int q = blockIdx.x; q < total; q += gridDim.x, ++i) {
             GItem it;
             g_decode(p, sh, q, it);
@@ -555,7 +555,24 @@ __global__ void __launch_bounds__(kGThreads, 1) bwd_gemm_kernel(const __grid_con
             tc_fence_after();
             const uint32_t tbase = tmem_base + ((uint32_t)(32 * q4) << 16) + (uint32_t)acc * 256u;
             const bool zero = it.nck == 0;
-            for (int c0 = 0; c0 < it.n_valid; c0 += 32) {
+            if (wgrad) {  // 64 columns per TMEM wait, two staging tiles, one store group
+                for (int c0 = 0; c0 < it.n_valid; c0 += 64) {
+                    const bool two = c0 + 32 < it.n_valid;
+                    uint32_t va[32], vb[32];
+                    if (!zero) {
+                        tmem_ld_32x32b_x32(tbase + (uint32_t)c0, va);
+                        if (two) tmem_ld_32x32b_x32(tbase + (uint32_t)c0 + 32u, vb);
+                        tmem_ld_wait();
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) va[j] = vb[j] = 0u;
+                    }
+                    g_store_wgrad(p, mp, it, q4, lane, c0, va, vb, two,
+                                  wstage + (size_t)(pairs & 3) * 4096);
+                    ++pairs;
+                }
+            }
+            for (int c0 = 0; !wgrad && c0 < it.n_valid; c0 += 32) {
                 uint32_t v[32];
                 if (!zero) {
                     tmem_ld_32x32b_x32(tbase + (uint32_t)c0, v);
@@ -564,11 +581,7 @@ __global__ void __launch_bounds__(kGThreads, 1) bwd_gemm_kernel(const __grid_con
 #pragma unroll
                     for (int j = 0; j < 32; ++j) v[j] = 0u;
                 }
-                if (wgrad) {
-                    g_store_wgrad(p, mp, it, q4, lane, c0, v,
-                                  wstage + (size_t)(q4 * nbuf + chunk % nbuf) * 2048, deep);
-                    ++chunk;
-                } else if (rowk) {
+                if (rowk) {
                     g_store_rows(p, it, m, et, c0, v, reinterpret_cast<float *>(epi));
                 } else {
                     g_store(p, it, m, c0, v, zero);
