@@ -221,7 +221,7 @@ struct TrainSpace {
     Workspace fw;
     void *gu;        // [hrows][2I]
     void *dy_perm;   // [rrows][d]
-    float *logits;   // [T][N]
+    float *logits;   // [kMaxLogitSplit][T][N]: partial logits, one per K part
     void *dl;        // [T][N]
     float *dx_r;     // [T][d]
     float *dw;       // [T][K]
@@ -241,7 +241,7 @@ static TrainSpace carve_train(const moge_config &c, void *base) {
     };
     s.gu = take(T * (K + c.S) * 2 * (size_t)c.I * 2);
     s.dy_perm = take(T * K * c.d * 2);
-    s.logits = (float *)take(T * c.N * 4);
+    s.logits = (float *)take((size_t)kMaxLogitSplit * T * c.N * 4);  // one [T][N] per K part
     s.dl = take(T * c.N * 2);
     s.dx_r = (float *)take(T * c.d * 4);
     s.dw = (float *)take(T * K * 4);
@@ -721,8 +721,8 @@ int moge_layer_backward(const moge_config *cfg, float alpha, const void *x, cons
     MOGE_CU(launch_combine_bwd(c, dy, ws.y_perm, ws.topk_w, ws.perm_dst, ts.dy_perm, ts.dw, st),
             "combine backward launch");
     MOGE_CU(launch_bwd_gemm(kLOGITS, c, ent, E, b, sms, st), "logits launch");
-    MOGE_CU(launch_router_bwd(c, alpha, ts.logits, ws.topk_idx, ts.dw, ws.counts, ts.dl, ts.part,
-                              aux, st), "router backward launch");
+    MOGE_CU(launch_router_bwd(c, alpha, ts.logits, logits_ksplit(c, sms), ws.topk_idx, ts.dw,
+                              ws.counts, ts.dl, ts.part, aux, st), "router backward launch");
     MOGE_CU(launch_bwd_gemm(kDH, c, ent, E, b, sms, st), "dh launch");
     MOGE_CU(launch_bwd_gemm(kDX, c, ent, E, b, sms, st), "dx launch");
     MOGE_CU(launch_bwd_gemm(kDWD, c, ent, E, b, sms, st), "dW_down launch");

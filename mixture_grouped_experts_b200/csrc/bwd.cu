@@ -78,10 +78,11 @@ __global__ void __launch_bounds__(kBwdThreads) combine_bwd_kernel(
 // l holding experts l, l + 32, ...; also each CTA's sums of p over its tokens
 // (part[blockIdx.x][e], fixed order) for the balance loss.
 __global__ void __launch_bounds__(32 * kRouterBwdWarps) router_bwd_kernel(
-    moge_config c, float alpha, const float *__restrict__ logits,
+    moge_config c, float alpha, const float *__restrict__ logits, int ksplit,
     const int32_t *__restrict__ topk_idx, const float *__restrict__ dw,
     const int32_t *__restrict__ counts, uint16_t *dl, float *part) {
     __shared__ float psum[kRouterBwdWarps][kMaxExperts];
+    const size_t part_stride = (size_t)c.T * c.N;  // the logit GEMM's K parts
     grid_dependency_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int N = c.N, K = c.M * c.Kp;
@@ -99,7 +100,12 @@ __global__ void __launch_bounds__(32 * kRouterBwdWarps) router_bwd_kernel(
 #pragma unroll
         for (int j = 0; j < kPer; ++j) {
             const int e = lane + 32 * j;
-            pr[j] = (j < per && e < N) ? logits[(size_t)t * N + e] : -INFINITY;
+            float l = -INFINITY;
+            if (j < per && e < N) {
+                l = logits[(size_t)t * N + e];
+                for (int k = 1; k < ksplit; ++k) l += logits[k * part_stride + (size_t)t * N + e];
+            }
+            pr[j] = l;
             mx = fmaxf(mx, pr[j]);
         }
         for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -210,12 +216,12 @@ cudaError_t launch_combine_bwd(const moge_config &c, const void *dy, const void 
 
 int router_bwd_parts(const moge_config &c) { return (c.T + kRouterBwdTokens - 1) / kRouterBwdTokens; }
 
-cudaError_t launch_router_bwd(const moge_config &c, float alpha, const float *logits,
+cudaError_t launch_router_bwd(const moge_config &c, float alpha, const float *logits, int ksplit,
                               const int32_t *topk_idx, const float *dw, const int32_t *counts,
                               void *dl, float *part, float *aux, cudaStream_t st) {
     const int parts = router_bwd_parts(c);
     cudaError_t e = launch_pdl(router_bwd_kernel, dim3(parts), dim3(32 * kRouterBwdWarps), 0, st, c,
-                               alpha, logits, topk_idx, dw, counts, (uint16_t *)dl, part);
+                               alpha, logits, ksplit, topk_idx, dw, counts, (uint16_t *)dl, part);
     if (e != cudaSuccess || !aux) return e;
     return launch_pdl(aux_loss_kernel, dim3(1), dim3(256), 0, st, c, alpha, (const float *)part,
                       parts, counts, aux);

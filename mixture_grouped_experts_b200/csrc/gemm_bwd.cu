@@ -54,6 +54,7 @@ struct GParams {
     int m_tiles;            // M tiles per entry (per part for kDWGU)
     int n_tiles, bn;        // weight-gradient and router kinds: N tiles and their width
     int kc;                 // K chunks of the fixed-K kinds
+    int ksplit;             // kLOGITS: K split into this many parts, partial logits per part
     int nst;                // pipeline stages in use (3 for the weight-gradient kinds, whose
                             // freed stage holds the epilogue's store staging tiles)
     void *out[4];
@@ -66,6 +67,7 @@ struct GParams {
 struct GItem {
     int entry, mt, nt, bn, n_valid, nck, kv_last;
     int a_sel, a_idx, b_sel, src_row0, dst_row0;
+    int ks, kc0;  // kLOGITS: K part and its first chunk
 };
 
 struct GShared {
@@ -87,6 +89,7 @@ __device__ __forceinline__ bool g_b_mn(int kind) {
 __device__ void g_decode(const GParams &p, const GShared &sh, int q, GItem &it) {
     it.kv_last = 64;
     it.a_sel = it.a_idx = it.b_sel = it.src_row0 = it.dst_row0 = 0;
+    it.ks = it.kc0 = 0;
     if (g_token_kind(p.kind)) {
         int lo = 0, hi = p.n_entries - 1;
         while (lo < hi) {  // last entry whose first item is <= q
@@ -120,12 +123,19 @@ __device__ void g_decode(const GParams &p, const GShared &sh, int q, GItem &it) 
         it.kv_last = rows - 64 * (it.nck - 1);
     } else {
         it.entry = 0;
+        const int ksp = p.kind == kLOGITS ? p.ksplit : 1;
+        it.ks = q % ksp;
+        q /= ksp;
         it.mt = q / p.n_tiles;
         it.nt = q % p.n_tiles;
         it.bn = p.bn;
         const int ncols = p.kind == kDWR ? p.d : p.T;
         it.n_valid = min(p.bn, ncols - it.nt * p.bn);
         it.nck = p.kind == kDWR ? (p.T + 63) / 64 : p.kc;
+        if (ksp > 1) {  // chunks [kc0, kc0 + nck) of this part
+            it.kc0 = it.ks * it.nck / ksp;
+            it.nck = (it.ks + 1) * it.nck / ksp - it.kc0;
+        }
     }
 }
 
@@ -133,7 +143,7 @@ __device__ void g_decode(const GParams &p, const GShared &sh, int q, GItem &it) 
 __device__ __forceinline__ void g_load(const GParams &p, const GMaps &mp, const GItem &it, int kc,
                                        int j, unsigned char *stage, uint64_t *bar, uint64_t pol_a,
                                        uint64_t pol_b) {
-    const int k = 64 * kc;
+    const int k = 64 * (kc + it.kc0);
     if (j < 2) {
         unsigned char *dst = stage + 8192 * j;
         const int mn = it.mt * 128 + 64 * j;
@@ -294,8 +304,8 @@ __device__ __forceinline__ void g_store(const GParams &p, const GItem &it, int m
         case kLOGITS: {
             const int e = it.mt * 128 + m;
             if (e >= p.N) return;
-            float *l = static_cast<float *>(p.out[0]);
-            const float b = p.bias ? p.bias[e] : 0.0f;
+            float *l = static_cast<float *>(p.out[0]) + (size_t)it.ks * p.T * p.N;
+            const float b = (p.bias && it.ks == 0) ? p.bias[e] : 0.0f;
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
                 const int c = c0 + j;
@@ -435,7 +445,7 @@ __global__ void __launch_bounds__(kGThreads, 1) bwd_gemm_kernel(const __grid_con
         } else if (g_wgrad_kind(p.kind)) {
             tot = p.n_entries * (p.kind == kDWGU ? 2 : 1) * p.m_tiles * p.n_tiles;
         } else {
-            tot = p.m_tiles * p.n_tiles;
+            tot = p.m_tiles * p.n_tiles * (p.kind == kLOGITS ? p.ksplit : 1);
         }
         sh.total = tot;
     }
@@ -634,6 +644,17 @@ static bool g_out(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows
               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// K parts of the recomputed router logits: enough items for the SMs (the
+// GEMM is small: one or two 128-row tiles of experts), at most kMaxLogitSplit
+int logits_ksplit(const moge_config &c, int num_sms) {
+    const int tiles = ((c.N + 127) / 128) * ((c.T + 255) / 256);
+    const int kc = (c.d + 63) / 64;
+    int ks = num_sms / (tiles > 0 ? tiles : 1);
+    ks = ks < kMaxLogitSplit ? ks : kMaxLogitSplit;
+    ks = ks < kc / 2 ? ks : kc / 2;
+    return ks > 1 ? ks : 1;
+}
+
 static size_t g_smem_bytes() {
     return 1024 + (size_t)kGStages * kGStageBytes + kGEpiBytes + sizeof(GShared);
 }
@@ -703,7 +724,8 @@ cudaError_t launch_bwd_gemm(int kind, const moge_config &c, const ExpertWork *en
             g_ntiles(T, p.n_tiles, p.bn);
             p.out[0] = b.logits;
             p.bias = b.bias;
-            total = p.m_tiles * p.n_tiles;
+            p.ksplit = logits_ksplit(c, num_sms);
+            total = p.m_tiles * p.n_tiles * p.ksplit;
             break;
         case kDWR:
             ok = g_rows(&mp.m[0], b.dl, N, T) && g_rows(&mp.m[1], b.x, d, T) &&

@@ -167,11 +167,15 @@ struct BwdTensors {
 enum : int { kDH = 0, kDX = 1, kDWD = 2, kDWGU = 3, kLOGITS = 4, kDWR = 5, kDXR = 6 };
 cudaError_t launch_bwd_gemm(int kind, const moge_config &c, const ExpertWork *ent, int n_entries,
                             const BwdTensors &b, int num_sms, cudaStream_t st);
+// K parts of the backward's router-logit GEMM (each writes its own [T][N]
+// partial, summed in order by the router backward); at most kMaxLogitSplit
+constexpr int kMaxLogitSplit = 16;
+int logits_ksplit(const moge_config &c, int num_sms);
 cudaError_t launch_combine_bwd(const moge_config &c, const void *dy, const void *y_perm,
                                const float *topk_w, const int32_t *perm_dst, void *dy_perm,
                                float *dw, cudaStream_t st);
 int router_bwd_parts(const moge_config &c);
-cudaError_t launch_router_bwd(const moge_config &c, float alpha, const float *logits,
+cudaError_t launch_router_bwd(const moge_config &c, float alpha, const float *logits, int ksplit,
                               const int32_t *topk_idx, const float *dw, const int32_t *counts,
                               void *dl, float *part, float *aux, cudaStream_t st);
 cudaError_t launch_unpermute_bwd(const moge_config &c, const void *dx_perm, const int32_t *perm_dst,
