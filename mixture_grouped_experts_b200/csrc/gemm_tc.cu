@@ -45,7 +45,7 @@ namespace moge {
 
 constexpr int kStages = 4;
 constexpr int kStageBytes = 48 * 1024;
-constexpr int kEpiBytes = 12 * 1024;
+constexpr int kEpiBytes = 16 * 1024;  // U fp32 [32][64], H and G bf16 [32][64]
 constexpr int kTcThreads = 192;
 constexpr int kChunkK = 64;          // bf16 elements per K-chunk (128 bytes, one swizzle row)
 constexpr int kBoxRows = 64;         // token rows per TMA box (one 8 KB copy per chunk)
@@ -391,15 +391,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
                     // lanes 0-63 hold gate and 64-127 up, or the reverse for an up-first tile
                     const bool gate_hi = p.gu_mode[it.w.a_sel] == kUpGateFused;
                     const bool is_gate = (q4 < 2) != gate_hi;
+                    uint16_t *G = reinterpret_cast<uint16_t *>(epi + 12288);  // [32 cols][64 features]
                     const int f = (q4 & 1) * 32 + lane;
-                    if (p.gu && it.fb * 64 + f < p.I) {  // keep g / u for the backward pass
-                        uint16_t *dst = p.gu + (row0 + c0) * 2 * (size_t)p.I + (is_gate ? 0 : p.I) +
-                                        it.fb * 64 + f;
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (c0 + j < it.n_valid)
-                                dst[(size_t)j * 2 * p.I] = to_bf16_bits(__uint_as_float(v[j]));
-                    }
                     if (!is_gate) {
 #pragma unroll
                         for (int j = 0; j < 32; ++j) U[j * 64 + f] = __uint_as_float(v[j]);
@@ -411,15 +404,26 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
                             const float g = __uint_as_float(v[j]);
                             const float hv = g / (1.0f + expf(-g)) * U[j * 64 + f];
                             H[j * 64 + f] = to_bf16_bits(hv);
+                            if (p.gu) G[j * 64 + f] = to_bf16_bits(g);
                         }
                     }
                     named_bar_sync(1, 128);
                     for (int idx = et; idx < 32 * 8; idx += 128) {
                         const int r = idx >> 3, vv = idx & 7;
                         const int col = c0 + r, feat = it.fb * 64 + vv * 8;
-                        if (col < it.n_valid && feat < p.I)
+                        if (col < it.n_valid && feat < p.I) {
                             *reinterpret_cast<uint4 *>(p.h + (row0 + col) * p.I + feat) =
                                 *reinterpret_cast<const uint4 *>(H + r * 64 + vv * 8);
+                            if (p.gu) {  // keep g and u (bf16) for the backward pass
+                                uint16_t *dst = p.gu + (row0 + col) * 2 * (size_t)p.I + feat;
+                                *reinterpret_cast<uint4 *>(dst) =
+                                    *reinterpret_cast<const uint4 *>(G + r * 64 + vv * 8);
+                                const float *u8 = U + r * 64 + vv * 8;
+                                *reinterpret_cast<uint4 *>(dst + p.I) =
+                                    make_uint4(pack_bf16x2(u8[0], u8[1]), pack_bf16x2(u8[2], u8[3]),
+                                               pack_bf16x2(u8[4], u8[5]), pack_bf16x2(u8[6], u8[7]));
+                            }
+                        }
                     }
                     named_bar_sync(1, 128);
                 } else {
