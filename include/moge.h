@@ -153,6 +153,25 @@ MOGE_API int moge_layer_forward_host(const moge_config *cfg, const void *x_host,
                             const void *s_down, void *y_host, void *x_dev, void *y_dev,
                             void *workspace, void *stream);
 
+/* A run of independent batches through the layer from and to host memory,
+ * with the copies overlapped with the compute: batch i's input x_host + i*T*d
+ * is copied in while batch i-1 is computed and batch i-2's output copied out
+ * (a host-to-device and a device-to-host stream of the library's own, per
+ * device, ordered by events; the layer runs on `stream`). x_host, y_host:
+ * [n_batches][T][d] in cfg->dtype, page-locked for the copies to overlap;
+ * x_dev2, y_dev2: caller-owned device buffers of 2*T*d elements (two per
+ * direction). Returns after every output has arrived in y_host. Same weights,
+ * workspace and rules as moge_layer_forward (no residual). The copy streams
+ * are shared by the calls on one device: do not run two such calls on one
+ * device at the same time (from two host threads). */
+MOGE_API int moge_layer_forward_host_stream(const moge_config *cfg, int64_t n_batches,
+                                            const void *x_host, const void *w_router,
+                                            const float *logit_bias, const void *w_gate,
+                                            const void *w_up, const void *w_down,
+                                            const void *s_gate, const void *s_up,
+                                            const void *s_down, void *y_host, void *x_dev2,
+                                            void *y_dev2, void *workspace, void *stream);
+
 /* Device pointers, inside `workspace`, of the routing written by the last
  * moge_layer_forward on it: topk_idx [T][K], topk_w [T][K], counts [N],
  * offsets [N+1] (any out pointer may be NULL). Host-only arithmetic. */

@@ -32,7 +32,8 @@ EXPORTS = ["moge_workspace_size", "moge_last_error", "moge_check_device_errors",
            "moge_rmsnorm", "moge_stage_timing", "moge_stage_times", "moge_route_noalloc",
            "moge_quantize_fp8_rows", "moge_layer_forward_fp8", "moge_selftest_waits",
            "moge_train_workspace_size", "moge_layer_forward_train", "moge_layer_backward",
-           "moge_ep_workspace_size", "moge_layer_forward_ep_local", "moge_ep_finish"]
+           "moge_ep_workspace_size", "moge_layer_forward_ep_local", "moge_ep_finish",
+           "moge_layer_forward_host_stream"]
 STAGES = ("router", "scan", "permute", "ffn", "combine")
 
 
@@ -116,6 +117,7 @@ def lib() -> ctypes.CDLL:
         L.moge_ep_workspace_size.restype = ctypes.c_size_t
         L.moge_layer_forward_ep_local.argtypes = [cp, i32, i32] + [vp] * 12
         L.moge_ep_finish.argtypes = [cp, ctypes.c_int64, vp, vp, vp, vp]
+        L.moge_layer_forward_host_stream.argtypes = [cp, ctypes.c_int64] + [vp] * 14
         for n in EXPORTS:
             if n not in ("moge_workspace_size", "moge_last_error", "moge_train_workspace_size",
                          "moge_ep_workspace_size"):
@@ -369,6 +371,20 @@ def moge_layer_forward_host(s: LayerShape, x_host, w: dict, workspace, y_host, x
                                        _p(w["w_down"]), _p(w.get("s_gate")), _p(w.get("s_up")),
                                        _p(w.get("s_down")), _p(y_host), _p(x_dev), _p(y_dev),
                                        _p(workspace), _stream(stream)))
+    return y_host
+
+
+def moge_layer_forward_host_stream(s: LayerShape, x_host, w: dict, workspace, y_host, x_dev2,
+                                   y_dev2, stream=None):
+    """A run of independent batches from and to (pinned) host memory, copies
+    overlapped with compute: x_host, y_host [n][T][d]; x_dev2, y_dev2 [2][T][d]
+    device buffers. Returns after every output is in y_host."""
+    _chk(lib().moge_layer_forward_host_stream(ctypes.byref(_cfg(s)), int(x_host.shape[0]),
+                                              _p(x_host), _p(w["w_router"]), _p(w.get("logit_bias")),
+                                              _p(w["w_gate"]), _p(w["w_up"]), _p(w["w_down"]),
+                                              _p(w.get("s_gate")), _p(w.get("s_up")),
+                                              _p(w.get("s_down")), _p(y_host), _p(x_dev2),
+                                              _p(y_dev2), _p(workspace), _stream(stream)))
     return y_host
 
 

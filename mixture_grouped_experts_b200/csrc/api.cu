@@ -1,6 +1,7 @@
 // C ABI of the MoGE layer (declared in include/moge.h): argument checks,
 // workspace carve-up and the launch sequences. No entry point allocates
 // device memory; all of them only enqueue work on the caller's stream.
+#include <mutex>
 #include <string.h>
 
 #include <string>
@@ -314,6 +315,37 @@ static EpSpace carve_ep(const moge_config &c, const moge_config &loc, const moge
     return e;
 }
 
+
+// Streams and events of the pipelined host-buffer call, created once per
+// device: a host-to-device and a device-to-host copy stream, and per device
+// buffer (two) "copied in", "computed" and "copied out" events.
+struct HostPipe {
+    cudaStream_t in = nullptr, out = nullptr;
+    cudaEvent_t copied_in[2] = {}, computed[2] = {}, copied_out[2] = {};
+    bool ready = false;
+};
+static int host_pipe(HostPipe *&hp) {
+    static HostPipe pipes[64];
+    static std::mutex mu;
+    int dev = 0;
+    MOGE_CU(cudaGetDevice(&dev), "cudaGetDevice");
+    if (dev < 0 || dev >= 64) return fail(MOGE_ERR_UNSUPPORTED, "device index >= 64");
+    std::lock_guard<std::mutex> lock(mu);
+    HostPipe &p = pipes[dev];
+    if (!p.ready) {
+        MOGE_CU(cudaStreamCreateWithFlags(&p.in, cudaStreamNonBlocking), "copy stream");
+        MOGE_CU(cudaStreamCreateWithFlags(&p.out, cudaStreamNonBlocking), "copy stream");
+        for (int b = 0; b < 2; ++b) {
+            MOGE_CU(cudaEventCreateWithFlags(&p.copied_in[b], cudaEventDisableTiming), "event");
+            MOGE_CU(cudaEventCreateWithFlags(&p.computed[b], cudaEventDisableTiming), "event");
+            MOGE_CU(cudaEventCreateWithFlags(&p.copied_out[b], cudaEventDisableTiming), "event");
+        }
+        p.ready = true;
+    }
+    hp = &p;
+    return MOGE_OK;
+}
+
 extern "C" {
 
 size_t moge_workspace_size(const moge_config *cfg) {
@@ -501,6 +533,56 @@ int moge_layer_forward_host(const moge_config *cfg, const void *x_host, const vo
                             s_down, nullptr, y_dev, workspace, stream);
     if (rc) return rc;
     MOGE_CU(cudaMemcpyAsync(y_host, y_dev, bytes, cudaMemcpyDeviceToHost, st), "copy y out");
+    MOGE_CU(cudaStreamSynchronize(st), "cudaStreamSynchronize");
+    return MOGE_OK;
+}
+
+int moge_layer_forward_host_stream(const moge_config *cfg, int64_t n_batches, const void *x_host,
+                                   const void *w_router, const float *logit_bias,
+                                   const void *w_gate, const void *w_up, const void *w_down,
+                                   const void *s_gate, const void *s_up, const void *s_down,
+                                   void *y_host, void *x_dev2, void *y_dev2, void *workspace,
+                                   void *stream) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    const moge_config c = *cfg;
+    if (n_batches < 0) return fail(MOGE_ERR_INVALID_ARG, "n_batches < 0");
+    if (c.T == 0 || n_batches == 0) return MOGE_OK;
+    if (!x_host || !y_host) return fail(MOGE_ERR_INVALID_ARG, "host buffer is NULL");
+    MOGE_NEED(x_dev2, "x_dev2");
+    MOGE_NEED(y_dev2, "y_dev2");
+    HostPipe *hp = nullptr;
+    if ((rc = host_pipe(hp))) return rc;
+    cudaStream_t st = (cudaStream_t)stream;
+    const size_t bytes = (size_t)c.T * c.d * (c.dtype == MOGE_BF16 ? 2 : 4);
+    const char *xh = static_cast<const char *>(x_host);
+    char *yh = static_cast<char *>(y_host);
+    char *xd = static_cast<char *>(x_dev2), *yd = static_cast<char *>(y_dev2);
+    // everything queued on `stream` before this call comes first
+    MOGE_CU(cudaEventRecord(hp->computed[1], st), "event");
+    MOGE_CU(cudaStreamWaitEvent(hp->in, hp->computed[1], 0), "wait");
+    MOGE_CU(cudaStreamWaitEvent(hp->out, hp->computed[1], 0), "wait");
+    for (int64_t i = 0; i < n_batches; ++i) {
+        const int b = (int)(i & 1);
+        // x buffer b: its previous batch (i - 2) has been read by its compute
+        if (i >= 2) MOGE_CU(cudaStreamWaitEvent(hp->in, hp->computed[b], 0), "wait");
+        MOGE_CU(cudaMemcpyAsync(xd + b * bytes, xh + i * bytes, bytes, cudaMemcpyHostToDevice,
+                                hp->in), "copy x in");
+        MOGE_CU(cudaEventRecord(hp->copied_in[b], hp->in), "event");
+        // y buffer b: its previous batch has been copied out
+        MOGE_CU(cudaStreamWaitEvent(st, hp->copied_in[b], 0), "wait");
+        if (i >= 2) MOGE_CU(cudaStreamWaitEvent(st, hp->copied_out[b], 0), "wait");
+        rc = moge_layer_forward(cfg, xd + b * bytes, w_router, logit_bias, w_gate, w_up, w_down,
+                                s_gate, s_up, s_down, nullptr, yd + b * bytes, workspace, stream);
+        if (rc) return rc;
+        MOGE_CU(cudaEventRecord(hp->computed[b], st), "event");
+        MOGE_CU(cudaStreamWaitEvent(hp->out, hp->computed[b], 0), "wait");
+        MOGE_CU(cudaMemcpyAsync(yh + i * bytes, yd + b * bytes, bytes, cudaMemcpyDeviceToHost,
+                                hp->out), "copy y out");
+        MOGE_CU(cudaEventRecord(hp->copied_out[b], hp->out), "event");
+    }
+    MOGE_CU(cudaStreamSynchronize(hp->out), "cudaStreamSynchronize");
+    MOGE_CU(cudaStreamSynchronize(hp->in), "cudaStreamSynchronize");
     MOGE_CU(cudaStreamSynchronize(st), "cudaStreamSynchronize");
     return MOGE_OK;
 }

@@ -75,6 +75,7 @@ struct GShared {
     uint32_t tmem_base;
     int abort;
     int total;
+    int epi_ok;  // the epilogue leader's wait result, shared with the other epilogue threads
     int start[kGMaxEntries + 1];  // token kinds: prefix sum of items per entry
 };
 
@@ -561,7 +562,13 @@ __global__ void __launch_bounds__(kGThreads, 1) bwd_gemm_kernel(const __grid_con
             GItem it;
             g_decode(p, sh, q, it);
             const int acc = i & 1;
-            if (!mbar_wait(&sh.tfull[acc], (uint32_t)(i >> 1) & 1u, abort)) break;
+            // one thread waits and all 128 act on its result (the row epilogues meet
+            // at named barriers, so they must all take or all skip an item)
+            if (et == 0) sh.epi_ok = mbar_wait(&sh.tfull[acc], (uint32_t)(i >> 1) & 1u, abort) ? 1 : 0;
+            named_bar_sync(1, 128);
+            const int ok_item = *(volatile int *)&sh.epi_ok;
+            named_bar_sync(1, 128);
+            if (!ok_item) break;
             tc_fence_after();
             const uint32_t tbase = tmem_base + ((uint32_t)(32 * q4) << 16) + (uint32_t)acc * 256u;
             const bool zero = it.nck == 0;
