@@ -349,6 +349,54 @@ def measure_train(cfg, inp, steps, warmup, alpha=0.01):
     return out
 
 
+def measure_stack(cfg, steps, warmup):
+    """Device-timed steps of the layer stack: for each of cfg.layers layers
+    (independent weights), u = RMSNorm(x), x = x + layer(u). Weights are drawn
+    on the device (seeded normal, std cfg.w_std): only timing depends on them;
+    the stack's numerics are checked against the oracle by the tests."""
+    import torch
+    import mixture_grouped_experts_b200 as mg
+    s = mg.shape_of(cfg)
+    g = torch.Generator(device="cuda").manual_seed(cfg.seed)
+
+    def rnd(*shape, std=cfg.w_std):
+        return (torch.randn(shape, generator=g, device="cuda") * std).to(torch.bfloat16)
+
+    E, I, d = cfg.N, cfg.I, cfg.d
+    layers = []
+    for _ in range(cfg.layers):
+        layers.append({"w_router": rnd(E, d), "logit_bias": None, "w_gate": rnd(E, I, d),
+                       "w_up": rnd(E, I, d), "w_down": rnd(E, d, I), "s_gate": rnd(cfg.S, I, d),
+                       "s_up": rnd(cfg.S, I, d), "s_down": rnd(cfg.S, d, I)})
+    x0 = rnd(cfg.T, d, std=cfg.x_std)
+    xa, xb, u = torch.empty_like(x0), torch.empty_like(x0), torch.empty_like(x0)
+    ws = mg.alloc_workspace(s)
+
+    def step():
+        cur, nxt = xa, xb
+        cur.copy_(x0)
+        for w in layers:
+            mg.moge_rmsnorm(s, cur, 1e-6, u)
+            mg.moge_layer_forward(s, u, w, ws, residual=cur, y=nxt)
+            cur, nxt = nxt, cur
+
+    for _ in range(max(warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    mg.check_device_errors()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(steps):
+        step()
+    end.record()
+    torch.cuda.synchronize()
+    mg.check_device_errors()
+    ms = start.elapsed_time(end) / steps
+    del layers, ws
+    torch.cuda.empty_cache()
+    return ms
+
+
 def max_over_ranks(v, dist_on):
     """Max of a per-rank scalar over all ranks (identity on one process).
     Uses a CUDA tensor under NCCL and a CPU tensor under gloo."""
@@ -465,6 +513,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--no-fp8", action="store_true", help="skip the 8-bit-weight side measurement")
     ap.add_argument("--no-train", action="store_true", help="skip the training-step side measurement")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the skewed-router and 12-layer-stack side measurements")
     ap.add_argument("--ref-tokens", type=int, default=2, help="tokens per step of --impl reference")
     ap.add_argument("--ep", action="store_true",
                     help="expert parallelism over the ranks instead of independent replicas")
@@ -601,6 +651,40 @@ def main():
                          "flops_per_step": train_flops(tcfg),
                          "peak_source": "%s bf16_tflops_sustained" % peak_kind},
             "backward_tflops": bwd_tf, "clocks": tclk}
+    if rank == 0 and n == 1 and not args.no_extra and args.config == "decode":
+        kcfg = synth.CONFIGS["skew"]
+        kinp = synth.layer_inputs(kcfg)
+        ks = ClockSampler(local)
+        ks.start()
+        km = measure(kcfg, kinp, 5, args.warmup, False, with_e2e=False)
+        kclk = ks.stop()
+        del kinp
+        tfs = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+        k_tf = layer_flops(kcfg) / (km["ms"] / 1e3) / 1e12
+        cnt = km["counts"]
+        line["skew"] = {
+            "workload": workload_config(kcfg)["workload"],
+            "value": kcfg.T / (km["ms"] / 1e3), "unit": "tokens/s", "ms_per_step": km["ms"],
+            "roofline": {"bound": "tensor", "achieved": k_tf, "peak": tfs, "unit": "TFLOP/s",
+                         "frac": k_tf / tfs, "peak_source": "%s bf16_tflops_sustained" % peak_kind},
+            "expert_rows": {"max": int(cnt.max()), "min": int(cnt.min())},
+            "group_rows": [int(cnt[g * (kcfg.N // kcfg.M):(g + 1) * (kcfg.N // kcfg.M)].sum())
+                           for g in range(kcfg.M)],
+            "stage_ms": km["stage_ms"], "clocks": kclk}
+        scfg = synth.CONFIGS["stack12"]
+        ss = ClockSampler(local)
+        ss.start()
+        sms = measure_stack(scfg, 5, args.warmup)
+        sclk = ss.stop()
+        sb = scfg.layers * layer_bytes(scfg, scfg.N) / (sms / 1e3) / 1e9
+        line["stack12"] = {
+            "workload": "12-layer stack of MoGE FFN blocks with pre-RMSNorm (eps 1e-6) and "
+                        "residual, decode: T=456, d=5120, per layer 64 experts / 8 groups / K'=1, "
+                        "4 shared, I=1344, bf16, independent weights per layer (33.8 GB)",
+            "value": scfg.T / (sms / 1e3), "unit": "tokens/s", "ms_per_step": sms,
+            "roofline": {"bound": "hbm", "achieved": sb, "peak": hbm, "unit": "GB/s",
+                         "frac": sb / hbm, "algorithmic_bytes": scfg.layers * layer_bytes(scfg, scfg.N)},
+            "clocks": sclk}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist_on:
