@@ -178,7 +178,8 @@ __global__ void __launch_bounds__(kRowThreads) combine_kernel(
         src_s[K + b] = static_cast<const char *>(shared_rows) + ((size_t)b * T + t) * row_bytes;
     __syncthreads();
     const int nsrc = K + n_shared;
-    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+    // CTA (t, part): vectors part*blockDim.x .. of the row (one per thread)
+    for (int v = blockIdx.y * blockDim.x + threadIdx.x; v < nvec; v += gridDim.y * blockDim.x) {
         float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
         for (int k0 = 0; k0 < nsrc; k0 += 8) {
             Raw8 raw[8];
@@ -220,7 +221,13 @@ cudaError_t launch_combine(const moge_config &c, const void *y_perm, const float
                            int n_shared_blocks, const void *residual, void *y, cudaStream_t st,
                            bool out_f32) {
     auto kern = c.dtype == MOGE_BF16 ? combine_kernel<MOGE_BF16> : combine_kernel<MOGE_F32>;
-    return launch_pdl(kern, dim3(c.T), dim3(kRowThreads), 0, st, c.T, c.d, c.N, y_perm, topk_w,
+    // few tokens (decode): a token's row spread over several CTAs, down to one
+    // 8-element vector per thread, for about 2048 CTAs; many tokens: one CTA each
+    const int nvec = c.d / 8;
+    const int max_parts = (nvec + kRowThreads - 1) / kRowThreads;
+    const int want = (2048 + c.T - 1) / (c.T > 0 ? c.T : 1);
+    const int parts = want < max_parts ? (want > 1 ? want : 1) : max_parts;
+    return launch_pdl(kern, dim3(c.T, parts), dim3(kRowThreads), 0, st, c.T, c.d, c.N, y_perm, topk_w,
                       perm_dst, K, shared_rows, n_shared_blocks, residual, y, out_f32 ? 1 : 0);
 }
 
