@@ -74,7 +74,7 @@ Workspace carve_workspace(const moge_config &c, void *base) {
     w.plan.down = (ExpertWork *)take(E * sizeof(ExpertWork));
     w.plan.up_start = (int *)take((E + 1) * 4);
     w.plan.down_start = (int *)take((E + 1) * 4);
-    w.plan.sync = (int *)take((E + 1) * 4);
+    w.plan.sync = (int *)take((E + 2) * 4);
     w.x_perm = take(T * K * c.d * esz);
     w.h = take(T * (K + c.S) * c.I * esz);
     w.y_perm = take(T * (K + c.S) * c.d * esz);
@@ -174,6 +174,10 @@ static int run_ffn(const moge_config &c, const Plan &plan, int n_entries, const 
 // combine) after the entry point validated its arguments. `op` carries the
 // expert weight pointers (and, for fp8, their row scales); the activation
 // pointers are filled in here.
+// Largest T*K whose permute runs inside the grouped GEMM launch (measured:
+// saves ~6 us at T = 456, costs ~30 us at T = 4096).
+constexpr long long kFusedPermuteRows = 8192;
+
 static int layer_run(const moge_config &c, const void *x, const void *w_router,
                      const float *logit_bias, FfnOperands op, bool fp8, const void *residual,
                      void *y, void *workspace, cudaStream_t st) {
@@ -187,8 +191,19 @@ static int layer_run(const moge_config &c, const void *x, const void *w_router,
     MOGE_CU(launch_scan(c, ws.hist, ws.base, ws.counts, ws.offsets, &ws.plan, true, c.S > 0, st),
             "scan launch");
     if (ev) MOGE_CU(cudaEventRecord(ev[2], st), "event");
-    MOGE_CU(launch_scatter_rows(c, x, ws.topk_idx, ws.rank, ws.base, ws.offsets, ws.perm_src,
-                                ws.perm_dst, ws.x_perm, st), "permute launch");
+    // bf16 decode-sized batches: the grouped GEMM launch does the permute itself
+    // (its epilogue warps copy the rows while the first, shared-expert items
+    // run); larger batches (the copy would hold the epilogue warps long enough to
+    // stall the first items), fp8 and fp32: a launch of its own
+    const bool fuse_permute = c.dtype == MOGE_BF16 && !fp8 &&
+                              (long long)c.T * c.M * c.Kp <= kFusedPermuteRows;
+    if (fuse_permute) {
+        op.pm_topk_idx = ws.topk_idx; op.pm_rank = ws.rank; op.pm_base = ws.base;
+        op.pm_offsets = ws.offsets; op.pm_perm_src = ws.perm_src; op.pm_perm_dst = ws.perm_dst;
+    } else {
+        MOGE_CU(launch_scatter_rows(c, x, ws.topk_idx, ws.rank, ws.base, ws.offsets, ws.perm_src,
+                                    ws.perm_dst, ws.x_perm, st), "permute launch");
+    }
     if (ev) MOGE_CU(cudaEventRecord(ev[3], st), "event");
     const int64_t rrows = (int64_t)c.T * K;
     op.b0 = ws.x_perm;

@@ -68,6 +68,12 @@ struct TcParams {
     uint16_t *y;         // [rows][d]
     int *sync;           // [0] queue counter, [1 + e] finished up items of entry e
     uint16_t *gu;        // null, or [rows][2I]: the up-projection's g and u (training forward)
+    // permute inside this launch (pm_topk_idx non-null): x (b1) -> x_perm (b0)
+    const int32_t *pm_topk_idx, *pm_rank, *pm_base, *pm_offsets;
+    int32_t *pm_perm_src, *pm_perm_dst;
+    const uint4 *pm_x;
+    uint4 *pm_x_perm;
+    int pm_T, pm_N, pm_K;
 };
 
 struct TcItem {
@@ -120,6 +126,7 @@ struct TcShared {
     uint32_t tmem_base;
     int abort;
     int epi_item;
+    int pm_rows[kMaxExperts];  // the fused permute: destination rows of the current token
 };
 
 // smem byte offsets of chunk c of a stage
@@ -227,6 +234,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
         uint32_t phase = 0;
         uint32_t armed = 0, armed_par = 0;  // lane 0: per stage, a load issued / its parity
         int next = lane == 0 ? atomicAdd(p.sync, 1) : 0;
+        bool permuted = p.pm_topk_idx == nullptr;  // x_perm complete (fused permute)
         for (int s = 0;; ++s) {
             const int slot = s % kSlots;
             int q = 0;
@@ -249,6 +257,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
                 if (lane == 0) ok = wait_counter(p.sync + 1 + it.entry, it.w.ntb * fb_up, abort);
                 if (!__shfl_sync(0xffffffffu, ok, 0)) break;
                 fence_proxy_async_global();
+            } else if (it.w.b_sel == 0 && !permuted) {  // routed rows: every CTA's permute share
+                int ok = 1;
+                if (lane == 0) ok = wait_counter(p.sync + 1 + p.n_entries, (int)gridDim.x, abort);
+                if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+                fence_proxy_async_global();
+                permuted = true;
             }
             const CUtensorMap *ma0, *ma1, *mb;
             if (it.up) {
@@ -357,6 +371,43 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
         // ------------------------------------------------------ epilogue
         const int q4 = warp & 3;           // TMEM lane quarter this warp may read
         const int et = threadIdx.x - 64;   // 0 .. 127
+        if (p.pm_topk_idx) {
+            // The permute, before this CTA's first accumulator exists: tokens
+            // blockIdx.x, + gridDim.x, ...; each token's K destination rows
+            // (expert offset + earlier tiles' rows + rank in its tile), then its
+            // row copied into each. Published with a release for the routed
+            // up-projection items, which read x_perm with TMA (async proxy).
+            const int K = p.pm_K, nvec = p.d / 8;
+            for (int t = blockIdx.x; t < p.pm_T; t += gridDim.x) {
+                for (int k = et; k < K; k += 128) {
+                    const size_t i = (size_t)t * K + k;
+                    const int e = p.pm_topk_idx[i];
+                    int row = -1;
+                    if (e >= 0 && e < p.pm_N) {
+                        row = p.pm_offsets[e] + p.pm_base[(size_t)(t / kRouterTile) * p.pm_N + e] +
+                              p.pm_rank[i];
+                        p.pm_perm_dst[i] = row;
+                        p.pm_perm_src[row] = t;
+                    } else {
+                        raise_error(ERRBIT_INVARIANT);
+                    }
+                    sh.pm_rows[k] = row;
+                }
+                named_bar_sync(1, 128);
+                for (int v = et; v < nvec; v += 128) {
+                    const uint4 val = p.pm_x[(size_t)t * nvec + v];
+                    for (int k = 0; k < K; ++k) {
+                        const int row = sh.pm_rows[k];
+                        if (row >= 0) p.pm_x_perm[(size_t)row * nvec + v] = val;
+                    }
+                }
+                named_bar_sync(1, 128);
+            }
+            fence_proxy_async_global();
+            __threadfence();
+            named_bar_sync(1, 128);
+            if (et == 0) atomicAdd(p.sync + 1 + p.n_entries, 1);
+        }
         for (int s = 0;; ++s) {
             // the leader takes the next item and waits for its accumulator;
             // all 128 threads then act on the same decision
@@ -551,6 +602,17 @@ cudaError_t launch_ffn_tc(const moge_config &c, const Plan &plan, int n_entries,
     p.y = (uint16_t *)op.y;
     p.sync = plan.sync;
     p.gu = (uint16_t *)op.gu;
+    p.pm_topk_idx = op.pm_topk_idx;
+    p.pm_rank = op.pm_rank;
+    p.pm_base = op.pm_base;
+    p.pm_offsets = op.pm_offsets;
+    p.pm_perm_src = op.pm_perm_src;
+    p.pm_perm_dst = op.pm_perm_dst;
+    p.pm_x = (const uint4 *)op.b1;
+    p.pm_x_perm = (uint4 *)op.b0;
+    p.pm_T = c.T;
+    p.pm_N = c.N;
+    p.pm_K = c.M * c.Kp;
 
     const size_t smem = tc_smem_bytes();
     cudaError_t e = cudaFuncSetAttribute(ffn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -43,8 +43,10 @@ struct Plan {
     ExpertWork *down;   // [n_entries]
     int *up_start;      // [n_entries + 1] prefix sum of items (ntb * feature blocks)
     int *down_start;    // [n_entries + 1]
-    int *sync;          // [n_entries + 1] work-queue counter and per-entry finished
-                        // up-projection items; zeroed by the kernel that writes the plan
+    int *sync;          // [n_entries + 2] work-queue counter, per-entry finished
+                        // up-projection items, and the CTAs done with a permute done
+                        // inside the grouped GEMM ([n_entries + 1]); zeroed by the
+                        // kernel that writes the plan
 };
 
 // Workspace carve-up (all regions 256-byte aligned).
@@ -128,6 +130,12 @@ struct FfnOperands {
     // Optional (bf16 tensor-core FFN only, training forward): the
     // up-projection's pre-activations, [h_rows][2I] = [g | u] per row.
     void *gu;
+    // Optional (bf16 tensor-core FFN only): the permute done inside the grouped
+    // GEMM launch -- x_perm (b0) is written from x (b1) by the kernel's epilogue
+    // warps before their first item, with the indices below (as the scatter
+    // kernel computes them); the routed up-projection items wait for it.
+    const int32_t *pm_topk_idx, *pm_rank, *pm_base, *pm_offsets;
+    int32_t *pm_perm_src, *pm_perm_dst;
     // FP8 weights only (launch_ffn_fp8): the w*/s* pointers above are E4M3
     // codes and these their per-row fp32 scales ([E][I], [E][I], [E][d])
     const float *wg_s, *wu_s, *wd_s;

@@ -554,7 +554,7 @@ __device__ void build_plan_block(const moge_config &c, const int32_t *offs, Plan
     const int i = threadIdx.x;
     ExpertWork u = {}, dn = {};
     int items_up = 0, items_down = 0;
-    if (i <= n) plan.sync[i] = 0;
+    if (i <= n + 1) plan.sync[i] = 0;
     if (i < n) {
         int rows, a_sel, a_idx, up_src, up_bsel, mid;
         if (i >= ns) {
