@@ -140,3 +140,15 @@ def test_expert_parallel_entry_points_validate_on_host(L):
     assert L.moge_layer_forward_ep_local(ctypes.byref(c), 0, 2, *args) == mg.ERR_INVALID_ARG  # y_part NULL
     assert L.moge_ep_finish(ctypes.byref(c), -1, None, None, None, None) == mg.ERR_INVALID_ARG
     assert L.moge_ep_finish(ctypes.byref(c), 4, 0x1008, None, 0x1000, None) == mg.ERR_UNSUPPORTED
+
+
+def test_streaming_host_call_validates_on_host(L):
+    c = mg.moge_config(64, 256, 16, 4, 1, 1, 128, mg.MOGE_BF16)
+    args = [None] * 14
+    assert L.moge_layer_forward_host_stream(ctypes.byref(c), -1, *args) == mg.ERR_INVALID_ARG
+    assert L.moge_layer_forward_host_stream(ctypes.byref(c), 0, *args) == mg.OK  # nothing to do
+    assert L.moge_layer_forward_host_stream(ctypes.byref(c), 2, *args) == mg.ERR_INVALID_ARG  # host NULL
+    # x_host, w_router, bias, w_gate, w_up, w_down, s_gate, s_up, s_down, y_host,
+    # x_dev2 (misaligned), y_dev2, workspace, stream
+    bad = [0x1000] + [None] * 8 + [0x2000, 0x3008, 0x4000, None, None]
+    assert L.moge_layer_forward_host_stream(ctypes.byref(c), 2, *bad) == mg.ERR_UNSUPPORTED
