@@ -147,6 +147,12 @@ cudaError_t launch_ffn_tc(const moge_config &c, const Plan &plan, int n_entries,
                           const FfnOperands &op, int num_sms, cudaStream_t st, cudaEvent_t mid);
 cudaError_t launch_ffn_f32(const moge_config &c, const Plan &plan, int n_entries,
                            const FfnOperands &op, cudaStream_t st, cudaEvent_t mid);
+namespace pair {
+// The same grouped FFN on CTA pairs (2-SM tcgen05 MMA, M = 256): bf16, no
+// saved g/u and no permute inside the launch; used for prefill-sized batches.
+cudaError_t launch_ffn_tc_pair(const moge_config &c, const Plan &plan, int n_entries,
+                               const FfnOperands &op, int num_sms, cudaStream_t st);
+}  // namespace pair
 // grouped FFN with FP8 (E4M3, per-row scale) weights and bf16 activations
 cudaError_t launch_ffn_fp8(const moge_config &c, const Plan &plan, int n_entries,
                            const FfnOperands &op, int num_sms, cudaStream_t st);

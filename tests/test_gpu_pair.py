@@ -1,0 +1,56 @@
+"""GPU parity of layers with at least 16384 routed rows (T * M * K'), whose
+grouped FFN runs on CTA pairs (2-SM tensor-core MMA, 256 weight rows per
+item): feature and output tiles split between the two CTAs with ragged ends
+(I and d not multiples of 128 / 256), experts of every size from streaming
+tiles (<= 64 rows) to several 256-row token tiles, and a hot expert."""
+import numpy as np
+import pytest
+import torch
+
+import mixture_grouped_experts_b200 as mg
+import synth
+from gpu_helpers import layer_parity
+
+pytestmark = pytest.mark.gpu
+
+PAIR_ROWS = 16384  # smallest T * M * K' that takes the pair kernel
+
+BASE = synth.Config("pair", T=2048, d=512, N=64, M=8, Kp=1, S=2, I=384, dtype="bf16", seed=91,
+                    w_std=0.05)
+CASES = {
+    # I = 384: three feature pairs, the last one half empty; d = 512: two output pairs
+    "even": (BASE, None),
+    # d = 520, I = 328: a last output pair of 8 rows, a last feature tile of 8
+    "odd": (BASE.replace(name="pair_odd", d=520, I=328, N=32, M=4, Kp=2, seed=92), 700),
+    # 256 experts of ~64 rows: streaming and tensor tiles side by side
+    "n256": (BASE.replace(name="pair_n256", N=256, S=1, seed=93), 700),
+    # no shared expert, 2 picks in each of 2 groups, > 1000 rows per expert
+    "s0": (BASE.replace(name="pair_s0", T=4096, N=16, M=2, Kp=2, S=0, seed=94), 600),
+}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    mg.lib()
+    yield
+    torch.cuda.synchronize()
+    mg.check_device_errors()
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_pair_layer(name):
+    cfg, n_sample = CASES[name]
+    assert cfg.T * cfg.M * cfg.Kp >= PAIR_ROWS
+    layer_parity(cfg, synth.layer_inputs(cfg), n_sample=n_sample)
+
+
+def test_pair_layer_hot_expert():
+    """A router bias sends most tokens of every group to its first expert:
+    those experts hold ~1500 rows (six 256-row token tiles), the rest few."""
+    cfg = BASE.replace(name="pair_hot", seed=95)
+    inp = synth.layer_inputs(cfg)
+    bias = np.zeros(cfg.N, dtype=np.float32)
+    bias[:: cfg.N // cfg.M] = 1.5
+    inp["logit_bias"] = bias
+    layer_parity(cfg, inp, n_sample=600)
