@@ -34,6 +34,13 @@ import synth  # noqa: E402
 
 METRIC = "MoGE layer tokens/s; % of HBM roofline (decode) / bf16 TC peak (prefill)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# The grouped FFN kernel a layer runs: the single-SM kernel below PAIR_ROWS
+# routed rows (T * M * K'), the CTA-pair kernel from there on.
+PAIR_ROWS = 16384
+FFN_KERNEL = ("ffn_tc_kernel (grouped gate+up GEMM with SwiGLU epilogue and down GEMM, one "
+              "persistent launch)")
+FFN_PAIR_KERNEL = ("ffn_tc_pair_kernel (the same grouped FFN on CTA pairs, 2-SM tcgen05 MMA, "
+                   "one persistent launch)")
 
 
 def load_peaks():
@@ -557,13 +564,20 @@ def main():
     hbm = peaks["hbm_gbs"]
     fb = ffn_bytes(cfg, m["n_used"])
     ach = fb / (su["ffn"] / 1e3) / 1e9
-    roofline = {"bound": "hbm",
-                "kernel": "ffn_tc_kernel (grouped gate+up GEMM with SwiGLU epilogue and down GEMM, one persistent launch)",
-                "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
-                "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
-                else "fallback 6650 GB/s", "traffic": None,
-                "algorithmic_bytes_per_launch": fb,
-                "kernel_ms": su["ffn"]}
+    if cfg.T * cfg.M * cfg.Kp < PAIR_ROWS:
+        roofline = {"bound": "hbm", "kernel": FFN_KERNEL,
+                    "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                    "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                    else "fallback 6650 GB/s", "traffic": None,
+                    "algorithmic_bytes_per_launch": fb,
+                    "kernel_ms": su["ffn"]}
+    else:  # prefill-sized batches: the contraction bounds the pair kernel
+        tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        ftf = ffn_flops(cfg) / (su["ffn"] / 1e3) / 1e12
+        roofline = {"bound": "tensor", "kernel": FFN_PAIR_KERNEL, "achieved": ftf, "peak": tf,
+                    "unit": "TFLOP/s", "frac": ftf / tf,
+                    "peak_source": "%s bf16_tflops (burst)" % peak_kind, "traffic": None,
+                    "algorithmic_flops_per_launch": ffn_flops(cfg), "kernel_ms": su["ffn"]}
     lb = layer_bytes(cfg, m["n_used"])
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": n, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -601,7 +615,7 @@ def main():
         line["prefill"] = {
             "workload": workload_config(pcfg)["workload"],
             "value": pcfg.T / (pm["ms"] / 1e3), "unit": "tokens/s", "ms_per_step": pm["ms"],
-            "roofline": {"bound": "tensor", "kernel": "ffn_tc_kernel", "achieved": ffn_tf,
+            "roofline": {"bound": "tensor", "kernel": FFN_PAIR_KERNEL, "achieved": ffn_tf,
                          "peak": tf, "unit": "TFLOP/s", "frac": ffn_tf / tf,
                          "peak_source": "%s bf16_tflops (burst)" % peak_kind},
             "layer_tflops": lay_tf, "layer_frac_sustained": lay_tf / tfs,
