@@ -177,10 +177,11 @@ static int run_ffn(const moge_config &c, const Plan &plan, int n_entries, const 
 // Largest T*K whose permute runs inside the grouped GEMM launch (measured:
 // saves ~6 us at T = 456, costs ~30 us at T = 4096).
 constexpr long long kFusedPermuteRows = 8192;
-// Smallest T*K whose grouped FFN runs on CTA pairs (2-SM MMA): the pair
-// halves the shared-memory bytes per MMA flop, which is what bounds the 1-SM
-// kernel on large token tiles; small batches keep the 1-SM kernel, whose
-// finer items balance better.
+// Smallest T*K whose grouped FFN runs on CTA pairs (2-SM MMA): each CTA of a
+// pair stages half of the token rows, a third fewer shared-memory bytes per
+// MMA flop, and shared-memory bandwidth and the copies' latency are what bound
+// the 1-SM kernel on large token tiles; small batches keep the 1-SM kernel,
+// whose finer items balance better.
 constexpr long long kPairRows = 16384;
 
 static int layer_run(const moge_config &c, const void *x, const void *w_router,
@@ -221,7 +222,7 @@ static int layer_run(const moge_config &c, const void *x, const void *w_router,
     if (fp8) {
         MOGE_CU(launch_ffn_fp8(c, ws.plan, c.N + c.S, op, num_sms(), st), "grouped FFN (fp8) launch");
     } else {
-        if (c.dtype == MOGE_BF16 && !fuse_permute && !op.gu && rrows >= kPairRows) {
+        if (c.dtype == MOGE_BF16 && !fuse_permute && rrows >= kPairRows) {
             MOGE_CU(pair::launch_ffn_tc_pair(c, ws.plan, c.N + c.S, op, num_sms(), st),
                     "grouped FFN (tcgen05 pairs) launch");
         } else {

@@ -5,8 +5,9 @@
 // down-projection (y rows out). CTAs work in pairs (clusters of 2) on the
 // 2-SM tensor-core MMA (tcgen05.mma.cta_group::2, M = 256): each item is two
 // weight tiles of 128 rows (one per CTA) against one token tile of N rows
-// (each CTA stages N/2 of them), so every byte staged in shared memory feeds
-// twice the MMA work of a single-SM tile. Warp roles in each CTA:
+// (each CTA stages N/2 of them): per CTA, 32 KB staged per 64-wide K-chunk of
+// 128 x 256 MMA work, where a single-SM tile stages 48 KB. The up-projection
+// can also keep g and u (bf16) for the backward pass. Warp roles in each CTA:
 //   warp 0    TMA producer; in the leader CTA also the scheduler, which takes
 //             work items from a global queue (an atomic counter) and publishes
 //             them to both CTAs through small shared-memory rings
@@ -49,7 +50,7 @@ namespace pair {
 
 constexpr int kStages = 6;
 constexpr int kStageBytes = 32 * 1024;  // one K-chunk: 16 KB of weights, <= 16 KB of token rows
-constexpr int kEpiBytes = 12 * 1024;
+constexpr int kEpiBytes = 16 * 1024;  // U fp32 [32][64], H and G bf16 [32][64]
 constexpr int kTcThreads = 192;
 constexpr int kChunkK = 64;          // bf16 elements per K-chunk (128 bytes, one swizzle row)
 constexpr int kBoxRows = 64;         // token rows per TMA box (one 8 KB copy per chunk)
@@ -73,6 +74,7 @@ struct TcParams {
     int I, d;
     uint16_t *h;         // [rows][I]
     uint16_t *y;         // [rows][d]
+    uint16_t *gu;        // [rows][2][I] g and u kept for the backward pass, or null
     int *sync;           // [0] queue counter, [1 + e] finished up-projection halves of entry e
 };
 
@@ -458,6 +460,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_pair_kernel(
                     // lanes 0-63 hold gate and 64-127 up, or the reverse for an up-first tile
                     const bool gate_hi = p.gu_mode[it.w.a_sel] == kUpGateFused;
                     const bool is_gate = (q4 < 2) != gate_hi;
+                    uint16_t *G = reinterpret_cast<uint16_t *>(epi + 12288);  // [32 cols][64 features]
                     const int f = (q4 & 1) * 32 + lane;
                     if (!is_gate) {
 #pragma unroll
@@ -470,15 +473,26 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_pair_kernel(
                             const float g = __uint_as_float(v[j]);
                             const float hv = g / (1.0f + expf(-g)) * U[j * 64 + f];
                             H[j * 64 + f] = to_bf16_bits(hv);
+                            if (p.gu) G[j * 64 + f] = to_bf16_bits(g);
                         }
                     }
                     named_bar_sync(1, 128);
                     for (int idx = et; idx < 32 * 8; idx += 128) {
                         const int r = idx >> 3, vv = idx & 7;
                         const int col = c0 + r, feat = tile * 64 + vv * 8;
-                        if (col < it.n_valid && feat < p.I)
+                        if (col < it.n_valid && feat < p.I) {
                             *reinterpret_cast<uint4 *>(p.h + (row0 + col) * p.I + feat) =
                                 *reinterpret_cast<const uint4 *>(H + r * 64 + vv * 8);
+                            if (p.gu) {  // keep g and u (bf16) for the backward pass
+                                uint16_t *dst = p.gu + (row0 + col) * 2 * (size_t)p.I + feat;
+                                *reinterpret_cast<uint4 *>(dst) =
+                                    *reinterpret_cast<const uint4 *>(G + r * 64 + vv * 8);
+                                const float *u8 = U + r * 64 + vv * 8;
+                                *reinterpret_cast<uint4 *>(dst + p.I) =
+                                    make_uint4(pack_bf16x2(u8[0], u8[1]), pack_bf16x2(u8[2], u8[3]),
+                                               pack_bf16x2(u8[4], u8[5]), pack_bf16x2(u8[6], u8[7]));
+                            }
+                        }
                     }
                     named_bar_sync(1, 128);
                 } else {
@@ -643,6 +657,7 @@ cudaError_t launch_ffn_tc_pair(const moge_config &c, const Plan &plan, int n_ent
     p.d = d;
     p.h = (uint16_t *)op.h;
     p.y = (uint16_t *)op.y;
+    p.gu = (uint16_t *)op.gu;
     p.sync = plan.sync;
 
     const size_t smem = tc_smem_bytes();

@@ -149,7 +149,8 @@ cudaError_t launch_ffn_f32(const moge_config &c, const Plan &plan, int n_entries
                            const FfnOperands &op, cudaStream_t st, cudaEvent_t mid);
 namespace pair {
 // The same grouped FFN on CTA pairs (2-SM tcgen05 MMA, M = 256): bf16, no
-// saved g/u and no permute inside the launch; used for prefill-sized batches.
+// permute inside the launch (g/u kept when op.gu is set); used for
+// prefill-sized batches.
 cudaError_t launch_ffn_tc_pair(const moge_config &c, const Plan &plan, int n_entries,
                                const FfnOperands &op, int num_sms, cudaStream_t st);
 }  // namespace pair

@@ -75,6 +75,10 @@ CASES = {
     # no shared experts, 64 experts in 8 groups, experts of > 256 rows (two token tiles)
     "n64": synth.Config("bw_n64", T=600, d=256, N=64, M=8, Kp=1, S=0, I=128, dtype="bf16",
                         seed=63, w_std=0.05),
+    # 16384 routed rows: the training forward runs the grouped FFN on CTA pairs
+    # (g and u kept by that kernel); I = 192: a half-empty last feature pair
+    "pair": synth.Config("bw_pair", T=2048, d=256, N=64, M=8, Kp=1, S=1, I=192, dtype="bf16",
+                         seed=65, w_std=0.05),
 }
 
 
