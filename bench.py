@@ -36,7 +36,7 @@ METRIC = "MoGE layer tokens/s; % of HBM roofline (decode) / bf16 TC peak (prefil
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # The grouped FFN kernel a layer runs: the single-SM kernel below PAIR_ROWS
 # routed rows (T * M * K'), the CTA-pair kernel from there on.
-PAIR_ROWS = 16384
+PAIR_ROWS = 8193
 FFN_KERNEL = ("ffn_tc_kernel (grouped gate+up GEMM with SwiGLU epilogue and down GEMM, one "
               "persistent launch)")
 FFN_PAIR_KERNEL = ("ffn_tc_pair_kernel (the same grouped FFN on CTA pairs, 2-SM tcgen05 MMA, "

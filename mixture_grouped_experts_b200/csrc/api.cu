@@ -180,9 +180,11 @@ constexpr long long kFusedPermuteRows = 8192;
 // Smallest T*K whose grouped FFN runs on CTA pairs (2-SM MMA): each CTA of a
 // pair stages half of the token rows, a third fewer shared-memory bytes per
 // MMA flop, and shared-memory bandwidth and the copies' latency are what bound
-// the 1-SM kernel on large token tiles; small batches keep the 1-SM kernel,
-// whose finer items balance better.
-constexpr long long kPairRows = 16384;
+// the 1-SM kernel on large token tiles. Every batch too large for the permute
+// inside the launch takes the pair (measured faster from T*K = 8800 on: 0.78
+// vs 0.83 ms at T = 1100 of the prefill layer); decode-sized ones keep the
+// 1-SM kernel and its fused permute.
+constexpr long long kPairRows = kFusedPermuteRows + 1;
 
 static int layer_run(const moge_config &c, const void *x, const void *w_router,
                      const float *logit_bias, FfnOperands op, bool fp8, const void *residual,

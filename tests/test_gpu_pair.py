@@ -1,4 +1,4 @@
-"""GPU parity of layers with at least 16384 routed rows (T * M * K'), whose
+"""GPU parity of layers with more than 8192 routed rows (T * M * K'), whose
 grouped FFN runs on CTA pairs (2-SM tensor-core MMA, 256 weight rows per
 item): feature and output tiles split between the two CTAs with ragged ends
 (I and d not multiples of 128 / 256), experts of every size from streaming
@@ -13,11 +13,13 @@ from gpu_helpers import layer_parity
 
 pytestmark = pytest.mark.gpu
 
-PAIR_ROWS = 16384  # smallest T * M * K' that takes the pair kernel
+PAIR_ROWS = 8193  # smallest T * M * K' that takes the pair kernel
 
 BASE = synth.Config("pair", T=2048, d=512, N=64, M=8, Kp=1, S=2, I=384, dtype="bf16", seed=91,
                     w_std=0.05)
 CASES = {
+    # 9000 routed rows: just past the decode-sized kernel's limit
+    "t1125": (BASE.replace(name="pair_t1125", T=1125, seed=96), None),
     # I = 384: three feature pairs, the last one half empty; d = 512: two output pairs
     "even": (BASE, None),
     # d = 520, I = 328: a last output pair of 8 rows, a last feature tile of 8
