@@ -39,6 +39,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 PAIR_ROWS = 8193
 FFN_KERNEL = ("ffn_tc_kernel (grouped gate+up GEMM with SwiGLU epilogue and down GEMM, one "
               "persistent launch)")
+# DRAM bytes of one decode-workload launch of ffn_tc_kernel as it stands, from
+# one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum, cold cache):
+# 2.868 GB read + 65.4 MB written.
+DECODE_FFN_TRAFFIC = 2867918848 + 65411072
 FFN_PAIR_KERNEL = ("ffn_tc_pair_kernel (the same grouped FFN on CTA pairs, 2-SM tcgen05 MMA, "
                    "one persistent launch)")
 
@@ -568,7 +572,8 @@ def main():
         roofline = {"bound": "hbm", "kernel": FFN_KERNEL,
                     "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
                     "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
-                    else "fallback 6650 GB/s", "traffic": None,
+                    else "fallback 6650 GB/s",
+                    "traffic": DECODE_FFN_TRAFFIC if args.config == "decode" else None,
                     "algorithmic_bytes_per_launch": fb,
                     "kernel_ms": su["ffn"]}
     else:  # prefill-sized batches: the contraction bounds the pair kernel
