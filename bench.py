@@ -39,6 +39,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 PAIR_ROWS = 8193
 FFN_KERNEL = ("ffn_tc_kernel (grouped gate+up GEMM with SwiGLU epilogue and down GEMM, one "
               "persistent launch)")
+# Nominal B200 figures, reported beside the measured denominators: HBM3e
+# ~8 TB/s and 2.25 PFLOP/s dense bf16.
+NOMINAL = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 # DRAM bytes of one decode-workload launch of ffn_tc_kernel as it stands, from
 # one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum, cold cache):
 # 2.868 GB read + 65.4 MB written.
@@ -574,6 +577,8 @@ def main():
                     "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
                     else "fallback 6650 GB/s",
                     "traffic": DECODE_FFN_TRAFFIC if args.config == "decode" else None,
+                    "nominal": {"peak": NOMINAL["hbm_gbs"], "unit": "GB/s",
+                                "frac": ach / NOMINAL["hbm_gbs"]},
                     "algorithmic_bytes_per_launch": fb,
                     "kernel_ms": su["ffn"]}
     else:  # prefill-sized batches: the contraction bounds the pair kernel
@@ -582,6 +587,8 @@ def main():
         roofline = {"bound": "tensor", "kernel": FFN_PAIR_KERNEL, "achieved": ftf, "peak": tf,
                     "unit": "TFLOP/s", "frac": ftf / tf,
                     "peak_source": "%s bf16_tflops (burst)" % peak_kind, "traffic": None,
+                    "nominal": {"peak": NOMINAL["bf16_tflops"], "unit": "TFLOP/s",
+                                "frac": ftf / NOMINAL["bf16_tflops"]},
                     "algorithmic_flops_per_launch": ffn_flops(cfg), "kernel_ms": su["ffn"]}
     lb = layer_bytes(cfg, m["n_used"])
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": n, "steps": args.steps,
@@ -591,6 +598,8 @@ def main():
             "roofline": roofline,
             "layer_roofline": {"bound": "hbm", "achieved": lb / (ms / 1e3) / 1e9, "peak": hbm,
                                "unit": "GB/s", "frac": lb / (ms / 1e3) / 1e9 / hbm,
+                               "nominal": {"peak": NOMINAL["hbm_gbs"], "unit": "GB/s",
+                                           "frac": lb / (ms / 1e3) / 1e9 / NOMINAL["hbm_gbs"]},
                                "algorithmic_bytes": lb},
             "stage_ms": su,
             "e2e": {"value": job_throughput(cfg.T, n, e2e_ms), "unit": "tokens/s",
@@ -622,7 +631,9 @@ def main():
             "value": pcfg.T / (pm["ms"] / 1e3), "unit": "tokens/s", "ms_per_step": pm["ms"],
             "roofline": {"bound": "tensor", "kernel": FFN_PAIR_KERNEL, "achieved": ffn_tf,
                          "peak": tf, "unit": "TFLOP/s", "frac": ffn_tf / tf,
-                         "peak_source": "%s bf16_tflops (burst)" % peak_kind},
+                         "peak_source": "%s bf16_tflops (burst)" % peak_kind,
+                         "nominal": {"peak": NOMINAL["bf16_tflops"], "unit": "TFLOP/s",
+                                     "frac": ffn_tf / NOMINAL["bf16_tflops"]}},
             "layer_tflops": lay_tf, "layer_frac_sustained": lay_tf / tfs,
             "stage_ms": pm["stage_ms"], "clocks": pclk}
     if rank == 0 and n == 1 and not args.no_fp8 and args.config == "decode":
