@@ -134,7 +134,10 @@ MOGE_API int moge_combine(const moge_config *cfg, const void *y_perm, const floa
                  void *stream);
 
 /* Whole layer: route, permute, one grouped-FFN launch covering both
- * projections of routed AND shared experts, combine.
+ * projections of routed AND shared experts, combine. bf16: up to 8192 routed
+ * rows (T*K) the FFN launch also does the permute and runs one CTA per SM;
+ * larger batches run it on CTA pairs (2-SM tcgen05 MMA, 256 weight rows per
+ * item). Both give results within the same tolerance of the oracle.
  *   y[t] = residual[t] (if not NULL) + MoGE(x)[t];  y may alias residual, not x.
  * s_* may be NULL when S == 0; logit_bias may be NULL. The routing of the
  * call stays readable in the workspace (moge_workspace_routing). */
