@@ -139,33 +139,6 @@ __device__ __forceinline__ int chunk_at(int i, int fp, int k_chunks) {
 // half of the token rows at offset 16 KB.
 constexpr uint32_t kBOff = 16384u;
 
-__device__ __forceinline__ int ld_acquire(const int *p) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-__device__ __forceinline__ void fence_proxy_async_global() {
-    asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
-// Bounded wait until *ctr >= need (an up-projection's h rows of one expert).
-__device__ bool wait_counter(const int *ctr, int need, volatile int *abort) {
-    if (ld_acquire(ctr) >= need) return true;
-    const uint64_t t0 = globaltimer_ns();
-    for (uint32_t it = 1;; ++it) {
-        __nanosleep(64);
-        if (ld_acquire(ctr) >= need) return true;
-        if ((it & 63u) == 0) {
-            if (*abort) return false;
-            if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
-                raise_error(ERRBIT_TIMEOUT);
-                *abort = 1;
-                return false;
-            }
-        }
-    }
-}
-
 // Token rows this CTA stages per chunk and the one TMA box that carries them
 // (32, 64 or 128 rows; rows past the tile are loaded and never used).
 __device__ __forceinline__ void b_boxes(int bn, int &half, int &nbox, int &box_rows) {
@@ -534,44 +507,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_pair_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// Host side: tensor maps and the launch.
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn get_encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    }
-    return fn;
-}
-
-static bool encode(CUtensorMap *m, const void *base, cuuint32_t rank, const cuuint64_t *dims,
-                   const cuuint64_t *strides, const cuuint32_t *box) {
-    EncodeTiledFn fn = get_encode_fn();
-    if (!fn) return false;
-    const cuuint32_t estr[4] = {1, 1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), dims, strides,
-              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// bf16 [experts][rows][cols] weights, box = [box_rows][64 cols] of one expert
-static bool encode_weights(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows,
-                           uint64_t experts, uint32_t box_rows) {
-    const cuuint64_t dims[3] = {cols, rows, experts};
-    const cuuint64_t strides[2] = {cols * 2, cols * rows * 2};
-    const cuuint32_t box[3] = {(cuuint32_t)kChunkK, box_rows, 1};
-    return encode(m, base, 3, dims, strides, box);
-}
-
+// Host side: tensor maps and the launch. The weight maps (encode_weights,
+// encode_gate_up) and the bounded counter wait are the single-SM kernel's;
+// token-row maps here take the box height.
 // bf16 [rows][cols] row matrix, box = [box_rows][64 cols]
 static bool encode_rows(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows,
                         uint32_t box_rows) {
@@ -579,36 +517,6 @@ static bool encode_rows(CUtensorMap *m, const void *base, uint64_t cols, uint64_
     const cuuint64_t strides[1] = {cols * 2};
     const cuuint32_t box[2] = {(cuuint32_t)kChunkK, box_rows};
     return encode(m, base, 2, dims, strides, box);
-}
-
-// One map over both the gate and the up tensor ([E][rows][cols] each, dense):
-// dims {cols, rows, E, 2}, the last dimension stepping from one tensor to the
-// other, so a {64, 64, 1, 2} box is one 16 KB copy of 64 gate rows followed by
-// the 64 matching up rows. Strides must increase, so this needs the two
-// tensors not to overlap; the tensor at the lower address becomes the first
-// half of the tile. Returns kGateUpSplit when they overlap (or on failure),
-// and the caller then uses two 3-D maps.
-static int encode_gate_up(CUtensorMap *m, const void *gate, const void *up, uint64_t cols,
-                          uint64_t rows, uint64_t experts) {
-    const int64_t bytes = (int64_t)(cols * rows * experts * 2);
-    const int64_t delta = static_cast<const char *>(up) - static_cast<const char *>(gate);
-    int mode;
-    const void *base;
-    if (delta >= bytes) {
-        mode = kGateUpFused;
-        base = gate;
-    } else if (-delta >= bytes) {
-        mode = kUpGateFused;
-        base = up;
-    } else {
-        return kGateUpSplit;
-    }
-    const uint64_t step = (uint64_t)(delta >= 0 ? delta : -delta);
-    if (step % 16 != 0 || step >= (1ull << 40)) return kGateUpSplit;
-    const cuuint64_t dims[4] = {cols, rows, experts, 2};
-    const cuuint64_t strides[3] = {cols * 2, cols * rows * 2, step};
-    const cuuint32_t box[4] = {(cuuint32_t)kChunkK, 64, 1, 2};
-    return encode(m, base, 4, dims, strides, box) ? mode : kGateUpSplit;
 }
 
 static size_t tc_smem_bytes() {
