@@ -1,7 +1,7 @@
-"""The expert-parallel decomposition run as two gloo ranks on the CPU (no
-GPU): each rank owns half of the tokens, all-gathers x, takes its share of
-the weights with the library's sharding helper (half of the expert groups and
-half of every shared expert's intermediate features), computes its partial of
+"""The expert-parallel decomposition run as two and four gloo ranks on the CPU
+(no GPU): each rank owns 1/R of the tokens, all-gathers x, takes its share of
+the weights with the library's sharding helper (1/R of the expert groups and
+of every shared expert's intermediate features), computes its partial of
 the layer with the oracle, and the partials are summed across the ranks (the
 reduce-scatter's arithmetic); every rank's rows must then equal the oracle's
 whole layer. This checks the sharding and the exchange pattern the CUDA path
@@ -11,6 +11,7 @@ import os
 import socket
 
 import numpy as np
+import pytest
 import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
@@ -63,8 +64,8 @@ def _worker(rank, world, port, out):
         dist.destroy_process_group()
 
 
-def test_two_gloo_ranks_expert_parallel_layer():
-    world = 2
+@pytest.mark.parametrize("world", [2, 4])
+def test_gloo_ranks_expert_parallel_layer(world):
     ctx = mp.get_context("spawn")
     mgr = ctx.Manager()
     out = mgr.dict()
@@ -81,4 +82,5 @@ def test_two_gloo_ranks_expert_parallel_layer():
     for r in range(world):
         assert out[r]["x_ok"]
         assert out[r]["err"] <= 1e-12, out[r]
-        assert out[r]["shapes"] == [(8, 24, 32), (2, 12, 32), (2, 32, 12)]
+        n_loc, i_loc = CFG.N // world, CFG.I // world
+        assert out[r]["shapes"] == [(n_loc, 24, 32), (2, i_loc, 32), (2, 32, i_loc)]
