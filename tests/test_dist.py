@@ -1,5 +1,5 @@
-"""The data-parallel (N > 1) path of the benchmark, run as two gloo ranks on
-the CPU: every rank owns a different token batch and the same weights, the
+"""The data-parallel (N > 1) path of the benchmark, run as two and four gloo
+ranks on the CPU: every rank owns a different token batch and the same weights, the
 step time is the maximum over ranks, and the job throughput counts every
 rank's tokens. No GPU and no collective on the data path."""
 import os
@@ -31,7 +31,7 @@ def _worker(rank, world, port, out):
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         inp = bench.rank_inputs(TINY, rank)
-        local_ms = 1.0 + 0.5 * rank                  # a slower second rank
+        local_ms = 1.0 + 0.5 * rank                  # later ranks slower
         ms = bench.max_over_ranks(local_ms, True)
         xs = [torch.zeros(TINY.T * TINY.d, dtype=torch.float32) for _ in range(world)]
         dist.all_gather(xs, torch.from_numpy(inp["x"].ravel().copy()))
@@ -40,15 +40,16 @@ def _worker(rank, world, port, out):
         out[rank] = {
             "ms": ms,
             "value": bench.job_throughput(TINY.T, world, ms),
-            "x_same": bool(torch.equal(xs[0], xs[1])),
-            "w_same": bool(torch.equal(ws[0], ws[1])),
+            "x_distinct": all(not torch.equal(xs[i], xs[j])
+                              for i in range(world) for j in range(i + 1, world)),
+            "w_same": all(torch.equal(ws[0], w) for w in ws[1:]),
         }
     finally:
         dist.destroy_process_group()
 
 
-def test_two_gloo_ranks_weak_scaling_aggregation():
-    world = 2
+@pytest.mark.parametrize("world", [2, 4])
+def test_gloo_ranks_weak_scaling_aggregation(world):
     ctx = mp.get_context("spawn")
     mgr = ctx.Manager()
     out = mgr.dict()
@@ -61,9 +62,10 @@ def test_two_gloo_ranks_weak_scaling_aggregation():
         assert p.exitcode == 0
     for r in range(world):
         o = out[r]
-        assert o["ms"] == 1.5                       # max over ranks, seen by every rank
-        assert o["value"] == pytest.approx(2 * TINY.T / 1.5e-3)
-        assert not o["x_same"] and o["w_same"]      # own batch, replicated weights
+        slowest = 1.0 + 0.5 * (world - 1)
+        assert o["ms"] == slowest                   # max over ranks, seen by every rank
+        assert o["value"] == pytest.approx(world * TINY.T / (slowest * 1e-3))
+        assert o["x_distinct"] and o["w_same"]      # own batch, replicated weights
 
 
 def test_single_process_is_identity():
