@@ -1,4 +1,5 @@
-"""Thin Python binding of libmoge.so, the B200 (sm_100a) MoGE layer forward.
+"""Thin Python binding of libmoge.so, the B200 (sm_100a) MoGE layer: forward,
+training forward + backward, and the expert-parallel local step.
 
 Argument marshalling only: every step of the layer runs in the library's CUDA
 kernels. PyTorch provides device memory and streams. The entry points carry
