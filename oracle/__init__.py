@@ -25,13 +25,24 @@ F32, BF16 = 0, 1
 _DT = {"f32": F32, "bf16": BF16}
 
 
+def compile_lib(src: str, out: str) -> str:
+    """gcc -O2, strict IEEE double (no contraction, no fast math), shared library."""
+    tmp = out + ".tmp%d" % os.getpid()
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
+                           "-shared", "-fPIC", src, "-o", tmp, "-lm"])
+    os.replace(tmp, out)
+    return out
+
+
 def build(force: bool = False) -> str:
-    """Compile liboracle.so (gcc -O2, strict IEEE double, one thread)."""
+    """Compile liboracle.so (one thread). The environment variable
+    ORACLE_LIB names another build of oracle.c to load instead; only the
+    planted-mistake tests set it (tests/test_oracle_plants.py)."""
+    override = os.environ.get("ORACLE_LIB")
+    if override:
+        return override
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        tmp = _LIB + ".tmp%d" % os.getpid()
-        subprocess.check_call(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
-                               "-shared", "-fPIC", _SRC, "-o", tmp, "-lm"])
-        os.replace(tmp, _LIB)
+        compile_lib(_SRC, _LIB)
     return _LIB
 
 
