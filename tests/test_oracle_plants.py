@@ -60,6 +60,11 @@ PLANTS = {
     # backward: W_down gradient without the combine weight
     "dw_down_unweighted": [("if (gd) gd[(size_t)o * I + i] += w * dyt[o] * h[i];",
                             "if (gd) gd[(size_t)o * I + i] += dyt[o] * h[i];", 0)],
+    # router rows read with a wrong stride
+    "router_row_stride": [("load_row(w_router, dtype, (size_t)e * d, d, w);",
+                           "load_row(w_router, dtype, (size_t)e * (d - 1), d, w);", 0)],
+    # routed experts' W_up pointer taken from W_gate (copy-paste slip)
+    "up_from_gate": [("expert_ptr(w_up, dtype, e, per),", "expert_ptr(w_gate, dtype, e, per),", 0)],
     # 8-bit weights: E4M3 exponent bias 8 instead of 7
     "e4m3_bias": [("ldexp(1.0 + m / 8.0, e - 7)", "ldexp(1.0 + m / 8.0, e - 8)", 0)],
     # expert-parallel partial: routed outputs not weighted by their scores
