@@ -221,12 +221,15 @@ def layer(x: np.ndarray, inp: dict, M: int, Kp: int, dtype: str,
 
 def layer_backward(x: np.ndarray, inp: dict, M: int, Kp: int, dtype: str, dy: np.ndarray,
                    alpha: float = 0.0, idx: Optional[np.ndarray] = None,
-                   tokens: Optional[Sequence[int]] = None, weights: bool = True) -> dict:
+                   tokens: Optional[Sequence[int]] = None, weights: bool = True,
+                   routed_weights: bool = True) -> dict:
     """Gradients of sum_t dy_t . y_t + L_aux (routing held fixed) -- oracle.c,
     oracle_layer_backward. x, dy: float64 [T][d]; idx: optional picks [T][M*Kp]
     to hold the routing at (default: the oracle's own); tokens: only these
     tokens' terms (their dx rows exact, weight gradients partial); weights=False:
-    dx alone (no weight-gradient arrays, for full-size samples). Returns float64 arrays
+    dx alone (no weight-gradient arrays, for full-size samples); routed_weights=False:
+    the router's and the shared experts' weight gradients but not the routed
+    experts' (whose arrays are the large ones). Returns float64 arrays
     dx [T][d], w_router [N][d], w_gate/w_up [N][I][d], w_down [N][d][I],
     s_gate/s_up [S][I][d], s_down [S][d][I], and the scalar aux."""
     x = np.ascontiguousarray(x, np.float64)
@@ -241,10 +244,11 @@ def layer_backward(x: np.ndarray, inp: dict, M: int, Kp: int, dtype: str, dy: np
     b = None if b is None else np.ascontiguousarray(b, np.float32)
     out = {"dx": np.empty((T, d))}
     if weights:
-        out.update({"w_router": np.empty((N, d)), "w_gate": np.empty((N, I, d)),
-                    "w_up": np.empty((N, I, d)), "w_down": np.empty((N, d, I)),
-                    "s_gate": np.empty((S, I, d)), "s_up": np.empty((S, I, d)),
-                    "s_down": np.empty((S, d, I))})
+        out.update({"w_router": np.empty((N, d)), "s_gate": np.empty((S, I, d)),
+                    "s_up": np.empty((S, I, d)), "s_down": np.empty((S, d, I))})
+        if routed_weights:
+            out.update({"w_gate": np.empty((N, I, d)), "w_up": np.empty((N, I, d)),
+                        "w_down": np.empty((N, d, I))})
     aux = np.zeros(1)
     picks = None if idx is None else np.ascontiguousarray(idx, np.int32)
     toks = None if tokens is None else np.ascontiguousarray(tokens, np.int32)

@@ -545,7 +545,9 @@ static double expert_token_backward(const double *xt, const double *dyt, double 
  * tokens (may be NULL): only these n_tokens tokens' terms are taken -- their
  * dx rows are then exact (other rows zero), the weight gradients partial; the
  * routing and the balance loss's f still come from the whole batch.
- * The weight-gradient outputs (dwr ... dsd) may all be NULL together: only dx.
+ * Each group of weight-gradient outputs may be NULL on its own (the router's
+ * dwr; the routed experts' dwg, dwu, dwd together; the shared experts' dsg,
+ * dsu, dsd together): that group is then not formed. All NULL: only dx.
  * Every output array is overwritten. Shapes: dx [T][d], dwr [N][d],
  * dwg/dwu [N][I][d], dwd [N][d][I], dsg/dsu [S][I][d], dsd [S][d][I].
  * aux_out (may be NULL) receives L_aux.
@@ -577,15 +579,15 @@ int oracle_layer_backward(const double *x, int T, int d, int N, int M, int Kp, i
         free(dh);
         return 2;
     }
-    const int wgt = dwg != NULL;
+    const int wgr = dwr != NULL, wge = dwg != NULL, wgs = dsg != NULL;
     memset(dx, 0, sizeof(double) * (size_t)T * d);
-    if (wgt) {
-        memset(dwr, 0, sizeof(double) * (size_t)N * d);
+    if (wgr) memset(dwr, 0, sizeof(double) * (size_t)N * d);
+    if (wge) {
         memset(dwg, 0, sizeof(double) * (size_t)N * per);
         memset(dwu, 0, sizeof(double) * (size_t)N * per);
         memset(dwd, 0, sizeof(double) * (size_t)N * per);
     }
-    if (wgt && S > 0) {
+    if (wgs && S > 0) {
         memset(dsg, 0, sizeof(double) * (size_t)S * per);
         memset(dsu, 0, sizeof(double) * (size_t)S * per);
         memset(dsd, 0, sizeof(double) * (size_t)S * per);
@@ -628,9 +630,9 @@ int oracle_layer_backward(const double *x, int T, int d, int N, int M, int Kp, i
                 routed ? expert_ptr(w_gate, dtype, e, per) : expert_ptr(s_gate, dtype, e, per),
                 routed ? expert_ptr(w_up, dtype, e, per) : expert_ptr(s_up, dtype, e, per),
                 routed ? expert_ptr(w_down, dtype, e, per) : expert_ptr(s_down, dtype, e, per),
-                dtype, d, I, wgt ? (routed ? dwg : dsg) + e * per : NULL,
-                wgt ? (routed ? dwu : dsu) + e * per : NULL,
-                wgt ? (routed ? dwd : dsd) + e * per : NULL, dxt, row, g, u, h, dh);
+                dtype, d, I, (routed ? wge : wgs) ? (routed ? dwg : dsg) + e * per : NULL,
+                (routed ? wge : wgs) ? (routed ? dwu : dsu) + e * per : NULL,
+                (routed ? wge : wgs) ? (routed ? dwd : dsd) + e * per : NULL, dxt, row, g, u, h, dh);
             if (routed) dp[e] += o_dot;
         }
         const double *pt = p + (size_t)t * N;
@@ -640,7 +642,7 @@ int oracle_layer_backward(const double *x, int T, int d, int N, int M, int Kp, i
             const double dl = pt[e] * (dp[e] - pdp);
             load_row(w_router, dtype, (size_t)e * d, d, row);
             for (int c = 0; c < d; ++c) {
-                if (wgt) dwr[(size_t)e * d + c] += dl * xt[c];
+                if (wgr) dwr[(size_t)e * d + c] += dl * xt[c];
                 dxt[c] += dl * row[c];
             }
         }

@@ -167,3 +167,20 @@ def test_dx_only():
     only = oracle.layer_backward(x, inp, cfg.M, cfg.Kp, "f32", dy, 0.2, weights=False)
     assert set(only) == {"dx", "aux"}
     assert np.array_equal(only["dx"], full["dx"])
+
+
+def test_backward_without_routed_weight_gradients_changes_nothing_else():
+    """routed_weights=False leaves out only the routed experts' gradient arrays:
+    dx, the router's and the shared experts' gradients and L_aux are the full
+    run's, bit for bit."""
+    cfg = synth.Config("bw_sel", T=12, d=48, N=8, M=4, Kp=1, S=2, I=24, dtype="f32", seed=71,
+                       w_std=0.3)
+    inp = synth.layer_inputs(cfg)
+    x = oracle.to_double(inp["x"], cfg.dtype)
+    dy = oracle.to_double(synth.upstream_grad(cfg), cfg.dtype)
+    full = oracle.layer_backward(x, inp, cfg.M, cfg.Kp, cfg.dtype, dy, 0.2)
+    part = oracle.layer_backward(x, inp, cfg.M, cfg.Kp, cfg.dtype, dy, 0.2, routed_weights=False)
+    assert "w_gate" not in part and "w_up" not in part and "w_down" not in part
+    for k in ("dx", "w_router", "s_gate", "s_up", "s_down"):
+        assert np.array_equal(full[k], part[k]), k
+    assert full["aux"] == part["aux"]
