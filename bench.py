@@ -42,12 +42,73 @@ FFN_KERNEL = ("ffn_tc_kernel (grouped gate+up GEMM with SwiGLU epilogue and down
 # Nominal B200 figures, reported beside the measured denominators: HBM3e
 # ~8 TB/s and 2.25 PFLOP/s dense bf16.
 NOMINAL = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
-# DRAM bytes of one decode-workload launch of ffn_tc_kernel as it stands, from
-# one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum, cold cache):
-# 2.868 GB read + 65.4 MB written.
-DECODE_FFN_TRAFFIC = 2867918848 + 65411072
+# DRAM traffic of the dominant kernel comes from an ncu capture summarised
+# under profiles/: a line "traffic-record: {json}" there names the kernel, the
+# workload, the DRAM bytes of one launch (dram__bytes_read.sum +
+# dram__bytes_write.sum) and a hash of the CUDA sources the capture ran. The
+# bench reports it only while the sources still hash the same (else null: the
+# kernel changed since the counters were taken).
+TRAFFIC_RECORDS = ("profiles/ffn_tc_decode.md", "profiles/ffn_tc_pair_prefill.md")
 FFN_PAIR_KERNEL = ("ffn_tc_pair_kernel (the same grouped FFN on CTA pairs, 2-SM tcgen05 MMA, "
                    "one persistent launch)")
+
+
+def source_sha16():
+    """Hash of the library's CUDA sources (csrc/*.cu, *.cuh, *.h and the ABI
+    header), the key under which a traffic record is valid."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "mixture_grouped_experts_b200", "csrc")
+    files = sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh"))
+                   + glob.glob(os.path.join(csrc, "*.h"))) + [os.path.join(ROOT, "include", "moge.h")]
+    for f in files:
+        h.update(os.path.basename(f).encode())
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def traffic_record(kernel, workload):
+    """(bytes per launch, source) of the committed ncu record for this kernel
+    and workload when it was taken on the current sources, else (None, why)."""
+    sha = source_sha16()
+    for rel in TRAFFIC_RECORDS:
+        path = os.path.join(ROOT, rel)
+        if not os.path.exists(path):
+            continue
+        for line in open(path):
+            if not line.startswith("traffic-record:"):
+                continue
+            rec = json.loads(line.split(":", 1)[1])
+            if rec.get("kernel") != kernel or rec.get("workload") != workload:
+                continue
+            if rec.get("src_sha16") != sha:
+                return None, "%s: captured on sources %s, now %s (kernel changed)" % (
+                    rel, rec.get("src_sha16"), sha)
+            return int(rec["dram_bytes_per_launch"]), "%s (ncu, sources %s)" % (rel, sha)
+    return None, "no ncu record for %s on the %s workload" % (kernel, workload)
+
+
+def layer_launches(cfg, fp8=False):
+    """Kernel launches of one moge_layer_forward call, by the library's rules:
+    router, scan, permute, grouped FFN, combine; bf16 layers of at most 8192
+    routed rows (T * M * K') copy the permute inside the FFN launch."""
+    if cfg.dtype == "bf16" and not fp8 and cfg.T * cfg.M * cfg.Kp <= 8192:
+        return 4
+    return 5
+
+
+def host_cpu():
+    """(logical CPUs, CPU model name) of this host."""
+    model = ""
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    return os.cpu_count(), model
 
 
 def load_peaks():
@@ -182,7 +243,9 @@ def oracle_sample(cfg, inp, tokens):
 def cpu_baseline(cfg, inp, n_tokens):
     toks = list(range(0, cfg.T, max(1, cfg.T // n_tokens)))[:n_tokens]
     dt = oracle_sample(cfg, inp, toks)
+    nproc, model = host_cpu()
     return {"value": len(toks) / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "nproc": nproc, "cpu_model": model,
             "sample": "%d of the %d tokens of the %s layer, full layer per token (routing over "
                       "%d experts, %d routed + %d shared SwiGLU experts), fp64 C, one thread; %.1f s"
                       % (len(toks), cfg.T, cfg.name, cfg.N, cfg.K, cfg.S, dt)}
@@ -215,8 +278,10 @@ def run_reference(args, cfg):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1000.0 * t / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded normal inputs)",
-            "config": workload_config(cfg),
+            "config": dict(workload_config(cfg),
+                           parallelism="replicas (dp%d), no collective" % args.gpus),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "nproc": host_cpu()[0], "cpu_model": host_cpu()[1],
                              "sample": "each step: %d random tokens of the %d-token batch, full layer "
                                        "per token, fp64 C oracle, one thread" % (per_step, cfg.T)},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -411,6 +476,39 @@ def measure_stack(cfg, steps, warmup):
     return ms
 
 
+def imbalance_score(counts, M, assignments):
+    """Imbalance score of one batch: (busiest group's load - idlest group's
+    load) / all (token, expert) assignments, the N experts in M contiguous
+    groups."""
+    import numpy as np
+    loads = np.asarray(counts).reshape(M, -1).sum(axis=1)
+    return {"score": float((loads.max() - loads.min()) / assignments),
+            "group_loads": [int(v) for v in loads]}
+
+
+def global_topk_imbalance(cfg, inp):
+    """Route the same batch (same x, router weights and bias) by conventional
+    global top-K (the library's router with one group of all N experts and K
+    picks) and report its imbalance score over the layer's M groups."""
+    import torch
+    import mixture_grouped_experts_b200 as mg
+    s1 = mg.shape_of(cfg, M=1, Kp=cfg.K, S=0)
+    x = mg.to_device(inp["x"], cfg.dtype)
+    wr = mg.to_device(inp["w_router"], cfg.dtype)
+    lb = inp.get("logit_bias")
+    lb = None if lb is None else torch.from_numpy(lb).cuda()
+    ws = mg.alloc_workspace(s1)
+    counts = mg.moge_route(s1, x, wr, lb, ws)[2]
+    torch.cuda.synchronize()
+    mg.check_device_errors()
+    out = imbalance_score(counts.cpu().numpy(), cfg.M, cfg.T * cfg.K)
+    out["routing"] = "global top-%d of %d experts on the same logits (library router, M=1)" % (
+        cfg.K, cfg.N)
+    del x, wr, ws
+    torch.cuda.empty_cache()
+    return out
+
+
 def max_over_ranks(v, dist_on):
     """Max of a per-rank scalar over all ranks (identity on one process).
     Uses a CUDA tensor under NCCL and a CPU tensor under gloo."""
@@ -569,28 +667,39 @@ def main():
 
     su = m["stage_ms"]
     hbm = peaks["hbm_gbs"]
-    fb = ffn_bytes(cfg, m["n_used"])
-    ach = fb / (su["ffn"] / 1e3) / 1e9
+    tf_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    tf_sust = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    lb = layer_bytes(cfg, m["n_used"])
     if cfg.T * cfg.M * cfg.Kp < PAIR_ROWS:
+        # algorithmic bytes of the layer (the used experts' three matrices once,
+        # the router, x in, y out: no padding, permute or intermediate rows) over
+        # the grouped FFN's live launch time
+        ach = lb / (su["ffn"] / 1e3) / 1e9
+        fb_incl = ffn_bytes(cfg, m["n_used"])
+        traffic, tsrc = traffic_record("ffn_tc_kernel", cfg.name)
         roofline = {"bound": "hbm", "kernel": FFN_KERNEL,
                     "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
                     "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
                     else "fallback 6650 GB/s",
-                    "traffic": DECODE_FFN_TRAFFIC if args.config == "decode" else None,
+                    "traffic": traffic, "traffic_source": tsrc,
                     "nominal": {"peak": NOMINAL["hbm_gbs"], "unit": "GB/s",
                                 "frac": ach / NOMINAL["hbm_gbs"]},
-                    "algorithmic_bytes_per_launch": fb,
+                    "algorithmic_bytes_per_launch": lb,
+                    "algorithmic_bytes_are": "used experts' three matrices once + router + x in + y out",
+                    "bytes_incl_intermediates": fb_incl,
+                    "frac_incl_intermediates": fb_incl / (su["ffn"] / 1e3) / 1e9 / hbm,
                     "kernel_ms": su["ffn"]}
     else:  # prefill-sized batches: the contraction bounds the pair kernel
-        tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
         ftf = ffn_flops(cfg) / (su["ffn"] / 1e3) / 1e12
-        roofline = {"bound": "tensor", "kernel": FFN_PAIR_KERNEL, "achieved": ftf, "peak": tf,
-                    "unit": "TFLOP/s", "frac": ftf / tf,
-                    "peak_source": "%s bf16_tflops (burst)" % peak_kind, "traffic": None,
+        traffic, tsrc = traffic_record("ffn_tc_pair_kernel", cfg.name)
+        roofline = {"bound": "tensor", "kernel": FFN_PAIR_KERNEL, "achieved": ftf, "peak": tf_burst,
+                    "unit": "TFLOP/s", "frac": ftf / tf_burst,
+                    "peak_source": "%s bf16_tflops (burst)" % peak_kind,
+                    "sustained": {"peak": tf_sust, "frac": ftf / tf_sust},
+                    "traffic": traffic, "traffic_source": tsrc,
                     "nominal": {"peak": NOMINAL["bf16_tflops"], "unit": "TFLOP/s",
                                 "frac": ftf / NOMINAL["bf16_tflops"]},
                     "algorithmic_flops_per_launch": ffn_flops(cfg), "kernel_ms": su["ffn"]}
-    lb = layer_bytes(cfg, m["n_used"])
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": n, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded normal inputs, random-init weights)",
@@ -610,7 +719,7 @@ def main():
                     "sync_per_step": {"value": job_throughput(cfg.T, n, max_over_ranks(
                         m.get("e2e_sync_ms", float("nan")), dist_on)), "unit": "tokens/s",
                         "api": "moge_layer_forward_host (one batch, synchronised per step)"}},
-            "gpu_launches": 5 * args.steps,
+            "gpu_launches": layer_launches(cfg) * args.steps,
             "clocks": clocks}
     if rank == 0 and n == 1 and args.cpu_tokens > 0:
         line["cpu_baseline"] = cpu_baseline(cfg, inp, args.cpu_tokens)
@@ -634,7 +743,11 @@ def main():
                          "peak_source": "%s bf16_tflops (burst)" % peak_kind,
                          "nominal": {"peak": NOMINAL["bf16_tflops"], "unit": "TFLOP/s",
                                      "frac": ffn_tf / NOMINAL["bf16_tflops"]}},
-            "layer_tflops": lay_tf, "layer_frac_sustained": lay_tf / tfs,
+            "layer_roofline": {"bound": "tensor", "achieved": lay_tf, "peak": tf, "unit": "TFLOP/s",
+                               "frac": lay_tf / tf, "peak_source": "%s bf16_tflops (burst)" % peak_kind,
+                               "sustained": {"peak": tfs, "frac": lay_tf / tfs},
+                               "algorithmic_flops": layer_flops(pcfg)},
+            "gpu_launches_per_step": layer_launches(pcfg),
             "stage_ms": pm["stage_ms"], "clocks": pclk}
     if rank == 0 and n == 1 and not args.no_fp8 and args.config == "decode":
         finp = synth.layer_inputs(cfg)
@@ -657,6 +770,7 @@ def main():
                          "kernel_ms": fm["stage_ms"]["ffn"]},
             "layer_roofline": {"achieved": lb8 / (fm["ms"] / 1e3) / 1e9, "peak": hbm, "unit": "GB/s",
                                "frac": lb8 / (fm["ms"] / 1e3) / 1e9 / hbm, "algorithmic_bytes": lb8},
+            "gpu_launches_per_step": layer_launches(cfg, fp8=True),
             "stage_ms": fm["stage_ms"], "clocks": fclk}
     if rank == 0 and n == 1 and not args.no_train and args.config == "decode":
         tcfg = synth.CONFIGS["prefill"]
@@ -666,6 +780,7 @@ def main():
         tm = measure_train(tcfg, tinp, max(5, args.steps // 2), args.warmup)
         tclk = ts.stop()
         del tinp
+        tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
         tfs = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
         ach = train_flops(tcfg) / (tm["step_ms"] / 1e3) / 1e12
         bwd_ms = tm["step_ms"] - tm["fwd_ms"]
@@ -677,9 +792,11 @@ def main():
             "value": tcfg.T / (tm["step_ms"] / 1e3), "unit": "tokens/s",
             "ms_per_step": tm["step_ms"], "forward_ms": tm["fwd_ms"], "backward_ms": bwd_ms,
             "roofline": {"bound": "tensor", "kernel": "training step (forward + backward GEMMs)",
-                         "achieved": ach, "peak": tfs, "unit": "TFLOP/s", "frac": ach / tfs,
+                         "achieved": ach, "peak": tf, "unit": "TFLOP/s", "frac": ach / tf,
                          "flops_per_step": train_flops(tcfg),
-                         "peak_source": "%s bf16_tflops_sustained" % peak_kind},
+                         "peak_source": "%s bf16_tflops (burst: the timed region is tens of "
+                                        "milliseconds)" % peak_kind,
+                         "sustained": {"peak": tfs, "frac": ach / tfs}},
             "backward_tflops": bwd_tf, "clocks": tclk}
     if rank == 0 and n == 1 and not args.no_extra and args.config == "decode":
         kcfg = synth.CONFIGS["skew"]
@@ -689,17 +806,25 @@ def main():
         km = measure(kcfg, kinp, 5, args.warmup, False, with_e2e=False)
         kclk = ks.stop()
         del kinp
+        tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
         tfs = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
         k_tf = layer_flops(kcfg) / (km["ms"] / 1e3) / 1e12
         cnt = km["counts"]
+        gim = global_topk_imbalance(kcfg, synth.layer_inputs(kcfg))
         line["skew"] = {
             "workload": workload_config(kcfg)["workload"],
             "value": kcfg.T / (km["ms"] / 1e3), "unit": "tokens/s", "ms_per_step": km["ms"],
-            "roofline": {"bound": "tensor", "achieved": k_tf, "peak": tfs, "unit": "TFLOP/s",
-                         "frac": k_tf / tfs, "peak_source": "%s bf16_tflops_sustained" % peak_kind},
+            "roofline": {"bound": "tensor", "kernel": "whole layer", "achieved": k_tf, "peak": tf,
+                         "unit": "TFLOP/s", "frac": k_tf / tf,
+                         "peak_source": "%s bf16_tflops (burst)" % peak_kind,
+                         "sustained": {"peak": tfs, "frac": k_tf / tfs},
+                         "algorithmic_flops": layer_flops(kcfg)},
             "expert_rows": {"max": int(cnt.max()), "min": int(cnt.min())},
             "group_rows": [int(cnt[g * (kcfg.N // kcfg.M):(g + 1) * (kcfg.N // kcfg.M)].sum())
                            for g in range(kcfg.M)],
+            "imbalance_moge": imbalance_score(cnt, kcfg.M, kcfg.T * kcfg.K),
+            "imbalance_global_top8": gim,
+            "gpu_launches_per_step": layer_launches(kcfg),
             "stage_ms": km["stage_ms"], "clocks": kclk}
         scfg = synth.CONFIGS["stack12"]
         ss = ClockSampler(local)

@@ -106,29 +106,44 @@ MOGE_API int moge_route(const moge_config *cfg, const void *x, const void *w_rou
                int32_t *offsets, int32_t *perm_src, int32_t *perm_dst, void *workspace,
                void *stream);
 
-/* Permute: x_perm[r] = x[perm_src[r]] for r < T*K (rows of d, dtype). */
+/* Permute: x_perm[r] = x[perm_src[r]] for r < T*K (rows of d, dtype).
+ * The dispatch of every token to the K' picked experts of each group
+ * (techwalker.com article, section 1: every group receives the tokens routed
+ * to its experts), laid out expert by expert as the grouped matmul of
+ * section 3 reads it. Rows of one expert in ascending token order. */
 MOGE_API int moge_permute(const moge_config *cfg, const void *x, const int32_t *perm_src, void *x_perm,
                  void *stream);
 
 /* Grouped routed-expert FFN over expert-major rows: for every expert e and
  * row r in [offsets[e], offsets[e+1]):
  *   y_perm[r] = W_down[e] (silu(W_gate[e] x_perm[r]) * (W_up[e] x_perm[r]))
+ * The grouped expert matmul ("GroupMatmul", whose SwiftGMM kernel picks a
+ * GEMV- or GEMM-like path by load: techwalker.com article, section 3, and the
+ * reportify.cn product digest); the pages do not give the expert's internals,
+ * the SwiGLU form is this library's reading.
  * x_perm, y_perm [T*K][d] dtype; offsets [N+1] int32 on the device.
  * bf16: tcgen05 tensor-core GEMMs (TMA-fed, TMEM accumulators), the SwiGLU
- * product rounded to bf16 between the two GEMMs. */
+ * product rounded to bf16 between the two GEMMs; above 8192 rows (T*K) on CTA
+ * pairs (2-SM MMA), as in moge_layer_forward. */
 MOGE_API int moge_grouped_ffn(const moge_config *cfg, const void *x_perm, const int32_t *offsets,
                      const void *w_gate, const void *w_up, const void *w_down, void *y_perm,
                      void *workspace, void *stream);
 
-/* Shared experts: y_shared[t] = sum_{s<S} FFN_s(x[t]); x, y_shared [T][d]. */
+/* Shared experts: y_shared[t] = sum_{s<S} FFN_s(x[t]); x, y_shared [T][d].
+ * The always-on shared experts (techwalker.com article, section 2: 4 shared
+ * beside the 64 routed experts; mokono.cn news page, item 1), each an FFN of
+ * the routed experts' form, entering with weight 1. Above 8192 rows (T*S) on
+ * CTA pairs. */
 MOGE_API int moge_shared_ffn(const moge_config *cfg, const void *x, const void *s_gate,
                     const void *s_up, const void *s_down, void *y_shared, void *workspace,
                     void *stream);
 
 /* Combine: y[t] = residual[t] + sum_{k<K} topk_w[t][k] * y_perm[perm_dst[t][k]]
  *                 + y_shared[t]
- * summed in fp32 in this order (k ascending); residual and y_shared may be
- * NULL (treated as zero). y may alias residual. */
+ * The picked experts' outputs weighted by their global softmax scores
+ * (techwalker.com article, section 1; no renormalisation) plus the shared
+ * experts' (section 2). Summed in fp32 in this order (k ascending); residual
+ * and y_shared may be NULL (treated as zero). y may alias residual. */
 MOGE_API int moge_combine(const moge_config *cfg, const void *y_perm, const float *topk_w,
                  const int32_t *perm_dst, const void *y_shared, const void *residual, void *y,
                  void *stream);
@@ -198,7 +213,8 @@ MOGE_API int moge_rmsnorm(const moge_config *cfg, const void *x, float eps, void
  * round256(T*K*4) <= 1048576 bytes (e.g. T <= 16384 at N = 64, K = 8);
  * larger batches return MOGE_ERR_UNSUPPORTED with a message. Allocates
  * nothing. The first call on a device (with that device current) looks up the
- * array's device address; make that first call before any stream capture.
+ * array's device address, and again the first call after the device's context
+ * changed (a cudaDeviceReset); make those calls before any stream capture.
  * All calls on a device share the array: calls that overlap on the GPU race,
  * so order them on one stream. Nothing in the array needs clearing between
  * calls (each call writes every scratch word it reads). */

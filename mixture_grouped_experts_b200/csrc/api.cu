@@ -459,6 +459,11 @@ int moge_grouped_ffn(const moge_config *cfg, const void *x_perm, const int32_t *
     const int64_t rows = (int64_t)c.T * c.M * c.Kp;
     FfnOperands op{x_perm, nullptr, rows, 0, w_gate, w_up, w_down, nullptr, nullptr, nullptr,
                    ws.h, rows, y_perm};
+    if (c.dtype == MOGE_BF16 && rows >= kPairRows) {  // prefill-sized: CTA pairs, as the layer does
+        MOGE_CU(pair::launch_ffn_tc_pair(c, ws.plan, c.N, op, num_sms(), st),
+                "grouped FFN (tcgen05 pairs) launch");
+        return MOGE_OK;
+    }
     return run_ffn(c, ws.plan, c.N, op, st);
 }
 
@@ -485,8 +490,13 @@ int moge_shared_ffn(const moge_config *cfg, const void *x, const void *s_gate, c
     const int64_t rows = (int64_t)c.T * c.S;
     FfnOperands op{nullptr, x, 0, c.T, nullptr, nullptr, nullptr, s_gate, s_up, s_down,
                    ws.h, rows, ws.y_perm};
-    rc = run_ffn(c, ws.plan, c.S, op, st);
-    if (rc) return rc;
+    if (c.dtype == MOGE_BF16 && rows >= kPairRows) {  // prefill-sized: CTA pairs, as the layer does
+        MOGE_CU(pair::launch_ffn_tc_pair(c, ws.plan, c.S, op, num_sms(), st),
+                "grouped FFN (tcgen05 pairs) launch");
+    } else {
+        rc = run_ffn(c, ws.plan, c.S, op, st);
+        if (rc) return rc;
+    }
     MOGE_CU(launch_combine(c, nullptr, nullptr, nullptr, 0, ws.y_perm, c.S, nullptr, y_shared, st),
             "shared sum launch");
     return MOGE_OK;

@@ -19,8 +19,10 @@
 // of every (token, pick)).
 //
 // In host code the array's name is only a host-side shadow, not a device
-// address; the device address is taken once per device with
-// cudaGetSymbolAddress, on the first call made while that device is current.
+// address; the device address is taken with cudaGetSymbolAddress on the first
+// call made while that device is current, and looked up again whenever the
+// device's context is a different one (after a cudaDeviceReset the module is
+// loaded anew, possibly at another address).
 #include <mutex>
 
 #include "common.cuh"
@@ -33,6 +35,26 @@ static __device__ __align__(256) unsigned char g_route_scratch[kRouteScratchByte
 
 static std::mutex g_route_scratch_mu;
 static void *g_route_scratch_dev[64] = {nullptr};
+static void *g_route_scratch_ctx[64] = {nullptr};  // the context each address belongs to
+
+// The calling thread's current driver context (through the runtime's driver
+// entry point: the library does not link libcuda); nullptr if unavailable.
+static void *current_context() {
+    typedef CUresult (*GetCurrentFn)(CUcontext *);
+    static GetCurrentFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<GetCurrentFn>(ptr);
+        tried = true;
+    }
+    CUcontext ctx = nullptr;
+    if (!fn || fn(&ctx) != CUDA_SUCCESS) return nullptr;
+    return ctx;
+}
 
 // Scratch layout: hist [tiles][N] | base [tiles][N] | rank [T][K], each
 // region rounded up to 256 bytes.
@@ -45,17 +67,21 @@ static size_t route_scratch_layout(const moge_config &c, size_t *off_base, size_
     return 2 * h + r;
 }
 
-// Device address of the scratch array on the current device (set up once per device).
+// Device address of the scratch array on the current device (set up once per
+// device and context).
 static int route_scratch_ptr(unsigned char **out) {
     int dev = -1;
     MOGE_CU(cudaGetDevice(&dev), "cudaGetDevice");
     if (dev < 0 || dev >= 64) return fail(MOGE_ERR_UNSUPPORTED, "device index above 63");
     std::lock_guard<std::mutex> lock(g_route_scratch_mu);
-    if (!g_route_scratch_dev[dev]) {
+    void *ctx = current_context();
+    if (!g_route_scratch_dev[dev] || !ctx || ctx != g_route_scratch_ctx[dev]) {
         void *p = nullptr;
         const cudaError_t e = cudaGetSymbolAddress(&p, g_route_scratch);
         if (e != cudaSuccess || !p) return cuda_fail(e, "cudaGetSymbolAddress(route scratch)");
         g_route_scratch_dev[dev] = p;
+        // the runtime creates the context on the lookup above if none was current
+        g_route_scratch_ctx[dev] = ctx ? ctx : current_context();
     }
     *out = static_cast<unsigned char *>(g_route_scratch_dev[dev]);
     return MOGE_OK;

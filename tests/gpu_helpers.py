@@ -86,6 +86,84 @@ def sample_tokens(T, n, seed=0):
     return np.array(out[:max(n, 1)] if len(out) > n else out, dtype=np.int64)
 
 
+# ------------------------------------------------------------------ oracle pool
+# The oracle is single-threaded; full-size checks of hundreds of tokens run it
+# in worker processes. Workers are started with "spawn" (never forked from a
+# process that has touched the GPU) and regenerate the seeded inputs of the
+# config themselves, so only token lists and results cross the pipe.
+def _pool_workers():
+    import os
+    return max(1, min(8, (os.cpu_count() or 2) // 2))
+
+
+def _oracle_layer_job(args):
+    cfg, tokens = args
+    inp = synth.layer_inputs(cfg)
+    xd = oracle.to_double(inp["x"], cfg.dtype)
+    return oracle.layer(xd, inp, cfg.M, cfg.Kp, cfg.dtype, tokens=tokens)[0]
+
+
+def _oracle_backward_job(args):
+    cfg, alpha, idx, tokens = args
+    inp = synth.layer_inputs(cfg)
+    xd = oracle.to_double(inp["x"], cfg.dtype)
+    dy = oracle.to_double(synth.upstream_grad(cfg), cfg.dtype)
+    return oracle.layer_backward(xd, inp, cfg.M, cfg.Kp, cfg.dtype, dy, alpha, idx=idx,
+                                 tokens=tokens, routed_weights=False)
+
+
+def _split(tokens, n):
+    tokens = np.asarray(tokens, dtype=np.int64)
+    return [c for c in np.array_split(tokens, n) if len(c)]
+
+
+def oracle_layer_pool(cfg, tokens):
+    """oracle.layer outputs of the listed tokens of the seeded config `cfg`
+    (its unmodified synth inputs), computed in spawned worker processes."""
+    import multiprocessing as mp
+    chunks = _split(tokens, min(_pool_workers(), max(1, len(tokens) // 4)))
+    with mp.get_context("spawn").Pool(len(chunks)) as pool:
+        parts = pool.map(_oracle_layer_job, [(cfg, c) for c in chunks])
+    return np.concatenate(parts, axis=0)
+
+
+def oracle_backward_pool(cfg, alpha, idx, tokens):
+    """oracle.layer_backward of the seeded config `cfg` at the picks idx,
+    without the routed experts' weight gradients: the token terms are split
+    over spawned workers and summed (every gradient is a sum over tokens; the
+    balance loss's f comes from the whole batch in each part)."""
+    import multiprocessing as mp
+    chunks = _split(tokens, _pool_workers())
+    with mp.get_context("spawn").Pool(len(chunks)) as pool:
+        parts = pool.map(_oracle_backward_job, [(cfg, alpha, idx, c) for c in chunks])
+    out = {k: sum(p[k] for p in parts) for k in parts[0] if k != "aux"}
+    out["aux"] = parts[0]["aux"]
+    return out
+
+
+def expert_tiles(rows, max_tile=256, stream_rows=64):
+    """Token tiles [start, end) of an expert with `rows` rows, by the grouped
+    FFN's tiling rule (one tile up to 64 rows, else ceil(rows / 256) balanced
+    tiles of a multiple-of-16 width). Used to pick tokens tile by tile."""
+    if rows <= 0:
+        return []
+    if rows <= stream_rows:
+        return [(0, rows)]
+    nt = -(-rows // max_tile)
+    bn = (-(-rows // nt) + 15) // 16 * 16
+    return [(a, min(rows, a + bn)) for a in range(0, rows, bn)]
+
+
+def tile_tokens(perm_src, offsets, e, tiles):
+    """Tokens held by the listed token tiles (indices into expert_tiles) of expert e."""
+    out = []
+    t_all = expert_tiles(int(offsets[e + 1] - offsets[e]))
+    for i in tiles:
+        a, b = t_all[i]
+        out += perm_src[offsets[e] + a:offsets[e] + b].tolist()
+    return out
+
+
 def run_layer(cfg, x_dev, w_dev, ws, residual=None):
     s = mg.shape_of(cfg)
     y = mg.moge_layer_forward(s, x_dev, w_dev, ws, residual=residual)
@@ -96,9 +174,13 @@ def run_layer(cfg, x_dev, w_dev, ws, residual=None):
             offsets.cpu().numpy())
 
 
-def layer_parity(cfg, inp, n_sample=None, tokens=None):
+def layer_parity(cfg, inp, n_sample=None, tokens=None, by_tiles=None):
     """Full layer on the GPU vs the oracle: routing of all tokens, outputs of
-    sampled tokens (all tokens when n_sample is None and tokens is None)."""
+    sampled tokens (all tokens when n_sample is None and tokens is None).
+    by_tiles (a function of (perm_src, offsets, counts) returning tokens):
+    more tokens chosen from the GPU's own dispatch, every token of whole token
+    tiles; they are run through the oracle in worker processes, which needs
+    `inp` to be the config's unmodified seeded inputs."""
     x, w = device_inputs(cfg, inp)
     ws = mg.alloc_workspace(mg.shape_of(cfg))
     y, idx_g, w_g, counts_g, offsets_g = run_layer(cfg, x, w, ws)
@@ -111,6 +193,13 @@ def layer_parity(cfg, inp, n_sample=None, tokens=None):
         tokens = np.arange(cfg.T) if n_sample is None else sample_tokens(cfg.T, n_sample)
     tokens = np.array([t for t in tokens if safe[t]], dtype=np.int64)
     y_ref, _, _, _ = oracle.layer(xd, inp, cfg.M, cfg.Kp, cfg.dtype, tokens=tokens)
+    if by_tiles is not None:
+        ps = oracle.dispatch(idx_g, cfg.N)[2]
+        extra = sorted(set(int(t) for t in by_tiles(ps, offsets_g, counts_g)
+                           if safe[t]) - set(tokens.tolist()))
+        if extra:
+            y_ref = np.concatenate([y_ref, oracle_layer_pool(cfg, extra)], axis=0)
+            tokens = np.concatenate([tokens, np.array(extra, dtype=np.int64)])
     y_g = to_host_f64(y)[tokens]
     err = normwise_err(y_g, y_ref)
     assert err <= TOL[cfg.dtype], (cfg.name, err)

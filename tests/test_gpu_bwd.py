@@ -19,7 +19,7 @@ import torch
 import mixture_grouped_experts_b200 as mg
 import oracle
 import synth
-from gpu_helpers import check_routing, sample_tokens, to_host_f64
+from gpu_helpers import check_routing, oracle_backward_pool, sample_tokens, to_host_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -148,3 +148,48 @@ def test_backward_full_size_prefill_sampled():
         assert err <= TOL, (k, e, len(rows), err)
     gr = grads["w_router"].float()
     assert float(gr.sum(0).abs().max() / gr.abs().max()) <= 0.05
+
+
+def test_backward_full_dims_small_batch_elementwise():
+    """The workload's layer dimensions (d = 5120, 64 experts in 8 groups,
+    K' = 1, 4 shared experts, I = 1344) on a batch of 128 tokens, small enough
+    for the oracle to form complete gradients: dx of every token, the router's
+    gradient and every shared expert's three gradients compared element-wise
+    (normwise per tensor), and the routed gradients of the experts with the
+    most and the fewest tokens."""
+    cfg = synth.Config("bw_full_dims", T=128, d=5120, N=64, M=8, Kp=1, S=4, I=1344,
+                       dtype="bf16", seed=66)
+    alpha = 0.01
+    inp = synth.layer_inputs(cfg)
+    x = oracle.to_double(inp["x"], cfg.dtype)
+    s = mg.shape_of(cfg)
+    xd = mg.to_device(inp["x"], cfg.dtype)
+    w = mg.weights_to_device(inp, cfg.dtype)
+    dy_h = synth.upstream_grad(cfg)
+    ws = mg.alloc_train_workspace(s)
+    aux = torch.zeros(1, dtype=torch.float32, device="cuda")
+    mg.moge_layer_forward_train(s, xd, w, ws)
+    idx_g, w_g, _, _ = mg.moge_workspace_routing(s, ws)
+    idx_g, w_g = idx_g.cpu().numpy(), w_g.cpu().numpy()
+    dx, grads = mg.moge_layer_backward(s, xd, w, mg.to_device(dy_h, "bf16"), ws, alpha=alpha,
+                                       aux=aux)
+    torch.cuda.synchronize()
+    mg.check_device_errors()
+    p = oracle.router_probs(x, inp["w_router"], None, cfg.dtype)
+    idx_o, _, mg_o = oracle.select_grouped(p, cfg.M, cfg.Kp)
+    check_routing(cfg, p, idx_o, mg_o, idx_g, w_g)
+    ref = oracle_backward_pool(cfg, alpha, idx_g, np.arange(cfg.T))
+    errs = {"dx": _normwise(to_host_f64(dx), ref["dx"])}
+    for k in ("w_router", "s_gate", "s_up", "s_down"):
+        errs[k] = _normwise(to_host_f64(grads[k]), ref[k])
+    dyd = oracle.to_double(dy_h, "bf16")
+    cnt = np.bincount(idx_g.ravel(), minlength=cfg.N)
+    for e in (int(np.argmax(cnt)), int(np.argmin(np.where(cnt > 0, cnt, 1 << 30)))):
+        rows = np.nonzero((idx_g == e).any(1))[0]
+        ref_w = oracle.expert_backward(x[rows], dyd[rows], p[rows, e], inp["w_gate"][e],
+                                       inp["w_up"][e], inp["w_down"][e], cfg.dtype)
+        for k, r in zip(("w_gate", "w_up", "w_down"), ref_w):
+            errs["%s[%d]" % (k, e)] = _normwise(to_host_f64(grads[k][e]), r)
+    for k, e in errs.items():
+        assert e <= TOL, (k, e, errs)
+    assert abs(float(aux.item()) - ref["aux"]) <= 1e-3 * abs(ref["aux"]), (aux.item(), ref["aux"])

@@ -11,7 +11,7 @@ import torch
 import mixture_grouped_experts_b200 as mg
 import oracle
 import synth
-from gpu_helpers import layer_parity
+from gpu_helpers import expert_tiles, layer_parity, tile_tokens
 
 pytestmark = pytest.mark.gpu
 
@@ -21,11 +21,30 @@ def _free():
     torch.cuda.empty_cache()
 
 
+def _by_tiles(name, T):
+    """Tokens to compare beyond the random sample, chosen tile by tile from the
+    GPU's dispatch: at decode every token; at prefill and skew every token of
+    the most-loaded expert's last token tile (ragged), the tile before it and a
+    middle one, and of the least-loaded expert's last tile. Every token also
+    exercises the shared experts' tiles it falls in."""
+    def pick(ps, offs, counts):
+        if name == "decode":
+            return range(T)
+        hot = int(np.argmax(counts))
+        cold = int(np.argmin(np.where(counts > 0, counts, 1 << 30)))
+        nt = len(expert_tiles(int(counts[hot])))
+        toks = tile_tokens(ps, offs, hot, sorted({nt - 1, max(nt - 2, 0), nt // 2}))
+        toks += tile_tokens(ps, offs, cold, [len(expert_tiles(int(counts[cold]))) - 1])
+        return toks
+    return pick
+
+
 @pytest.mark.parametrize("name,n_sample", [("decode", 12), ("prefill", 10), ("skew", 10)])
 def test_full_size_layer(name, n_sample):
     cfg = synth.CONFIGS[name]
     inp = synth.layer_inputs(cfg)
-    r = layer_parity(cfg, inp, n_sample=n_sample)
+    r = layer_parity(cfg, inp, n_sample=n_sample, by_tiles=_by_tiles(name, cfg.T))
+    assert len(r["tokens"]) >= (cfg.T - 8 if name == "decode" else 300), len(r["tokens"])
     counts = r["counts"]
     s_moge, loads = oracle.imbalance(r["idx"], cfg.N, cfg.M)
     assert s_moge == 0.0 and np.all(loads == cfg.T * cfg.Kp)

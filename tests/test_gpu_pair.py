@@ -56,3 +56,48 @@ def test_pair_layer_hot_expert():
     bias[:: cfg.N // cfg.M] = 1.5
     inp["logit_bias"] = bias
     layer_parity(cfg, inp, n_sample=600)
+
+
+def test_piecewise_entry_points_at_prefill_size():
+    """moge_grouped_ffn and moge_shared_ffn called on their own at the prefill
+    workload (32768 routed rows, 16384 shared rows: both above 8192, so both
+    run on CTA pairs): sampled rows against the oracle's expert FFN, and the
+    pieces composed with moge_combine against the layer call."""
+    import oracle
+    from gpu_helpers import TOL, device_inputs, normwise_err, to_host_f64, x_double
+    cfg = synth.CONFIGS["prefill"]
+    assert cfg.T * cfg.K >= PAIR_ROWS and cfg.T * cfg.S >= PAIR_ROWS
+    inp = synth.layer_inputs(cfg)
+    x, w = device_inputs(cfg, inp)
+    s = mg.shape_of(cfg)
+    ws = mg.alloc_workspace(s)
+    idx, wt, counts, offsets, ps, pd = mg.moge_route(s, x, w["w_router"], None, ws)
+    xp = mg.moge_permute(s, x, ps)
+    yp = mg.moge_grouped_ffn(s, xp, offsets, w["w_gate"], w["w_up"], w["w_down"], ws)
+    ysh = mg.moge_shared_ffn(s, x, w["s_gate"], w["s_up"], w["s_down"], ws)
+    y = mg.moge_combine(s, yp, wt, pd, y_shared=ysh)
+    y_layer = mg.moge_layer_forward(s, x, w, ws)
+    torch.cuda.synchronize()
+    mg.check_device_errors()
+    xd = x_double(inp, cfg)
+    ps_h, off_h = ps.cpu().numpy(), offsets.cpu().numpy()
+    yp_h = to_host_f64(yp)
+    # rows of every kind of token tile: first and last rows of the experts with
+    # the most and the fewest rows, and random rows
+    cnt = np.diff(off_h)
+    rows = []
+    for e in (int(cnt.argmax()), int(cnt.argmin()), 0, cfg.N - 1):
+        rows += [off_h[e], off_h[e] + cnt[e] // 2, off_h[e + 1] - 1]
+    rows += np.random.default_rng(3).choice(cfg.T * cfg.K, 20, replace=False).tolist()
+    for r in sorted(set(int(v) for v in rows)):
+        e = int(np.searchsorted(off_h, r, side="right") - 1)
+        ref = oracle.expert_ffn(xd[ps_h[r]], inp["w_gate"][e], inp["w_up"][e], inp["w_down"][e],
+                                "bf16")
+        assert normwise_err(yp_h[r], ref) <= TOL["bf16"], (r, e)
+    ysh_h = to_host_f64(ysh)
+    for t in (0, 255, 256, 2047, cfg.T - 1):
+        ref = sum(oracle.expert_ffn(xd[t], inp["s_gate"][k], inp["s_up"][k], inp["s_down"][k],
+                                    "bf16") for k in range(cfg.S))
+        assert normwise_err(ysh_h[t], ref) <= TOL["bf16"], t
+    # the layer call equals the composition of the pieces
+    assert normwise_err(to_host_f64(y_layer), to_host_f64(y)) <= 4e-3

@@ -17,18 +17,29 @@ import mixture_grouped_experts_b200 as mg
 import synth
 
 
-def _case(T, seed):
-    cfg = synth.Config("noalloc", T=T, d=512, N=16, M=4, Kp=1, S=0, I=64, dtype="bf16", seed=seed)
+def _case(T, seed, N=16, M=4):
+    cfg = synth.Config("noalloc", T=T, d=512, N=N, M=M, Kp=1, S=0, I=64, dtype="bf16", seed=seed)
     inp = synth.layer_inputs(cfg)
     return cfg, mg.to_device(inp["x"], "bf16"), mg.to_device(inp["w_router"], "bf16")
 
 
+def _scratch_bytes(T, N, K):
+    """Scratch the call needs: per-tile histograms and row bases, per-pick ranks."""
+    r256 = lambda v: (v + 255) // 256 * 256
+    return 2 * r256(-(-T // 16) * N * 4) + r256(T * K * 4)
+
+
 @pytest.mark.gpu
 def test_noalloc_route_matches_workspace_route_twice():
-    # two calls in a row: a larger batch first, then a smaller one, so that any
-    # read of the previous call's leftovers in the shared array would show
-    for T, seed in ((300, 31), (77, 32)):
-        cfg, x, wr = _case(T, seed)
+    # calls in a row, each larger batch before a smaller one, so that any read of
+    # the previous call's leftovers in the shared array would show: a batch that
+    # fills the 1 MiB array exactly (16384 tokens, 64 experts, 8 picks), one on
+    # the router's 64-token tiles (>= 1024 tokens with <= 64 experts), then two
+    # on its 16-token tiles
+    assert _scratch_bytes(16384, 64, 8) == 1 << 20
+    for T, seed, N, M in ((16384, 33, 64, 8), (1024, 34, 64, 8), (300, 31, 16, 4),
+                          (77, 32, 16, 4)):
+        cfg, x, wr = _case(T, seed, N, M)
         s = mg.shape_of(cfg)
         ws = mg.alloc_workspace(s)
         ref = mg.moge_route(s, x, wr, None, ws)
