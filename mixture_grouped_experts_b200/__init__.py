@@ -345,23 +345,116 @@ def moge_ep_finish(s: LayerShape, y_sum, residual=None, y=None, stream=None):
     return y
 
 
-def moge_layer_forward_ep(s: LayerShape, x_local, w_local: dict, workspace, group=None,
-                          residual=None):
+def ep_chunk_bounds(rows: int, chunks: int):
+    """Row ranges [a, b) of a rank's tokens, one per chunk of the pipelined
+    expert-parallel step (as even as possible; every rank uses the same)."""
+    chunks = max(1, min(int(chunks), rows)) if rows > 0 else 1
+    out, a = [], 0
+    for j in range(chunks):
+        b = a + rows // chunks + (1 if j < rows % chunks else 0)
+        out.append((a, b))
+        a = b
+    return out
+
+
+def ep_default_chunks(rows: int) -> int:
+    """Chunks of the pipelined step for `rows` tokens per rank: one for
+    decode-sized batches (each chunk streams this rank's expert weights again,
+    which only pays once the GEMMs are compute-bound), else about one per 256
+    tokens, at most 4."""
+    return 1 if rows < 512 else min(4, rows // 256)
+
+
+def ep_pipeline(x_local, bounds, gather, local, reduce, finish, comm_stream=None):
+    """The chunk schedule of the expert-parallel step, independent of the
+    device: for every chunk j (rows bounds[j] of this rank's x_local), gather
+    (all ranks' rows of the chunk) -> local (this rank's partial of those
+    tokens) -> reduce (sum over ranks, this rank's rows) -> finish (into the
+    output rows of the chunk). On CUDA, with comm_stream given, every gather is
+    issued at once on comm_stream, chunk j's local step waits only for its own
+    gather, and chunk j's reduce runs on comm_stream while chunk j + 1's local
+    step runs, so the collectives overlap the GEMMs. Returns the finish
+    results in chunk order."""
+    import torch
+    n = len(bounds)
+    if comm_stream is None:
+        outs = []
+        for a, b in bounds:
+            outs.append(finish(a, b, reduce(local(gather(x_local[a:b])))))
+        return outs
+    cur = torch.cuda.current_stream()
+    comm_stream.wait_stream(cur)
+    gathered, ev_g = [], []
+    with torch.cuda.stream(comm_stream):
+        for a, b in bounds:
+            gathered.append(gather(x_local[a:b]))
+            ev_g.append(comm_stream.record_event())
+    reduced, ev_r = [None] * n, [None] * n
+    for j, (a, b) in enumerate(bounds):
+        cur.wait_event(ev_g[j])
+        part = local(gathered[j])
+        comm_stream.wait_stream(cur)
+        with torch.cuda.stream(comm_stream):
+            reduced[j] = reduce(part)
+            ev_r[j] = comm_stream.record_event()
+            part.record_stream(comm_stream)
+        gathered[j].record_stream(cur)
+    outs = []
+    for j, (a, b) in enumerate(bounds):
+        cur.wait_event(ev_r[j])
+        reduced[j].record_stream(cur)
+        outs.append(finish(a, b, reduced[j]))
+    return outs
+
+
+def moge_layer_forward_ep(s: LayerShape, x_local, w_local: dict, workspace=None, group=None,
+                          residual=None, chunks=None, comm_stream=None):
     """One layer step under expert parallelism on the ranks of `group` (each
     with its own x_local [T/world][d]; s is the whole layer's shape, T = all
     ranks' tokens): all-gather x, this rank's partial, reduce-scatter of the
-    partials (NCCL), finish. Returns this rank's y [T/world][d]."""
+    partials (NCCL), finish. Returns this rank's y [T/world][d].
+
+    The step is pipelined over `chunks` token chunks (default
+    ep_default_chunks): the gathers run on a side stream (comm_stream, created
+    when not given) and chunk j's reduce-scatter overlaps chunk j + 1's local
+    GEMMs. workspace: an expert-parallel workspace for the largest chunk
+    (alloc_ep_workspace of that chunk's shape), allocated here when None."""
     import torch.distributed as dist
     world, rank = dist.get_world_size(group), dist.get_rank(group)
     rows = x_local.shape[0]
     if rows * world != s.T:
         raise ValueError("x_local must hold T / world rows")
-    x_all = torch.empty((s.T, s.d), dtype=x_local.dtype, device=x_local.device)
-    dist.all_gather_into_tensor(x_all, x_local, group=group)
-    y_part = moge_layer_forward_ep_local(s, rank, world, x_all, w_local, workspace)
-    y_sum = torch.empty((rows, s.d), dtype=torch.float32, device=x_local.device)
-    dist.reduce_scatter_tensor(y_sum, y_part, group=group)
-    return moge_ep_finish(s, y_sum, residual)
+    bounds = ep_chunk_bounds(rows, ep_default_chunks(rows) if chunks is None else chunks)
+    big = max(b - a for a, b in bounds)
+    if workspace is None:
+        workspace = alloc_ep_workspace(shape_of(s, T=big * world), world, x_local.device)
+    elif workspace.numel() < ep_workspace_size(shape_of(s, T=big * world), world):
+        raise ValueError("workspace smaller than the largest chunk needs")
+    y = torch.empty((rows, s.d), dtype=_TORCH_DT[s.dtype], device=x_local.device)
+
+    def gather(xc):
+        xa = torch.empty((xc.shape[0] * world, s.d), dtype=xc.dtype, device=xc.device)
+        dist.all_gather_into_tensor(xa, xc.contiguous(), group=group)
+        return xa
+
+    def local(xa):
+        return moge_layer_forward_ep_local(shape_of(s, T=xa.shape[0]), rank, world, xa, w_local,
+                                           workspace)
+
+    def reduce(part):
+        out = torch.empty((part.shape[0] // world, s.d), dtype=torch.float32, device=part.device)
+        dist.reduce_scatter_tensor(out, part, group=group)
+        return out
+
+    def finish(a, b, ysum):
+        res = None if residual is None else residual[a:b]
+        return moge_ep_finish(shape_of(s, T=b - a), ysum, res, y[a:b])
+
+    if comm_stream is None and len(bounds) > 1:
+        comm_stream = torch.cuda.Stream(device=x_local.device)
+    ep_pipeline(x_local, bounds, gather, local, reduce, finish,
+                comm_stream if len(bounds) > 1 else None)
+    return y
 
 
 def moge_layer_forward_host(s: LayerShape, x_host, w: dict, workspace, y_host, x_dev, y_dev,

@@ -112,7 +112,10 @@ def test_nccl_driver_world_one():
                             world_size=1)
     try:
         ws = mg.alloc_ep_workspace(s, 1)
-        y = mg.moge_layer_forward_ep(s, xd, mg.ep_shard_weights(w, 0, 1), ws)
+        y = mg.moge_layer_forward_ep(s, xd, mg.ep_shard_weights(w, 0, 1), ws, chunks=1)
+        # the pipelined schedule: 3 uneven token chunks, gathers on a side
+        # stream, each chunk's reduce-scatter overlapping the next chunk's GEMMs
+        yc = mg.moge_layer_forward_ep(s, xd, mg.ep_shard_weights(w, 0, 1), ws, chunks=3)
         torch.cuda.synchronize()
         mg.check_device_errors()
     finally:
@@ -123,6 +126,9 @@ def test_nccl_driver_world_one():
     assert normwise_err(to_host_f64(y)[toks], to_host_f64(y1)[toks]) <= TOL[cfg.dtype]
     y_ref, _, _, _ = oracle.layer(x, inp, cfg.M, cfg.Kp, cfg.dtype, tokens=toks)
     assert normwise_err(to_host_f64(y)[toks], y_ref) <= TOL[cfg.dtype]
+    # a token's result does not depend on the chunk it was computed in (up to
+    # the router's split of the hidden dimension, which follows the batch size)
+    assert normwise_err(to_host_f64(yc)[toks], to_host_f64(y)[toks]) <= 4e-3
 
 
 def test_full_size_decode_eight_ranks_sampled():
