@@ -99,5 +99,8 @@ def test_piecewise_entry_points_at_prefill_size():
         ref = sum(oracle.expert_ffn(xd[t], inp["s_gate"][k], inp["s_up"][k], inp["s_down"][k],
                                     "bf16") for k in range(cfg.S))
         assert normwise_err(ysh_h[t], ref) <= TOL["bf16"], t
-    # the layer call equals the composition of the pieces
-    assert normwise_err(to_host_f64(y_layer), to_host_f64(y)) <= 4e-3
+    # the layer call equals the composition of the pieces up to rounding: the
+    # pieces round the sum of the shared experts to bf16 (y_shared) before the
+    # combine, the layer adds each shared row in fp32 -- one bf16 rounding of
+    # a fraction of y more, within the bf16 tolerance
+    assert normwise_err(to_host_f64(y_layer), to_host_f64(y)) <= TOL["bf16"]
