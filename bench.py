@@ -53,16 +53,20 @@ FFN_PAIR_KERNEL = ("ffn_tc_pair_kernel (the same grouped FFN on CTA pairs, 2-SM 
                    "one persistent launch)")
 
 
-def source_sha16():
-    """Hash of the library's CUDA sources (csrc/*.cu, *.cuh, *.h and the ABI
-    header), the key under which a traffic record is valid."""
+def source_sha16(files=None):
+    """Hash of CUDA sources of the library: the listed files of csrc/ (or all
+    of csrc/*.cu, *.cuh, *.h and the ABI header when None), the key under
+    which a traffic record is valid."""
     import glob
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mixture_grouped_experts_b200", "csrc")
-    files = sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh"))
-                   + glob.glob(os.path.join(csrc, "*.h"))) + [os.path.join(ROOT, "include", "moge.h")]
-    for f in files:
+    if files is None:
+        paths = sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh"))
+                       + glob.glob(os.path.join(csrc, "*.h"))) + [os.path.join(ROOT, "include", "moge.h")]
+    else:
+        paths = [os.path.join(csrc, f) for f in files]
+    for f in paths:
         h.update(os.path.basename(f).encode())
         h.update(open(f, "rb").read())
     return h.hexdigest()[:16]
@@ -70,8 +74,8 @@ def source_sha16():
 
 def traffic_record(kernel, workload):
     """(bytes per launch, source) of the committed ncu record for this kernel
-    and workload when it was taken on the current sources, else (None, why)."""
-    sha = source_sha16()
+    and workload when it was taken on the current sources of that kernel (the
+    record's "files"), else (None, why)."""
     for rel in TRAFFIC_RECORDS:
         path = os.path.join(ROOT, rel)
         if not os.path.exists(path):
@@ -82,6 +86,7 @@ def traffic_record(kernel, workload):
             rec = json.loads(line.split(":", 1)[1])
             if rec.get("kernel") != kernel or rec.get("workload") != workload:
                 continue
+            sha = source_sha16(rec.get("files"))
             if rec.get("src_sha16") != sha:
                 return None, "%s: captured on sources %s, now %s (kernel changed)" % (
                     rel, rec.get("src_sha16"), sha)

@@ -79,6 +79,11 @@ CASES = {
     # (g and u kept by that kernel); I = 192: a half-empty last feature pair
     "pair": synth.Config("bw_pair", T=2048, d=256, N=64, M=8, Kp=1, S=1, I=192, dtype="bf16",
                          seed=65, w_std=0.05),
+    # 12000 routed rows (the training forward on CTA pairs); d = 320: a last
+    # 128-row tile of dx / dW_down half empty; ~375 rows per expert end inside
+    # a K chunk of the weight gradients (ragged rows zeroed); 2 picks per group
+    "pair_ragged": synth.Config("bw_pair_rag", T=1500, d=320, N=32, M=4, Kp=2, S=2, I=192,
+                                dtype="bf16", seed=67, w_std=0.05),
 }
 
 
