@@ -746,12 +746,14 @@ def main():
         tfs = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
         ffn_tf = ffn_flops(pcfg) / (pm["stage_ms"]["ffn"] / 1e3) / 1e12
         lay_tf = layer_flops(pcfg) / (pm["ms"] / 1e3) / 1e12
+        ptraffic, ptsrc = traffic_record("ffn_tc_pair_kernel", pcfg.name)
         line["prefill"] = {
             "workload": workload_config(pcfg)["workload"],
             "value": pcfg.T / (pm["ms"] / 1e3), "unit": "tokens/s", "ms_per_step": pm["ms"],
             "roofline": {"bound": "tensor", "kernel": FFN_PAIR_KERNEL, "achieved": ffn_tf,
                          "peak": tf, "unit": "TFLOP/s", "frac": ffn_tf / tf,
                          "peak_source": "%s bf16_tflops (burst)" % peak_kind,
+                         "traffic": ptraffic, "traffic_source": ptsrc,
                          "nominal": {"peak": NOMINAL["bf16_tflops"], "unit": "TFLOP/s",
                                      "frac": ffn_tf / NOMINAL["bf16_tflops"]}},
             "layer_roofline": {"bound": "tensor", "achieved": lay_tf, "peak": tf, "unit": "TFLOP/s",
