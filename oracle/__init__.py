@@ -75,6 +75,9 @@ def _l():
         lib.oracle_layer_fp8.argtypes = [vp, i32, i32, i32, i32, i32, i32, i32, i32, vp, vp,
                                          vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                          vp, i32, vp, vp, vp, vp]
+        lib.oracle_quantize_act_rows.argtypes = [vp, i64, i64, vp, vp]
+        lib.oracle_expert_ffn_w8a8.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, vp]
+        lib.oracle_layer_w8a8.argtypes = lib.oracle_layer_fp8.argtypes
         lib.oracle_layer_backward.argtypes = [vp, i32, i32, i32, i32, i32, i32, i32, i32,
                                               vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                               ctypes.c_double, vp, vp, i32, vp, vp, vp, vp, vp,
@@ -370,8 +373,42 @@ def expert_ffn_fp8(x_row: np.ndarray, qg, sg, qu, su, qd, sd) -> np.ndarray:
     return y
 
 
+def quantize_act_rows(v: np.ndarray):
+    """Per-row 8-bit activation quantisation (the W8A8 reading): each row of
+    v (any float dtype, [..., cols]) is taken in fp32, then scale = amax / 448
+    in fp32 (1 for an all-zero row) and q = E4M3(fp32(v / scale)).
+    Returns (q uint8 of v's shape, scale float32 of shape v.shape[:-1])."""
+    v = np.ascontiguousarray(v, np.float64)
+    cols = v.shape[-1]
+    rows = v.size // cols
+    q = np.empty(v.shape, np.uint8)
+    sc = np.empty(v.shape[:-1], np.float32)
+    _chk(_l().oracle_quantize_act_rows(_p(v), rows, cols, _p(q), _p(sc)), "quantize_act_rows")
+    return q, sc
+
+
+def expert_ffn_w8a8(x_row: np.ndarray, qg, sg, qu, su, qd, sd) -> np.ndarray:
+    """One SwiGLU expert on one token in W8A8: fp8 weights (qg, qu [I][d]; qd
+    [d][I]) and x, h quantised per token before their products."""
+    x = np.ascontiguousarray(x_row, np.float64)
+    qg, qu, qd = (np.ascontiguousarray(a, np.uint8) for a in (qg, qu, qd))
+    sg, su, sd = (np.ascontiguousarray(a, np.float32) for a in (sg, su, sd))
+    I, d = qg.shape
+    y = np.empty(d, np.float64)
+    _chk(_l().oracle_expert_ffn_w8a8(_p(x), _p(qg), _p(sg), _p(qu), _p(su), _p(qd), _p(sd),
+                                     d, I, _p(y)), "expert_ffn_w8a8")
+    return y
+
+
+def layer_w8a8(x: np.ndarray, inp: dict, q: dict, M: int, Kp: int, dtype: str,
+               tokens: Optional[Sequence[int]] = None):
+    """MoGE layer output in W8A8 (fp8 expert weights q in quantize_experts_fp8
+    form, activations quantised per token); router from inp. Same returns as layer()."""
+    return layer_fp8(x, inp, q, M, Kp, dtype, tokens, _act8=True)
+
+
 def layer_fp8(x: np.ndarray, inp: dict, q: dict, M: int, Kp: int, dtype: str,
-              tokens: Optional[Sequence[int]] = None):
+              tokens: Optional[Sequence[int]] = None, _act8: bool = False):
     """MoGE layer output with fp8 expert weights q (quantize_experts_fp8 form);
     router weights and logit bias from inp. Same returns as layer()."""
     x = np.ascontiguousarray(x, np.float64)
@@ -389,10 +426,10 @@ def layer_fp8(x: np.ndarray, inp: dict, q: dict, M: int, Kp: int, dtype: str,
     idx = np.empty((n, K), np.int32)
     w = np.empty((n, K), np.float64)
     mg = np.empty(n, np.float64)
-    _chk(_l().oracle_layer_fp8(_p(x), T, d, N, M, Kp, S, I, _DT[dtype], _p(wr), _p(b),
-                               _p(a["w_gate"]), _p(a["w_gate_scale"]), _p(a["w_up"]),
-                               _p(a["w_up_scale"]), _p(a["w_down"]), _p(a["w_down_scale"]),
-                               _p(a["s_gate"]), _p(a["s_gate_scale"]), _p(a["s_up"]),
-                               _p(a["s_up_scale"]), _p(a["s_down"]), _p(a["s_down_scale"]),
-                               _p(toks), n, _p(y), _p(idx), _p(w), _p(mg)), "layer_fp8")
+    fn = _l().oracle_layer_w8a8 if _act8 else _l().oracle_layer_fp8
+    _chk(fn(_p(x), T, d, N, M, Kp, S, I, _DT[dtype], _p(wr), _p(b),
+            _p(a["w_gate"]), _p(a["w_gate_scale"]), _p(a["w_up"]), _p(a["w_up_scale"]),
+            _p(a["w_down"]), _p(a["w_down_scale"]), _p(a["s_gate"]), _p(a["s_gate_scale"]),
+            _p(a["s_up"]), _p(a["s_up_scale"]), _p(a["s_down"]), _p(a["s_down_scale"]),
+            _p(toks), n, _p(y), _p(idx), _p(w), _p(mg)), "layer_w8a8" if _act8 else "layer_fp8")
     return y, idx, w, mg

@@ -422,17 +422,93 @@ int oracle_expert_ffn_fp8(const double *x, const uint8_t *qg, const float *sg, c
     return 0;
 }
 
-/* The layer [A][B][D] with fp8 expert weights (routed and shared), router
+/* ---------------------------------------------------------------------------
+ * 8-bit weights and 8-bit activations (W8A8). The same deployment section
+ * reports a W8A8 configuration; the pages fix neither the format nor where
+ * the activations are quantised. Reading taken: the weights as above, and the
+ * input of every expert matrix product quantised per token with the same
+ * rule: the token's row of x (for the gate and up products) and of h (for
+ * the down product), each taken in fp32 first, get
+ *   scale = amax / 448 (fp32 division; 1 for an all-zero row),
+ *   code  = E4M3 round-to-nearest-even, saturating, of fp32(v / scale),
+ * and the product uses decode(code) * scale. The router stays unquantised.
+ */
+
+/* per-row activation quantisation of fp64 rows v [rows][cols] (taken in fp32) */
+int oracle_quantize_act_rows(const double *v, int64_t rows, int64_t cols, uint8_t *q,
+                             float *scale) {
+    for (int64_t r = 0; r < rows; ++r) {
+        const double *vr = v + r * cols;
+        float amax = 0.0f;
+        for (int64_t c = 0; c < cols; ++c) {
+            float a = fabsf((float)vr[c]);
+            if (a > amax) amax = a;
+        }
+        volatile float s = amax > 0.0f ? amax / 448.0f : 1.0f;  /* one fp32 division */
+        scale[r] = s;
+        for (int64_t c = 0; c < cols; ++c) {
+            volatile float f = (float)vr[c];
+            volatile float qv = f / s;
+            q[r * cols + c] = oracle_e4m3_encode(qv);
+        }
+    }
+    return 0;
+}
+
+/* one activation row replaced by its dequantised 8-bit form, in place */
+static void quantize_act_inplace(double *v, int n, uint8_t *codes) {
+    float s;
+    oracle_quantize_act_rows(v, 1, n, codes, &s);
+    for (int j = 0; j < n; ++j) v[j] = oracle_e4m3_decode(codes[j]) * (double)s;
+}
+
+/* One expert on one token in W8A8: as oracle_expert_ffn_fp8, with x
+ * quantised before the gate and up products and h before the down product. */
+int oracle_expert_ffn_w8a8(const double *x, const uint8_t *qg, const float *sg, const uint8_t *qu,
+                           const float *su, const uint8_t *qd, const float *sd, int d, int I,
+                           double *y) {
+    int n = d > I ? d : I;
+    double *w = (double *)malloc(sizeof(double) * (size_t)n);
+    double *xq = (double *)malloc(sizeof(double) * (size_t)d);
+    double *h = (double *)malloc(sizeof(double) * (size_t)I);
+    uint8_t *codes = (uint8_t *)malloc((size_t)n);
+    if (!w || !xq || !h || !codes) { free(w); free(xq); free(h); free(codes); return 2; }
+    memcpy(xq, x, sizeof(double) * (size_t)d);
+    quantize_act_inplace(xq, d, codes);
+    for (int i = 0; i < I; ++i) {
+        load_row_fp8(qg, sg, (size_t)i, d, w);
+        double g = dot(xq, w, d);
+        load_row_fp8(qu, su, (size_t)i, d, w);
+        double u = dot(xq, w, d);
+        h[i] = (g / (1.0 + exp(-g))) * u;
+    }
+    quantize_act_inplace(h, I, codes);
+    for (int o = 0; o < d; ++o) {
+        load_row_fp8(qd, sd, (size_t)o, I, w);
+        y[o] = dot(h, w, I);
+    }
+    free(w);
+    free(xq);
+    free(h);
+    free(codes);
+    return 0;
+}
+
+typedef int (*expert_fn8)(const double *, const uint8_t *, const float *, const uint8_t *,
+                          const float *, const uint8_t *, const float *, int, int, double *);
+
+/* The layer [A][B][D] with 8-bit expert weights (routed and shared), router
  * weights and activations as in oracle_layer (dtype of x / w_router):
- * routed expert e uses qg + e I d, sg + e I, ..., qd + e d I, sd + e d. */
-int oracle_layer_fp8(const double *x, int T, int d, int N, int M, int Kp, int S, int I, int dtype,
-                     const void *w_router, const float *bias,
-                     const uint8_t *qg, const float *sg, const uint8_t *qu, const float *su,
-                     const uint8_t *qd, const float *sd,
-                     const uint8_t *sqg, const float *ssg, const uint8_t *squ, const float *ssu,
-                     const uint8_t *sqd, const float *ssd,
-                     const int32_t *tokens, int n, double *y_out,
-                     int32_t *idx_out, double *w_out, double *margin_out) {
+ * routed expert e uses qg + e I d, sg + e I, ..., qd + e d I, sd + e d;
+ * each expert evaluated by `ffn` (weights-only or W8A8). */
+static int layer_8bit(const double *x, int T, int d, int N, int M, int Kp, int S, int I, int dtype,
+                      const void *w_router, const float *bias,
+                      const uint8_t *qg, const float *sg, const uint8_t *qu, const float *su,
+                      const uint8_t *qd, const float *sd,
+                      const uint8_t *sqg, const float *ssg, const uint8_t *squ, const float *ssu,
+                      const uint8_t *sqd, const float *ssd,
+                      const int32_t *tokens, int n, double *y_out,
+                      int32_t *idx_out, double *w_out, double *margin_out, expert_fn8 ffn) {
     if (N % M != 0 || Kp < 1 || Kp > N / M) return 1;
     int K = M * Kp;
     size_t per = (size_t)I * d;
@@ -452,15 +528,15 @@ int oracle_layer_fp8(const double *x, int T, int d, int N, int M, int Kp, int S,
         for (int o = 0; o < d; ++o) yt[o] = 0.0;
         for (int k = 0; k < K; ++k) {
             size_t e = (size_t)idx[k];
-            rc = oracle_expert_ffn_fp8(xt, qg + e * per, sg + e * I, qu + e * per, su + e * I,
-                                       qd + e * per, sd + e * d, d, I, tmp);
+            rc = ffn(xt, qg + e * per, sg + e * I, qu + e * per, su + e * I, qd + e * per,
+                     sd + e * d, d, I, tmp);
             if (rc) break;
             for (int o = 0; o < d; ++o) yt[o] += w[k] * tmp[o];
         }
         for (int s = 0; s < S && rc == 0; ++s) {
             size_t e = (size_t)s;
-            rc = oracle_expert_ffn_fp8(xt, sqg + e * per, ssg + e * I, squ + e * per, ssu + e * I,
-                                       sqd + e * per, ssd + e * d, d, I, tmp);
+            rc = ffn(xt, sqg + e * per, ssg + e * I, squ + e * per, ssu + e * I, sqd + e * per,
+                     ssd + e * d, d, I, tmp);
             for (int o = 0; o < d; ++o) yt[o] += tmp[o];
         }
         if (idx_out) memcpy(idx_out + (size_t)q * K, idx, sizeof(int32_t) * (size_t)K);
@@ -471,6 +547,33 @@ int oracle_layer_fp8(const double *x, int T, int d, int N, int M, int Kp, int S,
     free(idx);
     free(w);
     return rc;
+}
+
+int oracle_layer_fp8(const double *x, int T, int d, int N, int M, int Kp, int S, int I, int dtype,
+                     const void *w_router, const float *bias,
+                     const uint8_t *qg, const float *sg, const uint8_t *qu, const float *su,
+                     const uint8_t *qd, const float *sd,
+                     const uint8_t *sqg, const float *ssg, const uint8_t *squ, const float *ssu,
+                     const uint8_t *sqd, const float *ssd,
+                     const int32_t *tokens, int n, double *y_out,
+                     int32_t *idx_out, double *w_out, double *margin_out) {
+    return layer_8bit(x, T, d, N, M, Kp, S, I, dtype, w_router, bias, qg, sg, qu, su, qd, sd, sqg,
+                      ssg, squ, ssu, sqd, ssd, tokens, n, y_out, idx_out, w_out, margin_out,
+                      oracle_expert_ffn_fp8);
+}
+
+/* The layer in W8A8 (oracle_expert_ffn_w8a8 per expert), otherwise as oracle_layer_fp8. */
+int oracle_layer_w8a8(const double *x, int T, int d, int N, int M, int Kp, int S, int I, int dtype,
+                      const void *w_router, const float *bias,
+                      const uint8_t *qg, const float *sg, const uint8_t *qu, const float *su,
+                      const uint8_t *qd, const float *sd,
+                      const uint8_t *sqg, const float *ssg, const uint8_t *squ, const float *ssu,
+                      const uint8_t *sqd, const float *ssd,
+                      const int32_t *tokens, int n, double *y_out,
+                      int32_t *idx_out, double *w_out, double *margin_out) {
+    return layer_8bit(x, T, d, N, M, Kp, S, I, dtype, w_router, bias, qg, sg, qu, su, qd, sd, sqg,
+                      ssg, squ, ssu, sqd, ssd, tokens, n, y_out, idx_out, w_out, margin_out,
+                      oracle_expert_ffn_w8a8);
 }
 
 /* One (token, expert) term of the backward pass below, with the expert's

@@ -20,7 +20,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "oracle.c")
 OUT = os.path.join(ROOT, "_build", "oracle_plants")
 PIN_SUITES = ["tests/test_oracle.py", "tests/test_oracle_bwd.py", "tests/test_oracle_fp8.py",
-              "tests/test_oracle_ep.py"]
+              "tests/test_oracle_w8a8.py", "tests/test_oracle_ep.py"]
 
 # name -> [(text in oracle.c, replacement, which occurrence (0-based))]
 PLANTS = {
@@ -67,6 +67,16 @@ PLANTS = {
     "up_from_gate": [("expert_ptr(w_up, dtype, e, per),", "expert_ptr(w_gate, dtype, e, per),", 0)],
     # 8-bit weights: E4M3 exponent bias 8 instead of 7
     "e4m3_bias": [("ldexp(1.0 + m / 8.0, e - 7)", "ldexp(1.0 + m / 8.0, e - 8)", 0)],
+    # W8A8: h left unquantised before the down product
+    "w8a8_h_unquantised": [("    quantize_act_inplace(h, I, codes);\n", "", 0)],
+    # W8A8: x left unquantised before the gate and up products
+    "w8a8_x_unquantised": [("    quantize_act_inplace(xq, d, codes);\n", "", 0)],
+    # W8A8: activation scale amax / 224 (codes saturate)
+    "w8a8_act_scale": [("volatile float s = amax > 0.0f ? amax / 448.0f : 1.0f;",
+                        "volatile float s = amax > 0.0f ? amax / 224.0f : 1.0f;", 1)],
+    # W8A8: the layer's routed experts evaluated without activation quantisation
+    "w8a8_layer_weights_only": [("                      oracle_expert_ffn_w8a8);",
+                                 "                      oracle_expert_ffn_fp8);", 0)],
     # expert-parallel partial: routed outputs not weighted by their scores
     "ep_partial_unweighted": [("            if (rc) break;\n"
                                "            for (int o = 0; o < d; ++o) yt[o] += w[k] * tmp[o];\n"
