@@ -295,28 +295,33 @@ def run_reference(args, cfg):
 
 
 # ----------------------------------------------------------------------------- GPU arm
-def measure(cfg, inp, steps, warmup, dist_on=False, with_e2e=True, fp8=False):
+def measure(cfg, inp, steps, warmup, dist_on=False, with_e2e=True, fp8=False, w8a8=False):
     """Device-timed layer steps (+ per-launch stage times, + end-to-end through
     the host-buffer entry point). Returns a dict of raw measurements. With
-    fp8, the expert weights are quantised on the device once (outside the
-    timed region) and the layer runs moge_layer_forward_fp8."""
+    fp8 or w8a8, the expert weights are quantised on the device once (outside
+    the timed region) and the layer runs moge_layer_forward_fp8 (weights-only
+    8-bit) or moge_layer_forward_w8a8 (activations quantised inside the call)."""
     import torch
     import mixture_grouped_experts_b200 as mg
 
     s = mg.shape_of(cfg)
     x = mg.to_device(inp["x"], cfg.dtype)
     w = mg.weights_to_device(inp, cfg.dtype)
-    ws = mg.alloc_workspace(s)
+    ws = mg.alloc_w8a8_workspace(s) if w8a8 else mg.alloc_workspace(s)
     y = torch.empty_like(x)
-    if fp8:
+    if fp8 or w8a8:
         w8 = mg.experts_to_fp8(w)
         torch.cuda.synchronize()
         for k in mg.FP8_KEYS:          # only the router stays in bf16
             w[k] = None
         torch.cuda.empty_cache()
 
-        def fwd():
-            mg.moge_layer_forward_fp8(s, x, w, w8, ws, y=y)
+        if w8a8:
+            def fwd():
+                mg.moge_layer_forward_w8a8(s, x, w, w8, ws, y=y)
+        else:
+            def fwd():
+                mg.moge_layer_forward_fp8(s, x, w, w8, ws, y=y)
     else:
         def fwd():
             mg.moge_layer_forward(s, x, w, ws, y=y)
@@ -353,7 +358,7 @@ def measure(cfg, inp, steps, warmup, dist_on=False, with_e2e=True, fp8=False):
     mg.check_device_errors()
     out = {"ms": ms, "stage_ms": {k: v / calls for k, v in stage_ms.items()}, "n_used": n_used,
            "counts": counts}
-    if with_e2e and not fp8:
+    if with_e2e and not (fp8 or w8a8):
         # end to end from pinned host memory: every step's x copied in and y
         # copied out inside the timed region. Headline: the streaming call (a
         # run of `steps` batches, copies overlapped with the neighbouring
@@ -384,7 +389,7 @@ def measure(cfg, inp, steps, warmup, dist_on=False, with_e2e=True, fp8=False):
         out["e2e_sync_ms"] = start.elapsed_time(end) / steps
         out["io_bytes"] = xh.numel() * xh.element_size()
     del x, w, ws, y
-    if fp8:
+    if fp8 or w8a8:
         del w8
     torch.cuda.empty_cache()
     return out

@@ -283,6 +283,33 @@ MOGE_API int moge_layer_forward_fp8(const moge_config *cfg, const void *x, const
                                     const moge_fp8_experts *shared, const void *residual, void *y,
                                     void *workspace, void *stream);
 
+/* W8A8: 8-bit weights and 8-bit activations. The same deployment section
+ * reports a W8A8 configuration (weights and activations in 8 bits), again
+ * without a format. This library's reading: the weights as above; the input
+ * of every expert matrix product quantised per token with the weight rule --
+ * a token's bf16 row of x (for the gate and up products) and its row of h,
+ * taken in fp32 (for the down product), each get scale = amax / 448 (fp32
+ * division; 1 for an all-zero row) and codes E4M3(fp32(v / scale)). Both
+ * operands of every expert GEMM are then E4M3 codes, multiplied by the tensor
+ * cores' 8-bit MMA with fp32 accumulation; the fp32 result times the weight
+ * row's scale times the token's scale is the product. The router stays bf16,
+ * y is bf16.
+ *
+ * moge_w8a8_workspace_size: bytes of the workspace moge_layer_forward_w8a8
+ * needs (larger than moge_workspace_size: it also holds the token codes, h in
+ * fp32 and the activation scales); 0 for an invalid config.
+ *
+ * moge_layer_forward_w8a8: the layer with W8A8 experts (routed and shared).
+ * cfg->dtype must be MOGE_BF16; d % 16 == 0 and I % 16 == 0. `shared` may be
+ * NULL when S == 0. x, y, residual, routing and aliasing rules as
+ * moge_layer_forward_fp8; `workspace` (device, caller-owned, 256-byte
+ * aligned) of moge_w8a8_workspace_size bytes. Asynchronous on `stream`. */
+MOGE_API size_t moge_w8a8_workspace_size(const moge_config *cfg);
+MOGE_API int moge_layer_forward_w8a8(const moge_config *cfg, const void *x, const void *w_router,
+                                     const float *logit_bias, const moge_fp8_experts *routed,
+                                     const moge_fp8_experts *shared, const void *residual,
+                                     void *y, void *workspace, void *stream);
+
 
 /* ---------------------------------------------------------------- training
  * Backward pass of the layer (the pages' models are trained, and they name a

@@ -34,7 +34,7 @@ EXPORTS = ["moge_workspace_size", "moge_last_error", "moge_check_device_errors",
            "moge_quantize_fp8_rows", "moge_layer_forward_fp8", "moge_selftest_waits",
            "moge_train_workspace_size", "moge_layer_forward_train", "moge_layer_backward",
            "moge_ep_workspace_size", "moge_layer_forward_ep_local", "moge_ep_finish",
-           "moge_layer_forward_host_stream"]
+           "moge_layer_forward_host_stream", "moge_w8a8_workspace_size", "moge_layer_forward_w8a8"]
 STAGES = ("router", "scan", "permute", "ffn", "combine")
 
 
@@ -110,6 +110,9 @@ def lib() -> ctypes.CDLL:
         L.moge_selftest_waits.argtypes = [ctypes.c_int64, vp, vp]
         fp = ctypes.POINTER(moge_fp8_experts)
         L.moge_layer_forward_fp8.argtypes = [cp, vp, vp, vp, fp, fp, vp, vp, vp, vp]
+        L.moge_layer_forward_w8a8.argtypes = [cp, vp, vp, vp, fp, fp, vp, vp, vp, vp]
+        L.moge_w8a8_workspace_size.argtypes = [cp]
+        L.moge_w8a8_workspace_size.restype = ctypes.c_size_t
         L.moge_train_workspace_size.argtypes = [cp]
         L.moge_train_workspace_size.restype = ctypes.c_size_t
         L.moge_layer_forward_train.argtypes = [cp] + [vp] * 12
@@ -121,7 +124,7 @@ def lib() -> ctypes.CDLL:
         L.moge_layer_forward_host_stream.argtypes = [cp, ctypes.c_int64] + [vp] * 14
         for n in EXPORTS:
             if n not in ("moge_workspace_size", "moge_last_error", "moge_train_workspace_size",
-                         "moge_ep_workspace_size"):
+                         "moge_ep_workspace_size", "moge_w8a8_workspace_size"):
                 getattr(L, n).restype = i32
         _lib = L
     return _lib
@@ -586,6 +589,33 @@ def moge_layer_forward_fp8(s: LayerShape, x, w: dict, w8: dict, workspace, resid
                                       ctypes.byref(routed) if routed is not None else None,
                                       ctypes.byref(shared) if shared is not None else None,
                                       _p(residual), _p(y), _p(workspace), _stream(stream)))
+    return y
+
+
+def w8a8_workspace_size(s: LayerShape) -> int:
+    n = lib().moge_w8a8_workspace_size(ctypes.byref(_cfg(s)))
+    if n == 0:
+        raise MogeError(ERR_INVALID_ARG, "invalid layer config %r" % (s,))
+    return n
+
+
+def alloc_w8a8_workspace(s: LayerShape, device=None) -> torch.Tensor:
+    return torch.empty(w8a8_workspace_size(s), dtype=torch.uint8, device=device or "cuda")
+
+
+def moge_layer_forward_w8a8(s: LayerShape, x, w: dict, w8: dict, workspace, residual=None,
+                            y=None, stream=None):
+    """Layer in W8A8: FP8 expert weights w8 (experts_to_fp8 form) and
+    activations quantised per token inside the call; w gives w_router and
+    logit_bias; workspace of w8a8_workspace_size bytes."""
+    if y is None:
+        y = torch.empty((s.T, s.d), dtype=x.dtype, device=x.device)
+    routed, shared = _fp8_side(w8, "w"), _fp8_side(w8, "s")
+    _chk(lib().moge_layer_forward_w8a8(ctypes.byref(_cfg(s)), _p(x), _p(w["w_router"]),
+                                       _p(w.get("logit_bias")),
+                                       ctypes.byref(routed) if routed is not None else None,
+                                       ctypes.byref(shared) if shared is not None else None,
+                                       _p(residual), _p(y), _p(workspace), _stream(stream)))
     return y
 
 

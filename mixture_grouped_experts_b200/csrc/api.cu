@@ -186,9 +186,47 @@ constexpr long long kFusedPermuteRows = 8192;
 // 1-SM kernel and its fused permute.
 constexpr long long kPairRows = kFusedPermuteRows + 1;
 
+// W8A8 workspace: the forward workspace (its x_perm region holds the routed
+// rows' codes, its h region the h codes), then the tokens' codes, the two
+// activation scale arrays, h in fp32 and its row amax words and scales.
+struct W8Space {
+    Workspace fw;
+    void *x8;        // [T][d] E4M3 codes
+    float *sx;       // [T]
+    float *sxp;      // [T*K]
+    float *h32;      // [T(K+S)][I]
+    uint32_t *hmax;  // [T(K+S)]
+    float *sh;       // [T(K+S)]
+    size_t total;
+};
+static W8Space carve_w8a8(const moge_config &c, void *base) {
+    W8Space s;
+    s.fw = carve_workspace(c, base);
+    const size_t K = (size_t)c.M * c.Kp, T = (size_t)c.T, hrows = T * (K + c.S);
+    char *p = static_cast<char *>(base);
+    size_t off = s.fw.total;
+    auto take = [&](size_t bytes) {
+        char *r = p ? p + off : nullptr;
+        off += align256(bytes > 0 ? bytes : 1);
+        return r;
+    };
+    s.x8 = take(T * c.d);
+    s.sx = (float *)take(T * 4);
+    s.sxp = (float *)take(T * K * 4);
+    s.h32 = (float *)take(hrows * c.I * 4);
+    s.hmax = (uint32_t *)take(hrows * 4);
+    s.sh = (float *)take(hrows * 4);
+    s.total = off;
+    return s;
+}
+
+// The layer's expert arithmetic: bf16 (or fp32), 8-bit weights, or W8A8.
+enum LayerMode { kModeDense = 0, kModeFp8Weights = 1, kModeW8A8 = 2 };
+
 static int layer_run(const moge_config &c, const void *x, const void *w_router,
-                     const float *logit_bias, FfnOperands op, bool fp8, const void *residual,
+                     const float *logit_bias, FfnOperands op, LayerMode mode, const void *residual,
                      void *y, void *workspace, cudaStream_t st) {
+    const bool fp8 = mode == kModeFp8Weights, w8a8 = mode == kModeW8A8;
     Workspace ws = carve_workspace(c, workspace);
     const int K = c.M * c.Kp;
     cudaEvent_t *ev = timer_slot();
@@ -203,9 +241,21 @@ static int layer_run(const moge_config &c, const void *x, const void *w_router,
     // (its epilogue warps copy the rows while the first, shared-expert items
     // run); larger batches (the copy would hold the epilogue warps long enough to
     // stall the first items), fp8 and fp32: a launch of its own
-    const bool fuse_permute = c.dtype == MOGE_BF16 && !fp8 &&
+    const bool fuse_permute = c.dtype == MOGE_BF16 && mode == kModeDense &&
                               (long long)c.T * c.M * c.Kp <= kFusedPermuteRows;
-    if (fuse_permute) {
+    op.b1 = x;
+    if (w8a8) {  // the tokens quantised, their codes permuted
+        W8Space w8 = carve_w8a8(c, workspace);
+        MOGE_CU(launch_quantize_scatter(c, x, ws.topk_idx, ws.rank, ws.base, ws.offsets,
+                                        ws.perm_src, ws.perm_dst, w8.x8, w8.sx, ws.x_perm, w8.sxp,
+                                        w8.hmax, st), "quantise + permute launch");
+        op.b1 = w8.x8;
+        op.cs_b0 = w8.sxp;
+        op.cs_b1 = w8.sx;
+        op.h32 = w8.h32;
+        op.hmax = w8.hmax;
+        op.sh = w8.sh;
+    } else if (fuse_permute) {
         op.pm_topk_idx = ws.topk_idx; op.pm_rank = ws.rank; op.pm_base = ws.base;
         op.pm_offsets = ws.offsets; op.pm_perm_src = ws.perm_src; op.pm_perm_dst = ws.perm_dst;
     } else {
@@ -215,7 +265,6 @@ static int layer_run(const moge_config &c, const void *x, const void *w_router,
     if (ev) MOGE_CU(cudaEventRecord(ev[3], st), "event");
     const int64_t rrows = (int64_t)c.T * K;
     op.b0 = ws.x_perm;
-    op.b1 = x;
     op.b0_rows = rrows;
     op.b1_rows = c.T;
     op.h = ws.h;
@@ -223,6 +272,9 @@ static int layer_run(const moge_config &c, const void *x, const void *w_router,
     op.y = ws.y_perm;
     if (fp8) {
         MOGE_CU(launch_ffn_fp8(c, ws.plan, c.N + c.S, op, num_sms(), st), "grouped FFN (fp8) launch");
+    } else if (w8a8) {
+        MOGE_CU(launch_ffn_w8a8(c, ws.plan, c.N + c.S, op, num_sms(), st),
+                "grouped FFN (W8A8) launch");
     } else {
         if (c.dtype == MOGE_BF16 && !fuse_permute && rrows >= kPairRows) {
             MOGE_CU(pair::launch_ffn_tc_pair(c, ws.plan, c.N + c.S, op, num_sms(), st),
@@ -548,7 +600,7 @@ int moge_layer_forward(const moge_config *cfg, const void *x, const void *w_rout
     FfnOperands wts{};
     wts.wg = w_gate; wts.wu = w_up; wts.wd = w_down;
     if (c.S > 0) { wts.sg = s_gate; wts.su = s_up; wts.sd = s_down; }
-    return layer_run(c, x, w_router, logit_bias, wts, false, residual, y, workspace,
+    return layer_run(c, x, w_router, logit_bias, wts, kModeDense, residual, y, workspace,
                      (cudaStream_t)stream);
 }
 
@@ -710,7 +762,43 @@ int moge_layer_forward_fp8(const moge_config *cfg, const void *x, const void *w_
         op.sg = shared->gate; op.su = shared->up; op.sd = shared->down;
         op.sg_s = shared->gate_scale; op.su_s = shared->up_scale; op.sd_s = shared->down_scale;
     }
-    return layer_run(c, x, w_router, logit_bias, op, true, residual, y, workspace,
+    return layer_run(c, x, w_router, logit_bias, op, kModeFp8Weights, residual, y, workspace,
+                     (cudaStream_t)stream);
+}
+
+size_t moge_w8a8_workspace_size(const moge_config *cfg) {
+    if (check_config(cfg) != MOGE_OK) return 0;
+    return carve_w8a8(*cfg, nullptr).total;
+}
+
+int moge_layer_forward_w8a8(const moge_config *cfg, const void *x, const void *w_router,
+                            const float *logit_bias, const moge_fp8_experts *routed,
+                            const moge_fp8_experts *shared, const void *residual, void *y,
+                            void *workspace, void *stream) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    const moge_config c = *cfg;
+    if (c.dtype != MOGE_BF16) return fail(MOGE_ERR_UNSUPPORTED, "W8A8 needs dtype MOGE_BF16");
+    if (c.d % 16 != 0 || c.I % 16 != 0)
+        return fail(MOGE_ERR_UNSUPPORTED, "W8A8 needs d % 16 == 0 and I % 16 == 0");
+    if (c.T == 0) return MOGE_OK;
+    MOGE_NEED(x, "x");
+    MOGE_NEED(w_router, "w_router");
+    if ((rc = check_fp8_side(routed, "routed"))) return rc;
+    if (c.S > 0 && (rc = check_fp8_side(shared, "shared"))) return rc;
+    if (logit_bias && !aligned4(logit_bias)) return fail(MOGE_ERR_UNSUPPORTED, "logit_bias misaligned");
+    if (residual && !aligned16(residual)) return fail(MOGE_ERR_UNSUPPORTED, "residual misaligned");
+    MOGE_NEED(y, "y");
+    MOGE_NEED(workspace, "workspace");
+    if (y == x) return fail(MOGE_ERR_INVALID_ARG, "y must not alias x");
+    FfnOperands op{};
+    op.wg = routed->gate; op.wu = routed->up; op.wd = routed->down;
+    op.wg_s = routed->gate_scale; op.wu_s = routed->up_scale; op.wd_s = routed->down_scale;
+    if (c.S > 0) {
+        op.sg = shared->gate; op.su = shared->up; op.sd = shared->down;
+        op.sg_s = shared->gate_scale; op.su_s = shared->up_scale; op.sd_s = shared->down_scale;
+    }
+    return layer_run(c, x, w_router, logit_bias, op, kModeW8A8, residual, y, workspace,
                      (cudaStream_t)stream);
 }
 
@@ -768,7 +856,7 @@ int moge_layer_forward_train(const moge_config *cfg, const void *x, const void *
     wts.wg = w_gate; wts.wu = w_up; wts.wd = w_down;
     if (c.S > 0) { wts.sg = s_gate; wts.su = s_up; wts.sd = s_down; }
     wts.gu = ts.gu;
-    return layer_run(c, x, w_router, logit_bias, wts, false, nullptr, y, workspace,
+    return layer_run(c, x, w_router, logit_bias, wts, kModeDense, nullptr, y, workspace,
                      (cudaStream_t)stream);
 }
 

@@ -326,6 +326,21 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t m, uint32_t n) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((n >> 3) << 17) | ((m >> 4) << 24);
 }
+// Instruction descriptor of kind::f8f6f4 with A and B both E4M3 (format code 0
+// in bits 7-9 and 10-12), fp32 accumulator, both K-major.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(uint32_t m, uint32_t n) {
+    return (1u << 4) | ((n >> 3) << 17) | ((m >> 4) << 24);
+}
+// D (tmem) (+)= A (smem desc) * B (smem desc), 8-bit operands: one instruction
+// covers 32 bytes (32 elements) of K per row, as kind::f16 covers 16 bf16.
+__device__ __forceinline__ void tc_mma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
 
 // Programmatic dependent launch: a kernel launched with programmatic stream
 // serialisation may start while its predecessor finishes; it must pass this
@@ -362,11 +377,12 @@ static inline EncodeTiledFn get_encode_fn() {
 }
 
 static inline bool encode(CUtensorMap *m, const void *base, cuuint32_t rank, const cuuint64_t *dims,
-                   const cuuint64_t *strides, const cuuint32_t *box) {
+                   const cuuint64_t *strides, const cuuint32_t *box,
+                   CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
     EncodeTiledFn fn = get_encode_fn();
     if (!fn) return false;
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), dims, strides,
+    return fn(m, dt, rank, const_cast<void *>(base), dims, strides,
               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }

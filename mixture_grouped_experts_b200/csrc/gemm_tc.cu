@@ -13,7 +13,7 @@
 //                           16-byte global stores, rows masked per expert)
 //
 // The queue hands out every up-projection item before any down-projection
-// item, shared experts first (the heaviest items go first, the tail is made
+// item (W8: with the quantisation items between them), shared experts first (the heaviest items go first, the tail is made
 // of small ones). A down-projection item of an expert waits -- bounded -- until
 // all up-projection items of that expert have stored their h rows (a per-
 // expert counter), so no kernel boundary separates the two phases. Every item
@@ -34,10 +34,26 @@
 // and lanes 64-127 hold up for the same 64 features; the epilogue pairs them
 // through shared memory. No repacking of the [E][I][d] weights is needed.
 //
+// W8A8 (the kernel's W8 instantiation): weights and activations are E4M3
+// codes, and the MMA is kind::f8f6f4. A K-chunk is still 128 bytes per row (128
+// codes), so the stages, boxes and descriptors keep their byte geometry. The
+// scales are applied in the epilogue: the weight row's scale per accumulator
+// lane and the token's scale per column. Each row of h needs its own scale,
+// which depends on all of the row's I features, so the up-projection items
+// store h in fp32 and fold each row's amax into a global word. The queue then
+// hands out quantisation items between the two projections: kQParts row
+// slices per token tile, each run by a CTA's epilogue warps once the expert's
+// up items are all done, each counting once more on the expert's counter. The
+// expert's down-projection items wait for those counts too. (Quantising a whole
+// expert in the CTA that finished its last up item chained: that CTA's delayed
+// items made it the last finisher of the next expert, and so on.)
+//
 // The grouped expert GEMM ("GroupMatmul") of the Pangu Pro MoE article
 // (techwalker.com, section 3) and its SwiftGMM GEMV/GEMM switch (reportify.cn
 // product digest) are prior art for Ascend; this is a B200 design of the
 // same operation.
+#include <cuda_fp8.h>
+
 #include "common.cuh"
 #include "moge_internal.h"
 
@@ -48,6 +64,8 @@ constexpr int kStageBytes = 48 * 1024;
 constexpr int kEpiBytes = 16 * 1024;  // U fp32 [32][64], H and G bf16 [32][64]
 constexpr int kTcThreads = 192;
 constexpr int kChunkK = 64;          // bf16 elements per K-chunk (128 bytes, one swizzle row)
+constexpr int kChunkK8 = 128;        // E4M3 elements per K-chunk (the same 128 bytes)
+constexpr int kKSteps = 4;           // MMAs per K-chunk: 32 bytes of K each
 constexpr int kBoxRows = 64;         // token rows per TMA box (one 8 KB copy per chunk)
 constexpr uint32_t kTmemCols = 512;  // two accumulators of 256 columns
 constexpr int kSlots = 8;            // depth of the work-item ring
@@ -76,23 +94,45 @@ struct TcParams {
     int pm_T, pm_N, pm_K;
 };
 
+// The W8A8 instantiation's extra operands (unused by the bf16 one).
+struct W8Params {
+    const float *sc_g[2], *sc_u[2], *sc_d[2];  // weight row scales, per a_sel
+    const float *cs_b0, *cs_b1;  // token scales of the up-projection's B rows (b_sel 0 / 1)
+    float *h32;                  // [rows][I] h in fp32, before quantisation
+    uint32_t *hmax;              // [rows] amax of each h row (fp32 bits; zeroed beforehand)
+    float *sh;                   // [rows] scale of each row of h codes
+    uint8_t *h8;                 // [rows][I] h codes: the down-projection's B
+};
+
 struct TcItem {
     ExpertWork w;
     int entry, fb, tb, n_valid;
     bool up, stream;
+    bool quant;  // W8: quantise part fb of token tile tb's h rows (no GEMM)
 };
 
-// Decode global item q: the up-projection items first, then the down-projection ones.
-__device__ __forceinline__ void decode_item(const TcParams &p, int tot_up, int q, TcItem &it) {
+// W8: every token tile's h rows are quantised by kQParts work items (row
+// slices of the tile), spread over the grid.
+constexpr int kQParts = 4;
+
+// Decode global item q: the up-projection items first, then (W8: tot_q > 0)
+// the quantisation items, kQParts per token tile in entry order, then the
+// down-projection items.
+__device__ __forceinline__ void decode_item(const TcParams &p, int tot_up, int tot_q, int q,
+                                            TcItem &it) {
     it.up = q < tot_up;
-    const int local = it.up ? q : q - tot_up;
-    const int *start = it.up ? p.plan.up_start : p.plan.down_start;
+    it.quant = !it.up && q < tot_up + tot_q;
+    const int fb_up = (p.I + 63) / 64;
+    // a quantisation item is looked up as the first up item of its tile
+    const int local = it.up ? q : it.quant ? ((q - tot_up) / kQParts) * fb_up : q - tot_up - tot_q;
+    const int *start = (it.up || it.quant) ? p.plan.up_start : p.plan.down_start;
     int lo = 0, hi = p.n_entries - 1;
     while (lo < hi) {  // last entry whose first item is <= local (entries may be empty)
         const int mid = (lo + hi + 1) >> 1;
         if (__ldg(start + mid) <= local) lo = mid; else hi = mid - 1;
     }
-    const int *wp = reinterpret_cast<const int *>((it.up ? p.plan.up : p.plan.down) + lo);
+    const int *wp =
+        reinterpret_cast<const int *>(((it.up || it.quant) ? p.plan.up : p.plan.down) + lo);
     it.w.rows = __ldg(wp + 0);
     it.w.src_row0 = __ldg(wp + 1);
     it.w.dst_row0 = __ldg(wp + 2);
@@ -103,8 +143,13 @@ __device__ __forceinline__ void decode_item(const TcParams &p, int tot_up, int q
     it.w.ntb = __ldg(wp + 7);
     it.entry = lo;
     const int r = local - __ldg(start + lo);
-    it.fb = r / it.w.ntb;  // feature block major, token tile fastest
-    it.tb = r % it.w.ntb;
+    if (it.quant) {
+        it.fb = (q - tot_up) % kQParts;
+        it.tb = r / fb_up;
+    } else {
+        it.fb = r / it.w.ntb;  // feature block major, token tile fastest
+        it.tb = r % it.w.ntb;
+    }
     it.n_valid = min(it.w.bn, it.w.rows - it.tb * it.w.bn);
     it.stream = it.w.rows <= kStreamRows;
 }
@@ -127,7 +172,45 @@ struct TcShared {
     int abort;
     int epi_item;
     int pm_rows[kMaxExperts];  // the fused permute: destination rows of the current token
+    float cs[32];              // W8: token scales of the columns being stored
 };
+
+// E4M3 codes of four fp32 values divided by s (IEEE fp32 division, then round
+// to nearest even, saturating), packed low byte first.
+__device__ __forceinline__ uint32_t e4m3x4_div(float4 f, float s) {
+    const uint32_t b0 = __nv_cvt_float_to_fp8(__fdiv_rn(f.x, s), __NV_SATFINITE, __NV_E4M3);
+    const uint32_t b1 = __nv_cvt_float_to_fp8(__fdiv_rn(f.y, s), __NV_SATFINITE, __NV_E4M3);
+    const uint32_t b2 = __nv_cvt_float_to_fp8(__fdiv_rn(f.z, s), __NV_SATFINITE, __NV_E4M3);
+    const uint32_t b3 = __nv_cvt_float_to_fp8(__fdiv_rn(f.w, s), __NV_SATFINITE, __NV_E4M3);
+    return b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+}
+
+// W8: quantise rows [r0, r0 + rows) of h (fp32 [.][I], I % 16 == 0) per row:
+// scale = amax / 448 (IEEE fp32 division; 1 for an all-zero row), code = E4M3
+// of fp32(h / scale). Called by the 128 epilogue threads (et), one warp per
+// row, four 16-byte loads in flight per lane. h and the amax words were
+// written by other CTAs: read through L2 only.
+__device__ void quantize_h_rows(const W8Params &w8, int I, int r0, int rows, int et) {
+    const int w = et >> 5, lane = et & 31;
+    const int nv = I / 4;
+    for (int r = w; r < rows; r += 4) {
+        const size_t row = (size_t)r0 + r;
+        const float amax = __uint_as_float(__ldcg(w8.hmax + row));
+        const float sc = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+        if (lane == 0) w8.sh[row] = sc;
+        const float4 *src = reinterpret_cast<const float4 *>(w8.h32 + row * I);
+        uint32_t *dst = reinterpret_cast<uint32_t *>(w8.h8 + row * I);
+        for (int v0 = lane; v0 < nv; v0 += 128) {
+            float4 f[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (v0 + 32 * u < nv) f[u] = __ldcg(src + v0 + 32 * u);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (v0 + 32 * u < nv) dst[v0 + 32 * u] = e4m3x4_div(f[u], sc);
+        }
+    }
+}
 
 // smem byte offsets of chunk c of a stage
 __device__ __forceinline__ uint32_t a_off(bool stream, int c) { return stream ? c * 24576u : 0u; }
@@ -165,8 +248,10 @@ __device__ bool wait_counter(const int *ctr, int need, volatile int *abort,
     }
 }
 
+template <bool W8>
 __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
-    const __grid_constant__ TcParams p, const __grid_constant__ CUtensorMap tmWg,
+    const __grid_constant__ TcParams p, const __grid_constant__ W8Params w8,
+    const __grid_constant__ CUtensorMap tmWg,
     const __grid_constant__ CUtensorMap tmWu, const __grid_constant__ CUtensorMap tmSg,
     const __grid_constant__ CUtensorMap tmSu, const __grid_constant__ CUtensorMap tmX0,
     const __grid_constant__ CUtensorMap tmX1, const __grid_constant__ CUtensorMap tmWd,
@@ -220,8 +305,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
     // everything above overlapped the previous kernel; its results are needed from here on
     grid_dependency_wait();
     const int tot_up = __ldg(p.plan.up_start + p.n_entries);
-    const int total = tot_up + __ldg(p.plan.down_start + p.n_entries);
     const int fb_up = (p.I + 63) / 64;
+    // W8: kQParts quantisation items per token tile (every entry's up items
+    // are its tiles x fb_up)
+    const int tot_q = W8 ? kQParts * (tot_up / fb_up) : 0;
+    const int total = tot_up + tot_q + __ldg(p.plan.down_start + p.n_entries);
+    constexpr int kCE = W8 ? kChunkK8 : kChunkK;  // elements per K-chunk
 
     if (warp == 0) {
         // ------------------------------------------------------ scheduler + producer
@@ -251,10 +340,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
             q = __shfl_sync(0xffffffffu, q, 0);
             if (q < 0 || q >= total) break;
             TcItem it;
-            decode_item(p, tot_up, q, it);
-            if (!it.up) {  // the h rows of this expert must all be stored
+            decode_item(p, tot_up, tot_q, q, it);
+            if (it.quant) continue;  // no operands: the epilogue warps do it
+            if (!it.up) {  // the h rows of this expert must all be stored (W8: and quantised)
                 int ok = 1;
-                if (lane == 0) ok = wait_counter(p.sync + 1 + it.entry, it.w.ntb * fb_up, abort);
+                if (lane == 0)
+                    ok = wait_counter(p.sync + 1 + it.entry,
+                                      it.w.ntb * (fb_up + (W8 ? kQParts : 0)), abort);
                 if (!__shfl_sync(0xffffffffu, ok, 0)) break;
                 fence_proxy_async_global();
             } else if (it.w.b_sel == 0 && !permuted) {  // routed rows: every CTA's permute share
@@ -298,7 +390,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
                 }
                 __syncwarp();
                 if (my_c < nch) {
-                    const int k = chunk_at(kc + my_c, it.fb, kcs) * kChunkK;
+                    const int k = chunk_at(kc + my_c, it.fb, kcs) * kCE;
                     unsigned char *sa = sbase + a_off(it.stream, my_c);
                     unsigned char *sb = sbase + b_off(it.stream, my_c);
                     if (my_r >= na) {
@@ -327,6 +419,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
+            int g = 0;  // GEMM items so far: the accumulators alternate over these
             for (int s = 0;; ++s) {
                 const int slot = s % kSlots;
                 if (!mbar_wait(&sh.slot_full[slot], (uint32_t)(s / kSlots) & 1u, abort)) break;
@@ -334,13 +427,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
                 mbar_arrive(&sh.slot_empty[slot]);
                 if (q >= total) break;
                 TcItem it;
-                decode_item(p, tot_up, q, it);
-                const int acc = s & 1;
-                const uint32_t use = (uint32_t)(s >> 1);
+                decode_item(p, tot_up, tot_q, q, it);
+                if (it.quant) continue;
+                const int acc = g & 1;
+                const uint32_t use = (uint32_t)(g >> 1);
+                ++g;
                 if (!mbar_wait(&sh.tempty[acc], (use & 1u) ^ 1u, abort)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)acc * 256u;
-                const uint32_t idesc = idesc_bf16_f32(128, (uint32_t)it.w.bn);
+                const uint32_t idesc = W8 ? idesc_e4m3_f32(128, (uint32_t)it.w.bn)
+                                          : idesc_bf16_f32(128, (uint32_t)it.w.bn);
                 const int kcs = it.up ? p.kc_up : p.kc_down;
                 const int per = it.stream ? 2 : 1;
                 bool ok = true;
@@ -353,10 +449,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
                         const uint32_t sa = sbase + a_off(it.stream, c);
                         const uint32_t sb = sbase + b_off(it.stream, c);
 #pragma unroll
-                        for (int j = 0; j < kChunkK / 16; ++j)  // 16-wide K steps: +32 bytes
-                            tc_mma_bf16(d_tmem, smem_desc_sw128(sa + 32u * j),
-                                        smem_desc_sw128(sb + 32u * j), idesc,
-                                        (kc + c + j) > 0 ? 1u : 0u);
+                        for (int j = 0; j < kKSteps; ++j) {  // K steps of 32 bytes
+                            const uint64_t da = smem_desc_sw128(sa + 32u * j);
+                            const uint64_t db = smem_desc_sw128(sb + 32u * j);
+                            if constexpr (W8)
+                                tc_mma_f8(d_tmem, da, db, idesc, (kc + c + j) > 0 ? 1u : 0u);
+                            else
+                                tc_mma_bf16(d_tmem, da, db, idesc, (kc + c + j) > 0 ? 1u : 0u);
+                        }
                     }
                     tc_commit(&sh.empty[stage]);  // frees the stage once these MMAs have read it
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -408,17 +508,25 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
             named_bar_sync(1, 128);
             if (et == 0) atomicAdd(p.sync + 1 + p.n_entries, 1);
         }
+        int g = 0;  // GEMM items so far (as the MMA issuer counts them)
         for (int s = 0;; ++s) {
-            // the leader takes the next item and waits for its accumulator;
-            // all 128 threads then act on the same decision
+            // the leader takes the next item and waits for its accumulator (a
+            // quantisation item: for the up items of its expert); all 128
+            // threads then act on the same decision
             if (et == 0) {
                 const int slot = s % kSlots;
                 int q = -1;
                 if (mbar_wait(&sh.slot_full[slot], (uint32_t)(s / kSlots) & 1u, abort)) {
                     q = sh.slot_item[slot];
                     mbar_arrive(&sh.slot_empty[slot]);
-                    if (q < total && !mbar_wait(&sh.tfull[s & 1], (uint32_t)(s >> 1) & 1u, abort))
-                        q = -1;
+                    if (q < total) {
+                        TcItem lt;
+                        decode_item(p, tot_up, tot_q, q, lt);
+                        const bool ok =
+                            lt.quant ? wait_counter(p.sync + 1 + lt.entry, lt.w.ntb * fb_up, abort)
+                                     : mbar_wait(&sh.tfull[g & 1], (uint32_t)(g >> 1) & 1u, abort);
+                        if (!ok) q = -1;
+                    }
                 }
                 sh.epi_item = q;
             }
@@ -426,16 +534,113 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
             const int q = *(volatile int *)&sh.epi_item;
             named_bar_sync(1, 128);
             if (q < 0 || q >= total) break;
-            tc_fence_after();
             TcItem it;
-            decode_item(p, tot_up, q, it);
-            const int acc = s & 1;
+            decode_item(p, tot_up, tot_q, q, it);
+            if constexpr (W8) {
+                if (it.quant) {
+                    // rows [lo, hi) of the tile's n_valid rows, then one count for
+                    // the expert's down-projection items
+                    const int per = (it.n_valid + kQParts - 1) / kQParts;
+                    const int lo = min(it.n_valid, it.fb * per), hi = min(it.n_valid, lo + per);
+                    quantize_h_rows(w8, p.I, it.w.dst_row0 + it.tb * it.w.bn + lo, hi - lo, et);
+                    fence_proxy_async_global();
+                    __threadfence();
+                    named_bar_sync(1, 128);
+                    if (et == 0) atomicAdd(p.sync + 1 + it.entry, 1);
+                    continue;
+                }
+            }
+            tc_fence_after();
+            const int acc = g & 1;
+            ++g;
             const uint32_t tbase = tmem_base + ((uint32_t)(32 * q4) << 16) + (uint32_t)acc * 256u;
             const size_t row0 = (size_t)it.w.dst_row0 + (size_t)it.tb * it.w.bn;
+            // W8: the scale of this thread's accumulator row (its weight row)
+            // and the token scales of the item's B rows
+            float rs = 1.0f;
+            const float *cs = nullptr;
+            if constexpr (W8) {
+                const int m = q4 * 32 + lane;
+                if (it.up) {
+                    const bool gate_hi = p.gu_mode[it.w.a_sel] == kUpGateFused;
+                    const bool is_gate = (q4 < 2) != gate_hi;
+                    const int f = it.fb * 64 + (m & 63);
+                    const float *sc = is_gate ? w8.sc_g[it.w.a_sel] : w8.sc_u[it.w.a_sel];
+                    rs = f < p.I ? __ldg(sc + (size_t)it.w.a_idx * p.I + f) : 0.0f;
+                    cs = it.w.b_sel ? w8.cs_b1 : w8.cs_b0;
+                } else {
+                    const int f = it.fb * 128 + m;
+                    rs = f < p.d ? __ldg(w8.sc_d[it.w.a_sel] + (size_t)it.w.a_idx * p.d + f) : 0.0f;
+                    cs = w8.sh;
+                }
+                cs += (size_t)it.w.src_row0 + (size_t)it.tb * it.w.bn;
+            }
             for (int c0 = 0; c0 < it.n_valid; c0 += 32) {
                 uint32_t v[32];
                 tmem_ld_32x32b_x32(tbase + (uint32_t)c0, v);
+                if constexpr (W8) {  // h scales were written in this launch: through L2
+                    if (et < 32) sh.cs[et] = c0 + et < it.n_valid ? __ldcg(cs + c0 + et) : 0.0f;
+                    named_bar_sync(1, 128);
+                }
                 tmem_ld_wait();
+                if constexpr (W8) {
+                    if (it.up) {
+                        float *U = reinterpret_cast<float *>(epi);           // [32 cols][64 features]
+                        float *H = reinterpret_cast<float *>(epi + 8192);    // [32 cols][64 features]
+                        const bool gate_hi = p.gu_mode[it.w.a_sel] == kUpGateFused;
+                        const bool is_gate = (q4 < 2) != gate_hi;
+                        const int f = (q4 & 1) * 32 + lane;
+                        if (!is_gate) {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                U[j * 64 + f] = __uint_as_float(v[j]) * rs * sh.cs[j];
+                        }
+                        named_bar_sync(1, 128);
+                        if (is_gate) {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) {
+                                const float g = __uint_as_float(v[j]) * rs * sh.cs[j];
+                                H[j * 64 + f] = g / (1.0f + expf(-g)) * U[j * 64 + f];
+                            }
+                        }
+                        named_bar_sync(1, 128);
+                        // fp32 h rows out, and each row's amax over these 64 features
+                        // folded into its global amax word (16 lanes per row)
+                        for (int idx = et; idx < 32 * 16; idx += 128) {
+                            const int r = idx >> 4, vv = idx & 15;
+                            const int col = c0 + r, feat = it.fb * 64 + vv * 4;
+                            const float4 hv = *reinterpret_cast<const float4 *>(H + r * 64 + vv * 4);
+                            float mx = 0.0f;
+                            if (col < it.n_valid && feat < p.I) {
+                                *reinterpret_cast<float4 *>(w8.h32 + (row0 + col) * p.I + feat) = hv;
+                                mx = fmaxf(fmaxf(fabsf(hv.x), fabsf(hv.y)),
+                                           fmaxf(fabsf(hv.z), fabsf(hv.w)));
+                            }
+#pragma unroll
+                            for (int o = 8; o > 0; o >>= 1)
+                                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                            if (vv == 0 && col < it.n_valid && mx > 0.0f)
+                                atomicMax(w8.hmax + row0 + col, __float_as_uint(mx));
+                        }
+                        named_bar_sync(1, 128);
+                    } else {
+                        uint16_t *Y = reinterpret_cast<uint16_t *>(epi);  // [32 cols][128 features]
+                        const int f = q4 * 32 + lane;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            Y[j * 128 + f] = to_bf16_bits(__uint_as_float(v[j]) * rs * sh.cs[j]);
+                        named_bar_sync(1, 128);
+                        for (int idx = et; idx < 32 * 16; idx += 128) {
+                            const int r = idx >> 4, vv = idx & 15;
+                            const int col = c0 + r, feat = it.fb * 128 + vv * 8;
+                            if (col < it.n_valid && feat < p.d)
+                                *reinterpret_cast<uint4 *>(p.y + (row0 + col) * p.d + feat) =
+                                    *reinterpret_cast<const uint4 *>(Y + r * 128 + vv * 8);
+                        }
+                        named_bar_sync(1, 128);
+                    }
+                    continue;
+                }
                 if (it.up) {
                     float *U = reinterpret_cast<float *>(epi);                 // [32 cols][64 features]
                     uint16_t *H = reinterpret_cast<uint16_t *>(epi + 8192);    // [32 cols][64 features]
@@ -512,22 +717,36 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// Host side: tensor maps and the launch.
-// bf16 [experts][rows][cols] weights, box = [box_rows][64 cols] of one expert
-static bool encode_weights(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows,
-                           uint64_t experts, uint32_t box_rows) {
-    const cuuint64_t dims[3] = {cols, rows, experts};
-    const cuuint64_t strides[2] = {cols * 2, cols * rows * 2};
-    const cuuint32_t box[3] = {(cuuint32_t)kChunkK, box_rows, 1};
-    return encode(m, base, 3, dims, strides, box);
+// Host side: tensor maps and the launch. Every map's box is 128 bytes wide:
+// 64 bf16 elements, or 128 E4M3 codes (w8).
+struct ElemType {
+    uint64_t size;
+    uint32_t chunk;
+    CUtensorMapDataType dt;
+};
+static ElemType elem_type(bool w8) {
+    return w8 ? ElemType{1, (uint32_t)kChunkK8, CU_TENSOR_MAP_DATA_TYPE_UINT8}
+              : ElemType{2, (uint32_t)kChunkK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16};
 }
 
-// bf16 [rows][cols] row matrix, box = [64 rows][64 cols]
-static bool encode_rows(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows) {
+// [experts][rows][cols] weights, box = [box_rows][one chunk] of one expert
+static bool encode_weights(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows,
+                           uint64_t experts, uint32_t box_rows, bool w8 = false) {
+    const ElemType et = elem_type(w8);
+    const cuuint64_t dims[3] = {cols, rows, experts};
+    const cuuint64_t strides[2] = {cols * et.size, cols * rows * et.size};
+    const cuuint32_t box[3] = {et.chunk, box_rows, 1};
+    return encode(m, base, 3, dims, strides, box, et.dt);
+}
+
+// [rows][cols] row matrix, box = [64 rows][one chunk]
+static bool encode_rows(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows,
+                        bool w8 = false) {
+    const ElemType et = elem_type(w8);
     const cuuint64_t dims[2] = {cols, rows};
-    const cuuint64_t strides[1] = {cols * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)kChunkK, (cuuint32_t)kBoxRows};
-    return encode(m, base, 2, dims, strides, box);
+    const cuuint64_t strides[1] = {cols * et.size};
+    const cuuint32_t box[2] = {et.chunk, (cuuint32_t)kBoxRows};
+    return encode(m, base, 2, dims, strides, box, et.dt);
 }
 
 // One map over both the gate and the up tensor ([E][rows][cols] each, dense):
@@ -538,8 +757,9 @@ static bool encode_rows(CUtensorMap *m, const void *base, uint64_t cols, uint64_
 // half of the tile. Returns kGateUpSplit when they overlap (or on failure),
 // and the caller then uses two 3-D maps.
 static int encode_gate_up(CUtensorMap *m, const void *gate, const void *up, uint64_t cols,
-                          uint64_t rows, uint64_t experts) {
-    const int64_t bytes = (int64_t)(cols * rows * experts * 2);
+                          uint64_t rows, uint64_t experts, bool w8 = false) {
+    const ElemType et = elem_type(w8);
+    const int64_t bytes = (int64_t)(cols * rows * experts * et.size);
     const int64_t delta = static_cast<const char *>(up) - static_cast<const char *>(gate);
     int mode;
     const void *base;
@@ -555,18 +775,21 @@ static int encode_gate_up(CUtensorMap *m, const void *gate, const void *up, uint
     const uint64_t step = (uint64_t)(delta >= 0 ? delta : -delta);
     if (step % 16 != 0 || step >= (1ull << 40)) return kGateUpSplit;
     const cuuint64_t dims[4] = {cols, rows, experts, 2};
-    const cuuint64_t strides[3] = {cols * 2, cols * rows * 2, step};
-    const cuuint32_t box[4] = {(cuuint32_t)kChunkK, 64, 1, 2};
-    return encode(m, base, 4, dims, strides, box) ? mode : kGateUpSplit;
+    const cuuint64_t strides[3] = {cols * et.size, cols * rows * et.size, step};
+    const cuuint32_t box[4] = {et.chunk, 64, 1, 2};
+    return encode(m, base, 4, dims, strides, box, et.dt) ? mode : kGateUpSplit;
 }
 
 static size_t tc_smem_bytes() {
     return 1024 + (size_t)kStages * kStageBytes + kEpiBytes + sizeof(TcShared);
 }
 
-cudaError_t launch_ffn_tc(const moge_config &c, const Plan &plan, int n_entries,
-                          const FfnOperands &op, int num_sms, cudaStream_t st, cudaEvent_t mid) {
-    (void)mid;
+// Both instantiations: maps, parameters and the launch. w8: the weights are
+// E4M3 codes with row scales (op.*_s), the B rows too (op.cs_b0 / cs_b1 their
+// token scales), op.h receives the h codes and op.h32 / hmax / sh the rest.
+static cudaError_t launch_ffn_tc_impl(bool w8, const moge_config &c, const Plan &plan,
+                                      int n_entries, const FfnOperands &op, int num_sms,
+                                      cudaStream_t st) {
     if (n_entries <= 0 || c.T <= 0) return cudaSuccess;
     const int N = c.N, S = c.S, d = c.d, I = c.I;
     // routed / shared weight tensors; a missing side borrows the other's
@@ -580,22 +803,23 @@ cudaError_t launch_ffn_tc(const moge_config &c, const Plan &plan, int n_entries,
 
     CUtensorMap mWg, mWu, mSg, mSu, mX0, mX1, mWd, mSd, mH;
     TcParams p;
-    p.gu_mode[0] = encode_gate_up(&mWg, wg, wu, d, I, ne);
-    p.gu_mode[1] = encode_gate_up(&mSg, sg, su, d, I, ns);
+    p.gu_mode[0] = encode_gate_up(&mWg, wg, wu, d, I, ne, w8);
+    p.gu_mode[1] = encode_gate_up(&mSg, sg, su, d, I, ns, w8);
     if (p.gu_mode[0] != kGateUpSplit) mWu = mWg;
-    else if (!encode_weights(&mWg, wg, d, I, ne, 64) || !encode_weights(&mWu, wu, d, I, ne, 64))
+    else if (!encode_weights(&mWg, wg, d, I, ne, 64, w8) || !encode_weights(&mWu, wu, d, I, ne, 64, w8))
         return cudaErrorInvalidValue;
     if (p.gu_mode[1] != kGateUpSplit) mSu = mSg;
-    else if (!encode_weights(&mSg, sg, d, I, ns, 64) || !encode_weights(&mSu, su, d, I, ns, 64))
+    else if (!encode_weights(&mSg, sg, d, I, ns, 64, w8) || !encode_weights(&mSu, su, d, I, ns, 64, w8))
         return cudaErrorInvalidValue;
-    if (!encode_rows(&mX0, b0, d, (uint64_t)r0) || !encode_rows(&mX1, b1, d, (uint64_t)r1) ||
-        !encode_weights(&mWd, wd, I, d, ne, 128) || !encode_weights(&mSd, sd, I, d, ns, 128) ||
-        !encode_rows(&mH, op.h, I, (uint64_t)op.h_rows))
+    if (!encode_rows(&mX0, b0, d, (uint64_t)r0, w8) || !encode_rows(&mX1, b1, d, (uint64_t)r1, w8) ||
+        !encode_weights(&mWd, wd, I, d, ne, 128, w8) || !encode_weights(&mSd, sd, I, d, ns, 128, w8) ||
+        !encode_rows(&mH, op.h, I, (uint64_t)op.h_rows, w8))
         return cudaErrorInvalidValue;
+    const int ce = w8 ? kChunkK8 : kChunkK;
     p.plan = plan;
     p.n_entries = n_entries;
-    p.kc_up = (d + kChunkK - 1) / kChunkK;
-    p.kc_down = (I + kChunkK - 1) / kChunkK;
+    p.kc_up = (d + ce - 1) / ce;
+    p.kc_down = (I + ce - 1) / ce;
     p.I = I;
     p.d = d;
     p.h = (uint16_t *)op.h;
@@ -613,13 +837,39 @@ cudaError_t launch_ffn_tc(const moge_config &c, const Plan &plan, int n_entries,
     p.pm_T = c.T;
     p.pm_N = c.N;
     p.pm_K = c.M * c.Kp;
+    W8Params q = {};
+    if (w8) {
+        const float *wgs = op.wg ? op.wg_s : op.sg_s, *wus = op.wg ? op.wu_s : op.su_s,
+                    *wds = op.wg ? op.wd_s : op.sd_s;
+        q.sc_g[0] = wgs; q.sc_u[0] = wus; q.sc_d[0] = wds;
+        q.sc_g[1] = op.sg ? op.sg_s : wgs;
+        q.sc_u[1] = op.sg ? op.su_s : wus;
+        q.sc_d[1] = op.sg ? op.sd_s : wds;
+        q.cs_b0 = op.cs_b0 ? op.cs_b0 : op.cs_b1;
+        q.cs_b1 = op.cs_b1 ? op.cs_b1 : op.cs_b0;
+        q.h32 = static_cast<float *>(op.h32);
+        q.hmax = op.hmax;
+        q.sh = op.sh;
+        q.h8 = static_cast<uint8_t *>(op.h);
+    }
 
     const size_t smem = tc_smem_bytes();
-    cudaError_t e = cudaFuncSetAttribute(ffn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    auto kern = w8 ? ffn_tc_kernel<true> : ffn_tc_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(ffn_tc_kernel, dim3(num_sms), dim3(kTcThreads), smem, st, p, mWg, mWu, mSg,
-                      mSu, mX0, mX1, mWd, mSd, mH);
+    return launch_pdl(kern, dim3(num_sms), dim3(kTcThreads), smem, st, p, q, mWg, mWu, mSg, mSu,
+                      mX0, mX1, mWd, mSd, mH);
+}
+
+cudaError_t launch_ffn_tc(const moge_config &c, const Plan &plan, int n_entries,
+                          const FfnOperands &op, int num_sms, cudaStream_t st, cudaEvent_t mid) {
+    (void)mid;
+    return launch_ffn_tc_impl(false, c, plan, n_entries, op, num_sms, st);
+}
+
+cudaError_t launch_ffn_w8a8(const moge_config &c, const Plan &plan, int n_entries,
+                            const FfnOperands &op, int num_sms, cudaStream_t st) {
+    return launch_ffn_tc_impl(true, c, plan, n_entries, op, num_sms, st);
 }
 
 }  // namespace moge

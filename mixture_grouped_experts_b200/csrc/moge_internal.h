@@ -140,11 +140,31 @@ struct FfnOperands {
     // codes and these their per-row fp32 scales ([E][I], [E][I], [E][d])
     const float *wg_s, *wu_s, *wd_s;
     const float *sg_s, *su_s, *sd_s;
+    // W8A8 only (launch_ffn_w8a8): b0 / b1 are E4M3 token rows with these
+    // per-row scales, h receives the h codes ([h_rows][I] bytes); h32
+    // ([h_rows][I] fp32), hmax ([h_rows], zeroed beforehand) and sh ([h_rows])
+    // hold h before quantisation, its row amax and its row scales
+    const float *cs_b0, *cs_b1;
+    void *h32;
+    uint32_t *hmax;
+    float *sh;
 };
 // `mid` (may be null) is recorded on the stream between the up- and the
 // down-projection launches.
 cudaError_t launch_ffn_tc(const moge_config &c, const Plan &plan, int n_entries,
                           const FfnOperands &op, int num_sms, cudaStream_t st, cudaEvent_t mid);
+cudaError_t launch_ffn_w8a8(const moge_config &c, const Plan &plan, int n_entries,
+                            const FfnOperands &op, int num_sms, cudaStream_t st);
+// W8A8 activations: per token t, scale sx[t] = amax / 448 of x's bf16 row
+// (fp32; 1 for a zero row) and the row's E4M3 codes into x8[t] and into each
+// of its K routed rows of x8p (sxp the same scale), with perm_src / perm_dst
+// as launch_scatter_rows; zeroes the amax word of each of the token's h rows
+// (hmax [T (K + S)]).
+cudaError_t launch_quantize_scatter(const moge_config &c, const void *x, const int32_t *topk_idx,
+                                    const int32_t *rank, const int32_t *base,
+                                    const int32_t *offsets, int32_t *perm_src, int32_t *perm_dst,
+                                    void *x8, float *sx, void *x8p, float *sxp, uint32_t *hmax,
+                                    cudaStream_t st);
 cudaError_t launch_ffn_f32(const moge_config &c, const Plan &plan, int n_entries,
                            const FfnOperands &op, cudaStream_t st, cudaEvent_t mid);
 namespace pair {

@@ -8,6 +8,8 @@
 // Combine weights are the picked experts' global softmax scores ("Huawei
 // releases Pangu Pro MoE", techwalker.com, section 1); shared experts are
 // always on with weight 1 (same page, section 2).
+#include <cuda_fp8.h>
+
 #include "common.cuh"
 #include "moge_internal.h"
 
@@ -66,6 +68,91 @@ cudaError_t launch_scatter_rows(const moge_config &c, const void *x, const int32
     return launch_pdl(scatter_rows_kernel, dim3(c.T, (nvec + kVecThreads - 1) / kVecThreads),
                       dim3(kVecThreads), 0, st, c, (const uint4 *)x, topk_idx, rank, base, offsets,
                       perm_src, perm_dst, (uint4 *)x_perm);
+}
+
+// W8A8 activations: one CTA per token t. The row's amax (exact in fp32),
+// scale = amax / 448 (IEEE fp32 division; 1 for an all-zero row), each code =
+// E4M3 (round to nearest even, saturating) of fp32(x / scale) -- the rule of
+// the weight quantiser -- written to x8[t] and to the token's K routed rows of
+// x8p, the scale beside each; the permutation indices as the scatter above;
+// the amax words of the token's h rows (routed and shared) zeroed for the
+// grouped FFN that follows.
+__global__ void __launch_bounds__(kVecThreads) quantize_scatter_kernel(
+    moge_config c, const uint4 *__restrict__ x, const int32_t *__restrict__ topk_idx,
+    const int32_t *__restrict__ rank, const int32_t *__restrict__ base,
+    const int32_t *__restrict__ offsets, int32_t *perm_src, int32_t *perm_dst, uint2 *x8,
+    float *sx, uint2 *x8p, float *sxp, uint32_t *hmax) {
+    __shared__ int dst_s[kMaxExperts];
+    __shared__ float red[kVecThreads / 32];
+    grid_dependency_wait();
+    const int t = blockIdx.x;
+    const int K = c.M * c.Kp;
+    const int nvec = c.d / 8;
+    for (int k = threadIdx.x; k < K; k += blockDim.x) {
+        const size_t i = (size_t)t * K + k;
+        const int e = topk_idx[i];
+        int row = -1;
+        if (e >= 0 && e < c.N) {
+            row = offsets[e] + base[(size_t)(t / kRouterTile) * c.N + e] + rank[i];
+            perm_dst[i] = row;
+            perm_src[row] = t;
+            hmax[row] = 0u;
+        } else {
+            raise_error(ERRBIT_INVARIANT);
+        }
+        dst_s[k] = row;
+    }
+    for (int s = threadIdx.x; s < c.S; s += blockDim.x)
+        hmax[(size_t)c.T * K + (size_t)s * c.T + t] = 0u;
+    const uint4 *xr = x + (size_t)t * nvec;
+    float amax = 0.0f;
+    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+        const uint4 u = xr[v];
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w[j])), fabsf(bf16_hi(w[j]))));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+    __syncthreads();  // also publishes dst_s
+    amax = red[0];
+    for (int w = 1; w < kVecThreads / 32; ++w) amax = fmaxf(amax, red[w]);
+    const float sc = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+    if (threadIdx.x == 0) sx[t] = sc;
+    for (int k = threadIdx.x; k < K; k += blockDim.x)
+        if (dst_s[k] >= 0) sxp[dst_s[k]] = sc;
+    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+        const uint4 u = xr[v];
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        uint32_t out[2] = {0u, 0u};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t b0 =
+                __nv_cvt_float_to_fp8(__fdiv_rn(bf16_lo(w[j]), sc), __NV_SATFINITE, __NV_E4M3);
+            const uint32_t b1 =
+                __nv_cvt_float_to_fp8(__fdiv_rn(bf16_hi(w[j]), sc), __NV_SATFINITE, __NV_E4M3);
+            out[j >> 1] |= (b0 | (b1 << 8)) << (16 * (j & 1));
+        }
+        const uint2 q = make_uint2(out[0], out[1]);
+        x8[(size_t)t * nvec + v] = q;
+        for (int k = 0; k < K; ++k) {
+            const int row = dst_s[k];
+            if (row >= 0) x8p[(size_t)row * nvec + v] = q;
+        }
+    }
+}
+
+cudaError_t launch_quantize_scatter(const moge_config &c, const void *x, const int32_t *topk_idx,
+                                    const int32_t *rank, const int32_t *base,
+                                    const int32_t *offsets, int32_t *perm_src, int32_t *perm_dst,
+                                    void *x8, float *sx, void *x8p, float *sxp, uint32_t *hmax,
+                                    cudaStream_t st) {
+    if (c.T <= 0) return cudaSuccess;
+    return launch_pdl(quantize_scatter_kernel, dim3(c.T), dim3(kVecThreads), 0, st, c,
+                      (const uint4 *)x, topk_idx, rank, base, offsets, perm_src, perm_dst,
+                      (uint2 *)x8, sx, (uint2 *)x8p, sxp, hmax);
 }
 
 // x_perm[r] = x[perm_src[r]], one CTA per destination row
