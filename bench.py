@@ -51,6 +51,8 @@ NOMINAL = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 TRAFFIC_RECORDS = ("profiles/ffn_tc_decode.md", "profiles/ffn_tc_pair_prefill.md")
 FFN_PAIR_KERNEL = ("ffn_tc_pair_kernel (the same grouped FFN on CTA pairs, 2-SM tcgen05 MMA, "
                    "one persistent launch)")
+FFN_W8A8_KERNEL = ("ffn_tc_kernel<W8> (the single-SM grouped FFN on 8-bit operands, tcgen05 "
+                   "kind::f8f6f4, h quantised per token between the projections, one launch)")
 
 
 def source_sha16(files=None):
@@ -790,6 +792,32 @@ def main():
                                "frac": lb8 / (fm["ms"] / 1e3) / 1e9 / hbm, "algorithmic_bytes": lb8},
             "gpu_launches_per_step": layer_launches(cfg, fp8=True),
             "stage_ms": fm["stage_ms"], "clocks": fclk}
+        # W8A8: the same 8-bit weights, x and h quantised per token inside the
+        # call, both operands of every expert GEMM E4M3 on the 8-bit MMA
+        ainp = synth.layer_inputs(cfg)
+        as_ = ClockSampler(local)
+        as_.start()
+        am = measure(cfg, ainp, args.steps, args.warmup, False, with_e2e=False, w8a8=True)
+        aclk = as_.stop()
+        del ainp
+        lba = layer_bytes_fp8(cfg, am["n_used"])
+        ach_a = lba / (am["stage_ms"]["ffn"] / 1e3) / 1e9
+        line["decode_w8a8"] = {
+            "workload": workload_config(cfg)["workload"],
+            "weights": "expert weights as OCP E4M3 codes + one fp32 scale per row; x and h "
+                       "quantised per token (E4M3, fp32 scale amax/448) inside the call; router "
+                       "bf16, y bf16; weights quantised on the device before the timed region",
+            "value": cfg.T / (am["ms"] / 1e3), "unit": "tokens/s", "ms_per_step": am["ms"],
+            "vs_bf16_layer": ms / am["ms"] if n == 1 else None,
+            "roofline": {"bound": "hbm", "kernel": FFN_W8A8_KERNEL, "achieved": ach_a, "peak": hbm,
+                         "unit": "GB/s", "frac": ach_a / hbm, "algorithmic_bytes_per_launch": lba,
+                         "algorithmic_bytes_are": "used experts' 8-bit matrices and row scales "
+                                                  "once + router + x in + y out",
+                         "kernel_ms": am["stage_ms"]["ffn"]},
+            "layer_roofline": {"achieved": lba / (am["ms"] / 1e3) / 1e9, "peak": hbm, "unit": "GB/s",
+                               "frac": lba / (am["ms"] / 1e3) / 1e9 / hbm, "algorithmic_bytes": lba},
+            "gpu_launches_per_step": layer_launches(cfg, fp8=True),
+            "stage_ms": am["stage_ms"], "clocks": aclk}
     if rank == 0 and n == 1 and not args.no_train and args.config == "decode":
         tcfg = synth.CONFIGS["prefill"]
         tinp = synth.layer_inputs(tcfg)

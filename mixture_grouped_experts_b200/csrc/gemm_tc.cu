@@ -63,6 +63,7 @@ constexpr int kStages = 4;
 constexpr int kStageBytes = 48 * 1024;
 constexpr int kEpiBytes = 16 * 1024;  // U fp32 [32][64], H and G bf16 [32][64]
 constexpr int kTcThreads = 192;
+constexpr int kTcThreadsW8 = 320;    // + warps 6-9: the h quantisers
 constexpr int kChunkK = 64;          // bf16 elements per K-chunk (128 bytes, one swizzle row)
 constexpr int kChunkK8 = 128;        // E4M3 elements per K-chunk (the same 128 bytes)
 constexpr int kKSteps = 4;           // MMAs per K-chunk: 32 bytes of K each
@@ -111,9 +112,9 @@ struct TcItem {
     bool quant;  // W8: quantise part fb of token tile tb's h rows (no GEMM)
 };
 
-// W8: every token tile's h rows are quantised by kQParts work items (row
-// slices of the tile), spread over the grid.
-constexpr int kQParts = 4;
+// W8: every token tile's h rows are quantised by kQParts work items (part p
+// takes the tile's rows p, p + kQParts, ...), spread over the grid.
+constexpr int kQParts = 16;
 
 // Decode global item q: the up-projection items first, then (W8: tot_q > 0)
 // the quantisation items, kQParts per token tile in entry order, then the
@@ -173,6 +174,7 @@ struct TcShared {
     int epi_item;
     int pm_rows[kMaxExperts];  // the fused permute: destination rows of the current token
     float cs[32];              // W8: token scales of the columns being stored
+    int q_item;                // W8: the quantisers' current item
 };
 
 // E4M3 codes of four fp32 values divided by s (IEEE fp32 division, then round
@@ -185,29 +187,46 @@ __device__ __forceinline__ uint32_t e4m3x4_div(float4 f, float s) {
     return b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
 }
 
-// W8: quantise rows [r0, r0 + rows) of h (fp32 [.][I], I % 16 == 0) per row:
-// scale = amax / 448 (IEEE fp32 division; 1 for an all-zero row), code = E4M3
-// of fp32(h / scale). Called by the 128 epilogue threads (et), one warp per
-// row, four 16-byte loads in flight per lane. h and the amax words were
-// written by other CTAs: read through L2 only.
-__device__ void quantize_h_rows(const W8Params &w8, int I, int r0, int rows, int et) {
-    const int w = et >> 5, lane = et & 31;
-    const int nv = I / 4;
-    for (int r = w; r < rows; r += 4) {
-        const size_t row = (size_t)r0 + r;
-        const float amax = __uint_as_float(__ldcg(w8.hmax + row));
-        const float sc = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-        if (lane == 0) w8.sh[row] = sc;
-        const float4 *src = reinterpret_cast<const float4 *>(w8.h32 + row * I);
-        uint32_t *dst = reinterpret_cast<uint32_t *>(w8.h8 + row * I);
-        for (int v0 = lane; v0 < nv; v0 += 128) {
-            float4 f[4];
+// W8: quantise rows row0 + first, row0 + first + step, ... (tile-relative
+// indices < n) of h (fp32 [.][I], I % 16 == 0), each with its own scale:
+// amax / 448 (IEEE fp32 division; 1 for an all-zero row), code = E4M3 of
+// fp32(h / scale). The 128 epilogue threads (et) take four rows at a time,
+// every thread loading its vectors of all four before converting any. h and
+// the amax words were written by other CTAs: read through L2 only.
+__device__ void quantize_h_rows(const W8Params &w8, int I, size_t row0, int first, int step, int n,
+                                int et) {
+    const int nv = I / 4;  // 16-byte vectors per row
+    for (int r = first; r < n; r += 4 * step) {
+        size_t row[4];
+        float sc[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
-                if (v0 + 32 * u < nv) f[u] = __ldcg(src + v0 + 32 * u);
+        for (int j = 0; j < 4; ++j) {
+            row[j] = row0 + (size_t)(r + j * step);
+            sc[j] = 1.0f;
+            if (r + j * step < n) {
+                const float amax = __uint_as_float(__ldcg(w8.hmax + row[j]));
+                if (amax > 0.0f) sc[j] = __fdiv_rn(amax, 448.0f);
+                if (et == 0) w8.sh[row[j]] = sc[j];
+            }
+        }
+        for (int v0 = 0; v0 < nv; v0 += 3 * 128) {
+            float4 f[4][3];
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
-                if (v0 + 32 * u < nv) dst[v0 + 32 * u] = e4m3x4_div(f[u], sc);
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int k = 0; k < 3; ++k) {
+                    const int v = v0 + et + 128 * k;
+                    if (r + j * step < n && v < nv)
+                        f[j][k] = __ldcg(reinterpret_cast<const float4 *>(w8.h32 + row[j] * I) + v);
+                }
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int k = 0; k < 3; ++k) {
+                    const int v = v0 + et + 128 * k;
+                    if (r + j * step < n && v < nv)
+                        reinterpret_cast<uint32_t *>(w8.h8 + row[j] * I)[v] = e4m3x4_div(f[j][k], sc[j]);
+                }
         }
     }
 }
@@ -231,11 +250,11 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 // Gives up (records ERRBIT_TIMEOUT, sets *abort) after limit_ns, or at once
 // when *abort is set; abort may be NULL.
 __device__ bool wait_counter(const int *ctr, int need, volatile int *abort,
-                             uint64_t limit_ns = kWaitTimeoutNs) {
+                             uint64_t limit_ns = kWaitTimeoutNs, uint32_t sleep_ns = 64) {
     if (ld_acquire(ctr) >= need) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
-        __nanosleep(64);
+        __nanosleep(sleep_ns);
         if (ld_acquire(ctr) >= need) return true;
         if ((it & 63u) == 0) {
             if (abort && *abort) return false;
@@ -249,7 +268,7 @@ __device__ bool wait_counter(const int *ctr, int need, volatile int *abort,
 }
 
 template <bool W8>
-__global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
+__global__ void __launch_bounds__(W8 ? kTcThreadsW8 : kTcThreads, 1) ffn_tc_kernel(
     const __grid_constant__ TcParams p, const __grid_constant__ W8Params w8,
     const __grid_constant__ CUtensorMap tmWg,
     const __grid_constant__ CUtensorMap tmWu, const __grid_constant__ CUtensorMap tmSg,
@@ -307,9 +326,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
     const int tot_up = __ldg(p.plan.up_start + p.n_entries);
     const int fb_up = (p.I + 63) / 64;
     // W8: kQParts quantisation items per token tile (every entry's up items
-    // are its tiles x fb_up)
+    // are its tiles x fb_up), taken from their own queue by warps 6-9
     const int tot_q = W8 ? kQParts * (tot_up / fb_up) : 0;
-    const int total = tot_up + tot_q + __ldg(p.plan.down_start + p.n_entries);
+    const int total = tot_up + __ldg(p.plan.down_start + p.n_entries);
     constexpr int kCE = W8 ? kChunkK8 : kChunkK;  // elements per K-chunk
 
     if (warp == 0) {
@@ -340,8 +359,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
             q = __shfl_sync(0xffffffffu, q, 0);
             if (q < 0 || q >= total) break;
             TcItem it;
-            decode_item(p, tot_up, tot_q, q, it);
-            if (it.quant) continue;  // no operands: the epilogue warps do it
+            decode_item(p, tot_up, 0, q, it);
             if (!it.up) {  // the h rows of this expert must all be stored (W8: and quantised)
                 int ok = 1;
                 if (lane == 0)
@@ -419,7 +437,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            int g = 0;  // GEMM items so far: the accumulators alternate over these
             for (int s = 0;; ++s) {
                 const int slot = s % kSlots;
                 if (!mbar_wait(&sh.slot_full[slot], (uint32_t)(s / kSlots) & 1u, abort)) break;
@@ -427,11 +444,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
                 mbar_arrive(&sh.slot_empty[slot]);
                 if (q >= total) break;
                 TcItem it;
-                decode_item(p, tot_up, tot_q, q, it);
-                if (it.quant) continue;
-                const int acc = g & 1;
-                const uint32_t use = (uint32_t)(g >> 1);
-                ++g;
+                decode_item(p, tot_up, 0, q, it);
+                const int acc = s & 1;
+                const uint32_t use = (uint32_t)(s >> 1);
                 if (!mbar_wait(&sh.tempty[acc], (use & 1u) ^ 1u, abort)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)acc * 256u;
@@ -466,6 +481,40 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
             }
             tc_commit(&sh.drain);  // every MMA of this CTA has completed after this
             mbar_wait(&sh.drain, 0, nullptr);
+        }
+    } else if (W8 && warp >= 6) {
+        // ------------------------------------------------------ h quantisers (W8)
+        // Items from their own queue (sync[1 + n_entries]: no permute runs in
+        // this launch), each once the up items of its expert are all done;
+        // they run beside the GEMM roles instead of holding up the epilogue.
+        const int qt = threadIdx.x - 6 * 32;  // 0 .. 127
+        for (;;) {
+            if (qt == 0) {
+                int i = atomicAdd(p.sync + 1 + p.n_entries, 1);
+                if (i < tot_q) {
+                    TcItem lt;
+                    decode_item(p, tot_up, tot_q, tot_up + i, lt);
+                    // (polled sparsely: up to 148 CTAs may wait here at once)
+                    if (!wait_counter(p.sync + 1 + lt.entry, lt.w.ntb * fb_up, abort,
+                                      kWaitTimeoutNs, 512))
+                        i = tot_q;
+                }
+                sh.q_item = i;
+            }
+            named_bar_sync(2, 128);
+            const int i = *(volatile int *)&sh.q_item;
+            named_bar_sync(2, 128);
+            if (i >= tot_q) break;
+            TcItem it;
+            decode_item(p, tot_up, tot_q, tot_up + i, it);
+            // rows fb, fb + kQParts, ... of the tile, then one count for the
+            // expert's down-projection items
+            quantize_h_rows(w8, p.I, (size_t)it.w.dst_row0 + (size_t)it.tb * it.w.bn, it.fb,
+                            kQParts, it.n_valid, qt);
+            fence_proxy_async_global();
+            __threadfence();
+            named_bar_sync(2, 128);
+            if (qt == 0) atomicAdd(p.sync + 1 + it.entry, 1);
         }
     } else {
         // ------------------------------------------------------ epilogue
@@ -508,25 +557,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
             named_bar_sync(1, 128);
             if (et == 0) atomicAdd(p.sync + 1 + p.n_entries, 1);
         }
-        int g = 0;  // GEMM items so far (as the MMA issuer counts them)
         for (int s = 0;; ++s) {
-            // the leader takes the next item and waits for its accumulator (a
-            // quantisation item: for the up items of its expert); all 128
-            // threads then act on the same decision
+            // the leader takes the next item and waits for its accumulator;
+            // all 128 threads then act on the same decision
             if (et == 0) {
                 const int slot = s % kSlots;
                 int q = -1;
                 if (mbar_wait(&sh.slot_full[slot], (uint32_t)(s / kSlots) & 1u, abort)) {
                     q = sh.slot_item[slot];
                     mbar_arrive(&sh.slot_empty[slot]);
-                    if (q < total) {
-                        TcItem lt;
-                        decode_item(p, tot_up, tot_q, q, lt);
-                        const bool ok =
-                            lt.quant ? wait_counter(p.sync + 1 + lt.entry, lt.w.ntb * fb_up, abort)
-                                     : mbar_wait(&sh.tfull[g & 1], (uint32_t)(g >> 1) & 1u, abort);
-                        if (!ok) q = -1;
-                    }
+                    if (q < total && !mbar_wait(&sh.tfull[s & 1], (uint32_t)(s >> 1) & 1u, abort))
+                        q = -1;
                 }
                 sh.epi_item = q;
             }
@@ -534,25 +575,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(
             const int q = *(volatile int *)&sh.epi_item;
             named_bar_sync(1, 128);
             if (q < 0 || q >= total) break;
-            TcItem it;
-            decode_item(p, tot_up, tot_q, q, it);
-            if constexpr (W8) {
-                if (it.quant) {
-                    // rows [lo, hi) of the tile's n_valid rows, then one count for
-                    // the expert's down-projection items
-                    const int per = (it.n_valid + kQParts - 1) / kQParts;
-                    const int lo = min(it.n_valid, it.fb * per), hi = min(it.n_valid, lo + per);
-                    quantize_h_rows(w8, p.I, it.w.dst_row0 + it.tb * it.w.bn + lo, hi - lo, et);
-                    fence_proxy_async_global();
-                    __threadfence();
-                    named_bar_sync(1, 128);
-                    if (et == 0) atomicAdd(p.sync + 1 + it.entry, 1);
-                    continue;
-                }
-            }
             tc_fence_after();
-            const int acc = g & 1;
-            ++g;
+            TcItem it;
+            decode_item(p, tot_up, 0, q, it);
+            const int acc = s & 1;
             const uint32_t tbase = tmem_base + ((uint32_t)(32 * q4) << 16) + (uint32_t)acc * 256u;
             const size_t row0 = (size_t)it.w.dst_row0 + (size_t)it.tb * it.w.bn;
             // W8: the scale of this thread's accumulator row (its weight row)
@@ -857,7 +883,8 @@ static cudaError_t launch_ffn_tc_impl(bool w8, const moge_config &c, const Plan 
     auto kern = w8 ? ffn_tc_kernel<true> : ffn_tc_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(kern, dim3(num_sms), dim3(kTcThreads), smem, st, p, q, mWg, mWu, mSg, mSu,
+    return launch_pdl(kern, dim3(num_sms), dim3(w8 ? kTcThreadsW8 : kTcThreads), smem, st, p, q,
+                      mWg, mWu, mSg, mSu,
                       mX0, mX1, mWd, mSd, mH);
 }
 
