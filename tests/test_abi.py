@@ -122,6 +122,32 @@ def test_fp8_entry_points_validate_on_host(L):
     assert rc == mg.ERR_UNSUPPORTED and b"gate_scale" in L.moge_last_error()
 
 
+def test_w8a8_entry_points_validate_on_host(L):
+    s = _shape(dtype="bf16")
+    K, hrows = s.M * s.Kp, s.T * (s.M * s.Kp + s.S)
+    # the forward workspace, then x's codes, two scale arrays, h in fp32 and
+    # its amax words and scales
+    extra = s.T * s.d + s.T * 4 + s.T * K * 4 + hrows * s.I * 4 + 2 * hrows * 4
+    n = mg.w8a8_workspace_size(s)
+    assert mg.workspace_size(s) + extra <= n <= mg.workspace_size(s) + extra + 6 * 256
+    assert L.moge_w8a8_workspace_size(ctypes.byref(mg._cfg(_shape(M=3)))) == 0
+    f8 = mg.moge_fp8_experts(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000)
+    args = (0x7000, 0x8000, None, ctypes.byref(f8), ctypes.byref(f8), None, 0x9000, 0xA000, None)
+    rc = L.moge_layer_forward_w8a8(ctypes.byref(mg._cfg(_shape(dtype="f32"))), *args)
+    assert rc == mg.ERR_UNSUPPORTED and b"BF16" in L.moge_last_error()
+    rc = L.moge_layer_forward_w8a8(ctypes.byref(mg._cfg(_shape(dtype="bf16", d=264))), *args)
+    assert rc == mg.ERR_UNSUPPORTED and b"% 16" in L.moge_last_error()
+    rc = L.moge_layer_forward_w8a8(ctypes.byref(mg._cfg(s)), 0x7000, 0x8000, None, None,
+                                   ctypes.byref(f8), None, 0x9000, 0xA000, None)
+    assert rc == mg.ERR_INVALID_ARG and b"routed" in L.moge_last_error()
+    rc = L.moge_layer_forward_w8a8(ctypes.byref(mg._cfg(s)), 0x7000, 0x8000, None,
+                                   ctypes.byref(f8), ctypes.byref(f8), None, 0x7000, 0xA000, None)
+    assert rc == mg.ERR_INVALID_ARG and b"alias" in L.moge_last_error()
+    rc = L.moge_layer_forward_w8a8(ctypes.byref(mg._cfg(s)), 0x7000, 0x8000, None,
+                                   ctypes.byref(f8), ctypes.byref(f8), None, 0x9000, None, None)
+    assert rc == mg.ERR_INVALID_ARG and b"workspace" in L.moge_last_error()
+
+
 def test_wait_selftest_validates_on_host(L):
     assert L.moge_selftest_waits(0, 0x1000, None) == mg.ERR_INVALID_ARG
     assert L.moge_selftest_waits(2000001, 0x1000, None) == mg.ERR_INVALID_ARG
