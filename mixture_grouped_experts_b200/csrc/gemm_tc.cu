@@ -173,7 +173,7 @@ struct TcShared {
     int abort;
     int epi_item;
     int pm_rows[kMaxExperts];  // the fused permute: destination rows of the current token
-    float cs[32];              // W8: token scales of the columns being stored
+    float cs[kMaxTileN];       // W8: token scales of the current item's columns
     int q_item;                // W8: the quantisers' current item
 };
 
@@ -600,14 +600,14 @@ __global__ void __launch_bounds__(W8 ? kTcThreadsW8 : kTcThreads, 1) ffn_tc_kern
                     cs = w8.sh;
                 }
                 cs += (size_t)it.w.src_row0 + (size_t)it.tb * it.w.bn;
+                // all of the item's token scales at once (h scales were written in
+                // this launch: through L2); one load latency per item
+                for (int j = et; j < it.n_valid; j += 128) sh.cs[j] = __ldcg(cs + j);
+                named_bar_sync(1, 128);
             }
             for (int c0 = 0; c0 < it.n_valid; c0 += 32) {
                 uint32_t v[32];
                 tmem_ld_32x32b_x32(tbase + (uint32_t)c0, v);
-                if constexpr (W8) {  // h scales were written in this launch: through L2
-                    if (et < 32) sh.cs[et] = c0 + et < it.n_valid ? __ldcg(cs + c0 + et) : 0.0f;
-                    named_bar_sync(1, 128);
-                }
                 tmem_ld_wait();
                 if constexpr (W8) {
                     if (it.up) {
@@ -619,13 +619,13 @@ __global__ void __launch_bounds__(W8 ? kTcThreadsW8 : kTcThreads, 1) ffn_tc_kern
                         if (!is_gate) {
 #pragma unroll
                             for (int j = 0; j < 32; ++j)
-                                U[j * 64 + f] = __uint_as_float(v[j]) * rs * sh.cs[j];
+                                U[j * 64 + f] = __uint_as_float(v[j]) * rs * sh.cs[c0 + j];
                         }
                         named_bar_sync(1, 128);
                         if (is_gate) {
 #pragma unroll
                             for (int j = 0; j < 32; ++j) {
-                                const float g = __uint_as_float(v[j]) * rs * sh.cs[j];
+                                const float g = __uint_as_float(v[j]) * rs * sh.cs[c0 + j];
                                 H[j * 64 + f] = g / (1.0f + expf(-g)) * U[j * 64 + f];
                             }
                         }
@@ -654,7 +654,7 @@ __global__ void __launch_bounds__(W8 ? kTcThreadsW8 : kTcThreads, 1) ffn_tc_kern
                         const int f = q4 * 32 + lane;
 #pragma unroll
                         for (int j = 0; j < 32; ++j)
-                            Y[j * 128 + f] = to_bf16_bits(__uint_as_float(v[j]) * rs * sh.cs[j]);
+                            Y[j * 128 + f] = to_bf16_bits(__uint_as_float(v[j]) * rs * sh.cs[c0 + j]);
                         named_bar_sync(1, 128);
                         for (int idx = et; idx < 32 * 16; idx += 128) {
                             const int r = idx >> 4, vv = idx & 15;
