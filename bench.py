@@ -48,7 +48,8 @@ NOMINAL = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 # dram__bytes_write.sum) and a hash of the CUDA sources the capture ran. The
 # bench reports it only while the sources still hash the same (else null: the
 # kernel changed since the counters were taken).
-TRAFFIC_RECORDS = ("profiles/ffn_tc_decode.md", "profiles/ffn_tc_pair_prefill.md")
+TRAFFIC_RECORDS = ("profiles/ffn_tc_decode.md", "profiles/ffn_tc_pair_prefill.md",
+                   "profiles/ffn_tc_w8a8_decode.md")
 FFN_PAIR_KERNEL = ("ffn_tc_pair_kernel (the same grouped FFN on CTA pairs, 2-SM tcgen05 MMA, "
                    "one persistent launch)")
 FFN_W8A8_KERNEL = ("ffn_tc_kernel<W8> (the single-SM grouped FFN on 8-bit operands, tcgen05 "
@@ -641,7 +642,11 @@ def main():
     ap.add_argument("--no-secondary", action="store_true", help="skip the prefill side measurement")
     ap.add_argument("--cpu-tokens", type=int, default=16, help="tokens in the CPU-baseline sample (0: skip)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
-    ap.add_argument("--no-fp8", action="store_true", help="skip the 8-bit-weight side measurement")
+    ap.add_argument("--no-fp8", action="store_true",
+                    help="skip the 8-bit side measurements (weights-only and W8A8)")
+    ap.add_argument("--arith", default="bf16", choices=["bf16", "w8a8"],
+                    help="arithmetic of the main line: the bf16 layer, or the W8A8 layer "
+                         "(8-bit weights and per-token 8-bit activations; no host-buffer leg)")
     ap.add_argument("--no-train", action="store_true", help="skip the training-step side measurement")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the skewed-router and 12-layer-stack side measurements")
@@ -676,7 +681,9 @@ def main():
     inp = rank_inputs(cfg, rank)
     sampler = ClockSampler(local)
     sampler.start()
-    m = measure(cfg, inp, args.steps, args.warmup, dist_on, with_e2e=not args.no_e2e)
+    w8 = args.arith == "w8a8"
+    m = measure(cfg, inp, args.steps, args.warmup, dist_on, with_e2e=not (args.no_e2e or w8),
+                w8a8=w8)
     clocks = sampler.stop()
     ms = max_over_ranks(m["ms"], dist_on)
     e2e_ms = max_over_ranks(m.get("e2e_ms", float("nan")), dist_on)
@@ -687,8 +694,30 @@ def main():
     hbm = peaks["hbm_gbs"]
     tf_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     tf_sust = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
-    lb = layer_bytes(cfg, m["n_used"])
-    if cfg.T * cfg.M * cfg.Kp < PAIR_ROWS:
+    lb = layer_bytes_fp8(cfg, m["n_used"]) if w8 else layer_bytes(cfg, m["n_used"])
+    if w8:
+        # the W8A8 grouped FFN: the layer's 8-bit algorithmic bytes over its live
+        # time (HBM-bound at decode), or its flops against the 8-bit dense rate
+        # (twice the measured bf16 burst peak, the nominal fp8 / bf16 ratio)
+        traffic, tsrc = traffic_record("ffn_tc_kernel<W8>", cfg.name)
+        if cfg.T * cfg.M * cfg.Kp < PAIR_ROWS:
+            ach = lb / (su["ffn"] / 1e3) / 1e9
+            roofline = {"bound": "hbm", "kernel": FFN_W8A8_KERNEL, "achieved": ach, "peak": hbm,
+                        "unit": "GB/s", "frac": ach / hbm,
+                        "peak_source": "%s hbm_gbs" % peak_kind,
+                        "algorithmic_bytes_per_launch": lb,
+                        "algorithmic_bytes_are": "used experts' 8-bit matrices and row scales "
+                                                 "once + router + x in + y out",
+                        "traffic": traffic, "traffic_source": tsrc, "kernel_ms": su["ffn"]}
+        else:
+            ftf = ffn_flops(cfg) / (su["ffn"] / 1e3) / 1e12
+            roofline = {"bound": "tensor", "kernel": FFN_W8A8_KERNEL, "achieved": ftf,
+                        "peak": 2 * tf_burst, "unit": "TFLOP/s", "frac": ftf / (2 * tf_burst),
+                        "peak_source": "2 x %s bf16_tflops (burst): the nominal fp8/bf16 ratio"
+                                       % peak_kind,
+                        "algorithmic_flops_per_launch": ffn_flops(cfg),
+                        "traffic": traffic, "traffic_source": tsrc, "kernel_ms": su["ffn"]}
+    elif cfg.T * cfg.M * cfg.Kp < PAIR_ROWS:
         # algorithmic bytes of the layer (the used experts' three matrices once,
         # the router, x in, y out: no padding, permute or intermediate rows) over
         # the grouped FFN's live launch time
@@ -739,6 +768,13 @@ def main():
                         "api": "moge_layer_forward_host (one batch, synchronised per step)"}},
             "gpu_launches": layer_launches(cfg) * args.steps,
             "clocks": clocks}
+    if w8:
+        line["dtype"] = "e4m3 (W8A8: expert weights and activations; router bf16, fp32 accumulation)"
+        line["e2e"] = {"value": None, "unit": "tokens/s", "h2d_bytes_per_step": None,
+                       "d2h_bytes_per_step": None,
+                       "note": "the host-buffer entry points run the bf16 layer; the W8A8 layer "
+                               "is device-timed only"}
+        line["gpu_launches"] = layer_launches(cfg, fp8=True) * args.steps
     if rank == 0 and n == 1 and args.cpu_tokens > 0:
         line["cpu_baseline"] = cpu_baseline(cfg, inp, args.cpu_tokens)
     del inp
@@ -769,7 +805,7 @@ def main():
                                "algorithmic_flops": layer_flops(pcfg)},
             "gpu_launches_per_step": layer_launches(pcfg),
             "stage_ms": pm["stage_ms"], "clocks": pclk}
-    if rank == 0 and n == 1 and not args.no_fp8 and args.config == "decode":
+    if rank == 0 and n == 1 and not args.no_fp8 and not w8 and args.config == "decode":
         finp = synth.layer_inputs(cfg)
         fs = ClockSampler(local)
         fs.start()
@@ -802,6 +838,7 @@ def main():
         del ainp
         lba = layer_bytes_fp8(cfg, am["n_used"])
         ach_a = lba / (am["stage_ms"]["ffn"] / 1e3) / 1e9
+        atraffic, atsrc = traffic_record("ffn_tc_kernel<W8>", cfg.name)
         line["decode_w8a8"] = {
             "workload": workload_config(cfg)["workload"],
             "weights": "expert weights as OCP E4M3 codes + one fp32 scale per row; x and h "
@@ -813,6 +850,7 @@ def main():
                          "unit": "GB/s", "frac": ach_a / hbm, "algorithmic_bytes_per_launch": lba,
                          "algorithmic_bytes_are": "used experts' 8-bit matrices and row scales "
                                                   "once + router + x in + y out",
+                         "traffic": atraffic, "traffic_source": atsrc,
                          "kernel_ms": am["stage_ms"]["ffn"]},
             "layer_roofline": {"achieved": lba / (am["ms"] / 1e3) / 1e9, "peak": hbm, "unit": "GB/s",
                                "frac": lba / (am["ms"] / 1e3) / 1e9 / hbm, "algorithmic_bytes": lba},
