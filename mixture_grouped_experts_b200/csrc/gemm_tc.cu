@@ -611,31 +611,32 @@ __global__ void __launch_bounds__(W8 ? kTcThreadsW8 : kTcThreads, 1) ffn_tc_kern
                 tmem_ld_wait();
                 if constexpr (W8) {
                     if (it.up) {
-                        float *U = reinterpret_cast<float *>(epi);           // [32 cols][64 features]
-                        float *H = reinterpret_cast<float *>(epi + 8192);    // [32 cols][64 features]
+                        // the scaled gate and up accumulators staged side by side,
+                        // then every thread forms h for 16 of the block's 2048
+                        // (column, feature) pairs (the 8-bit MMA leaves the epilogue
+                        // half the time of a bf16 item, so the SwiGLU is spread over
+                        // all four warps, with the fast exponential and division)
+                        float *G = reinterpret_cast<float *>(epi);           // [32 cols][64 features]
+                        float *U = reinterpret_cast<float *>(epi + 8192);    // [32 cols][64 features]
                         const bool gate_hi = p.gu_mode[it.w.a_sel] == kUpGateFused;
-                        const bool is_gate = (q4 < 2) != gate_hi;
+                        float *D = ((q4 < 2) != gate_hi) ? G : U;
                         const int f = (q4 & 1) * 32 + lane;
-                        if (!is_gate) {
 #pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                U[j * 64 + f] = __uint_as_float(v[j]) * rs * sh.cs[c0 + j];
-                        }
-                        named_bar_sync(1, 128);
-                        if (is_gate) {
-#pragma unroll
-                            for (int j = 0; j < 32; ++j) {
-                                const float g = __uint_as_float(v[j]) * rs * sh.cs[c0 + j];
-                                H[j * 64 + f] = g / (1.0f + expf(-g)) * U[j * 64 + f];
-                            }
-                        }
+                        for (int j = 0; j < 32; ++j)
+                            D[j * 64 + f] = __uint_as_float(v[j]) * rs * sh.cs[c0 + j];
                         named_bar_sync(1, 128);
                         // fp32 h rows out, and each row's amax over these 64 features
                         // folded into its global amax word (16 lanes per row)
                         for (int idx = et; idx < 32 * 16; idx += 128) {
                             const int r = idx >> 4, vv = idx & 15;
                             const int col = c0 + r, feat = it.fb * 64 + vv * 4;
-                            const float4 hv = *reinterpret_cast<const float4 *>(H + r * 64 + vv * 4);
+                            const float4 g = *reinterpret_cast<const float4 *>(G + r * 64 + vv * 4);
+                            const float4 u = *reinterpret_cast<const float4 *>(U + r * 64 + vv * 4);
+                            float4 hv;
+                            hv.x = __fdividef(g.x, 1.0f + __expf(-g.x)) * u.x;
+                            hv.y = __fdividef(g.y, 1.0f + __expf(-g.y)) * u.y;
+                            hv.z = __fdividef(g.z, 1.0f + __expf(-g.z)) * u.z;
+                            hv.w = __fdividef(g.w, 1.0f + __expf(-g.w)) * u.w;
                             float mx = 0.0f;
                             if (col < it.n_valid && feat < p.I) {
                                 *reinterpret_cast<float4 *>(w8.h32 + (row0 + col) * p.I + feat) = hv;
