@@ -63,7 +63,7 @@ constexpr int kStages = 4;
 constexpr int kStageBytes = 48 * 1024;
 constexpr int kEpiBytes = 16 * 1024;  // U fp32 [32][64], H and G bf16 [32][64]
 constexpr int kTcThreads = 192;
-constexpr int kTcThreadsW8 = 320;    // + warps 6-9: the h quantisers
+constexpr int kTcThreadsW8 = 448;    // warps 2-9 epilogue (two per TMEM lane quarter), 10-13 the h quantisers
 constexpr int kChunkK = 64;          // bf16 elements per K-chunk (128 bytes, one swizzle row)
 constexpr int kChunkK8 = 128;        // E4M3 elements per K-chunk (the same 128 bytes)
 constexpr int kKSteps = 4;           // MMAs per K-chunk: 32 bytes of K each
@@ -292,7 +292,7 @@ __global__ void __launch_bounds__(W8 ? kTcThreadsW8 : kTcThreads, 1) ffn_tc_kern
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&sh.tfull[a], 1);
-            mbar_init(&sh.tempty[a], 128);
+            mbar_init(&sh.tempty[a], W8 ? 256 : 128);  // every epilogue thread
         }
         for (int s = 0; s < kSlots; ++s) {
             mbar_init(&sh.slot_full[s], 1);
@@ -326,7 +326,7 @@ __global__ void __launch_bounds__(W8 ? kTcThreadsW8 : kTcThreads, 1) ffn_tc_kern
     const int tot_up = __ldg(p.plan.up_start + p.n_entries);
     const int fb_up = (p.I + 63) / 64;
     // W8: kQParts quantisation items per token tile (every entry's up items
-    // are its tiles x fb_up), taken from their own queue by warps 6-9
+    // are its tiles x fb_up), taken from their own queue by warps 10-13
     const int tot_q = W8 ? kQParts * (tot_up / fb_up) : 0;
     const int total = tot_up + __ldg(p.plan.down_start + p.n_entries);
     constexpr int kCE = W8 ? kChunkK8 : kChunkK;  // elements per K-chunk
@@ -482,12 +482,12 @@ __global__ void __launch_bounds__(W8 ? kTcThreadsW8 : kTcThreads, 1) ffn_tc_kern
             tc_commit(&sh.drain);  // every MMA of this CTA has completed after this
             mbar_wait(&sh.drain, 0, nullptr);
         }
-    } else if (W8 && warp >= 6) {
+    } else if (W8 && warp >= 10) {
         // ------------------------------------------------------ h quantisers (W8)
         // Items from their own queue (sync[1 + n_entries]: no permute runs in
         // this launch), each once the up items of its expert are all done;
         // they run beside the GEMM roles instead of holding up the epilogue.
-        const int qt = threadIdx.x - 6 * 32;  // 0 .. 127
+        const int qt = threadIdx.x - 10 * 32;  // 0 .. 127
         for (;;) {
             if (qt == 0) {
                 int i = atomicAdd(p.sync + 1 + p.n_entries, 1);
@@ -519,7 +519,11 @@ __global__ void __launch_bounds__(W8 ? kTcThreadsW8 : kTcThreads, 1) ffn_tc_kern
     } else {
         // ------------------------------------------------------ epilogue
         const int q4 = warp & 3;           // TMEM lane quarter this warp may read
-        const int et = threadIdx.x - 64;   // 0 .. 127
+        const int et = threadIdx.x - 64;   // 0 .. kEpi - 1
+        // W8: eight epilogue warps, two per lane quarter, each taking 16 of
+        // every 32 accumulator columns (the 8-bit MMA halves an item's time)
+        constexpr int kEpi = W8 ? 256 : 128;
+        const int eh = W8 ? (warp - 2) >> 2 : 0;
         if (p.pm_topk_idx) {
             // The permute, before this CTA's first accumulator exists: tokens
             // blockIdx.x, + gridDim.x, ...; each token's K destination rows
@@ -542,7 +546,7 @@ __global__ void __launch_bounds__(W8 ? kTcThreadsW8 : kTcThreads, 1) ffn_tc_kern
                     }
                     sh.pm_rows[k] = row;
                 }
-                named_bar_sync(1, 128);
+                named_bar_sync(1, kEpi);
                 for (int v = et; v < nvec; v += 128) {
                     const uint4 val = p.pm_x[(size_t)t * nvec + v];
                     for (int k = 0; k < K; ++k) {
@@ -550,16 +554,16 @@ __global__ void __launch_bounds__(W8 ? kTcThreadsW8 : kTcThreads, 1) ffn_tc_kern
                         if (row >= 0) p.pm_x_perm[(size_t)row * nvec + v] = val;
                     }
                 }
-                named_bar_sync(1, 128);
+                named_bar_sync(1, kEpi);
             }
             fence_proxy_async_global();
             __threadfence();
-            named_bar_sync(1, 128);
+            named_bar_sync(1, kEpi);
             if (et == 0) atomicAdd(p.sync + 1 + p.n_entries, 1);
         }
         for (int s = 0;; ++s) {
             // the leader takes the next item and waits for its accumulator;
-            // all 128 threads then act on the same decision
+            // all epilogue threads then act on the same decision
             if (et == 0) {
                 const int slot = s % kSlots;
                 int q = -1;
@@ -571,9 +575,9 @@ __global__ void __launch_bounds__(W8 ? kTcThreadsW8 : kTcThreads, 1) ffn_tc_kern
                 }
                 sh.epi_item = q;
             }
-            named_bar_sync(1, 128);
+            named_bar_sync(1, kEpi);
             const int q = *(volatile int *)&sh.epi_item;
-            named_bar_sync(1, 128);
+            named_bar_sync(1, kEpi);
             if (q < 0 || q >= total) break;
             tc_fence_after();
             TcItem it;
@@ -602,12 +606,15 @@ __global__ void __launch_bounds__(W8 ? kTcThreadsW8 : kTcThreads, 1) ffn_tc_kern
                 cs += (size_t)it.w.src_row0 + (size_t)it.tb * it.w.bn;
                 // all of the item's token scales at once (h scales were written in
                 // this launch: through L2); one load latency per item
-                for (int j = et; j < it.n_valid; j += 128) sh.cs[j] = __ldcg(cs + j);
-                named_bar_sync(1, 128);
+                for (int j = et; j < it.n_valid; j += kEpi) sh.cs[j] = __ldcg(cs + j);
+                named_bar_sync(1, kEpi);
             }
             for (int c0 = 0; c0 < it.n_valid; c0 += 32) {
                 uint32_t v[32];
-                tmem_ld_32x32b_x32(tbase + (uint32_t)c0, v);
+                if constexpr (W8)
+                    tmem_ld_32x32b_x16(tbase + (uint32_t)(c0 + 16 * eh), v);
+                else
+                    tmem_ld_32x32b_x32(tbase + (uint32_t)c0, v);
                 tmem_ld_wait();
                 if constexpr (W8) {
                     if (it.up) {
@@ -622,12 +629,14 @@ __global__ void __launch_bounds__(W8 ? kTcThreadsW8 : kTcThreads, 1) ffn_tc_kern
                         float *D = ((q4 < 2) != gate_hi) ? G : U;
                         const int f = (q4 & 1) * 32 + lane;
 #pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            D[j * 64 + f] = __uint_as_float(v[j]) * rs * sh.cs[c0 + j];
-                        named_bar_sync(1, 128);
+                        for (int j = 0; j < 16; ++j) {
+                            const int cj = 16 * eh + j;
+                            D[cj * 64 + f] = __uint_as_float(v[j]) * rs * sh.cs[c0 + cj];
+                        }
+                        named_bar_sync(1, kEpi);
                         // fp32 h rows out, and each row's amax over these 64 features
                         // folded into its global amax word (16 lanes per row)
-                        for (int idx = et; idx < 32 * 16; idx += 128) {
+                        for (int idx = et; idx < 32 * 16; idx += kEpi) {
                             const int r = idx >> 4, vv = idx & 15;
                             const int col = c0 + r, feat = it.fb * 64 + vv * 4;
                             const float4 g = *reinterpret_cast<const float4 *>(G + r * 64 + vv * 4);
@@ -649,22 +658,24 @@ __global__ void __launch_bounds__(W8 ? kTcThreadsW8 : kTcThreads, 1) ffn_tc_kern
                             if (vv == 0 && col < it.n_valid && mx > 0.0f)
                                 atomicMax(w8.hmax + row0 + col, __float_as_uint(mx));
                         }
-                        named_bar_sync(1, 128);
+                        named_bar_sync(1, kEpi);
                     } else {
                         uint16_t *Y = reinterpret_cast<uint16_t *>(epi);  // [32 cols][128 features]
                         const int f = q4 * 32 + lane;
 #pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            Y[j * 128 + f] = to_bf16_bits(__uint_as_float(v[j]) * rs * sh.cs[c0 + j]);
-                        named_bar_sync(1, 128);
-                        for (int idx = et; idx < 32 * 16; idx += 128) {
+                        for (int j = 0; j < 16; ++j) {
+                            const int cj = 16 * eh + j;
+                            Y[cj * 128 + f] = to_bf16_bits(__uint_as_float(v[j]) * rs * sh.cs[c0 + cj]);
+                        }
+                        named_bar_sync(1, kEpi);
+                        for (int idx = et; idx < 32 * 16; idx += kEpi) {
                             const int r = idx >> 4, vv = idx & 15;
                             const int col = c0 + r, feat = it.fb * 128 + vv * 8;
                             if (col < it.n_valid && feat < p.d)
                                 *reinterpret_cast<uint4 *>(p.y + (row0 + col) * p.d + feat) =
                                     *reinterpret_cast<const uint4 *>(Y + r * 128 + vv * 8);
                         }
-                        named_bar_sync(1, 128);
+                        named_bar_sync(1, kEpi);
                     }
                     continue;
                 }
@@ -680,7 +691,7 @@ __global__ void __launch_bounds__(W8 ? kTcThreadsW8 : kTcThreads, 1) ffn_tc_kern
 #pragma unroll
                         for (int j = 0; j < 32; ++j) U[j * 64 + f] = __uint_as_float(v[j]);
                     }
-                    named_bar_sync(1, 128);
+                    named_bar_sync(1, kEpi);
                     if (is_gate) {
 #pragma unroll
                         for (int j = 0; j < 32; ++j) {
@@ -690,8 +701,8 @@ __global__ void __launch_bounds__(W8 ? kTcThreadsW8 : kTcThreads, 1) ffn_tc_kern
                             if (p.gu) G[j * 64 + f] = to_bf16_bits(g);
                         }
                     }
-                    named_bar_sync(1, 128);
-                    for (int idx = et; idx < 32 * 8; idx += 128) {
+                    named_bar_sync(1, kEpi);
+                    for (int idx = et; idx < 32 * 8; idx += kEpi) {
                         const int r = idx >> 3, vv = idx & 7;
                         const int col = c0 + r, feat = it.fb * 64 + vv * 8;
                         if (col < it.n_valid && feat < p.I) {
@@ -708,21 +719,21 @@ __global__ void __launch_bounds__(W8 ? kTcThreadsW8 : kTcThreads, 1) ffn_tc_kern
                             }
                         }
                     }
-                    named_bar_sync(1, 128);
+                    named_bar_sync(1, kEpi);
                 } else {
                     uint16_t *Y = reinterpret_cast<uint16_t *>(epi);  // [32 cols][128 features]
                     const int f = q4 * 32 + lane;
 #pragma unroll
                     for (int j = 0; j < 32; ++j) Y[j * 128 + f] = to_bf16_bits(__uint_as_float(v[j]));
-                    named_bar_sync(1, 128);
-                    for (int idx = et; idx < 32 * 16; idx += 128) {
+                    named_bar_sync(1, kEpi);
+                    for (int idx = et; idx < 32 * 16; idx += kEpi) {
                         const int r = idx >> 4, vv = idx & 15;
                         const int col = c0 + r, feat = it.fb * 128 + vv * 8;
                         if (col < it.n_valid && feat < p.d)
                             *reinterpret_cast<uint4 *>(p.y + (row0 + col) * p.d + feat) =
                                 *reinterpret_cast<const uint4 *>(Y + r * 128 + vv * 8);
                     }
-                    named_bar_sync(1, 128);
+                    named_bar_sync(1, kEpi);
                 }
             }
             tc_fence_before();
@@ -731,7 +742,7 @@ __global__ void __launch_bounds__(W8 ? kTcThreadsW8 : kTcThreads, 1) ffn_tc_kern
                 // publish this item's h rows to the down-projection items of the expert
                 fence_proxy_async_global();
                 __threadfence();
-                named_bar_sync(1, 128);
+                named_bar_sync(1, kEpi);
                 if (et == 0) atomicAdd(p.sync + 1 + it.entry, 1);
             }
         }
