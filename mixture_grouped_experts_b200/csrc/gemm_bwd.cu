@@ -15,10 +15,16 @@
 //   kDWR    dWr   = dl^T x         (K = T)
 //   kDXR    dx_r  = dl Wr          (K = N, fp32)
 // D = A B^T with the MMA's M = 128 rows of A in TMEM lanes and N <= 256
-// columns. Operands are staged by TMA in 64 x 64 boxes with the 128-byte
-// swizzle; a row-major matrix read along its rows is a "K-major" operand, read
-// across them an "MN-major" one (tcgen05 descriptor: 8-row groups 1024 bytes
-// apart, 64-element blocks 8 KB apart). Gradients over an expert's rows have a
+// columns. Operands are staged by TMA with the 128-byte swizzle; a row-major
+// matrix read along its rows is a "K-major" operand, read across them an
+// "MN-major" one (tcgen05 descriptor: 8-row groups 1024 bytes apart,
+// 64-element blocks 8 KB apart). Few, large copies: a copy's issue cost, not
+// its bytes, bounded these GEMMs with 8 KB boxes. So a K-major operand comes
+// in 128-row boxes, and an MN-major one -- whose 128-byte swizzle row holds
+// only 64 of its MN elements -- through a view of the matrix whose outermost
+// dimension steps over its 64-column blocks ({64 columns, rows, column
+// blocks}, the blocks 128 bytes apart): one copy lands several 64-wide blocks
+// one after another, 8 KB apart, which is the descriptor's layout. Gradients over an expert's rows have a
 // ragged last K-chunk: its rows past the expert are zeroed in shared memory in
 // the A operand (they belong to the next expert) and the MMAs past them are
 // skipped.
@@ -60,6 +66,7 @@ struct GParams {
     void *out[4];
     const uint16_t *gu;     // kDH: [rows][2I]
     const float *bias;      // kLOGITS, nullable
+    int a_wide, b_wide;     // A: one 128-column copy; B: one 256-column copy (MN-major views)
 };
 
 // One work item, with its plan entry's fields held in registers (the copy
@@ -140,31 +147,49 @@ __device__ void g_decode(const GParams &p, const GShared &sh, int q, GItem &it) 
     }
 }
 
-// Issue box `j` of operand A (j < 2) or B (j >= 2: box j - 2) of chunk kc.
+// Copies of one chunk: A in na copies, B in nb (g_copies); lane j issues
+// copy j (A's first). A wide copy (p.a_wide / p.b_wide) is one copy of a
+// column-block view (see the file comment); otherwise 64 x 64 boxes, or
+// 128-row boxes for the K-major B rows of the token kinds.
+__device__ __forceinline__ void g_copies(const GParams &p, const GItem &it, int &na, int &nb,
+                                         uint32_t &bytes) {
+    na = p.a_wide ? 1 : 2;
+    if (p.b_wide) nb = 1;
+    else if (g_token_kind(p.kind)) nb = (it.bn + 127) / 128;
+    else nb = (it.bn + 63) / 64;
+    const uint32_t bbox = p.b_wide ? (uint32_t)p.bn * 128u : g_token_kind(p.kind) ? 16384u : 8192u;
+    bytes = 16384u + bbox * (uint32_t)nb;
+}
+
 __device__ __forceinline__ void g_load(const GParams &p, const GMaps &mp, const GItem &it, int kc,
-                                       int j, unsigned char *stage, uint64_t *bar, uint64_t pol_a,
-                                       uint64_t pol_b) {
+                                       int j, int na, unsigned char *stage, uint64_t *bar,
+                                       uint64_t pol_a, uint64_t pol_b) {
     const int k = 64 * (kc + it.kc0);
-    if (j < 2) {
+    if (j < na) {
         unsigned char *dst = stage + 8192 * j;
         const int mn = it.mt * 128 + 64 * j;
         switch (p.kind) {
             case kDH:  // Wd[e] as [d][I]: rows are K
-                tma_load_3d(dst, &mp.m[it.a_sel], bar, mn, k, it.a_idx, pol_a);
+                if (p.a_wide) tma_load_4d(dst, &mp.m[it.a_sel], bar, 0, k, mn / 64, it.a_idx, pol_a);
+                else tma_load_3d(dst, &mp.m[it.a_sel], bar, mn, k, it.a_idx, pol_a);
                 break;
             case kDX: {  // Wg[e] then Wu[e], as [I][d]: rows are K
                 const int kh = p.I / 64;
                 const int sel = (kc < kh ? 0 : 2) + it.a_sel;
-                tma_load_3d(dst, &mp.m[sel], bar, mn, kc < kh ? k : k - p.I, it.a_idx, pol_a);
+                const int kk = kc < kh ? k : k - p.I;
+                if (p.a_wide) tma_load_4d(dst, &mp.m[sel], bar, 0, kk, mn / 64, it.a_idx, pol_a);
+                else tma_load_3d(dst, &mp.m[sel], bar, mn, kk, it.a_idx, pol_a);
                 break;
             }
             case kDWD:  // dy rows (dy_perm / dy) read across: rows are K
-                tma_load_2d(dst, &mp.m[it.b_sel], bar, mn, it.src_row0 + k, pol_a);
+                if (p.a_wide) tma_load_3d(dst, &mp.m[it.b_sel], bar, 0, it.src_row0 + k, mn / 64, pol_a);
+                else tma_load_2d(dst, &mp.m[it.b_sel], bar, mn, it.src_row0 + k, pol_a);
                 break;
             case kDWGU: {  // [g | u] rows read across
                 const int part = it.mt / p.m_tiles;
                 const int m0 = (it.mt - part * p.m_tiles) * 128 + 64 * j + part * p.I;
-                tma_load_2d(dst, &mp.m[0], bar, m0, it.dst_row0 + k, pol_a);
+                if (p.a_wide) tma_load_3d(dst, &mp.m[0], bar, 0, it.dst_row0 + k, m0 / 64, pol_a);
+                else tma_load_2d(dst, &mp.m[0], bar, m0, it.dst_row0 + k, pol_a);
                 break;
             }
             case kLOGITS:  // Wr rows, K-major
@@ -175,9 +200,10 @@ __device__ __forceinline__ void g_load(const GParams &p, const GMaps &mp, const 
                 break;
         }
     } else {
-        const int jb = j - 2;
-        unsigned char *dst = stage + 16384 + 8192 * jb;
-        const int r0 = it.nt * it.bn + 64 * jb;  // first N element of the box
+        const int jb = j - na;
+        const int brows = p.b_wide ? 256 : g_token_kind(p.kind) ? 128 : 64;
+        unsigned char *dst = stage + 16384 + brows * 128 * jb;
+        const int r0 = it.nt * it.bn + brows * jb;  // first N element of the copy
         switch (p.kind) {
             case kDH:  // dy rows, K-major
                 tma_load_2d(dst, &mp.m[2 + it.b_sel], bar, k, it.src_row0 + r0, pol_b);
@@ -186,10 +212,12 @@ __device__ __forceinline__ void g_load(const GParams &p, const GMaps &mp, const 
                 tma_load_2d(dst, &mp.m[4], bar, k, it.dst_row0 + r0, pol_b);
                 break;
             case kDWD:  // h rows read across
-                tma_load_2d(dst, &mp.m[2], bar, r0, it.dst_row0 + k, pol_b);
+                if (p.b_wide) tma_load_3d(dst, &mp.m[2], bar, 0, it.dst_row0 + k, r0 / 64, pol_b);
+                else tma_load_2d(dst, &mp.m[2], bar, r0, it.dst_row0 + k, pol_b);
                 break;
             case kDWGU:  // x rows (x_perm / x) read across
-                tma_load_2d(dst, &mp.m[2 + it.b_sel], bar, r0, it.src_row0 + k, pol_b);
+                if (p.b_wide) tma_load_3d(dst, &mp.m[2 + it.b_sel], bar, 0, it.src_row0 + k, r0 / 64, pol_b);
+                else tma_load_2d(dst, &mp.m[2 + it.b_sel], bar, r0, it.src_row0 + k, pol_b);
                 break;
             case kDWR:  // x read across
                 tma_load_2d(dst, &mp.m[1], bar, r0, k, pol_b);
@@ -466,8 +494,9 @@ __global__ void __launch_bounds__(kGThreads, 1) bwd_gemm_kernel(const __grid_con
         for (int q = blockIdx.x; q < total && ok; q += gridDim.x) {
             GItem it;
             g_decode(p, sh, q, it);
-            const int nbb = (it.bn + 63) / 64;
-            const uint32_t bytes = 16384u + 8192u * (uint32_t)nbb;
+            int na, nb;
+            uint32_t bytes;
+            g_copies(p, it, na, nb, bytes);
             for (int kc = 0; kc < it.nck; ++kc) {
                 int got = 1;
                 if (lane == 0) got = mbar_wait(&sh.empty[stage], phase ^ 1u, abort);
@@ -479,7 +508,8 @@ __global__ void __launch_bounds__(kGThreads, 1) bwd_gemm_kernel(const __grid_con
                     armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
                 }
                 __syncwarp();
-                if (lane < 2 + nbb) g_load(p, mp, it, kc, lane, sbase, &sh.full[stage], pol_a, pol_b);
+                if (lane < na + nb)
+                    g_load(p, mp, it, kc, lane, na, sbase, &sh.full[stage], pol_a, pol_b);
                 if (++stage == nst) { stage = 0; phase ^= 1u; }
             }
         }
@@ -619,11 +649,31 @@ __global__ void __launch_bounds__(kGThreads, 1) bwd_gemm_kernel(const __grid_con
 
 // ---------------------------------------------------------------------------
 // Host side.
-static bool g_rows(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows) {
+static bool g_rows(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows,
+                   uint32_t box_rows = 64) {
     const cuuint64_t dims[2] = {cols, rows};
     const cuuint64_t strides[1] = {cols * 2};
-    const cuuint32_t box[2] = {64, 64};
+    const cuuint32_t box[2] = {64, box_rows};
     return encode(m, base, 2, dims, strides, box);
+}
+// MN-major view of a row-major bf16 [rows][cols] matrix (cols % 64 == 0):
+// {64 columns, rows, cols / 64 column blocks}, the blocks 128 bytes apart; a
+// {64, 64, nblk} box lands nblk 64-column blocks of 64 rows one after
+// another, 8 KB apart
+static bool g_rows_mn(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows,
+                      uint32_t nblk) {
+    const cuuint64_t dims[3] = {64, rows, cols / 64};
+    const cuuint64_t strides[2] = {cols * 2, 128};
+    const cuuint32_t box[3] = {64, 64, nblk};
+    return encode(m, base, 3, dims, strides, box);
+}
+// the same view of [E][rows][cols] expert matrices: {64, rows, cols / 64, E}
+static bool g_experts_mn(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows,
+                         uint64_t E, uint32_t nblk) {
+    const cuuint64_t dims[4] = {64, rows, cols / 64, E};
+    const cuuint64_t strides[3] = {cols * 2, 128, cols * rows * 2};
+    const cuuint32_t box[4] = {64, 64, nblk, 1};
+    return encode(m, base, 4, dims, strides, box);
 }
 static bool g_experts(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint64_t E) {
     const cuuint64_t dims[3] = {cols, rows, E};
@@ -637,6 +687,16 @@ static void g_ntiles(int n, int &tiles, int &bn, int align = 16) {
     if (tiles < 1) tiles = 1;
     bn = (((n + tiles - 1) / tiles) + align - 1) / align * align;
     if (bn < align) bn = align;
+}
+// N tiles of 64-column blocks (a wide B copy starts on a block): the width
+// out of 256, 192, 128, 64 that covers n with the fewest columns (the widest
+// on a tie)
+static void g_ntiles64(int n, int &tiles, int &bn) {
+    int best = 0;
+    for (int w = 256; w >= 64; w -= 64) {
+        const int t = (n + w - 1) / w;
+        if (best == 0 || t * w < tiles * bn) { tiles = t; bn = w; best = 1; }
+    }
 }
 // bf16 [E][rows][cols] gradient written in [32 rows][32 cols] boxes (64-byte swizzle)
 static bool g_out(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint64_t E) {
@@ -684,8 +744,11 @@ cudaError_t launch_bwd_gemm(int kind, const moge_config &c, const ExpertWork *en
     int total = -1;  // unknown on the host (token kinds)
     switch (kind) {
         case kDH:
-            ok = g_experts(&mp.m[0], b.wd, I, d, N) && g_experts(&mp.m[1], sd, I, d, ns) &&
-                 g_rows(&mp.m[2], b.dy_perm, d, rrows) && g_rows(&mp.m[3], b.dy, d, T);
+            p.a_wide = I % 64 == 0;
+            ok = (p.a_wide ? g_experts_mn(&mp.m[0], b.wd, I, d, N, 2) &&
+                                 g_experts_mn(&mp.m[1], sd, I, d, ns, 2)
+                           : g_experts(&mp.m[0], b.wd, I, d, N) && g_experts(&mp.m[1], sd, I, d, ns)) &&
+                 g_rows(&mp.m[2], b.dy_perm, d, rrows, 128) && g_rows(&mp.m[3], b.dy, d, T, 128);
             mp.m[4] = mp.m[5] = mp.m[0];
             p.m_tiles = (I + 127) / 128;
             p.kc = (d + 63) / 64;
@@ -693,33 +756,51 @@ cudaError_t launch_bwd_gemm(int kind, const moge_config &c, const ExpertWork *en
             p.gu = (const uint16_t *)b.gu;
             break;
         case kDX:
-            ok = g_experts(&mp.m[0], b.wg, d, I, N) && g_experts(&mp.m[1], sg, d, I, ns) &&
-                 g_experts(&mp.m[2], b.wu, d, I, N) && g_experts(&mp.m[3], su, d, I, ns) &&
-                 g_rows(&mp.m[4], b.dgu, 2 * (uint64_t)I, hrows);
+            p.a_wide = d % 64 == 0;
+            ok = (p.a_wide ? g_experts_mn(&mp.m[0], b.wg, d, I, N, 2) &&
+                                 g_experts_mn(&mp.m[1], sg, d, I, ns, 2) &&
+                                 g_experts_mn(&mp.m[2], b.wu, d, I, N, 2) &&
+                                 g_experts_mn(&mp.m[3], su, d, I, ns, 2)
+                           : g_experts(&mp.m[0], b.wg, d, I, N) && g_experts(&mp.m[1], sg, d, I, ns) &&
+                                 g_experts(&mp.m[2], b.wu, d, I, N) &&
+                                 g_experts(&mp.m[3], su, d, I, ns)) &&
+                 g_rows(&mp.m[4], b.dgu, 2 * (uint64_t)I, hrows, 128);
             mp.m[5] = mp.m[0];
             p.m_tiles = (d + 127) / 128;
             p.kc = 2 * I / 64;
             p.out[0] = b.dx_perm;
             break;
         case kDWD:
-            ok = g_rows(&mp.m[0], b.dy_perm, d, rrows) && g_rows(&mp.m[1], b.dy, d, T) &&
-                 g_rows(&mp.m[2], b.h, I, hrows);
+            p.a_wide = d % 64 == 0;
+            p.b_wide = I % 64 == 0;
+            if (p.b_wide) g_ntiles64(I, p.n_tiles, p.bn);
+            else g_ntiles(I, p.n_tiles, p.bn, 32);
+            ok = (p.a_wide ? g_rows_mn(&mp.m[0], b.dy_perm, d, rrows, 2) &&
+                                 g_rows_mn(&mp.m[1], b.dy, d, T, 2)
+                           : g_rows(&mp.m[0], b.dy_perm, d, rrows) && g_rows(&mp.m[1], b.dy, d, T)) &&
+                 (p.b_wide ? g_rows_mn(&mp.m[2], b.h, I, hrows, (uint32_t)p.bn / 64)
+                           : g_rows(&mp.m[2], b.h, I, hrows));
             ok = ok && g_out(&mp.m[6], b.dwd, I, d, N) && g_out(&mp.m[7], S ? b.dsd : b.dwd, I, d, ns);
             mp.m[3] = mp.m[4] = mp.m[5] = mp.m[0];
             mp.m[8] = mp.m[9] = mp.m[6];
             p.m_tiles = (d + 127) / 128;
-            g_ntiles(I, p.n_tiles, p.bn, 32);
             p.out[0] = b.dwd; p.out[1] = b.dsd;
             total = n_entries * p.m_tiles * p.n_tiles;
             break;
         case kDWGU:
-            ok = g_rows(&mp.m[0], b.dgu, 2 * (uint64_t)I, hrows) &&
-                 g_rows(&mp.m[2], b.x_perm, d, rrows) && g_rows(&mp.m[3], b.x, d, T);
+            p.a_wide = I % 64 == 0;
+            p.b_wide = d % 64 == 0;
+            if (p.b_wide) g_ntiles64(d, p.n_tiles, p.bn);
+            else g_ntiles(d, p.n_tiles, p.bn, 32);
+            ok = (p.a_wide ? g_rows_mn(&mp.m[0], b.dgu, 2 * (uint64_t)I, hrows, 2)
+                           : g_rows(&mp.m[0], b.dgu, 2 * (uint64_t)I, hrows)) &&
+                 (p.b_wide ? g_rows_mn(&mp.m[2], b.x_perm, d, rrows, (uint32_t)p.bn / 64) &&
+                                 g_rows_mn(&mp.m[3], b.x, d, T, (uint32_t)p.bn / 64)
+                           : g_rows(&mp.m[2], b.x_perm, d, rrows) && g_rows(&mp.m[3], b.x, d, T));
             ok = ok && g_out(&mp.m[6], b.dwg, d, I, N) && g_out(&mp.m[7], S ? b.dsg : b.dwg, d, I, ns) &&
                  g_out(&mp.m[8], b.dwu, d, I, N) && g_out(&mp.m[9], S ? b.dsu : b.dwu, d, I, ns);
             mp.m[1] = mp.m[4] = mp.m[5] = mp.m[0];
             p.m_tiles = (I + 127) / 128;
-            g_ntiles(d, p.n_tiles, p.bn, 32);
             p.out[0] = b.dwg; p.out[1] = b.dsg; p.out[2] = b.dwu; p.out[3] = b.dsu;
             total = n_entries * 2 * p.m_tiles * p.n_tiles;
             break;
