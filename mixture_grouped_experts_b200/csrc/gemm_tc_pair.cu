@@ -50,7 +50,7 @@ namespace pair {
 
 constexpr int kStages = 6;
 constexpr int kStageBytes = 32 * 1024;  // one K-chunk: 16 KB of weights, <= 16 KB of token rows
-constexpr int kEpiBytes = 16 * 1024;  // U fp32 [32][64], H and G bf16 [32][64]
+constexpr int kEpiBytes = 16 * 1024;  // G and U fp32 [32][64] (up), Y bf16 [32][128] (down)
 constexpr int kTcThreads = 192;
 constexpr int kChunkK = 64;          // bf16 elements per K-chunk (128 bytes, one swizzle row)
 constexpr int kBoxRows = 64;         // token rows per TMA box (one 8 KB copy per chunk)
@@ -428,39 +428,41 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_pair_kernel(
                 tmem_ld_32x32b_x32(tbase + (uint32_t)c0, v);
                 tmem_ld_wait();
                 if (it.up) {
-                    float *U = reinterpret_cast<float *>(epi);                 // [32 cols][64 features]
-                    uint16_t *H = reinterpret_cast<uint16_t *>(epi + 8192);    // [32 cols][64 features]
+                    // the gate and up accumulators staged side by side (fp32), then
+                    // every thread forms h for 16 of the block's 2048 (column,
+                    // feature) pairs: the SwiGLU spread over all four warps, with the
+                    // fast exponential and division (half the warps doing all of it
+                    // held the accumulator up: the MMA thread waited for it)
+                    float *G = reinterpret_cast<float *>(epi);         // [32 cols][64 features]
+                    float *U = reinterpret_cast<float *>(epi + 8192);  // [32 cols][64 features]
                     // lanes 0-63 hold gate and 64-127 up, or the reverse for an up-first tile
                     const bool gate_hi = p.gu_mode[it.w.a_sel] == kUpGateFused;
-                    const bool is_gate = (q4 < 2) != gate_hi;
-                    uint16_t *G = reinterpret_cast<uint16_t *>(epi + 12288);  // [32 cols][64 features]
+                    float *D = ((q4 < 2) != gate_hi) ? G : U;
                     const int f = (q4 & 1) * 32 + lane;
-                    if (!is_gate) {
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) U[j * 64 + f] = __uint_as_float(v[j]);
-                    }
-                    named_bar_sync(1, 128);
-                    if (is_gate) {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const float g = __uint_as_float(v[j]);
-                            const float hv = g / (1.0f + expf(-g)) * U[j * 64 + f];
-                            H[j * 64 + f] = to_bf16_bits(hv);
-                            if (p.gu) G[j * 64 + f] = to_bf16_bits(g);
-                        }
-                    }
+                    for (int j = 0; j < 32; ++j) D[j * 64 + f] = __uint_as_float(v[j]);
                     named_bar_sync(1, 128);
                     for (int idx = et; idx < 32 * 8; idx += 128) {
                         const int r = idx >> 3, vv = idx & 7;
                         const int col = c0 + r, feat = tile * 64 + vv * 8;
                         if (col < it.n_valid && feat < p.I) {
+                            const float4 *g4 = reinterpret_cast<const float4 *>(G + r * 64 + vv * 8);
+                            const float4 *u4 = reinterpret_cast<const float4 *>(U + r * 64 + vv * 8);
+                            const float4 ga = g4[0], gb = g4[1], ua = u4[0], ub = u4[1];
+                            const float g8[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+                            const float u8[8] = {ua.x, ua.y, ua.z, ua.w, ub.x, ub.y, ub.z, ub.w};
+                            float h8[8];
+#pragma unroll
+                            for (int k = 0; k < 8; ++k)
+                                h8[k] = __fdividef(g8[k], 1.0f + __expf(-g8[k])) * u8[k];
                             *reinterpret_cast<uint4 *>(p.h + (row0 + col) * p.I + feat) =
-                                *reinterpret_cast<const uint4 *>(H + r * 64 + vv * 8);
+                                make_uint4(pack_bf16x2(h8[0], h8[1]), pack_bf16x2(h8[2], h8[3]),
+                                           pack_bf16x2(h8[4], h8[5]), pack_bf16x2(h8[6], h8[7]));
                             if (p.gu) {  // keep g and u (bf16) for the backward pass
                                 uint16_t *dst = p.gu + (row0 + col) * 2 * (size_t)p.I + feat;
                                 *reinterpret_cast<uint4 *>(dst) =
-                                    *reinterpret_cast<const uint4 *>(G + r * 64 + vv * 8);
-                                const float *u8 = U + r * 64 + vv * 8;
+                                    make_uint4(pack_bf16x2(g8[0], g8[1]), pack_bf16x2(g8[2], g8[3]),
+                                               pack_bf16x2(g8[4], g8[5]), pack_bf16x2(g8[6], g8[7]));
                                 *reinterpret_cast<uint4 *>(dst + p.I) =
                                     make_uint4(pack_bf16x2(u8[0], u8[1]), pack_bf16x2(u8[2], u8[3]),
                                                pack_bf16x2(u8[4], u8[5]), pack_bf16x2(u8[6], u8[7]));
