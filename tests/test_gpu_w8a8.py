@@ -7,7 +7,7 @@ both operands of every expert GEMM are E4M3 codes on the 8-bit tensor-core MMA.
   GPU layer must match under the usual rules: routing bit-exact above the
   1e-4 margin, outputs within 1e-2 normwise. This is checked at sizes that
   span several tiles with ragged K-chunks and token tails, and at the decode
-  workload on sampled tokens.
+  and prefill workloads on sampled tokens.
 * The two sides quantise x identically: bf16 inputs, an exact amax, an IEEE
   fp32 division and round-to-nearest-even.
 * h is computed in fp32 on the GPU and in fp64 rounded to fp32 in the oracle.
@@ -112,5 +112,16 @@ def test_layer_w8a8_decode_workload_sampled():
     cfg = synth.CONFIGS["decode"]
     inp = synth.layer_inputs(cfg)
     r = _w8a8_parity(cfg, inp, tokens=sample_tokens(cfg.T, 8, seed=5))
+    del r
+    torch.cuda.empty_cache()
+
+
+def test_layer_w8a8_prefill_workload_sampled():
+    """The prefill workload (T = 4096: about 512 rows per routed expert in two
+    256-row token tiles, 16 tiles per shared expert, quantisation items over
+    ~190 tiles) on sampled tokens."""
+    cfg = synth.CONFIGS["prefill"]
+    inp = synth.layer_inputs(cfg)
+    r = _w8a8_parity(cfg, inp, tokens=sample_tokens(cfg.T, 6, seed=6))
     del r
     torch.cuda.empty_cache()
