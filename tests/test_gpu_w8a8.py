@@ -6,8 +6,8 @@ both operands of every expert GEMM are E4M3 codes on the 8-bit tensor-core MMA.
   W8A8 layer in fp64 (x and h quantised per token with the same rule). The
   GPU layer must match under the usual rules: routing bit-exact above the
   1e-4 margin, outputs within 1e-2 normwise. This is checked at sizes that
-  span several tiles with ragged K-chunks and token tails, and at the decode
-  and prefill workloads on sampled tokens.
+  span several tiles with ragged K-chunks and token tails, above 8192 routed
+  rows too, and at the decode and prefill workloads on sampled tokens.
 * The two sides quantise x identically: bf16 inputs, an exact amax, an IEEE
   fp32 division and round-to-nearest-even.
 * h is computed in fp32 on the GPU and in fp64 rounded to fp32 in the oracle.
@@ -38,6 +38,9 @@ CASES = {
     "s0": MED.replace(name="a8s0", T=50, S=0, seed=45),               # no shared expert
     "big": MED.replace(name="a8big", T=1100, N=8, M=2, S=1, seed=46),  # > 256 rows per expert
     "i16": MED.replace(name="a8i16", T=96, d=256, I=16, seed=47),     # one partial K-chunk of h
+    # above 8192 routed rows (where the bf16 layer takes the CTA-pair kernel)
+    "pair": MED.replace(name="a8pair", T=1100, M=8, seed=51),
+    "pair_odd": MED.replace(name="a8pairodd", T=1040, M=8, d=528, I=336, seed=52),
 }
 
 
