@@ -45,9 +45,10 @@ NOMINAL = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 # DRAM traffic of the dominant kernel comes from an ncu capture summarised
 # under profiles/: a line "traffic-record: {json}" there names the kernel, the
 # workload, the DRAM bytes of one launch (dram__bytes_read.sum +
-# dram__bytes_write.sum) and a hash of the CUDA sources the capture ran. The
-# bench reports it only while the sources still hash the same (else null: the
-# kernel changed since the counters were taken).
+# dram__bytes_write.sum) and a hash of the code (comments left out) of the
+# CUDA sources the capture ran. The bench reports it only while the sources
+# still hash the same (else null: the kernel changed since the counters were
+# taken).
 TRAFFIC_RECORDS = ("profiles/ffn_tc_decode.md", "profiles/ffn_tc_pair_prefill.md",
                    "profiles/ffn_tc_w8a8_decode.md")
 FFN_PAIR_KERNEL = ("ffn_tc_pair_kernel (the same grouped FFN on CTA pairs, 2-SM tcgen05 MMA, "
@@ -56,10 +57,37 @@ FFN_W8A8_KERNEL = ("ffn_tc_kernel<W8> (the single-SM grouped FFN on 8-bit operan
                    "kind::f8f6f4, h quantised per token between the projections, one launch)")
 
 
+def code_of(text):
+    """C / CUDA source without its comments and with runs of white space
+    collapsed: what the compiler sees, so that editing a comment does not
+    change a source's hash. String and character literals are kept as they
+    are (a // inside one is not a comment)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            out.append(" ")
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def source_sha16(files=None):
-    """Hash of CUDA sources of the library: the listed files of csrc/ (or all
-    of csrc/*.cu, *.cuh, *.h and the ABI header when None), the key under
-    which a traffic record is valid."""
+    """Hash of the code (comments left out, code_of) of CUDA sources of the
+    library: the listed files of csrc/ (or all of csrc/*.cu, *.cuh, *.h and
+    the ABI header when None), the key under which a traffic record is valid."""
     import glob
     import hashlib
     h = hashlib.sha256()
@@ -71,7 +99,7 @@ def source_sha16(files=None):
         paths = [os.path.join(csrc, f) for f in files]
     for f in paths:
         h.update(os.path.basename(f).encode())
-        h.update(open(f, "rb").read())
+        h.update(code_of(open(f, encoding="utf-8").read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -10,10 +10,12 @@
 //   warp 1    MMA issuer   (tcgen05.mma kind::f16, M = 128, N = token tile,
 //                           fp32 accumulators in TMEM, double-buffered)
 //   warps 2-5 epilogue     (tcgen05.ld -> registers -> smem -> coalesced
-//                           16-byte global stores, rows masked per expert)
+//                           16-byte global stores, rows masked per expert;
+//                           W8: warps 2-9, two per TMEM lane quarter)
+//   warps 10-13 (W8 only)  h quantisers, on a queue of their own
 //
 // The queue hands out every up-projection item before any down-projection
-// item (W8: with the quantisation items between them), shared experts first (the heaviest items go first, the tail is made
+// item, shared experts first (the heaviest items go first, the tail is made
 // of small ones). A down-projection item of an expert waits -- bounded -- until
 // all up-projection items of that expert have stored their h rows (a per-
 // expert counter), so no kernel boundary separates the two phases. Every item
@@ -40,13 +42,16 @@
 // scales are applied in the epilogue: the weight row's scale per accumulator
 // lane and the token's scale per column. Each row of h needs its own scale,
 // which depends on all of the row's I features, so the up-projection items
-// store h in fp32 and fold each row's amax into a global word. The queue then
-// hands out quantisation items between the two projections: kQParts row
-// slices per token tile, each run by a CTA's epilogue warps once the expert's
-// up items are all done, each counting once more on the expert's counter. The
-// expert's down-projection items wait for those counts too. (Quantising a whole
-// expert in the CTA that finished its last up item chained: that CTA's delayed
-// items made it the last finisher of the next expert, and so on.)
+// store h in fp32 and fold each row's amax into a global word. Quantisation
+// items -- kQParts row slices per token tile -- come from a second queue and
+// run on four quantiser warps per CTA beside the GEMM roles, each once the
+// expert's up items are all done, each counting once more on the expert's
+// counter; the expert's down-projection items wait for those counts too. (Run
+// by the CTA that finished an expert's last up item, quantisation chained:
+// that CTA's delayed items made it the last finisher of the next expert, and
+// so on; run on the epilogue warps, it stalled the GEMM pipeline.) The 8-bit
+// MMA halves an item's time, so the W8 epilogue has eight warps and spreads
+// the SwiGLU over all of them.
 //
 // The grouped expert GEMM ("GroupMatmul") of the Pangu Pro MoE article
 // (techwalker.com, section 3) and its SwiftGMM GEMV/GEMM switch (reportify.cn
