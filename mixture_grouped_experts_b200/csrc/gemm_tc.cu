@@ -195,7 +195,7 @@ __device__ __forceinline__ uint32_t e4m3x4_div(float4 f, float s) {
 // W8: quantise rows row0 + first, row0 + first + step, ... (tile-relative
 // indices < n) of h (fp32 [.][I], I % 16 == 0), each with its own scale:
 // amax / 448 (IEEE fp32 division; 1 for an all-zero row), code = E4M3 of
-// fp32(h / scale). The 128 epilogue threads (et) take four rows at a time,
+// fp32(h / scale). The 128 quantiser threads (et) take four rows at a time,
 // every thread loading its vectors of all four before converting any. h and
 // the amax words were written by other CTAs: read through L2 only.
 __device__ void quantize_h_rows(const W8Params &w8, int I, size_t row0, int first, int step, int n,
