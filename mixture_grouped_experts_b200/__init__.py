@@ -247,8 +247,17 @@ def moge_combine(s: LayerShape, y_perm, topk_w, perm_dst, y_shared=None, residua
     return y
 
 
+def _need_workspace(workspace, nbytes: int, what: str):
+    """A torch workspace smaller than the call needs is refused on the host
+    (the C ABI takes a bare pointer and cannot check its size)."""
+    if isinstance(workspace, torch.Tensor) and workspace.numel() * workspace.element_size() < nbytes:
+        raise MogeError(ERR_INVALID_ARG, "workspace of %d bytes, %s needs %d" % (
+            workspace.numel() * workspace.element_size(), what, nbytes))
+
+
 def moge_layer_forward(s: LayerShape, x, w: dict, workspace, residual=None, y=None, stream=None):
     """w: dict with w_router, logit_bias (or None), w_gate, w_up, w_down, s_gate, s_up, s_down."""
+    _need_workspace(workspace, workspace_size(s), "moge_layer_forward")
     if y is None:
         y = torch.empty((s.T, s.d), dtype=x.dtype, device=x.device)
     _chk(lib().moge_layer_forward(ctypes.byref(_cfg(s)), _p(x), _p(w["w_router"]),
@@ -261,6 +270,7 @@ def moge_layer_forward(s: LayerShape, x, w: dict, workspace, residual=None, y=No
 
 def moge_layer_forward_train(s: LayerShape, x, w: dict, workspace, y=None, stream=None):
     """Forward that keeps what moge_layer_backward needs in `workspace` (a training workspace)."""
+    _need_workspace(workspace, train_workspace_size(s), "moge_layer_forward_train")
     if y is None:
         y = torch.empty((s.T, s.d), dtype=x.dtype, device=x.device)
     _chk(lib().moge_layer_forward_train(ctypes.byref(_cfg(s)), _p(x), _p(w["w_router"]),
@@ -279,6 +289,7 @@ def moge_layer_backward(s: LayerShape, x, w: dict, dy, workspace, alpha: float =
     """Gradients for the preceding moge_layer_forward_train on the same workspace.
     Returns (dx, grads) with grads keyed like the weights (GRAD_KEYS); `aux` (a
     device float32 tensor of one element, optional) receives the balance loss."""
+    _need_workspace(workspace, train_workspace_size(s), "moge_layer_backward")
     if dx is None:
         dx = torch.empty_like(x)
     if grads is None:
@@ -581,6 +592,7 @@ def moge_layer_forward_fp8(s: LayerShape, x, w: dict, w8: dict, workspace, resid
                            stream=None):
     """Layer with FP8 expert weights w8 (experts_to_fp8 form); w gives w_router
     and logit_bias."""
+    _need_workspace(workspace, workspace_size(s), "moge_layer_forward_fp8")
     if y is None:
         y = torch.empty((s.T, s.d), dtype=x.dtype, device=x.device)
     routed, shared = _fp8_side(w8, "w"), _fp8_side(w8, "s")
@@ -608,6 +620,7 @@ def moge_layer_forward_w8a8(s: LayerShape, x, w: dict, w8: dict, workspace, resi
     """Layer in W8A8: FP8 expert weights w8 (experts_to_fp8 form) and
     activations quantised per token inside the call; w gives w_router and
     logit_bias; workspace of w8a8_workspace_size bytes."""
+    _need_workspace(workspace, w8a8_workspace_size(s), "moge_layer_forward_w8a8")
     if y is None:
         y = torch.empty((s.T, s.d), dtype=x.dtype, device=x.device)
     routed, shared = _fp8_side(w8, "w"), _fp8_side(w8, "s")

@@ -6,6 +6,7 @@ import re
 import subprocess
 
 import pytest
+import torch
 
 import mixture_grouped_experts_b200 as mg
 from mixture_grouped_experts_b200 import build as mbuild
@@ -146,6 +147,19 @@ def test_w8a8_entry_points_validate_on_host(L):
     rc = L.moge_layer_forward_w8a8(ctypes.byref(mg._cfg(s)), 0x7000, 0x8000, None,
                                    ctypes.byref(f8), ctypes.byref(f8), None, 0x9000, None, None)
     assert rc == mg.ERR_INVALID_ARG and b"workspace" in L.moge_last_error()
+
+
+def test_undersized_workspace_refused_before_the_call(L):
+    # the C ABI cannot see a workspace's size; the binding checks torch ones
+    s = _shape(dtype="bf16")
+    small = torch.empty(mg.workspace_size(s), dtype=torch.uint8)   # the plain layer's size
+    w8 = {k: None for k in mg.FP8_KEYS}
+    with pytest.raises(mg.MogeError, match="moge_layer_forward_w8a8 needs"):
+        mg.moge_layer_forward_w8a8(s, None, {}, w8, small)
+    with pytest.raises(mg.MogeError, match="moge_layer_forward needs"):
+        mg.moge_layer_forward(s, None, {}, small[:-1])
+    with pytest.raises(mg.MogeError, match="moge_layer_backward needs"):
+        mg.moge_layer_backward(s, None, {}, None, small)
 
 
 def test_wait_selftest_validates_on_host(L):
