@@ -735,16 +735,20 @@ static int check_fp8_side(const moge_fp8_experts *e, const char *side) {
     return MOGE_OK;
 }
 
-int moge_layer_forward_fp8(const moge_config *cfg, const void *x, const void *w_router,
-                           const float *logit_bias, const moge_fp8_experts *routed,
-                           const moge_fp8_experts *shared, const void *residual, void *y,
-                           void *workspace, void *stream) {
+// The two 8-bit layers share their host checks and operands: E4M3 expert
+// weights with one fp32 scale per row, bf16 x and y.
+static int forward_8bit(const moge_config *cfg, const void *x, const void *w_router,
+                        const float *logit_bias, const moge_fp8_experts *routed,
+                        const moge_fp8_experts *shared, const void *residual, void *y,
+                        void *workspace, void *stream, LayerMode mode) {
     int rc = check_config(cfg);
     if (rc) return rc;
     const moge_config c = *cfg;
-    if (c.dtype != MOGE_BF16) return fail(MOGE_ERR_UNSUPPORTED, "fp8 experts need dtype MOGE_BF16");
+    const char *what = mode == kModeW8A8 ? "W8A8 needs" : "fp8 experts need";
+    if (c.dtype != MOGE_BF16)
+        return fail(MOGE_ERR_UNSUPPORTED, std::string(what) + " dtype MOGE_BF16");
     if (c.d % 16 != 0 || c.I % 16 != 0)
-        return fail(MOGE_ERR_UNSUPPORTED, "fp8 experts need d % 16 == 0 and I % 16 == 0");
+        return fail(MOGE_ERR_UNSUPPORTED, std::string(what) + " d % 16 == 0 and I % 16 == 0");
     if (c.T == 0) return MOGE_OK;
     MOGE_NEED(x, "x");
     MOGE_NEED(w_router, "w_router");
@@ -762,8 +766,16 @@ int moge_layer_forward_fp8(const moge_config *cfg, const void *x, const void *w_
         op.sg = shared->gate; op.su = shared->up; op.sd = shared->down;
         op.sg_s = shared->gate_scale; op.su_s = shared->up_scale; op.sd_s = shared->down_scale;
     }
-    return layer_run(c, x, w_router, logit_bias, op, kModeFp8Weights, residual, y, workspace,
+    return layer_run(c, x, w_router, logit_bias, op, mode, residual, y, workspace,
                      (cudaStream_t)stream);
+}
+
+int moge_layer_forward_fp8(const moge_config *cfg, const void *x, const void *w_router,
+                           const float *logit_bias, const moge_fp8_experts *routed,
+                           const moge_fp8_experts *shared, const void *residual, void *y,
+                           void *workspace, void *stream) {
+    return forward_8bit(cfg, x, w_router, logit_bias, routed, shared, residual, y, workspace,
+                        stream, kModeFp8Weights);
 }
 
 size_t moge_w8a8_workspace_size(const moge_config *cfg) {
@@ -775,31 +787,8 @@ int moge_layer_forward_w8a8(const moge_config *cfg, const void *x, const void *w
                             const float *logit_bias, const moge_fp8_experts *routed,
                             const moge_fp8_experts *shared, const void *residual, void *y,
                             void *workspace, void *stream) {
-    int rc = check_config(cfg);
-    if (rc) return rc;
-    const moge_config c = *cfg;
-    if (c.dtype != MOGE_BF16) return fail(MOGE_ERR_UNSUPPORTED, "W8A8 needs dtype MOGE_BF16");
-    if (c.d % 16 != 0 || c.I % 16 != 0)
-        return fail(MOGE_ERR_UNSUPPORTED, "W8A8 needs d % 16 == 0 and I % 16 == 0");
-    if (c.T == 0) return MOGE_OK;
-    MOGE_NEED(x, "x");
-    MOGE_NEED(w_router, "w_router");
-    if ((rc = check_fp8_side(routed, "routed"))) return rc;
-    if (c.S > 0 && (rc = check_fp8_side(shared, "shared"))) return rc;
-    if (logit_bias && !aligned4(logit_bias)) return fail(MOGE_ERR_UNSUPPORTED, "logit_bias misaligned");
-    if (residual && !aligned16(residual)) return fail(MOGE_ERR_UNSUPPORTED, "residual misaligned");
-    MOGE_NEED(y, "y");
-    MOGE_NEED(workspace, "workspace");
-    if (y == x) return fail(MOGE_ERR_INVALID_ARG, "y must not alias x");
-    FfnOperands op{};
-    op.wg = routed->gate; op.wu = routed->up; op.wd = routed->down;
-    op.wg_s = routed->gate_scale; op.wu_s = routed->up_scale; op.wd_s = routed->down_scale;
-    if (c.S > 0) {
-        op.sg = shared->gate; op.su = shared->up; op.sd = shared->down;
-        op.sg_s = shared->gate_scale; op.su_s = shared->up_scale; op.sd_s = shared->down_scale;
-    }
-    return layer_run(c, x, w_router, logit_bias, op, kModeW8A8, residual, y, workspace,
-                     (cudaStream_t)stream);
+    return forward_8bit(cfg, x, w_router, logit_bias, routed, shared, residual, y, workspace,
+                        stream, kModeW8A8);
 }
 
 int moge_stage_timing(int enable) {
