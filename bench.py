@@ -660,7 +660,7 @@ def job_throughput(tokens_per_rank, world, max_ms):
     return world * tokens_per_rank / (max_ms / 1e3)
 
 
-def main():
+def arg_parser() -> argparse.ArgumentParser:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
@@ -681,7 +681,11 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=2, help="tokens per step of --impl reference")
     ap.add_argument("--ep", action="store_true",
                     help="expert parallelism over the ranks instead of independent replicas")
-    args = ap.parse_args()
+    return ap
+
+
+def main():
+    args = arg_parser().parse_args()
     cfg = synth.CONFIGS[args.config]
     if args.impl == "reference":
         run_reference(args, cfg)
