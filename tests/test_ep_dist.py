@@ -158,3 +158,20 @@ def test_gloo_ranks_pipelined_chunks(world, chunks):
         assert out[r]["bounds"] == want
         assert out[r]["seen"] == [world * (b - a) for a, b in want]
         assert out[r]["err"] <= 1e-12, out[r]
+
+
+def test_chunk_bounds_partition_every_rank_alike():
+    """The chunks cover a rank's rows in order, without gaps or empty chunks,
+    their sizes differ by at most one, and more chunks than rows are clipped;
+    decode-sized batches stay one chunk."""
+    for rows in (0, 1, 2, 7, 8, 100, 457):
+        for chunks in (1, 2, 3, 4, 9, 1000):
+            b = mg.ep_chunk_bounds(rows, chunks)
+            assert len(b) == (max(1, min(chunks, rows)) if rows else 1)
+            assert b[0][0] == 0 and b[-1][1] == rows
+            assert all(b[j][1] == b[j + 1][0] for j in range(len(b) - 1))
+            sizes = [hi - lo for lo, hi in b]
+            assert max(sizes) - min(sizes) <= 1
+            assert rows == 0 or min(sizes) >= 1
+    assert [mg.ep_default_chunks(r) for r in (1, 456, 511, 512, 767, 768, 1024, 4096)] == \
+        [1, 1, 1, 2, 2, 3, 4, 4]
