@@ -17,6 +17,7 @@ import torch
 
 import mixture_grouped_experts_b200 as mg
 import oracle
+import oracle_par
 import synth
 
 MARGIN = 1e-4
@@ -87,20 +88,14 @@ def sample_tokens(T, n, seed=0):
 
 
 # ------------------------------------------------------------------ oracle pool
-# The oracle is single-threaded; full-size checks of hundreds of tokens run it
-# in worker processes. Workers are started with "spawn" (never forked from a
-# process that has touched the GPU) and regenerate the seeded inputs of the
-# config themselves, so only token lists and results cross the pipe.
+# The oracle is single-threaded. Layer outputs of many tokens are spread over
+# host threads (oracle_par); the backward's token terms run in worker
+# processes, started with "spawn" (never forked from a process that has
+# touched the GPU), which regenerate the seeded inputs of the config
+# themselves, so only token lists and results cross the pipe.
 def _pool_workers():
     import os
     return max(1, min(8, (os.cpu_count() or 2) // 2))
-
-
-def _oracle_layer_job(args):
-    cfg, tokens = args
-    inp = synth.layer_inputs(cfg)
-    xd = oracle.to_double(inp["x"], cfg.dtype)
-    return oracle.layer(xd, inp, cfg.M, cfg.Kp, cfg.dtype, tokens=tokens)[0]
 
 
 def _oracle_backward_job(args):
@@ -115,16 +110,6 @@ def _oracle_backward_job(args):
 def _split(tokens, n):
     tokens = np.asarray(tokens, dtype=np.int64)
     return [c for c in np.array_split(tokens, n) if len(c)]
-
-
-def oracle_layer_pool(cfg, tokens):
-    """oracle.layer outputs of the listed tokens of the seeded config `cfg`
-    (its unmodified synth inputs), computed in spawned worker processes."""
-    import multiprocessing as mp
-    chunks = _split(tokens, min(_pool_workers(), max(1, len(tokens) // 4)))
-    with mp.get_context("spawn").Pool(len(chunks)) as pool:
-        parts = pool.map(_oracle_layer_job, [(cfg, c) for c in chunks])
-    return np.concatenate(parts, axis=0)
 
 
 def oracle_backward_pool(cfg, alpha, idx, tokens):
@@ -179,8 +164,7 @@ def layer_parity(cfg, inp, n_sample=None, tokens=None, by_tiles=None):
     sampled tokens (all tokens when n_sample is None and tokens is None).
     by_tiles (a function of (perm_src, offsets, counts) returning tokens):
     more tokens chosen from the GPU's own dispatch, every token of whole token
-    tiles; they are run through the oracle in worker processes, which needs
-    `inp` to be the config's unmodified seeded inputs."""
+    tiles, run through the oracle on host threads."""
     x, w = device_inputs(cfg, inp)
     ws = mg.alloc_workspace(mg.shape_of(cfg))
     y, idx_g, w_g, counts_g, offsets_g = run_layer(cfg, x, w, ws)
@@ -192,13 +176,14 @@ def layer_parity(cfg, inp, n_sample=None, tokens=None, by_tiles=None):
     if tokens is None:
         tokens = np.arange(cfg.T) if n_sample is None else sample_tokens(cfg.T, n_sample)
     tokens = np.array([t for t in tokens if safe[t]], dtype=np.int64)
-    y_ref, _, _, _ = oracle.layer(xd, inp, cfg.M, cfg.Kp, cfg.dtype, tokens=tokens)
+    y_ref, _, _, _ = oracle_par.layer(xd, inp, cfg.M, cfg.Kp, cfg.dtype, tokens=tokens)
     if by_tiles is not None:
         ps = oracle.dispatch(idx_g, cfg.N)[2]
         extra = sorted(set(int(t) for t in by_tiles(ps, offsets_g, counts_g)
                            if safe[t]) - set(tokens.tolist()))
         if extra:
-            y_ref = np.concatenate([y_ref, oracle_layer_pool(cfg, extra)], axis=0)
+            y_ref = np.concatenate([y_ref, oracle_par.layer(xd, inp, cfg.M, cfg.Kp, cfg.dtype,
+                                                            tokens=extra)[0]], axis=0)
             tokens = np.concatenate([tokens, np.array(extra, dtype=np.int64)])
     y_g = to_host_f64(y)[tokens]
     err = normwise_err(y_g, y_ref)

@@ -16,6 +16,7 @@ import torch
 
 import mixture_grouped_experts_b200 as mg
 import oracle
+import oracle_par
 import synth
 from gpu_helpers import (TOL, check_counts, check_routing, device_inputs, normwise_err,
                          sample_tokens, to_host_f64, x_double)
@@ -58,7 +59,7 @@ def _fp8_parity(cfg, inp, tokens=None):
     s = mg.shape_of(cfg)
     ws = mg.alloc_workspace(s)
     w8 = mg.experts_to_fp8(w)
-    q_o = oracle.quantize_experts_fp8(inp)
+    q_o = oracle_par.quantize_experts_fp8(inp)
     for k in mg.FP8_KEYS:                       # the oracle quantised the same weights alike
         if inp[k].size:
             assert np.array_equal(w8[k].cpu().numpy(), q_o[k]), k
@@ -76,7 +77,7 @@ def _fp8_parity(cfg, inp, tokens=None):
     if tokens is None:
         tokens = np.arange(cfg.T)
     tokens = np.array([t for t in tokens if safe[t]], dtype=np.int64)
-    y_ref, _, _, _ = oracle.layer_fp8(xd, inp, q_o, cfg.M, cfg.Kp, cfg.dtype, tokens=tokens)
+    y_ref, _, _, _ = oracle_par.layer_fp8(xd, inp, q_o, cfg.M, cfg.Kp, cfg.dtype, tokens=tokens)
     err = normwise_err(to_host_f64(y)[tokens], y_ref)
     assert err <= TOL["bf16"], (cfg.name, err)
     return dict(err=err, y=y, x=x, w=w, w8=w8, ws=ws, s=s)

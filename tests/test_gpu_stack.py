@@ -27,6 +27,7 @@ import torch
 
 import mixture_grouped_experts_b200 as mg
 import oracle
+import oracle_par
 import synth
 from gpu_helpers import MARGIN, TOL, normwise_err, to_host_f64
 
@@ -67,7 +68,7 @@ def test_stack12_teacher_forced_and_end_to_end():
         p_all.append(p)
         # teacher forcing on two tokens per layer
         tf = np.array([(37 * l + 11) % cfg.T, (91 * l + 5) % cfg.T])
-        y_ref, idx_ref, _, mg_ref = oracle.layer(u_h, inp, cfg.M, cfg.Kp, "bf16", tokens=tf)
+        y_ref, idx_ref, _, mg_ref = oracle_par.layer(u_h, inp, cfg.M, cfg.Kp, "bf16", tokens=tf)
         yg = to_host_f64(y_only)[tf]
         for j, t in enumerate(tf):
             if mg_ref[j] > MARGIN:
@@ -84,7 +85,7 @@ def test_stack12_teacher_forced_and_end_to_end():
     for l in range(cfg.layers):                   # pass 2: the oracle's fp64 stack
         inp = synth.layer_inputs(cfg, layer=l, with_x=False)
         uo = oracle.rmsnorm(xo, 1e-6)
-        yo, idx_o, _, mg_o = oracle.layer(uo, inp, cfg.M, cfg.Kp, "bf16")
+        yo, idx_o, _, mg_o = oracle_par.layer(uo, inp, cfg.M, cfg.Kp, "bf16")
         drift = np.abs(oracle.router_probs(uo, inp["w_router"], None, "bf16") - p_all[l][cand])
         idx_g = idx_all[l][cand]
         for j in range(len(cand)):
