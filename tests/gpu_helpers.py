@@ -88,42 +88,23 @@ def sample_tokens(T, n, seed=0):
 
 
 # ------------------------------------------------------------------ oracle pool
-# The oracle is single-threaded. Layer outputs of many tokens are spread over
-# host threads (oracle_par); the backward's token terms run in worker
-# processes, started with "spawn" (never forked from a process that has
-# touched the GPU), which regenerate the seeded inputs of the config
-# themselves, so only token lists and results cross the pipe.
+# The oracle is single-threaded; full-size checks spread its tokens over host
+# threads (oracle_par), whose ctypes calls run at once.
 def _pool_workers():
     import os
     return max(1, min(8, (os.cpu_count() or 2) // 2))
 
 
-def _oracle_backward_job(args):
-    cfg, alpha, idx, tokens = args
-    inp = synth.layer_inputs(cfg)
-    xd = oracle.to_double(inp["x"], cfg.dtype)
-    dy = oracle.to_double(synth.upstream_grad(cfg), cfg.dtype)
-    return oracle.layer_backward(xd, inp, cfg.M, cfg.Kp, cfg.dtype, dy, alpha, idx=idx,
-                                 tokens=tokens, routed_weights=False)
-
-
-def _split(tokens, n):
-    tokens = np.asarray(tokens, dtype=np.int64)
-    return [c for c in np.array_split(tokens, n) if len(c)]
-
-
 def oracle_backward_pool(cfg, alpha, idx, tokens):
     """oracle.layer_backward of the seeded config `cfg` at the picks idx,
     without the routed experts' weight gradients: the token terms are split
-    over spawned workers and summed (every gradient is a sum over tokens; the
+    over host threads and summed (every gradient is a sum over tokens; the
     balance loss's f comes from the whole batch in each part)."""
-    import multiprocessing as mp
-    chunks = _split(tokens, _pool_workers())
-    with mp.get_context("spawn").Pool(len(chunks)) as pool:
-        parts = pool.map(_oracle_backward_job, [(cfg, alpha, idx, c) for c in chunks])
-    out = {k: sum(p[k] for p in parts) for k in parts[0] if k != "aux"}
-    out["aux"] = parts[0]["aux"]
-    return out
+    inp = synth.layer_inputs(cfg)
+    xd = oracle.to_double(inp["x"], cfg.dtype)
+    dy = oracle.to_double(synth.upstream_grad(cfg), cfg.dtype)
+    return oracle_par.layer_backward_sum(xd, inp, cfg.M, cfg.Kp, cfg.dtype, dy, alpha, idx,
+                                         tokens, _pool_workers())
 
 
 def expert_tiles(rows, max_tile=256, stream_rows=64):

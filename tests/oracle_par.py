@@ -72,3 +72,19 @@ def quantize_experts_fp8(inp: dict) -> dict:
         else:   # no expert of this kind (S = 0)
             out[k], out[k + "_scale"] = oracle.quantize_rows_fp8(inp[k])
     return out
+
+
+def layer_backward_sum(x, inp, M, Kp, dtype, dy, alpha, idx, tokens, parts):
+    """oracle.layer_backward without the routed experts' weight gradients,
+    its token terms split into `parts` lists on threads and summed in list
+    order (every gradient is a sum over tokens; the balance loss's batch
+    shares come from the whole batch in every part, so aux is part 0's)."""
+    toks = _tokens(x, tokens)
+    chunks = [c for c in np.array_split(toks, max(1, min(parts, len(toks)))) if len(c)] or [toks]
+    with ThreadPoolExecutor(len(chunks)) as ex:
+        outs = list(ex.map(lambda c: oracle.layer_backward(x, inp, M, Kp, dtype, dy, alpha,
+                                                           idx=idx, tokens=c,
+                                                           routed_weights=False), chunks))
+    out = {k: sum(o[k] for o in outs) for k in outs[0] if k != "aux"}
+    out["aux"] = outs[0]["aux"]
+    return out

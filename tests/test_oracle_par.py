@@ -34,3 +34,21 @@ def test_threaded_quantiser_without_shared_experts():
     inp = synth.layer_inputs(cfg)
     q, q2 = oracle.quantize_experts_fp8(inp), oracle_par.quantize_experts_fp8(inp)
     assert sorted(q) == sorted(q2) and _same([q[k] for k in sorted(q)], [q2[k] for k in sorted(q)])
+
+
+def test_threaded_backward_sum_equals_one_oracle_call():
+    """The token terms summed part by part equal one call over all tokens, up
+    to the order of the sums; each part's aux is the whole batch's."""
+    inp = synth.layer_inputs(CFG)
+    xd = oracle.to_double(inp["x"], CFG.dtype)
+    dy = oracle.to_double(synth.upstream_grad(CFG), CFG.dtype)
+    one = oracle.layer_backward(xd, inp, CFG.M, CFG.Kp, CFG.dtype, dy, 0.01, routed_weights=False)
+    idx = oracle.route(xd, inp["w_router"], inp["logit_bias"], CFG.dtype, CFG.M, CFG.Kp)[0]
+    for parts in (1, 3, 8):
+        got = oracle_par.layer_backward_sum(xd, inp, CFG.M, CFG.Kp, CFG.dtype, dy, 0.01, idx,
+                                            None, parts)
+        assert sorted(got) == sorted(one)
+        assert got["aux"] == one["aux"]
+        for k in one:
+            if k != "aux":
+                assert np.allclose(got[k], one[k], rtol=0, atol=1e-12 * np.abs(one[k]).max()), k
