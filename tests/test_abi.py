@@ -60,6 +60,21 @@ def test_workspace_size_matches_layout(L):
     assert mg.workspace_size(_shape(T=0)) > 0
 
 
+def test_w8a8_workspace_is_the_forward_workspace_plus_its_regions(L):
+    """The W8A8 workspace: the forward workspace, then x's codes [T][d] bytes,
+    the token scales [T] and [T*K] fp32, h in fp32 [T(K+S)][I], its row amax
+    words and row scales [T(K+S)], every region 256-byte aligned (at least
+    one 256-byte slot each, even when empty)."""
+    a256 = lambda n: (max(n, 1) + 255) // 256 * 256
+    for kw in (dict(), dict(T=1), dict(T=0), dict(T=456, d=5120, N=64, M=8, S=4, I=1344),
+               dict(Kp=2, S=0, I=336, d=528)):
+        s = _shape(dtype="bf16", **kw)
+        K, hrows = s.M * s.Kp, s.T * (s.M * s.Kp + s.S)
+        want = (mg.workspace_size(s) + a256(s.T * s.d) + a256(s.T * 4) + a256(s.T * K * 4)
+                + a256(hrows * s.I * 4) + 2 * a256(hrows * 4))
+        assert mg.w8a8_workspace_size(s) == want, kw
+
+
 @pytest.mark.parametrize("kw,code", [
     (dict(N=15), mg.ERR_UNSUPPORTED),               # N % M != 0
     (dict(Kp=5), mg.ERR_UNSUPPORTED),               # Kp > N/M
