@@ -33,6 +33,19 @@ def test_header_declares_the_boundary():
     assert set(names) == set(mg.EXPORTS)
 
 
+def test_boundary_calls_cite_their_passage():
+    """Each piecewise call of the boundary states, in its own comment, the
+    page and section that define its operation."""
+    txt = open(HEADER).read()
+    pages = ("techwalker", "reportify", "mokono", "hwcomputing")
+    for name in ("moge_route", "moge_permute", "moge_grouped_ffn", "moge_shared_ffn",
+                 "moge_combine"):
+        decl = re.search(r"MOGE_API\s+int\s+%s\s*\(" % name, txt)
+        assert decl, name
+        comment = txt[:decl.start()].rsplit("/*", 1)[1]
+        assert any(p in comment for p in pages) and "section" in comment, name
+
+
 def test_library_exports_every_declared_symbol(L):
     out = subprocess.check_output(["nm", "-D", "--defined-only", mg.LIB_PATH], text=True)
     exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
