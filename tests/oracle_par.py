@@ -21,12 +21,19 @@ def threads() -> int:
     return max(1, min(16, os.cpu_count() or 1))
 
 
+def _load():
+    """Load the oracle's library in the calling thread before any worker
+    starts (its first use may compile it, which must happen once)."""
+    oracle.e4m3_decode(0)
+
+
 def _tokens(x, tokens):
     n = np.asarray(x).shape[0]
     return np.arange(n, dtype=np.int64) if tokens is None else np.asarray(tokens, np.int64)
 
 
 def _split_tokens(fn, x, tokens, *args, **kw):
+    _load()
     toks = _tokens(x, tokens)
     nt = min(threads(), len(toks))
     if nt <= 1:
@@ -55,6 +62,7 @@ def layer_w8a8(x, inp, q, M, Kp, dtype, tokens=None):
 def quantize_experts_fp8(inp: dict) -> dict:
     """oracle.quantize_experts_fp8, each matrix's experts spread over threads
     (rows are quantised independently); same returns."""
+    _load()
     jobs = []
     for k in ("w_gate", "w_up", "w_down", "s_gate", "s_up", "s_down"):
         w = inp[k]
@@ -79,6 +87,7 @@ def layer_backward_sum(x, inp, M, Kp, dtype, dy, alpha, idx, tokens, parts):
     its token terms split into `parts` lists on threads and summed in list
     order (every gradient is a sum over tokens; the balance loss's batch
     shares come from the whole batch in every part, so aux is part 0's)."""
+    _load()
     toks = _tokens(x, tokens)
     chunks = [c for c in np.array_split(toks, max(1, min(parts, len(toks)))) if len(c)] or [toks]
     with ThreadPoolExecutor(len(chunks)) as ex:
